@@ -1,0 +1,515 @@
+#!/usr/bin/env python
+"""Throughput of the CSA + HCA compressed-attention hot path on B200.
+
+One step = one decode step of the decode_1m workload through the C ABI:
+4 sequences x 4 layers (CSA, HCA, CSA, HCA) at a cached context of 1,048,576
+tokens (CSA 4:1 with e4m3 indexer keys and top-1024, HCA 128:1 dense, 128-token
+window, 64 heads of 512 dims).  `value` = tokens/s over all ranks (each rank
+runs its own 4 sequences: weak scaling, no collective on the data path).
+With --prefill the line also carries the csa_prefill_128k layer (one CSA
+prefill of 131,072 tokens: both compressors, indexer top-k, attention).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the float64 CPU oracle (the only reference that
+exists for this path) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes as C
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_compressed_overlapped_b200 import api, native, synth  # noqa: E402
+
+METRIC = "CSA+HCA attention tokens/s (decode@1M, prefill@128K); % HBM / TC roofline"
+L2_BYTES = 126 * 2**20
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------ distributed ----
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks ----
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms (this GPU)."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.uuid = None
+        try:
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            pass
+        self.proc = None
+        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "200"]
+            if self.uuid:
+                cmd[1:1] = ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    sm.append(float(parts[2]))
+                    smax = float(parts[3])
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[6:10]):
+                    if val.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        busy = [x for x in sm if smax and x > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------- decode step ----
+
+class DecodeStep:
+    """Pre-marshalled C-ABI calls of one decode step (all layers)."""
+
+    def __init__(self, wl, layers, stream):
+        self.lib = native.lib()
+        self.wl = wl
+        self.layers = layers
+        self.stream = stream
+        self.sh = stream.cuda_stream
+        self.calls = []
+        for L in layers:
+            kw = dict(m=L["m"], rope_dims=wl.r, q_gain=L["q_gain"])
+            if L["kind"] == "csa":
+                kw.update(k=wl.k, qI=L["qI"], wI=L["w"], kI=L["kI"], kI_scale=L["kI_scale"])
+            args, out, keep = api.decode_args(L["kind"], L["q"], L["pos"], L["kv"], L["win"],
+                                              L["sinks"], **kw)
+            nbytes = self.lib.csahca_decode_workspace_size(C.byref(args))
+            ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=L["q"].device)
+            args.workspace = ws.data_ptr()
+            args.workspace_bytes = ws.numel()
+            L["out"] = out
+            self.calls.append((args, out, keep, ws))
+
+    def __call__(self):
+        for args, _, _, _ in self.calls:
+            st = self.lib.compressed_attn_decode(C.byref(args), self.sh)
+            if st != 0:
+                native.check(st, "compressed_attn_decode")
+
+
+def decode_bytes_per_kernel(wl, ctx):
+    """Algorithmic bytes per launch of each traced decode kernel (one launch
+    covers the B sequences of one layer)."""
+    B, d, H, HI, dI, k, w = wl.B, wl.d, wl.H, wl.HI, wl.dI, wl.k, wl.w
+    vc = (ctx + 1) // wl.m
+    vh = (ctx + 1) // wl.m_hca
+    key_row = dI + 4 * (dI // 128) if wl.fp8_keys else 2 * dI
+    qo = 2 * H * d * 2
+    return {
+        "indexer_scores": B * (vc * key_row + HI * dI * 2 + HI * 4),
+        "topk_rows": B * (vc * 4 + k * 4),
+        "attn_decode_csa": B * ((k + w) * d * 2 + qo),
+        "attn_decode_hca": B * ((vh + w) * d * 2 + qo),
+    }
+
+
+def decode_step_bytes(wl, ctx):
+    """Algorithmic HBM bytes of one whole decode step (all layers)."""
+    per = decode_bytes_per_kernel(wl, ctx)
+    tot = 0
+    for kind in wl.layers:
+        if kind == "csa":
+            tot += per["indexer_scores"] + per["attn_decode_csa"]
+        else:
+            tot += per["attn_decode_hca"]
+    return tot
+
+
+def kernel_bytes_key(name):
+    if name.startswith("indexer_scores"):
+        return "indexer_scores"
+    if name.startswith("topk"):
+        return "topk_rows"
+    if "decode_csa" in name:
+        return "attn_decode_csa"
+    if "decode_hca" in name:
+        return "attn_decode_hca"
+    return None
+
+
+def time_steps(step, K, stream, flush, world):
+    """K steps, each bracketed by CUDA events on `stream`, L2 flushed between
+    steps (outside the events).  Returns the max over ranks of the summed
+    device time in ms."""
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(K):
+            flush()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    total = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    return max_over_ranks(total, world)
+
+
+# -------------------------------------------------------------- prefill ----
+
+def prefill_layer_fn(wl, dev, stream):
+    inp = synth.prefill_inputs(wl, dev)
+    kvi, ik = inp["kv"], inp["ik"]
+    q_pos = torch.arange(wl.n, device=dev, dtype=torch.int32)[None].repeat(wl.B, 1).contiguous()
+    idx = torch.empty(wl.B, wl.n, wl.k, dtype=torch.int32, device=dev)
+    out = torch.empty_like(inp["q"])
+
+    def step():
+        with torch.cuda.stream(stream):
+            kv = api.csa_compress(kvi["a"], kvi["b"], kvi["za"], kvi["zb"], kvi["bias_a"],
+                                  kvi["bias_b"], wl.m, gain=inp["kv_gain"], rope_dims=wl.r,
+                                  stream=stream)
+            kI = api.csa_compress(ik["a"], ik["b"], ik["za"], ik["zb"], ik["bias_a"],
+                                  ik["bias_b"], wl.m, rms_norm=False, stream=stream)
+            api.indexer_topk(inp["qI"], inp["w"], kI, q_pos, wl.m, wl.k, idx=idx, stream=stream)
+            api.compressed_attn_prefill("csa", inp["q"], kv, inp["kv_win"], inp["sinks"], m=wl.m,
+                                        w=wl.w, rope_dims=wl.r, idx=idx, q_gain=inp["q_gain"],
+                                        kv_gain=inp["kv_gain"], out=out, stream=stream)
+    return step
+
+
+def prefill_flops(wl):
+    n, m, k, w = wl.n, wl.m, wl.k, wl.w
+    t = np.arange(n, dtype=np.int64)
+    vis = (t + 1) // m
+    pairs = int(vis.sum())
+    keys = int(np.minimum(vis, k).sum() + np.minimum(w, t + 1).sum())
+    idx_fl = pairs * wl.HI * wl.dI * 2
+    att_fl = keys * wl.H * wl.d * 4
+    return idx_fl, att_fl
+
+
+# ------------------------------------------------------------ CPU oracle ----
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads", 0) for i in info if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def oracle_decode_sequence(wl, layers, b):
+    """The oracle's decode step for sequence b over all layers."""
+    from oracle import csahca_oracle as O
+
+    def npy(t):
+        return t.detach().cpu().to(torch.float64).numpy() if t.dtype != torch.uint8 else t.cpu().numpy()
+
+    outs = []
+    for L in layers:
+        pos = int(L["pos"][b])
+        sel = None
+        if L["kind"] == "csa":
+            v = min(O.n_visible(pos, L["m"]), L["kv"].shape[1])
+            if L["kI_scale"] is not None:
+                K = O.dequant_e4m3_rows(npy(L["kI"][b, :v]), npy(L["kI_scale"][b, :v]))
+            else:
+                K = npy(L["kI"][b, :v])
+            s = O.indexer_scores(npy(L["qI"][b]), npy(L["w"][b]), K)
+            sel = O.top_k_select(s, wl.k)
+        outs.append(O.decode_attention(L["kind"], npy(L["q"][b]), pos, npy(L["kv"][b]),
+                                       npy(L["win"][b]), npy(L["sinks"]), m=L["m"], w=wl.w,
+                                       r=wl.r, q_gain=npy(L["q_gain"]), sel=sel))
+    return outs
+
+
+def host_layers(layers):
+    """Host copies of the layer tensors the oracle reads (one sequence's worth
+    is sliced later)."""
+    out = []
+    for L in layers:
+        H = {}
+        for k_, v in L.items():
+            H[k_] = v.cpu() if isinstance(v, torch.Tensor) else v
+        out.append(H)
+    return out
+
+
+def cpu_baseline(wl, layers_host, budget_s=12.0):
+    """Oracle decode steps on whole sequences until ~budget_s of CPU work."""
+    t0 = time.perf_counter()
+    seqs = 0
+    while True:
+        oracle_decode_sequence(wl, layers_host, seqs % wl.B)
+        seqs += 1
+        if time.perf_counter() - t0 >= budget_s or seqs >= wl.B:
+            break
+    el = time.perf_counter() - t0
+    return {"value": seqs / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{seqs} of {wl.B} sequences of one decode step, all {len(wl.layers)} layers "
+                      f"(float64 NumPy, {el:.1f} s)"}
+
+
+# ------------------------------------------------------------------ main ----
+
+def run_reference(args, world, rank):
+    """Reference arm: the float64 oracle on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS[args.workload]
+    layers = synth.decode_inputs(wl, "cpu" if not torch.cuda.is_available() else "cuda")
+    layers_host = host_layers(layers)
+    del layers
+    for _ in range(args.warmup):
+        oracle_decode_sequence(wl, layers_host, 0)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_decode_sequence(wl, layers_host, i % wl.B)
+    el = time.perf_counter() - t0
+    value = args.steps / el
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "global_batch": 1, "seq_len": wl.ctx, "layers": list(wl.layers),
+                   "sample": "one sequence per step (of 4), all layers", "parallelism": "none"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": "one of the 4 sequences per step, all 4 layers, float64 NumPy"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode_1m")
+    ap.add_argument("--prefill", action="store_true", help="also time csa_prefill_128k")
+    ap.add_argument("--prefill-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world, rank, local = dist_setup() if torch.cuda.is_available() else (1, 0, 0)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device=dev)
+    wl = synth.WORKLOADS[args.workload]
+    wl_r = synth.Workload(**{**wl.__dict__, "seed": wl.seed + 1000 * rank})
+    layers = synth.decode_inputs(wl_r, dev)
+    step = DecodeStep(wl, layers, stream)
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.random_(0, 255)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize()
+    if api.device_error(stream) != 0:
+        raise RuntimeError("device error flag set during warm-up")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    total_ms = time_steps(step, args.steps, stream, flush, world)
+    clk = clocks.stop()
+    ms_per_step = total_ms / args.steps
+    tokens = world * wl.B * args.steps
+    value = tokens / (total_ms / 1000.0)
+
+    # traced pass: per-kernel device time of the same K steps
+    api.trace_enable(True)
+    time_steps(step, args.steps, stream, flush, world)
+    traced = api.trace_collect()
+    api.trace_enable(False)
+
+    pk = peaks()
+    per_bytes = decode_bytes_per_kernel(wl, wl.ctx)
+    dom = max(traced.items(), key=lambda kv: kv[1][1])
+    dname, (dl, dms) = dom
+    key = kernel_bytes_key(dname)
+    roof = None
+    if key is not None:
+        ach = per_bytes[key] / (dms / dl / 1000.0) / 1e9
+        roof = {"kernel": dname, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": ach / pk["hbm_gbs"], "traffic": None,
+                "peak_source": pk["source"], "launches": dl, "avg_us": 1000 * dms / dl}
+    step_bytes = decode_step_bytes(wl, wl.ctx)
+    step_frac = step_bytes / (ms_per_step / 1000.0) / 1e9 / pk["hbm_gbs"]
+
+    # end to end: pinned host inputs copied in and outputs read back per step
+    host_in, host_out = [], []
+    for L in layers:
+        for name in ("q", "qI", "w", "pos"):
+            if name in L:
+                host_in.append((L[name], L[name].cpu().pin_memory()))
+        host_out.append((L["out"], torch.empty(L["out"].shape, dtype=L["out"].dtype).pin_memory()))
+    h2d = sum(h.numel() * h.element_size() for _, h in host_in)
+    d2h = sum(h.numel() * h.element_size() for _, h in host_out)
+
+    def e2e_step():
+        for dv, hv in host_in:
+            dv.copy_(hv, non_blocking=True)
+        step()
+        for dv, hv in host_out:
+            hv.copy_(dv, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = time_steps(e2e_step, args.steps, stream, flush, world)
+    e2e_val = tokens / (e2e_ms / 1000.0)
+
+    prefill = None
+    if args.prefill:
+        pw = synth.WORKLOADS["csa_prefill_128k"]
+        pstep = prefill_layer_fn(pw, dev, stream)
+        for _ in range(max(1, args.warmup // 3)):
+            pstep()
+        torch.cuda.synchronize()
+        api.trace_enable(True)
+        p_ms = time_steps(pstep, args.prefill_steps, stream, flush, world)
+        ptr = api.trace_collect()
+        api.trace_enable(False)
+        idx_fl, att_fl = prefill_flops(pw)
+        tot_fl = idx_fl + att_fl
+        peak_tf = pk["bf16_tflops_sustained"]
+        prefill = {"workload": pw.name, "tokens_per_s": world * pw.n * args.prefill_steps / (p_ms / 1000),
+                   "ms_per_layer": p_ms / args.prefill_steps,
+                   "tflops": tot_fl / (p_ms / args.prefill_steps / 1000) / 1e12,
+                   "frac_of_bf16_peak": tot_fl / (p_ms / args.prefill_steps / 1000) / 1e12 / peak_tf,
+                   "peak_tflops": peak_tf, "algorithmic_flops": tot_fl,
+                   "kernels_ms_per_layer": {k_: v[1] / args.prefill_steps for k_, v in ptr.items()}}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, host_layers(layers))
+
+    if api.device_error(stream) != 0:
+        raise RuntimeError("device error flag set during the timed region")
+    launches = sum(v[0] for v in traced.values()) // args.steps * args.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "global_batch": world * wl.B, "seq_len": wl.ctx,
+                   "layers": list(wl.layers), "heads": wl.H, "head_dim": wl.d, "top_k": wl.k,
+                   "window": wl.w, "indexer_keys": "e4m3" if wl.fp8_keys else "bf16",
+                   "parallelism": f"replicas{world}" if world > 1 else "none",
+                   "l2": "flushed between timed steps"},
+        "roofline": roof,
+        "step_hbm": {"algorithmic_bytes": step_bytes, "frac": step_frac, "peak": pk["hbm_gbs"]},
+        "clocks": clk,
+        "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "kernels_ms_per_step": {k_: v[1] / args.steps for k_, v in traced.items()},
+        "cpu_baseline": cpu,
+        "prefill": prefill,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        barrier(world)
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,292 @@
+/*
+ * csahca.h -- C ABI of the B200 (sm_100a) compressed-attention library
+ * (libcsahca.so): the forward hot path of DeepSeek-V4's hybrid attention,
+ * CSA (compressed sparse attention) and HCA (heavily compressed attention).
+ *
+ * Sources, cited by page title and section:
+ *   [P2] "Paper Breakdown: DeepSeek-V4", section 4 "Hybrid Attention: CSA + HCA":
+ *        CSA KV compression (two streams C^a, C^b, logits Z^a, Z^b, 2m entries
+ *        per block, softmax with positional biases B^a, B^b), DSA on compressed
+ *        KV (indexer keys compressed the same way, top-k, MQA core attention),
+ *        sliding window KV, HCA (single stream, ratio 1/m', no overlap, dense),
+ *        Additional Techniques (query/KV RMSNorm, partial RoPE on the last 64
+ *        dims, attention sink logit per head).
+ *   [P4] "How DeepSeek-V4 architecture and training work together", section
+ *        "Two compressed views of one history": 1,024 selected entries per
+ *        query, 128-token local window.
+ *   [P5] "Inside DeepSeek V4": "Two compression regimes" (overlapping 4x,
+ *        non-overlapping 128x) and "Local window" (128 uncompressed entries in
+ *        every CSA and HCA layer).
+ *
+ * Conventions (all entry points):
+ *   - Every tensor argument is a DEVICE pointer owned by the caller, row-major
+ *     and contiguous in the layout stated, 16-byte aligned.  The library keeps
+ *     no pointer after the call returns and allocates no device memory: where
+ *     a call needs scratch it takes `workspace` / `workspace_bytes`, sized by
+ *     the matching *_workspace_size() query (NULL / 0 is fine when that query
+ *     returns 0).
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  A return of CSAHCA_OK means the work was
+ *     enqueued; errors found on the device surface through
+ *     csahca_device_error().
+ *   - Shapes are validated on the host before any launch; a bad argument
+ *     returns a negative status and launches nothing.  There is no fallback
+ *     path: a shape the kernels do not cover returns CSAHCA_ERR_UNSUPPORTED.
+ *   - dtypes: F32 (float), BF16 (bfloat16), E4M3 (float8 e4m3 "fn" bytes, with
+ *     one fp32 scale per 128 contiguous elements).  Arithmetic is fp32.
+ *   - Fixed readings of the pages (stated once here, used by every call):
+ *       entry i of ratio m covers tokens i*m .. (i+1)*m-1 and is visible to
+ *       query t iff (i+1)*m-1 <= t; an incomplete trailing block forms no
+ *       entry; RoPE rotates interleaved pairs (2j, 2j+1) of the last r dims by
+ *       pos * base^(-2j/r); compressed entry i sits at position i*m; RMSNorm is
+ *       x / sqrt(mean(x^2) + eps) * gain; softmax scale defaults to 1/sqrt(d);
+ *       K = V = the compressed (or window) row; the sink adds e^{z_h} to the
+ *       softmax denominator only; the rope dims of each output row are rotated
+ *       back by -t (t = query position).
+ */
+#ifndef CSAHCA_H_
+#define CSAHCA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CSAHCA_ABI_VERSION 1
+
+/* ---- status codes ------------------------------------------------------- */
+enum {
+  CSAHCA_OK = 0,
+  CSAHCA_ERR_INVALID_ARG = -1,   /* NULL pointer, negative size, bad enum      */
+  CSAHCA_ERR_UNSUPPORTED = -2,   /* valid but not covered by the kernels       */
+  CSAHCA_ERR_ALIGNMENT = -3,     /* a pointer is not 16-byte aligned           */
+  CSAHCA_ERR_WORKSPACE = -4,     /* workspace NULL or smaller than required    */
+  CSAHCA_ERR_LAUNCH = -5,        /* a CUDA launch or driver call failed        */
+  CSAHCA_ERR_DEVICE_TIMEOUT = -6,/* a bounded device wait gave up (see below)  */
+  CSAHCA_ERR_NO_DEVICE = -7      /* no usable sm_100 device                    */
+};
+
+/* ---- enums ---------------------------------------------------------------- */
+enum { CSAHCA_F32 = 0, CSAHCA_BF16 = 1, CSAHCA_E4M3 = 2 };
+enum { CSAHCA_CSA = 0, CSAHCA_HCA = 1 };
+
+/* ---- csa_compress / hca_compress ----------------------------------------
+ * [P2] CSA KV compression; HCA; Additional Techniques (RMSNorm, RoPE).
+ *
+ * CSA (overlapped, ratio 1/m, 2m tokens per entry), for entry i, channel c:
+ *   la_r = za[i*m + r, c] + bias_a[r, c],  lb_r = zb[(i-1)*m + r, c] + bias_b[r, c]
+ *   (lb = -inf for i = 0), S = softmax over the 2m logits jointly,
+ *   C_i[c] = sum_r Sa_r a[i*m + r, c] + sum_r Sb_r b[(i-1)*m + r, c].
+ * HCA (non-overlapped, ratio 1/m'): C_i[c] = sum_r softmax_r(za + bias_a) a.
+ *   (b, zb, bias_b are ignored.)
+ * Then, if rms_norm != 0: C_i <- C_i / sqrt(mean(C_i^2) + eps) * gain (gain
+ * NULL = ones); if rope_dims > 0: RoPE at position i*m on the last rope_dims.
+ * Indexer keys use the same pooling with rms_norm = 0 and rope_dims = 0.
+ *
+ * Layout: a, b, za, zb [B, n, c] (dtype); bias_a, bias_b [m, c] f32;
+ * gain [c] f32; out [B, num_blocks, c] (dtype) holding entries
+ * first_block .. first_block + num_blocks - 1, each of which must be complete
+ * (first_block + num_blocks <= n / m).  num_blocks = -1 means all n / m
+ * entries from first_block.  Constraints: dtype F32 (c % 4 == 0) or BF16
+ * (c % 8 == 0); rope_dims even, <= c, (c - rope_dims) even; m >= 1.
+ */
+typedef struct {
+  int32_t dtype;
+  int32_t B, n, c;
+  int32_t m;
+  int32_t first_block, num_blocks;
+  int32_t rms_norm;
+  int32_t rope_dims;
+  float rope_base;     /* 0 -> 10000 */
+  float eps;           /* 0 -> 1e-6  */
+  int32_t reserved0;
+  const void* a;
+  const void* b;
+  const void* za;
+  const void* zb;
+  const float* bias_a;
+  const float* bias_b;
+  const float* gain;
+  void* out;
+} csahca_compress_args;
+
+int csa_compress(const csahca_compress_args* args, void* stream);
+int hca_compress(const csahca_compress_args* args, void* stream);
+
+/* ---- indexer_topk ---------------------------------------------------------
+ * [P2] DSA on Compressed KV (lightning indexer, top-k); [P4] 1,024 entries.
+ * For query q of sequence b at absolute position t = q_pos[b, q]:
+ *   I_{t,i} = sum_j w[b,q,j] * max(0, qI[b,q,j,:] . kI[b,i,:])  for the
+ *   visible entries i < v = min(N, (t+1)/m);  kI row i = decode(codes) * scale
+ *   per 128-element block when k_dtype = E4M3.
+ *   idx[b,q,:] = the k entries with the largest I (ties to the lower index),
+ *   sorted ascending, padded with -1 when v < k.
+ * Layout: qI [B, nq, HI, dI] (q_dtype F32/BF16); w [B, nq, HI] f32;
+ *   kI [B, N, dI] (k_dtype F32/BF16/E4M3); kI_scale [B, N, dI/128] f32 (E4M3
+ *   only, else NULL); q_pos [B, nq] int32 on the device; idx [B, nq, k] int32.
+ *   scores_out: optional [B, nq, N] f32; entries i < v of each row receive
+ *   I_{t,i}, the rest is left untouched.  q_pos values < 0 give v = 0.
+ * Constraints: k >= 1; dI % 8 == 0; E4M3 needs dI % 128 == 0 and the same
+ *   q_dtype rules; q_dtype == k_dtype unless k_dtype is E4M3 (queries BF16).
+ * Workspace: csahca_indexer_workspace_size().
+ */
+typedef struct {
+  int32_t q_dtype, k_dtype;
+  int32_t B, nq, HI, dI;
+  int32_t N;
+  int32_t m;
+  int32_t k;
+  int32_t reserved0;
+  const void* qI;
+  const float* w;
+  const void* kI;
+  const float* kI_scale;
+  const int32_t* q_pos;
+  int32_t* idx;
+  float* scores_out;
+  void* workspace;
+  size_t workspace_bytes;
+} csahca_indexer_args;
+
+int indexer_topk(const csahca_indexer_args* args, void* stream);
+size_t csahca_indexer_workspace_size(const csahca_indexer_args* args);
+
+/* ---- compressed_attn_prefill ----------------------------------------------
+ * [P2] MQA core attention, sliding window, HCA dense attention, Additional
+ * Techniques; [P5] Local window.  For sequence b, query t (position t), head h:
+ *   q = RoPE_t(RMSNorm(q_raw[b,t,h,:]) * q_gain)     (norm only if q_norm)
+ *   keys J_t = { kv_comp[b, idx[b,t,j]] : idx >= 0 }           (kind CSA)
+ *            = { kv_comp[b, i] : i < min(N, (t+1)/m) }          (kind HCA)
+ *     plus window rows s = max(0, t-w+1) .. t, each
+ *     RoPE_s(RMSNorm(kv_win[b,s,:]) * kv_gain)        (norm only if kv_norm)
+ *   o = sum_j e^{s_j} row_j / (e^{sinks[h]} + sum_j e^{s_j}),
+ *   s_j = scale * q . row_j, then the last rope_dims of o rotated by -t.
+ * Layout: q [B, n, H, d]; kv_comp [B, N, d] (final rows from csa/hca_compress);
+ *   kv_win [B, n, d] raw per-token rows; q_gain, kv_gain [d] f32 or NULL
+ *   (ones); idx [B, n, k] int32 (CSA; entries < 0 are skipped, entries must be
+ *   < N); sinks [H] f32; out [B, n, H, d].  q, kv_comp, kv_win, out share
+ *   `dtype` (F32 or BF16).
+ * Constraints: d % 8 == 0, rope_dims even and <= d, w >= 0, H >= 1.
+ * Workspace: csahca_prefill_workspace_size().
+ */
+typedef struct {
+  int32_t kind;
+  int32_t dtype;
+  int32_t B, n, H, d;
+  int32_t N;
+  int32_t m;
+  int32_t k;
+  int32_t w;
+  int32_t rope_dims;
+  float rope_base;     /* 0 -> 10000 */
+  float eps;           /* 0 -> 1e-6 */
+  float scale;         /* 0 -> 1/sqrt(d) */
+  int32_t q_norm, kv_norm;
+  const void* q;
+  const void* kv_comp;
+  const void* kv_win;
+  const float* q_gain;
+  const float* kv_gain;
+  const int32_t* idx;
+  const float* sinks;
+  void* out;
+  void* workspace;
+  size_t workspace_bytes;
+} csahca_attn_args;
+
+int compressed_attn_prefill(const csahca_attn_args* args, void* stream);
+size_t csahca_prefill_workspace_size(const csahca_attn_args* args);
+
+/* ---- compressed_attn_decode -----------------------------------------------
+ * One decode step of one layer (CSA or HCA) for B sequences, one new query
+ * token each at position pos[b] (device int32).  Caches hold final rows
+ * (already normed and roped): kv_cache [B, N_cap, d] with entry i valid iff
+ * i < min(N_cap, (pos+1)/m); win [B, w, d] ring buffer, slot p % w holding
+ * the row of position p, for p = max(0, pos-w+1) .. pos (the new token's own
+ * row included).  q [B, H, d] raw, normed (q_norm) and roped at pos here.
+ * CSA: the selection is the lightning-indexer top-k over the visible entries
+ *   (qI [B, HI, dI], wI [B, HI] f32, kI [B, N_cap, dI], kI_scale as in
+ *   indexer_topk) unless idx_in [B, k] is given, which is then used as is.
+ *   idx_out [B, k] (optional) receives the selection used.
+ * HCA: dense over every visible entry.  Output and sink exactly as in
+ * compressed_attn_prefill; out [B, H, d] (dtype).
+ * Workspace: csahca_decode_workspace_size().
+ */
+typedef struct {
+  int32_t kind;
+  int32_t dtype;
+  int32_t B, H, d;
+  int32_t N_cap;
+  int32_t m;
+  int32_t w;
+  int32_t rope_dims;
+  float rope_base;
+  float eps;
+  float scale;
+  int32_t q_norm;
+  int32_t k;
+  int32_t HI, dI;
+  int32_t qI_dtype, kI_dtype;
+  const void* q;
+  const int32_t* pos;
+  const float* q_gain;
+  const void* kv_cache;
+  const void* win;
+  const float* sinks;
+  const void* qI;
+  const float* wI;
+  const void* kI;
+  const float* kI_scale;
+  const int32_t* idx_in;
+  int32_t* idx_out;
+  void* out;
+  void* workspace;
+  size_t workspace_bytes;
+} csahca_decode_args;
+
+int compressed_attn_decode(const csahca_decode_args* args, void* stream);
+size_t csahca_decode_workspace_size(const csahca_decode_args* args);
+
+/* ---- utilities ------------------------------------------------------------ */
+
+/* Human-readable name of a status code (static string). */
+const char* csahca_status_string(int status);
+
+/* CSAHCA_ABI_VERSION of the loaded library. */
+int csahca_abi_version(void);
+
+/* sizeof() of the argument structs, for bindings to check their mirrors:
+ * which = 0 compress, 1 indexer, 2 prefill, 3 decode; -1 for an unknown id. */
+int64_t csahca_struct_size(int which);
+
+/* Device-side error word of the current device: every bounded wait in the
+ * kernels that gives up ORs a code into it and the kernel returns early
+ * instead of hanging.  Synchronises `stream`, stores the word in *code (0 =
+ * no error) and clears it.  Returns CSAHCA_OK, or CSAHCA_ERR_LAUNCH if the
+ * stream itself reports a CUDA error. */
+int csahca_device_error(void* stream, int32_t* code);
+
+/* ---- tracing ---------------------------------------------------------------
+ * Optional per-kernel timing.  While enabled, every kernel the library
+ * launches is bracketed by two CUDA events recorded on its stream (events are
+ * created once and reused; at most 65536 launches are held between collects,
+ * later ones are not traced).  csahca_trace_collect() synchronises those
+ * events, adds the elapsed times up per kernel name, writes at most
+ * max_entries entries, stores how many it wrote in *n_entries and forgets
+ * the recorded launches.  Not thread-safe: trace from one host thread. */
+typedef struct {
+  char name[48];
+  int64_t launches;
+  double total_ms;
+} csahca_trace_entry;
+
+int csahca_trace_enable(int enable);
+int csahca_trace_collect(csahca_trace_entry* out, int max_entries, int* n_entries);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSAHCA_H_ */

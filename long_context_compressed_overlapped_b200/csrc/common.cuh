@@ -1,0 +1,97 @@
+// Shared device helpers: storage-type conversion, 16-byte vector access,
+// warp/block reductions, RoPE angles and the device error word.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+namespace csahca {
+
+// Error codes ORed into g_device_error by a bounded wait that gave up.
+enum : int32_t {
+  DEVERR_MBAR_TIMEOUT = 1,     // an mbarrier wait exceeded its iteration limit
+  DEVERR_BAD_INDEX = 2,        // a selection index outside [0, N) was skipped
+};
+
+__device__ int32_t g_device_error;
+
+__device__ __forceinline__ void raise_device_error(int32_t code) {
+  atomicOr(&g_device_error, code);
+}
+
+// ---- storage types --------------------------------------------------------
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Elements of T per 16-byte vector.
+template <typename T> struct Vec16 { static constexpr int N = 16 / sizeof(T); };
+
+__device__ __forceinline__ void load16(const float* p, float* o) {
+  float4 v = __ldg(reinterpret_cast<const float4*>(p));
+  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+}
+__device__ __forceinline__ void load16(const __nv_bfloat16* p, float* o) {
+  uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(h[i]);
+    o[2 * i] = f.x; o[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void store16(float* p, const float* o) {
+  *reinterpret_cast<float4*>(p) = make_float4(o[0], o[1], o[2], o[3]);
+}
+__device__ __forceinline__ void store16(__nv_bfloat16* p, const float* o) {
+  uint4 v;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+  *reinterpret_cast<uint4*>(p) = v;
+}
+
+// e4m3 ("fn") byte -> float, through the CUDA fp8 conversion intrinsic.
+__device__ __forceinline__ float e4m3_to_f32(uint8_t code) {
+  __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code), __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+// ---- reductions -------------------------------------------------------------
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// ---- RoPE -----------------------------------------------------------------------
+// Pair j of the last r dims at position pos rotates by pos * base^(-2j/r).  The
+// angle is formed and reduced in double so that positions up to 2^20 keep the
+// phase exact to fp32 rounding; cos/sin are returned in float.
+__device__ __forceinline__ void rope_cos_sin(double pos, int j, int r, double base,
+                                             float* c, float* s) {
+  double theta = pow(base, -2.0 * (double)j / (double)r);
+  double sn, cs;
+  sincos(pos * theta, &sn, &cs);
+  *c = (float)cs;
+  *s = (float)sn;
+}
+
+__host__ __device__ __forceinline__ int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace csahca

@@ -1,0 +1,609 @@
+// C ABI of libcsahca.so (declared in include/csahca.h).  Host-side argument
+// validation, workspace sizing and kernel dispatch; every step of the path
+// runs in the kernels included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <vector>
+
+#include "../../include/csahca.h"
+#include "common.cuh"
+#include "compress.cuh"
+#include "indexer_simt.cuh"
+#include "topk.cuh"
+#include "attention_simt.cuh"
+
+using namespace csahca;
+
+namespace {
+
+// ---------------------------------------------------------------- tracing --
+namespace trace {
+constexpr size_t kMaxRecords = 65536;
+struct Record { cudaEvent_t begin, end; const char* name; };
+bool g_enabled = false;
+std::vector<cudaEvent_t> g_pool;      // free events
+std::vector<Record> g_records;
+
+cudaEvent_t take_event() {
+  if (!g_pool.empty()) { cudaEvent_t e = g_pool.back(); g_pool.pop_back(); return e; }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) { (void)cudaGetLastError(); return nullptr; }
+  return e;
+}
+
+// Bracket one launch: begin() before it, end() after it, on the same stream.
+struct Scope {
+  cudaEvent_t b = nullptr;
+  const char* name;
+  cudaStream_t s;
+  Scope(const char* n, cudaStream_t st) : name(n), s(st) {
+    if (!g_enabled || g_records.size() >= kMaxRecords) return;
+    b = take_event();
+    if (b) cudaEventRecord(b, s);
+  }
+  ~Scope() {
+    if (!b) return;
+    cudaEvent_t e = take_event();
+    if (!e) { g_pool.push_back(b); return; }
+    cudaEventRecord(e, s);
+    g_records.push_back({b, e, name});
+  }
+};
+}  // namespace trace
+
+#define CSAHCA_TRACE(name, stream) trace::Scope trace_scope_##__LINE__(name, stream)
+
+constexpr double kDefaultRopeBase = 10000.0;
+constexpr float kDefaultEps = 1e-6f;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+#define CSAHCA_CHECK_LAUNCH()                                  \
+  do {                                                         \
+    if (cudaPeekAtLastError() != cudaSuccess) {                \
+      (void)cudaGetLastError();                                \
+      return CSAHCA_ERR_LAUNCH;                                \
+    }                                                          \
+  } while (0)
+
+int dtype_size(int dt) {
+  switch (dt) {
+    case CSAHCA_F32: return 4;
+    case CSAHCA_BF16: return 2;
+    case CSAHCA_E4M3: return 1;
+    default: return 0;
+  }
+}
+
+int device_ok() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { (void)cudaGetLastError(); return CSAHCA_ERR_NO_DEVICE; }
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return CSAHCA_ERR_NO_DEVICE;
+  }
+  return major == 10 ? CSAHCA_OK : CSAHCA_ERR_NO_DEVICE;
+}
+
+// ---------------------------------------------------------------- compress --
+
+int validate_compress(const csahca_compress_args* a, bool csa, int* nblocks) {
+  if (!a) return CSAHCA_ERR_INVALID_ARG;
+  if (a->dtype != CSAHCA_F32 && a->dtype != CSAHCA_BF16) return CSAHCA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->n < 0 || a->c <= 0 || a->m < 1 || a->first_block < 0) return CSAHCA_ERR_INVALID_ARG;
+  const int vec = 16 / dtype_size(a->dtype);
+  if (a->c % vec) return CSAHCA_ERR_UNSUPPORTED;
+  if (a->c > 128 * vec) return CSAHCA_ERR_UNSUPPORTED;
+  if (a->rope_dims < 0 || a->rope_dims > a->c || (a->rope_dims & 1) || ((a->c - a->rope_dims) & 1))
+    return CSAHCA_ERR_INVALID_ARG;
+  const int total = a->n / a->m;
+  int nb = a->num_blocks < 0 ? total - a->first_block : a->num_blocks;
+  if (nb < 0 || a->first_block + nb > total) return CSAHCA_ERR_INVALID_ARG;
+  *nblocks = nb;
+  if (nb == 0 || a->B == 0) return CSAHCA_OK;
+  if (!a->a || !a->za || !a->bias_a || !a->out) return CSAHCA_ERR_INVALID_ARG;
+  if (csa && (!a->b || !a->zb || !a->bias_b)) return CSAHCA_ERR_INVALID_ARG;
+  const void* ptrs[] = {a->a, a->za, a->bias_a, a->out, a->gain, csa ? a->b : nullptr,
+                        csa ? a->zb : nullptr, csa ? a->bias_b : nullptr};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return CSAHCA_ERR_ALIGNMENT;
+  return CSAHCA_OK;
+}
+
+int run_compress(const csahca_compress_args* a, void* stream, bool csa) {
+  int nb = 0;
+  int st = validate_compress(a, csa, &nb);
+  if (st != CSAHCA_OK) return st;
+  if (nb == 0 || a->B == 0) return CSAHCA_OK;
+  if ((st = device_ok()) != CSAHCA_OK) return st;
+  CompressParams p;
+  p.a = a->a; p.b = a->b; p.za = a->za; p.zb = a->zb;
+  p.bias_a = a->bias_a; p.bias_b = a->bias_b; p.gain = a->gain; p.out = a->out;
+  p.B = a->B; p.n = a->n; p.c = a->c; p.m = a->m; p.first_block = a->first_block;
+  p.num_blocks = nb; p.rms_norm = a->rms_norm; p.rope_dims = a->rope_dims;
+  p.rope_base = a->rope_base > 0 ? a->rope_base : kDefaultRopeBase;
+  p.eps = a->eps > 0 ? a->eps : kDefaultEps;
+  const int64_t warps = (int64_t)a->B * nb;
+  const int threads = 256;
+  const int64_t blocks = ceil_div64(warps * 32, threads);
+  if (blocks > INT32_MAX) return CSAHCA_ERR_UNSUPPORTED;
+  cudaStream_t s = as_stream(stream);
+  CSAHCA_TRACE(csa ? "csa_compress" : "hca_compress", s);
+  if (a->dtype == CSAHCA_F32) {
+    if (csa) compress_kernel<float, true><<<(unsigned)blocks, threads, 0, s>>>(p);
+    else compress_kernel<float, false><<<(unsigned)blocks, threads, 0, s>>>(p);
+  } else {
+    if (csa) compress_kernel<__nv_bfloat16, true><<<(unsigned)blocks, threads, 0, s>>>(p);
+    else compress_kernel<__nv_bfloat16, false><<<(unsigned)blocks, threads, 0, s>>>(p);
+  }
+  CSAHCA_CHECK_LAUNCH();
+  return CSAHCA_OK;
+}
+
+// ------------------------------------------------------------------ indexer --
+
+int validate_indexer(const csahca_indexer_args* a, bool shapes_only = false) {
+  if (!a) return CSAHCA_ERR_INVALID_ARG;
+  if (a->q_dtype != CSAHCA_F32 && a->q_dtype != CSAHCA_BF16) return CSAHCA_ERR_INVALID_ARG;
+  if (a->k_dtype != CSAHCA_F32 && a->k_dtype != CSAHCA_BF16 && a->k_dtype != CSAHCA_E4M3)
+    return CSAHCA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->nq < 0 || a->HI < 1 || a->dI < 1 || a->N < 0 || a->m < 1 || a->k < 1)
+    return CSAHCA_ERR_INVALID_ARG;
+  if (a->dI % 8) return CSAHCA_ERR_UNSUPPORTED;
+  if (a->k_dtype == CSAHCA_E4M3) {
+    if (a->dI % 128) return CSAHCA_ERR_UNSUPPORTED;
+    if (a->q_dtype != CSAHCA_BF16 && a->q_dtype != CSAHCA_F32) return CSAHCA_ERR_UNSUPPORTED;
+  } else if (a->k_dtype != a->q_dtype) {
+    return CSAHCA_ERR_UNSUPPORTED;
+  }
+  if (a->HI > kIdxSimtMaxHeads) return CSAHCA_ERR_UNSUPPORTED;
+  if (shapes_only || a->B == 0 || a->nq == 0) return CSAHCA_OK;
+  if (!a->qI || !a->w || !a->q_pos || !a->idx) return CSAHCA_ERR_INVALID_ARG;
+  if (a->N > 0 && !a->kI) return CSAHCA_ERR_INVALID_ARG;
+  if (a->k_dtype == CSAHCA_E4M3 && a->N > 0 && !a->kI_scale) return CSAHCA_ERR_INVALID_ARG;
+  const void* ptrs[] = {a->qI, a->w, a->kI, a->kI_scale, a->q_pos, a->idx, a->scores_out, a->workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return CSAHCA_ERR_ALIGNMENT;
+  return CSAHCA_OK;
+}
+
+// Query chunk so that a chunk of scores stays below ~2 GiB of workspace.
+int indexer_chunk_rows(const csahca_indexer_args* a) {
+  const int64_t per_q = (int64_t)a->B * (a->N > 0 ? a->N : 1) * 4;
+  int64_t rows = ((int64_t)2 << 30) / (per_q > 0 ? per_q : 1);
+  if (rows < 1) rows = 1;
+  if (rows > a->nq) rows = a->nq;
+  if (rows > 65535) rows = 65535;
+  return (int)rows;
+}
+
+size_t indexer_workspace(const csahca_indexer_args* a) {
+  if (a->scores_out || a->B == 0 || a->nq == 0) return 0;
+  return align_up((size_t)a->B * indexer_chunk_rows(a) * (size_t)(a->N > 0 ? a->N : 1) * 4, 256);
+}
+
+template <typename TQ, typename TK, bool kFP8>
+void launch_indexer_simt(const IndexerParams& p, cudaStream_t s) {
+  const size_t smem = ((size_t)p.HI * p.dI + p.HI) * sizeof(float);
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(indexer_scores_simt<TQ, TK, kFP8>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  dim3 grid((unsigned)ceil_div64(p.N, 256), (unsigned)p.q_count, (unsigned)p.B);
+  CSAHCA_TRACE("indexer_scores_simt", s);
+  indexer_scores_simt<TQ, TK, kFP8><<<grid, 256, smem, s>>>(p);
+}
+
+int run_indexer(const csahca_indexer_args* a, void* stream) {
+  int st = validate_indexer(a);
+  if (st != CSAHCA_OK) return st;
+  if (a->B == 0 || a->nq == 0) return CSAHCA_OK;
+  if ((st = device_ok()) != CSAHCA_OK) return st;
+  const size_t need = indexer_workspace(a);
+  if (need && (!a->workspace || a->workspace_bytes < need)) return CSAHCA_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  const int chunk = a->scores_out ? (a->nq < 65535 ? a->nq : 65535) : indexer_chunk_rows(a);
+  for (int q0 = 0; q0 < a->nq; q0 += chunk) {
+    const int qc = (a->nq - q0) < chunk ? (a->nq - q0) : chunk;
+    IndexerParams p;
+    p.qI = a->qI; p.w = a->w; p.kI = a->kI; p.kI_scale = a->kI_scale; p.q_pos = a->q_pos;
+    p.B = a->B; p.nq = a->nq; p.HI = a->HI; p.dI = a->dI; p.N = a->N; p.m = a->m;
+    p.q_begin = q0; p.q_count = qc;
+    // scores rows of this chunk: row (b, q) -> b * qc + (q - q0); with
+    // scores_out the full [B, nq, N] layout is addressed through the stride.
+    float* base;
+    int64_t stride = a->N > 0 ? a->N : 1;
+    if (a->scores_out) {
+      // one launch per batch entry keeps the [B, nq, N] layout
+      for (int b = 0; b < a->B; ++b) {
+        IndexerParams pb = p;
+        pb.B = 1;
+        pb.qI = static_cast<const char*>(a->qI) + (int64_t)b * a->nq * a->HI * a->dI * dtype_size(a->q_dtype);
+        pb.w = a->w + (int64_t)b * a->nq * a->HI;
+        pb.kI = a->kI ? static_cast<const char*>(a->kI) + (int64_t)b * a->N * a->dI * dtype_size(a->k_dtype) : nullptr;
+        pb.kI_scale = a->kI_scale ? a->kI_scale + (int64_t)b * a->N * (a->dI / 128) : nullptr;
+        pb.q_pos = a->q_pos + (int64_t)b * a->nq;
+        pb.scores = a->scores_out + ((int64_t)b * a->nq + q0) * stride;
+        pb.score_row_stride = stride;
+        if (a->N > 0) {
+          if (a->k_dtype == CSAHCA_E4M3) {
+            if (a->q_dtype == CSAHCA_BF16) launch_indexer_simt<__nv_bfloat16, uint8_t, true>(pb, s);
+            else launch_indexer_simt<float, uint8_t, true>(pb, s);
+          } else if (a->q_dtype == CSAHCA_BF16) {
+            launch_indexer_simt<__nv_bfloat16, __nv_bfloat16, false>(pb, s);
+          } else {
+            launch_indexer_simt<float, float, false>(pb, s);
+          }
+          CSAHCA_CHECK_LAUNCH();
+        }
+        TopkParams tp;
+        tp.scores = pb.scores; tp.row_stride = stride; tp.q_pos = pb.q_pos;
+        tp.idx = a->idx + (int64_t)b * a->nq * a->k;
+        tp.B = 1; tp.nq = a->nq; tp.N = a->N; tp.m = a->m; tp.k = a->k;
+        tp.q_begin = q0; tp.q_count = qc;
+        {
+          CSAHCA_TRACE("topk_rows", s);
+          topk_rows_kernel<<<qc, kTopkThreads, 0, s>>>(tp);
+        }
+        CSAHCA_CHECK_LAUNCH();
+      }
+      continue;
+    }
+    base = static_cast<float*>(a->workspace);
+    p.scores = base;
+    p.score_row_stride = stride;
+    if (a->N > 0) {
+      if (a->k_dtype == CSAHCA_E4M3) {
+        if (a->q_dtype == CSAHCA_BF16) launch_indexer_simt<__nv_bfloat16, uint8_t, true>(p, s);
+        else launch_indexer_simt<float, uint8_t, true>(p, s);
+      } else if (a->q_dtype == CSAHCA_BF16) {
+        launch_indexer_simt<__nv_bfloat16, __nv_bfloat16, false>(p, s);
+      } else {
+        launch_indexer_simt<float, float, false>(p, s);
+      }
+      CSAHCA_CHECK_LAUNCH();
+    }
+    TopkParams tp;
+    tp.scores = base; tp.row_stride = stride; tp.q_pos = a->q_pos; tp.idx = a->idx;
+    tp.B = a->B; tp.nq = a->nq; tp.N = a->N; tp.m = a->m; tp.k = a->k;
+    tp.q_begin = q0; tp.q_count = qc;
+    {
+      CSAHCA_TRACE("topk_rows", s);
+      topk_rows_kernel<<<(unsigned)(a->B * qc), kTopkThreads, 0, s>>>(tp);
+    }
+    CSAHCA_CHECK_LAUNCH();
+  }
+  return CSAHCA_OK;
+}
+
+// ----------------------------------------------------------------- prefill --
+
+int validate_attn(const csahca_attn_args* a, bool shapes_only = false) {
+  if (!a) return CSAHCA_ERR_INVALID_ARG;
+  if (a->kind != CSAHCA_CSA && a->kind != CSAHCA_HCA) return CSAHCA_ERR_INVALID_ARG;
+  if (a->dtype != CSAHCA_F32 && a->dtype != CSAHCA_BF16) return CSAHCA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->n < 0 || a->H < 1 || a->d < 1 || a->N < 0 || a->m < 1 || a->w < 0)
+    return CSAHCA_ERR_INVALID_ARG;
+  if (a->kind == CSAHCA_CSA && a->k < 1) return CSAHCA_ERR_INVALID_ARG;
+  if (a->rope_dims < 0 || a->rope_dims > a->d || (a->rope_dims & 1)) return CSAHCA_ERR_INVALID_ARG;
+  if (a->d % 32 || a->d > 32 * kSimtMaxDPL) return CSAHCA_ERR_UNSUPPORTED;
+  if (shapes_only || a->B == 0 || a->n == 0) return CSAHCA_OK;
+  if (!a->q || !a->sinks || !a->out) return CSAHCA_ERR_INVALID_ARG;
+  if (a->N > 0 && !a->kv_comp) return CSAHCA_ERR_INVALID_ARG;
+  if (a->w > 0 && !a->kv_win) return CSAHCA_ERR_INVALID_ARG;
+  if (a->kind == CSAHCA_CSA && !a->idx) return CSAHCA_ERR_INVALID_ARG;
+  const void* ptrs[] = {a->q, a->kv_comp, a->kv_win, a->q_gain, a->kv_gain, a->idx, a->sinks,
+                        a->out, a->workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return CSAHCA_ERR_ALIGNMENT;
+  return CSAHCA_OK;
+}
+
+size_t prefill_workspace(const csahca_attn_args* a) {
+  if (a->B == 0 || a->n == 0 || a->w == 0) return 0;
+  return align_up((size_t)a->B * a->n * a->d * dtype_size(a->dtype), 256);
+}
+
+template <typename T>
+int launch_finish(const void* x, void* out, const float* gain, int64_t rows, int c, int group,
+                  int npos, int rms, int r, double base, float eps, cudaStream_t s) {
+  FinishParams f;
+  f.x = x; f.out = out; f.gain = gain; f.rows = rows; f.c = c; f.group = group; f.npos = npos;
+  f.rms_norm = rms; f.rope_dims = r; f.rope_base = base; f.eps = eps;
+  const int64_t blocks = ceil_div64(rows * 32, 256);
+  CSAHCA_TRACE("finish_rows", s);
+  finish_rows_kernel<T><<<(unsigned)blocks, 256, 0, s>>>(f);
+  CSAHCA_CHECK_LAUNCH();
+  return CSAHCA_OK;
+}
+
+template <typename T>
+int launch_simt_attn(const SimtAttnParams& p, int nq_total, cudaStream_t s, const char* name) {
+  const size_t smem = ((size_t)kSimtHG * p.d + (size_t)kSimtKeys * (p.d + 1)) * sizeof(float);
+  cudaFuncSetAttribute(attn_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  dim3 grid((unsigned)nq_total, (unsigned)ceil_div64(p.H, kSimtHG), (unsigned)p.splits);
+  CSAHCA_TRACE(name, s);
+  attn_simt_kernel<T><<<grid, 32 * kSimtHG, smem, s>>>(p);
+  CSAHCA_CHECK_LAUNCH();
+  return CSAHCA_OK;
+}
+
+template <typename T>
+int run_prefill_t(const csahca_attn_args* a, cudaStream_t s) {
+  const double base = a->rope_base > 0 ? a->rope_base : kDefaultRopeBase;
+  const float eps = a->eps > 0 ? a->eps : kDefaultEps;
+  void* win_final = nullptr;
+  if (a->w > 0) {
+    win_final = a->workspace;
+    int st = launch_finish<T>(a->kv_win, win_final, a->kv_gain, (int64_t)a->B * a->n, a->d, 1,
+                              a->n, a->kv_norm, a->rope_dims, base, eps, s);
+    if (st != CSAHCA_OK) return st;
+  }
+  SimtAttnParams p;
+  memset(&p, 0, sizeof(p));
+  p.q = a->q; p.q_gain = a->q_gain; p.sinks = a->sinks; p.pos = nullptr;
+  p.q_norm = a->q_norm; p.eps = eps; p.scale = a->scale > 0 ? a->scale : 1.0f / sqrtf((float)a->d);
+  p.rope_dims = a->rope_dims; p.rope_base = base;
+  p.B = a->B; p.nq = a->n; p.H = a->H; p.d = a->d;
+  p.kv_comp = a->kv_comp; p.N = a->N;
+  p.idx = a->kind == CSAHCA_CSA ? a->idx : nullptr; p.k = a->k; p.m = a->m;
+  p.win = win_final; p.w = a->w; p.decode = 0;
+  p.splits = 1; p.keys_per_split = INT32_MAX / 2;
+  p.out = a->out; p.partial = nullptr;
+  return launch_simt_attn<T>(p, a->B * a->n, s,
+                             a->kind == CSAHCA_CSA ? "attn_prefill_csa_simt" : "attn_prefill_hca_simt");
+}
+
+int run_prefill(const csahca_attn_args* a, void* stream) {
+  int st = validate_attn(a);
+  if (st != CSAHCA_OK) return st;
+  if (a->B == 0 || a->n == 0) return CSAHCA_OK;
+  if ((st = device_ok()) != CSAHCA_OK) return st;
+  const size_t need = prefill_workspace(a);
+  if (need && (!a->workspace || a->workspace_bytes < need)) return CSAHCA_ERR_WORKSPACE;
+  if ((int64_t)a->B * a->n > INT32_MAX) return CSAHCA_ERR_UNSUPPORTED;
+  cudaStream_t s = as_stream(stream);
+  return a->dtype == CSAHCA_F32 ? run_prefill_t<float>(a, s) : run_prefill_t<__nv_bfloat16>(a, s);
+}
+
+// ------------------------------------------------------------------ decode --
+
+constexpr int kDecodeKeysPerSplit = 256;
+
+int validate_decode(const csahca_decode_args* a, bool shapes_only = false) {
+  if (!a) return CSAHCA_ERR_INVALID_ARG;
+  if (a->kind != CSAHCA_CSA && a->kind != CSAHCA_HCA) return CSAHCA_ERR_INVALID_ARG;
+  if (a->dtype != CSAHCA_F32 && a->dtype != CSAHCA_BF16) return CSAHCA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->H < 1 || a->d < 1 || a->N_cap < 0 || a->m < 1 || a->w < 0)
+    return CSAHCA_ERR_INVALID_ARG;
+  if (a->rope_dims < 0 || a->rope_dims > a->d || (a->rope_dims & 1)) return CSAHCA_ERR_INVALID_ARG;
+  if (a->d % 32 || a->d > 32 * kSimtMaxDPL) return CSAHCA_ERR_UNSUPPORTED;
+  if (a->kind == CSAHCA_CSA) {
+    if (a->k < 1) return CSAHCA_ERR_INVALID_ARG;
+    if (!a->idx_in) {
+      csahca_indexer_args ia;
+      memset(&ia, 0, sizeof(ia));
+      ia.q_dtype = a->qI_dtype; ia.k_dtype = a->kI_dtype; ia.B = a->B; ia.nq = 1; ia.HI = a->HI;
+      ia.dI = a->dI; ia.N = a->N_cap; ia.m = a->m; ia.k = a->k;
+      ia.qI = a->qI; ia.w = a->wI; ia.kI = a->kI; ia.kI_scale = a->kI_scale;
+      int st = validate_indexer(&ia, /*shapes_only=*/true);
+      if (st != CSAHCA_OK) return st;
+    }
+  }
+  if (shapes_only || a->B == 0) return CSAHCA_OK;
+  if (!a->q || !a->pos || !a->sinks || !a->out) return CSAHCA_ERR_INVALID_ARG;
+  if (a->kind == CSAHCA_CSA && !a->idx_in && (!a->qI || !a->wI || (a->N_cap > 0 && !a->kI) ||
+                                              (a->kI_dtype == CSAHCA_E4M3 && a->N_cap > 0 && !a->kI_scale)))
+    return CSAHCA_ERR_INVALID_ARG;
+  if (a->N_cap > 0 && !a->kv_cache) return CSAHCA_ERR_INVALID_ARG;
+  if (a->w > 0 && !a->win) return CSAHCA_ERR_INVALID_ARG;
+  const void* ptrs[] = {a->q, a->pos, a->q_gain, a->kv_cache, a->win, a->sinks, a->qI, a->wI,
+                        a->kI, a->kI_scale, a->idx_in, a->idx_out, a->out, a->workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return CSAHCA_ERR_ALIGNMENT;
+  return CSAHCA_OK;
+}
+
+struct DecodeLayout {
+  size_t scores_off, idx_off, partial_off, total;
+  int splits;
+};
+
+DecodeLayout decode_layout(const csahca_decode_args* a) {
+  DecodeLayout L;
+  const bool csa = a->kind == CSAHCA_CSA;
+  const bool run_indexer = csa && !a->idx_in;
+  const int64_t jmax = (csa ? (int64_t)a->k : (int64_t)a->N_cap) + a->w;
+  L.splits = (int)(jmax > 0 ? ceil_div64(jmax, kDecodeKeysPerSplit) : 1);
+  size_t off = 0;
+  L.scores_off = off;
+  if (run_indexer) off += align_up((size_t)a->B * (a->N_cap > 0 ? a->N_cap : 1) * 4, 256);
+  L.idx_off = off;
+  if (csa && !a->idx_out) off += align_up((size_t)a->B * a->k * 4, 256);
+  L.partial_off = off;
+  off += align_up((size_t)a->B * a->H * L.splits * (a->d + 2) * 4, 256);
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+int run_decode_t(const csahca_decode_args* a, cudaStream_t s, char* ws) {
+  const DecodeLayout L = decode_layout(a);
+  const double base = a->rope_base > 0 ? a->rope_base : kDefaultRopeBase;
+  const float eps = a->eps > 0 ? a->eps : kDefaultEps;
+  const int32_t* sel = nullptr;
+  if (a->kind == CSAHCA_CSA) {
+    if (a->idx_in) {
+      sel = a->idx_in;
+      if (a->idx_out)
+        cudaMemcpyAsync(a->idx_out, a->idx_in, (size_t)a->B * a->k * 4, cudaMemcpyDeviceToDevice, s);
+    } else {
+      int32_t* idx = a->idx_out ? a->idx_out : reinterpret_cast<int32_t*>(ws + L.idx_off);
+      csahca_indexer_args ia;
+      memset(&ia, 0, sizeof(ia));
+      ia.q_dtype = a->qI_dtype; ia.k_dtype = a->kI_dtype; ia.B = a->B; ia.nq = 1; ia.HI = a->HI;
+      ia.dI = a->dI; ia.N = a->N_cap; ia.m = a->m; ia.k = a->k;
+      ia.qI = a->qI; ia.w = a->wI; ia.kI = a->kI; ia.kI_scale = a->kI_scale;
+      ia.q_pos = a->pos; ia.idx = idx;
+      ia.workspace = ws + L.scores_off;
+      ia.workspace_bytes = L.idx_off - L.scores_off;
+      int st = run_indexer(&ia, s);
+      if (st != CSAHCA_OK) return st;
+      sel = idx;
+    }
+  }
+  SimtAttnParams p;
+  memset(&p, 0, sizeof(p));
+  p.q = a->q; p.q_gain = a->q_gain; p.sinks = a->sinks; p.pos = a->pos;
+  p.q_norm = a->q_norm; p.eps = eps; p.scale = a->scale > 0 ? a->scale : 1.0f / sqrtf((float)a->d);
+  p.rope_dims = a->rope_dims; p.rope_base = base;
+  p.B = a->B; p.nq = 1; p.H = a->H; p.d = a->d;
+  p.kv_comp = a->kv_cache; p.N = a->N_cap;
+  p.idx = sel; p.k = a->k; p.m = a->m;
+  p.win = a->win; p.w = a->w; p.decode = 1;
+  p.splits = L.splits; p.keys_per_split = kDecodeKeysPerSplit;
+  p.out = nullptr; p.partial = reinterpret_cast<float*>(ws + L.partial_off);
+  int st = launch_simt_attn<T>(p, a->B, s,
+                               a->kind == CSAHCA_CSA ? "attn_decode_csa_simt" : "attn_decode_hca_simt");
+  if (st != CSAHCA_OK) return st;
+  CombineParams c;
+  c.partial = p.partial; c.sinks = a->sinks; c.pos = a->pos; c.out = a->out;
+  c.B = a->B; c.nq = 1; c.H = a->H; c.d = a->d; c.splits = L.splits;
+  c.rope_dims = a->rope_dims; c.decode = 1; c.rope_base = base;
+  {
+    CSAHCA_TRACE("attn_combine", s);
+    attn_combine_kernel<T><<<(unsigned)(a->B * a->H), 256, 0, s>>>(c);
+  }
+  CSAHCA_CHECK_LAUNCH();
+  return CSAHCA_OK;
+}
+
+int run_decode(const csahca_decode_args* a, void* stream, char* ws, size_t ws_bytes) {
+  int st = validate_decode(a);
+  if (st != CSAHCA_OK) return st;
+  if (a->B == 0) return CSAHCA_OK;
+  if ((st = device_ok()) != CSAHCA_OK) return st;
+  const DecodeLayout L = decode_layout(a);
+  if (!ws || ws_bytes < L.total) return CSAHCA_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  return a->dtype == CSAHCA_F32 ? run_decode_t<float>(a, s, ws) : run_decode_t<__nv_bfloat16>(a, s, ws);
+}
+
+}  // namespace
+
+// ============================================================== C ABI ======
+
+extern "C" {
+
+int csa_compress(const csahca_compress_args* args, void* stream) { return run_compress(args, stream, true); }
+int hca_compress(const csahca_compress_args* args, void* stream) { return run_compress(args, stream, false); }
+
+int indexer_topk(const csahca_indexer_args* args, void* stream) { return run_indexer(args, stream); }
+
+size_t csahca_indexer_workspace_size(const csahca_indexer_args* args) {
+  if (validate_indexer(args, true) != CSAHCA_OK) return 0;
+  return indexer_workspace(args);
+}
+
+int compressed_attn_prefill(const csahca_attn_args* args, void* stream) { return run_prefill(args, stream); }
+
+size_t csahca_prefill_workspace_size(const csahca_attn_args* args) {
+  if (validate_attn(args, true) != CSAHCA_OK) return 0;
+  return prefill_workspace(args);
+}
+
+int compressed_attn_decode(const csahca_decode_args* args, void* stream) {
+  if (!args) return CSAHCA_ERR_INVALID_ARG;
+  return run_decode(args, stream, static_cast<char*>(args->workspace), args->workspace_bytes);
+}
+
+size_t csahca_decode_workspace_size(const csahca_decode_args* args) {
+  if (validate_decode(args, true) != CSAHCA_OK) return 0;
+  if (args->B == 0) return 0;
+  return decode_layout(args).total;
+}
+
+const char* csahca_status_string(int status) {
+  switch (status) {
+    case CSAHCA_OK: return "ok";
+    case CSAHCA_ERR_INVALID_ARG: return "invalid argument";
+    case CSAHCA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case CSAHCA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case CSAHCA_ERR_WORKSPACE: return "workspace missing or too small";
+    case CSAHCA_ERR_LAUNCH: return "CUDA launch or driver error";
+    case CSAHCA_ERR_DEVICE_TIMEOUT: return "a bounded device wait gave up";
+    case CSAHCA_ERR_NO_DEVICE: return "no sm_100 CUDA device";
+    default: return "unknown status";
+  }
+}
+
+int csahca_abi_version(void) { return CSAHCA_ABI_VERSION; }
+
+int64_t csahca_struct_size(int which) {
+  switch (which) {
+    case 0: return (int64_t)sizeof(csahca_compress_args);
+    case 1: return (int64_t)sizeof(csahca_indexer_args);
+    case 2: return (int64_t)sizeof(csahca_attn_args);
+    case 3: return (int64_t)sizeof(csahca_decode_args);
+    default: return -1;
+  }
+}
+
+int csahca_trace_enable(int enable) {
+  trace::g_enabled = enable != 0;
+  return CSAHCA_OK;
+}
+
+int csahca_trace_collect(csahca_trace_entry* out, int max_entries, int* n_entries) {
+  if (!n_entries || (max_entries > 0 && !out) || max_entries < 0) return CSAHCA_ERR_INVALID_ARG;
+  *n_entries = 0;
+  std::vector<csahca_trace_entry> acc;
+  int status = CSAHCA_OK;
+  for (const auto& r : trace::g_records) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.end) != cudaSuccess || cudaEventElapsedTime(&ms, r.begin, r.end) != cudaSuccess) {
+      (void)cudaGetLastError();
+      status = CSAHCA_ERR_LAUNCH;
+    }
+    size_t i = 0;
+    for (; i < acc.size(); ++i)
+      if (strncmp(acc[i].name, r.name, sizeof(acc[i].name)) == 0) break;
+    if (i == acc.size()) {
+      csahca_trace_entry e;
+      memset(&e, 0, sizeof(e));
+      strncpy(e.name, r.name, sizeof(e.name) - 1);
+      acc.push_back(e);
+    }
+    acc[i].launches += 1;
+    acc[i].total_ms += ms;
+    trace::g_pool.push_back(r.begin);
+    trace::g_pool.push_back(r.end);
+  }
+  trace::g_records.clear();
+  int n = 0;
+  for (; n < (int)acc.size() && n < max_entries; ++n) out[n] = acc[n];
+  *n_entries = n;
+  return status;
+}
+
+int csahca_device_error(void* stream, int32_t* code) {
+  if (!code) return CSAHCA_ERR_INVALID_ARG;
+  *code = 0;
+  cudaStream_t s = as_stream(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) { (void)cudaGetLastError(); return CSAHCA_ERR_LAUNCH; }
+  int32_t v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return CSAHCA_ERR_LAUNCH;
+  }
+  *code = v;
+  return CSAHCA_OK;
+}
+
+}  // extern "C"

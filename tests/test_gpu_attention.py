@@ -1,0 +1,111 @@
+"""GPU parity of compressed_attn_prefill against the float64 oracle
+("Paper Breakdown: DeepSeek-V4", section 4: MQA core attention, sliding
+window, HCA dense attention, attention sink, RMSNorm, partial RoPE; "Inside
+DeepSeek V4", "Local window")."""
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_compressed_overlapped_b200 import api, synth
+from oracle import csahca_oracle as O
+from tests.helpers import check_close, npy
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _sample(n, extra, seed=0, count=24):
+    rng = np.random.default_rng(seed)
+    s = np.unique(np.r_[extra, rng.integers(0, n, count)])
+    return s[(s >= 0) & (s < n)]
+
+
+def _prefill_layer(wl, n, B):
+    """Compressed rows (GPU compressor; both sides then read the same rows),
+    raw window rows and queries."""
+    inp = synth.prefill_inputs(wl, DEV, n=n, B=B)
+    kvi = inp["kv"]
+    m = wl.m if wl.kind == "csa" else wl.m_hca
+    if wl.kind == "csa":
+        kv = api.csa_compress(kvi["a"], kvi["b"], kvi["za"], kvi["zb"], kvi["bias_a"],
+                              kvi["bias_b"], m, gain=inp["kv_gain"], rope_dims=wl.r)
+    else:
+        kv = api.hca_compress(kvi["a"], kvi["za"], kvi["bias_a"], m, gain=inp["kv_gain"],
+                              rope_dims=wl.r)
+    return inp, kv, m
+
+
+def _oracle_rows(kind, inp, kv, idx, wl, m, b, rows):
+    return O.prefill_attention(kind, npy(inp["q"][b]), npy(kv[b]), npy(inp["kv_win"][b]),
+                               npy(inp["sinks"]), m=m, w=wl.w, r=wl.r,
+                               q_gain=npy(inp["q_gain"]), kv_gain=npy(inp["kv_gain"]),
+                               idx=None if idx is None else npy(idx[b]), rows=rows)
+
+
+def test_prefill_csa_tiny_f32():
+    """tiny_csa_f32 end to end on the GPU (compress -> indexer -> attention);
+    output parity uses the GPU's own index set on the oracle side."""
+    wl = synth.WORKLOADS["tiny_csa_f32"]
+    inp, kv, m = _prefill_layer(wl, wl.n, wl.B)
+    ik = inp["ik"]
+    kI = api.csa_compress(ik["a"], ik["b"], ik["za"], ik["zb"], ik["bias_a"], ik["bias_b"], m,
+                          rms_norm=False)
+    q_pos = torch.arange(wl.n, device=DEV, dtype=torch.int32)[None]
+    idx = api.indexer_topk(inp["qI"], inp["w"], kI, q_pos, m, wl.k)
+    out = api.compressed_attn_prefill("csa", inp["q"], kv, inp["kv_win"], inp["sinks"], m=m,
+                                      w=wl.w, rope_dims=wl.r, idx=idx, q_gain=inp["q_gain"],
+                                      kv_gain=inp["kv_gain"])
+    ref = _oracle_rows("csa", inp, kv, idx, wl, m, 0, np.arange(wl.n))
+    check_close(npy(out[0]), ref, "f32", "tiny csa prefill")
+    assert api.device_error() == 0
+
+
+def test_prefill_hca_8k_bf16_full_size():
+    """hca_8k_bf16 at full size (B = 2, n = 8192, H = 16, d = 128, m' = 128,
+    w = 128) on sampled queries, including t < m', t < w and t = n - 1."""
+    wl = synth.WORKLOADS["hca_8k_bf16"]
+    inp, kv, m = _prefill_layer(wl, wl.n, wl.B)
+    out = api.compressed_attn_prefill("hca", inp["q"], kv, inp["kv_win"], inp["sinks"], m=m,
+                                      w=wl.w, rope_dims=wl.r, q_gain=inp["q_gain"],
+                                      kv_gain=inp["kv_gain"])
+    for b in range(wl.B):
+        rows = _sample(wl.n, [0, 1, 126, 127, 128, 255, 256, wl.n - 1], seed=b)
+        ref = _oracle_rows("hca", inp, kv, None, wl, m, b, rows)
+        check_close(npy(out[b, rows]), ref, "bf16", f"hca b={b}")
+    assert api.device_error() == 0
+
+
+def test_prefill_csa_bf16_prefill_shapes():
+    """csa_prefill_128k head shapes (H = 64, d = 512, r = 64, k = 1024,
+    w = 128) at n = 4096 + 3, with the GPU's selection."""
+    wl = synth.WORKLOADS["csa_prefill_128k"]
+    n = 4096 + 3
+    inp, kv, m = _prefill_layer(wl, n, 1)
+    ik = inp["ik"]
+    kI = api.csa_compress(ik["a"], ik["b"], ik["za"], ik["zb"], ik["bias_a"], ik["bias_b"], m,
+                          rms_norm=False)
+    q_pos = torch.arange(n, device=DEV, dtype=torch.int32)[None]
+    idx = api.indexer_topk(inp["qI"], inp["w"], kI, q_pos, m, wl.k)
+    out = api.compressed_attn_prefill("csa", inp["q"], kv, inp["kv_win"], inp["sinks"], m=m,
+                                      w=wl.w, rope_dims=wl.r, idx=idx, q_gain=inp["q_gain"],
+                                      kv_gain=inp["kv_gain"])
+    rows = _sample(n, [0, 3, 4, 127, 128, 4095, 4096, n - 1], count=12)
+    ref = _oracle_rows("csa", inp, kv, idx, wl, m, 0, rows)
+    check_close(npy(out[0, rows]), ref, "bf16", "csa prefill")
+    assert api.device_error() == 0
+
+
+def test_prefill_no_window_no_sink_edge():
+    """w = 0 with the first queries (no visible entry): the output is 0 for
+    t < m - 1 (only the sink in the denominator)."""
+    wl = synth.WORKLOADS["hca_8k_bf16"]
+    inp, kv, m = _prefill_layer(wl, 512, 1)
+    out = api.compressed_attn_prefill("hca", inp["q"], kv, inp["kv_win"], inp["sinks"], m=m,
+                                      w=0, rope_dims=wl.r)
+    assert torch.count_nonzero(out[0, : m - 1]) == 0
+    rows = np.array([m - 1, m, 300, 511])
+    ref = O.prefill_attention("hca", npy(inp["q"][0]), npy(kv[0]), npy(inp["kv_win"][0]),
+                              npy(inp["sinks"]), m=m, w=0, r=wl.r, rows=rows)
+    check_close(npy(out[0, rows]), ref, "bf16", "hca w=0")
+    assert api.device_error() == 0

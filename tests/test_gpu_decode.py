@@ -1,0 +1,106 @@
+"""GPU parity of compressed_attn_decode (one decode step per layer; CSA with
+the lightning-indexer top-k, HCA dense; window ring and sink) against the
+float64 oracle ("Paper Breakdown: DeepSeek-V4", section 4; "How DeepSeek-V4
+architecture and training work together", "Two compressed views of one
+history": interleaved CSA / HCA layers, top-1,024 and a 128-token window)."""
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_compressed_overlapped_b200 import api, synth
+from oracle import csahca_oracle as O
+from tests.helpers import check_close, check_topk, npy
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _decode_layer(L, wl, idx_out=None, idx_in=None):
+    kw = dict(m=L["m"], rope_dims=wl.r, q_gain=L["q_gain"])
+    if L["kind"] == "csa":
+        kw.update(k=wl.k, qI=L["qI"], wI=L["w"], kI=L["kI"], kI_scale=L["kI_scale"],
+                  idx_out=idx_out, idx_in=idx_in)
+    return api.compressed_attn_decode(L["kind"], L["q"], L["pos"], L["kv"], L["win"], L["sinks"],
+                                      **kw)
+
+
+def _check_layer(L, wl, out, idx, seqs):
+    for b in seqs:
+        pos = int(L["pos"][b])
+        sel = None
+        if L["kind"] == "csa":
+            v = min(O.n_visible(pos, L["m"]), L["kv"].shape[1])
+            if L["kI_scale"] is not None:
+                K = O.dequant_e4m3_rows(npy(L["kI"][b, :v]), npy(L["kI_scale"][b, :v]))
+            else:
+                K = npy(L["kI"][b, :v])
+            s = O.indexer_scores(npy(L["qI"][b]), npy(L["w"][b]), K)
+            check_topk(npy(idx[b]), s, wl.k, f"{L['kind']} b={b}")
+            sel = npy(idx[b])
+        ref = O.decode_attention(L["kind"], npy(L["q"][b]), pos, npy(L["kv"][b]), npy(L["win"][b]),
+                                 npy(L["sinks"]), m=L["m"], w=wl.w, r=wl.r,
+                                 q_gain=npy(L["q_gain"]), sel=sel)
+        check_close(npy(out[b]), ref, wl.dtype, f"{L['kind']} b={b}")
+
+
+@pytest.mark.parametrize("wl_name,ctx", [("decode_256k", 16384 + 7), ("decode_1m", 32768 + 130)])
+def test_decode_layers(wl_name, ctx):
+    """Interleaved layers of decode_256k (bf16 keys) and decode_1m (e4m3
+    keys) at reduced context, positions including a ragged block tail."""
+    wl = synth.WORKLOADS[wl_name]
+    layers = synth.decode_inputs(wl, DEV, ctx=ctx, B=2)
+    for L in layers:
+        L["pos"] = torch.tensor([ctx, ctx - 200], device=DEV, dtype=torch.int32)
+        idx = torch.empty(2, wl.k, dtype=torch.int32, device=DEV) if L["kind"] == "csa" else None
+        out = _decode_layer(L, wl, idx_out=idx)
+        _check_layer(L, wl, out, idx, range(2))
+    assert api.device_error() == 0
+
+
+def test_decode_short_context_edges():
+    """pos < m - 1 (no entry visible), pos < w (partial window), visible <= k."""
+    wl = synth.WORKLOADS["decode_256k"]
+    layers = synth.decode_inputs(wl, DEV, ctx=4096, B=4)
+    for L in layers:
+        L["pos"] = torch.tensor([0, 2, 100, 4095], device=DEV, dtype=torch.int32)
+        idx = torch.empty(4, wl.k, dtype=torch.int32, device=DEV) if L["kind"] == "csa" else None
+        out = _decode_layer(L, wl, idx_out=idx)
+        _check_layer(L, wl, out, idx, range(4))
+    assert api.device_error() == 0
+
+
+def test_decode_tiny_f32():
+    """tiny_csa_f32 head shapes in fp32: tolerance 1e-5."""
+    wl = synth.WORKLOADS["tiny_csa_f32"]
+    wl = synth.Workload(**{**wl.__dict__, "layers": ("csa", "hca"), "m_hca": 16})
+    layers = synth.decode_inputs(wl, DEV, ctx=512, B=2)
+    for L in layers:
+        L["pos"] = torch.tensor([511, 300], device=DEV, dtype=torch.int32)
+        idx = torch.empty(2, wl.k, dtype=torch.int32, device=DEV) if L["kind"] == "csa" else None
+        out = _decode_layer(L, wl, idx_out=idx)
+        _check_layer(L, wl, out, idx, range(2))
+    assert api.device_error() == 0
+
+
+def test_decode_idx_in_matches_internal_selection():
+    wl = synth.WORKLOADS["decode_256k"]
+    L = synth.decode_inputs(wl, DEV, ctx=8192, B=2, layers=("csa",))[0]
+    idx = torch.empty(2, wl.k, dtype=torch.int32, device=DEV)
+    out1 = _decode_layer(L, wl, idx_out=idx)
+    out2 = _decode_layer(L, wl, idx_in=idx)
+    assert torch.equal(out1, out2)
+    assert api.device_error() == 0
+
+
+@pytest.mark.slow
+def test_decode_1m_full_size_one_sequence_checked():
+    """decode_1m at full context (1,048,576 tokens, 262,144 CSA entries with
+    e4m3 keys, 8,192 HCA entries), all four layers; sequence 0 checked."""
+    wl = synth.WORKLOADS["decode_1m"]
+    layers = synth.decode_inputs(wl, DEV)
+    for L in layers:
+        idx = torch.empty(wl.B, wl.k, dtype=torch.int32, device=DEV) if L["kind"] == "csa" else None
+        out = _decode_layer(L, wl, idx_out=idx)
+        _check_layer(L, wl, out, idx, [0])
+    assert api.device_error() == 0
