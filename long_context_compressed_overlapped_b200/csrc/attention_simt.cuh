@@ -32,9 +32,9 @@ struct SimtAttnParams {
   int decode;
   // split-KV
   int splits, keys_per_split;
-  // outputs
-  void* out;                         // final [B, nq, H, d] (splits == 1)
-  float* partial;                    // [B, nq, H, splits, d + 2] (splits > 1)
+  // outputs: partial == NULL -> final rows in out (one split); else partials
+  void* out;                         // final [B, nq, H, d]
+  float* partial;                    // [B, nq, H, splits, d + 2]
 };
 
 template <typename T>
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(32 * kSimtHG) attn_simt_kernel(SimtAttnParams 
   }
   if (h >= p.H) return;
 
-  if (p.splits == 1) {
+  if (p.partial == nullptr) {
     // final: o = acc / (e^{z} + lsum) in the max-shifted frame, rope dims back by -t
     const float z = p.sinks[h];
     const float M = fmaxf(mx, z);

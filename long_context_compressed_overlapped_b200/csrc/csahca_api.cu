@@ -2,6 +2,7 @@
 // validation, workspace sizing and kernel dispatch; every step of the path
 // runs in the kernels included below.
 #include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
@@ -14,6 +15,7 @@
 #include "indexer_simt.cuh"
 #include "topk.cuh"
 #include "attention_simt.cuh"
+#include "indexer_tc.cuh"
 
 using namespace csahca;
 
@@ -70,6 +72,44 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
       return CSAHCA_ERR_LAUNCH;                                \
     }                                                          \
   } while (0)
+
+// ---- device facts and TMA descriptors -------------------------------------
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+    return n;
+  (void)cudaGetLastError();
+  return 148;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// 2D row-major tensor [rows, inner] of `dt`, box [box_rows, box_inner].
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* ptr, uint64_t inner,
+               uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(inner * elem_bytes)};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 int dtype_size(int dt) {
   switch (dt) {
@@ -199,6 +239,60 @@ void launch_indexer_simt(const IndexerParams& p, cudaStream_t s) {
   indexer_scores_simt<TQ, TK, kFP8><<<grid, 256, smem, s>>>(p);
 }
 
+bool indexer_tc_eligible(const csahca_indexer_args* a) {
+  return a->q_dtype == CSAHCA_BF16 && (a->k_dtype == CSAHCA_BF16 || a->k_dtype == CSAHCA_E4M3) &&
+         a->HI == 64 && a->dI == kIdxTcDim && a->N > 0;
+}
+
+template <int QT, bool kFP8>
+int launch_indexer_tc_t(const csahca_indexer_args* a, IdxTcParams p, cudaStream_t s) {
+  using Cfg = IdxTcCfg<QT, 64, kFP8>;
+  CUtensorMap kmap, qmap;
+  bool ok;
+  if (kFP8)
+    ok = encode_2d(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->kI, (uint64_t)a->dI, (uint64_t)a->B * a->N, 128, 128,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+  else
+    ok = encode_2d(&kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a->kI, (uint64_t)a->dI, (uint64_t)a->B * a->N, 64,
+                   128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && encode_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a->qI, (uint64_t)a->dI,
+                       (uint64_t)a->B * a->nq * a->HI, 64, (uint32_t)Cfg::NCOL, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return CSAHCA_ERR_LAUNCH;
+  auto kern = indexer_tc_kernel<QT, 64, kFP8>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+  if (grid <= 0) return CSAHCA_OK;
+  CSAHCA_TRACE(QT == 1 ? "indexer_scores_tc_decode" : "indexer_scores_tc_prefill", s);
+  kern<<<grid, kIdxTcThreads, Cfg::SMEM, s>>>(kmap, qmap, p);
+  CSAHCA_CHECK_LAUNCH();
+  return CSAHCA_OK;
+}
+
+// Tensor-core scores for queries [q0, q0 + qc) into scores (row stride N).
+int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* scores, int64_t stride,
+                      cudaStream_t s) {
+  IdxTcParams p;
+  memset(&p, 0, sizeof(p));
+  p.w = a->w; p.kI_scale = a->kI_scale; p.q_pos = a->q_pos;
+  p.scores = scores; p.score_row_stride = stride;
+  p.B = a->B; p.nq = a->nq; p.HI = a->HI; p.N = a->N; p.m = a->m;
+  p.q_begin = q0; p.q_count = qc;
+  const bool fp8 = a->k_dtype == CSAHCA_E4M3;
+  if (qc == 1) {
+    const int tiles = (int)ceil_div64(a->N, 128);
+    int splits = (int)ceil_div64(2 * num_sms(), a->B);
+    if (splits > tiles) splits = tiles;
+    if (splits < 1) splits = 1;
+    p.tiles_per_split = (int)ceil_div64(tiles, splits);
+    p.splits = (int)ceil_div64(tiles, p.tiles_per_split);
+    p.n_items = a->B * p.splits;
+    return fp8 ? launch_indexer_tc_t<1, true>(a, p, s) : launch_indexer_tc_t<1, false>(a, p, s);
+  }
+  p.splits = 0;
+  p.n_items = a->B * (int)ceil_div64(qc, 4);
+  return fp8 ? launch_indexer_tc_t<4, true>(a, p, s) : launch_indexer_tc_t<4, false>(a, p, s);
+}
+
 int run_indexer(const csahca_indexer_args* a, void* stream) {
   int st = validate_indexer(a);
   if (st != CSAHCA_OK) return st;
@@ -230,7 +324,12 @@ int run_indexer(const csahca_indexer_args* a, void* stream) {
         pb.q_pos = a->q_pos + (int64_t)b * a->nq;
         pb.scores = a->scores_out + ((int64_t)b * a->nq + q0) * stride;
         pb.score_row_stride = stride;
-        if (a->N > 0) {
+        if (indexer_tc_eligible(a)) {
+          csahca_indexer_args ab = *a;
+          ab.B = 1; ab.qI = pb.qI; ab.w = pb.w; ab.kI = pb.kI; ab.kI_scale = pb.kI_scale; ab.q_pos = pb.q_pos;
+          int st2 = launch_indexer_tc(&ab, q0, qc, pb.scores, stride, s);
+          if (st2 != CSAHCA_OK) return st2;
+        } else if (a->N > 0) {
           if (a->k_dtype == CSAHCA_E4M3) {
             if (a->q_dtype == CSAHCA_BF16) launch_indexer_simt<__nv_bfloat16, uint8_t, true>(pb, s);
             else launch_indexer_simt<float, uint8_t, true>(pb, s);
@@ -257,7 +356,10 @@ int run_indexer(const csahca_indexer_args* a, void* stream) {
     base = static_cast<float*>(a->workspace);
     p.scores = base;
     p.score_row_stride = stride;
-    if (a->N > 0) {
+    if (indexer_tc_eligible(a)) {
+      int st2 = launch_indexer_tc(a, q0, qc, base, stride, s);
+      if (st2 != CSAHCA_OK) return st2;
+    } else if (a->N > 0) {
       if (a->k_dtype == CSAHCA_E4M3) {
         if (a->q_dtype == CSAHCA_BF16) launch_indexer_simt<__nv_bfloat16, uint8_t, true>(p, s);
         else launch_indexer_simt<float, uint8_t, true>(p, s);

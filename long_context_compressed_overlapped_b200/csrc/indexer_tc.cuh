@@ -1,0 +1,289 @@
+// Lightning-indexer scores on the tensor cores ("Paper Breakdown: DeepSeek-V4",
+// section 4, DSA on Compressed KV):  I_{t,i} = sum_j w_{t,j} ReLU(qI_{t,j} . kI_i).
+//
+// One 128-key tile of compressed indexer keys is the M = 128 operand (A,
+// K-major, SW128); the QT queries x HI heads of a work item are the N operand
+// (B, QT*HI <= 256 rows); K = dI = 128.  The fp32 accumulator sits in TMEM
+// with one key per lane, so the ReLU and the weighted sum over heads are
+// thread-local in the epilogue: thread i of the 4 epilogue warps reads the
+// QT*HI columns of lane i and writes QT scores of key i.
+//
+// Roles (320 threads): warps 0-3 epilogue, warp 4 TMA producer, warp 5 MMA
+// issuer (and TMEM owner), warps 6-9 convert e4m3 key tiles to bf16 (exact)
+// when the keys are stored in e4m3; for e4m3 keys the per-row fp32 scale is
+// applied to the score (a positive per-row factor commutes with ReLU).
+//
+// Work items: prefill = (sequence, tile of QT queries, every key tile any of
+// its queries can see), longest first; decode = (sequence, contiguous range of
+// key tiles).  CTAs stride over the item list.
+#pragma once
+#include "tc_common.cuh"
+
+namespace csahca {
+
+constexpr int kIdxTcThreads = 320;
+constexpr int kIdxTcDim = 128;       // dI handled by the tensor-core path
+
+struct IdxTcParams {
+  const float* w; const float* kI_scale; const int* q_pos;
+  float* scores; int64_t score_row_stride;
+  int B, nq, HI, N, m;
+  int q_begin, q_count;
+  int n_items;
+  int splits;                 // > 0: decode items (b, split); 0: prefill items (b, query tile)
+  int tiles_per_split;
+};
+
+template <int QT, int HI, bool kFP8>
+struct IdxTcCfg {
+  static constexpr int NCOL = QT * HI;                          // MMA N
+  static constexpr int NSTAGE = kFP8 ? 4 : 4;
+  static constexpr int NACC = (512 / NCOL) > 4 ? 4 : (512 / NCOL);
+  static constexpr int TMEM_COLS = NCOL * NACC <= 32 ? 32 : (NCOL * NACC <= 64 ? 64 : (NCOL * NACC <= 128 ? 128 : (NCOL * NACC <= 256 ? 256 : 512)));
+  static constexpr int B_CHUNK = NCOL * 128;                    // bytes per 64-dim chunk of B
+  static constexpr int B_BYTES = 2 * B_CHUNK;
+  static constexpr int A_BYTES = 2 * 128 * 128;                 // 128 keys x 128 dims bf16
+  static constexpr int RAW_BYTES = kFP8 ? 128 * 128 : 0;        // 128 keys x 128 e4m3
+  static constexpr int SMEM = 1024 + B_BYTES + NSTAGE * (A_BYTES + RAW_BYTES) + QT * HI * 4 + 1024;
+  static_assert(NCOL % 16 == 0 && NCOL <= 256, "MMA N");
+  static_assert(HI % 32 == 0, "heads per query must be a multiple of 32");
+};
+
+struct IdxItem { int b, q0, qn, kt0, kt1; };
+
+__device__ __forceinline__ int idx_visible(const IdxTcParams& p, int b, int q) {
+  const int t = p.q_pos[(int64_t)b * p.nq + q];
+  if (t < 0) return 0;
+  const int64_t v = ((int64_t)t + 1) / p.m;
+  return (int)(v < p.N ? v : p.N);
+}
+
+template <int QT>
+__device__ __forceinline__ IdxItem idx_item(const IdxTcParams& p, int id) {
+  IdxItem it;
+  if (p.splits > 0) {
+    it.b = id / p.splits;
+    const int sp = id % p.splits;
+    it.q0 = p.q_begin; it.qn = 1;
+    const int v = idx_visible(p, it.b, it.q0);
+    const int nt = (v + 127) / 128;
+    it.kt0 = sp * p.tiles_per_split;
+    it.kt1 = min(nt, it.kt0 + p.tiles_per_split);
+  } else {
+    const int nqt = (p.q_count + QT - 1) / QT;
+    const int r = id / p.B;
+    it.b = id % p.B;
+    const int qt = nqt - 1 - r;                       // longest (latest) query tiles first
+    it.q0 = p.q_begin + qt * QT;
+    it.qn = min(QT, p.q_begin + p.q_count - it.q0);
+    int vmax = 0;
+    for (int q = 0; q < it.qn; ++q) vmax = max(vmax, idx_visible(p, it.b, it.q0 + q));
+    it.kt0 = 0;
+    it.kt1 = (vmax + 127) / 128;
+  }
+  return it;
+}
+
+template <int QT, int HI, bool kFP8>
+__global__ void __launch_bounds__(kIdxTcThreads, 1)
+indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                  IdxTcParams p) {
+  using Cfg = IdxTcCfg<QT, HI, kFP8>;
+  constexpr int NS = Cfg::NSTAGE, NACC = Cfg::NACC, NCOL = Cfg::NCOL;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sB = base;
+  uint8_t* sA = sB + Cfg::B_BYTES;
+  uint8_t* sRaw = sA + NS * Cfg::A_BYTES;
+  float* sW = reinterpret_cast<float*>(sRaw + NS * Cfg::RAW_BYTES);
+  __shared__ uint64_t bar_a_full[NS], bar_a_empty[NS], bar_raw_full[NS], bar_raw_empty[NS];
+  __shared__ uint64_t bar_acc_full[NACC], bar_acc_empty[NACC];
+  __shared__ uint64_t bar_b_full, bar_b_empty, bar_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bar_a_full[s], kFP8 ? 128 : 1);
+      mbar_init(&bar_a_empty[s], 1);
+      mbar_init(&bar_raw_full[s], 1);
+      mbar_init(&bar_raw_empty[s], 128);
+    }
+    for (int j = 0; j < NACC; ++j) { mbar_init(&bar_acc_full[j], 1); mbar_init(&bar_acc_empty[j], 128); }
+    mbar_init(&bar_b_full, 1);
+    mbar_init(&bar_b_empty, 1);
+    mbar_init(&bar_done, 1);
+    mbar_fence_init();
+  }
+  if (warp == 5) tmem_alloc(&tmem_base_sh, Cfg::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&qmap);
+      uint32_t a_iter = 0, b_iter = 0;
+      for (int id = blockIdx.x; id < p.n_items && !abort_flag; id += gridDim.x) {
+        const IdxItem it = idx_item<QT>(p, id);
+        if (it.kt1 <= it.kt0) continue;
+        if (!mbar_wait(&bar_b_empty, (b_iter & 1) ^ 1, &abort_flag)) break;
+        mbar_expect_tx(&bar_b_full, Cfg::B_BYTES);
+        const int qrow = (it.b * p.nq + it.q0) * HI;
+        tma_load_2d(sB, &qmap, 0, qrow, &bar_b_full);
+        tma_load_2d(sB + Cfg::B_CHUNK, &qmap, 64, qrow, &bar_b_full);
+        ++b_iter;
+        for (int kt = it.kt0; kt < it.kt1; ++kt, ++a_iter) {
+          const int s = a_iter % NS;
+          const uint32_t ph = (a_iter / NS) & 1;
+          const int krow = it.b * p.N + kt * 128;
+          if (kFP8) {
+            if (!mbar_wait(&bar_raw_empty[s], ph ^ 1, &abort_flag)) break;
+            mbar_expect_tx(&bar_raw_full[s], Cfg::RAW_BYTES);
+            tma_load_2d(sRaw + s * Cfg::RAW_BYTES, &kmap, 0, krow, &bar_raw_full[s]);
+          } else {
+            if (!mbar_wait(&bar_a_empty[s], ph ^ 1, &abort_flag)) break;
+            mbar_expect_tx(&bar_a_full[s], Cfg::A_BYTES);
+            tma_load_2d(sA + s * Cfg::A_BYTES, &kmap, 0, krow, &bar_a_full[s]);
+            tma_load_2d(sA + s * Cfg::A_BYTES + 16384, &kmap, 64, krow, &bar_a_full[s]);
+          }
+        }
+      }
+      // drain: every issued fill has landed before the CTA may exit
+      for (uint32_t i = (a_iter > NS ? a_iter - NS : 0); i < a_iter; ++i) {
+        const int s = i % NS;
+        const uint32_t ph = (i / NS) & 1;
+        if (kFP8) mbar_wait(&bar_raw_full[s], ph, &abort_flag);
+        else mbar_wait(&bar_a_full[s], ph, &abort_flag);
+      }
+      if (b_iter) mbar_wait(&bar_b_full, (b_iter - 1) & 1, &abort_flag);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(128, NCOL, 0, 0);
+      uint32_t a_iter = 0, b_iter = 0, acc_iter = 0;
+      const uint32_t sA0 = smem_u32(sA), sB0 = smem_u32(sB);
+      for (int id = blockIdx.x; id < p.n_items && !abort_flag; id += gridDim.x) {
+        const IdxItem it = idx_item<QT>(p, id);
+        if (it.kt1 <= it.kt0) continue;
+        if (!mbar_wait(&bar_b_full, b_iter & 1, &abort_flag)) break;
+        ++b_iter;
+        for (int kt = it.kt0; kt < it.kt1; ++kt, ++a_iter, ++acc_iter) {
+          const int s = a_iter % NS;
+          const uint32_t ph = (a_iter / NS) & 1;
+          const int j = acc_iter % NACC;
+          const uint32_t aph = (acc_iter / NACC) & 1;
+          if (!mbar_wait(&bar_a_full[s], ph, &abort_flag)) break;
+          if (!mbar_wait(&bar_acc_empty[j], aph ^ 1, &abort_flag)) break;
+          tc_fence_after();
+          const uint32_t d = tmem + j * NCOL;
+#pragma unroll
+          for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              umma_bf16(d, umma_desc_kmajor(sA0 + s * Cfg::A_BYTES + kc * 16384 + ks * 32),
+                        umma_desc_kmajor(sB0 + kc * Cfg::B_CHUNK + ks * 32), idesc, (kc | ks) != 0);
+          umma_commit(&bar_a_empty[s]);
+          umma_commit(&bar_acc_full[j]);
+        }
+        umma_commit(&bar_b_empty);
+      }
+      umma_commit(&bar_done);
+      mbar_wait(&bar_done, 0, &abort_flag);
+    }
+  } else if (warp >= 6) {
+    // ------------------------------------------------------------ e4m3 -> bf16
+    if (kFP8) {
+      const int ct = threadIdx.x - 192;                 // 0..127
+      uint32_t a_iter = 0;
+      for (int id = blockIdx.x; id < p.n_items && !abort_flag; id += gridDim.x) {
+        const IdxItem it = idx_item<QT>(p, id);
+        for (int kt = it.kt0; kt < it.kt1; ++kt, ++a_iter) {
+          const int s = a_iter % NS;
+          const uint32_t ph = (a_iter / NS) & 1;
+          if (!mbar_wait(&bar_raw_full[s], ph, &abort_flag)) break;
+          if (!mbar_wait(&bar_a_empty[s], ph ^ 1, &abort_flag)) break;
+          const uint8_t* raw = sRaw + s * Cfg::RAW_BYTES;
+          uint8_t* dst = sA + s * Cfg::A_BYTES;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int piece = ct + 128 * i;             // 16-byte piece of the raw tile
+            const int row = piece >> 3, pin = piece & 7;
+            const uint4 v = *reinterpret_cast<const uint4*>(raw + piece * 16);
+            const uint16_t* h = reinterpret_cast<const uint16_t*>(&v);
+            uint4 o0, o1;
+            o0.x = e4m3x2_to_bf16x2(h[0]); o0.y = e4m3x2_to_bf16x2(h[1]);
+            o0.z = e4m3x2_to_bf16x2(h[2]); o0.w = e4m3x2_to_bf16x2(h[3]);
+            o1.x = e4m3x2_to_bf16x2(h[4]); o1.y = e4m3x2_to_bf16x2(h[5]);
+            o1.z = e4m3x2_to_bf16x2(h[6]); o1.w = e4m3x2_to_bf16x2(h[7]);
+            // elements pin*16 .. pin*16+15 of the row: chunk pin/4, bytes (pin%4)*32 ..
+            uint8_t* chunk = dst + (pin >> 2) * 16384;
+            const int byte = (pin & 3) * 32;
+            *reinterpret_cast<uint4*>(chunk + sw128_offset(row, byte)) = o0;
+            *reinterpret_cast<uint4*>(chunk + sw128_offset(row, byte + 16)) = o1;
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&bar_a_full[s]);
+          mbar_arrive(&bar_raw_empty[s]);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 0-3)
+    const int et = threadIdx.x;                         // key lane 0..127
+    uint32_t acc_iter = 0;
+    bool stop = false;                                  // uniform over the 128 threads
+    for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
+      const IdxItem it = idx_item<QT>(p, id);
+      if (it.kt1 <= it.kt0) continue;
+      named_sync128();
+      for (int x = et; x < QT * HI; x += 128) {
+        const int q = x / HI;
+        sW[x] = q < it.qn ? p.w[((int64_t)it.b * p.nq + it.q0 + q) * HI + (x % HI)] : 0.f;
+      }
+      named_sync128();
+      int vq[QT];
+#pragma unroll
+      for (int q = 0; q < QT; ++q) vq[q] = q < it.qn ? idx_visible(p, it.b, it.q0 + q) : 0;
+      for (int kt = it.kt0; kt < it.kt1; ++kt, ++acc_iter) {
+        const int j = acc_iter % NACC;
+        const uint32_t aph = (acc_iter / NACC) & 1;
+        if (!mbar_wait128(&bar_acc_full[j], aph, &abort_flag)) { stop = true; break; }
+        tc_fence_after();
+        const int key = kt * 128 + et;
+        float scale = 1.f;
+        if (kFP8 && key < p.N) scale = __ldg(p.kI_scale + (int64_t)it.b * p.N + key);
+        const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + j * NCOL;
+#pragma unroll
+        for (int q = 0; q < QT; ++q) {
+          float acc = 0.f;
+#pragma unroll
+          for (int c = 0; c < HI / 32; ++c) {
+            float v[32];
+            tmem_ld32(tbase + q * HI + c * 32, v);
+            tmem_wait_ld();
+            const float* wq = sW + q * HI + c * 32;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) acc = fmaf(wq[e], fmaxf(v[e], 0.f), acc);
+          }
+          if (key < vq[q])
+            p.scores[((int64_t)it.b * p.q_count + (it.q0 + q - p.q_begin)) * p.score_row_stride + key] = acc * scale;
+        }
+        tc_fence_before();
+        mbar_arrive(&bar_acc_empty[j]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem, Cfg::TMEM_COLS);
+}
+
+}  // namespace csahca
