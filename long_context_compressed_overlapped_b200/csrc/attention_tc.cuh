@@ -1,0 +1,514 @@
+// Sink attention on the tensor cores ("Paper Breakdown: DeepSeek-V4", section
+// 4: MQA core attention over selected compressed entries (CSA) or every
+// visible entry (HCA), plus the uncompressed sliding window and a per-head
+// sink; query RMSNorm and partial RoPE; "Inside DeepSeek V4", "Local window").
+//
+// MQA: all H heads of a query share the key rows, and K = V.  Both products
+// are written transposed so that every MMA has M = 128 and one operand copy
+// serves both:
+//   S^T [128 keys x H]  = K [128 keys x D]  . Q^T      (A = key tile, K-major)
+//   O^T [D x H]        += V^T [D x 128 keys] . P^T     (A = the SAME key tile
+//                                                       read MN-major; B = P^T)
+// S^T lives in TMEM (H columns); O^T in TMEM as D/128 M-tiles of H columns.
+// Thread i of the 4 softmax warps owns key slot i of S^T and dim slot i of
+// each O^T M-tile.  Per-head max and sum over the 128 keys are warp
+// transpose-reductions (62 shuffles) plus a 4-way shared-memory step; the
+// running max is raised lazily (only when a head's tile max exceeds it by
+// more than 2^8), so O^T is rescaled in TMEM rarely.
+//
+// Roles (192 threads): warps 0-3 query prologue, softmax, epilogue; warp 4
+// TMA producer (4-row gathers for selected entries, 2D tiles for contiguous
+// rows); warp 5 MMA issuer and TMEM owner.  Key tiles arrive in 8 chunks of
+// 64 dims with their own barriers; chunk pair (2j, 2j+1) is released as soon
+// as the P.V of O^T M-tile j has read it, so the next tile's loads overlap
+// the tail of the current one.
+//
+// Work items: prefill = one query (all its tiles, final output); decode = one
+// query x a range of its tiles (partial max / sum / O for the combine).
+#pragma once
+#include "tc_common.cuh"
+
+namespace csahca {
+
+constexpr int kAttnTcThreads = 192;
+constexpr int kAttnH = 64;          // heads (MMA N of both products)
+constexpr int kAttnD = 512;         // head dim
+constexpr int kAttnChunks = kAttnD / 64;
+constexpr int kAttnMT = kAttnD / 128;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+struct AttnTcParams {
+  const __nv_bfloat16* q; const float* q_gain; const float* sinks; const int* pos;
+  int q_norm; float eps; float scale_log2; int rope_dims; double rope_base;
+  int B, nq, N, m, k, w;
+  int csa;                      // 1: keys = idx rows; 0: every visible entry
+  const int* idx;               // [B, nq, k]
+  int decode;                   // window = ring [B, w, d] (decode) or finished rows [B, nq, d]
+  int n_items, splits, tiles_per_split;
+  __nv_bfloat16* out;           // final [B, nq, H, D]
+  float* partial;               // [B, nq, H, splits, D + 2]
+};
+
+struct AttnItem { int b, qi, t, tile0, tile1, split, ncomp_tiles, nwin_tiles; };
+struct AttnTile { int src; int row0; int lo, hi; int list_off; };   // src 0 gather, 1 comp rows, 2 window rows
+
+__device__ __forceinline__ int attn_visible(const AttnTcParams& p, int t) {
+  if (t < 0) return 0;
+  const int64_t v = ((int64_t)t + 1) / p.m;
+  return (int)(v < p.N ? v : p.N);
+}
+
+__device__ __forceinline__ AttnItem attn_item(const AttnTcParams& p, int id) {
+  AttnItem it;
+  int qid;
+  if (p.decode) { qid = id / p.splits; it.split = id % p.splits; }
+  else {
+    // HCA prefill: latest queries (most tiles) first; CSA: all alike.
+    qid = p.csa ? id : (p.n_items - 1 - id);
+    it.split = 0;
+  }
+  it.b = qid / p.nq;
+  it.qi = qid % p.nq;
+  it.t = p.decode ? p.pos[it.b] : it.qi;
+  const int ncomp = p.csa ? p.k : attn_visible(p, it.t);
+  it.ncomp_tiles = (ncomp + 127) / 128;
+  it.nwin_tiles = (p.w + 127) / 128;
+  const int total = it.ncomp_tiles + it.nwin_tiles;
+  if (p.decode) {
+    it.tile0 = it.split * p.tiles_per_split;
+    it.tile1 = min(total, it.tile0 + p.tiles_per_split);
+  } else {
+    it.tile0 = 0;
+    it.tile1 = total;
+  }
+  return it;
+}
+
+__device__ __forceinline__ AttnTile attn_tile(const AttnTcParams& p, const AttnItem& it, int tile) {
+  AttnTile T;
+  if (tile < it.ncomp_tiles) {
+    if (p.csa) {
+      T.src = 0;
+      T.list_off = tile * 128;
+      T.row0 = 0;
+      T.lo = 0;
+      T.hi = min(128, p.k - tile * 128);
+    } else {
+      T.src = 1;
+      T.row0 = it.b * p.N + tile * 128;
+      T.lo = 0;
+      T.hi = min(128, attn_visible(p, it.t) - tile * 128);
+      T.list_off = 0;
+    }
+  } else {
+    const int wt = tile - it.ncomp_tiles;
+    T.src = 2;
+    T.list_off = 0;
+    if (p.decode) {
+      // ring slots [wt*128, wt*128 + 128); slot s is valid iff it holds a
+      // position in [pos - w + 1, pos] that is >= 0
+      T.row0 = it.b * p.w + wt * 128;
+      T.lo = 0;
+      const int nslot = min(128, p.w - wt * 128);
+      T.hi = (it.t >= p.w - 1) ? nslot : max(0, min(nslot, it.t + 1 - wt * 128));
+    } else {
+      // positions [t - w + 1 + wt*128, ...] clipped to [0, t]
+      const int p0 = it.t - p.w + 1 + wt * 128;
+      T.row0 = it.b * p.nq + p0;
+      T.lo = p0 < 0 ? -p0 : 0;
+      T.hi = min(128, min(p.w - wt * 128, it.t - p0 + 1));
+    }
+  }
+  return T;
+}
+
+// 64 per-thread values -> per-head reduction over the 128 threads of warps
+// 0-3.  Returns in out[64] (shared).  kMax: max, else sum.
+template <bool kMax>
+__device__ __forceinline__ void reduce_heads(float (&v)[kAttnH], float* red, float* out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
+#pragma unroll
+    for (int j = 0; j < n; ++j) {
+      const bool hi = lane & o;
+      const float keep = hi ? v[n + j] : v[j];
+      const float send = hi ? v[j] : v[n + j];
+      const float got = __shfl_xor_sync(0xffffffffu, send, o);
+      v[j] = kMax ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  red[warp * kAttnH + 2 * lane] = v[0];
+  red[warp * kAttnH + 2 * lane + 1] = v[1];
+  named_sync128();
+  if (threadIdx.x < kAttnH) {
+    const int h = threadIdx.x;
+    float r = red[h];
+#pragma unroll
+    for (int w = 1; w < 4; ++w) r = kMax ? fmaxf(r, red[w * kAttnH + h]) : r + red[w * kAttnH + h];
+    out[h] = r;
+  }
+  named_sync128();
+}
+
+// S^T row of this thread (64 heads) from TMEM, scaled to log2 units; -inf
+// for a masked key.
+__device__ __forceinline__ void load_scores(uint32_t taddr, bool valid, float scale_log2, float (&s)[kAttnH]) {
+  float v[32];
+  tmem_ld32(taddr, v);
+  tmem_wait_ld();
+#pragma unroll
+  for (int e = 0; e < 32; ++e) s[e] = valid ? v[e] * scale_log2 : -INFINITY;
+  tmem_ld32(taddr + 32, v);
+  tmem_wait_ld();
+#pragma unroll
+  for (int e = 0; e < 32; ++e) s[32 + e] = valid ? v[e] * scale_log2 : -INFINITY;
+}
+
+struct AttnSmem {
+  static constexpr int Q_CHUNK = kAttnH * 128;               // 8 KB
+  static constexpr int Q_BYTES = kAttnChunks * Q_CHUNK;      // 64 KB
+  static constexpr int K_CHUNK = 128 * 128;                  // 16 KB
+  static constexpr int K_BYTES = kAttnChunks * K_CHUNK;      // 128 KB
+  static constexpr int P_BYTES = 128 * 128;                  // 16 KB
+  static constexpr int TOTAL = 1024 + Q_BYTES + K_BYTES + P_BYTES;
+};
+
+__global__ void __launch_bounds__(kAttnTcThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_constant__ CUtensorMap comp_gather,
+               const __grid_constant__ CUtensorMap win_rows, AttnTcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = base;
+  uint8_t* sK = sQ + AttnSmem::Q_BYTES;
+  uint8_t* sP = sK + AttnSmem::K_BYTES;
+  __shared__ uint64_t bar_kfull[kAttnChunks], bar_kempty[kAttnChunks];
+  __shared__ uint64_t bar_q_full, bar_s_full, bar_s_empty, bar_p_full, bar_pv_done, bar_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+  __shared__ float red[4 * kAttnH];
+  __shared__ float stat_a[kAttnH], stat_b[kAttnH];
+  __shared__ float m_use[kAttnH], alpha[kAttnH], l_run[kAttnH];
+  __shared__ float rope_cs[64], rope_sn[64];
+  __shared__ int need_rescale;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int c = 0; c < kAttnChunks; ++c) { mbar_init(&bar_kfull[c], 1); mbar_init(&bar_kempty[c], 1); }
+    mbar_init(&bar_q_full, 128);
+    mbar_init(&bar_s_full, 1);
+    mbar_init(&bar_s_empty, 128);
+    mbar_init(&bar_p_full, 128);
+    mbar_init(&bar_pv_done, 1);
+    mbar_init(&bar_done, 1);
+    mbar_fence_init();
+  }
+  if (warp == 5) tmem_alloc(&tmem_base_sh, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const uint32_t tS = tmem;                 // S^T: columns [0, H)
+  const uint32_t tO = tmem + 128;           // O^T M-tile j: columns [128 + j*H, ...)
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    tma_prefetch_desc(&comp_rows);
+    tma_prefetch_desc(&comp_gather);
+    tma_prefetch_desc(&win_rows);
+    uint32_t tcount = 0;
+    bool stop = false;                       // warp-uniform
+    for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
+      const AttnItem it = attn_item(p, id);
+      for (int tile = it.tile0; tile < it.tile1 && !stop; ++tile, ++tcount) {
+        const AttnTile T = attn_tile(p, it, tile);
+        const uint32_t ph = tcount & 1;
+        int r[4] = {0, 0, 0, 0};
+        if (T.src == 0) {
+          const int* L = p.idx + ((int64_t)it.b * p.nq + it.qi) * p.k + T.list_off;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * lane + e;
+            int v = (j < T.hi) ? __ldg(L + j) : 0;
+            v = (v < 0 || v >= p.N) ? 0 : v;
+            r[e] = it.b * p.N + v;
+          }
+        }
+        for (int c = 0; c < kAttnChunks; ++c) {
+          int ok = 1;
+          if (lane == 0) {
+            ok = mbar_wait(&bar_kempty[c], ph ^ 1, &abort_flag);
+            if (ok) mbar_expect_tx(&bar_kfull[c], AttnSmem::K_CHUNK);
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) { stop = true; break; }
+          uint8_t* dst = sK + c * AttnSmem::K_CHUNK;
+          if (T.src == 0) {
+            tma_gather4(dst + (4 * lane) * 128, &comp_gather, c * 64, r[0], r[1], r[2], r[3], &bar_kfull[c]);
+          } else if (lane == 0) {
+            tma_load_2d(dst, T.src == 1 ? &comp_rows : &win_rows, c * 64, T.row0, &bar_kfull[c]);
+          }
+        }
+      }
+    }
+    // drain the last tile's loads before the CTA may exit
+    if (lane == 0 && tcount > 0)
+      for (int c = 0; c < kAttnChunks; ++c) mbar_wait(&bar_kfull[c], (tcount - 1) & 1, &abort_flag);
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = umma_idesc_bf16(128, kAttnH, 0, 0);
+      constexpr uint32_t idesc_pv = umma_idesc_bf16(128, kAttnH, 1, 1);
+      const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), p0 = smem_u32(sP);
+      uint32_t tcount = 0, icount = 0;
+      for (int id = blockIdx.x; id < p.n_items && !abort_flag; id += gridDim.x) {
+        const AttnItem it = attn_item(p, id);
+        if (it.tile1 <= it.tile0) continue;
+        if (!mbar_wait(&bar_q_full, icount & 1, &abort_flag)) break;
+        ++icount;
+        for (int tile = it.tile0; tile < it.tile1; ++tile, ++tcount) {
+          const uint32_t ph = tcount & 1;
+          if (!mbar_wait(&bar_s_empty, ph ^ 1, &abort_flag)) break;
+          tc_fence_after();
+          for (int c = 0; c < kAttnChunks; ++c) {
+            if (!mbar_wait(&bar_kfull[c], ph, &abort_flag)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              umma_bf16(tS, umma_desc_kmajor(k0 + c * AttnSmem::K_CHUNK + ks * 32),
+                        umma_desc_kmajor(q0 + c * AttnSmem::Q_CHUNK + ks * 32), idesc_s, (c | ks) != 0);
+          }
+          umma_commit(&bar_s_full);
+          if (!mbar_wait(&bar_p_full, ph, &abort_flag)) break;
+          tc_fence_after();
+          const bool first = tile == it.tile0;
+#pragma unroll
+          for (int mt = 0; mt < kAttnMT; ++mt) {
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+              umma_bf16(tO + mt * kAttnH,
+                        umma_desc_mnmajor(k0 + (2 * mt) * AttnSmem::K_CHUNK + ks * 2048, AttnSmem::K_CHUNK),
+                        umma_desc_mnmajor(p0 + ks * 2048, AttnSmem::P_BYTES), idesc_pv, !(first && ks == 0));
+            umma_commit(&bar_kempty[2 * mt]);
+            umma_commit(&bar_kempty[2 * mt + 1]);
+          }
+          umma_commit(&bar_pv_done);
+        }
+      }
+      umma_commit(&bar_done);
+      mbar_wait(&bar_done, 0, &abort_flag);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue (warps 0-3)
+    const int tid = threadIdx.x;               // key slot / dim slot
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    uint32_t tcount = 0;
+    const int r0 = kAttnD - p.rope_dims;
+    bool stop = false;                       // uniform over the 128 threads
+    for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
+      const AttnItem it = attn_item(p, id);
+      const bool empty = it.tile1 <= it.tile0;
+      // ---- query prologue: RMSNorm * gain, RoPE at t -> bf16, K-major SW128
+      if (!empty) {
+        if (tid < p.rope_dims / 2) {
+          float cs, sn;
+          rope_cos_sin((double)it.t, tid, p.rope_dims, p.rope_base, &cs, &sn);
+          rope_cs[tid] = cs;
+          rope_sn[tid] = sn;
+        }
+        named_sync128();
+        const __nv_bfloat16* Q = p.q + ((int64_t)it.b * p.nq + it.qi) * kAttnH * kAttnD;
+        for (int hh = 0; hh < kAttnH / 4; ++hh) {
+          const int h = warp * (kAttnH / 4) + hh;
+          float x[16];
+          load16(Q + (int64_t)h * kAttnD + lane * 16, x);
+          load16(Q + (int64_t)h * kAttnD + lane * 16 + 8, x + 8);
+          float ss = 0.f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) ss = fmaf(x[e], x[e], ss);
+          const float inv = p.q_norm ? rsqrtf(warp_sum(ss) / (float)kAttnD + p.eps) : 1.f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int dim = lane * 16 + e;
+            x[e] *= inv * (p.q_norm && p.q_gain ? __ldg(p.q_gain + dim) : 1.f);
+          }
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            const int dim = lane * 16 + e;
+            if (dim >= r0) {
+              const int j = (dim - r0) >> 1;
+              const float x0 = x[e], x1 = x[e + 1];
+              x[e] = x0 * rope_cs[j] - x1 * rope_sn[j];
+              x[e + 1] = x0 * rope_sn[j] + x1 * rope_cs[j];
+            }
+          }
+          // dims lane*16 .. +15 -> chunk lane/4, bytes (lane%4)*32 .. +31 of row h
+          uint8_t* chunk = sQ + (lane >> 2) * AttnSmem::Q_CHUNK;
+          uint4 o0, o1;
+          store16(reinterpret_cast<__nv_bfloat16*>(&o0), x);
+          store16(reinterpret_cast<__nv_bfloat16*>(&o1), x + 8);
+          *reinterpret_cast<uint4*>(chunk + sw128_offset(h, (lane & 3) * 32)) = o0;
+          *reinterpret_cast<uint4*>(chunk + sw128_offset(h, (lane & 3) * 32 + 16)) = o1;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bar_q_full);
+        if (tid < kAttnH) m_use[tid] = -INFINITY;
+      }
+      if (tid < kAttnH) l_run[tid] = 0.f;
+      named_sync128();
+
+      for (int tile = it.tile0; tile < it.tile1; ++tile, ++tcount) {
+        const uint32_t ph = tcount & 1;
+        const AttnTile T = attn_tile(p, it, tile);
+        bool valid = tid >= T.lo && tid < T.hi;
+        if (valid && T.src == 0) {
+          const int e = __ldg(p.idx + ((int64_t)it.b * p.nq + it.qi) * p.k + T.list_off + tid);
+          valid = e >= 0 && e < p.N;
+        }
+        if (!mbar_wait128(&bar_s_full, ph, &abort_flag)) { stop = true; break; }
+        tc_fence_after();
+        float s[kAttnH];
+        load_scores(tS + lane_base, valid, p.scale_log2, s);
+        reduce_heads<true>(s, red, stat_a);             // stat_a = tile max per head
+        if (tid == 0) need_rescale = 0;
+        named_sync128();
+        if (tid < kAttnH) {
+          const float mt = stat_a[tid], mo = m_use[tid];
+          float a = 1.f;
+          if (mt > mo + kRescaleThreshold || (mo == -INFINITY && mt != -INFINITY)) {
+            a = (mo == -INFINITY) ? 0.f : exp2f(mo - mt);
+            m_use[tid] = mt;
+            if (tile != it.tile0) need_rescale = 1;
+          }
+          alpha[tid] = a;
+        }
+        named_sync128();
+        // the previous tile's P.V has finished: P^T may be overwritten and O^T rescaled
+        if (tile != it.tile0) {
+          if (!mbar_wait128(&bar_pv_done, ph ^ 1, &abort_flag)) { stop = true; break; }
+          tc_fence_after();
+          if (need_rescale) {
+#pragma unroll 1
+            for (int mt = 0; mt < kAttnMT; ++mt) {
+#pragma unroll
+              for (int half = 0; half < 2; ++half) {
+                float v[32];
+                const uint32_t a = tO + lane_base + mt * kAttnH + half * 32;
+                tmem_ld32(a, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] *= alpha[half * 32 + e];
+                tmem_st32(a, v);
+              }
+            }
+            tmem_wait_st();
+          }
+        }
+        // probabilities from a second read of S (the first was consumed by the reduction)
+        load_scores(tS + lane_base, valid, p.scale_log2, s);
+        tc_fence_before();
+        mbar_arrive(&bar_s_empty);
+#pragma unroll
+        for (int h = 0; h < kAttnH; ++h) s[h] = (s[h] == -INFINITY) ? 0.f : exp2f(s[h] - m_use[h]);
+        // P^T row tid (64 heads, bf16) into the MN-major SW128 tile
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          uint4 o;
+          store16(reinterpret_cast<__nv_bfloat16*>(&o), s + 8 * j);
+          *reinterpret_cast<uint4*>(sP + sw128_offset(tid, j * 16)) = o;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bar_p_full);
+        // running per-head sum of p (overlaps the P.V on the tensor cores)
+        reduce_heads<false>(s, red, stat_b);
+        if (tid < kAttnH) l_run[tid] = l_run[tid] * alpha[tid] + stat_b[tid];
+      }
+      if (stop) break;
+      if (empty && !p.decode) {
+        // no key at all: only the sink is in the denominator, o = 0
+        __nv_bfloat16* O = p.out + ((int64_t)it.b * p.nq + it.qi) * kAttnH * kAttnD;
+        for (int x = tid; x < kAttnH * kAttnD; x += 128) O[x] = __float2bfloat16_rn(0.f);
+        continue;
+      }
+      // ---- epilogue: wait for the last P.V, reduce the sums, write out
+      if (!empty) {
+        if (!mbar_wait128(&bar_pv_done, (tcount - 1) & 1, &abort_flag)) { stop = true; break; }
+        tc_fence_after();
+      }
+      named_sync128();                                 // l_run / m_use complete
+      if (p.decode) {
+        float* P = p.partial + (((int64_t)it.b * p.nq + it.qi) * kAttnH * p.splits + it.split) * (kAttnD + 2);
+        const int64_t hstride = (int64_t)p.splits * (kAttnD + 2);
+        if (tid < kAttnH) {
+          P[tid * hstride + 0] = empty ? -INFINITY : m_use[tid] * 0.6931471805599453f;
+          P[tid * hstride + 1] = empty ? 0.f : l_run[tid];
+        }
+#pragma unroll 1
+        for (int mt = 0; mt < kAttnMT; ++mt) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            float v[32];
+            if (!empty) {
+              tmem_ld32(tO + lane_base + mt * kAttnH + half * 32, v);
+              tmem_wait_ld();
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = 0.f;
+            }
+            const int dim = mt * 128 + tid;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) P[(half * 32 + e) * hstride + 2 + dim] = v[e];
+          }
+        }
+      } else {
+        // final rows: o = O / (l + e^{z - m}), rope dims rotated back by -t
+        if (tid < kAttnH) {
+          const float z2 = p.sinks[tid] * kLog2e;
+          const float mu = m_use[tid];
+          const float M = fmaxf(mu, z2);
+          const float den = exp2f(z2 - M) + (mu == -INFINITY ? 0.f : l_run[tid] * exp2f(mu - M));
+          stat_a[tid] = (mu == -INFINITY) ? 0.f : exp2f(mu - M) / den;   // factor on O
+        }
+        if (tid < p.rope_dims / 2) {
+          float cs, sn;
+          rope_cos_sin(-(double)it.t, tid, p.rope_dims, p.rope_base, &cs, &sn);
+          rope_cs[tid] = cs;
+          rope_sn[tid] = sn;
+        }
+        named_sync128();
+        __nv_bfloat16* O = p.out + ((int64_t)it.b * p.nq + it.qi) * kAttnH * kAttnD;
+#pragma unroll 1
+        for (int mt = 0; mt < kAttnMT; ++mt) {
+          const int dim = mt * 128 + tid;
+          const bool rot = dim >= r0;
+          const int j = (dim - r0) >> 1;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            float v[32];
+            tmem_ld32(tO + lane_base + mt * kAttnH + half * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int h = half * 32 + e;
+              float o = v[e] * stat_a[h];
+              const float partner = __shfl_xor_sync(0xffffffffu, o, 1);
+              if (rot) o = (dim & 1) ? fmaf(partner, rope_sn[j], o * rope_cs[j]) : fmaf(-partner, rope_sn[j], o * rope_cs[j]);
+              O[(int64_t)h * kAttnD + dim] = __float2bfloat16_rn(o);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      named_sync128();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace csahca

@@ -16,6 +16,7 @@
 #include "topk.cuh"
 #include "attention_simt.cuh"
 #include "indexer_tc.cuh"
+#include "attention_tc.cuh"
 
 using namespace csahca;
 
@@ -435,6 +436,34 @@ int launch_simt_attn(const SimtAttnParams& p, int nq_total, cudaStream_t s, cons
   return CSAHCA_OK;
 }
 
+// ---- tensor-core attention (H = 64, d = 512, bf16) ---------------------------
+
+bool attn_tc_shape_ok(int dtype, int H, int d, int rope_dims, int64_t comp_rows, int64_t win_rows) {
+  return dtype == CSAHCA_BF16 && H == kAttnH && d == kAttnD && rope_dims <= 128 && comp_rows >= 128 &&
+         win_rows >= 128;
+}
+
+int launch_attn_tc(const AttnTcParams& p, const void* kv_comp, int64_t comp_rows, const void* win,
+                   int64_t win_rows, cudaStream_t s, const char* name) {
+  CUtensorMap m_rows, m_gather, m_win;
+  bool ok = encode_2d(&m_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv_comp, kAttnD, (uint64_t)comp_rows, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&m_gather, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv_comp, kAttnD, (uint64_t)comp_rows, 64, 1,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+  if (win) ok = ok && encode_2d(&m_win, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, win, kAttnD, (uint64_t)win_rows, 64,
+                                128, CU_TENSOR_MAP_SWIZZLE_128B);
+  else m_win = m_rows;
+  if (!ok) return CSAHCA_ERR_LAUNCH;
+  const int smem = AttnSmem::TOTAL;
+  cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+  if (grid <= 0) return CSAHCA_OK;
+  CSAHCA_TRACE(name, s);
+  attn_tc_kernel<<<grid, kAttnTcThreads, smem, s>>>(m_rows, m_gather, m_win, p);
+  CSAHCA_CHECK_LAUNCH();
+  return CSAHCA_OK;
+}
+
 template <typename T>
 int run_prefill_t(const csahca_attn_args* a, cudaStream_t s) {
   const double base = a->rope_base > 0 ? a->rope_base : kDefaultRopeBase;
@@ -446,10 +475,23 @@ int run_prefill_t(const csahca_attn_args* a, cudaStream_t s) {
                               a->n, a->kv_norm, a->rope_dims, base, eps, s);
     if (st != CSAHCA_OK) return st;
   }
+  const float scale = a->scale > 0 ? a->scale : 1.0f / sqrtf((float)a->d);
+  if (attn_tc_shape_ok(a->dtype, a->H, a->d, a->rope_dims, (int64_t)a->B * a->N, (int64_t)a->B * a->n)) {
+    AttnTcParams t;
+    memset(&t, 0, sizeof(t));
+    t.q = static_cast<const __nv_bfloat16*>(a->q); t.q_gain = a->q_gain; t.sinks = a->sinks; t.pos = nullptr;
+    t.q_norm = a->q_norm; t.eps = eps; t.scale_log2 = scale * kLog2e; t.rope_dims = a->rope_dims;
+    t.rope_base = base; t.B = a->B; t.nq = a->n; t.N = a->N; t.m = a->m; t.k = a->k; t.w = a->w;
+    t.csa = a->kind == CSAHCA_CSA; t.idx = a->idx; t.decode = 0;
+    t.n_items = a->B * a->n; t.splits = 1; t.tiles_per_split = 0;
+    t.out = static_cast<__nv_bfloat16*>(a->out); t.partial = nullptr;
+    return launch_attn_tc(t, a->kv_comp, (int64_t)a->B * a->N, win_final, (int64_t)a->B * a->n, s,
+                          a->kind == CSAHCA_CSA ? "attn_prefill_csa_tc" : "attn_prefill_hca_tc");
+  }
   SimtAttnParams p;
   memset(&p, 0, sizeof(p));
   p.q = a->q; p.q_gain = a->q_gain; p.sinks = a->sinks; p.pos = nullptr;
-  p.q_norm = a->q_norm; p.eps = eps; p.scale = a->scale > 0 ? a->scale : 1.0f / sqrtf((float)a->d);
+  p.q_norm = a->q_norm; p.eps = eps; p.scale = scale;
   p.rope_dims = a->rope_dims; p.rope_base = base;
   p.B = a->B; p.nq = a->n; p.H = a->H; p.d = a->d;
   p.kv_comp = a->kv_comp; p.N = a->N;
@@ -514,14 +556,31 @@ int validate_decode(const csahca_decode_args* a, bool shapes_only = false) {
 struct DecodeLayout {
   size_t scores_off, idx_off, partial_off, total;
   int splits;
+  bool tc;
+  int tiles_per_split;
 };
+
+bool decode_tc(const csahca_decode_args* a) {
+  return attn_tc_shape_ok(a->dtype, a->H, a->d, a->rope_dims, (int64_t)a->B * a->N_cap, (int64_t)a->B * a->w);
+}
 
 DecodeLayout decode_layout(const csahca_decode_args* a) {
   DecodeLayout L;
   const bool csa = a->kind == CSAHCA_CSA;
   const bool run_indexer = csa && !a->idx_in;
   const int64_t jmax = (csa ? (int64_t)a->k : (int64_t)a->N_cap) + a->w;
-  L.splits = (int)(jmax > 0 ? ceil_div64(jmax, kDecodeKeysPerSplit) : 1);
+  L.tc = decode_tc(a);
+  L.tiles_per_split = 0;
+  if (L.tc) {
+    // tensor-core path: split each query's tiles so that B x splits ~ one wave
+    const int tiles = (int)(ceil_div64(csa ? a->k : a->N_cap, 128) + ceil_div64(a->w, 128));
+    int want = (int)ceil_div64(num_sms(), a->B > 0 ? a->B : 1);
+    if (want < 1) want = 1;
+    L.tiles_per_split = (int)ceil_div64(tiles > 0 ? tiles : 1, want);
+    L.splits = (int)ceil_div64(tiles > 0 ? tiles : 1, L.tiles_per_split);
+  } else {
+    L.splits = (int)(jmax > 0 ? ceil_div64(jmax, kDecodeKeysPerSplit) : 1);
+  }
   size_t off = 0;
   L.scores_off = off;
   if (run_indexer) off += align_up((size_t)a->B * (a->N_cap > 0 ? a->N_cap : 1) * 4, 256);
@@ -559,22 +618,37 @@ int run_decode_t(const csahca_decode_args* a, cudaStream_t s, char* ws) {
       sel = idx;
     }
   }
-  SimtAttnParams p;
-  memset(&p, 0, sizeof(p));
-  p.q = a->q; p.q_gain = a->q_gain; p.sinks = a->sinks; p.pos = a->pos;
-  p.q_norm = a->q_norm; p.eps = eps; p.scale = a->scale > 0 ? a->scale : 1.0f / sqrtf((float)a->d);
-  p.rope_dims = a->rope_dims; p.rope_base = base;
-  p.B = a->B; p.nq = 1; p.H = a->H; p.d = a->d;
-  p.kv_comp = a->kv_cache; p.N = a->N_cap;
-  p.idx = sel; p.k = a->k; p.m = a->m;
-  p.win = a->win; p.w = a->w; p.decode = 1;
-  p.splits = L.splits; p.keys_per_split = kDecodeKeysPerSplit;
-  p.out = nullptr; p.partial = reinterpret_cast<float*>(ws + L.partial_off);
-  int st = launch_simt_attn<T>(p, a->B, s,
-                               a->kind == CSAHCA_CSA ? "attn_decode_csa_simt" : "attn_decode_hca_simt");
+  const float scale = a->scale > 0 ? a->scale : 1.0f / sqrtf((float)a->d);
+  float* partial = reinterpret_cast<float*>(ws + L.partial_off);
+  int st;
+  if (L.tc) {
+    AttnTcParams t;
+    memset(&t, 0, sizeof(t));
+    t.q = static_cast<const __nv_bfloat16*>(a->q); t.q_gain = a->q_gain; t.sinks = a->sinks; t.pos = a->pos;
+    t.q_norm = a->q_norm; t.eps = eps; t.scale_log2 = scale * kLog2e; t.rope_dims = a->rope_dims;
+    t.rope_base = base; t.B = a->B; t.nq = 1; t.N = a->N_cap; t.m = a->m; t.k = a->k; t.w = a->w;
+    t.csa = a->kind == CSAHCA_CSA; t.idx = sel; t.decode = 1;
+    t.splits = L.splits; t.tiles_per_split = L.tiles_per_split; t.n_items = a->B * L.splits;
+    t.out = nullptr; t.partial = partial;
+    st = launch_attn_tc(t, a->kv_cache, (int64_t)a->B * a->N_cap, a->w > 0 ? a->win : nullptr,
+                        (int64_t)a->B * a->w, s, a->kind == CSAHCA_CSA ? "attn_decode_csa_tc" : "attn_decode_hca_tc");
+  } else {
+    SimtAttnParams p;
+    memset(&p, 0, sizeof(p));
+    p.q = a->q; p.q_gain = a->q_gain; p.sinks = a->sinks; p.pos = a->pos;
+    p.q_norm = a->q_norm; p.eps = eps; p.scale = scale;
+    p.rope_dims = a->rope_dims; p.rope_base = base;
+    p.B = a->B; p.nq = 1; p.H = a->H; p.d = a->d;
+    p.kv_comp = a->kv_cache; p.N = a->N_cap;
+    p.idx = sel; p.k = a->k; p.m = a->m;
+    p.win = a->win; p.w = a->w; p.decode = 1;
+    p.splits = L.splits; p.keys_per_split = kDecodeKeysPerSplit;
+    p.out = nullptr; p.partial = partial;
+    st = launch_simt_attn<T>(p, a->B, s, a->kind == CSAHCA_CSA ? "attn_decode_csa_simt" : "attn_decode_hca_simt");
+  }
   if (st != CSAHCA_OK) return st;
   CombineParams c;
-  c.partial = p.partial; c.sinks = a->sinks; c.pos = a->pos; c.out = a->out;
+  c.partial = partial; c.sinks = a->sinks; c.pos = a->pos; c.out = a->out;
   c.B = a->B; c.nq = 1; c.H = a->H; c.d = a->d; c.splits = L.splits;
   c.rope_dims = a->rope_dims; c.decode = 1; c.rope_base = base;
   {

@@ -302,23 +302,26 @@ def attend_query(q_final, key_rows, sinks, t: int, r: int, tau: float,
 def prefill_attention(kind: str, q_raw, kv_comp, kv_win_raw, sinks, *, m: int,
                       w: int, r: int, q_gain=None, kv_gain=None, idx=None,
                       tau=None, base: float = ROPE_BASE, rows=None,
-                      q_norm: bool = True, kv_norm: bool = True) -> np.ndarray:
+                      q_norm: bool = True, kv_norm: bool = True,
+                      q_holds_rows: bool = False) -> np.ndarray:
     """Prefill attention for one sequence.
 
     kind: "csa" (keys = kv_comp[idx[t]]) or "hca" (keys = every visible entry).
-    q_raw: [n, H, d]; kv_comp: [N, d] final compressed rows; kv_win_raw: [n, d]
-    per-token rows, finished here at their own positions; idx: [n, k] (csa).
-    Returns o for the query positions in ``rows`` (default all): [len, H, d].
+    q_raw: [n, H, d] (or, with q_holds_rows, [len(rows), H, d] holding only the
+    queries of ``rows``); kv_comp: [N, d] final compressed rows; kv_win_raw:
+    [n, d] per-token rows, finished here at their own positions; idx: [n, k]
+    (csa).  Returns o for the query positions in ``rows`` (default all).
     """
     q_raw = np.asarray(q_raw, np.float64)
-    n, H, d = q_raw.shape
+    _, H, d = q_raw.shape
+    n = np.asarray(kv_win_raw).shape[0]
     tau = 1.0 / np.sqrt(d) if tau is None else tau
     kv_comp = np.asarray(kv_comp, np.float64)
     rows = np.arange(n) if rows is None else np.asarray(rows)
     out = np.zeros((len(rows), H, d))
     for oi, t in enumerate(rows):
         t = int(t)
-        qt = finish_rows(q_raw[t], t, q_gain, r, base, normalize=q_norm)
+        qt = finish_rows(q_raw[oi if q_holds_rows else t], t, q_gain, r, base, normalize=q_norm)
         if kind == "csa":
             sel = np.asarray(idx[t])
             sel = sel[sel >= 0]

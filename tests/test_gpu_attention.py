@@ -37,10 +37,13 @@ def _prefill_layer(wl, n, B):
 
 
 def _oracle_rows(kind, inp, kv, idx, wl, m, b, rows):
-    return O.prefill_attention(kind, npy(inp["q"][b]), npy(kv[b]), npy(inp["kv_win"][b]),
-                               npy(inp["sinks"]), m=m, w=wl.w, r=wl.r,
+    rows = np.asarray(rows)
+    sel = torch.as_tensor(rows, device=inp["q"].device)
+    return O.prefill_attention(kind, npy(inp["q"][b].index_select(0, sel)), npy(kv[b]),
+                               npy(inp["kv_win"][b]), npy(inp["sinks"]), m=m, w=wl.w, r=wl.r,
                                q_gain=npy(inp["q_gain"]), kv_gain=npy(inp["kv_gain"]),
-                               idx=None if idx is None else npy(idx[b]), rows=rows)
+                               idx=None if idx is None else npy(idx[b]), rows=rows,
+                               q_holds_rows=True)
 
 
 def test_prefill_csa_tiny_f32():
@@ -108,4 +111,21 @@ def test_prefill_no_window_no_sink_edge():
     ref = O.prefill_attention("hca", npy(inp["q"][0]), npy(kv[0]), npy(inp["kv_win"][0]),
                               npy(inp["sinks"]), m=m, w=0, r=wl.r, rows=rows)
     check_close(npy(out[0, rows]), ref, "bf16", "hca w=0")
+    assert api.device_error() == 0
+
+
+@pytest.mark.parametrize("n,w", [(16384 + 37, 128), (8192 + 5, 64), (600, 64)])
+def test_prefill_hca_64_heads_512_dims(n, w):
+    """HCA prefill at the 64-head / 512-dim shape (m' = 128), including
+    queries with no visible entry yet, a partial window and a ragged tail
+    (the two larger cases run on the tensor cores, the smallest on CUDA cores)."""
+    wl = synth.Workload(**{**synth.WORKLOADS["csa_prefill_128k"].__dict__, "kind": "hca", "w": w})
+    inp, kv, m = _prefill_layer(wl, n, 2)
+    out = api.compressed_attn_prefill("hca", inp["q"], kv, inp["kv_win"], inp["sinks"], m=m,
+                                      w=wl.w, rope_dims=wl.r, q_gain=inp["q_gain"],
+                                      kv_gain=inp["kv_gain"])
+    for b in range(2):
+        rows = _sample(n, [0, 1, 126, 127, 128, 255, 256, n - 1], seed=10 + b, count=10)
+        ref = _oracle_rows("hca", inp, kv, None, wl, m, b, rows)
+        check_close(npy(out[b, rows]), ref, "bf16", f"hca64 b={b}")
     assert api.device_error() == 0
