@@ -35,7 +35,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from long_context_compressed_overlapped_b200 import api, native, synth  # noqa: E402
+from long_context_compressed_overlapped_b200 import api, native, runtime, synth  # noqa: E402
 
 METRIC = "CSA+HCA attention tokens/s (decode@1M, prefill@128K); % HBM / TC roofline"
 L2_BYTES = 126 * 2**20
@@ -75,11 +75,7 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
+    return runtime.max_over_ranks(x) if world > 1 else x
 
 
 # ------------------------------------------------------------------ clocks ----
@@ -94,7 +90,8 @@ class ClockSampler:
     def __init__(self, device: int):
         self.uuid = None
         try:
-            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            u = str(torch.cuda.get_device_properties(device).uuid)
+            self.uuid = u if u.startswith("GPU-") else "GPU-" + u
         except Exception:
             pass
         self.proc = None
@@ -105,8 +102,6 @@ class ClockSampler:
             self.fh = open(self.path, "w")
             cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                    "-lms", "200"]
-            if self.uuid:
-                cmd[1:1] = ["-i", self.uuid]
             self.proc = subprocess.Popen(cmd, stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -127,6 +122,8 @@ class ClockSampler:
                 parts = [p.strip() for p in line.split(",")]
                 if len(parts) < 10:
                     continue
+                if self.uuid and parts[1] != self.uuid and not (len(parts[1]) > 4 and self.uuid.endswith(parts[1][4:])):
+                    continue
                 try:
                     sm.append(float(parts[2]))
                     smax = float(parts[3])
@@ -142,36 +139,6 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------- decode step ----
-
-class DecodeStep:
-    """Pre-marshalled C-ABI calls of one decode step (all layers)."""
-
-    def __init__(self, wl, layers, stream):
-        self.lib = native.lib()
-        self.wl = wl
-        self.layers = layers
-        self.stream = stream
-        self.sh = stream.cuda_stream
-        self.calls = []
-        for L in layers:
-            kw = dict(m=L["m"], rope_dims=wl.r, q_gain=L["q_gain"])
-            if L["kind"] == "csa":
-                kw.update(k=wl.k, qI=L["qI"], wI=L["w"], kI=L["kI"], kI_scale=L["kI_scale"])
-            args, out, keep = api.decode_args(L["kind"], L["q"], L["pos"], L["kv"], L["win"],
-                                              L["sinks"], **kw)
-            nbytes = self.lib.csahca_decode_workspace_size(C.byref(args))
-            ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=L["q"].device)
-            args.workspace = ws.data_ptr()
-            args.workspace_bytes = ws.numel()
-            L["out"] = out
-            self.calls.append((args, out, keep, ws))
-
-    def __call__(self):
-        for args, _, _, _ in self.calls:
-            st = self.lib.compressed_attn_decode(C.byref(args), self.sh)
-            if st != 0:
-                native.check(st, "compressed_attn_decode")
-
 
 def decode_bytes_per_kernel(wl, ctx):
     """Algorithmic bytes per launch of each traced decode kernel (one launch
@@ -376,6 +343,7 @@ def main():
     ap.add_argument("--prefill", action="store_true", help="also time csa_prefill_128k")
     ap.add_argument("--prefill-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the decode step eagerly")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -390,9 +358,13 @@ def main():
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(device=dev)
     wl = synth.WORKLOADS[args.workload]
-    wl_r = synth.Workload(**{**wl.__dict__, "seed": wl.seed + 1000 * rank})
-    layers = synth.decode_inputs(wl_r, dev)
-    step = DecodeStep(wl, layers, stream)
+    layers = synth.decode_inputs(runtime.shard_workload(wl, rank), dev)
+    eager = runtime.DecodeStep(wl, layers, stream)
+    step = eager
+    launch_mode = "eager"
+    if not args.no_graph:
+        step = runtime.DecodeGraph(eager)
+        launch_mode = "cuda_graph"
     flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
 
     def flush():
@@ -413,9 +385,10 @@ def main():
     tokens = world * wl.B * args.steps
     value = tokens / (total_ms / 1000.0)
 
-    # traced pass: per-kernel device time of the same K steps
+    # traced pass: per-kernel device time of the same K steps (eager launches,
+    # so every kernel is bracketed by its own events)
     api.trace_enable(True)
-    time_steps(step, args.steps, stream, flush, world)
+    time_steps(eager, args.steps, stream, flush, world)
     traced = api.trace_collect()
     api.trace_enable(False)
 
@@ -493,7 +466,7 @@ def main():
                    "layers": list(wl.layers), "heads": wl.H, "head_dim": wl.d, "top_k": wl.k,
                    "window": wl.w, "indexer_keys": "e4m3" if wl.fp8_keys else "bf16",
                    "parallelism": f"replicas{world}" if world > 1 else "none",
-                   "l2": "flushed between timed steps"},
+                   "launch": launch_mode, "l2": "flushed between timed steps"},
         "roofline": roof,
         "step_hbm": {"algorithmic_bytes": step_bytes, "frac": step_frac, "peak": pk["hbm_gbs"]},
         "clocks": clk,

@@ -34,7 +34,7 @@ struct SimtAttnParams {
   int splits, keys_per_split;
   // outputs: partial == NULL -> final rows in out (one split); else partials
   void* out;                         // final [B, nq, H, d]
-  float* partial;                    // [B, nq, H, splits, d + 2]
+  float* partial;                    // [B, nq, H, splits, d + 4]: m, l, -, -, acc[d]
 };
 
 template <typename T>
@@ -181,10 +181,10 @@ __global__ void __launch_bounds__(32 * kSimtHG) attn_simt_kernel(SimtAttnParams 
       }
     }
   } else {
-    float* P = p.partial + ((((int64_t)b * p.nq + qi) * p.H + h) * p.splits + split) * (d + 2);
+    float* P = p.partial + ((((int64_t)b * p.nq + qi) * p.H + h) * p.splits + split) * (d + 4);
 #pragma unroll
     for (int e = 0; e < kSimtMaxDPL; ++e)
-      if (e < dpl) P[2 + lane + 32 * e] = acc[e];
+      if (e < dpl) P[4 + lane + 32 * e] = acc[e];
     if (lane == 0) { P[0] = mx; P[1] = lsum; }
   }
 }
@@ -205,26 +205,27 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(CombineParams p) {
   const int64_t bq = bqh / p.H;
   const int qi = (int)(bq % p.nq), b = (int)(bq / p.nq);
   const int t = p.decode ? p.pos[b] : qi;
-  const float* P = p.partial + bqh * p.splits * (p.d + 2);
+  const int64_t ps = p.d + 4;                       // partial row: m, l, -, -, acc[d]
+  const float* P = p.partial + bqh * p.splits * ps;
   const float z = p.sinks[h];
   float M = z;
-  for (int s = 0; s < p.splits; ++s) M = fmaxf(M, P[(int64_t)s * (p.d + 2)]);
+  for (int s = 0; s < p.splits; ++s) M = fmaxf(M, P[(int64_t)s * ps]);
   float den = expf(z - M);
   for (int s = 0; s < p.splits; ++s) {
-    const float ms = P[(int64_t)s * (p.d + 2)];
-    if (ms != -INFINITY) den += P[(int64_t)s * (p.d + 2) + 1] * expf(ms - M);
+    const float ms = P[(int64_t)s * ps];
+    if (ms != -INFINITY) den += P[(int64_t)s * ps + 1] * expf(ms - M);
   }
   const int r0 = p.d - p.rope_dims;
   T* O = static_cast<T*>(p.out) + bqh * p.d;
   for (int dim2 = threadIdx.x * 2; dim2 < p.d; dim2 += blockDim.x * 2) {
     float o0 = 0.f, o1 = 0.f;
     for (int s = 0; s < p.splits; ++s) {
-      const float* Ps = P + (int64_t)s * (p.d + 2);
+      const float* Ps = P + (int64_t)s * ps;
       const float ms = Ps[0];
       if (ms == -INFINITY) continue;
       const float f = expf(ms - M);
-      o0 = fmaf(Ps[2 + dim2], f, o0);
-      o1 = fmaf(Ps[3 + dim2], f, o1);
+      o0 = fmaf(Ps[4 + dim2], f, o0);
+      o1 = fmaf(Ps[5 + dim2], f, o1);
     }
     o0 /= den; o1 /= den;
     if (dim2 >= r0) {

@@ -47,7 +47,7 @@ struct AttnTcParams {
   int decode;                   // window = ring [B, w, d] (decode) or finished rows [B, nq, d]
   int n_items, splits, tiles_per_split;
   __nv_bfloat16* out;           // final [B, nq, H, D]
-  float* partial;               // [B, nq, H, splits, D + 2]
+  float* partial;               // [B, nq, H, splits, D + 4]
 };
 
 struct AttnItem { int b, qi, t, tile0, tile1, split, ncomp_tiles, nwin_tiles; };
@@ -177,14 +177,16 @@ struct AttnSmem {
 
 __global__ void __launch_bounds__(kAttnTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_constant__ CUtensorMap comp_gather,
-               const __grid_constant__ CUtensorMap win_rows, AttnTcParams p) {
+               const __grid_constant__ CUtensorMap win_rows, const __grid_constant__ CUtensorMap q_rows,
+               AttnTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
   uint8_t* sK = sQ + AttnSmem::Q_BYTES;
   uint8_t* sP = sK + AttnSmem::K_BYTES;
   __shared__ uint64_t bar_kfull[kAttnChunks], bar_kempty[kAttnChunks];
-  __shared__ uint64_t bar_q_full, bar_s_full, bar_s_empty, bar_p_full, bar_pv_done, bar_done;
+  __shared__ uint64_t bar_q_raw, bar_q_empty, bar_q_full, bar_s_full, bar_s_empty, bar_p_full, bar_pv_done,
+      bar_done;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
   __shared__ float red[4 * kAttnH];
@@ -197,6 +199,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int c = 0; c < kAttnChunks; ++c) { mbar_init(&bar_kfull[c], 1); mbar_init(&bar_kempty[c], 1); }
+    mbar_init(&bar_q_raw, 1);
+    mbar_init(&bar_q_empty, 1);
     mbar_init(&bar_q_full, 128);
     mbar_init(&bar_s_full, 1);
     mbar_init(&bar_s_empty, 128);
@@ -218,10 +222,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     tma_prefetch_desc(&comp_rows);
     tma_prefetch_desc(&comp_gather);
     tma_prefetch_desc(&win_rows);
-    uint32_t tcount = 0;
+    tma_prefetch_desc(&q_rows);
+    uint32_t tcount = 0, icount = 0;
     bool stop = false;                       // warp-uniform
     for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
       const AttnItem it = attn_item(p, id);
+      if (it.tile1 <= it.tile0) continue;
+      {
+        // raw Q of this item into the Q buffer once the previous item's
+        // score MMAs have read it; normed and roped there by warps 0-3
+        int ok = 1;
+        if (lane == 0) {
+          ok = mbar_wait(&bar_q_empty, (icount & 1) ^ 1, &abort_flag);
+          if (ok) {
+            mbar_expect_tx(&bar_q_raw, AttnSmem::Q_BYTES);
+            const int qrow = (it.b * p.nq + it.qi) * kAttnH;
+            for (int c = 0; c < kAttnChunks; ++c)
+              tma_load_2d(sQ + c * AttnSmem::Q_CHUNK, &q_rows, c * 64, qrow, &bar_q_raw);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) { stop = true; break; }
+        ++icount;
+      }
       for (int tile = it.tile0; tile < it.tile1 && !stop; ++tile, ++tcount) {
         const AttnTile T = attn_tile(p, it, tile);
         const uint32_t ph = tcount & 1;
@@ -253,9 +276,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
         }
       }
     }
-    // drain the last tile's loads before the CTA may exit
+    // drain the last loads before the CTA may exit
     if (lane == 0 && tcount > 0)
       for (int c = 0; c < kAttnChunks; ++c) mbar_wait(&bar_kfull[c], (tcount - 1) & 1, &abort_flag);
+    if (lane == 0 && icount > 0) mbar_wait(&bar_q_raw, (icount - 1) & 1, &abort_flag);
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -281,6 +305,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
                         umma_desc_kmajor(q0 + c * AttnSmem::Q_CHUNK + ks * 32), idesc_s, (c | ks) != 0);
           }
           umma_commit(&bar_s_full);
+          if (tile == it.tile1 - 1) umma_commit(&bar_q_empty);
           if (!mbar_wait(&bar_p_full, ph, &abort_flag)) break;
           tc_fence_after();
           const bool first = tile == it.tile0;
@@ -304,13 +329,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     // ------------------------------------------------------------ softmax / epilogue (warps 0-3)
     const int tid = threadIdx.x;               // key slot / dim slot
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    uint32_t tcount = 0;
+    uint32_t tcount = 0, qcount = 0;
     const int r0 = kAttnD - p.rope_dims;
     bool stop = false;                       // uniform over the 128 threads
     for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
       const AttnItem it = attn_item(p, id);
       const bool empty = it.tile1 <= it.tile0;
-      // ---- query prologue: RMSNorm * gain, RoPE at t -> bf16, K-major SW128
+      // ---- query prologue: raw Q (landed by TMA in the K-major SW128 layout)
+      // -> RMSNorm * gain, RoPE at t, in place
       if (!empty) {
         if (tid < p.rope_dims / 2) {
           float cs, sn;
@@ -318,13 +344,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
           rope_cs[tid] = cs;
           rope_sn[tid] = sn;
         }
-        named_sync128();
-        const __nv_bfloat16* Q = p.q + ((int64_t)it.b * p.nq + it.qi) * kAttnH * kAttnD;
+        if (tid < kAttnH) { m_use[tid] = -INFINITY; l_run[tid] = 0.f; }
+        if (!mbar_wait128(&bar_q_raw, qcount & 1, &abort_flag)) { stop = true; break; }
+        ++qcount;
+        uint8_t* chunk = sQ + (lane >> 2) * AttnSmem::Q_CHUNK;
         for (int hh = 0; hh < kAttnH / 4; ++hh) {
           const int h = warp * (kAttnH / 4) + hh;
+          uint4* a0 = reinterpret_cast<uint4*>(chunk + sw128_offset(h, (lane & 3) * 32));
+          uint4* a1 = reinterpret_cast<uint4*>(chunk + sw128_offset(h, (lane & 3) * 32 + 16));
+          uint4 r0v = *a0, r1v = *a1;
           float x[16];
-          load16(Q + (int64_t)h * kAttnD + lane * 16, x);
-          load16(Q + (int64_t)h * kAttnD + lane * 16 + 8, x + 8);
+          {
+            const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&r0v);
+            const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&r1v);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              float2 f0 = __bfloat1622float2(h0[i]), f1 = __bfloat1622float2(h1[i]);
+              x[2 * i] = f0.x; x[2 * i + 1] = f0.y; x[8 + 2 * i] = f1.x; x[8 + 2 * i + 1] = f1.y;
+            }
+          }
           float ss = 0.f;
 #pragma unroll
           for (int e = 0; e < 16; ++e) ss = fmaf(x[e], x[e], ss);
@@ -344,19 +382,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
               x[e + 1] = x0 * rope_sn[j] + x1 * rope_cs[j];
             }
           }
-          // dims lane*16 .. +15 -> chunk lane/4, bytes (lane%4)*32 .. +31 of row h
-          uint8_t* chunk = sQ + (lane >> 2) * AttnSmem::Q_CHUNK;
           uint4 o0, o1;
           store16(reinterpret_cast<__nv_bfloat16*>(&o0), x);
           store16(reinterpret_cast<__nv_bfloat16*>(&o1), x + 8);
-          *reinterpret_cast<uint4*>(chunk + sw128_offset(h, (lane & 3) * 32)) = o0;
-          *reinterpret_cast<uint4*>(chunk + sw128_offset(h, (lane & 3) * 32 + 16)) = o1;
+          *a0 = o0;
+          *a1 = o1;
         }
         fence_proxy_async_smem();
         mbar_arrive(&bar_q_full);
-        if (tid < kAttnH) m_use[tid] = -INFINITY;
       }
-      if (tid < kAttnH) l_run[tid] = 0.f;
       named_sync128();
 
       for (int tile = it.tile0; tile < it.tile1; ++tile, ++tcount) {
@@ -440,15 +474,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       }
       named_sync128();                                 // l_run / m_use complete
       if (p.decode) {
-        float* P = p.partial + (((int64_t)it.b * p.nq + it.qi) * kAttnH * p.splits + it.split) * (kAttnD + 2);
-        const int64_t hstride = (int64_t)p.splits * (kAttnD + 2);
+        // partial rows [H][D + 4]: m (natural log units), l, -, -, O^T[.][h]
+        float* P = p.partial + (((int64_t)it.b * p.nq + it.qi) * kAttnH * p.splits + it.split) * (kAttnD + 4);
+        const int64_t hstride = (int64_t)p.splits * (kAttnD + 4);
         if (tid < kAttnH) {
           P[tid * hstride + 0] = empty ? -INFINITY : m_use[tid] * 0.6931471805599453f;
           P[tid * hstride + 1] = empty ? 0.f : l_run[tid];
         }
+        float* stage = reinterpret_cast<float*>(sP);   // [32 heads][128 dims] f32 = 16 KB
 #pragma unroll 1
         for (int mt = 0; mt < kAttnMT; ++mt) {
-#pragma unroll
+#pragma unroll 1
           for (int half = 0; half < 2; ++half) {
             float v[32];
             if (!empty) {
@@ -458,9 +494,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
 #pragma unroll
               for (int e = 0; e < 32; ++e) v[e] = 0.f;
             }
-            const int dim = mt * 128 + tid;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) P[(half * 32 + e) * hstride + 2 + dim] = v[e];
+            for (int e = 0; e < 32; ++e) stage[e * 128 + tid] = v[e];
+            named_sync128();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int piece = tid + 128 * i;           // 16-byte piece: head e = piece / 32
+              const int e = piece >> 5, off = (piece & 31) * 4;
+              const float4 val = *reinterpret_cast<const float4*>(stage + e * 128 + off);
+              *reinterpret_cast<float4*>(P + (half * 32 + e) * hstride + 4 + mt * 128 + off) = val;
+            }
+            named_sync128();
           }
         }
       } else {
@@ -480,6 +524,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
         }
         named_sync128();
         __nv_bfloat16* O = p.out + ((int64_t)it.b * p.nq + it.qi) * kAttnH * kAttnD;
+        __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sP);   // [64 heads][128 dims] bf16
 #pragma unroll 1
         for (int mt = 0; mt < kAttnMT; ++mt) {
           const int dim = mt * 128 + tid;
@@ -496,9 +541,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
               float o = v[e] * stat_a[h];
               const float partner = __shfl_xor_sync(0xffffffffu, o, 1);
               if (rot) o = (dim & 1) ? fmaf(partner, rope_sn[j], o * rope_cs[j]) : fmaf(-partner, rope_sn[j], o * rope_cs[j]);
-              O[(int64_t)h * kAttnD + dim] = __float2bfloat16_rn(o);
+              stage[h * 128 + tid] = __float2bfloat16_rn(o);
             }
           }
+          named_sync128();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int piece = tid + 128 * i;             // 16-byte piece: head = piece / 16
+            const int h = piece >> 4, off = (piece & 15) * 8;
+            const uint4 val = *reinterpret_cast<const uint4*>(stage + h * 128 + off);
+            *reinterpret_cast<uint4*>(O + (int64_t)h * kAttnD + mt * 128 + off) = val;
+          }
+          named_sync128();
         }
       }
       tc_fence_before();

@@ -14,6 +14,7 @@
 #include "compress.cuh"
 #include "indexer_simt.cuh"
 #include "topk.cuh"
+#include "topk_large.cuh"
 #include "attention_simt.cuh"
 #include "indexer_tc.cuh"
 #include "attention_tc.cuh"
@@ -224,9 +225,87 @@ int indexer_chunk_rows(const csahca_indexer_args* a) {
   return (int)rows;
 }
 
-size_t indexer_workspace(const csahca_indexer_args* a) {
+constexpr int kTopkSmallMaxN = 32768;      // rows up to this length: one CTA per row
+
+bool topk_uses_large(const csahca_indexer_args* a) { return a->N > kTopkSmallMaxN; }
+
+// Scratch of the multi-CTA top-k for `rows` rows of length N.
+struct TopkLargeLayout { size_t hist, counters, above, cand, total; };
+TopkLargeLayout topk_large_layout(int64_t rows, int N, int k) {
+  TopkLargeLayout L;
+  size_t off = 0;
+  L.hist = off; off += align_up((size_t)rows * kHistBins * 4, 256);
+  L.counters = off; off += align_up((size_t)rows * 4 * 4, 256);
+  L.above = off; off += align_up((size_t)rows * k * 4, 256);
+  L.cand = off; off += align_up((size_t)rows * N * 8, 256);
+  L.total = off;
+  return L;
+}
+
+size_t indexer_scores_bytes(const csahca_indexer_args* a) {
   if (a->scores_out || a->B == 0 || a->nq == 0) return 0;
   return align_up((size_t)a->B * indexer_chunk_rows(a) * (size_t)(a->N > 0 ? a->N : 1) * 4, 256);
+}
+
+size_t indexer_workspace(const csahca_indexer_args* a) {
+  if (a->B == 0 || a->nq == 0) return 0;
+  size_t w = indexer_scores_bytes(a);
+  if (topk_uses_large(a)) {
+    const int64_t rows = a->scores_out ? (a->nq < 65535 ? a->nq : 65535) : (int64_t)a->B * indexer_chunk_rows(a);
+    w += topk_large_layout(rows, a->N, a->k).total;
+  }
+  return w;
+}
+
+// Top-k of `rows` score rows (row r at scores + r * stride, position q_pos[r]).
+int launch_topk(const csahca_indexer_args* a, const float* scores, int64_t stride, const int* q_pos, int* idx,
+                int rows, char* scratch, cudaStream_t s) {
+  if (!topk_uses_large(a)) {
+    TopkParams tp;
+    tp.scores = scores; tp.row_stride = stride; tp.q_pos = q_pos; tp.idx = idx;
+    tp.B = 1; tp.nq = rows; tp.N = a->N; tp.m = a->m; tp.k = a->k;
+    tp.q_begin = 0; tp.q_count = rows;
+    CSAHCA_TRACE("topk_rows", s);
+    topk_rows_kernel<<<rows, kTopkThreads, 0, s>>>(tp);
+    CSAHCA_CHECK_LAUNCH();
+    return CSAHCA_OK;
+  }
+  if (a->N > kTopkLargeMaxN) return CSAHCA_ERR_UNSUPPORTED;
+  const TopkLargeLayout L = topk_large_layout(rows, a->N, a->k);
+  TopkLargeParams tp;
+  tp.scores = scores; tp.row_stride = stride; tp.q_pos = q_pos; tp.idx = idx;
+  tp.rows = rows; tp.N = a->N; tp.m = a->m; tp.k = a->k;
+  int slices = (int)ceil_div64(2 * num_sms(), rows);
+  const int max_slices = (int)ceil_div64(a->N, 2048);
+  if (slices > max_slices) slices = max_slices;
+  if (slices < 1) slices = 1;
+  tp.slices = slices;
+  tp.hist = reinterpret_cast<uint32_t*>(scratch + L.hist);
+  tp.counters = reinterpret_cast<uint32_t*>(scratch + L.counters);
+  tp.above = reinterpret_cast<int*>(scratch + L.above);
+  tp.cand = reinterpret_cast<uint2*>(scratch + L.cand);
+  if (cudaMemsetAsync(scratch + L.hist, 0, L.above - L.hist, s) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return CSAHCA_ERR_LAUNCH;
+  }
+  {
+    CSAHCA_TRACE("topk_hist", s);
+    topk_hist_kernel<<<rows * slices, 512, 0, s>>>(tp);
+  }
+  CSAHCA_CHECK_LAUNCH();
+  {
+    CSAHCA_TRACE("topk_split", s);
+    topk_split_kernel<<<rows * slices, 512, 0, s>>>(tp);
+  }
+  CSAHCA_CHECK_LAUNCH();
+  const int smem = 2 * (int)ceil_div64(a->N, 32) * 4;
+  cudaFuncSetAttribute(topk_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  {
+    CSAHCA_TRACE("topk_finish", s);
+    topk_finish_kernel<<<rows, 1024, smem, s>>>(tp);
+  }
+  CSAHCA_CHECK_LAUNCH();
+  return CSAHCA_OK;
 }
 
 template <typename TQ, typename TK, bool kFP8>
@@ -341,16 +420,9 @@ int run_indexer(const csahca_indexer_args* a, void* stream) {
           }
           CSAHCA_CHECK_LAUNCH();
         }
-        TopkParams tp;
-        tp.scores = pb.scores; tp.row_stride = stride; tp.q_pos = pb.q_pos;
-        tp.idx = a->idx + (int64_t)b * a->nq * a->k;
-        tp.B = 1; tp.nq = a->nq; tp.N = a->N; tp.m = a->m; tp.k = a->k;
-        tp.q_begin = q0; tp.q_count = qc;
-        {
-          CSAHCA_TRACE("topk_rows", s);
-          topk_rows_kernel<<<qc, kTopkThreads, 0, s>>>(tp);
-        }
-        CSAHCA_CHECK_LAUNCH();
+        int st3 = launch_topk(a, pb.scores, stride, pb.q_pos + q0, a->idx + ((int64_t)b * a->nq + q0) * a->k, qc,
+                              static_cast<char*>(a->workspace), s);
+        if (st3 != CSAHCA_OK) return st3;
       }
       continue;
     }
@@ -371,15 +443,19 @@ int run_indexer(const csahca_indexer_args* a, void* stream) {
       }
       CSAHCA_CHECK_LAUNCH();
     }
-    TopkParams tp;
-    tp.scores = base; tp.row_stride = stride; tp.q_pos = a->q_pos; tp.idx = a->idx;
-    tp.B = a->B; tp.nq = a->nq; tp.N = a->N; tp.m = a->m; tp.k = a->k;
-    tp.q_begin = q0; tp.q_count = qc;
-    {
-      CSAHCA_TRACE("topk_rows", s);
-      topk_rows_kernel<<<(unsigned)(a->B * qc), kTopkThreads, 0, s>>>(tp);
+    // rows of this chunk: (b, q) -> b * qc + (q - q0); positions and outputs are
+    // addressed per batch entry, so launch per b unless the chunk is the whole nq
+    char* scratch = static_cast<char*>(a->workspace) + indexer_scores_bytes(a);
+    if (qc == a->nq) {
+      int st3 = launch_topk(a, base, stride, a->q_pos, a->idx, a->B * qc, scratch, s);
+      if (st3 != CSAHCA_OK) return st3;
+    } else {
+      for (int b = 0; b < a->B; ++b) {
+        int st3 = launch_topk(a, base + (int64_t)b * qc * stride, stride, a->q_pos + (int64_t)b * a->nq + q0,
+                              a->idx + ((int64_t)b * a->nq + q0) * a->k, qc, scratch, s);
+        if (st3 != CSAHCA_OK) return st3;
+      }
     }
-    CSAHCA_CHECK_LAUNCH();
   }
   return CSAHCA_OK;
 }
@@ -445,7 +521,7 @@ bool attn_tc_shape_ok(int dtype, int H, int d, int rope_dims, int64_t comp_rows,
 
 int launch_attn_tc(const AttnTcParams& p, const void* kv_comp, int64_t comp_rows, const void* win,
                    int64_t win_rows, cudaStream_t s, const char* name) {
-  CUtensorMap m_rows, m_gather, m_win;
+  CUtensorMap m_rows, m_gather, m_win, m_q;
   bool ok = encode_2d(&m_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv_comp, kAttnD, (uint64_t)comp_rows, 64, 128,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_2d(&m_gather, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv_comp, kAttnD, (uint64_t)comp_rows, 64, 1,
@@ -453,13 +529,15 @@ int launch_attn_tc(const AttnTcParams& p, const void* kv_comp, int64_t comp_rows
   if (win) ok = ok && encode_2d(&m_win, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, win, kAttnD, (uint64_t)win_rows, 64,
                                 128, CU_TENSOR_MAP_SWIZZLE_128B);
   else m_win = m_rows;
+  ok = ok && encode_2d(&m_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.q, kAttnD, (uint64_t)p.B * p.nq * kAttnH, 64,
+                       kAttnH, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return CSAHCA_ERR_LAUNCH;
   const int smem = AttnSmem::TOTAL;
   cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   if (grid <= 0) return CSAHCA_OK;
   CSAHCA_TRACE(name, s);
-  attn_tc_kernel<<<grid, kAttnTcThreads, smem, s>>>(m_rows, m_gather, m_win, p);
+  attn_tc_kernel<<<grid, kAttnTcThreads, smem, s>>>(m_rows, m_gather, m_win, m_q, p);
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
 }
@@ -583,11 +661,17 @@ DecodeLayout decode_layout(const csahca_decode_args* a) {
   }
   size_t off = 0;
   L.scores_off = off;
-  if (run_indexer) off += align_up((size_t)a->B * (a->N_cap > 0 ? a->N_cap : 1) * 4, 256);
+  if (run_indexer) {
+    csahca_indexer_args ia;
+    memset(&ia, 0, sizeof(ia));
+    ia.q_dtype = a->qI_dtype; ia.k_dtype = a->kI_dtype; ia.B = a->B; ia.nq = 1; ia.HI = a->HI;
+    ia.dI = a->dI; ia.N = a->N_cap; ia.m = a->m; ia.k = a->k;
+    off += align_up(indexer_workspace(&ia), 256);
+  }
   L.idx_off = off;
   if (csa && !a->idx_out) off += align_up((size_t)a->B * a->k * 4, 256);
   L.partial_off = off;
-  off += align_up((size_t)a->B * a->H * L.splits * (a->d + 2) * 4, 256);
+  off += align_up((size_t)a->B * a->H * L.splits * (a->d + 4) * 4, 256);
   L.total = off;
   return L;
 }

@@ -1,0 +1,84 @@
+"""Host runtime around the C ABI: per-rank sharding of decode work, max-over-
+ranks timing, a pre-marshalled decode step (all layers of the interleaved
+CSA / HCA schedule) and its CUDA-graph capture.
+
+Sharding: decode sequences are independent, so N ranks run N replicas, each on
+its own sequences (weak scaling); no collective touches the data path.  The
+only collective is the max over ranks of a measured time.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import dataclasses
+
+import torch
+
+from . import api, native, synth
+
+
+def shard_workload(wl: synth.Workload, rank: int) -> synth.Workload:
+    """The workload rank `rank` runs: same shapes, its own sequences (seed)."""
+    return dataclasses.replace(wl, seed=wl.seed + 1000 * int(rank))
+
+
+def max_over_ranks(x: float, group=None) -> float:
+    """Max of a per-rank float over the default (or given) process group; x
+    itself when torch.distributed is not initialised."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+        return float(x)
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend(group) == "nccl" \
+        else torch.device("cpu")
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())
+
+
+class DecodeStep:
+    """One decode step over every layer of `layers` (as made by
+    synth.decode_inputs): the C-ABI argument structs and workspaces are
+    built once, so a call only enqueues the library's kernels on `stream`."""
+
+    def __init__(self, wl: synth.Workload, layers, stream: torch.cuda.Stream):
+        self.lib = native.lib()
+        self.stream = stream
+        self.calls = []
+        for L in layers:
+            kw = dict(m=L["m"], rope_dims=wl.r, q_gain=L["q_gain"])
+            if L["kind"] == "csa":
+                kw.update(k=wl.k, qI=L["qI"], wI=L["w"], kI=L["kI"], kI_scale=L["kI_scale"])
+            args, out, keep = api.decode_args(L["kind"], L["q"], L["pos"], L["kv"], L["win"],
+                                              L["sinks"], **kw)
+            nbytes = self.lib.csahca_decode_workspace_size(C.byref(args))
+            ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=L["q"].device)
+            args.workspace = ws.data_ptr()
+            args.workspace_bytes = ws.numel()
+            L["out"] = out
+            self.calls.append((args, out, keep, ws))
+        self.outputs = [c[1] for c in self.calls]
+
+    def __call__(self):
+        sh = self.stream.cuda_stream
+        for args, _, _, _ in self.calls:
+            st = self.lib.compressed_attn_decode(C.byref(args), sh)
+            if st != 0:
+                native.check(st, "compressed_attn_decode")
+
+
+class DecodeGraph:
+    """A DecodeStep captured once into a CUDA graph and replayed: the same
+    kernels with the same arguments, without per-launch host work."""
+
+    def __init__(self, step: DecodeStep):
+        self.step = step
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(step.stream):
+            step()                               # warm the lazy set-up outside capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(self.graph, stream=step.stream, capture_error_mode="thread_local"):
+            step()
+        torch.cuda.synchronize()
+
+    def __call__(self):
+        self.graph.replay()
