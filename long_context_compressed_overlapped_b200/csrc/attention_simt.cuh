@@ -17,6 +17,7 @@ namespace csahca {
 constexpr int kSimtHG = 4;           // heads per CTA (one warp each)
 constexpr int kSimtKeys = 32;        // keys per shared-memory chunk
 constexpr int kSimtMaxDPL = 16;      // d <= 512
+constexpr int kCombineMaxSplits = 1024;
 
 struct SimtAttnParams {
   // query side
@@ -199,7 +200,10 @@ struct CombineParams {
 };
 
 template <typename T>
-__global__ void __launch_bounds__(256) attn_combine_kernel(CombineParams p) {
+__global__ void __launch_bounds__(128) attn_combine_kernel(CombineParams p) {
+  // one CTA per (b, q, h); the split weights f_s = e^{m_s - M} / den are
+  // computed once into shared memory, then each thread sums 4 dims
+  __shared__ float wsplit[kCombineMaxSplits];
   const int64_t bqh = blockIdx.x;                   // (b * nq + qi) * H + h
   const int h = (int)(bqh % p.H);
   const int64_t bq = bqh / p.H;
@@ -208,35 +212,58 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(CombineParams p) {
   const int64_t ps = p.d + 4;                       // partial row: m, l, -, -, acc[d]
   const float* P = p.partial + bqh * p.splits * ps;
   const float z = p.sinks[h];
-  float M = z;
-  for (int s = 0; s < p.splits; ++s) M = fmaxf(M, P[(int64_t)s * ps]);
-  float den = expf(z - M);
-  for (int s = 0; s < p.splits; ++s) {
-    const float ms = P[(int64_t)s * ps];
-    if (ms != -INFINITY) den += P[(int64_t)s * ps + 1] * expf(ms - M);
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    float M = z;
+    for (int s = lane; s < p.splits; s += 32) M = fmaxf(M, P[(int64_t)s * ps]);
+    M = warp_max(M);
+    float den = 0.f;
+    for (int s = lane; s < p.splits; s += 32) {
+      const float ms = P[(int64_t)s * ps];
+      const float f = (ms == -INFINITY) ? 0.f : expf(ms - M);
+      wsplit[s] = f;
+      den += P[(int64_t)s * ps + 1] * f;
+    }
+    den = warp_sum(den) + expf(z - M);
+    const float inv = 1.f / den;
+    for (int s = lane; s < p.splits; s += 32) wsplit[s] *= inv;
   }
+  __syncthreads();
   const int r0 = p.d - p.rope_dims;
   T* O = static_cast<T*>(p.out) + bqh * p.d;
-  for (int dim2 = threadIdx.x * 2; dim2 < p.d; dim2 += blockDim.x * 2) {
-    float o0 = 0.f, o1 = 0.f;
-    for (int s = 0; s < p.splits; ++s) {
-      const float* Ps = P + (int64_t)s * ps;
-      const float ms = Ps[0];
-      if (ms == -INFINITY) continue;
-      const float f = expf(ms - M);
-      o0 = fmaf(Ps[4 + dim2], f, o0);
-      o1 = fmaf(Ps[5 + dim2], f, o1);
+  for (int dim4 = threadIdx.x * 4; dim4 < p.d; dim4 += blockDim.x * 4) {
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    int s = 0;
+    for (; s + 4 <= p.splits; s += 4) {
+      float4 a[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) a[u] = *reinterpret_cast<const float4*>(P + (int64_t)(s + u) * ps + 4 + dim4);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float f = wsplit[s + u];
+        o.x = fmaf(a[u].x, f, o.x); o.y = fmaf(a[u].y, f, o.y);
+        o.z = fmaf(a[u].z, f, o.z); o.w = fmaf(a[u].w, f, o.w);
+      }
     }
-    o0 /= den; o1 /= den;
-    if (dim2 >= r0) {
-      float cs, sn;
-      rope_cos_sin(-(double)t, (dim2 - r0) >> 1, p.rope_dims, p.rope_base, &cs, &sn);
-      const float x0 = o0, x1 = o1;
-      o0 = x0 * cs - x1 * sn;
-      o1 = x0 * sn + x1 * cs;
+    for (; s < p.splits; ++s) {
+      const float4 a = *reinterpret_cast<const float4*>(P + (int64_t)s * ps + 4 + dim4);
+      const float f = wsplit[s];
+      o.x = fmaf(a.x, f, o.x); o.y = fmaf(a.y, f, o.y); o.z = fmaf(a.z, f, o.z); o.w = fmaf(a.w, f, o.w);
     }
-    O[dim2] = from_f32<T>(o0);
-    O[dim2 + 1] = from_f32<T>(o1);
+    float v[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+    for (int e = 0; e < 4; e += 2) {
+      const int dim = dim4 + e;
+      if (dim >= r0) {
+        float cs, sn;
+        rope_cos_sin(-(double)t, (dim - r0) >> 1, p.rope_dims, p.rope_base, &cs, &sn);
+        const float x0 = v[e], x1 = v[e + 1];
+        v[e] = x0 * cs - x1 * sn;
+        v[e + 1] = x0 * sn + x1 * cs;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) O[dim4 + e] = from_f32<T>(v[e]);
   }
 }
 

@@ -30,7 +30,7 @@
 
 namespace csahca {
 
-constexpr int kAttnTcThreads = 192;
+constexpr int kAttnTcThreads = 224;   // warps 0-3 softmax, 4 and 6 loads, 5 MMA
 constexpr int kAttnH = 64;          // heads (MMA N of both products)
 constexpr int kAttnD = 512;         // head dim
 constexpr int kAttnChunks = kAttnD / 64;
@@ -40,6 +40,7 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 struct AttnTcParams {
   const __nv_bfloat16* q; const float* q_gain; const float* sinks; const int* pos;
+  const __nv_bfloat16* kv_comp_ptr;  // [B * N, D] compressed rows (gather source)
   int q_norm; float eps; float scale_log2; int rope_dims; double rope_base;
   int B, nq, N, m, k, w;
   int csa;                      // 1: keys = idx rows; 0: every visible entry
@@ -190,15 +191,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
   __shared__ float red[4 * kAttnH];
-  __shared__ float stat_a[kAttnH], stat_b[kAttnH];
-  __shared__ float m_use[kAttnH], alpha[kAttnH], l_run[kAttnH];
+  __shared__ __align__(16) float stat_a[kAttnH];
+  __shared__ float stat_b[kAttnH];
+  __shared__ __align__(16) float m_use[kAttnH];
+  __shared__ float alpha[kAttnH], l_run[kAttnH];
   __shared__ float rope_cs[64], rope_sn[64];
+  __shared__ __align__(16) float gain_s[kAttnD];
+  __shared__ int rows_s[2][128];
   __shared__ int need_rescale;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (int c = 0; c < kAttnChunks; ++c) { mbar_init(&bar_kfull[c], 1); mbar_init(&bar_kempty[c], 1); }
+    for (int c = 0; c < kAttnChunks; ++c) { mbar_init(&bar_kfull[c], 32); mbar_init(&bar_kempty[c], 1); }
     mbar_init(&bar_q_raw, 1);
     mbar_init(&bar_q_empty, 1);
     mbar_init(&bar_q_full, 128);
@@ -216,9 +221,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
   const uint32_t tmem = tmem_base_sh;
   const uint32_t tS = tmem;                 // S^T: columns [0, H)
   const uint32_t tO = tmem + 128;           // O^T M-tile j: columns [128 + j*H, ...)
+  const uint32_t tL = tmem + 128 + kAttnMT * kAttnH;   // per-key-slot partial sums of p: H columns
 
-  if (warp == 4) {
-    // ------------------------------------------------------------ producer
+  if (warp == 4 || warp == 6) {
+    // ------------------------------------------------------------ producers
+    // warp 4 loads chunks 0,1,4,5 (and the raw Q); warp 6 chunks 2,3,6,7
+    const int pw = warp == 4 ? 0 : 1;
     tma_prefetch_desc(&comp_rows);
     tma_prefetch_desc(&comp_gather);
     tma_prefetch_desc(&win_rows);
@@ -228,7 +236,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
       const AttnItem it = attn_item(p, id);
       if (it.tile1 <= it.tile0) continue;
-      {
+      if (pw == 0) {
         // raw Q of this item into the Q buffer once the previous item's
         // score MMAs have read it; normed and roped there by warps 0-3
         int ok = 1;
@@ -248,38 +256,55 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       for (int tile = it.tile0; tile < it.tile1 && !stop; ++tile, ++tcount) {
         const AttnTile T = attn_tile(p, it, tile);
         const uint32_t ph = tcount & 1;
-        int r[4] = {0, 0, 0, 0};
         if (T.src == 0) {
+          // selected rows of this tile (clamped; masked later by the softmax)
           const int* L = p.idx + ((int64_t)it.b * p.nq + it.qi) * p.k + T.list_off;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int j = 4 * lane + e;
+            const int j = lane + 32 * e;
             int v = (j < T.hi) ? __ldg(L + j) : 0;
             v = (v < 0 || v >= p.N) ? 0 : v;
-            r[e] = it.b * p.N + v;
+            rows_s[pw][j] = it.b * p.N + v;
           }
+          __syncwarp();
         }
-        for (int c = 0; c < kAttnChunks; ++c) {
+        for (int cc = 0; cc < kAttnChunks / 2; ++cc) {
+          const int c = 4 * (cc >> 1) + 2 * pw + (cc & 1);
           int ok = 1;
-          if (lane == 0) {
-            ok = mbar_wait(&bar_kempty[c], ph ^ 1, &abort_flag);
-            if (ok) mbar_expect_tx(&bar_kfull[c], AttnSmem::K_CHUNK);
-          }
+          if (lane == 0) ok = mbar_wait(&bar_kempty[c], ph ^ 1, &abort_flag);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) { stop = true; break; }
           uint8_t* dst = sK + c * AttnSmem::K_CHUNK;
           if (T.src == 0) {
-            tma_gather4(dst + (4 * lane) * 128, &comp_gather, c * 64, r[0], r[1], r[2], r[3], &bar_kfull[c]);
-          } else if (lane == 0) {
-            tma_load_2d(dst, T.src == 1 ? &comp_rows : &win_rows, c * 64, T.row0, &bar_kfull[c]);
+            // gathered rows: 8 lanes per 128-byte row segment (coalesced,
+            // conflict-free), 4 rows per instruction, 32 instructions per
+            // chunk; each lane arrives on the chunk's barrier when its copies
+            // have landed, without waiting for them
+            const int piece = lane & 7, rg = lane >> 3;
+            const __nv_bfloat16* base = p.kv_comp_ptr + c * 64 + piece * 8;
+#pragma unroll 8
+            for (int j = 0; j < 32; ++j) {
+              const int r = 4 * j + rg;
+              cp_async16(dst + sw128_offset(r, piece * 16), base + (int64_t)rows_s[pw][r] * kAttnD);
+            }
+            cp_async_arrive_noinc(&bar_kfull[c]);
+          } else {
+            if (lane == 0) {
+              mbar_expect_tx(&bar_kfull[c], AttnSmem::K_CHUNK);
+              tma_load_2d(dst, T.src == 1 ? &comp_rows : &win_rows, c * 64, T.row0, &bar_kfull[c]);
+            } else {
+              mbar_arrive(&bar_kfull[c]);
+            }
           }
         }
       }
     }
     // drain the last loads before the CTA may exit
+    cp_async_wait<0>();
     if (lane == 0 && tcount > 0)
-      for (int c = 0; c < kAttnChunks; ++c) mbar_wait(&bar_kfull[c], (tcount - 1) & 1, &abort_flag);
-    if (lane == 0 && icount > 0) mbar_wait(&bar_q_raw, (icount - 1) & 1, &abort_flag);
+      for (int cc = 0; cc < kAttnChunks / 2; ++cc)
+        mbar_wait(&bar_kfull[4 * (cc >> 1) + 2 * pw + (cc & 1)], (tcount - 1) & 1, &abort_flag);
+    if (pw == 0 && lane == 0 && icount > 0) mbar_wait(&bar_q_raw, (icount - 1) & 1, &abort_flag);
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -298,6 +323,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
           tc_fence_after();
           for (int c = 0; c < kAttnChunks; ++c) {
             if (!mbar_wait(&bar_kfull[c], ph, &abort_flag)) break;
+            fence_proxy_async_smem();
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
@@ -332,6 +358,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     uint32_t tcount = 0, qcount = 0;
     const int r0 = kAttnD - p.rope_dims;
     bool stop = false;                       // uniform over the 128 threads
+    // q gain (same for every head and query) staged once in shared memory
+    for (int x = tid; x < kAttnD; x += 128) gain_s[x] = (p.q_norm && p.q_gain) ? __ldg(p.q_gain + x) : 1.f;
+    named_sync128();
     for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
       const AttnItem it = attn_item(p, id);
       const bool empty = it.tile1 <= it.tile0;
@@ -344,49 +373,66 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
           rope_cs[tid] = cs;
           rope_sn[tid] = sn;
         }
-        if (tid < kAttnH) { m_use[tid] = -INFINITY; l_run[tid] = 0.f; }
+        if (tid < kAttnH) m_use[tid] = -INFINITY;
         if (!mbar_wait128(&bar_q_raw, qcount & 1, &abort_flag)) { stop = true; break; }
         ++qcount;
         uint8_t* chunk = sQ + (lane >> 2) * AttnSmem::Q_CHUNK;
-        for (int hh = 0; hh < kAttnH / 4; ++hh) {
-          const int h = warp * (kAttnH / 4) + hh;
-          uint4* a0 = reinterpret_cast<uint4*>(chunk + sw128_offset(h, (lane & 3) * 32));
-          uint4* a1 = reinterpret_cast<uint4*>(chunk + sw128_offset(h, (lane & 3) * 32 + 16));
-          uint4 r0v = *a0, r1v = *a1;
-          float x[16];
-          {
+        for (int hh = 0; hh < kAttnH / 4; hh += 4) {
+          // four heads at a time: independent reduction chains interleave
+          float x[4][16];
+          uint4* a0[4];
+          uint4* a1[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int h = warp * (kAttnH / 4) + hh + u;
+            a0[u] = reinterpret_cast<uint4*>(chunk + sw128_offset(h, (lane & 3) * 32));
+            a1[u] = reinterpret_cast<uint4*>(chunk + sw128_offset(h, (lane & 3) * 32 + 16));
+            const uint4 r0v = *a0[u], r1v = *a1[u];
             const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&r0v);
             const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&r1v);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              float2 f0 = __bfloat1622float2(h0[i]), f1 = __bfloat1622float2(h1[i]);
-              x[2 * i] = f0.x; x[2 * i + 1] = f0.y; x[8 + 2 * i] = f1.x; x[8 + 2 * i + 1] = f1.y;
+              const float2 f0 = __bfloat1622float2(h0[i]), f1 = __bfloat1622float2(h1[i]);
+              x[u][2 * i] = f0.x; x[u][2 * i + 1] = f0.y; x[u][8 + 2 * i] = f1.x; x[u][8 + 2 * i + 1] = f1.y;
             }
           }
-          float ss = 0.f;
+          float ss[4];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) ss = fmaf(x[e], x[e], ss);
-          const float inv = p.q_norm ? rsqrtf(warp_sum(ss) / (float)kAttnD + p.eps) : 1.f;
+          for (int u = 0; u < 4; ++u) {
+            ss[u] = 0.f;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int dim = lane * 16 + e;
-            x[e] *= inv * (p.q_norm && p.q_gain ? __ldg(p.q_gain + dim) : 1.f);
+            for (int e = 0; e < 16; ++e) ss[u] = fmaf(x[u][e], x[u][e], ss[u]);
           }
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            const int dim = lane * 16 + e;
-            if (dim >= r0) {
-              const int j = (dim - r0) >> 1;
-              const float x0 = x[e], x1 = x[e + 1];
-              x[e] = x0 * rope_cs[j] - x1 * rope_sn[j];
-              x[e + 1] = x0 * rope_sn[j] + x1 * rope_cs[j];
+          for (int o = 16; o >= 1; o >>= 1)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], o);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float inv = p.q_norm ? rsqrtf(ss[u] / (float)kAttnD + p.eps) : 1.f;
+#pragma unroll
+            for (int e = 0; e < 16; e += 4) {
+              const float4 g4 = *reinterpret_cast<const float4*>(gain_s + lane * 16 + e);
+              x[u][e] *= inv * g4.x; x[u][e + 1] *= inv * g4.y; x[u][e + 2] *= inv * g4.z; x[u][e + 3] *= inv * g4.w;
             }
+            if (lane * 16 + 15 >= r0) {
+#pragma unroll
+              for (int e = 0; e < 16; e += 2) {
+                const int dim = lane * 16 + e;
+                if (dim >= r0) {
+                  const int j = (dim - r0) >> 1;
+                  const float x0 = x[u][e], x1 = x[u][e + 1];
+                  x[u][e] = x0 * rope_cs[j] - x1 * rope_sn[j];
+                  x[u][e + 1] = x0 * rope_sn[j] + x1 * rope_cs[j];
+                }
+              }
+            }
+            uint4 o0, o1;
+            store16(reinterpret_cast<__nv_bfloat16*>(&o0), x[u]);
+            store16(reinterpret_cast<__nv_bfloat16*>(&o1), x[u] + 8);
+            *a0[u] = o0;
+            *a1[u] = o1;
           }
-          uint4 o0, o1;
-          store16(reinterpret_cast<__nv_bfloat16*>(&o0), x);
-          store16(reinterpret_cast<__nv_bfloat16*>(&o1), x + 8);
-          *a0 = o0;
-          *a1 = o1;
         }
         fence_proxy_async_smem();
         mbar_arrive(&bar_q_full);
@@ -395,6 +441,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
 
       for (int tile = it.tile0; tile < it.tile1; ++tile, ++tcount) {
         const uint32_t ph = tcount & 1;
+        const bool first = tile == it.tile0;
         const AttnTile T = attn_tile(p, it, tile);
         bool valid = tid >= T.lo && tid < T.hi;
         if (valid && T.src == 0) {
@@ -403,62 +450,113 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
         }
         if (!mbar_wait128(&bar_s_full, ph, &abort_flag)) { stop = true; break; }
         tc_fence_after();
-        float s[kAttnH];
-        load_scores(tS + lane_base, valid, p.scale_log2, s);
-        reduce_heads<true>(s, red, stat_a);             // stat_a = tile max per head
-        if (tid == 0) need_rescale = 0;
-        named_sync128();
-        if (tid < kAttnH) {
-          const float mt = stat_a[tid], mo = m_use[tid];
-          float a = 1.f;
-          if (mt > mo + kRescaleThreshold || (mo == -INFINITY && mt != -INFINITY)) {
-            a = (mo == -INFINITY) ? 0.f : exp2f(mo - mt);
-            m_use[tid] = mt;
-            if (tile != it.tile0) need_rescale = 1;
+        // The running max m_use is raised only when some score of this tile
+        // exceeds it by more than 2^8 (or on the item's first tile); else the
+        // per-tile max is not needed at all.  S stays in TMEM until p_full.
+        bool exceed = first;
+        if (!first) {
+          const float4* mu4 = reinterpret_cast<const float4*>(m_use);
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            float v[32];
+            tmem_ld32(tS + lane_base + half * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 mu = mu4[half * 8 + e4];
+              exceed |= (v[4 * e4 + 0] * p.scale_log2 > mu.x + kRescaleThreshold) |
+                        (v[4 * e4 + 1] * p.scale_log2 > mu.y + kRescaleThreshold) |
+                        (v[4 * e4 + 2] * p.scale_log2 > mu.z + kRescaleThreshold) |
+                        (v[4 * e4 + 3] * p.scale_log2 > mu.w + kRescaleThreshold);
+            }
           }
-          alpha[tid] = a;
+          exceed = exceed && valid;
         }
-        named_sync128();
-        // the previous tile's P.V has finished: P^T may be overwritten and O^T rescaled
-        if (tile != it.tile0) {
+        exceed = group128_any(exceed);
+        bool rescale = false;
+        if (exceed) {
+          {
+            float v[kAttnH];
+            load_scores(tS + lane_base, valid, p.scale_log2, v);
+            reduce_heads<true>(v, red, stat_a);           // stat_a = tile max per head
+          }
+          if (tid == 0) need_rescale = 0;
+          named_sync128();
+          if (tid < kAttnH) {
+            const float mt = stat_a[tid], mo = m_use[tid];
+            float a = 1.f;
+            if (mt > mo + kRescaleThreshold || (mo == -INFINITY && mt != -INFINITY)) {
+              a = (mo == -INFINITY) ? 0.f : exp2f(mo - mt);
+              m_use[tid] = mt;
+              if (!first) need_rescale = 1;
+            }
+            alpha[tid] = a;
+          }
+          named_sync128();
+          rescale = need_rescale != 0;
+        }
+        // the previous tile's P.V has finished: P^T may be overwritten and
+        // O^T / the partial sums rescaled
+        if (!first) {
           if (!mbar_wait128(&bar_pv_done, ph ^ 1, &abort_flag)) { stop = true; break; }
           tc_fence_after();
-          if (need_rescale) {
-#pragma unroll 1
-            for (int mt = 0; mt < kAttnMT; ++mt) {
-#pragma unroll
-              for (int half = 0; half < 2; ++half) {
-                float v[32];
-                const uint32_t a = tO + lane_base + mt * kAttnH + half * 32;
-                tmem_ld32(a, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] *= alpha[half * 32 + e];
-                tmem_st32(a, v);
-              }
-            }
-            tmem_wait_st();
-          }
         }
-        // probabilities from a second read of S (the first was consumed by the reduction)
-        load_scores(tS + lane_base, valid, p.scale_log2, s);
-        tc_fence_before();
-        mbar_arrive(&bar_s_empty);
+        if (rescale) {
+#pragma unroll 1
+          for (int mt = 0; mt <= kAttnMT; ++mt) {            // O^T M-tiles, then the partial sums
 #pragma unroll
-        for (int h = 0; h < kAttnH; ++h) s[h] = (s[h] == -INFINITY) ? 0.f : exp2f(s[h] - m_use[h]);
-        // P^T row tid (64 heads, bf16) into the MN-major SW128 tile
+            for (int half = 0; half < 2; ++half) {
+              float v[32];
+              const uint32_t a = (mt < kAttnMT ? tO + mt * kAttnH : tL) + lane_base + half * 32;
+              tmem_ld32(a, v);
+              tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          uint4 o;
-          store16(reinterpret_cast<__nv_bfloat16*>(&o), s + 8 * j);
-          *reinterpret_cast<uint4*>(sP + sw128_offset(tid, j * 16)) = o;
+              for (int e = 0; e < 32; ++e) v[e] *= alpha[half * 32 + e];
+              tmem_st32(a, v);
+            }
+          }
+          tmem_wait_st();
+        }
+        // p = 2^(S * scale - m) (masked keys give 0), in two halves of 32
+        // heads: P^T row tid into the MN-major SW128 tile, and this key slot's
+        // running sums per head in TMEM
+        {
+          const float4* mu4 = reinterpret_cast<const float4*>(m_use);
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            float v[32];
+            tmem_ld32(tS + lane_base + half * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 mu = mu4[half * 8 + e4];
+              v[4 * e4 + 0] = valid ? fast_exp2(fmaf(v[4 * e4 + 0], p.scale_log2, -mu.x)) : 0.f;
+              v[4 * e4 + 1] = valid ? fast_exp2(fmaf(v[4 * e4 + 1], p.scale_log2, -mu.y)) : 0.f;
+              v[4 * e4 + 2] = valid ? fast_exp2(fmaf(v[4 * e4 + 2], p.scale_log2, -mu.z)) : 0.f;
+              v[4 * e4 + 3] = valid ? fast_exp2(fmaf(v[4 * e4 + 3], p.scale_log2, -mu.w)) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 o;
+              store16(reinterpret_cast<__nv_bfloat16*>(&o), v + 8 * j);
+              *reinterpret_cast<uint4*>(sP + sw128_offset(tid, (half * 4 + j) * 16)) = o;
+            }
+            const uint32_t la = tL + lane_base + half * 32;
+            if (!first) {
+              float l[32];
+              tmem_ld32(la, l);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] += l[e];
+            }
+            tmem_st32(la, v);
+          }
+          tmem_wait_st();
         }
         fence_proxy_async_smem();
         tc_fence_before();
+        mbar_arrive(&bar_s_empty);
         mbar_arrive(&bar_p_full);
-        // running per-head sum of p (overlaps the P.V on the tensor cores)
-        reduce_heads<false>(s, red, stat_b);
-        if (tid < kAttnH) l_run[tid] = l_run[tid] * alpha[tid] + stat_b[tid];
       }
       if (stop) break;
       if (empty && !p.decode) {
@@ -471,6 +569,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       if (!empty) {
         if (!mbar_wait128(&bar_pv_done, (tcount - 1) & 1, &abort_flag)) { stop = true; break; }
         tc_fence_after();
+      }
+      if (!empty) {
+        float v[kAttnH];
+        tmem_ld32(tL + lane_base, *reinterpret_cast<float(*)[32]>(v));
+        tmem_wait_ld();
+        tmem_ld32(tL + lane_base + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+        tmem_wait_ld();
+        reduce_heads<false>(v, red, l_run);            // l_run = sum of p per head
       }
       named_sync128();                                 // l_run / m_use complete
       if (p.decode) {
@@ -525,24 +631,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
         named_sync128();
         __nv_bfloat16* O = p.out + ((int64_t)it.b * p.nq + it.qi) * kAttnH * kAttnD;
         __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sP);   // [64 heads][128 dims] bf16
+        const float4* fac4 = reinterpret_cast<const float4*>(stat_a);
 #pragma unroll 1
         for (int mt = 0; mt < kAttnMT; ++mt) {
           const int dim = mt * 128 + tid;
+          const bool mt_rope = mt * 128 + 127 >= r0;     // uniform over the CTA
           const bool rot = dim >= r0;
-          const int j = (dim - r0) >> 1;
+          const int j = rot ? (dim - r0) >> 1 : 0;
+          const float cs = rot ? rope_cs[j] : 1.f, sn = rot ? rope_sn[j] : 0.f;
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             float v[32];
             tmem_ld32(tO + lane_base + mt * kAttnH + half * 32, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int h = half * 32 + e;
-              float o = v[e] * stat_a[h];
-              const float partner = __shfl_xor_sync(0xffffffffu, o, 1);
-              if (rot) o = (dim & 1) ? fmaf(partner, rope_sn[j], o * rope_cs[j]) : fmaf(-partner, rope_sn[j], o * rope_cs[j]);
-              stage[h * 128 + tid] = __float2bfloat16_rn(o);
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 f = fac4[half * 8 + e4];
+              v[e4 * 4 + 0] *= f.x; v[e4 * 4 + 1] *= f.y; v[e4 * 4 + 2] *= f.z; v[e4 * 4 + 3] *= f.w;
             }
+            if (mt_rope) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const float partner = __shfl_xor_sync(0xffffffffu, v[e], 1);
+                if (rot) v[e] = (dim & 1) ? fmaf(partner, sn, v[e] * cs) : fmaf(-partner, sn, v[e] * cs);
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 32; ++e) stage[(half * 32 + e) * 128 + tid] = __float2bfloat16_rn(v[e]);
           }
           named_sync128();
 #pragma unroll

@@ -17,6 +17,7 @@
 #include "topk_large.cuh"
 #include "attention_simt.cuh"
 #include "indexer_tc.cuh"
+#include "indexer_f8.cuh"
 #include "attention_tc.cuh"
 
 using namespace csahca;
@@ -225,7 +226,7 @@ int indexer_chunk_rows(const csahca_indexer_args* a) {
   return (int)rows;
 }
 
-constexpr int kTopkSmallMaxN = 32768;      // rows up to this length: one CTA per row
+constexpr int kTopkSmallMaxN = kTopkSmemMaxN;   // rows up to this length: one CTA per row
 
 bool topk_uses_large(const csahca_indexer_args* a) { return a->N > kTopkSmallMaxN; }
 
@@ -265,8 +266,10 @@ int launch_topk(const csahca_indexer_args* a, const float* scores, int64_t strid
     tp.scores = scores; tp.row_stride = stride; tp.q_pos = q_pos; tp.idx = idx;
     tp.B = 1; tp.nq = rows; tp.N = a->N; tp.m = a->m; tp.k = a->k;
     tp.q_begin = 0; tp.q_count = rows;
+    const int smem = topk_rows_smem_bytes(a->N > 0 ? a->N : 1);
+    cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     CSAHCA_TRACE("topk_rows", s);
-    topk_rows_kernel<<<rows, kTopkThreads, 0, s>>>(tp);
+    topk_rows_kernel<<<rows, kTopkThreads, smem, s>>>(tp);
     CSAHCA_CHECK_LAUNCH();
     return CSAHCA_OK;
   }
@@ -357,7 +360,34 @@ int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* score
   p.scores = scores; p.score_row_stride = stride;
   p.B = a->B; p.nq = a->nq; p.HI = a->HI; p.N = a->N; p.m = a->m;
   p.q_begin = q0; p.q_count = qc;
-  const bool fp8 = a->k_dtype == CSAHCA_E4M3;
+  if (a->k_dtype == CSAHCA_E4M3) {
+    // e4m3 keys straight into the FP8 tensor cores, one query per work item;
+    // decode spreads each sequence's key tiles over about one CTA per SM
+    const int tiles = (int)ceil_div64(a->N, 128);
+    if (qc == 1) {
+      int splits = num_sms() / (a->B > 0 ? a->B : 1);
+      if (splits > tiles) splits = tiles;
+      if (splits < 1) splits = 1;
+      p.tiles_per_split = (int)ceil_div64(tiles, splits);
+      p.splits = (int)ceil_div64(tiles, p.tiles_per_split);
+      p.n_items = a->B * p.splits;
+    } else {
+      p.splits = 0;
+      p.n_items = a->B * qc;
+    }
+    using Cfg = IdxF8Cfg<64>;
+    CUtensorMap kmap;
+    if (!encode_2d(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->kI, (uint64_t)a->dI, (uint64_t)a->B * a->N, 128, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return CSAHCA_ERR_LAUNCH;
+    cudaFuncSetAttribute(indexer_f8_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+    if (grid <= 0) return CSAHCA_OK;
+    CSAHCA_TRACE("indexer_scores_f8", s);
+    indexer_f8_kernel<64><<<grid, kIdxF8Threads, Cfg::SMEM, s>>>(kmap, static_cast<const __nv_bfloat16*>(a->qI), p);
+    CSAHCA_CHECK_LAUNCH();
+    return CSAHCA_OK;
+  }
   if (qc == 1) {
     const int tiles = (int)ceil_div64(a->N, 128);
     int splits = (int)ceil_div64(2 * num_sms(), a->B);
@@ -366,11 +396,11 @@ int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* score
     p.tiles_per_split = (int)ceil_div64(tiles, splits);
     p.splits = (int)ceil_div64(tiles, p.tiles_per_split);
     p.n_items = a->B * p.splits;
-    return fp8 ? launch_indexer_tc_t<1, true>(a, p, s) : launch_indexer_tc_t<1, false>(a, p, s);
+    return launch_indexer_tc_t<1, false>(a, p, s);
   }
   p.splits = 0;
   p.n_items = a->B * (int)ceil_div64(qc, 4);
-  return fp8 ? launch_indexer_tc_t<4, true>(a, p, s) : launch_indexer_tc_t<4, false>(a, p, s);
+  return launch_indexer_tc_t<4, false>(a, p, s);
 }
 
 int run_indexer(const csahca_indexer_args* a, void* stream) {
@@ -558,6 +588,7 @@ int run_prefill_t(const csahca_attn_args* a, cudaStream_t s) {
     AttnTcParams t;
     memset(&t, 0, sizeof(t));
     t.q = static_cast<const __nv_bfloat16*>(a->q); t.q_gain = a->q_gain; t.sinks = a->sinks; t.pos = nullptr;
+    t.kv_comp_ptr = static_cast<const __nv_bfloat16*>(a->kv_comp);
     t.q_norm = a->q_norm; t.eps = eps; t.scale_log2 = scale * kLog2e; t.rope_dims = a->rope_dims;
     t.rope_base = base; t.B = a->B; t.nq = a->n; t.N = a->N; t.m = a->m; t.k = a->k; t.w = a->w;
     t.csa = a->kind == CSAHCA_CSA; t.idx = a->idx; t.decode = 0;
@@ -709,6 +740,7 @@ int run_decode_t(const csahca_decode_args* a, cudaStream_t s, char* ws) {
     AttnTcParams t;
     memset(&t, 0, sizeof(t));
     t.q = static_cast<const __nv_bfloat16*>(a->q); t.q_gain = a->q_gain; t.sinks = a->sinks; t.pos = a->pos;
+    t.kv_comp_ptr = static_cast<const __nv_bfloat16*>(a->kv_cache);
     t.q_norm = a->q_norm; t.eps = eps; t.scale_log2 = scale * kLog2e; t.rope_dims = a->rope_dims;
     t.rope_base = base; t.B = a->B; t.nq = 1; t.N = a->N_cap; t.m = a->m; t.k = a->k; t.w = a->w;
     t.csa = a->kind == CSAHCA_CSA; t.idx = sel; t.decode = 1;
@@ -737,7 +769,7 @@ int run_decode_t(const csahca_decode_args* a, cudaStream_t s, char* ws) {
   c.rope_dims = a->rope_dims; c.decode = 1; c.rope_base = base;
   {
     CSAHCA_TRACE("attn_combine", s);
-    attn_combine_kernel<T><<<(unsigned)(a->B * a->H), 256, 0, s>>>(c);
+    attn_combine_kernel<T><<<(unsigned)(a->B * a->H), 128, 0, s>>>(c);
   }
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
@@ -749,6 +781,7 @@ int run_decode(const csahca_decode_args* a, void* stream, char* ws, size_t ws_by
   if (a->B == 0) return CSAHCA_OK;
   if ((st = device_ok()) != CSAHCA_OK) return st;
   const DecodeLayout L = decode_layout(a);
+  if (L.splits > kCombineMaxSplits) return CSAHCA_ERR_UNSUPPORTED;
   if (!ws || ws_bytes < L.total) return CSAHCA_ERR_WORKSPACE;
   cudaStream_t s = as_stream(stream);
   return a->dtype == CSAHCA_F32 ? run_decode_t<float>(a, s, ws) : run_decode_t<__nv_bfloat16>(a, s, ws);

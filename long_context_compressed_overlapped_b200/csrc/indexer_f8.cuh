@@ -1,0 +1,246 @@
+// Lightning-indexer scores for e4m3 indexer keys on the FP8 tensor cores
+// ("Paper Breakdown: DeepSeek-V4", section 4, DSA on Compressed KV:
+// I_{t,i} = sum_j w_{t,j} ReLU(qI_{t,j} . kI_i); the keys are stored as e4m3
+// with one fp32 scale per 128-element row).
+//
+// The keys stream from HBM by TMA straight into the A operand of
+// tcgen05.mma.kind::f8f6f4 (128 keys x 128 e4m3 bytes, SW128), with no
+// conversion.  The bf16 indexer query is made an exact e4m3 operand: with a
+// per-head power of two s_h = 2^(E_h - 8), E_h the exponent of the head's
+// largest |q| (so |q / s_h| < 256), every bf16 value x = q / s_h is the sum
+// t0 + t1 of two e4m3 values, t0 = RNE_e4m3(x) and t1 = x - t0.  (x has 8
+// significant bits; t0 keeps the top 4 after rounding, so t1 is an integer
+// multiple of x's last-bit weight of magnitude <= 8 of them, which e4m3
+// holds exactly whenever that weight is >= 2^-9, i.e. for every element of
+// magnitude >= 2^-9 of the head's largest; smaller elements are rounded to
+// within 2^-10 s_h.)  The B operand is therefore the two terms side by side
+// along K, and one accumulation over K = 2 x 128 against the same key tile
+// gives D[i, h] = kI_i . q_h / s_h.  Since s_h > 0 and the key row scale
+// c_i > 0 commute with ReLU, I_{t,i} = c_i sum_h (w_h s_h) ReLU(D[i, h]).
+// Heads whose largest |q| is below 2^-118 (s_h would leave the normal fp32
+// range) contribute nothing.
+//
+// Roles (320 threads): two epilogue groups of 4 warps (warps 0-3, 4-7) take
+// alternate key tiles, so the ReLU / weighted-sum epilogue of one tile
+// overlaps the next; group 0 also writes the split query of each work item.
+// Warp 8 issues the TMA key loads into a 10-stage ring, warp 9 issues the MMAs
+// (N = HI, 8 MMAs of K = 32 per tile) into 4 TMEM accumulators and owns TMEM.
+// Work items as in indexer_tc.cuh: decode = (sequence, range of key tiles),
+// prefill = (sequence, one query, every visible key tile).
+#pragma once
+#include "indexer_tc.cuh"
+
+namespace csahca {
+
+constexpr int kIdxF8Threads = 320;
+constexpr int kIdxF8Stages = 10;
+constexpr int kIdxF8Acc = 4;
+
+template <int HI>
+struct IdxF8Cfg {
+  static constexpr int B_TERM = HI * 128;           // one e4m3 term: HI rows x 128 bytes
+  static constexpr int B_BYTES = 2 * B_TERM;
+  static constexpr int A_BYTES = 128 * 128;         // 128 keys x 128 e4m3
+  static constexpr int SMEM = 1024 + B_BYTES + kIdxF8Stages * A_BYTES;
+  static constexpr int TMEM_COLS = kIdxF8Acc * HI <= 256 ? 256 : 512;
+  static_assert(HI == 64, "two threads per head of a 128-thread group build the split query");
+  static_assert(B_TERM % 1024 == 0, "SW128 operands start on 1024-byte boundaries");
+};
+
+// kind::f8f6f4 instruction descriptor: e4m3 x e4m3 -> fp32, both K-major.
+__host__ __device__ constexpr uint32_t umma_idesc_e4m3(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+template <int HI>
+__global__ void __launch_bounds__(kIdxF8Threads, 1)
+indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* __restrict__ qI, IdxTcParams p) {
+  using Cfg = IdxF8Cfg<HI>;
+  constexpr int NS = kIdxF8Stages, NACC = kIdxF8Acc;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sB = base;
+  uint8_t* sA = sB + Cfg::B_BYTES;
+  __shared__ uint64_t bar_a_full[NS], bar_a_empty[NS];
+  __shared__ uint64_t bar_acc_full[NACC], bar_acc_empty[NACC];
+  __shared__ uint64_t bar_b_full, bar_b_empty, bar_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+  __shared__ float sW[2][HI];                     // per group: w_h * s_h of its current item
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < NS; ++s) { mbar_init(&bar_a_full[s], 1); mbar_init(&bar_a_empty[s], 1); }
+    for (int j = 0; j < NACC; ++j) { mbar_init(&bar_acc_full[j], 1); mbar_init(&bar_acc_empty[j], 128); }
+    mbar_init(&bar_b_full, 128);
+    mbar_init(&bar_b_empty, 1);
+    mbar_init(&bar_done, 1);
+    mbar_fence_init();
+  }
+  if (warp == 9) tmem_alloc(&tmem_base_sh, Cfg::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&kmap);
+      uint32_t a_iter = 0;
+      for (int id = blockIdx.x; id < p.n_items && !abort_flag; id += gridDim.x) {
+        const IdxItem it = idx_item<1>(p, id);
+        for (int kt = it.kt0; kt < it.kt1; ++kt, ++a_iter) {
+          const int s = a_iter % NS;
+          const uint32_t ph = (a_iter / NS) & 1;
+          if (!mbar_wait(&bar_a_empty[s], ph ^ 1, &abort_flag)) break;
+          mbar_expect_tx(&bar_a_full[s], Cfg::A_BYTES);
+          tma_load_2d(sA + s * Cfg::A_BYTES, &kmap, 0, it.b * p.N + kt * 128, &bar_a_full[s]);
+        }
+      }
+      // drain: every issued fill has landed before the CTA may exit
+      for (uint32_t i = (a_iter > NS ? a_iter - NS : 0); i < a_iter; ++i)
+        mbar_wait(&bar_a_full[i % NS], (i / NS) & 1, &abort_flag);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_e4m3(128, HI);
+      uint32_t a_iter = 0, b_iter = 0, acc_iter = 0;
+      const uint32_t sA0 = smem_u32(sA), sB0 = smem_u32(sB);
+      for (int id = blockIdx.x; id < p.n_items && !abort_flag; id += gridDim.x) {
+        const IdxItem it = idx_item<1>(p, id);
+        if (it.kt1 <= it.kt0) continue;
+        if (!mbar_wait(&bar_b_full, b_iter & 1, &abort_flag)) break;
+        ++b_iter;
+        bool ok = true;
+        for (int kt = it.kt0; kt < it.kt1; ++kt, ++a_iter, ++acc_iter) {
+          const int s = a_iter % NS;
+          const uint32_t ph = (a_iter / NS) & 1;
+          const int j = acc_iter % NACC;
+          const uint32_t aph = (acc_iter / NACC) & 1;
+          if (!mbar_wait(&bar_a_full[s], ph, &abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&bar_acc_empty[j], aph ^ 1, &abort_flag)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              umma_e4m3(tmem + j * HI, umma_desc_kmajor(sA0 + s * Cfg::A_BYTES + ks * 32),
+                        umma_desc_kmajor(sB0 + t * Cfg::B_TERM + ks * 32), idesc, (t | ks) != 0);
+          umma_commit(&bar_a_empty[s]);
+          umma_commit(&bar_acc_full[j]);
+        }
+        if (!ok) break;
+        umma_commit(&bar_b_empty);
+      }
+      umma_commit(&bar_done);
+      mbar_wait(&bar_done, 0, &abort_flag);
+    }
+  } else {
+    // ------------------------------------------------------------ split query + epilogue (2 groups)
+    const int g = warp >> 2;                         // group 0: warps 0-3, group 1: warps 4-7
+    const int bar_id = 1 + g;
+    const int et = threadIdx.x & 127;                // key lane within a tile
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    uint32_t acc_iter = 0, b_iter = 0;
+    bool stop = false;                               // uniform over the group
+    for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
+      const IdxItem it = idx_item<1>(p, id);
+      if (it.kt1 <= it.kt0) continue;
+      // group 0 rewrites B once the previous item's MMAs have read it
+      if (g == 0 && !mbar_wait_group(bar_id, &bar_b_empty, (b_iter & 1) ^ 1, &abort_flag)) { stop = true; break; }
+      ++b_iter;
+      {
+        // thread (h = et / 2, half = et % 2) owns 64 dims of head h
+        const int h = et >> 1, half = et & 1;
+        const int64_t qrow = ((int64_t)it.b * p.nq + it.q0) * HI + h;
+        const __nv_bfloat16* src = qI + qrow * 128 + half * 64;
+        float r[64];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) load16(src + 8 * i, r + 8 * i);
+        float mx = 0.f;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) mx = fmaxf(mx, fabsf(r[e]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        int E = 0;
+        frexpf(mx, &E);                              // mx = f * 2^E, f in [0.5, 1)
+        const bool live = mx >= 0x1p-118f;
+        const float s_h = live ? ldexpf(1.f, E - 8) : 0.f;
+        const float inv = live ? ldexpf(1.f, 8 - E) : 0.f;
+        if (g == 0) {
+#pragma unroll
+          for (int pc = 0; pc < 4; ++pc) {           // 16 dims -> 16 bytes of each term
+            uint32_t w0[4], w1[4];                   // packed explicitly: element e in byte e % 4
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) {
+              uint32_t lo0 = 0, lo1 = 0;
+#pragma unroll
+              for (int pr = 0; pr < 2; ++pr) {
+                const int e = pc * 16 + wd * 4 + pr * 2;
+                const float x0 = r[e] * inv, x1 = r[e + 1] * inv;
+                const __nv_fp8x2_storage_t c0 =
+                    __nv_cvt_float2_to_fp8x2(make_float2(x0, x1), __NV_SATFINITE, __NV_E4M3);
+                const float2 back = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(c0, __NV_E4M3)));
+                const __nv_fp8x2_storage_t c1 =
+                    __nv_cvt_float2_to_fp8x2(make_float2(x0 - back.x, x1 - back.y), __NV_SATFINITE, __NV_E4M3);
+                lo0 |= (uint32_t)c0 << (16 * pr);
+                lo1 |= (uint32_t)c1 << (16 * pr);
+              }
+              w0[wd] = lo0;
+              w1[wd] = lo1;
+            }
+            *reinterpret_cast<uint4*>(sB + sw128_offset(h, half * 64 + pc * 16)) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+            *reinterpret_cast<uint4*>(sB + Cfg::B_TERM + sw128_offset(h, half * 64 + pc * 16)) =
+                make_uint4(w1[0], w1[1], w1[2], w1[3]);
+          }
+        }
+        if (half == 0) sW[g][h] = p.w[((int64_t)it.b * p.nq + it.q0) * HI + h] * s_h;
+        if (g == 0) {
+          fence_proxy_async_smem();
+          mbar_arrive(&bar_b_full);
+        }
+        group_sync(bar_id);                          // sW[g] complete
+      }
+      const int v = idx_visible(p, it.b, it.q0);
+      float* srow = p.scores + ((int64_t)it.b * p.q_count + (it.q0 - p.q_begin)) * p.score_row_stride;
+      for (int kt = it.kt0; kt < it.kt1; ++kt, ++acc_iter) {
+        if ((int)(acc_iter & 1) != g) continue;      // the other group's tile
+        const int j = acc_iter % NACC;
+        const uint32_t aph = (acc_iter / NACC) & 1;
+        if (!mbar_wait_group(bar_id, &bar_acc_full[j], aph, &abort_flag)) { stop = true; break; }
+        tc_fence_after();
+        const int key = kt * 128 + et;
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < HI / 32; ++c) {
+          float d[32];
+          tmem_ld32(tmem + lane_base + j * HI + c * 32, d);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) acc = fmaf(sW[g][c * 32 + e], fmaxf(d[e], 0.f), acc);
+        }
+        tc_fence_before();
+        mbar_arrive(&bar_acc_empty[j]);
+        if (key < v) srow[key] = acc * __ldg(p.kI_scale + (int64_t)it.b * p.N + key);
+      }
+      if (stop) break;
+      group_sync(bar_id);                            // sW[g] may be rewritten
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) tmem_dealloc(tmem, Cfg::TMEM_COLS);
+}
+
+}  // namespace csahca

@@ -286,4 +286,5 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
   if (warp == 5) tmem_dealloc(tmem, Cfg::TMEM_COLS);
 }
 
+
 }  // namespace csahca

@@ -78,10 +78,38 @@ __device__ __forceinline__ bool group128_all(bool ok) {
       : "memory");
   return r != 0;
 }
+// OR of `v` over the 128 threads of named barrier 1.
+__device__ __forceinline__ bool group128_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
 __device__ __forceinline__ bool mbar_wait128(uint64_t* bar, uint32_t parity, volatile int* abort) {
   return group128_all(mbar_wait(bar, parity, abort));
 }
 __device__ __forceinline__ void named_sync128() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// The same three group operations on named barrier `id` (128 threads), for
+// kernels with more than one 128-thread group.
+__device__ __forceinline__ bool group_all(int id, bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)ok), "r"(id)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void group_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+__device__ __forceinline__ bool mbar_wait_group(int id, uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return group_all(id, mbar_wait(bar, parity, abort));
+}
 
 // ---- TMA ----------------------------------------------------------------------
 
@@ -102,6 +130,26 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, i
         "r"(smem_u32(bar))
       : "memory");
 }
+// 16-byte global -> shared copy (L2 only); completion is tracked per thread
+// and signalled to an mbarrier with cp_async_arrive_noinc().
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src_gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Arrive once on `bar` when every cp.async this thread issued so far has
+// landed (counted in the barrier's expected arrivals; the thread does not wait).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Wait until at most N of this thread's committed cp.async groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -227,14 +227,10 @@ __global__ void __launch_bounds__(1024) topk_finish_kernel(TopkLargeParams p) {
       if ((key & mask) == prefix) atomicAdd(&hist8[(key >> sh) & dm], 1u);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      uint32_t cum = 0, digit = 0, nd = sh_need;
-      for (int d = (int)dm; d >= 0; --d) {
-        if (cum + hist8[d] >= nd) { digit = (uint32_t)d; break; }
-        cum += hist8[d];
-      }
-      sh_digit = digit;
-      sh_need = nd - cum;
+    if ((threadIdx.x >> 5) == 0) {
+      const uint32_t nd = sh_need;
+      __syncwarp();
+      find_digit_warp(hist8, (int)dm + 1 >= 32 ? (int)dm + 1 : 32, nd, &sh_digit, &sh_need);
     }
     __syncthreads();
     prefix |= sh_digit << sh;
