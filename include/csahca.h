@@ -153,6 +153,31 @@ typedef struct {
 int indexer_topk(const csahca_indexer_args* args, void* stream);
 size_t csahca_indexer_workspace_size(const csahca_indexer_args* args);
 
+/* ---- indexer_topk_noalloc --------------------------------------------------
+ * No counterpart on the pages: an addition of this library for callers that
+ * cannot allocate device memory when they call it (for example code running
+ * inside a pre-planned memory pool, or a host thread that must not touch the
+ * allocator).  Computes exactly what indexer_topk computes, with the same
+ * arguments and results, but allocates nothing and takes no workspace: the
+ * score rows and top-k buffers live in one fixed __device__ array of
+ * CSAHCA_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits.  args->workspace and
+ * args->workspace_bytes are ignored.
+ *   - A problem whose scratch (csahca_indexer_workspace_size of the same
+ *     args) exceeds CSAHCA_NOALLOC_SCRATCH_BYTES is rejected with
+ *     CSAHCA_ERR_WORKSPACE before any launch.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current, and caches it; make that
+ *     first call outside any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents (the parts that must start at zero are cleared by each call).
+ *     Calls whose work overlaps on the GPU (other streams, or other host
+ *     threads) race on it: serialise them.
+ *   - Calls no cudaMalloc / cudaFree and no allocating library routine. */
+#define CSAHCA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+int indexer_topk_noalloc(const csahca_indexer_args* args, void* stream);
+
 /* ---- compressed_attn_prefill ----------------------------------------------
  * [P2] MQA core attention, sliding window, HCA dense attention, Additional
  * Techniques; [P5] Local window.  For sequence b, query t (position t), head h:

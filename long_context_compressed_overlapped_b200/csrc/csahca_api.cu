@@ -7,6 +7,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
 #include <vector>
 
 #include "../../include/csahca.h"
@@ -900,3 +901,56 @@ int csahca_device_error(void* stream, int32_t* code) {
 }
 
 }  // extern "C"
+
+// ======================================================= allocation-free ======
+// indexer_topk_noalloc: indexer_topk with its scratch (score rows and the
+// multi-CTA top-k buffers) in a fixed device array of this library instead of
+// a caller-provided workspace.  It exists for callers that cannot allocate
+// device memory at the point of the call.  The array is a file-scope
+// __device__ object, so every GPU that loads the library holds it until the
+// process exits.
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = CSAHCA_NOALLOC_SCRATCH_BYTES;
+constexpr int kNoAllocMaxDevices = 64;
+
+// Host code must not pass the array's name to a kernel: on the host it is only
+// a stand-in symbol.  Its device address comes from cudaGetSymbolAddress, once
+// per device (with that device current), and is cached here.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices];
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { (void)cudaGetLastError(); return CSAHCA_ERR_NO_DEVICE; }
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return CSAHCA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      (void)cudaGetLastError();
+      return CSAHCA_ERR_LAUNCH;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return CSAHCA_OK;
+}
+
+}  // namespace
+
+extern "C" int indexer_topk_noalloc(const csahca_indexer_args* args, void* stream) {
+  int st = validate_indexer(args);
+  if (st != CSAHCA_OK) return st;
+  if (args->B == 0 || args->nq == 0) return CSAHCA_OK;
+  if (indexer_workspace(args) > kNoAllocScratchBytes) return CSAHCA_ERR_WORKSPACE;
+  if ((st = device_ok()) != CSAHCA_OK) return st;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != CSAHCA_OK) return st;
+  csahca_indexer_args a = *args;
+  a.workspace = scratch;
+  a.workspace_bytes = kNoAllocScratchBytes;
+  return run_indexer(&a, stream);
+}

@@ -21,6 +21,8 @@ ERR_LAUNCH = -5
 ERR_DEVICE_TIMEOUT = -6
 ERR_NO_DEVICE = -7
 
+NOALLOC_SCRATCH_BYTES = 32 << 20    # CSAHCA_NOALLOC_SCRATCH_BYTES
+
 F32, BF16, E4M3 = 0, 1, 2
 CSA, HCA = 0, 1
 
@@ -75,6 +77,7 @@ SIGNATURES = {
     "hca_compress": (C.c_int, [C.POINTER(CompressArgs), vp]),
     "indexer_topk": (C.c_int, [C.POINTER(IndexerArgs), vp]),
     "csahca_indexer_workspace_size": (sz, [C.POINTER(IndexerArgs)]),
+    "indexer_topk_noalloc": (C.c_int, [C.POINTER(IndexerArgs), vp]),
     "compressed_attn_prefill": (C.c_int, [C.POINTER(AttnArgs), vp]),
     "csahca_prefill_workspace_size": (sz, [C.POINTER(AttnArgs)]),
     "compressed_attn_decode": (C.c_int, [C.POINTER(DecodeArgs), vp]),
