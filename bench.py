@@ -81,61 +81,127 @@ def max_over_ranks(x: float, world: int) -> float:
 # ------------------------------------------------------------------ clocks ----
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples every 200 ms (this GPU)."""
+    """SM clock and throttle reasons of this GPU, sampled through NVML every
+    2 ms by a host thread while the timed loop runs (nvidia-smi reads the same
+    counters; its 200 ms period is too coarse for a timed region of tens of
+    milliseconds).  Falls back to nvidia-smi -lms 200 if NVML is unavailable."""
 
-    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device: int):
-        self.uuid = None
-        try:
-            u = str(torch.cuda.get_device_properties(device).uuid)
-            self.uuid = u if u.startswith("GPU-") else "GPU-" + u
-        except Exception:
-            pass
+    def __init__(self, device: int, period_s: float = 0.002):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.handle = None
+        self.thread = None
         self.proc = None
-        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.handle = None
+
+    def _loop(self):
+        n = self.nvml
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append(float(n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)))
+                bits = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                for name, bit in self.REASONS.items():
+                    if bits & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def start(self):
+        self.samples, self.reasons = [], set()
+        if self.handle is not None:
+            self.stop_flag = threading.Event()
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
+            return
         try:
+            self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
             self.fh = open(self.path, "w")
-            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                   "-lms", "200"]
+            cmd = ["nvidia-smi", "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                   "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                   "clocks_event_reasons.sw_power_cap", "--format=csv,noheader,nounits", "-lms", "200"]
             self.proc = subprocess.Popen(cmd, stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.fh.close()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join()
+            src = "nvml"
+        elif self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            with open(self.path) as f:
+                for line in f:
+                    parts = [x.strip() for x in line.split(",")]
+                    try:
+                        self.samples.append(float(parts[0]))
+                        self.max_mhz = float(parts[1])
+                    except (ValueError, IndexError):
+                        continue
+                    for nm, val in zip(names, parts[2:6]):
+                        if val.lower().startswith("active"):
+                            self.reasons.add(nm)
+            os.unlink(self.path)
+            src = "nvidia-smi"
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"], "samples": 0}
+        sm = self.samples
+        busy = [x for x in sm if self.max_mhz and x > 0.5 * self.max_mhz] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(sm), "source": src}
+
+
+# ------------------------------------------------------- committed ncu data ----
+
+def ncu_traffic(kernel_name):
+    """DRAM bytes per launch of `kernel_name` from the committed ncu summary
+    (profiles/*.md lines `kernel:`, `source_sha256:`, `dram_bytes_per_launch:`),
+    used only while the kernel's source file still has the hash the capture
+    was taken with; None otherwise."""
+    import glob
+    import hashlib
+    for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        meta = {}
+        with open(path) as f:
             for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 10:
-                    continue
-                if self.uuid and parts[1] != self.uuid and not (len(parts[1]) > 4 and self.uuid.endswith(parts[1][4:])):
-                    continue
-                try:
-                    sm.append(float(parts[2]))
-                    smax = float(parts[3])
-                except ValueError:
-                    continue
-                for nm, val in zip(names, parts[6:10]):
-                    if val.lower().startswith("active"):
-                        reasons.add(nm)
-        os.unlink(self.path)
-        busy = [x for x in sm if smax and x > 0.5 * smax] or sm
-        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                if ":" in line and line.split(":", 1)[0].strip() in ("kernel", "source", "source_sha256",
+                                                                      "dram_bytes_per_launch"):
+                    k_, v_ = line.split(":", 1)
+                    meta[k_.strip()] = v_.strip().strip("`")
+        if meta.get("kernel") != kernel_name or "source" not in meta:
+            continue
+        src = os.path.join(ROOT, meta["source"])
+        if not os.path.exists(src):
+            continue
+        with open(src, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != meta.get("source_sha256"):
+                continue
+        try:
+            return float(meta["dram_bytes_per_launch"])
+        except (KeyError, ValueError):
+            return None
+    return None
 
 
 # ----------------------------------------------------------- decode step ----
@@ -336,7 +402,7 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode_1m")
@@ -401,7 +467,7 @@ def main():
     if key is not None:
         ach = per_bytes[key] / (dms / dl / 1000.0) / 1e9
         roof = {"kernel": dname, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": ach / pk["hbm_gbs"], "traffic": None,
+                "unit": "GB/s", "frac": ach / pk["hbm_gbs"], "traffic": ncu_traffic(dname),
                 "peak_source": pk["source"], "launches": dl, "avg_us": 1000 * dms / dl}
     step_bytes = decode_step_bytes(wl, wl.ctx)
     step_frac = step_bytes / (ms_per_step / 1000.0) / 1e9 / pk["hbm_gbs"]

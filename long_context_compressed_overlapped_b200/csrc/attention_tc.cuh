@@ -153,18 +153,19 @@ __device__ __forceinline__ void reduce_heads(float (&v)[kAttnH], float* red, flo
   named_sync128();
 }
 
-// S^T row of this thread (64 heads) from TMEM, scaled to log2 units; -inf
-// for a masked key.
-__device__ __forceinline__ void load_scores(uint32_t taddr, bool valid, float scale_log2, float (&s)[kAttnH]) {
+// S^T row of this thread (64 heads) from TMEM, times each head's scale (log2
+// units); -inf for a masked key.
+__device__ __forceinline__ void load_scores(uint32_t taddr, bool valid, const float* scale_log2,
+                                            float (&s)[kAttnH]) {
   float v[32];
   tmem_ld32(taddr, v);
   tmem_wait_ld();
 #pragma unroll
-  for (int e = 0; e < 32; ++e) s[e] = valid ? v[e] * scale_log2 : -INFINITY;
+  for (int e = 0; e < 32; ++e) s[e] = valid ? v[e] * scale_log2[e] : -INFINITY;
   tmem_ld32(taddr + 32, v);
   tmem_wait_ld();
 #pragma unroll
-  for (int e = 0; e < 32; ++e) s[32 + e] = valid ? v[e] * scale_log2 : -INFINITY;
+  for (int e = 0; e < 32; ++e) s[32 + e] = valid ? v[e] * scale_log2[32 + e] : -INFINITY;
 }
 
 struct AttnSmem {
@@ -175,6 +176,15 @@ struct AttnSmem {
   static constexpr int P_BYTES = 128 * 128;                  // 16 KB
   static constexpr int TOTAL = 1024 + Q_BYTES + K_BYTES + P_BYTES;
 };
+
+// Decode partial of one (query, split): m[H], l[H] fp32, then O / l fp16 [D][H].
+constexpr int kTcPartialHeader = 2 * kAttnH * 4;
+constexpr int kTcPartialBytes = kTcPartialHeader + kAttnD * kAttnH * 2;
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  const __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
 
 __global__ void __launch_bounds__(kAttnTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_constant__ CUtensorMap comp_gather,
@@ -192,8 +202,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
   __shared__ volatile int abort_flag;
   __shared__ float red[4 * kAttnH];
   __shared__ __align__(16) float stat_a[kAttnH];
-  __shared__ float stat_b[kAttnH];
   __shared__ __align__(16) float m_use[kAttnH];
+  __shared__ __align__(16) float sc_h[kAttnH];     // softmax scale of head h (log2 units, times inv_rms_h)
   __shared__ float alpha[kAttnH], l_run[kAttnH];
   __shared__ float rope_cs[64], rope_sn[64];
   __shared__ __align__(16) float gain_s[kAttnD];
@@ -222,6 +232,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
   const uint32_t tS = tmem;                 // S^T: columns [0, H)
   const uint32_t tO = tmem + 128;           // O^T M-tile j: columns [128 + j*H, ...)
   const uint32_t tL = tmem + 128 + kAttnMT * kAttnH;   // per-key-slot partial sums of p: H columns
+  griddep_launch_dependents();
 
   if (warp == 4 || warp == 6) {
     // ------------------------------------------------------------ producers
@@ -253,6 +264,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
         if (!ok) { stop = true; break; }
         ++icount;
       }
+      // key rows and selections may come from earlier kernels of this stream;
+      // the query (a caller input) was already on its way
+      griddep_wait();
       for (int tile = it.tile0; tile < it.tile1 && !stop; ++tile, ++tcount) {
         const AttnTile T = attn_tile(p, it, tile);
         const uint32_t ph = tcount & 1;
@@ -310,7 +324,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     if (lane == 0) {
       constexpr uint32_t idesc_s = umma_idesc_bf16(128, kAttnH, 0, 0);
       constexpr uint32_t idesc_pv = umma_idesc_bf16(128, kAttnH, 1, 1);
-      const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), p0 = smem_u32(sP);
+      // base descriptors; chunk / K-step offsets are adds in 16-byte units
+      const uint64_t kdesc = umma_desc_kmajor(smem_u32(sK)), qdesc = umma_desc_kmajor(smem_u32(sQ));
+      const uint64_t vdesc = umma_desc_mnmajor(smem_u32(sK), AttnSmem::K_CHUNK);
+      const uint64_t pdesc = umma_desc_mnmajor(smem_u32(sP), AttnSmem::P_BYTES);
       uint32_t tcount = 0, icount = 0;
       for (int id = blockIdx.x; id < p.n_items && !abort_flag; id += gridDim.x) {
         const AttnItem it = attn_item(p, id);
@@ -325,10 +342,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
             if (!mbar_wait(&bar_kfull[c], ph, &abort_flag)) break;
             fence_proxy_async_smem();
             tc_fence_after();
+            const uint64_t kd = kdesc + (uint64_t)(c * (AttnSmem::K_CHUNK >> 4));
+            const uint64_t qd = qdesc + (uint64_t)(c * (AttnSmem::Q_CHUNK >> 4));
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-              umma_bf16(tS, umma_desc_kmajor(k0 + c * AttnSmem::K_CHUNK + ks * 32),
-                        umma_desc_kmajor(q0 + c * AttnSmem::Q_CHUNK + ks * 32), idesc_s, (c | ks) != 0);
+            for (int ks = 0; ks < 4; ++ks) umma_bf16(tS, kd + 2 * ks, qd + 2 * ks, idesc_s, (c | ks) != 0);
           }
           umma_commit(&bar_s_full);
           if (tile == it.tile1 - 1) umma_commit(&bar_q_empty);
@@ -337,11 +354,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
           const bool first = tile == it.tile0;
 #pragma unroll
           for (int mt = 0; mt < kAttnMT; ++mt) {
+            const uint64_t vd = vdesc + (uint64_t)((2 * mt) * (AttnSmem::K_CHUNK >> 4));
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-              umma_bf16(tO + mt * kAttnH,
-                        umma_desc_mnmajor(k0 + (2 * mt) * AttnSmem::K_CHUNK + ks * 2048, AttnSmem::K_CHUNK),
-                        umma_desc_mnmajor(p0 + ks * 2048, AttnSmem::P_BYTES), idesc_pv, !(first && ks == 0));
+              umma_bf16(tO + mt * kAttnH, vd + 128 * ks, pdesc + 128 * ks, idesc_pv, !(first && ks == 0));
             umma_commit(&bar_kempty[2 * mt]);
             umma_commit(&bar_kempty[2 * mt + 1]);
           }
@@ -358,14 +374,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     uint32_t tcount = 0, qcount = 0;
     const int r0 = kAttnD - p.rope_dims;
     bool stop = false;                       // uniform over the 128 threads
-    // q gain (same for every head and query) staged once in shared memory
-    for (int x = tid; x < kAttnD; x += 128) gain_s[x] = (p.q_norm && p.q_gain) ? __ldg(p.q_gain + x) : 1.f;
-    named_sync128();
+    // q gain (same for every head and query) staged once in shared memory;
+    // an all-ones gain (or none) leaves the non-rope dims of q untouched
+    bool ones = true;
+    for (int x = tid; x < kAttnD; x += 128) {
+      const float g = (p.q_norm && p.q_gain) ? __ldg(p.q_gain + x) : 1.f;
+      gain_s[x] = g;
+      ones = ones && g == 1.f;
+    }
+    const bool gain_ones = group128_all(ones);
     for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
       const AttnItem it = attn_item(p, id);
       const bool empty = it.tile1 <= it.tile0;
-      // ---- query prologue: raw Q (landed by TMA in the K-major SW128 layout)
-      // -> RMSNorm * gain, RoPE at t, in place
+      // ---- query prologue.  RoPE is linear and the RMSNorm factor is one
+      // scalar per head, so RoPE_t(RMSNorm(q) * g) = inv_rms_h * RoPE_t(q * g):
+      // the MMA operand is RoPE_t(q * g) (with an all-ones gain only the rope
+      // dims are rewritten), and inv_rms_h joins the softmax scale of head h.
       if (!empty) {
         if (tid < p.rope_dims / 2) {
           float cs, sn;
@@ -376,68 +400,86 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
         if (tid < kAttnH) m_use[tid] = -INFINITY;
         if (!mbar_wait128(&bar_q_raw, qcount & 1, &abort_flag)) { stop = true; break; }
         ++qcount;
-        uint8_t* chunk = sQ + (lane >> 2) * AttnSmem::Q_CHUNK;
-        for (int hh = 0; hh < kAttnH / 4; hh += 4) {
-          // four heads at a time: independent reduction chains interleave
-          float x[4][16];
-          uint4* a0[4];
-          uint4* a1[4];
+        // thread (head h, half) owns dims [256 * half, 256 * half + 256) of row h
+        const int h = tid >> 1, half = tid & 1;
+        float ss = 0.f;
+        if (!gain_ones) {
+          // q * g on every dim (sum of squares from the raw values), RoPE on the rope dims
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            const int chunk = 4 * half + c;
+            uint8_t* row = sQ + chunk * AttnSmem::Q_CHUNK;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int h = warp * (kAttnH / 4) + hh + u;
-            a0[u] = reinterpret_cast<uint4*>(chunk + sw128_offset(h, (lane & 3) * 32));
-            a1[u] = reinterpret_cast<uint4*>(chunk + sw128_offset(h, (lane & 3) * 32 + 16));
-            const uint4 r0v = *a0[u], r1v = *a1[u];
-            const __nv_bfloat162* h0 = reinterpret_cast<const __nv_bfloat162*>(&r0v);
-            const __nv_bfloat162* h1 = reinterpret_cast<const __nv_bfloat162*>(&r1v);
+            for (int pc = 0; pc < 8; ++pc) {
+              uint4* a = reinterpret_cast<uint4*>(row + sw128_offset(h, pc * 16));
+              float x[8];
+              {
+                const uint4 raw = *a;
+                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float2 f0 = __bfloat1622float2(h0[i]), f1 = __bfloat1622float2(h1[i]);
-              x[u][2 * i] = f0.x; x[u][2 * i + 1] = f0.y; x[u][8 + 2 * i] = f1.x; x[u][8 + 2 * i + 1] = f1.y;
-            }
-          }
-          float ss[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            ss[u] = 0.f;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) ss[u] = fmaf(x[u][e], x[u][e], ss[u]);
-          }
-#pragma unroll
-          for (int o = 16; o >= 1; o >>= 1)
-#pragma unroll
-            for (int u = 0; u < 4; ++u) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], o);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float inv = p.q_norm ? rsqrtf(ss[u] / (float)kAttnD + p.eps) : 1.f;
-#pragma unroll
-            for (int e = 0; e < 16; e += 4) {
-              const float4 g4 = *reinterpret_cast<const float4*>(gain_s + lane * 16 + e);
-              x[u][e] *= inv * g4.x; x[u][e + 1] *= inv * g4.y; x[u][e + 2] *= inv * g4.z; x[u][e + 3] *= inv * g4.w;
-            }
-            if (lane * 16 + 15 >= r0) {
-#pragma unroll
-              for (int e = 0; e < 16; e += 2) {
-                const int dim = lane * 16 + e;
-                if (dim >= r0) {
-                  const int j = (dim - r0) >> 1;
-                  const float x0 = x[u][e], x1 = x[u][e + 1];
-                  x[u][e] = x0 * rope_cs[j] - x1 * rope_sn[j];
-                  x[u][e + 1] = x0 * rope_sn[j] + x1 * rope_cs[j];
+                for (int i = 0; i < 4; ++i) {
+                  const float2 f = __bfloat1622float2(h2[i]);
+                  x[2 * i] = f.x; x[2 * i + 1] = f.y;
                 }
               }
+              const int d0 = chunk * 64 + pc * 8;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) { ss = fmaf(x[e], x[e], ss); x[e] *= gain_s[d0 + e]; }
+              if (d0 + 7 >= r0) {
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                  if (d0 + e >= r0) {
+                    const int j = (d0 + e - r0) >> 1;
+                    const float x0 = x[e], x1 = x[e + 1];
+                    x[e] = x0 * rope_cs[j] - x1 * rope_sn[j];
+                    x[e + 1] = x0 * rope_sn[j] + x1 * rope_cs[j];
+                  }
+                }
+              }
+              uint4 o;
+              store16(reinterpret_cast<__nv_bfloat16*>(&o), x);
+              *a = o;
             }
-            uint4 o0, o1;
-            store16(reinterpret_cast<__nv_bfloat16*>(&o0), x[u]);
-            store16(reinterpret_cast<__nv_bfloat16*>(&o1), x[u] + 8);
-            *a0[u] = o0;
-            *a1[u] = o1;
+          }
+        } else {
+          // RoPE on the rope dims only: pairs (r0 + 2j, r0 + 2j + 1), this
+          // thread taking j = half, half + 2, ...
+          for (int j = half; j < p.rope_dims / 2; j += 2) {
+            const int dim = r0 + 2 * j;
+            __nv_bfloat162* a = reinterpret_cast<__nv_bfloat162*>(sQ + (dim >> 6) * AttnSmem::Q_CHUNK +
+                                                                   sw128_offset(h, (dim & 63) * 2));
+            const float2 f = __bfloat1622float2(*a);
+            *a = __floats2bfloat162_rn(f.x * rope_cs[j] - f.y * rope_sn[j], f.x * rope_sn[j] + f.y * rope_cs[j]);
           }
         }
         fence_proxy_async_smem();
         mbar_arrive(&bar_q_full);
+        if (p.q_norm) {
+          if (gain_ones) {
+            // the rotation keeps every pair's norm: sum the squares of the operand
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              const uint8_t* row = sQ + (4 * half + c) * AttnSmem::Q_CHUNK;
+#pragma unroll
+              for (int pc = 0; pc < 8; ++pc) {
+                const uint4 raw = *reinterpret_cast<const uint4*>(row + sw128_offset(h, pc * 16));
+                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const float2 f = __bfloat1622float2(h2[i]);
+                  ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+                }
+              }
+            }
+          }
+          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+          if (half == 0) sc_h[h] = p.scale_log2 * rsqrtf(ss / (float)kAttnD + p.eps);
+        } else if (half == 0) {
+          sc_h[h] = p.scale_log2;
+        }
       }
       named_sync128();
+      griddep_wait();                                // selections read, outputs written below
 
       for (int tile = it.tile0; tile < it.tile1; ++tile, ++tcount) {
         const uint32_t ph = tcount & 1;
@@ -464,10 +506,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
 #pragma unroll
             for (int e4 = 0; e4 < 8; ++e4) {
               const float4 mu = mu4[half * 8 + e4];
-              exceed |= (v[4 * e4 + 0] * p.scale_log2 > mu.x + kRescaleThreshold) |
-                        (v[4 * e4 + 1] * p.scale_log2 > mu.y + kRescaleThreshold) |
-                        (v[4 * e4 + 2] * p.scale_log2 > mu.z + kRescaleThreshold) |
-                        (v[4 * e4 + 3] * p.scale_log2 > mu.w + kRescaleThreshold);
+              const float4 sc = reinterpret_cast<const float4*>(sc_h)[half * 8 + e4];
+              exceed |= (v[4 * e4 + 0] * sc.x > mu.x + kRescaleThreshold) |
+                        (v[4 * e4 + 1] * sc.y > mu.y + kRescaleThreshold) |
+                        (v[4 * e4 + 2] * sc.z > mu.z + kRescaleThreshold) |
+                        (v[4 * e4 + 3] * sc.w > mu.w + kRescaleThreshold);
             }
           }
           exceed = exceed && valid;
@@ -477,7 +520,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
         if (exceed) {
           {
             float v[kAttnH];
-            load_scores(tS + lane_base, valid, p.scale_log2, v);
+            load_scores(tS + lane_base, valid, sc_h, v);
             reduce_heads<true>(v, red, stat_a);           // stat_a = tile max per head
           }
           if (tid == 0) need_rescale = 0;
@@ -530,10 +573,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
 #pragma unroll
             for (int e4 = 0; e4 < 8; ++e4) {
               const float4 mu = mu4[half * 8 + e4];
-              v[4 * e4 + 0] = valid ? fast_exp2(fmaf(v[4 * e4 + 0], p.scale_log2, -mu.x)) : 0.f;
-              v[4 * e4 + 1] = valid ? fast_exp2(fmaf(v[4 * e4 + 1], p.scale_log2, -mu.y)) : 0.f;
-              v[4 * e4 + 2] = valid ? fast_exp2(fmaf(v[4 * e4 + 2], p.scale_log2, -mu.z)) : 0.f;
-              v[4 * e4 + 3] = valid ? fast_exp2(fmaf(v[4 * e4 + 3], p.scale_log2, -mu.w)) : 0.f;
+              const float4 sc = reinterpret_cast<const float4*>(sc_h)[half * 8 + e4];
+              v[4 * e4 + 0] = valid ? fast_exp2(fmaf(v[4 * e4 + 0], sc.x, -mu.x)) : 0.f;
+              v[4 * e4 + 1] = valid ? fast_exp2(fmaf(v[4 * e4 + 1], sc.y, -mu.y)) : 0.f;
+              v[4 * e4 + 2] = valid ? fast_exp2(fmaf(v[4 * e4 + 2], sc.z, -mu.z)) : 0.f;
+              v[4 * e4 + 3] = valid ? fast_exp2(fmaf(v[4 * e4 + 3], sc.w, -mu.w)) : 0.f;
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -580,37 +624,45 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       }
       named_sync128();                                 // l_run / m_use complete
       if (p.decode) {
-        // partial rows [H][D + 4]: m (natural log units), l, -, -, O^T[.][h]
-        float* P = p.partial + (((int64_t)it.b * p.nq + it.qi) * kAttnH * p.splits + it.split) * (kAttnD + 4);
-        const int64_t hstride = (int64_t)p.splits * (kAttnD + 4);
+        // partial block of (query, split): m[H] (log2 units) and l[H] in fp32,
+        // then O / l as fp16 [D][H] (a thread writes its dim's 64 heads, 128
+        // contiguous bytes, straight from TMEM); an empty split writes only
+        // m = -inf, which the combine skips
+        char* P = reinterpret_cast<char*>(p.partial) +
+                  (((int64_t)it.b * p.nq + it.qi) * p.splits + it.split) * kTcPartialBytes;
+        float* hdr = reinterpret_cast<float*>(P);
         if (tid < kAttnH) {
-          P[tid * hstride + 0] = empty ? -INFINITY : m_use[tid] * 0.6931471805599453f;
-          P[tid * hstride + 1] = empty ? 0.f : l_run[tid];
+          const float l = empty ? 0.f : l_run[tid];
+          hdr[tid] = empty ? -INFINITY : m_use[tid];
+          hdr[kAttnH + tid] = l;
+          stat_a[tid] = l > 0.f ? 1.f / l : 0.f;
         }
-        float* stage = reinterpret_cast<float*>(sP);   // [32 heads][128 dims] f32 = 16 KB
+        named_sync128();
+        if (!empty) {
+          const float4* f4 = reinterpret_cast<const float4*>(stat_a);
 #pragma unroll 1
-        for (int mt = 0; mt < kAttnMT; ++mt) {
-#pragma unroll 1
-          for (int half = 0; half < 2; ++half) {
-            float v[32];
-            if (!empty) {
+          for (int mt = 0; mt < kAttnMT; ++mt) {
+            uint4* dst = reinterpret_cast<uint4*>(P + kTcPartialHeader + (int64_t)(mt * 128 + tid) * kAttnH * 2);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              float v[32];
               tmem_ld32(tO + lane_base + mt * kAttnH + half * 32, v);
               tmem_wait_ld();
-            } else {
 #pragma unroll
-              for (int e = 0; e < 32; ++e) v[e] = 0.f;
+              for (int e4 = 0; e4 < 8; ++e4) {
+                const float4 f = f4[half * 8 + e4];
+                v[4 * e4 + 0] *= f.x; v[4 * e4 + 1] *= f.y; v[4 * e4 + 2] *= f.z; v[4 * e4 + 3] *= f.w;
+              }
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                uint4 o;
+                o.x = pack_half2(v[8 * q + 0], v[8 * q + 1]);
+                o.y = pack_half2(v[8 * q + 2], v[8 * q + 3]);
+                o.z = pack_half2(v[8 * q + 4], v[8 * q + 5]);
+                o.w = pack_half2(v[8 * q + 6], v[8 * q + 7]);
+                dst[half * 4 + q] = o;
+              }
             }
-#pragma unroll
-            for (int e = 0; e < 32; ++e) stage[e * 128 + tid] = v[e];
-            named_sync128();
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int piece = tid + 128 * i;           // 16-byte piece: head e = piece / 32
-              const int e = piece >> 5, off = (piece & 31) * 4;
-              const float4 val = *reinterpret_cast<const float4*>(stage + e * 128 + off);
-              *reinterpret_cast<float4*>(P + (half * 32 + e) * hstride + 4 + mt * 128 + off) = val;
-            }
-            named_sync128();
           }
         }
       } else {
@@ -678,6 +730,102 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
   __syncthreads();
   tc_fence_after();
   if (warp == 5) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------
+// Split-KV combine of the tensor-core decode partials, with the sink and the
+// output de-rotation: o = sum_s f_s (O_s / l_s), f_s = l_s 2^(m_s - M) / den,
+// den = 2^(z_h log2 e - M) + sum_s l_s 2^(m_s - M), M the largest of them; the
+// rope dims of o are then rotated by -t.  One CTA per (query, 16 dims): thread
+// (dim dl = tid / 8, heads 8 * (tid % 8) ..) reads 16 contiguous bytes of
+// every split; the split weights of the 64 heads are formed once in shared
+// memory (dynamic: splits x 3 x 64 floats, the weights and the staged m, l
+// headers).
+struct TcCombineParams {
+  const char* partial;        // [B * nq][splits] blocks of kTcPartialBytes
+  const float* sinks;         // [H]
+  const int* pos;             // [B] query positions (decode)
+  __nv_bfloat16* out;         // [B * nq, H, D]
+  int rows, splits, rope_dims;
+  double rope_base;
+};
+
+__global__ void __launch_bounds__(128) attn_combine_tc_kernel(TcCombineParams p) {
+  griddep_launch_dependents();
+  griddep_wait();
+  extern __shared__ float wsplit[];                       // [splits][H]
+  __shared__ __align__(16) __nv_bfloat16 ostage[kAttnH][16];
+  constexpr int kChunks = kAttnD / 16;
+  const int row = blockIdx.x / kChunks, dc = blockIdx.x % kChunks;
+  const char* P0 = p.partial + (int64_t)row * p.splits * kTcPartialBytes;
+  const int tid = threadIdx.x;
+  // every split's m[H], l[H] into shared memory (independent loads in flight),
+  // then the weights of head h = tid from there
+  for (int x = tid; x < p.splits * 2 * kAttnH; x += blockDim.x) {
+    const int sp = x / (2 * kAttnH), e = x % (2 * kAttnH);
+    wsplit[p.splits * kAttnH + x] = __ldcg(reinterpret_cast<const float*>(P0 + (int64_t)sp * kTcPartialBytes) + e);
+  }
+  __syncthreads();
+  if (tid < kAttnH) {
+    const int h = tid;
+    const float* hs = wsplit + p.splits * kAttnH;          // [splits][m[H], l[H]]
+    const float z2 = p.sinks[h] * kLog2e;
+    float M = z2;
+    for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, hs[sp * 2 * kAttnH + h]);
+    float den = exp2f(z2 - M);
+    for (int sp = 0; sp < p.splits; ++sp) {
+      const float ms = hs[sp * 2 * kAttnH + h];
+      const float f = ms == -INFINITY ? 0.f : hs[sp * 2 * kAttnH + kAttnH + h] * exp2f(ms - M);
+      wsplit[sp * kAttnH + h] = f;
+      den += f;
+    }
+    const float inv = 1.f / den;
+    for (int sp = 0; sp < p.splits; ++sp) wsplit[sp * kAttnH + h] *= inv;
+  }
+  __syncthreads();
+  const int dl = tid >> 3, hg = tid & 7;
+  const int dim = dc * 16 + dl;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 4
+  for (int s = 0; s < p.splits; ++s) {
+    const float4 w0 = *reinterpret_cast<const float4*>(wsplit + s * kAttnH + hg * 8);
+    const float4 w1 = *reinterpret_cast<const float4*>(wsplit + s * kAttnH + hg * 8 + 4);
+    if (w0.x == 0.f && w0.y == 0.f && w0.z == 0.f && w0.w == 0.f && w1.x == 0.f && w1.y == 0.f &&
+        w1.z == 0.f && w1.w == 0.f)
+      continue;                                            // empty split: O was not written
+    const uint4 raw = __ldcg(reinterpret_cast<const uint4*>(P0 + (int64_t)s * kTcPartialBytes + kTcPartialHeader +
+                                                           ((int64_t)dim * kAttnH + hg * 8) * 2));
+    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(h2[i]);
+      acc[2 * i] = fmaf(wv[2 * i], f.x, acc[2 * i]);
+      acc[2 * i + 1] = fmaf(wv[2 * i + 1], f.y, acc[2 * i + 1]);
+    }
+  }
+  // rope dims: the pair partner (dim ^ 1) is thread tid ^ 8
+  const int r0 = kAttnD - p.rope_dims;
+  float partner[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) partner[i] = __shfl_xor_sync(0xffffffffu, acc[i], 8);
+  if (dim >= r0) {
+    float cs, sn;
+    rope_cos_sin(-(double)p.pos[row], (dim - r0) >> 1, p.rope_dims, p.rope_base, &cs, &sn);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      acc[i] = (dim & 1) ? fmaf(partner[i], sn, acc[i] * cs) : fmaf(-partner[i], sn, acc[i] * cs);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ostage[hg * 8 + i][dl] = __float2bfloat16_rn(acc[i]);
+  __syncthreads();
+  {
+    const int h = tid >> 1, piece = tid & 1;
+    *reinterpret_cast<uint4*>(p.out + ((int64_t)row * kAttnH + h) * kAttnD + dc * 16 + piece * 8) =
+        *reinterpret_cast<const uint4*>(&ostage[h][piece * 8]);
+  }
 }
 
 }  // namespace csahca

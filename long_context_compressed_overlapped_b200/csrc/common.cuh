@@ -94,4 +94,18 @@ __device__ __forceinline__ void rope_cos_sin(double pos, int j, int r, double ba
 
 __host__ __device__ __forceinline__ int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// ---- programmatic dependent launch --------------------------------------------
+// Every kernel of the library is launched so that it may start while the
+// previous kernel in the stream finishes.  Before its first read of global
+// data that an earlier kernel of the library may write (compressed rows,
+// scores, selections, partials) and before its first global write, a thread
+// calls griddep_wait(), which returns once every prerequisite grid has
+// completed and its writes are visible (at once when there is none).  Work
+// before it touches only shared memory, TMEM, kernel parameters and the
+// caller's inputs that no kernel of the library writes.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel in the stream be scheduled once every CTA of this grid
+// has issued it or exited.
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 }  // namespace csahca

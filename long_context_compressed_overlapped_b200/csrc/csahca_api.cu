@@ -5,9 +5,11 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "../../include/csahca.h"
@@ -68,6 +70,36 @@ constexpr float kDefaultEps = 1e-6f;
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Every launch goes through launch_k: programmatic dependent launch lets a
+// kernel start (barrier set-up, TMEM allocation, loads of caller inputs)
+// while the previous kernel in the stream finishes; each kernel waits
+// (griddep_wait) before touching what earlier kernels write.  CSAHCA_PDL=0 in
+// the environment launches plainly instead.
+bool pdl_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = getenv("CSAHCA_PDL");
+    on = (e && e[0] == '0') ? 0 : 1;
+  }
+  return on == 1;
+}
+
+template <typename... KArgs, typename... Args>
+void launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  (void)cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 #define CSAHCA_CHECK_LAUNCH()                                  \
   do {                                                         \
@@ -180,11 +212,11 @@ int run_compress(const csahca_compress_args* a, void* stream, bool csa) {
   cudaStream_t s = as_stream(stream);
   CSAHCA_TRACE(csa ? "csa_compress" : "hca_compress", s);
   if (a->dtype == CSAHCA_F32) {
-    if (csa) compress_kernel<float, true><<<(unsigned)blocks, threads, 0, s>>>(p);
-    else compress_kernel<float, false><<<(unsigned)blocks, threads, 0, s>>>(p);
+    if (csa) launch_k(compress_kernel<float, true>, dim3((unsigned)blocks), dim3(threads), 0, s, p);
+    else launch_k(compress_kernel<float, false>, dim3((unsigned)blocks), dim3(threads), 0, s, p);
   } else {
-    if (csa) compress_kernel<__nv_bfloat16, true><<<(unsigned)blocks, threads, 0, s>>>(p);
-    else compress_kernel<__nv_bfloat16, false><<<(unsigned)blocks, threads, 0, s>>>(p);
+    if (csa) launch_k(compress_kernel<__nv_bfloat16, true>, dim3((unsigned)blocks), dim3(threads), 0, s, p);
+    else launch_k(compress_kernel<__nv_bfloat16, false>, dim3((unsigned)blocks), dim3(threads), 0, s, p);
   }
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
@@ -260,8 +292,10 @@ size_t indexer_workspace(const csahca_indexer_args* a) {
 }
 
 // Top-k of `rows` score rows (row r at scores + r * stride, position q_pos[r]).
+// Long rows use the multi-CTA path; hist_ready means the indexer has already
+// zeroed the scratch and built the row histograms (pass 1) while scoring.
 int launch_topk(const csahca_indexer_args* a, const float* scores, int64_t stride, const int* q_pos, int* idx,
-                int rows, char* scratch, cudaStream_t s) {
+                int rows, char* scratch, cudaStream_t s, bool hist_ready = false) {
   if (!topk_uses_large(a)) {
     TopkParams tp;
     tp.scores = scores; tp.row_stride = stride; tp.q_pos = q_pos; tp.idx = idx;
@@ -270,7 +304,7 @@ int launch_topk(const csahca_indexer_args* a, const float* scores, int64_t strid
     const int smem = topk_rows_smem_bytes(a->N > 0 ? a->N : 1);
     cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     CSAHCA_TRACE("topk_rows", s);
-    topk_rows_kernel<<<rows, kTopkThreads, smem, s>>>(tp);
+    launch_k(topk_rows_kernel, dim3(rows), dim3(kTopkThreads), smem, s, tp);
     CSAHCA_CHECK_LAUNCH();
     return CSAHCA_OK;
   }
@@ -288,25 +322,22 @@ int launch_topk(const csahca_indexer_args* a, const float* scores, int64_t strid
   tp.counters = reinterpret_cast<uint32_t*>(scratch + L.counters);
   tp.above = reinterpret_cast<int*>(scratch + L.above);
   tp.cand = reinterpret_cast<uint2*>(scratch + L.cand);
-  if (cudaMemsetAsync(scratch + L.hist, 0, L.above - L.hist, s) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return CSAHCA_ERR_LAUNCH;
+  if (!hist_ready) {
+    if (cudaMemsetAsync(scratch + L.hist, 0, L.above - L.hist, s) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return CSAHCA_ERR_LAUNCH;
+    }
+    {
+      CSAHCA_TRACE("topk_hist", s);
+      launch_k(topk_hist_kernel, dim3(rows * slices), dim3(512), 0, s, tp);
+    }
+    CSAHCA_CHECK_LAUNCH();
   }
+  const int smem = topk_select_smem_bytes(a->N);
+  cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   {
-    CSAHCA_TRACE("topk_hist", s);
-    topk_hist_kernel<<<rows * slices, 512, 0, s>>>(tp);
-  }
-  CSAHCA_CHECK_LAUNCH();
-  {
-    CSAHCA_TRACE("topk_split", s);
-    topk_split_kernel<<<rows * slices, 512, 0, s>>>(tp);
-  }
-  CSAHCA_CHECK_LAUNCH();
-  const int smem = 2 * (int)ceil_div64(a->N, 32) * 4;
-  cudaFuncSetAttribute(topk_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  {
-    CSAHCA_TRACE("topk_finish", s);
-    topk_finish_kernel<<<rows, 1024, smem, s>>>(tp);
+    CSAHCA_TRACE("topk_select", s);
+    launch_k(topk_select_kernel, dim3(rows * slices), dim3(kTopkSelectThreads), smem, s, tp);
   }
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
@@ -320,7 +351,7 @@ void launch_indexer_simt(const IndexerParams& p, cudaStream_t s) {
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid((unsigned)ceil_div64(p.N, 256), (unsigned)p.q_count, (unsigned)p.B);
   CSAHCA_TRACE("indexer_scores_simt", s);
-  indexer_scores_simt<TQ, TK, kFP8><<<grid, 256, smem, s>>>(p);
+  launch_k(indexer_scores_simt<TQ, TK, kFP8>, dim3(grid), dim3(256), smem, s, p);
 }
 
 bool indexer_tc_eligible(const csahca_indexer_args* a) {
@@ -347,16 +378,17 @@ int launch_indexer_tc_t(const csahca_indexer_args* a, IdxTcParams p, cudaStream_
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   if (grid <= 0) return CSAHCA_OK;
   CSAHCA_TRACE(QT == 1 ? "indexer_scores_tc_decode" : "indexer_scores_tc_prefill", s);
-  kern<<<grid, kIdxTcThreads, Cfg::SMEM, s>>>(kmap, qmap, p);
+  launch_k(kern, dim3(grid), dim3(kIdxTcThreads), Cfg::SMEM, s, kmap, qmap, p);
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
 }
 
 // Tensor-core scores for queries [q0, q0 + qc) into scores (row stride N).
 int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* scores, int64_t stride,
-                      cudaStream_t s) {
+                      cudaStream_t s, uint32_t* hist = nullptr) {
   IdxTcParams p;
   memset(&p, 0, sizeof(p));
+  p.hist = hist;
   p.w = a->w; p.kI_scale = a->kI_scale; p.q_pos = a->q_pos;
   p.scores = scores; p.score_row_stride = stride;
   p.B = a->B; p.nq = a->nq; p.HI = a->HI; p.N = a->N; p.m = a->m;
@@ -385,7 +417,7 @@ int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* score
     const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
     if (grid <= 0) return CSAHCA_OK;
     CSAHCA_TRACE("indexer_scores_f8", s);
-    indexer_f8_kernel<64><<<grid, kIdxF8Threads, Cfg::SMEM, s>>>(kmap, static_cast<const __nv_bfloat16*>(a->qI), p);
+    launch_k(indexer_f8_kernel<64>, dim3(grid), dim3(kIdxF8Threads), Cfg::SMEM, s, kmap, static_cast<const __nv_bfloat16*>(a->qI), p);
     CSAHCA_CHECK_LAUNCH();
     return CSAHCA_OK;
   }
@@ -460,8 +492,22 @@ int run_indexer(const csahca_indexer_args* a, void* stream) {
     base = static_cast<float*>(a->workspace);
     p.scores = base;
     p.score_row_stride = stride;
+    char* scratch = static_cast<char*>(a->workspace) + indexer_scores_bytes(a);
+    // decode with e4m3 keys: the FP8 indexer builds the top-k row histograms
+    // while it writes the scores (the scratch it adds into is zeroed first)
+    const bool fuse_hist = qc == a->nq && topk_uses_large(a) && indexer_tc_eligible(a) &&
+                           a->k_dtype == CSAHCA_E4M3 && a->N <= kTopkLargeMaxN;
+    uint32_t* hist = nullptr;
+    if (fuse_hist) {
+      const TopkLargeLayout L = topk_large_layout((int64_t)a->B * qc, a->N, a->k);
+      if (cudaMemsetAsync(scratch + L.hist, 0, L.above - L.hist, s) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return CSAHCA_ERR_LAUNCH;
+      }
+      hist = reinterpret_cast<uint32_t*>(scratch + L.hist);
+    }
     if (indexer_tc_eligible(a)) {
-      int st2 = launch_indexer_tc(a, q0, qc, base, stride, s);
+      int st2 = launch_indexer_tc(a, q0, qc, base, stride, s, hist);
       if (st2 != CSAHCA_OK) return st2;
     } else if (a->N > 0) {
       if (a->k_dtype == CSAHCA_E4M3) {
@@ -476,9 +522,8 @@ int run_indexer(const csahca_indexer_args* a, void* stream) {
     }
     // rows of this chunk: (b, q) -> b * qc + (q - q0); positions and outputs are
     // addressed per batch entry, so launch per b unless the chunk is the whole nq
-    char* scratch = static_cast<char*>(a->workspace) + indexer_scores_bytes(a);
     if (qc == a->nq) {
-      int st3 = launch_topk(a, base, stride, a->q_pos, a->idx, a->B * qc, scratch, s);
+      int st3 = launch_topk(a, base, stride, a->q_pos, a->idx, a->B * qc, scratch, s, fuse_hist);
       if (st3 != CSAHCA_OK) return st3;
     } else {
       for (int b = 0; b < a->B; ++b) {
@@ -527,7 +572,7 @@ int launch_finish(const void* x, void* out, const float* gain, int64_t rows, int
   f.rms_norm = rms; f.rope_dims = r; f.rope_base = base; f.eps = eps;
   const int64_t blocks = ceil_div64(rows * 32, 256);
   CSAHCA_TRACE("finish_rows", s);
-  finish_rows_kernel<T><<<(unsigned)blocks, 256, 0, s>>>(f);
+  launch_k(finish_rows_kernel<T>, dim3((unsigned)blocks), dim3(256), 0, s, f);
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
 }
@@ -538,7 +583,7 @@ int launch_simt_attn(const SimtAttnParams& p, int nq_total, cudaStream_t s, cons
   cudaFuncSetAttribute(attn_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   dim3 grid((unsigned)nq_total, (unsigned)ceil_div64(p.H, kSimtHG), (unsigned)p.splits);
   CSAHCA_TRACE(name, s);
-  attn_simt_kernel<T><<<grid, 32 * kSimtHG, smem, s>>>(p);
+  launch_k(attn_simt_kernel<T>, dim3(grid), dim3(32 * kSimtHG), smem, s, p);
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
 }
@@ -568,7 +613,7 @@ int launch_attn_tc(const AttnTcParams& p, const void* kv_comp, int64_t comp_rows
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   if (grid <= 0) return CSAHCA_OK;
   CSAHCA_TRACE(name, s);
-  attn_tc_kernel<<<grid, kAttnTcThreads, smem, s>>>(m_rows, m_gather, m_win, m_q, p);
+  launch_k(attn_tc_kernel, dim3(grid), dim3(kAttnTcThreads), smem, s, m_rows, m_gather, m_win, m_q, p);
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
 }
@@ -703,7 +748,8 @@ DecodeLayout decode_layout(const csahca_decode_args* a) {
   L.idx_off = off;
   if (csa && !a->idx_out) off += align_up((size_t)a->B * a->k * 4, 256);
   L.partial_off = off;
-  off += align_up((size_t)a->B * a->H * L.splits * (a->d + 4) * 4, 256);
+  if (L.tc) off += align_up((size_t)a->B * L.splits * kTcPartialBytes, 256);
+  else off += align_up((size_t)a->B * a->H * L.splits * (a->d + 4) * 4, 256);
   L.total = off;
   return L;
 }
@@ -764,13 +810,28 @@ int run_decode_t(const csahca_decode_args* a, cudaStream_t s, char* ws) {
     st = launch_simt_attn<T>(p, a->B, s, a->kind == CSAHCA_CSA ? "attn_decode_csa_simt" : "attn_decode_hca_simt");
   }
   if (st != CSAHCA_OK) return st;
+  if (L.tc) {
+    TcCombineParams c;
+    c.partial = reinterpret_cast<const char*>(partial); c.sinks = a->sinks; c.pos = a->pos;
+    c.out = static_cast<__nv_bfloat16*>(a->out);
+    c.rows = a->B; c.splits = L.splits; c.rope_dims = a->rope_dims; c.rope_base = base;
+    const int smem = L.splits * 3 * kAttnH * 4;
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(attn_combine_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    {
+      CSAHCA_TRACE("attn_combine", s);
+      launch_k(attn_combine_tc_kernel, dim3((unsigned)(a->B * (kAttnD / 16))), dim3(128), smem, s, c);
+    }
+    CSAHCA_CHECK_LAUNCH();
+    return CSAHCA_OK;
+  }
   CombineParams c;
   c.partial = partial; c.sinks = a->sinks; c.pos = a->pos; c.out = a->out;
   c.B = a->B; c.nq = 1; c.H = a->H; c.d = a->d; c.splits = L.splits;
   c.rope_dims = a->rope_dims; c.decode = 1; c.rope_base = base;
   {
     CSAHCA_TRACE("attn_combine", s);
-    attn_combine_kernel<T><<<(unsigned)(a->B * a->H), 128, 0, s>>>(c);
+    launch_k(attn_combine_kernel<T>, dim3((unsigned)(a->B * a->H)), dim3(128), 0, s, c);
   }
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;

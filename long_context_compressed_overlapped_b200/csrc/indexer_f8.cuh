@@ -13,26 +13,36 @@
 // multiple of x's last-bit weight of magnitude <= 8 of them, which e4m3
 // holds exactly whenever that weight is >= 2^-9, i.e. for every element of
 // magnitude >= 2^-9 of the head's largest; smaller elements are rounded to
-// within 2^-10 s_h.)  The B operand is therefore the two terms side by side
-// along K, and one accumulation over K = 2 x 128 against the same key tile
-// gives D[i, h] = kI_i . q_h / s_h.  Since s_h > 0 and the key row scale
-// c_i > 0 commute with ReLU, I_{t,i} = c_i sum_h (w_h s_h) ReLU(D[i, h]).
+// within 2^-10 s_h.)  The B operand holds the two terms as 2 x HI rows (term
+// t of head h in row t*HI + h), so one MMA chain of N = 2*HI over K = 128
+// against the key tile gives D[i, t*HI + h] = kI_i . t_{t,h}, and
+// kI_i . q_h / s_h = D[i, h] + D[i, HI + h] exactly in fp32.  Since s_h > 0 and
+// the key row scale c_i > 0 commute with ReLU,
+// I_{t,i} = c_i sum_h (w_h s_h) ReLU(D[i, h] + D[i, HI + h]).
 // Heads whose largest |q| is below 2^-118 (s_h would leave the normal fp32
 // range) contribute nothing.
 //
-// Roles (320 threads): two epilogue groups of 4 warps (warps 0-3, 4-7) take
+// Roles (352 threads): two epilogue groups of 4 warps (warps 0-3, 4-7) take
 // alternate key tiles, so the ReLU / weighted-sum epilogue of one tile
 // overlaps the next; group 0 also writes the split query of each work item.
-// Warp 8 issues the TMA key loads into a 10-stage ring, warp 9 issues the MMAs
-// (N = HI, 8 MMAs of K = 32 per tile) into 4 TMEM accumulators and owns TMEM.
+// Warp 8 issues the TMA key loads (and copies the keys' row scales) into a
+// 10-stage ring; warps 9 and 10 issue the MMAs of alternate tiles (N = 2*HI,
+// 4 MMAs of K = 32 per tile, descriptors precomputed so that each issue is one
+// add) into 4 TMEM accumulators; warp 9 owns TMEM.
 // Work items as in indexer_tc.cuh: decode = (sequence, range of key tiles),
 // prefill = (sequence, one query, every visible key tile).
+//
+// With p.hist set, the epilogue also counts each written score into a
+// 2048-bin shared histogram of its order key's top 11 bits and adds it to the
+// row's global histogram at the end of each work item: pass 1 of the
+// multi-CTA top-k (topk_large.cuh), done while the scores are in registers.
 #pragma once
 #include "indexer_tc.cuh"
+#include "topk_large.cuh"
 
 namespace csahca {
 
-constexpr int kIdxF8Threads = 320;
+constexpr int kIdxF8Threads = 352;
 constexpr int kIdxF8Stages = 10;
 constexpr int kIdxF8Acc = 4;
 
@@ -42,7 +52,10 @@ struct IdxF8Cfg {
   static constexpr int B_BYTES = 2 * B_TERM;
   static constexpr int A_BYTES = 128 * 128;         // 128 keys x 128 e4m3
   static constexpr int SMEM = 1024 + B_BYTES + kIdxF8Stages * A_BYTES;
-  static constexpr int TMEM_COLS = kIdxF8Acc * HI <= 256 ? 256 : 512;
+  static constexpr int NCOL = 2 * HI;               // MMA N: both terms of every head
+  static constexpr int TMEM_COLS = kIdxF8Acc * NCOL <= 256 ? 256 : 512;
+  static_assert(kIdxF8Acc * NCOL <= 512, "accumulators fit in TMEM");
+  static_assert(kIdxF8Stages % 2 == 0 && kIdxF8Acc % 2 == 0, "tile parity picks issuer, stage and accumulator");
   static_assert(HI == 64, "two threads per head of a 128-thread group build the split query");
   static_assert(B_TERM % 1024 == 0, "SW128 operands start on 1024-byte boundaries");
 };
@@ -60,6 +73,25 @@ __device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t adesc, uint6
       ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
+// 4-byte global -> shared copy; src_bytes = 0 fills zero without reading.
+__device__ __forceinline__ void cp_async4_zfill(void* dst_smem, const void* src_gmem, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem), "r"(src_bytes)
+               : "memory");
+}
+
+// Named barrier 3 over the 256 threads of both epilogue groups.
+__device__ __forceinline__ void epi_sync256() { asm volatile("bar.sync 3, 256;" ::: "memory"); }
+__device__ __forceinline__ bool epi_any256(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 3, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
 template <int HI>
 __global__ void __launch_bounds__(kIdxF8Threads, 1)
 indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* __restrict__ qI, IdxTcParams p) {
@@ -75,15 +107,20 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
   __shared__ float sW[2][HI];                     // per group: w_h * s_h of its current item
+  __shared__ uint32_t hist_s[kHistBins];          // this item's score histogram (p.hist set)
+  __shared__ float sScale[NS][128];               // key row scales of each stage
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (int s = 0; s < NS; ++s) { mbar_init(&bar_a_full[s], 1); mbar_init(&bar_a_empty[s], 1); }
+    // a stage is full once its key tile (TMA bytes, lane 0's arrive) and its
+    // scales (one cp.async arrive per producer lane) have landed; it is empty
+    // once the MMAs have read the keys and the owning epilogue group the scales
+    for (int s = 0; s < NS; ++s) { mbar_init(&bar_a_full[s], 1 + 32); mbar_init(&bar_a_empty[s], 1 + 128); }
     for (int j = 0; j < NACC; ++j) { mbar_init(&bar_acc_full[j], 1); mbar_init(&bar_acc_empty[j], 128); }
     mbar_init(&bar_b_full, 128);
-    mbar_init(&bar_b_empty, 1);
-    mbar_init(&bar_done, 1);
+    mbar_init(&bar_b_empty, 2);                    // both MMA issuers, once per item
+    mbar_init(&bar_done, 2);
     mbar_fence_init();
   }
   if (warp == 9) tmem_alloc(&tmem_base_sh, Cfg::TMEM_COLS);
@@ -91,32 +128,58 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  griddep_launch_dependents();
+  griddep_wait();                                  // keys may come from this stream's compress kernel
 
   if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&kmap);
-      uint32_t a_iter = 0;
-      for (int id = blockIdx.x; id < p.n_items && !abort_flag; id += gridDim.x) {
-        const IdxItem it = idx_item<1>(p, id);
-        for (int kt = it.kt0; kt < it.kt1; ++kt, ++a_iter) {
-          const int s = a_iter % NS;
-          const uint32_t ph = (a_iter / NS) & 1;
-          if (!mbar_wait(&bar_a_empty[s], ph ^ 1, &abort_flag)) break;
-          mbar_expect_tx(&bar_a_full[s], Cfg::A_BYTES);
-          tma_load_2d(sA + s * Cfg::A_BYTES, &kmap, 0, it.b * p.N + kt * 128, &bar_a_full[s]);
+    // ------------------------------------------------------------ producer
+    // lane 0: the key tile by TMA; all lanes: the tile's 128 row scales by
+    // cp.async (4 each, zero past the row's end)
+    if (lane == 0) tma_prefetch_desc(&kmap);
+    uint32_t a_iter = 0;
+    bool stop = false;                               // warp-uniform
+    for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
+      const IdxItem it = idx_item<1>(p, id);
+      const float* srow = p.kI_scale + (int64_t)it.b * p.N;
+      for (int kt = it.kt0; kt < it.kt1; ++kt, ++a_iter) {
+        const int s = a_iter % NS;
+        const uint32_t ph = (a_iter / NS) & 1;
+        int ok = 1;
+        if (lane == 0) {
+          ok = mbar_wait(&bar_a_empty[s], ph ^ 1, &abort_flag);
+          if (ok) {
+            mbar_expect_tx(&bar_a_full[s], Cfg::A_BYTES);
+            tma_load_2d(sA + s * Cfg::A_BYTES, &kmap, 0, it.b * p.N + kt * 128, &bar_a_full[s]);
+          }
         }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) { stop = true; break; }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = kt * 128 + lane + 32 * e;
+          const bool in = key < p.N;
+          cp_async4_zfill(&sScale[s][lane + 32 * e], srow + (in ? key : 0), in ? 4u : 0u);
+        }
+        cp_async_arrive_noinc(&bar_a_full[s]);
       }
-      // drain: every issued fill has landed before the CTA may exit
+    }
+    // drain: every issued fill has landed before the CTA may exit
+    cp_async_wait<0>();
+    if (lane == 0)
       for (uint32_t i = (a_iter > NS ? a_iter - NS : 0); i < a_iter; ++i)
         mbar_wait(&bar_a_full[i % NS], (i / NS) & 1, &abort_flag);
-    }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 9 || warp == 10) {
+    // ------------------------------------------------------------ MMA issuers
+    // issuer e takes the tiles of parity e (their stages and accumulators have
+    // that parity too), so two threads keep the tensor pipe fed
     if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_e4m3(128, HI);
+      const uint32_t e = (uint32_t)(warp - 9);
+      constexpr uint32_t idesc = umma_idesc_e4m3(128, Cfg::NCOL);
       uint32_t a_iter = 0, b_iter = 0, acc_iter = 0;
-      const uint32_t sA0 = smem_u32(sA), sB0 = smem_u32(sB);
+      // the start address is the descriptor's low field (in 16-byte units):
+      // stage / K-step offsets are plain adds to the base descriptors
+      const uint64_t adesc0 = umma_desc_kmajor(smem_u32(sA));
+      const uint64_t bdesc0 = umma_desc_kmajor(smem_u32(sB));
       for (int id = blockIdx.x; id < p.n_items && !abort_flag; id += gridDim.x) {
         const IdxItem it = idx_item<1>(p, id);
         if (it.kt1 <= it.kt0) continue;
@@ -124,6 +187,7 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
         ++b_iter;
         bool ok = true;
         for (int kt = it.kt0; kt < it.kt1; ++kt, ++a_iter, ++acc_iter) {
+          if ((a_iter & 1u) != e) continue;
           const int s = a_iter % NS;
           const uint32_t ph = (a_iter / NS) & 1;
           const int j = acc_iter % NACC;
@@ -131,12 +195,10 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
           if (!mbar_wait(&bar_a_full[s], ph, &abort_flag)) { ok = false; break; }
           if (!mbar_wait(&bar_acc_empty[j], aph ^ 1, &abort_flag)) { ok = false; break; }
           tc_fence_after();
+          const uint64_t ad = adesc0 + (uint64_t)((s * Cfg::A_BYTES) >> 4);
+          const uint32_t d = tmem + j * Cfg::NCOL;
 #pragma unroll
-          for (int t = 0; t < 2; ++t)
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-              umma_e4m3(tmem + j * HI, umma_desc_kmajor(sA0 + s * Cfg::A_BYTES + ks * 32),
-                        umma_desc_kmajor(sB0 + t * Cfg::B_TERM + ks * 32), idesc, (t | ks) != 0);
+          for (int ks = 0; ks < 4; ++ks) umma_e4m3(d, ad + 2 * ks, bdesc0 + 2 * ks, idesc, ks != 0);
           umma_commit(&bar_a_empty[s]);
           umma_commit(&bar_acc_full[j]);
         }
@@ -151,16 +213,23 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
     const int g = warp >> 2;                         // group 0: warps 0-3, group 1: warps 4-7
     const int bar_id = 1 + g;
     const int et = threadIdx.x & 127;                // key lane within a tile
+    const int ept = threadIdx.x;                     // 0..255 over both groups
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const bool do_hist = p.hist != nullptr;
+    if (do_hist)
+      for (int i = ept; i < kHistBins; i += 256) hist_s[i] = 0;
+    epi_sync256();
     uint32_t acc_iter = 0, b_iter = 0;
-    bool stop = false;                               // uniform over the group
-    for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
+    for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
       const IdxItem it = idx_item<1>(p, id);
       if (it.kt1 <= it.kt0) continue;
+      // `bad` is uniform over a group; a group that gives up skips the rest of
+      // the item and both groups leave together at its end
+      bool bad = false;
       // group 0 rewrites B once the previous item's MMAs have read it
-      if (g == 0 && !mbar_wait_group(bar_id, &bar_b_empty, (b_iter & 1) ^ 1, &abort_flag)) { stop = true; break; }
+      if (g == 0 && !mbar_wait_group(bar_id, &bar_b_empty, (b_iter & 1) ^ 1, &abort_flag)) bad = true;
       ++b_iter;
-      {
+      if (!bad) {
         // thread (h = et / 2, half = et % 2) owns 64 dims of head h
         const int h = et >> 1, half = et & 1;
         const int64_t qrow = ((int64_t)it.b * p.nq + it.q0) * HI + h;
@@ -209,32 +278,48 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
           fence_proxy_async_smem();
           mbar_arrive(&bar_b_full);
         }
-        group_sync(bar_id);                          // sW[g] complete
       }
+      group_sync(bar_id);                            // sW[g] complete
       const int v = idx_visible(p, it.b, it.q0);
       float* srow = p.scores + ((int64_t)it.b * p.q_count + (it.q0 - p.q_begin)) * p.score_row_stride;
       for (int kt = it.kt0; kt < it.kt1; ++kt, ++acc_iter) {
-        if ((int)(acc_iter & 1) != g) continue;      // the other group's tile
+        if ((int)(acc_iter & 1) != g || bad) continue;   // the other group's tile, or giving up
         const int j = acc_iter % NACC;
         const uint32_t aph = (acc_iter / NACC) & 1;
-        if (!mbar_wait_group(bar_id, &bar_acc_full[j], aph, &abort_flag)) { stop = true; break; }
+        if (!mbar_wait_group(bar_id, &bar_acc_full[j], aph, &abort_flag)) { bad = true; continue; }
         tc_fence_after();
         const int key = kt * 128 + et;
-        float acc = 0.f;
+        const int st = acc_iter % NS;                // this tile's stage (one stage per tile)
+        const float kscale = sScale[st][et];
+        mbar_arrive(&bar_a_empty[st]);
+        float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < HI / 32; ++c) {
-          float d[32];
-          tmem_ld32(tmem + lane_base + j * HI + c * 32, d);
+          float d0[32], d1[32];
+          tmem_ld32(tmem + lane_base + j * Cfg::NCOL + c * 32, d0);
+          tmem_ld32(tmem + lane_base + j * Cfg::NCOL + HI + c * 32, d1);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) acc = fmaf(sW[g][c * 32 + e], fmaxf(d[e], 0.f), acc);
+          for (int e = 0; e < 32; ++e) a4[e & 3] = fmaf(sW[g][c * 32 + e], fmaxf(d0[e] + d1[e], 0.f), a4[e & 3]);
         }
+        const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
         tc_fence_before();
         mbar_arrive(&bar_acc_empty[j]);
-        if (key < v) srow[key] = acc * __ldg(p.kI_scale + (int64_t)it.b * p.N + key);
+        if (key < v) {
+          const float score = acc * kscale;
+          srow[key] = score;
+          if (do_hist) atomicAdd(&hist_s[order_key(score) >> kHistShift], 1u);
+        }
       }
-      if (stop) break;
-      group_sync(bar_id);                            // sW[g] may be rewritten
+      if (epi_any256(bad)) break;                    // also: both groups are done with the item
+      if (do_hist) {
+        uint32_t* gh = p.hist + ((int64_t)it.b * p.q_count + (it.q0 - p.q_begin)) * kHistBins;
+        for (int i = ept; i < kHistBins; i += 256) {
+          const uint32_t c = hist_s[i];
+          if (c) { atomicAdd(gh + i, c); hist_s[i] = 0; }
+        }
+        epi_sync256();
+      }
     }
   }
   tc_fence_before();

@@ -32,6 +32,7 @@ struct IdxTcParams {
   int n_items;
   int splits;                 // > 0: decode items (b, split); 0: prefill items (b, query tile)
   int tiles_per_split;
+  uint32_t* hist;             // optional [rows][2048] score histograms (decode, e4m3 keys)
 };
 
 template <int QT, int HI, bool kFP8>
@@ -122,6 +123,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  griddep_launch_dependents();
+  griddep_wait();                                  // keys may come from this stream's compress kernel
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer

@@ -26,8 +26,9 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive block scan of 0/1 flags (blockDim.x == kTopkThreads); returns the
-// exclusive prefix of this thread and writes the block total to *total.
+// Exclusive block scan of 0/1 flags (blockDim.x a multiple of 32, <= 1024);
+// returns the exclusive prefix of this thread and writes the block total to
+// *total.
 __device__ __forceinline__ int block_excl_scan(int flag, int* warp_buf, int* total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   unsigned ballot = __ballot_sync(0xffffffffu, flag);
@@ -35,7 +36,7 @@ __device__ __forceinline__ int block_excl_scan(int flag, int* warp_buf, int* tot
   if (lane == 0) warp_buf[wid] = __popc(ballot);
   __syncthreads();
   if (wid == 0) {
-    int x = warp_buf[lane];
+    int x = lane < (int)(blockDim.x >> 5) ? warp_buf[lane] : 0;
     int incl = x;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -52,7 +53,8 @@ __device__ __forceinline__ int block_excl_scan(int flag, int* warp_buf, int* tot
   return res;
 }
 
-// Exclusive block prefix sum of per-thread counts (blockDim.x == 1024).
+// Exclusive block prefix sum of per-thread counts (blockDim.x a multiple of
+// 32, <= 1024).
 __device__ __forceinline__ int block_excl_count(int c, int* warp_buf, int* total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   int incl = c;
@@ -64,7 +66,7 @@ __device__ __forceinline__ int block_excl_count(int c, int* warp_buf, int* total
   if (lane == 31) warp_buf[wid] = incl;
   __syncthreads();
   if (wid == 0) {
-    const int x = warp_buf[lane];
+    const int x = lane < (int)(blockDim.x >> 5) ? warp_buf[lane] : 0;
     int wi = x;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -122,6 +124,8 @@ __host__ __device__ __forceinline__ int kslot(int j) { return j + (j >> 5); }
 __host__ __device__ __forceinline__ int topk_rows_smem_bytes(int n) { return (kslot(n) + 1) * 4; }
 
 __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(TopkParams p) {
+  griddep_launch_dependents();
+  griddep_wait();
   extern __shared__ uint32_t keys[];           // order keys of the row at kslot(j)
   __shared__ uint32_t hist[kTopkSubHist * 256];
   __shared__ int warp_buf[72];

@@ -1,20 +1,24 @@
 // Top-k over long score rows (decode: one query against every visible
-// compressed entry, up to 2^20 of them), spread over many CTAs.
+// compressed entry, up to 786,432 of them), spread over many CTAs.
 // ("Paper Breakdown: DeepSeek-V4", section 4, DSA on Compressed KV: the top-k
 // entries by I_{t,s}; "How DeepSeek-V4 architecture and training work
 // together": 1,024 entries per query.)
 //
-//   1. topk_hist:   each CTA histograms its slice of the row on the top 11
-//                   bits of the order-preserving key; global atomics merge.
-//   2. topk_split:  every CTA finds the row's threshold bin T (fewer than k
-//                   keys above it, at least k from it up) and routes its keys:
-//                   bins above T are taken, bin T keys become candidates.
-//   3. topk_finish: one CTA per row: exact radix select of the remaining
-//                   count among the candidates (21 low bits), ties to the
-//                   lower index through a bitmap scan in index order, and the
-//                   taken set is written in ascending index order through a
-//                   second bitmap scan.
+//   1. histogram:   a 2048-bin histogram per row of the top 11 bits of the
+//                   order-preserving key, either built by the tensor-core
+//                   decode indexer while it writes the scores, or by
+//                   topk_hist_kernel (each CTA a slice, merged by atomics).
+//   2. topk_select: every CTA finds the row's threshold bin T (fewer than k
+//                   keys above it, at least k from it up) and routes its slice:
+//                   bins above T are taken, bin T keys become candidates.  The
+//                   last CTA of a row to finish (atomic count after a fence)
+//                   then selects exactly: radix select of the remaining count
+//                   among the candidates (21 low bits), ties to the lower index
+//                   through a bitmap scan in index order, and the taken set
+//                   written in ascending index order through a second bitmap
+//                   scan.
 #pragma once
+#include <limits.h>
 #include "topk.cuh"
 
 namespace csahca {
@@ -31,7 +35,7 @@ struct TopkLargeParams {
   int slices;                              // CTAs per row in passes 1 and 2
   // workspace (per row)
   uint32_t* hist;                          // [rows][kHistBins]
-  uint32_t* counters;                      // [rows][4]: n_above, n_cand
+  uint32_t* counters;                      // [rows][4]: n_above, n_cand, slices done
   int* above;                              // [rows][k]
   uint2* cand;                             // [rows][N]: (key, index)
 };
@@ -44,6 +48,8 @@ __device__ __forceinline__ int topk_visible(const TopkLargeParams& p, int row) {
 }
 
 __global__ void __launch_bounds__(512) topk_hist_kernel(TopkLargeParams p) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ uint32_t h[kHistBins];
   const int row = blockIdx.x / p.slices, slice = blockIdx.x % p.slices;
   const int v = topk_visible(p, row);
@@ -95,53 +101,9 @@ __device__ __forceinline__ int threshold_bin(const uint32_t* g, int k, uint32_t*
   return sh_T;
 }
 
-__global__ void __launch_bounds__(512) topk_split_kernel(TopkLargeParams p) {
-  __shared__ uint32_t sh[1024];
-  const int row = blockIdx.x / p.slices, slice = blockIdx.x % p.slices;
-  const int v = topk_visible(p, row);
-  if (v <= p.k) return;
-  uint32_t n_above;
-  const int T = threshold_bin(p.hist + (int64_t)row * kHistBins, p.k, sh, &n_above);
-  const int per = (v + p.slices - 1) / p.slices;
-  const int j0 = slice * per, j1 = min(v, j0 + per);
-  const float* s = p.scores + (int64_t)row * p.row_stride;
-  uint32_t* cnt = p.counters + (int64_t)row * 4;
-  int* above = p.above + (int64_t)row * p.k;
-  uint2* cand = p.cand + (int64_t)row * p.N;
-  const int lane = threadIdx.x & 31;
-  for (int base = j0; base < j1; base += blockDim.x) {
-    const int j = base + threadIdx.x;
-    const uint32_t key = j < j1 ? order_key(s[j]) : 0u;
-    const int bin = (int)(key >> kHistShift);
-    const bool take = j < j1 && bin > T;
-    const bool cnd = j < j1 && bin == T;
-    // warp-aggregated appends
-    const unsigned mt = __ballot_sync(0xffffffffu, take);
-    if (mt) {
-      uint32_t basei = 0;
-      if (lane == 0) basei = atomicAdd(&cnt[0], (uint32_t)__popc(mt));
-      basei = __shfl_sync(0xffffffffu, basei, 0);
-      if (take) {
-        const uint32_t pos = basei + __popc(mt & ((1u << lane) - 1u));
-        if (pos < (uint32_t)p.k) above[pos] = j;
-      }
-    }
-    const unsigned mc = __ballot_sync(0xffffffffu, cnd);
-    if (mc) {
-      uint32_t basei = 0;
-      if (lane == 0) basei = atomicAdd(&cnt[1], (uint32_t)__popc(mc));
-      basei = __shfl_sync(0xffffffffu, basei, 0);
-      if (cnd) {
-        const uint32_t pos = basei + __popc(mc & ((1u << lane) - 1u));
-        if (pos < (uint32_t)p.N) cand[pos] = make_uint2(key, (uint32_t)j);
-      }
-    }
-  }
-}
-
 // Index-ordered scan of a bitmap of `words` 32-bit words: calls out(i) for the
 // set bits in ascending order, at most `limit` of them; returns how many.
-// blockDim.x == 1024; warp_buf as for block_excl_scan.
+// blockDim.x a multiple of 32 (<= 1024); warp_buf holds at least 65 ints.
 template <typename F>
 __device__ __forceinline__ int bitmap_scan(const uint32_t* bm, int words, int limit, int* warp_buf, F out) {
   int done = 0;
@@ -159,7 +121,7 @@ __device__ __forceinline__ int bitmap_scan(const uint32_t* bm, int words, int li
     if (lane == 31) warp_buf[wid] = incl;
     __syncthreads();
     if (wid == 0) {
-      const int x = warp_buf[lane];
+      const int x = lane < (int)(blockDim.x >> 5) ? warp_buf[lane] : 0;
       int wincl = x;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -186,31 +148,128 @@ __device__ __forceinline__ int bitmap_scan(const uint32_t* bm, int words, int li
   return done < limit ? done : limit;
 }
 
-__global__ void __launch_bounds__(1024) topk_finish_kernel(TopkLargeParams p) {
+constexpr int kTopkSelectThreads = 512;
+constexpr int kTopkCandCache = 4096;       // candidates staged in shared memory (8 bytes each)
+constexpr int kTopkSortCap = 2048;         // selected / tie indices sorted in shared memory
+
+__host__ __device__ __forceinline__ int next_pow2(int x) {
+  int n = 1;
+  while (n < x) n <<= 1;
+  return n;
+}
+
+// Dynamic shared memory of topk_select_kernel: the larger of the bitmap path
+// (two bitmaps of N bits) and the sort path (candidate cache, selected and
+// tie buffers).
+__host__ __device__ __forceinline__ int topk_select_smem_bytes(int N) {
+  const int bitmaps = 2 * ((N + 31) / 32) * 4;
+  const int sorted = kTopkCandCache * 8 + 2 * kTopkSortCap * 4;
+  return bitmaps > sorted ? bitmaps : sorted;
+}
+
+// Ascending bitonic sort of n (a power of two) ints in shared memory by the
+// whole block; ends with a barrier.
+__device__ __forceinline__ void bitonic_sort_smem(int* a, int n) {
+  for (int k2 = 2; k2 <= n; k2 <<= 1) {
+    for (int j = k2 >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const int x = a[i], y = a[ixj];
+          const bool up = (i & k2) == 0;
+          if ((x > y) == up) { a[i] = y; a[ixj] = x; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  __syncthreads();
+}
+
+// Routing of one slice (pass 2) and, in the last CTA of the row, the exact
+// selection.  Dynamic shared memory: topk_select_smem_bytes(N) (two bitmaps).
+__global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLargeParams p) {
+  griddep_launch_dependents();
+  griddep_wait();
   extern __shared__ uint32_t bm_sel[];               // [words] taken, then [words] ties
+  __shared__ uint32_t sh[1024];
   __shared__ uint32_t hist8[256];
   __shared__ int warp_buf[72];
-  __shared__ uint32_t sh_digit, sh_need;
-  const int row = blockIdx.x;
+  __shared__ uint32_t sh_digit, sh_need, sh_eq, sh_nsel, sh_base_t, sh_base_c;
+  __shared__ int sh_last;
+  const int row = blockIdx.x / p.slices, slice = blockIdx.x % p.slices;
   const int v = topk_visible(p, row);
   int* out = p.idx + (int64_t)row * p.k;
   if (v <= p.k) {
-    for (int j = threadIdx.x; j < p.k; j += blockDim.x) out[j] = j < v ? j : -1;
+    if (slice == 0)
+      for (int j = threadIdx.x; j < p.k; j += blockDim.x) out[j] = j < v ? j : -1;
     return;
   }
-  const int words = (v + 31) / 32;
-  uint32_t* bm_eq = bm_sel + words;
-  for (int i = threadIdx.x; i < 2 * words; i += blockDim.x) bm_sel[i] = 0;
-  const uint32_t* cnt = p.counters + (int64_t)row * 4;
-  const uint32_t n_above = min(cnt[0], (uint32_t)p.k);
-  const uint32_t n_cand = min(cnt[1], (uint32_t)p.N);
-  const uint2* cand = p.cand + (int64_t)row * p.N;
-  const int* above = p.above + (int64_t)row * p.k;
-  __syncthreads();
-  for (uint32_t i = threadIdx.x; i < n_above; i += blockDim.x) {
-    const int j = above[i];
-    atomicOr(&bm_sel[j >> 5], 1u << (j & 31));
+  uint32_t* cnt = p.counters + (int64_t)row * 4;
+  int* above = p.above + (int64_t)row * p.k;
+  uint2* cand = p.cand + (int64_t)row * p.N;
+  {
+    uint32_t n_above_T;
+    const int T = threshold_bin(p.hist + (int64_t)row * kHistBins, p.k, sh, &n_above_T);
+    const int per = (v + p.slices - 1) / p.slices;
+    const int j0 = slice * per, j1 = min(v, j0 + per);
+    const float* s = p.scores + (int64_t)row * p.row_stride;
+    // 8 keys per thread per round; the CTA reserves its ranges of the row's
+    // taken / candidate lists with one atomic each (a block prefix sum places
+    // every thread's entries), so the row counters see one atomic per CTA
+    constexpr int kPer = 8;
+    for (int base = j0; base < j1; base += kPer * (int)blockDim.x) {
+      uint32_t key[kPer];
+      int nt = 0, nc = 0;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int j = base + u * (int)blockDim.x + (int)threadIdx.x;
+        key[u] = j < j1 ? order_key(__ldcg(s + j)) : 0u;
+        const int bin = (int)(key[u] >> kHistShift);
+        nt += (j < j1 && bin > T);
+        nc += (j < j1 && bin == T);
+      }
+      int tot;
+      const int off = block_excl_count(nt | (nc << 16), warp_buf, &tot);
+      if (threadIdx.x == 0) {
+        sh_base_t = atomicAdd(&cnt[0], (uint32_t)(tot & 0xFFFF));
+        sh_base_c = atomicAdd(&cnt[1], (uint32_t)(tot >> 16));
+      }
+      __syncthreads();
+      uint32_t pt = sh_base_t + (uint32_t)(off & 0xFFFF), pc = sh_base_c + (uint32_t)(off >> 16);
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int j = base + u * (int)blockDim.x + (int)threadIdx.x;
+        const int bin = (int)(key[u] >> kHistShift);
+        if (j < j1 && bin > T) {
+          if (pt < (uint32_t)p.k) above[pt] = j;
+          ++pt;
+        } else if (j < j1 && bin == T) {
+          if (pc < (uint32_t)p.N) cand[pc] = make_uint2(key[u], (uint32_t)j);
+          ++pc;
+        }
+      }
+      __syncthreads();
+    }
   }
+  // publish this slice, then let the last CTA of the row finish it
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) sh_last = atomicAdd(&cnt[2], 1u) == (uint32_t)(p.slices - 1);
+  __syncthreads();
+  if (!sh_last) return;
+  __threadfence();
+
+  const uint32_t n_above = min(__ldcg(&cnt[0]), (uint32_t)p.k);
+  const uint32_t n_cand = min(__ldcg(&cnt[1]), (uint32_t)p.N);
+  // candidates staged in shared memory when they fit (the usual case), else
+  // read from the scratch in every pass
+  uint2* cand_s = reinterpret_cast<uint2*>(bm_sel);
+  const bool cand_local = n_cand <= (uint32_t)kTopkCandCache;
+  if (cand_local)
+    for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) cand_s[i] = __ldcg(cand + i);
+  const uint2* C = cand_local ? cand_s : cand;
+  __syncthreads();
   // radix select of the need-th largest key among the candidates (bits 20..0)
   uint32_t need = (uint32_t)p.k - n_above;
   uint32_t prefix = 0, mask = 0;
@@ -218,13 +277,13 @@ __global__ void __launch_bounds__(1024) topk_finish_kernel(TopkLargeParams p) {
   const int shifts[3] = {13, 5, 0};
   const int widths[3] = {8, 8, 5};
   for (int pass = 0; pass < 3; ++pass) {
-    const int sh = shifts[pass];
+    const int shf = shifts[pass];
     const uint32_t dm = (1u << widths[pass]) - 1u;
     for (int i = threadIdx.x; i < 256; i += blockDim.x) hist8[i] = 0;
     __syncthreads();
     for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
-      const uint32_t key = cand[i].x & ((1u << kHistShift) - 1u);
-      if ((key & mask) == prefix) atomicAdd(&hist8[(key >> sh) & dm], 1u);
+      const uint32_t key = (cand_local ? C[i].x : __ldcg(&cand[i].x)) & ((1u << kHistShift) - 1u);
+      if ((key & mask) == prefix) atomicAdd(&hist8[(key >> shf) & dm], 1u);
     }
     __syncthreads();
     if ((threadIdx.x >> 5) == 0) {
@@ -233,13 +292,73 @@ __global__ void __launch_bounds__(1024) topk_finish_kernel(TopkLargeParams p) {
       find_digit_warp(hist8, (int)dm + 1 >= 32 ? (int)dm + 1 : 32, nd, &sh_digit, &sh_need);
     }
     __syncthreads();
-    prefix |= sh_digit << sh;
-    mask |= dm << sh;
+    prefix |= sh_digit << shf;
+    mask |= dm << shf;
     __syncthreads();
   }
   need = sh_need;                              // keys equal to the threshold still to take
+  // count the keys equal to the threshold
+  if (threadIdx.x == 0) { sh_eq = 0; sh_nsel = 0; }
+  __syncthreads();
+  {
+    uint32_t ne = 0;
+    for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
+      const uint32_t low = (cand_local ? C[i].x : __ldcg(&cand[i].x)) & ((1u << kHistShift) - 1u);
+      ne += low == prefix;
+    }
+    if (ne) atomicAdd(&sh_eq, ne);
+  }
+  __syncthreads();
+  const uint32_t n_eq = sh_eq;
+  const int nsort = next_pow2(p.k);
+  if (nsort <= kTopkSortCap && (n_eq == need || n_eq <= (uint32_t)kTopkSortCap)) {
+    // ---- sort path: gather the k selected indices, then sort them ascending
+    int* sel = reinterpret_cast<int*>(bm_sel) + 2 * kTopkCandCache;   // after the candidate cache
+    int* ties = sel + kTopkSortCap;
+    for (uint32_t i = threadIdx.x; i < n_above; i += blockDim.x) sel[i] = __ldcg(above + i);
+    if (threadIdx.x == 0) sh_nsel = n_above;
+    __syncthreads();
+    if (threadIdx.x == 0) sh_eq = 0;
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
+      const uint2 c = cand_local ? C[i] : __ldcg(cand + i);
+      const uint32_t low = c.x & ((1u << kHistShift) - 1u);
+      if (low > prefix) sel[atomicAdd(&sh_nsel, 1u)] = (int)c.y;
+      else if (low == prefix) {
+        if (n_eq == need) sel[atomicAdd(&sh_nsel, 1u)] = (int)c.y;   // every tie is taken
+        else ties[atomicAdd(&sh_eq, 1u)] = (int)c.y;
+      }
+    }
+    __syncthreads();
+    if (n_eq != need) {
+      // the `need` lowest indices among the ties
+      const int nt = next_pow2((int)n_eq);
+      for (int i = (int)n_eq + threadIdx.x; i < nt; i += blockDim.x) ties[i] = INT_MAX;
+      __syncthreads();
+      bitonic_sort_smem(ties, nt);
+      const uint32_t base = sh_nsel;
+      for (uint32_t i = threadIdx.x; i < need; i += blockDim.x) sel[base + i] = ties[i];
+      __syncthreads();
+    }
+    for (int i = p.k + threadIdx.x; i < nsort; i += blockDim.x) sel[i] = INT_MAX;
+    __syncthreads();
+    bitonic_sort_smem(sel, nsort);
+    for (int i = threadIdx.x; i < p.k; i += blockDim.x) out[i] = sel[i];
+    return;
+  }
+  // ---- bitmap path (large k, or more ties than the sort buffers hold):
+  // index order through bitmaps of v bits
+  __syncthreads();
+  const int words = (v + 31) / 32;
+  uint32_t* bm_eq = bm_sel + words;
+  for (int i = threadIdx.x; i < 2 * words; i += blockDim.x) bm_sel[i] = 0;
+  __syncthreads();
+  for (uint32_t i = threadIdx.x; i < n_above; i += blockDim.x) {
+    const int j = __ldcg(above + i);
+    atomicOr(&bm_sel[j >> 5], 1u << (j & 31));
+  }
   for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
-    const uint2 c = cand[i];
+    const uint2 c = __ldcg(cand + i);
     const uint32_t low = c.x & ((1u << kHistShift) - 1u);
     if (low > prefix) atomicOr(&bm_sel[c.y >> 5], 1u << (c.y & 31));
     else if (low == prefix) atomicOr(&bm_eq[c.y >> 5], 1u << (c.y & 31));

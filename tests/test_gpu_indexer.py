@@ -93,6 +93,26 @@ def test_indexer_decode_shapes(fp8):
     assert api.device_error() == 0
 
 
+def test_indexer_decode_e4m3_long_rows():
+    """e4m3 keys with rows longer than one CTA's top-k (the FP8 indexer builds
+    the row histograms while scoring): a ragged key count, v > k, v = k + 1
+    and v < k rows."""
+    wl = synth.WORKLOADS["decode_1m"]
+    D = synth.Draw(14, DEV)
+    B, N = 4, 40001
+    qI = D.normal("qI", (B, 1, wl.HI, wl.dI), 1.0, torch.bfloat16)
+    w = D.normal("w", (B, 1, wl.HI), 1 / np.sqrt(wl.HI))
+    kI, scale = synth.quantize_e4m3_rows(D.normal("kI", (B, N, wl.dI), 1.0, torch.bfloat16))
+    q_pos = torch.tensor([[4 * N + 3], [4 * N - 9], [4 * (wl.k + 1) - 1], [4 * 700 + 2]], device=DEV,
+                         dtype=torch.int32)
+    idx = api.indexer_topk(qI, w, kI, q_pos, wl.m, wl.k, kI_scale=scale)
+    _check_rows(idx, qI, w, kI, scale, q_pos, wl.m, wl.k, [(b, 0) for b in range(B)])
+    # the same selection a second time (the scratch is reused)
+    idx2 = api.indexer_topk(qI, w, kI, q_pos, wl.m, wl.k, kI_scale=scale)
+    assert torch.equal(idx, idx2)
+    assert api.device_error() == 0
+
+
 def test_indexer_edge_cases():
     """No visible entry (t < m - 1, negative t), exactly k visible, k = 1,
     and all-equal scores (ties go to the lower index)."""
