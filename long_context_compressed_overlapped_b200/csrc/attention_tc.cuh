@@ -16,9 +16,11 @@
 // running max is raised lazily (only when a head's tile max exceeds it by
 // more than 2^8), so O^T is rescaled in TMEM rarely.
 //
-// Roles (192 threads): warps 0-3 query prologue, softmax, epilogue; warp 4
-// TMA producer (4-row gathers for selected entries, 2D tiles for contiguous
-// rows); warp 5 MMA issuer and TMEM owner.  Key tiles arrive in 8 chunks of
+// Roles (384 threads): warps 0-7 query prologue, softmax and epilogue in two
+// groups of four warps, group g owning heads [32g, 32g + 32); warps 8 and 9
+// load key tiles (cp.async gathers of selected rows, 2D TMA tiles of
+// contiguous rows); warp 10 issues the S MMAs and owns TMEM, warp 11 the P.V
+// MMAs.  Key tiles arrive in 8 chunks of
 // 64 dims with their own barriers; chunk pair (2j, 2j+1) is released as soon
 // as the P.V of O^T M-tile j has read it, so the next tile's loads overlap
 // the tail of the current one.
@@ -30,7 +32,7 @@
 
 namespace csahca {
 
-constexpr int kAttnTcThreads = 224;   // warps 0-3 softmax, 4 and 6 loads, 5 MMA
+constexpr int kAttnTcThreads = 384;   // warps 0-7 softmax (two head groups), 8-9 loads, 10-11 MMA
 constexpr int kAttnH = 64;          // heads (MMA N of both products)
 constexpr int kAttnD = 512;         // head dim
 constexpr int kAttnChunks = kAttnD / 64;
@@ -124,13 +126,50 @@ __device__ __forceinline__ AttnTile attn_tile(const AttnTcParams& p, const AttnI
   return T;
 }
 
-// 64 per-thread values -> per-head reduction over the 128 threads of warps
-// 0-3.  Returns in out[64] (shared).  kMax: max, else sum.
+// Named barrier 3 over the 256 softmax threads (both head groups).
+__device__ __forceinline__ void softmax_sync256() { asm volatile("bar.sync 3, 256;" ::: "memory"); }
+__device__ __forceinline__ bool softmax_any256(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 3, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ bool softmax_all256(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 3, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+// OR of v over the 128 threads of named barrier `id`.
+__device__ __forceinline__ bool group_any(int id, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
+// 32 per-thread values (one per head of the group) -> per-head reduction over
+// the group's 128 key slots: a warp transpose-reduction (31 shuffles) leaves
+// head `lane` in lane `lane`, then the 4 warps combine through shared memory.
+// red: 4 x 32 floats of this group; out: the group's 32 heads.  kMax: max,
+// else sum.  Ends with a group barrier.
 template <bool kMax>
-__device__ __forceinline__ void reduce_heads(float (&v)[kAttnH], float* red, float* out) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__device__ __forceinline__ void reduce_group32(float (&v)[32], float* red, float* out, int gid) {
+  const int lane = threadIdx.x & 31, wq = (threadIdx.x >> 5) & 3;
 #pragma unroll
-  for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
+  for (int o = 16, n = 16; o >= 1; o >>= 1, n >>= 1) {
 #pragma unroll
     for (int j = 0; j < n; ++j) {
       const bool hi = lane & o;
@@ -140,32 +179,16 @@ __device__ __forceinline__ void reduce_heads(float (&v)[kAttnH], float* red, flo
       v[j] = kMax ? fmaxf(keep, got) : keep + got;
     }
   }
-  red[warp * kAttnH + 2 * lane] = v[0];
-  red[warp * kAttnH + 2 * lane + 1] = v[1];
-  named_sync128();
-  if (threadIdx.x < kAttnH) {
-    const int h = threadIdx.x;
+  red[wq * 32 + lane] = v[0];
+  group_sync(gid);
+  if ((threadIdx.x & 127) < 32) {
+    const int h = threadIdx.x & 31;
     float r = red[h];
 #pragma unroll
-    for (int w = 1; w < 4; ++w) r = kMax ? fmaxf(r, red[w * kAttnH + h]) : r + red[w * kAttnH + h];
+    for (int w = 1; w < 4; ++w) r = kMax ? fmaxf(r, red[w * 32 + h]) : r + red[w * 32 + h];
     out[h] = r;
   }
-  named_sync128();
-}
-
-// S^T row of this thread (64 heads) from TMEM, times each head's scale (log2
-// units); -inf for a masked key.
-__device__ __forceinline__ void load_scores(uint32_t taddr, bool valid, const float* scale_log2,
-                                            float (&s)[kAttnH]) {
-  float v[32];
-  tmem_ld32(taddr, v);
-  tmem_wait_ld();
-#pragma unroll
-  for (int e = 0; e < 32; ++e) s[e] = valid ? v[e] * scale_log2[e] : -INFINITY;
-  tmem_ld32(taddr + 32, v);
-  tmem_wait_ld();
-#pragma unroll
-  for (int e = 0; e < 32; ++e) s[32 + e] = valid ? v[e] * scale_log2[32 + e] : -INFINITY;
+  group_sync(gid);
 }
 
 struct AttnSmem {
@@ -180,6 +203,10 @@ struct AttnSmem {
 // Decode partial of one (query, split): m[H], l[H] fp32, then O / l fp16 [D][H].
 constexpr int kTcPartialHeader = 2 * kAttnH * 4;
 constexpr int kTcPartialBytes = kTcPartialHeader + kAttnD * kAttnH * 2;
+// The same blocks seen as 128-byte rows (64 fp16), as the TMA store writes them.
+constexpr int kTcPartialRows = kTcPartialBytes / 128;
+constexpr int kTcPartialHeaderRows = kTcPartialHeader / 128;
+static_assert(kTcPartialBytes % 128 == 0 && kTcPartialHeader % 128 == 0, "partial blocks are whole 128-byte rows");
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   const __half2 h = __floats2half2_rn(a, b);
@@ -189,7 +216,7 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 __global__ void __launch_bounds__(kAttnTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_constant__ CUtensorMap comp_gather,
                const __grid_constant__ CUtensorMap win_rows, const __grid_constant__ CUtensorMap q_rows,
-               AttnTcParams p) {
+               const __grid_constant__ CUtensorMap part_rows, AttnTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
@@ -200,15 +227,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       bar_done;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
-  __shared__ float red[4 * kAttnH];
+  __shared__ float red[2][4 * 32];
   __shared__ __align__(16) float stat_a[kAttnH];
   __shared__ __align__(16) float m_use[kAttnH];
   __shared__ __align__(16) float sc_h[kAttnH];     // softmax scale of head h (log2 units, times inv_rms_h)
-  __shared__ float alpha[kAttnH], l_run[kAttnH];
+  __shared__ __align__(16) float alpha[kAttnH];
+  __shared__ float l_run[kAttnH];
   __shared__ float rope_cs[64], rope_sn[64];
+  __shared__ double theta_s[64];                   // RoPE frequency of pair j
   __shared__ __align__(16) float gain_s[kAttnD];
   __shared__ int rows_s[2][128];
-  __shared__ int need_rescale;
+  __shared__ int need_rescale[2];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -216,15 +245,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     for (int c = 0; c < kAttnChunks; ++c) { mbar_init(&bar_kfull[c], 32); mbar_init(&bar_kempty[c], 1); }
     mbar_init(&bar_q_raw, 1);
     mbar_init(&bar_q_empty, 1);
-    mbar_init(&bar_q_full, 128);
+    mbar_init(&bar_q_full, 256);
     mbar_init(&bar_s_full, 1);
-    mbar_init(&bar_s_empty, 128);
-    mbar_init(&bar_p_full, 128);
+    mbar_init(&bar_s_empty, 256);
+    mbar_init(&bar_p_full, 256);
     mbar_init(&bar_pv_done, 1);
-    mbar_init(&bar_done, 1);
+    mbar_init(&bar_done, 2);                       // both MMA issuers
     mbar_fence_init();
   }
-  if (warp == 5) tmem_alloc(&tmem_base_sh, 512);
+  if (warp == 10) tmem_alloc(&tmem_base_sh, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -234,10 +263,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
   const uint32_t tL = tmem + 128 + kAttnMT * kAttnH;   // per-key-slot partial sums of p: H columns
   griddep_launch_dependents();
 
-  if (warp == 4 || warp == 6) {
+  if (warp == 8 || warp == 9) {
     // ------------------------------------------------------------ producers
-    // warp 4 loads chunks 0,1,4,5 (and the raw Q); warp 6 chunks 2,3,6,7
-    const int pw = warp == 4 ? 0 : 1;
+    // warp 8 loads chunks 0,1,4,5 (and the raw Q); warp 9 chunks 2,3,6,7
+    const int pw = warp - 8;
     tma_prefetch_desc(&comp_rows);
     tma_prefetch_desc(&comp_gather);
     tma_prefetch_desc(&win_rows);
@@ -249,7 +278,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       if (it.tile1 <= it.tile0) continue;
       if (pw == 0) {
         // raw Q of this item into the Q buffer once the previous item's
-        // score MMAs have read it; normed and roped there by warps 0-3
+        // score MMAs have read it; roped there by the softmax warps
         int ok = 1;
         if (lane == 0) {
           ok = mbar_wait(&bar_q_empty, (icount & 1) ^ 1, &abort_flag);
@@ -270,6 +299,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       for (int tile = it.tile0; tile < it.tile1 && !stop; ++tile, ++tcount) {
         const AttnTile T = attn_tile(p, it, tile);
         const uint32_t ph = tcount & 1;
+        // L2 prefetch of the next tile's rows: HBM streams while this tile is
+        // processed, and the next tile's shared-memory loads hit L2 (the
+        // current tile is loaded right away, so it is not prefetched)
+        if (pw == 0 && tile + 1 < it.tile1) {
+          const AttnTile Tn = attn_tile(p, it, tile + 1);
+          if (Tn.src == 0) {
+            const int* L = p.idx + ((int64_t)it.b * p.nq + it.qi) * p.k + Tn.list_off;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = lane + 32 * e;
+              if (j < Tn.hi) {
+                const int v = __ldg(L + j);
+                if (v >= 0 && v < p.N) bulk_prefetch_l2(p.kv_comp_ptr + ((int64_t)it.b * p.N + v) * kAttnD, kAttnD * 2);
+              }
+            }
+          } else if (lane < kAttnChunks && Tn.row0 >= 0) {
+            tma_prefetch_l2_2d(Tn.src == 1 ? &comp_rows : &win_rows, lane * 64, Tn.row0);
+          }
+        }
         if (T.src == 0) {
           // selected rows of this tile (clamped; masked later by the softmax)
           const int* L = p.idx + ((int64_t)it.b * p.nq + it.qi) * p.k + T.list_off;
@@ -295,11 +343,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
             // chunk; each lane arrives on the chunk's barrier when its copies
             // have landed, without waiting for them
             const int piece = lane & 7, rg = lane >> 3;
-            const __nv_bfloat16* base = p.kv_comp_ptr + c * 64 + piece * 8;
+            const __nv_bfloat16* src = p.kv_comp_ptr + c * 64 + piece * 8;
 #pragma unroll 8
             for (int j = 0; j < 32; ++j) {
               const int r = 4 * j + rg;
-              cp_async16(dst + sw128_offset(r, piece * 16), base + (int64_t)rows_s[pw][r] * kAttnD);
+              cp_async16(dst + sw128_offset(r, piece * 16), src + (int64_t)rows_s[pw][r] * kAttnD);
             }
             cp_async_arrive_noinc(&bar_kfull[c]);
           } else {
@@ -319,27 +367,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       for (int cc = 0; cc < kAttnChunks / 2; ++cc)
         mbar_wait(&bar_kfull[4 * (cc >> 1) + 2 * pw + (cc & 1)], (tcount - 1) & 1, &abort_flag);
     if (pw == 0 && lane == 0 && icount > 0) mbar_wait(&bar_q_raw, (icount - 1) & 1, &abort_flag);
-  } else if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ S MMA issuer
+    // (a separate thread issues the P.V MMAs, so the S MMAs of tile t+1 go out
+    // while those of P.V(t) still do)
     if (lane == 0) {
       constexpr uint32_t idesc_s = umma_idesc_bf16(128, kAttnH, 0, 0);
-      constexpr uint32_t idesc_pv = umma_idesc_bf16(128, kAttnH, 1, 1);
       // base descriptors; chunk / K-step offsets are adds in 16-byte units
       const uint64_t kdesc = umma_desc_kmajor(smem_u32(sK)), qdesc = umma_desc_kmajor(smem_u32(sQ));
-      const uint64_t vdesc = umma_desc_mnmajor(smem_u32(sK), AttnSmem::K_CHUNK);
-      const uint64_t pdesc = umma_desc_mnmajor(smem_u32(sP), AttnSmem::P_BYTES);
       uint32_t tcount = 0, icount = 0;
-      for (int id = blockIdx.x; id < p.n_items && !abort_flag; id += gridDim.x) {
+      bool stop = false;
+      for (int id = blockIdx.x; id < p.n_items && !stop && !abort_flag; id += gridDim.x) {
         const AttnItem it = attn_item(p, id);
         if (it.tile1 <= it.tile0) continue;
         if (!mbar_wait(&bar_q_full, icount & 1, &abort_flag)) break;
         ++icount;
-        for (int tile = it.tile0; tile < it.tile1; ++tile, ++tcount) {
+        for (int tile = it.tile0; tile < it.tile1 && !stop; ++tile, ++tcount) {
           const uint32_t ph = tcount & 1;
-          if (!mbar_wait(&bar_s_empty, ph ^ 1, &abort_flag)) break;
+          if (!mbar_wait(&bar_s_empty, ph ^ 1, &abort_flag)) { stop = true; break; }
           tc_fence_after();
           for (int c = 0; c < kAttnChunks; ++c) {
-            if (!mbar_wait(&bar_kfull[c], ph, &abort_flag)) break;
+            if (!mbar_wait(&bar_kfull[c], ph, &abort_flag)) { stop = true; break; }
             fence_proxy_async_smem();
             tc_fence_after();
             const uint64_t kd = kdesc + (uint64_t)(c * (AttnSmem::K_CHUNK >> 4));
@@ -347,9 +395,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) umma_bf16(tS, kd + 2 * ks, qd + 2 * ks, idesc_s, (c | ks) != 0);
           }
+          if (stop) break;
           umma_commit(&bar_s_full);
           if (tile == it.tile1 - 1) umma_commit(&bar_q_empty);
-          if (!mbar_wait(&bar_p_full, ph, &abort_flag)) break;
+        }
+      }
+      umma_commit(&bar_done);
+      mbar_wait(&bar_done, 0, &abort_flag);
+    }
+  } else if (warp == 11) {
+    // ------------------------------------------------------------ P.V MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_pv = umma_idesc_bf16(128, kAttnH, 1, 1);
+      const uint64_t vdesc = umma_desc_mnmajor(smem_u32(sK), AttnSmem::K_CHUNK);
+      const uint64_t pdesc = umma_desc_mnmajor(smem_u32(sP), AttnSmem::P_BYTES);
+      uint32_t tcount = 0;
+      bool stop = false;
+      for (int id = blockIdx.x; id < p.n_items && !stop && !abort_flag; id += gridDim.x) {
+        const AttnItem it = attn_item(p, id);
+        for (int tile = it.tile0; tile < it.tile1; ++tile, ++tcount) {
+          const uint32_t ph = tcount & 1;
+          if (!mbar_wait(&bar_p_full, ph, &abort_flag)) { stop = true; break; }
           tc_fence_after();
           const bool first = tile == it.tile0;
 #pragma unroll
@@ -367,121 +433,139 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       umma_commit(&bar_done);
       mbar_wait(&bar_done, 0, &abort_flag);
     }
-  } else {
-    // ------------------------------------------------------------ softmax / epilogue (warps 0-3)
-    const int tid = threadIdx.x;               // key slot / dim slot
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax / epilogue
+    // Two groups of 4 warps; group g owns heads [32g, 32g + 32): its columns
+    // of S^T, O^T and the row sums in TMEM, and its 64 bytes of each P^T row.
+    // Thread tid of a group is key slot tid of a tile and dim slot tid of
+    // each O^T M-tile (TMEM lane).
+    const int g = warp >> 2;
+    const int gid = 1 + g;                   // the group's named barrier
+    const int tid = threadIdx.x & 127;
+    const int st = threadIdx.x;              // 0..255 over both groups
+    const int h0 = 32 * g;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     uint32_t tcount = 0, qcount = 0;
     const int r0 = kAttnD - p.rope_dims;
-    bool stop = false;                       // uniform over the 128 threads
     // q gain (same for every head and query) staged once in shared memory;
     // an all-ones gain (or none) leaves the non-rope dims of q untouched
     bool ones = true;
-    for (int x = tid; x < kAttnD; x += 128) {
-      const float g = (p.q_norm && p.q_gain) ? __ldg(p.q_gain + x) : 1.f;
-      gain_s[x] = g;
-      ones = ones && g == 1.f;
+    for (int x = st; x < kAttnD; x += 256) {
+      const float gv = (p.q_norm && p.q_gain) ? __ldg(p.q_gain + x) : 1.f;
+      gain_s[x] = gv;
+      ones = ones && gv == 1.f;
     }
-    const bool gain_ones = group128_all(ones);
-    for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
+    if (st < p.rope_dims / 2) theta_s[st] = rope_theta(st, p.rope_dims, p.rope_base);
+    const bool gain_ones = softmax_all256(ones);
+    for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
       const AttnItem it = attn_item(p, id);
       const bool empty = it.tile1 <= it.tile0;
+      bool bad = false;                      // uniform over the group; both groups leave together
       // ---- query prologue.  RoPE is linear and the RMSNorm factor is one
       // scalar per head, so RoPE_t(RMSNorm(q) * g) = inv_rms_h * RoPE_t(q * g):
       // the MMA operand is RoPE_t(q * g) (with an all-ones gain only the rope
       // dims are rewritten), and inv_rms_h joins the softmax scale of head h.
       if (!empty) {
-        if (tid < p.rope_dims / 2) {
+        if (st < p.rope_dims / 2) {
           float cs, sn;
-          rope_cos_sin((double)it.t, tid, p.rope_dims, p.rope_base, &cs, &sn);
-          rope_cs[tid] = cs;
-          rope_sn[tid] = sn;
+          rope_sincos((double)it.t, theta_s[st], &cs, &sn);
+          rope_cs[st] = cs;
+          rope_sn[st] = sn;
         }
-        if (tid < kAttnH) m_use[tid] = -INFINITY;
-        if (!mbar_wait128(&bar_q_raw, qcount & 1, &abort_flag)) { stop = true; break; }
+        if (st < kAttnH) m_use[st] = -INFINITY;
+        // (the 256-thread reduction also publishes rope_cs / rope_sn)
+        bad = !softmax_all256(mbar_wait(&bar_q_raw, qcount & 1, &abort_flag));
         ++qcount;
-        // thread (head h, half) owns dims [256 * half, 256 * half + 256) of row h
-        const int h = tid >> 1, half = tid & 1;
-        float ss = 0.f;
-        if (!gain_ones) {
-          // q * g on every dim (sum of squares from the raw values), RoPE on the rope dims
+        if (!bad) {
+          // thread (head h, quarter qq) owns dims [128 qq, 128 qq + 128) of row h
+          const int h = st >> 2, qq = st & 3;
+          float ss = 0.f;
+          if (!gain_ones) {
+            // q * g on every dim (sum of squares from the raw values), RoPE on the rope dims
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            const int chunk = 4 * half + c;
-            uint8_t* row = sQ + chunk * AttnSmem::Q_CHUNK;
+            for (int c = 0; c < 2; ++c) {
+              const int chunk = 2 * qq + c;
+              uint8_t* row = sQ + chunk * AttnSmem::Q_CHUNK;
 #pragma unroll
-            for (int pc = 0; pc < 8; ++pc) {
-              uint4* a = reinterpret_cast<uint4*>(row + sw128_offset(h, pc * 16));
-              float x[8];
-              {
-                const uint4 raw = *a;
-                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+              for (int pc = 0; pc < 8; ++pc) {
+                uint4* a = reinterpret_cast<uint4*>(row + sw128_offset(h, pc * 16));
+                float x[8];
+                {
+                  const uint4 raw = *a;
+                  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const float2 f = __bfloat1622float2(h2[i]);
-                  x[2 * i] = f.x; x[2 * i + 1] = f.y;
+                  for (int i = 0; i < 4; ++i) {
+                    const float2 f = __bfloat1622float2(h2[i]);
+                    x[2 * i] = f.x; x[2 * i + 1] = f.y;
+                  }
                 }
+                const int d0 = chunk * 64 + pc * 8;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) { ss = fmaf(x[e], x[e], ss); x[e] *= gain_s[d0 + e]; }
+                if (d0 + 7 >= r0) {
+#pragma unroll
+                  for (int e = 0; e < 8; e += 2) {
+                    if (d0 + e >= r0) {
+                      const int j = (d0 + e - r0) >> 1;
+                      const float x0 = x[e], x1 = x[e + 1];
+                      x[e] = x0 * rope_cs[j] - x1 * rope_sn[j];
+                      x[e + 1] = x0 * rope_sn[j] + x1 * rope_cs[j];
+                    }
+                  }
+                }
+                uint4 o;
+                store16(reinterpret_cast<__nv_bfloat16*>(&o), x);
+                *a = o;
               }
-              const int d0 = chunk * 64 + pc * 8;
+            }
+          } else {
+            // RoPE on the rope dims only: pairs (r0 + 2j, r0 + 2j + 1), this
+            // thread taking j = qq, qq + 4, ...
+            for (int j = qq; j < p.rope_dims / 2; j += 4) {
+              const int dim = r0 + 2 * j;
+              __nv_bfloat162* a = reinterpret_cast<__nv_bfloat162*>(sQ + (dim >> 6) * AttnSmem::Q_CHUNK +
+                                                                     sw128_offset(h, (dim & 63) * 2));
+              const float2 f = __bfloat1622float2(*a);
+              *a = __floats2bfloat162_rn(f.x * rope_cs[j] - f.y * rope_sn[j], f.x * rope_sn[j] + f.y * rope_cs[j]);
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&bar_q_full);
+          if (p.q_norm) {
+            if (gain_ones) {
+              // the rotation keeps every pair's norm: sum the squares of the
+              // operand once every pair is rotated (the MMAs already run)
+              softmax_sync256();
+#pragma unroll 1
+              for (int c = 0; c < 2; ++c) {
+                const uint8_t* row = sQ + (2 * qq + c) * AttnSmem::Q_CHUNK;
 #pragma unroll
-              for (int e = 0; e < 8; ++e) { ss = fmaf(x[e], x[e], ss); x[e] *= gain_s[d0 + e]; }
-              if (d0 + 7 >= r0) {
+                for (int pc = 0; pc < 8; ++pc) {
+                  const uint4 raw = *reinterpret_cast<const uint4*>(row + sw128_offset(h, pc * 16));
+                  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                  if (d0 + e >= r0) {
-                    const int j = (d0 + e - r0) >> 1;
-                    const float x0 = x[e], x1 = x[e + 1];
-                    x[e] = x0 * rope_cs[j] - x1 * rope_sn[j];
-                    x[e + 1] = x0 * rope_sn[j] + x1 * rope_cs[j];
+                  for (int i = 0; i < 4; ++i) {
+                    const float2 f = __bfloat1622float2(h2[i]);
+                    ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
                   }
                 }
               }
-              uint4 o;
-              store16(reinterpret_cast<__nv_bfloat16*>(&o), x);
-              *a = o;
             }
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+            if (qq == 0) sc_h[h] = p.scale_log2 * rsqrtf(ss / (float)kAttnD + p.eps);
+          } else if (qq == 0) {
+            sc_h[h] = p.scale_log2;
           }
-        } else {
-          // RoPE on the rope dims only: pairs (r0 + 2j, r0 + 2j + 1), this
-          // thread taking j = half, half + 2, ...
-          for (int j = half; j < p.rope_dims / 2; j += 2) {
-            const int dim = r0 + 2 * j;
-            __nv_bfloat162* a = reinterpret_cast<__nv_bfloat162*>(sQ + (dim >> 6) * AttnSmem::Q_CHUNK +
-                                                                   sw128_offset(h, (dim & 63) * 2));
-            const float2 f = __bfloat1622float2(*a);
-            *a = __floats2bfloat162_rn(f.x * rope_cs[j] - f.y * rope_sn[j], f.x * rope_sn[j] + f.y * rope_cs[j]);
-          }
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&bar_q_full);
-        if (p.q_norm) {
-          if (gain_ones) {
-            // the rotation keeps every pair's norm: sum the squares of the operand
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              const uint8_t* row = sQ + (4 * half + c) * AttnSmem::Q_CHUNK;
-#pragma unroll
-              for (int pc = 0; pc < 8; ++pc) {
-                const uint4 raw = *reinterpret_cast<const uint4*>(row + sw128_offset(h, pc * 16));
-                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const float2 f = __bfloat1622float2(h2[i]);
-                  ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
-                }
-              }
-            }
-          }
-          ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-          if (half == 0) sc_h[h] = p.scale_log2 * rsqrtf(ss / (float)kAttnD + p.eps);
-        } else if (half == 0) {
-          sc_h[h] = p.scale_log2;
         }
       }
-      named_sync128();
-      griddep_wait();                                // selections read, outputs written below
+      softmax_sync256();                     // sc_h, m_use complete
+      griddep_wait();                        // selections read, outputs written below
 
+      const float4* sc4 = reinterpret_cast<const float4*>(sc_h + h0);
+      const float4* mu4 = reinterpret_cast<const float4*>(m_use + h0);
       for (int tile = it.tile0; tile < it.tile1; ++tile, ++tcount) {
+        if (bad) continue;
         const uint32_t ph = tcount & 1;
         const bool first = tile == it.tile0;
         const AttnTile T = attn_tile(p, it, tile);
@@ -490,111 +574,105 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
           const int e = __ldg(p.idx + ((int64_t)it.b * p.nq + it.qi) * p.k + T.list_off + tid);
           valid = e >= 0 && e < p.N;
         }
-        if (!mbar_wait128(&bar_s_full, ph, &abort_flag)) { stop = true; break; }
+        if (!mbar_wait_group(gid, &bar_s_full, ph, &abort_flag)) { bad = true; continue; }
         tc_fence_after();
+        // this key's scores for the group's heads, scaled to log2 units
+        float v[32];
+        tmem_ld32(tS + lane_base + h0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 sc = sc4[e4];
+          v[4 * e4 + 0] = valid ? v[4 * e4 + 0] * sc.x : -INFINITY;
+          v[4 * e4 + 1] = valid ? v[4 * e4 + 1] * sc.y : -INFINITY;
+          v[4 * e4 + 2] = valid ? v[4 * e4 + 2] * sc.z : -INFINITY;
+          v[4 * e4 + 3] = valid ? v[4 * e4 + 3] * sc.w : -INFINITY;
+        }
         // The running max m_use is raised only when some score of this tile
-        // exceeds it by more than 2^8 (or on the item's first tile); else the
-        // per-tile max is not needed at all.  S stays in TMEM until p_full.
+        // exceeds it by more than 2^8 (or on the item's first tile).
         bool exceed = first;
         if (!first) {
-          const float4* mu4 = reinterpret_cast<const float4*>(m_use);
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            float v[32];
-            tmem_ld32(tS + lane_base + half * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-              const float4 mu = mu4[half * 8 + e4];
-              const float4 sc = reinterpret_cast<const float4*>(sc_h)[half * 8 + e4];
-              exceed |= (v[4 * e4 + 0] * sc.x > mu.x + kRescaleThreshold) |
-                        (v[4 * e4 + 1] * sc.y > mu.y + kRescaleThreshold) |
-                        (v[4 * e4 + 2] * sc.z > mu.z + kRescaleThreshold) |
-                        (v[4 * e4 + 3] * sc.w > mu.w + kRescaleThreshold);
-            }
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 mu = mu4[e4];
+            exceed |= (v[4 * e4 + 0] > mu.x + kRescaleThreshold) | (v[4 * e4 + 1] > mu.y + kRescaleThreshold) |
+                      (v[4 * e4 + 2] > mu.z + kRescaleThreshold) | (v[4 * e4 + 3] > mu.w + kRescaleThreshold);
           }
-          exceed = exceed && valid;
         }
-        exceed = group128_any(exceed);
+        exceed = group_any(gid, exceed);
         bool rescale = false;
         if (exceed) {
           {
-            float v[kAttnH];
-            load_scores(tS + lane_base, valid, sc_h, v);
-            reduce_heads<true>(v, red, stat_a);           // stat_a = tile max per head
+            float t[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) t[e] = v[e];
+            reduce_group32<true>(t, red[g], stat_a + h0, gid);      // stat_a = tile max per head
           }
-          if (tid == 0) need_rescale = 0;
-          named_sync128();
-          if (tid < kAttnH) {
-            const float mt = stat_a[tid], mo = m_use[tid];
+          if (tid == 0) need_rescale[g] = 0;
+          group_sync(gid);
+          if (tid < 32) {
+            const int h = h0 + tid;
+            const float mt = stat_a[h], mo = m_use[h];
             float a = 1.f;
             if (mt > mo + kRescaleThreshold || (mo == -INFINITY && mt != -INFINITY)) {
               a = (mo == -INFINITY) ? 0.f : exp2f(mo - mt);
-              m_use[tid] = mt;
-              if (!first) need_rescale = 1;
+              m_use[h] = mt;
+              if (!first) need_rescale[g] = 1;
             }
-            alpha[tid] = a;
+            alpha[h] = a;
           }
-          named_sync128();
-          rescale = need_rescale != 0;
+          group_sync(gid);
+          rescale = need_rescale[g] != 0;
         }
         // the previous tile's P.V has finished: P^T may be overwritten and
         // O^T / the partial sums rescaled
         if (!first) {
-          if (!mbar_wait128(&bar_pv_done, ph ^ 1, &abort_flag)) { stop = true; break; }
+          if (!mbar_wait_group(gid, &bar_pv_done, ph ^ 1, &abort_flag)) { bad = true; continue; }
           tc_fence_after();
         }
         if (rescale) {
+          const float4* al4 = reinterpret_cast<const float4*>(alpha + h0);
 #pragma unroll 1
           for (int mt = 0; mt <= kAttnMT; ++mt) {            // O^T M-tiles, then the partial sums
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              float v[32];
-              const uint32_t a = (mt < kAttnMT ? tO + mt * kAttnH : tL) + lane_base + half * 32;
-              tmem_ld32(a, v);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) v[e] *= alpha[half * 32 + e];
-              tmem_st32(a, v);
-            }
-          }
-          tmem_wait_st();
-        }
-        // p = 2^(S * scale - m) (masked keys give 0), in two halves of 32
-        // heads: P^T row tid into the MN-major SW128 tile, and this key slot's
-        // running sums per head in TMEM
-        {
-          const float4* mu4 = reinterpret_cast<const float4*>(m_use);
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            float v[32];
-            tmem_ld32(tS + lane_base + half * 32, v);
+            float o[32];
+            const uint32_t a = (mt < kAttnMT ? tO + mt * kAttnH : tL) + lane_base + h0;
+            tmem_ld32(a, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e4 = 0; e4 < 8; ++e4) {
-              const float4 mu = mu4[half * 8 + e4];
-              const float4 sc = reinterpret_cast<const float4*>(sc_h)[half * 8 + e4];
-              v[4 * e4 + 0] = valid ? fast_exp2(fmaf(v[4 * e4 + 0], sc.x, -mu.x)) : 0.f;
-              v[4 * e4 + 1] = valid ? fast_exp2(fmaf(v[4 * e4 + 1], sc.y, -mu.y)) : 0.f;
-              v[4 * e4 + 2] = valid ? fast_exp2(fmaf(v[4 * e4 + 2], sc.z, -mu.z)) : 0.f;
-              v[4 * e4 + 3] = valid ? fast_exp2(fmaf(v[4 * e4 + 3], sc.w, -mu.w)) : 0.f;
+              const float4 al = al4[e4];
+              o[4 * e4 + 0] *= al.x; o[4 * e4 + 1] *= al.y; o[4 * e4 + 2] *= al.z; o[4 * e4 + 3] *= al.w;
             }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              uint4 o;
-              store16(reinterpret_cast<__nv_bfloat16*>(&o), v + 8 * j);
-              *reinterpret_cast<uint4*>(sP + sw128_offset(tid, (half * 4 + j) * 16)) = o;
-            }
-            const uint32_t la = tL + lane_base + half * 32;
-            if (!first) {
-              float l[32];
-              tmem_ld32(la, l);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) v[e] += l[e];
-            }
-            tmem_st32(la, v);
+            tmem_st32(a, o);
           }
+          tmem_wait_st();
+        }
+        // p = 2^(s - m) (masked keys give 0): P^T row tid, bytes [64g, 64g + 64),
+        // and this key slot's running sums per head in TMEM
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 mu = mu4[e4];
+          v[4 * e4 + 0] = valid ? fast_exp2(v[4 * e4 + 0] - mu.x) : 0.f;
+          v[4 * e4 + 1] = valid ? fast_exp2(v[4 * e4 + 1] - mu.y) : 0.f;
+          v[4 * e4 + 2] = valid ? fast_exp2(v[4 * e4 + 2] - mu.z) : 0.f;
+          v[4 * e4 + 3] = valid ? fast_exp2(v[4 * e4 + 3] - mu.w) : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 o;
+          store16(reinterpret_cast<__nv_bfloat16*>(&o), v + 8 * j);
+          *reinterpret_cast<uint4*>(sP + sw128_offset(tid, (4 * g + j) * 16)) = o;
+        }
+        {
+          const uint32_t la = tL + lane_base + h0;
+          if (!first) {
+            float l[32];
+            tmem_ld32(la, l);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] += l[e];
+          }
+          tmem_st32(la, v);
           tmem_wait_st();
         }
         fence_proxy_async_smem();
@@ -602,134 +680,134 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
         mbar_arrive(&bar_s_empty);
         mbar_arrive(&bar_p_full);
       }
-      if (stop) break;
-      if (empty && !p.decode) {
-        // no key at all: only the sink is in the denominator, o = 0
-        __nv_bfloat16* O = p.out + ((int64_t)it.b * p.nq + it.qi) * kAttnH * kAttnD;
-        for (int x = tid; x < kAttnH * kAttnD; x += 128) O[x] = __float2bfloat16_rn(0.f);
-        continue;
-      }
       // ---- epilogue: wait for the last P.V, reduce the sums, write out
-      if (!empty) {
-        if (!mbar_wait128(&bar_pv_done, (tcount - 1) & 1, &abort_flag)) { stop = true; break; }
-        tc_fence_after();
+      if (!empty && !bad) {
+        if (!mbar_wait_group(gid, &bar_pv_done, (tcount - 1) & 1, &abort_flag)) bad = true;
+        else tc_fence_after();
       }
-      if (!empty) {
-        float v[kAttnH];
-        tmem_ld32(tL + lane_base, *reinterpret_cast<float(*)[32]>(v));
+      if (!empty && !bad) {
+        float v[32];
+        tmem_ld32(tL + lane_base + h0, v);
         tmem_wait_ld();
-        tmem_ld32(tL + lane_base + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-        tmem_wait_ld();
-        reduce_heads<false>(v, red, l_run);            // l_run = sum of p per head
+        reduce_group32<false>(v, red[g], l_run + h0, gid);     // l_run = sum of p per head
       }
-      named_sync128();                                 // l_run / m_use complete
-      if (p.decode) {
-        // partial block of (query, split): m[H] (log2 units) and l[H] in fp32,
-        // then O / l as fp16 [D][H] (a thread writes its dim's 64 heads, 128
-        // contiguous bytes, straight from TMEM); an empty split writes only
-        // m = -inf, which the combine skips
-        char* P = reinterpret_cast<char*>(p.partial) +
-                  (((int64_t)it.b * p.nq + it.qi) * p.splits + it.split) * kTcPartialBytes;
-        float* hdr = reinterpret_cast<float*>(P);
-        if (tid < kAttnH) {
-          const float l = empty ? 0.f : l_run[tid];
-          hdr[tid] = empty ? -INFINITY : m_use[tid];
-          hdr[kAttnH + tid] = l;
-          stat_a[tid] = l > 0.f ? 1.f / l : 0.f;
-        }
-        named_sync128();
-        if (!empty) {
-          const float4* f4 = reinterpret_cast<const float4*>(stat_a);
+      bad = softmax_any256(bad);             // the output stage is entered by both groups or neither
+      if (!bad) {
+        if (p.decode) {
+          // partial block of (query, split): m[H] (log2 units) and l[H] in
+          // fp32, then O / l as fp16 [D][H] (a thread writes its dim's 32
+          // heads, 64 contiguous bytes, straight from TMEM); an empty split
+          // writes only m = -inf, which the combine skips
+          char* P = reinterpret_cast<char*>(p.partial) +
+                    (((int64_t)it.b * p.nq + it.qi) * p.splits + it.split) * kTcPartialBytes;
+          float* hdr = reinterpret_cast<float*>(P);
+          if (tid < 32) {
+            const int h = h0 + tid;
+            const float l = empty ? 0.f : l_run[h];
+            hdr[h] = empty ? -INFINITY : m_use[h];
+            hdr[kAttnH + h] = l;
+            stat_a[h] = l > 0.f ? 1.f / l : 0.f;
+          }
+          group_sync(gid);
+          if (!empty) {
+            // O / l of M-tile mt: 128 dims x 64 heads fp16 = 128-byte rows,
+            // staged in P's buffer with the 128-byte swizzle (group g writes
+            // pieces 4g..4g+3 of row tid) and stored by one TMA box
+            const float4* f4 = reinterpret_cast<const float4*>(stat_a + h0);
+            const int blk = ((it.b * p.nq + it.qi) * p.splits + it.split);
 #pragma unroll 1
-          for (int mt = 0; mt < kAttnMT; ++mt) {
-            uint4* dst = reinterpret_cast<uint4*>(P + kTcPartialHeader + (int64_t)(mt * 128 + tid) * kAttnH * 2);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              float v[32];
-              tmem_ld32(tO + lane_base + mt * kAttnH + half * 32, v);
+            for (int mt = 0; mt < kAttnMT; ++mt) {
+              float o[32];
+              tmem_ld32(tO + lane_base + mt * kAttnH + h0, o);
               tmem_wait_ld();
 #pragma unroll
               for (int e4 = 0; e4 < 8; ++e4) {
-                const float4 f = f4[half * 8 + e4];
-                v[4 * e4 + 0] *= f.x; v[4 * e4 + 1] *= f.y; v[4 * e4 + 2] *= f.z; v[4 * e4 + 3] *= f.w;
+                const float4 f = f4[e4];
+                o[4 * e4 + 0] *= f.x; o[4 * e4 + 1] *= f.y; o[4 * e4 + 2] *= f.z; o[4 * e4 + 3] *= f.w;
               }
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                uint4 o;
-                o.x = pack_half2(v[8 * q + 0], v[8 * q + 1]);
-                o.y = pack_half2(v[8 * q + 2], v[8 * q + 3]);
-                o.z = pack_half2(v[8 * q + 4], v[8 * q + 5]);
-                o.w = pack_half2(v[8 * q + 6], v[8 * q + 7]);
-                dst[half * 4 + q] = o;
+                uint4 w;
+                w.x = pack_half2(o[8 * q + 0], o[8 * q + 1]);
+                w.y = pack_half2(o[8 * q + 2], o[8 * q + 3]);
+                w.z = pack_half2(o[8 * q + 4], o[8 * q + 5]);
+                w.w = pack_half2(o[8 * q + 6], o[8 * q + 7]);
+                *reinterpret_cast<uint4*>(sP + sw128_offset(tid, (4 * g + q) * 16)) = w;
               }
+              fence_proxy_async_smem();
+              softmax_sync256();
+              if (st == 0) {
+                tma_store_2d(&part_rows, sP, 0, blk * kTcPartialRows + kTcPartialHeaderRows + mt * 128);
+                bulk_commit();
+                bulk_wait_read<0>();                 // sP may be rewritten
+              }
+              softmax_sync256();
             }
+            if (st == 0) bulk_wait<0>();
           }
-        }
-      } else {
-        // final rows: o = O / (l + e^{z - m}), rope dims rotated back by -t
-        if (tid < kAttnH) {
-          const float z2 = p.sinks[tid] * kLog2e;
-          const float mu = m_use[tid];
-          const float M = fmaxf(mu, z2);
-          const float den = exp2f(z2 - M) + (mu == -INFINITY ? 0.f : l_run[tid] * exp2f(mu - M));
-          stat_a[tid] = (mu == -INFINITY) ? 0.f : exp2f(mu - M) / den;   // factor on O
-        }
-        if (tid < p.rope_dims / 2) {
-          float cs, sn;
-          rope_cos_sin(-(double)it.t, tid, p.rope_dims, p.rope_base, &cs, &sn);
-          rope_cs[tid] = cs;
-          rope_sn[tid] = sn;
-        }
-        named_sync128();
-        __nv_bfloat16* O = p.out + ((int64_t)it.b * p.nq + it.qi) * kAttnH * kAttnD;
-        __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sP);   // [64 heads][128 dims] bf16
-        const float4* fac4 = reinterpret_cast<const float4*>(stat_a);
+        } else {
+          // final rows: o = O / (l + e^{z - m}), rope dims rotated back by -t
+          __nv_bfloat16* O = p.out + ((int64_t)it.b * p.nq + it.qi) * kAttnH * kAttnD;
+          if (empty) {
+            // no key at all: only the sink is in the denominator, o = 0
+            for (int x = tid; x < 32 * kAttnD; x += 128) O[(int64_t)h0 * kAttnD + x] = __float2bfloat16_rn(0.f);
+          } else {
+            if (tid < 32) {
+              const int h = h0 + tid;
+              const float z2 = p.sinks[h] * kLog2e;
+              const float mu = m_use[h];
+              const float M = fmaxf(mu, z2);
+              const float den = exp2f(z2 - M) + (mu == -INFINITY ? 0.f : l_run[h] * exp2f(mu - M));
+              stat_a[h] = (mu == -INFINITY) ? 0.f : exp2f(mu - M) / den;   // factor on O
+            }
+            group_sync(gid);
+            __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sP) + g * 32 * 128;   // [32 heads][128 dims]
+            const float4* fac4 = reinterpret_cast<const float4*>(stat_a + h0);
 #pragma unroll 1
-        for (int mt = 0; mt < kAttnMT; ++mt) {
-          const int dim = mt * 128 + tid;
-          const bool mt_rope = mt * 128 + 127 >= r0;     // uniform over the CTA
-          const bool rot = dim >= r0;
-          const int j = rot ? (dim - r0) >> 1 : 0;
-          const float cs = rot ? rope_cs[j] : 1.f, sn = rot ? rope_sn[j] : 0.f;
+            for (int mt = 0; mt < kAttnMT; ++mt) {
+              const int dim = mt * 128 + tid;
+              const bool mt_rope = mt * 128 + 127 >= r0;     // uniform over the group
+              const bool rot = dim >= r0;
+              float cs = 1.f, sn = 0.f;
+              if (rot) rope_sincos(-(double)it.t, theta_s[(dim - r0) >> 1], &cs, &sn);
+              float o[32];
+              tmem_ld32(tO + lane_base + mt * kAttnH + h0, o);
+              tmem_wait_ld();
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            float v[32];
-            tmem_ld32(tO + lane_base + mt * kAttnH + half * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-              const float4 f = fac4[half * 8 + e4];
-              v[e4 * 4 + 0] *= f.x; v[e4 * 4 + 1] *= f.y; v[e4 * 4 + 2] *= f.z; v[e4 * 4 + 3] *= f.w;
-            }
-            if (mt_rope) {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const float partner = __shfl_xor_sync(0xffffffffu, v[e], 1);
-                if (rot) v[e] = (dim & 1) ? fmaf(partner, sn, v[e] * cs) : fmaf(-partner, sn, v[e] * cs);
+              for (int e4 = 0; e4 < 8; ++e4) {
+                const float4 f = fac4[e4];
+                o[e4 * 4 + 0] *= f.x; o[e4 * 4 + 1] *= f.y; o[e4 * 4 + 2] *= f.z; o[e4 * 4 + 3] *= f.w;
               }
+              if (mt_rope) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                  const float partner = __shfl_xor_sync(0xffffffffu, o[e], 1);
+                  if (rot) o[e] = (dim & 1) ? fmaf(partner, sn, o[e] * cs) : fmaf(-partner, sn, o[e] * cs);
+                }
+              }
+#pragma unroll
+              for (int e = 0; e < 32; ++e) stage[e * 128 + tid] = __float2bfloat16_rn(o[e]);
+              group_sync(gid);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int piece = tid + 128 * i;             // 16-byte piece: head = piece / 16
+                const int h = piece >> 4, off = (piece & 15) * 8;
+                const uint4 val = *reinterpret_cast<const uint4*>(stage + h * 128 + off);
+                *reinterpret_cast<uint4*>(O + (int64_t)(h0 + h) * kAttnD + mt * 128 + off) = val;
+              }
+              group_sync(gid);
             }
-#pragma unroll
-            for (int e = 0; e < 32; ++e) stage[(half * 32 + e) * 128 + tid] = __float2bfloat16_rn(v[e]);
           }
-          named_sync128();
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int piece = tid + 128 * i;             // 16-byte piece: head = piece / 16
-            const int h = piece >> 4, off = (piece & 15) * 8;
-            const uint4 val = *reinterpret_cast<const uint4*>(stage + h * 128 + off);
-            *reinterpret_cast<uint4*>(O + (int64_t)h * kAttnD + mt * 128 + off) = val;
-          }
-          named_sync128();
         }
       }
       tc_fence_before();
-      named_sync128();
+      if (softmax_any256(bad)) break;        // also: both groups are done with the item
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, 512);
+  if (warp == 10) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------------------
@@ -761,9 +839,24 @@ __global__ void __launch_bounds__(128) attn_combine_tc_kernel(TcCombineParams p)
   const int tid = threadIdx.x;
   // every split's m[H], l[H] into shared memory (independent loads in flight),
   // then the weights of head h = tid from there
-  for (int x = tid; x < p.splits * 2 * kAttnH; x += blockDim.x) {
-    const int sp = x / (2 * kAttnH), e = x % (2 * kAttnH);
-    wsplit[p.splits * kAttnH + x] = __ldcg(reinterpret_cast<const float*>(P0 + (int64_t)sp * kTcPartialBytes) + e);
+  {
+    // 8 independent loads in flight per thread
+    const int n = p.splits * 2 * kAttnH;
+    for (int base = tid; base < n; base += 8 * (int)blockDim.x) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int x = base + u * (int)blockDim.x;
+        v[u] = x < n ? __ldcg(reinterpret_cast<const float*>(P0 + (int64_t)(x / (2 * kAttnH)) * kTcPartialBytes) +
+                              x % (2 * kAttnH))
+                     : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int x = base + u * (int)blockDim.x;
+        if (x < n) wsplit[p.splits * kAttnH + x] = v[u];
+      }
+    }
   }
   __syncthreads();
   if (tid < kAttnH) {
@@ -788,22 +881,36 @@ __global__ void __launch_bounds__(128) attn_combine_tc_kernel(TcCombineParams p)
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-#pragma unroll 4
-  for (int s = 0; s < p.splits; ++s) {
-    const float4 w0 = *reinterpret_cast<const float4*>(wsplit + s * kAttnH + hg * 8);
-    const float4 w1 = *reinterpret_cast<const float4*>(wsplit + s * kAttnH + hg * 8 + 4);
-    if (w0.x == 0.f && w0.y == 0.f && w0.z == 0.f && w0.w == 0.f && w1.x == 0.f && w1.y == 0.f &&
-        w1.z == 0.f && w1.w == 0.f)
-      continue;                                            // empty split: O was not written
-    const uint4 raw = __ldcg(reinterpret_cast<const uint4*>(P0 + (int64_t)s * kTcPartialBytes + kTcPartialHeader +
-                                                           ((int64_t)dim * kAttnH + hg * 8) * 2));
-    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
-    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+  // splits in groups of 8: the group's loads are issued before its FMAs; an
+  // empty split (all weights 0) was not written and is not read
+  for (int s0 = 0; s0 < p.splits; s0 += 8) {
+    uint4 raw[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __half22float2(h2[i]);
-      acc[2 * i] = fmaf(wv[2 * i], f.x, acc[2 * i]);
-      acc[2 * i + 1] = fmaf(wv[2 * i + 1], f.y, acc[2 * i + 1]);
+    for (int u = 0; u < 8; ++u) {
+      const int s = s0 + u;
+      raw[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (s < p.splits) {
+        const float4 w0 = *reinterpret_cast<const float4*>(wsplit + s * kAttnH + hg * 8);
+        const float4 w1 = *reinterpret_cast<const float4*>(wsplit + s * kAttnH + hg * 8 + 4);
+        const bool live = w0.x != 0.f || w0.y != 0.f || w0.z != 0.f || w0.w != 0.f || w1.x != 0.f ||
+                          w1.y != 0.f || w1.z != 0.f || w1.w != 0.f;
+        if (live)
+          raw[u] = __ldcg(reinterpret_cast<const uint4*>(P0 + (int64_t)s * kTcPartialBytes + kTcPartialHeader +
+                                                         ((int64_t)dim * kAttnH + hg * 8) * 2));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int s = s0 + u;
+      if (s >= p.splits) break;
+      const float* w = wsplit + s * kAttnH + hg * 8;
+      const __half2* h2 = reinterpret_cast<const __half2*>(&raw[u]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h2[i]);
+        acc[2 * i] = fmaf(w[2 * i], f.x, acc[2 * i]);
+        acc[2 * i + 1] = fmaf(w[2 * i + 1], f.y, acc[2 * i + 1]);
+      }
     }
   }
   // rope dims: the pair partner (dim ^ 1) is thread tid ^ 8

@@ -80,19 +80,33 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // ---- RoPE -----------------------------------------------------------------------
-// Pair j of the last r dims at position pos rotates by pos * base^(-2j/r).  The
-// angle is formed and reduced in double so that positions up to 2^20 keep the
-// phase exact to fp32 rounding; cos/sin are returned in float.
-__device__ __forceinline__ void rope_cos_sin(double pos, int j, int r, double base,
-                                             float* c, float* s) {
-  double theta = pow(base, -2.0 * (double)j / (double)r);
-  double sn, cs;
-  sincos(pos * theta, &sn, &cs);
-  *c = (float)cs;
-  *s = (float)sn;
+// Pair j of the last r dims at position pos rotates by pos * theta_j,
+// theta_j = base^(-2j/r).  The angle pos * theta_j is formed in double (its
+// error is ~2^-53 of |angle|, about 1e-10 rad at pos = 2^20) and reduced to
+// [-pi, pi] by Cody-Waite reduction with 2*pi split into a double head and
+// tail, k = rint(angle / 2pi): r = (angle - k*hi) - k*lo, each step one fma.
+// cos/sin of the reduced float angle then come from sincosf (|r| <= pi).
+__device__ __forceinline__ double rope_theta(int j, int r, double base) {
+  return pow(base, -2.0 * (double)j / (double)r);
+}
+__device__ __forceinline__ void rope_sincos(double pos, double theta, float* c, float* s) {
+  const double kTwoPiHi = 6.283185307179586;           // 2*pi rounded to double
+  const double kTwoPiLo = 2.4492935982947064e-16;      // 2*pi - kTwoPiHi
+  const double x = pos * theta;
+  const double k = rint(x * (1.0 / kTwoPiHi));
+  const double red = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, x));
+  sincosf((float)red, s, c);
+}
+__device__ __forceinline__ void rope_cos_sin(double pos, int j, int r, double base, float* c, float* s) {
+  rope_sincos(pos, rope_theta(j, r, base), c, s);
 }
 
 __host__ __device__ __forceinline__ int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// L2 prefetch of `bytes` contiguous bytes (16-byte aligned address, multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 
 // ---- programmatic dependent launch --------------------------------------------
 // Every kernel of the library is launched so that it may start while the

@@ -269,7 +269,7 @@ TopkLargeLayout topk_large_layout(int64_t rows, int N, int k) {
   TopkLargeLayout L;
   size_t off = 0;
   L.hist = off; off += align_up((size_t)rows * kHistBins * 4, 256);
-  L.counters = off; off += align_up((size_t)rows * 4 * 4, 256);
+  L.counters = off; off += align_up((size_t)rows * kTopkCounters * 4, 256);
   L.above = off; off += align_up((size_t)rows * k * 4, 256);
   L.cand = off; off += align_up((size_t)rows * N * 8, 256);
   L.total = off;
@@ -291,11 +291,26 @@ size_t indexer_workspace(const csahca_indexer_args* a) {
   return w;
 }
 
+// Zeroes `bytes` (a multiple of 16, 16-byte aligned) of scratch in the stream.
+int launch_zero(char* ptr, size_t bytes, cudaStream_t s) {
+  const int64_t n16 = (int64_t)(bytes / 16);
+  if (n16 == 0) return CSAHCA_OK;
+  int64_t blocks = ceil_div64(n16, 256);
+  if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
+  {
+    CSAHCA_TRACE("zero_scratch", s);
+    launch_k(zero16_kernel, dim3((unsigned)blocks), dim3(256), 0, s, reinterpret_cast<uint4*>(ptr), n16);
+  }
+  CSAHCA_CHECK_LAUNCH();
+  return CSAHCA_OK;
+}
+
 // Top-k of `rows` score rows (row r at scores + r * stride, position q_pos[r]).
 // Long rows use the multi-CTA path; hist_ready means the indexer has already
 // zeroed the scratch and built the row histograms (pass 1) while scoring.
 int launch_topk(const csahca_indexer_args* a, const float* scores, int64_t stride, const int* q_pos, int* idx,
-                int rows, char* scratch, cudaStream_t s, bool hist_ready = false) {
+                int rows, char* scratch, cudaStream_t s, bool hist_ready = false,
+                const void* prefetch_base = nullptr, int64_t prefetch_row_bytes = 0) {
   if (!topk_uses_large(a)) {
     TopkParams tp;
     tp.scores = scores; tp.row_stride = stride; tp.q_pos = q_pos; tp.idx = idx;
@@ -322,10 +337,13 @@ int launch_topk(const csahca_indexer_args* a, const float* scores, int64_t strid
   tp.counters = reinterpret_cast<uint32_t*>(scratch + L.counters);
   tp.above = reinterpret_cast<int*>(scratch + L.above);
   tp.cand = reinterpret_cast<uint2*>(scratch + L.cand);
+  tp.thresh_ready = hist_ready ? 1 : 0;
+  tp.prefetch_base = static_cast<const char*>(prefetch_base);
+  tp.prefetch_row_bytes = prefetch_row_bytes;
   if (!hist_ready) {
-    if (cudaMemsetAsync(scratch + L.hist, 0, L.above - L.hist, s) != cudaSuccess) {
-      (void)cudaGetLastError();
-      return CSAHCA_ERR_LAUNCH;
+    {
+      const int st = launch_zero(scratch + L.hist, L.above - L.hist, s);
+      if (st != CSAHCA_OK) return st;
     }
     {
       CSAHCA_TRACE("topk_hist", s);
@@ -385,10 +403,12 @@ int launch_indexer_tc_t(const csahca_indexer_args* a, IdxTcParams p, cudaStream_
 
 // Tensor-core scores for queries [q0, q0 + qc) into scores (row stride N).
 int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* scores, int64_t stride,
-                      cudaStream_t s, uint32_t* hist = nullptr) {
+                      cudaStream_t s, uint32_t* hist = nullptr, uint32_t* counters = nullptr) {
   IdxTcParams p;
   memset(&p, 0, sizeof(p));
   p.hist = hist;
+  p.counters = counters;
+  p.k = a->k;
   p.w = a->w; p.kI_scale = a->kI_scale; p.q_pos = a->q_pos;
   p.scores = scores; p.score_row_stride = stride;
   p.B = a->B; p.nq = a->nq; p.HI = a->HI; p.N = a->N; p.m = a->m;
@@ -408,6 +428,7 @@ int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* score
       p.splits = 0;
       p.n_items = a->B * qc;
     }
+    p.items_per_row = p.splits > 0 ? p.splits : 1;
     using Cfg = IdxF8Cfg<64>;
     CUtensorMap kmap;
     if (!encode_2d(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->kI, (uint64_t)a->dI, (uint64_t)a->B * a->N, 128, 128,
@@ -436,7 +457,10 @@ int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* score
   return launch_indexer_tc_t<4, false>(a, p, s);
 }
 
-int run_indexer(const csahca_indexer_args* a, void* stream) {
+// prefetch_base / prefetch_row_bytes (internal, decode only): every selected
+// row of a long row's top-k is prefetched into L2 from that [B][N] table.
+int run_indexer(const csahca_indexer_args* a, void* stream, const void* prefetch_base = nullptr,
+                int64_t prefetch_row_bytes = 0) {
   int st = validate_indexer(a);
   if (st != CSAHCA_OK) return st;
   if (a->B == 0 || a->nq == 0) return CSAHCA_OK;
@@ -498,16 +522,16 @@ int run_indexer(const csahca_indexer_args* a, void* stream) {
     const bool fuse_hist = qc == a->nq && topk_uses_large(a) && indexer_tc_eligible(a) &&
                            a->k_dtype == CSAHCA_E4M3 && a->N <= kTopkLargeMaxN;
     uint32_t* hist = nullptr;
+    uint32_t* counters = nullptr;
     if (fuse_hist) {
       const TopkLargeLayout L = topk_large_layout((int64_t)a->B * qc, a->N, a->k);
-      if (cudaMemsetAsync(scratch + L.hist, 0, L.above - L.hist, s) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return CSAHCA_ERR_LAUNCH;
-      }
+      const int zst = launch_zero(scratch + L.hist, L.above - L.hist, s);
+      if (zst != CSAHCA_OK) return zst;
       hist = reinterpret_cast<uint32_t*>(scratch + L.hist);
+      counters = reinterpret_cast<uint32_t*>(scratch + L.counters);
     }
     if (indexer_tc_eligible(a)) {
-      int st2 = launch_indexer_tc(a, q0, qc, base, stride, s, hist);
+      int st2 = launch_indexer_tc(a, q0, qc, base, stride, s, hist, counters);
       if (st2 != CSAHCA_OK) return st2;
     } else if (a->N > 0) {
       if (a->k_dtype == CSAHCA_E4M3) {
@@ -523,7 +547,8 @@ int run_indexer(const csahca_indexer_args* a, void* stream) {
     // rows of this chunk: (b, q) -> b * qc + (q - q0); positions and outputs are
     // addressed per batch entry, so launch per b unless the chunk is the whole nq
     if (qc == a->nq) {
-      int st3 = launch_topk(a, base, stride, a->q_pos, a->idx, a->B * qc, scratch, s, fuse_hist);
+      int st3 = launch_topk(a, base, stride, a->q_pos, a->idx, a->B * qc, scratch, s, fuse_hist,
+                            a->nq == 1 ? prefetch_base : nullptr, prefetch_row_bytes);
       if (st3 != CSAHCA_OK) return st3;
     } else {
       for (int b = 0; b < a->B; ++b) {
@@ -607,13 +632,18 @@ int launch_attn_tc(const AttnTcParams& p, const void* kv_comp, int64_t comp_rows
   else m_win = m_rows;
   ok = ok && encode_2d(&m_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.q, kAttnD, (uint64_t)p.B * p.nq * kAttnH, 64,
                        kAttnH, CU_TENSOR_MAP_SWIZZLE_128B);
+  // decode partials as 128-byte fp16 rows, stored 128 rows (one O^T M-tile) per box
+  CUtensorMap m_part = m_rows;
+  if (p.decode)
+    ok = ok && encode_2d(&m_part, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.partial, kAttnH,
+                         (uint64_t)p.B * p.nq * p.splits * kTcPartialRows, kAttnH, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return CSAHCA_ERR_LAUNCH;
   const int smem = AttnSmem::TOTAL;
   cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   if (grid <= 0) return CSAHCA_OK;
   CSAHCA_TRACE(name, s);
-  launch_k(attn_tc_kernel, dim3(grid), dim3(kAttnTcThreads), smem, s, m_rows, m_gather, m_win, m_q, p);
+  launch_k(attn_tc_kernel, dim3(grid), dim3(kAttnTcThreads), smem, s, m_rows, m_gather, m_win, m_q, m_part, p);
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
 }

@@ -22,11 +22,12 @@
 // Heads whose largest |q| is below 2^-118 (s_h would leave the normal fp32
 // range) contribute nothing.
 //
-// Roles (352 threads): two epilogue groups of 4 warps (warps 0-3, 4-7) take
+// Roles (384 threads): two epilogue groups of 4 warps (warps 0-3, 4-7) take
 // alternate key tiles, so the ReLU / weighted-sum epilogue of one tile
 // overlaps the next; group 0 also writes the split query of each work item.
-// Warp 8 issues the TMA key loads (and copies the keys' row scales) into a
-// 10-stage ring; warps 9 and 10 issue the MMAs of alternate tiles (N = 2*HI,
+// Warps 8 and 11 issue the TMA key loads (and copy the keys' row scales) of
+// alternate tiles into a 10-stage ring; warps 9 and 10 issue the MMAs of
+// alternate tiles (N = 2*HI,
 // 4 MMAs of K = 32 per tile, descriptors precomputed so that each issue is one
 // add) into 4 TMEM accumulators; warp 9 owns TMEM.
 // Work items as in indexer_tc.cuh: decode = (sequence, range of key tiles),
@@ -35,14 +36,15 @@
 // With p.hist set, the epilogue also counts each written score into a
 // 2048-bin shared histogram of its order key's top 11 bits and adds it to the
 // row's global histogram at the end of each work item: pass 1 of the
-// multi-CTA top-k (topk_large.cuh), done while the scores are in registers.
+// multi-CTA top-k (topk_large.cuh), done while the scores are in registers;
+// the last item of a row then finds the row's threshold bin.
 #pragma once
 #include "indexer_tc.cuh"
 #include "topk_large.cuh"
 
 namespace csahca {
 
-constexpr int kIdxF8Threads = 352;
+constexpr int kIdxF8Threads = 384;
 constexpr int kIdxF8Stages = 10;
 constexpr int kIdxF8Acc = 4;
 
@@ -92,6 +94,44 @@ __device__ __forceinline__ bool epi_any256(bool v) {
   return r != 0;
 }
 
+// Last work item of a top-k row (counted after a fence): the row's histogram
+// is complete, so the 256 epilogue threads find its threshold bin T (fewer
+// than k keys in bins above T, at least k from T up) and store T and the
+// count above it for the select kernel.  All 256 threads call this.
+__device__ __forceinline__ void idx_row_done(const IdxTcParams& p, int row, uint32_t* scan, int* sh_flag) {
+  const int ept = threadIdx.x;
+  uint32_t* cnt = p.counters + (int64_t)row * kTopkCounters;
+  __threadfence();                                   // this item's histogram adds
+  epi_sync256();
+  if (ept == 0) *sh_flag = atomicAdd(&cnt[kCntItems], 1u) == (uint32_t)(p.items_per_row - 1);
+  epi_sync256();
+  if (!*sh_flag) return;
+  __threadfence();
+  const uint32_t* g = p.hist + (int64_t)row * kHistBins;
+  uint32_t c[8], tot = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) { c[e] = __ldcg(g + ept * 8 + e); tot += c[e]; }
+  uint32_t* a = scan;
+  uint32_t* b = scan + 256;
+  a[ept] = tot;
+  epi_sync256();
+  for (int off = 1; off < 256; off <<= 1) {          // inclusive suffix sums of the group totals
+    b[ept] = a[ept] + (ept + off < 256 ? a[ept + off] : 0u);
+    epi_sync256();
+    uint32_t* t = a; a = b; b = t;
+  }
+  uint32_t run = a[ept] - tot;                        // keys in groups above this one
+  const uint32_t k = (uint32_t)p.k;
+  if (run < k && run + tot >= k) {
+#pragma unroll
+    for (int e = 7; e >= 0; --e) {
+      if (run + c[e] >= k) { cnt[kCntT] = (uint32_t)(ept * 8 + e); cnt[kCntAboveT] = run; break; }
+      run += c[e];
+    }
+  }
+  epi_sync256();
+}
+
 template <int HI>
 __global__ void __launch_bounds__(kIdxF8Threads, 1)
 indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* __restrict__ qI, IdxTcParams p) {
@@ -109,6 +149,8 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
   __shared__ float sW[2][HI];                     // per group: w_h * s_h of its current item
   __shared__ uint32_t hist_s[kHistBins];          // this item's score histogram (p.hist set)
   __shared__ float sScale[NS][128];               // key row scales of each stage
+  __shared__ uint32_t scan_s[512];                // threshold search of a finished row
+  __shared__ int row_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -117,6 +159,7 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
     // scales (one cp.async arrive per producer lane) have landed; it is empty
     // once the MMAs have read the keys and the owning epilogue group the scales
     for (int s = 0; s < NS; ++s) { mbar_init(&bar_a_full[s], 1 + 32); mbar_init(&bar_a_empty[s], 1 + 128); }
+    // (the producer of tile i is warp 8 + (i & 1); its stage has that parity too)
     for (int j = 0; j < NACC; ++j) { mbar_init(&bar_acc_full[j], 1); mbar_init(&bar_acc_empty[j], 128); }
     mbar_init(&bar_b_full, 128);
     mbar_init(&bar_b_empty, 2);                    // both MMA issuers, once per item
@@ -131,10 +174,12 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
   griddep_launch_dependents();
   griddep_wait();                                  // keys may come from this stream's compress kernel
 
-  if (warp == 8) {
-    // ------------------------------------------------------------ producer
-    // lane 0: the key tile by TMA; all lanes: the tile's 128 row scales by
-    // cp.async (4 each, zero past the row's end)
+  if (warp == 8 || warp == 11) {
+    // ------------------------------------------------------------ producers
+    // warps 8 and 11 take alternate tiles; lane 0: the key tile by TMA; all
+    // lanes: the tile's 128 row scales by cp.async (4 each, zero past the
+    // row's end)
+    const uint32_t pe = warp == 8 ? 0u : 1u;
     if (lane == 0) tma_prefetch_desc(&kmap);
     uint32_t a_iter = 0;
     bool stop = false;                               // warp-uniform
@@ -142,6 +187,7 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
       const IdxItem it = idx_item<1>(p, id);
       const float* srow = p.kI_scale + (int64_t)it.b * p.N;
       for (int kt = it.kt0; kt < it.kt1; ++kt, ++a_iter) {
+        if ((a_iter & 1u) != pe) continue;
         const int s = a_iter % NS;
         const uint32_t ph = (a_iter / NS) & 1;
         int ok = 1;
@@ -163,11 +209,11 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
         cp_async_arrive_noinc(&bar_a_full[s]);
       }
     }
-    // drain: every issued fill has landed before the CTA may exit
+    // drain: every fill this warp issued has landed before the CTA may exit
     cp_async_wait<0>();
     if (lane == 0)
       for (uint32_t i = (a_iter > NS ? a_iter - NS : 0); i < a_iter; ++i)
-        mbar_wait(&bar_a_full[i % NS], (i / NS) & 1, &abort_flag);
+        if ((i & 1u) == pe) mbar_wait(&bar_a_full[i % NS], (i / NS) & 1, &abort_flag);
   } else if (warp == 9 || warp == 10) {
     // ------------------------------------------------------------ MMA issuers
     // issuer e takes the tiles of parity e (their stages and accumulators have
@@ -222,7 +268,11 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
     uint32_t acc_iter = 0, b_iter = 0;
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
       const IdxItem it = idx_item<1>(p, id);
-      if (it.kt1 <= it.kt0) continue;
+      const int row = it.b * p.q_count + (it.q0 - p.q_begin);
+      if (it.kt1 <= it.kt0) {
+        if (do_hist) idx_row_done(p, row, scan_s, &row_flag);   // an empty item still counts
+        continue;
+      }
       // `bad` is uniform over a group; a group that gives up skips the rest of
       // the item and both groups leave together at its end
       bool bad = false;
@@ -313,12 +363,12 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
       }
       if (epi_any256(bad)) break;                    // also: both groups are done with the item
       if (do_hist) {
-        uint32_t* gh = p.hist + ((int64_t)it.b * p.q_count + (it.q0 - p.q_begin)) * kHistBins;
+        uint32_t* gh = p.hist + (int64_t)row * kHistBins;
         for (int i = ept; i < kHistBins; i += 256) {
           const uint32_t c = hist_s[i];
           if (c) { atomicAdd(gh + i, c); hist_s[i] = 0; }
         }
-        epi_sync256();
+        idx_row_done(p, row, scan_s, &row_flag);
       }
     }
   }

@@ -33,6 +33,9 @@ struct IdxTcParams {
   int splits;                 // > 0: decode items (b, split); 0: prefill items (b, query tile)
   int tiles_per_split;
   uint32_t* hist;             // optional [rows][2048] score histograms (decode, e4m3 keys)
+  uint32_t* counters;         // with hist: [rows][8] top-k counters (threshold bin stored here)
+  int items_per_row;          // with hist: work items per row
+  int k;                      // with hist: the top-k size
 };
 
 template <int QT, int HI, bool kFP8>

@@ -13,10 +13,11 @@
 //                   bins above T are taken, bin T keys become candidates.  The
 //                   last CTA of a row to finish (atomic count after a fence)
 //                   then selects exactly: radix select of the remaining count
-//                   among the candidates (21 low bits), ties to the lower index
-//                   through a bitmap scan in index order, and the taken set
-//                   written in ascending index order through a second bitmap
-//                   scan.
+//                   among the candidates (21 low bits), then the selected set
+//                   in a bitmap of the row, read out in ascending index order
+//                   (one block prefix sum over per-thread word ranges); when
+//                   more keys tie at the threshold than are still to take, the
+//                   lowest-index ones through a bitmap scan in index order.
 #pragma once
 #include <limits.h>
 #include "topk.cuh"
@@ -24,6 +25,14 @@
 namespace csahca {
 
 constexpr int kHistBins = 2048;            // top 11 bits of the key
+// per-row counters of the multi-CTA top-k scratch
+constexpr int kTopkCounters = 8;
+constexpr int kCntAbove = 0;               // keys routed to the taken list
+constexpr int kCntCand = 1;                // keys routed to the candidate list
+constexpr int kCntSlices = 2;              // select CTAs done with the row
+constexpr int kCntItems = 3;               // indexer work items done with the row
+constexpr int kCntT = 4;                   // threshold bin (set by the indexer's last item)
+constexpr int kCntAboveT = 5;              // keys in bins above it
 constexpr int kHistShift = 21;
 constexpr int kTopkLargeMaxN = 786432;     // two bitmaps of N bits in shared memory
 
@@ -35,9 +44,15 @@ struct TopkLargeParams {
   int slices;                              // CTAs per row in passes 1 and 2
   // workspace (per row)
   uint32_t* hist;                          // [rows][kHistBins]
-  uint32_t* counters;                      // [rows][4]: n_above, n_cand, slices done
+  uint32_t* counters;                      // [rows][kTopkCounters]: see kCnt* below
+  int thresh_ready;                        // the indexer stored T and n_above_T in the counters
   int* above;                              // [rows][k]
   uint2* cand;                             // [rows][N]: (key, index)
+  // optional: row j of sequence `row` of a [rows][N] table of prefetch_row_bytes
+  // rows is prefetched into L2 for every selected j (decode: the KV rows the
+  // attention kernel gathers next)
+  const char* prefetch_base;
+  int64_t prefetch_row_bytes;
 };
 
 __device__ __forceinline__ int topk_visible(const TopkLargeParams& p, int row) {
@@ -45,6 +60,17 @@ __device__ __forceinline__ int topk_visible(const TopkLargeParams& p, int row) {
   if (t < 0) return 0;
   const int64_t v = ((int64_t)t + 1) / p.m;
   return (int)(v < p.N ? v : p.N);
+}
+
+// Zeroes n16 16-byte words of top-k scratch (histograms and counters).  A
+// kernel rather than a memset node, so that the stream's chain of
+// programmatic dependent launches is not broken; it writes only after the
+// previous kernel has completed.
+__global__ void __launch_bounds__(256) zero16_kernel(uint4* p, int64_t n16) {
+  griddep_launch_dependents();
+  griddep_wait();
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (int64_t)gridDim.x * blockDim.x)
+    p[i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 __global__ void __launch_bounds__(512) topk_hist_kernel(TopkLargeParams p) {
@@ -150,40 +176,15 @@ __device__ __forceinline__ int bitmap_scan(const uint32_t* bm, int words, int li
 
 constexpr int kTopkSelectThreads = 512;
 constexpr int kTopkCandCache = 4096;       // candidates staged in shared memory (8 bytes each)
-constexpr int kTopkSortCap = 2048;         // selected / tie indices sorted in shared memory
 
-__host__ __device__ __forceinline__ int next_pow2(int x) {
-  int n = 1;
-  while (n < x) n <<= 1;
-  return n;
-}
-
-// Dynamic shared memory of topk_select_kernel: the larger of the bitmap path
-// (two bitmaps of N bits) and the sort path (candidate cache, selected and
-// tie buffers).
+// Dynamic shared memory of topk_select_kernel: the larger of the tie path
+// (two bitmaps of N bits) and the common path (candidate cache, then one
+// bitmap of N bits).
 __host__ __device__ __forceinline__ int topk_select_smem_bytes(int N) {
-  const int bitmaps = 2 * ((N + 31) / 32) * 4;
-  const int sorted = kTopkCandCache * 8 + 2 * kTopkSortCap * 4;
-  return bitmaps > sorted ? bitmaps : sorted;
-}
-
-// Ascending bitonic sort of n (a power of two) ints in shared memory by the
-// whole block; ends with a barrier.
-__device__ __forceinline__ void bitonic_sort_smem(int* a, int n) {
-  for (int k2 = 2; k2 <= n; k2 <<= 1) {
-    for (int j = k2 >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const int x = a[i], y = a[ixj];
-          const bool up = (i & k2) == 0;
-          if ((x > y) == up) { a[i] = y; a[ixj] = x; }
-        }
-      }
-      __syncthreads();
-    }
-  }
-  __syncthreads();
+  const int words = (N + 31) / 32;
+  const int ties = 2 * words * 4;
+  const int common = kTopkCandCache * 8 + words * 4;
+  return ties > common ? ties : common;
 }
 
 // Routing of one slice (pass 2) and, in the last CTA of the row, the exact
@@ -195,7 +196,7 @@ __global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLar
   __shared__ uint32_t sh[1024];
   __shared__ uint32_t hist8[256];
   __shared__ int warp_buf[72];
-  __shared__ uint32_t sh_digit, sh_need, sh_eq, sh_nsel, sh_base_t, sh_base_c;
+  __shared__ uint32_t sh_digit, sh_need, sh_eq, sh_base_t, sh_base_c;
   __shared__ int sh_last;
   const int row = blockIdx.x / p.slices, slice = blockIdx.x % p.slices;
   const int v = topk_visible(p, row);
@@ -205,12 +206,18 @@ __global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLar
       for (int j = threadIdx.x; j < p.k; j += blockDim.x) out[j] = j < v ? j : -1;
     return;
   }
-  uint32_t* cnt = p.counters + (int64_t)row * 4;
+  uint32_t* cnt = p.counters + (int64_t)row * kTopkCounters;
   int* above = p.above + (int64_t)row * p.k;
   uint2* cand = p.cand + (int64_t)row * p.N;
   {
     uint32_t n_above_T;
-    const int T = threshold_bin(p.hist + (int64_t)row * kHistBins, p.k, sh, &n_above_T);
+    int T;
+    if (p.thresh_ready) {
+      T = (int)__ldcg(&cnt[kCntT]);
+      n_above_T = __ldcg(&cnt[kCntAboveT]);
+    } else {
+      T = threshold_bin(p.hist + (int64_t)row * kHistBins, p.k, sh, &n_above_T);
+    }
     const int per = (v + p.slices - 1) / p.slices;
     const int j0 = slice * per, j1 = min(v, j0 + per);
     const float* s = p.scores + (int64_t)row * p.row_stride;
@@ -232,8 +239,8 @@ __global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLar
       int tot;
       const int off = block_excl_count(nt | (nc << 16), warp_buf, &tot);
       if (threadIdx.x == 0) {
-        sh_base_t = atomicAdd(&cnt[0], (uint32_t)(tot & 0xFFFF));
-        sh_base_c = atomicAdd(&cnt[1], (uint32_t)(tot >> 16));
+        sh_base_t = atomicAdd(&cnt[kCntAbove], (uint32_t)(tot & 0xFFFF));
+        sh_base_c = atomicAdd(&cnt[kCntCand], (uint32_t)(tot >> 16));
       }
       __syncthreads();
       uint32_t pt = sh_base_t + (uint32_t)(off & 0xFFFF), pc = sh_base_c + (uint32_t)(off >> 16);
@@ -255,13 +262,13 @@ __global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLar
   // publish this slice, then let the last CTA of the row finish it
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) sh_last = atomicAdd(&cnt[2], 1u) == (uint32_t)(p.slices - 1);
+  if (threadIdx.x == 0) sh_last = atomicAdd(&cnt[kCntSlices], 1u) == (uint32_t)(p.slices - 1);
   __syncthreads();
   if (!sh_last) return;
   __threadfence();
 
-  const uint32_t n_above = min(__ldcg(&cnt[0]), (uint32_t)p.k);
-  const uint32_t n_cand = min(__ldcg(&cnt[1]), (uint32_t)p.N);
+  const uint32_t n_above = min(__ldcg(&cnt[kCntAbove]), (uint32_t)p.k);
+  const uint32_t n_cand = min(__ldcg(&cnt[kCntCand]), (uint32_t)p.N);
   // candidates staged in shared memory when they fit (the usual case), else
   // read from the scratch in every pass
   uint2* cand_s = reinterpret_cast<uint2*>(bm_sel);
@@ -298,7 +305,7 @@ __global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLar
   }
   need = sh_need;                              // keys equal to the threshold still to take
   // count the keys equal to the threshold
-  if (threadIdx.x == 0) { sh_eq = 0; sh_nsel = 0; }
+  if (threadIdx.x == 0) sh_eq = 0;
   __syncthreads();
   {
     uint32_t ne = 0;
@@ -310,44 +317,48 @@ __global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLar
   }
   __syncthreads();
   const uint32_t n_eq = sh_eq;
-  const int nsort = next_pow2(p.k);
-  if (nsort <= kTopkSortCap && (n_eq == need || n_eq <= (uint32_t)kTopkSortCap)) {
-    // ---- sort path: gather the k selected indices, then sort them ascending
-    int* sel = reinterpret_cast<int*>(bm_sel) + 2 * kTopkCandCache;   // after the candidate cache
-    int* ties = sel + kTopkSortCap;
-    for (uint32_t i = threadIdx.x; i < n_above; i += blockDim.x) sel[i] = __ldcg(above + i);
-    if (threadIdx.x == 0) sh_nsel = n_above;
+  if (n_eq == need) {
+    // ---- common path: every key equal to the threshold is taken.  The
+    // selected set goes into a v-bit bitmap (after the candidate cache); each
+    // thread then owns a contiguous range of words, and one block prefix sum
+    // of their popcounts places its indices: the output is in index order.
+    const int words = (v + 31) / 32;
+    uint32_t* bm = bm_sel + 2 * kTopkCandCache;
+    for (int i = threadIdx.x; i < words; i += blockDim.x) bm[i] = 0u;
     __syncthreads();
-    if (threadIdx.x == 0) sh_eq = 0;
-    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < n_above; i += blockDim.x) {
+      const int j = __ldcg(above + i);
+      atomicOr(&bm[j >> 5], 1u << (j & 31));
+    }
     for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
       const uint2 c = cand_local ? C[i] : __ldcg(cand + i);
-      const uint32_t low = c.x & ((1u << kHistShift) - 1u);
-      if (low > prefix) sel[atomicAdd(&sh_nsel, 1u)] = (int)c.y;
-      else if (low == prefix) {
-        if (n_eq == need) sel[atomicAdd(&sh_nsel, 1u)] = (int)c.y;   // every tie is taken
-        else ties[atomicAdd(&sh_eq, 1u)] = (int)c.y;
+      if ((c.x & ((1u << kHistShift) - 1u)) >= prefix) atomicOr(&bm[c.y >> 5], 1u << (c.y & 31));
+    }
+    __syncthreads();
+    const int wpt = (words + (int)blockDim.x - 1) / (int)blockDim.x;
+    const int w0 = (int)threadIdx.x * wpt, w1 = min(words, w0 + wpt);
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+    int tot;
+    int pos = block_excl_count(cnt, warp_buf, &tot);
+    for (int w = w0; w < w1; ++w) {
+      uint32_t bits = bm[w];
+      while (bits) {
+        const int j = w * 32 + __ffs(bits) - 1;
+        bits &= bits - 1u;
+        if (pos < p.k) {
+          out[pos] = j;
+          if (p.prefetch_base)
+            bulk_prefetch_l2(p.prefetch_base + ((int64_t)row * p.N + j) * p.prefetch_row_bytes,
+                             (uint32_t)p.prefetch_row_bytes);
+        }
+        ++pos;
       }
     }
-    __syncthreads();
-    if (n_eq != need) {
-      // the `need` lowest indices among the ties
-      const int nt = next_pow2((int)n_eq);
-      for (int i = (int)n_eq + threadIdx.x; i < nt; i += blockDim.x) ties[i] = INT_MAX;
-      __syncthreads();
-      bitonic_sort_smem(ties, nt);
-      const uint32_t base = sh_nsel;
-      for (uint32_t i = threadIdx.x; i < need; i += blockDim.x) sel[base + i] = ties[i];
-      __syncthreads();
-    }
-    for (int i = p.k + threadIdx.x; i < nsort; i += blockDim.x) sel[i] = INT_MAX;
-    __syncthreads();
-    bitonic_sort_smem(sel, nsort);
-    for (int i = threadIdx.x; i < p.k; i += blockDim.x) out[i] = sel[i];
     return;
   }
-  // ---- bitmap path (large k, or more ties than the sort buffers hold):
-  // index order through bitmaps of v bits
+  // ---- tie path (more keys equal to the threshold than still to take):
+  // the lowest-index ties through a bitmap scan in index order
   __syncthreads();
   const int words = (v + 31) / 32;
   uint32_t* bm_eq = bm_sel + words;
@@ -368,7 +379,11 @@ __global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLar
   bitmap_scan(bm_eq, words, (int)need, warp_buf,
               [&](int, int j) { atomicOr(&bm_sel[j >> 5], 1u << (j & 31)); });
   __syncthreads();
-  bitmap_scan(bm_sel, words, p.k, warp_buf, [&](int pos, int j) { out[pos] = j; });
+  bitmap_scan(bm_sel, words, p.k, warp_buf, [&](int pos, int j) {
+    out[pos] = j;
+    if (p.prefetch_base) bulk_prefetch_l2(p.prefetch_base + ((int64_t)row * p.N + j) * p.prefetch_row_bytes,
+                                          (uint32_t)p.prefetch_row_bytes);
+  });
 }
 
 }  // namespace csahca
