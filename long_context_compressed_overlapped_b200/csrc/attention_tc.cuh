@@ -49,6 +49,7 @@ struct AttnTcParams {
   const int* idx;               // [B, nq, k]
   int decode;                   // window = ring [B, w, d] (decode) or finished rows [B, nq, d]
   int n_items, splits, tiles_per_split;
+  int gtile;                    // CSA: selected rows per tile (128, 64 or 32); rows gtile..127 stay zero
   __nv_bfloat16* out;           // final [B, nq, H, D]
   float* partial;               // [B, nq, H, splits, D + 4]
 };
@@ -74,8 +75,7 @@ __device__ __forceinline__ AttnItem attn_item(const AttnTcParams& p, int id) {
   it.b = qid / p.nq;
   it.qi = qid % p.nq;
   it.t = p.decode ? p.pos[it.b] : it.qi;
-  const int ncomp = p.csa ? p.k : attn_visible(p, it.t);
-  it.ncomp_tiles = (ncomp + 127) / 128;
+  it.ncomp_tiles = p.csa ? (p.k + p.gtile - 1) / p.gtile : (attn_visible(p, it.t) + 127) / 128;
   it.nwin_tiles = (p.w + 127) / 128;
   const int total = it.ncomp_tiles + it.nwin_tiles;
   if (p.decode) {
@@ -93,10 +93,10 @@ __device__ __forceinline__ AttnTile attn_tile(const AttnTcParams& p, const AttnI
   if (tile < it.ncomp_tiles) {
     if (p.csa) {
       T.src = 0;
-      T.list_off = tile * 128;
+      T.list_off = tile * p.gtile;
       T.row0 = 0;
       T.lo = 0;
-      T.hi = min(128, p.k - tile * 128);
+      T.hi = min(p.gtile, p.k - T.list_off);
     } else {
       T.src = 1;
       T.row0 = it.b * p.N + tile * 128;
@@ -214,9 +214,9 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 }
 
 __global__ void __launch_bounds__(kAttnTcThreads, 1)
-attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_constant__ CUtensorMap comp_gather,
-               const __grid_constant__ CUtensorMap win_rows, const __grid_constant__ CUtensorMap q_rows,
-               const __grid_constant__ CUtensorMap part_rows, AttnTcParams p) {
+attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_constant__ CUtensorMap win_rows,
+               const __grid_constant__ CUtensorMap q_rows, const __grid_constant__ CUtensorMap part_rows,
+               AttnTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
@@ -254,6 +254,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     mbar_fence_init();
   }
   if (warp == 10) tmem_alloc(&tmem_base_sh, 512);
+  if (p.gtile < 128) {
+    // rows [gtile, 128) of the key buffer are never written by a gathered
+    // tile; zeros there keep the score and P.V MMAs finite (P = 0 there)
+    const int per_chunk = (128 - p.gtile) * 8;     // 16-byte pieces
+    for (int x = threadIdx.x; x < kAttnChunks * per_chunk; x += blockDim.x) {
+      const int c = x / per_chunk, o = x - c * per_chunk;
+      *reinterpret_cast<uint4*>(sK + c * AttnSmem::K_CHUNK + p.gtile * 128 + o * 16) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -268,7 +278,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     // warp 8 loads chunks 0,1,4,5 (and the raw Q); warp 9 chunks 2,3,6,7
     const int pw = warp - 8;
     tma_prefetch_desc(&comp_rows);
-    tma_prefetch_desc(&comp_gather);
     tma_prefetch_desc(&win_rows);
     tma_prefetch_desc(&q_rows);
     uint32_t tcount = 0, icount = 0;
@@ -284,9 +293,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
           ok = mbar_wait(&bar_q_empty, (icount & 1) ^ 1, &abort_flag);
           if (ok) {
             mbar_expect_tx(&bar_q_raw, AttnSmem::Q_BYTES);
-            const int qrow = (it.b * p.nq + it.qi) * kAttnH;
-            for (int c = 0; c < kAttnChunks; ++c)
-              tma_load_2d(sQ + c * AttnSmem::Q_CHUNK, &q_rows, c * 64, qrow, &bar_q_raw);
+            tma_load_3d(sQ, &q_rows, 0, (it.b * p.nq + it.qi) * kAttnH, 0, &bar_q_raw);
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -315,7 +322,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
               }
             }
           } else if (lane < kAttnChunks && Tn.row0 >= 0) {
-            tma_prefetch_l2_2d(Tn.src == 1 ? &comp_rows : &win_rows, lane * 64, Tn.row0);
+            tma_prefetch_l2_3d(Tn.src == 1 ? &comp_rows : &win_rows, 0, Tn.row0, lane);
           }
         }
         if (T.src == 0) {
@@ -339,21 +346,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
           uint8_t* dst = sK + c * AttnSmem::K_CHUNK;
           if (T.src == 0) {
             // gathered rows: 8 lanes per 128-byte row segment (coalesced,
-            // conflict-free), 4 rows per instruction, 32 instructions per
-            // chunk; each lane arrives on the chunk's barrier when its copies
-            // have landed, without waiting for them
+            // conflict-free), 4 rows per instruction, gtile / 4 instructions
+            // per chunk; each lane arrives on the chunk's barrier when its
+            // copies have landed, without waiting for them
             const int piece = lane & 7, rg = lane >> 3;
             const __nv_bfloat16* src = p.kv_comp_ptr + c * 64 + piece * 8;
+            const int nj = p.gtile >> 2;
 #pragma unroll 8
-            for (int j = 0; j < 32; ++j) {
+            for (int j = 0; j < nj; ++j) {
               const int r = 4 * j + rg;
               cp_async16(dst + sw128_offset(r, piece * 16), src + (int64_t)rows_s[pw][r] * kAttnD);
             }
             cp_async_arrive_noinc(&bar_kfull[c]);
           } else {
+            // contiguous rows: one 16 KB box per chunk, so the score MMAs of
+            // a chunk start as soon as it lands
             if (lane == 0) {
               mbar_expect_tx(&bar_kfull[c], AttnSmem::K_CHUNK);
-              tma_load_2d(dst, T.src == 1 ? &comp_rows : &win_rows, c * 64, T.row0, &bar_kfull[c]);
+              tma_load_3d(dst, T.src == 1 ? &comp_rows : &win_rows, 0, T.row0, c, &bar_kfull[c]);
             } else {
               mbar_arrive(&bar_kfull[c]);
             }
@@ -364,8 +374,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     // drain the last loads before the CTA may exit
     cp_async_wait<0>();
     if (lane == 0 && tcount > 0)
-      for (int cc = 0; cc < kAttnChunks / 2; ++cc)
-        mbar_wait(&bar_kfull[4 * (cc >> 1) + 2 * pw + (cc & 1)], (tcount - 1) & 1, &abort_flag);
+      for (int c = 0; c < kAttnChunks; ++c) mbar_wait(&bar_kfull[c], (tcount - 1) & 1, &abort_flag);
     if (pw == 0 && lane == 0 && icount > 0) mbar_wait(&bar_q_raw, (icount - 1) & 1, &abort_flag);
   } else if (warp == 10) {
     // ------------------------------------------------------------ S MMA issuer
@@ -418,11 +427,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
           if (!mbar_wait(&bar_p_full, ph, &abort_flag)) { stop = true; break; }
           tc_fence_after();
           const bool first = tile == it.tile0;
+          // key steps past the tile's last valid row hold P = 0 and are skipped
+          const int hi = attn_tile(p, it, tile).hi;
+          const int nks = hi <= 16 ? 1 : min(8, (hi + 15) >> 4);
+          // M-tile by M-tile, so that chunk pair (2 mt, 2 mt + 1) is released
+          // for the next tile's loads as soon as its MMAs complete
 #pragma unroll
           for (int mt = 0; mt < kAttnMT; ++mt) {
             const uint64_t vd = vdesc + (uint64_t)((2 * mt) * (AttnSmem::K_CHUNK >> 4));
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
+            for (int ks = 0; ks < nks; ++ks)
               umma_bf16(tO + mt * kAttnH, vd + 128 * ks, pdesc + 128 * ks, idesc_pv, !(first && ks == 0));
             umma_commit(&bar_kempty[2 * mt]);
             umma_commit(&bar_kempty[2 * mt + 1]);
@@ -715,8 +728,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
             // pieces 4g..4g+3 of row tid) and stored by one TMA box
             const float4* f4 = reinterpret_cast<const float4*>(stat_a + h0);
             const int blk = ((it.b * p.nq + it.qi) * p.splits + it.split);
+            // a CTA with a single item stages all four M-tiles in the key
+            // buffer (its last P.V has completed and no further keys come),
+            // so the four stores go out back to back
+            const bool own_k = p.n_items <= (int)gridDim.x;
 #pragma unroll 1
             for (int mt = 0; mt < kAttnMT; ++mt) {
+              uint8_t* stg = own_k ? sK + mt * AttnSmem::K_CHUNK : sP;
               float o[32];
               tmem_ld32(tO + lane_base + mt * kAttnH + h0, o);
               tmem_wait_ld();
@@ -732,18 +750,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
                 w.y = pack_half2(o[8 * q + 2], o[8 * q + 3]);
                 w.z = pack_half2(o[8 * q + 4], o[8 * q + 5]);
                 w.w = pack_half2(o[8 * q + 6], o[8 * q + 7]);
-                *reinterpret_cast<uint4*>(sP + sw128_offset(tid, (4 * g + q) * 16)) = w;
+                *reinterpret_cast<uint4*>(stg + sw128_offset(tid, (4 * g + q) * 16)) = w;
               }
               fence_proxy_async_smem();
               softmax_sync256();
               if (st == 0) {
-                tma_store_2d(&part_rows, sP, 0, blk * kTcPartialRows + kTcPartialHeaderRows + mt * 128);
+                tma_store_2d(&part_rows, stg, 0, blk * kTcPartialRows + kTcPartialHeaderRows + mt * 128);
                 bulk_commit();
-                bulk_wait_read<0>();                 // sP may be rewritten
+                if (!own_k) bulk_wait_read<0>();     // sP may be rewritten
               }
-              softmax_sync256();
+              if (!own_k) softmax_sync256();
             }
-            if (st == 0) bulk_wait<0>();
+            if (st == 0) bulk_wait_read<0>();       // the stores complete before the grid does
           }
         } else {
           // final rows: o = O / (l + e^{z - m}), rope dims rotated back by -t
@@ -814,11 +832,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
 // Split-KV combine of the tensor-core decode partials, with the sink and the
 // output de-rotation: o = sum_s f_s (O_s / l_s), f_s = l_s 2^(m_s - M) / den,
 // den = 2^(z_h log2 e - M) + sum_s l_s 2^(m_s - M), M the largest of them; the
-// rope dims of o are then rotated by -t.  One CTA per (query, 16 dims): thread
-// (dim dl = tid / 8, heads 8 * (tid % 8) ..) reads 16 contiguous bytes of
-// every split; the split weights of the 64 heads are formed once in shared
-// memory (dynamic: splits x 3 x 64 floats, the weights and the staged m, l
-// headers).
+// rope dims of o are then rotated by -t.  One CTA per (query, 16 dims).  The
+// m, l headers of every split and the 16-dim slices (16 x 64 fp16 per split)
+// reach shared memory by two TMA boxes, so the kernel pays about one memory
+// latency, not one per split.  With more splits than slice slots the slices
+// go in rounds.
+constexpr int kTcCombineMaxSplits = 160;
+constexpr int kTcCombineSlots = 64;
+constexpr int kTcCombineDims = 16;
+constexpr int kTcCombineSlice = kTcCombineDims * kAttnH * 2;
+
 struct TcCombineParams {
   const char* partial;        // [B * nq][splits] blocks of kTcPartialBytes
   const float* sinks;         // [H]
@@ -828,91 +851,121 @@ struct TcCombineParams {
   double rope_base;
 };
 
-__global__ void __launch_bounds__(128) attn_combine_tc_kernel(TcCombineParams p) {
+// dynamic shared memory of the combine: headers of all splits + slice slots
+__host__ __device__ inline int tc_combine_smem_bytes(int splits) {
+  const int slots = splits < kTcCombineSlots ? splits : kTcCombineSlots;
+  return splits * kTcPartialHeader + slots * kTcCombineSlice;
+}
+
+// hdr_map: the partials as [blocks][516 rows][64 fp16], box [splits][4][64]
+// (the m, l headers of all splits of one query); slc_map: the same tensor,
+// box [min(splits, 64)][16][64] (16 dims of up to 64 splits).  A bulk copy per
+// split was measured to complete one copy at a time; a box covering every
+// split goes out as one transfer.
+__global__ void __launch_bounds__(128) attn_combine_tc_kernel(const __grid_constant__ CUtensorMap hdr_map,
+                                                              const __grid_constant__ CUtensorMap slc_map,
+                                                              TcCombineParams p) {
+  extern __shared__ __align__(128) uint8_t cmb_smem[];
+  __shared__ uint64_t bar_hdr, bar_slc;
+  __shared__ float red[2][kAttnH];
+  __shared__ float inv_s[kAttnH];
+  __shared__ __align__(16) __nv_bfloat16 ostage[kAttnH][kTcCombineDims];
+  __shared__ volatile int abort_flag;
+  constexpr int kChunks = kAttnD / kTcCombineDims;
+  float* hdr = reinterpret_cast<float*>(cmb_smem);              // [splits][m[H], l[H]]; m slots -> weights
+  uint8_t* slots = cmb_smem + p.splits * kTcPartialHeader;        // [slots][16 dims][H] fp16
+  const int nslots = p.splits < kTcCombineSlots ? p.splits : kTcCombineSlots;
+  const int row = blockIdx.x / kChunks, dc = blockIdx.x % kChunks;
+  const int blk0 = row * p.splits, srow = kTcPartialHeaderRows + dc * kTcCombineDims;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    abort_flag = 0;
+    mbar_init(&bar_hdr, 1);
+    mbar_init(&bar_slc, 1);
+    mbar_fence_init();
+    tma_prefetch_desc(&hdr_map);
+    tma_prefetch_desc(&slc_map);
+  }
+  __syncthreads();
   griddep_launch_dependents();
   griddep_wait();
-  extern __shared__ float wsplit[];                       // [splits][H]
-  __shared__ __align__(16) __nv_bfloat16 ostage[kAttnH][16];
-  constexpr int kChunks = kAttnD / 16;
-  const int row = blockIdx.x / kChunks, dc = blockIdx.x % kChunks;
-  const char* P0 = p.partial + (int64_t)row * p.splits * kTcPartialBytes;
-  const int tid = threadIdx.x;
-  // every split's m[H], l[H] into shared memory (independent loads in flight),
-  // then the weights of head h = tid from there
-  {
-    // 8 independent loads in flight per thread
-    const int n = p.splits * 2 * kAttnH;
-    for (int base = tid; base < n; base += 8 * (int)blockDim.x) {
-      float v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int x = base + u * (int)blockDim.x;
-        v[u] = x < n ? __ldcg(reinterpret_cast<const float*>(P0 + (int64_t)(x / (2 * kAttnH)) * kTcPartialBytes) +
-                              x % (2 * kAttnH))
-                     : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int x = base + u * (int)blockDim.x;
-        if (x < n) wsplit[p.splits * kAttnH + x] = v[u];
-      }
-    }
+  if (tid == 0) {
+    mbar_expect_tx(&bar_hdr, (uint32_t)(p.splits * kTcPartialHeader));
+    tma_load_3d(hdr, &hdr_map, 0, 0, blk0, &bar_hdr);
+    // a last round shorter than the box reads past this query's splits (or
+    // zero fill past the tensor); those slots are not used
+    mbar_expect_tx(&bar_slc, (uint32_t)(nslots * kTcCombineSlice));
+    tma_load_3d(slots, &slc_map, 0, srow, blk0, &bar_slc);
   }
+  // split weights: thread (head h, half) takes the splits of its parity
+  const int h = tid & (kAttnH - 1), half = tid >> 6;
+  bool ok = mbar_wait(&bar_hdr, 0, &abort_flag);
+  const float z2 = p.sinks[h] * kLog2e;
+  float mx = -INFINITY;
+  if (ok) {
+#pragma unroll 4
+    for (int s = half; s < p.splits; s += 2) mx = fmaxf(mx, hdr[s * 2 * kAttnH + h]);
+  }
+  red[half][h] = mx;
   __syncthreads();
-  if (tid < kAttnH) {
-    const int h = tid;
-    const float* hs = wsplit + p.splits * kAttnH;          // [splits][m[H], l[H]]
-    const float z2 = p.sinks[h] * kLog2e;
-    float M = z2;
-    for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, hs[sp * 2 * kAttnH + h]);
-    float den = exp2f(z2 - M);
-    for (int sp = 0; sp < p.splits; ++sp) {
-      const float ms = hs[sp * 2 * kAttnH + h];
-      const float f = ms == -INFINITY ? 0.f : hs[sp * 2 * kAttnH + kAttnH + h] * exp2f(ms - M);
-      wsplit[sp * kAttnH + h] = f;
+  const float M = fmaxf(z2, fmaxf(red[0][h], red[1][h]));
+  float den = 0.f;
+  if (ok)
+#pragma unroll 4
+    for (int s = half; s < p.splits; s += 2) {
+      const float ms = hdr[s * 2 * kAttnH + h];
+      const float f = ms == -INFINITY ? 0.f : hdr[s * 2 * kAttnH + kAttnH + h] * exp2f(ms - M);
+      hdr[s * 2 * kAttnH + h] = f;
       den += f;
     }
-    const float inv = 1.f / den;
-    for (int sp = 0; sp < p.splits; ++sp) wsplit[sp * kAttnH + h] *= inv;
-  }
+  __syncthreads();                                 // every read of red[] (M) is done
+  red[half][h] = den;
   __syncthreads();
+  if (half == 0) inv_s[h] = 1.f / (exp2f(z2 - M) + red[0][h] + red[1][h]);
+  __syncthreads();
+  // weighted sum over the splits: thread (dim dl, heads 8 hg ..)
   const int dl = tid >> 3, hg = tid & 7;
-  const int dim = dc * 16 + dl;
+  const int dim = dc * kTcCombineDims + dl;
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  // splits in groups of 8: the group's loads are issued before its FMAs; an
-  // empty split (all weights 0) was not written and is not read
-  for (int s0 = 0; s0 < p.splits; s0 += 8) {
-    uint4 raw[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int s = s0 + u;
-      raw[u] = make_uint4(0u, 0u, 0u, 0u);
-      if (s < p.splits) {
-        const float4 w0 = *reinterpret_cast<const float4*>(wsplit + s * kAttnH + hg * 8);
-        const float4 w1 = *reinterpret_cast<const float4*>(wsplit + s * kAttnH + hg * 8 + 4);
-        const bool live = w0.x != 0.f || w0.y != 0.f || w0.z != 0.f || w0.w != 0.f || w1.x != 0.f ||
-                          w1.y != 0.f || w1.z != 0.f || w1.w != 0.f;
-        if (live)
-          raw[u] = __ldcg(reinterpret_cast<const uint4*>(P0 + (int64_t)s * kTcPartialBytes + kTcPartialHeader +
-                                                         ((int64_t)dim * kAttnH + hg * 8) * 2));
+  for (int s0 = 0, round = 0; s0 < p.splits; s0 += nslots, ++round) {
+    if (round > 0) {
+      __syncthreads();                             // every slot of the last round is consumed
+      if (tid == 0) {
+        mbar_expect_tx(&bar_slc, (uint32_t)(nslots * kTcCombineSlice));
+        tma_load_3d(slots, &slc_map, 0, srow, blk0 + s0, &bar_slc);
       }
     }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int s = s0 + u;
-      if (s >= p.splits) break;
-      const float* w = wsplit + s * kAttnH + hg * 8;
-      const __half2* h2 = reinterpret_cast<const __half2*>(&raw[u]);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __half22float2(h2[i]);
-        acc[2 * i] = fmaf(w[2 * i], f.x, acc[2 * i]);
-        acc[2 * i + 1] = fmaf(w[2 * i + 1], f.y, acc[2 * i + 1]);
+    // a timed-out wait leaves ok false; the loop still runs to the end so
+    // that every thread reaches the same barriers
+    ok = mbar_wait(&bar_slc, round & 1, &abort_flag) && ok;
+    if (ok) {
+      const int n = min(p.splits, s0 + nslots) - s0;
+      const float* wb = hdr + s0 * 2 * kAttnH + hg * 8;
+      const uint8_t* sb = slots + dl * (kAttnH * 2) + hg * 16;
+#pragma unroll 4
+      for (int i = 0; i < n; ++i) {
+        const float4 w0 = *reinterpret_cast<const float4*>(wb + i * 2 * kAttnH);
+        const float4 w1 = *reinterpret_cast<const float4*>(wb + i * 2 * kAttnH + 4);
+        uint4 raw = *reinterpret_cast<const uint4*>(sb + i * kTcCombineSlice);
+        // an empty split (all weights 0) has a header but no written slice
+        const bool live = (w0.x != 0.f) | (w0.y != 0.f) | (w0.z != 0.f) | (w0.w != 0.f) | (w1.x != 0.f) |
+                          (w1.y != 0.f) | (w1.z != 0.f) | (w1.w != 0.f);
+        raw.x = live ? raw.x : 0u; raw.y = live ? raw.y : 0u; raw.z = live ? raw.z : 0u; raw.w = live ? raw.w : 0u;
+        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+        const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&raw.z));
+        const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&raw.w));
+        acc[0] = fmaf(w0.x, f0.x, acc[0]); acc[1] = fmaf(w0.y, f0.y, acc[1]);
+        acc[2] = fmaf(w0.z, f1.x, acc[2]); acc[3] = fmaf(w0.w, f1.y, acc[3]);
+        acc[4] = fmaf(w1.x, f2.x, acc[4]); acc[5] = fmaf(w1.y, f2.y, acc[5]);
+        acc[6] = fmaf(w1.z, f3.x, acc[6]); acc[7] = fmaf(w1.w, f3.y, acc[7]);
       }
     }
   }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] *= inv_s[hg * 8 + i];
   // rope dims: the pair partner (dim ^ 1) is thread tid ^ 8
   const int r0 = kAttnD - p.rope_dims;
   float partner[8];
@@ -927,11 +980,12 @@ __global__ void __launch_bounds__(128) attn_combine_tc_kernel(TcCombineParams p)
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) ostage[hg * 8 + i][dl] = __float2bfloat16_rn(acc[i]);
-  __syncthreads();
+  ok = __syncthreads_and(ok);
+  if (!ok) return;
   {
-    const int h = tid >> 1, piece = tid & 1;
-    *reinterpret_cast<uint4*>(p.out + ((int64_t)row * kAttnH + h) * kAttnD + dc * 16 + piece * 8) =
-        *reinterpret_cast<const uint4*>(&ostage[h][piece * 8]);
+    const int hh = tid >> 1, piece = tid & 1;
+    *reinterpret_cast<uint4*>(p.out + ((int64_t)row * kAttnH + hh) * kAttnD + dc * kTcCombineDims + piece * 8) =
+        *reinterpret_cast<const uint4*>(&ostage[hh][piece * 8]);
   }
 }
 

@@ -147,6 +147,22 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const v
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D tensor [d2][d1][d0] of `dt` with byte strides s1 (between d1 rows) and
+// s2 (between d2 blocks), box [b2][b1][b0], no swizzle.
+bool encode_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+               uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2,
+               CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_NONE) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d0, (cuuint64_t)d1, (cuuint64_t)d2};
+  cuuint64_t strides[2] = {(cuuint64_t)s1, (cuuint64_t)s2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int dtype_size(int dt) {
   switch (dt) {
     case CSAHCA_F32: return 4;
@@ -622,16 +638,18 @@ bool attn_tc_shape_ok(int dtype, int H, int d, int rope_dims, int64_t comp_rows,
 
 int launch_attn_tc(const AttnTcParams& p, const void* kv_comp, int64_t comp_rows, const void* win,
                    int64_t win_rows, cudaStream_t s, const char* name) {
-  CUtensorMap m_rows, m_gather, m_win, m_q;
-  bool ok = encode_2d(&m_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv_comp, kAttnD, (uint64_t)comp_rows, 64, 128,
-                      CU_TENSOR_MAP_SWIZZLE_128B) &&
-            encode_2d(&m_gather, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv_comp, kAttnD, (uint64_t)comp_rows, 64, 1,
-                      CU_TENSOR_MAP_SWIZZLE_128B);
-  if (win) ok = ok && encode_2d(&m_win, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, win, kAttnD, (uint64_t)win_rows, 64,
-                                128, CU_TENSOR_MAP_SWIZZLE_128B);
+  // rows of d = 512 bf16 seen as [chunk 8][row][64]: a key box is one chunk
+  // of 128 rows (16 KB); the query box is all 8 chunks x 64 heads (64 KB),
+  // landing chunk-major with the 128-byte swizzle as the MMA operand wants it
+  CUtensorMap m_rows, m_win, m_q;
+  const uint64_t rs = kAttnD * 2;
+  bool ok = encode_3d(&m_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv_comp, 64, (uint64_t)comp_rows, kAttnChunks, rs,
+                      128, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (win) ok = ok && encode_3d(&m_win, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, win, 64, (uint64_t)win_rows, kAttnChunks,
+                                rs, 128, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B);
   else m_win = m_rows;
-  ok = ok && encode_2d(&m_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.q, kAttnD, (uint64_t)p.B * p.nq * kAttnH, 64,
-                       kAttnH, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && encode_3d(&m_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.q, 64, (uint64_t)p.B * p.nq * kAttnH, kAttnChunks,
+                       rs, 128, 64, kAttnH, kAttnChunks, CU_TENSOR_MAP_SWIZZLE_128B);
   // decode partials as 128-byte fp16 rows, stored 128 rows (one O^T M-tile) per box
   CUtensorMap m_part = m_rows;
   if (p.decode)
@@ -643,7 +661,7 @@ int launch_attn_tc(const AttnTcParams& p, const void* kv_comp, int64_t comp_rows
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   if (grid <= 0) return CSAHCA_OK;
   CSAHCA_TRACE(name, s);
-  launch_k(attn_tc_kernel, dim3(grid), dim3(kAttnTcThreads), smem, s, m_rows, m_gather, m_win, m_q, m_part, p);
+  launch_k(attn_tc_kernel, dim3(grid), dim3(kAttnTcThreads), smem, s, m_rows, m_win, m_q, m_part, p);
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
 }
@@ -668,7 +686,7 @@ int run_prefill_t(const csahca_attn_args* a, cudaStream_t s) {
     t.q_norm = a->q_norm; t.eps = eps; t.scale_log2 = scale * kLog2e; t.rope_dims = a->rope_dims;
     t.rope_base = base; t.B = a->B; t.nq = a->n; t.N = a->N; t.m = a->m; t.k = a->k; t.w = a->w;
     t.csa = a->kind == CSAHCA_CSA; t.idx = a->idx; t.decode = 0;
-    t.n_items = a->B * a->n; t.splits = 1; t.tiles_per_split = 0;
+    t.n_items = a->B * a->n; t.splits = 1; t.tiles_per_split = 0; t.gtile = 128;
     t.out = static_cast<__nv_bfloat16*>(a->out); t.partial = nullptr;
     return launch_attn_tc(t, a->kv_comp, (int64_t)a->B * a->N, win_final, (int64_t)a->B * a->n, s,
                           a->kind == CSAHCA_CSA ? "attn_prefill_csa_tc" : "attn_prefill_hca_tc");
@@ -743,6 +761,7 @@ struct DecodeLayout {
   int splits;
   bool tc;
   int tiles_per_split;
+  int gtile;                    // gathered rows per CSA tile
 };
 
 bool decode_tc(const csahca_decode_args* a) {
@@ -756,10 +775,16 @@ DecodeLayout decode_layout(const csahca_decode_args* a) {
   const int64_t jmax = (csa ? (int64_t)a->k : (int64_t)a->N_cap) + a->w;
   L.tc = decode_tc(a);
   L.tiles_per_split = 0;
+  L.gtile = 128;
   if (L.tc) {
-    // tensor-core path: split each query's tiles so that B x splits ~ one wave
-    const int tiles = (int)(ceil_div64(csa ? a->k : a->N_cap, 128) + ceil_div64(a->w, 128));
-    int want = (int)ceil_div64(num_sms(), a->B > 0 ? a->B : 1);
+    // tensor-core path: split each query's tiles so that B x splits ~ one
+    // wave (gathered CSA tiles of 128 rows: smaller ones, 64 or 32 rows,
+    // measured slower at decode_1m, the per-tile fixed costs dominating)
+    const int B = a->B > 0 ? a->B : 1;
+    const int64_t wt = ceil_div64(a->w, 128);
+    const int tiles = (int)(ceil_div64(csa ? a->k : a->N_cap, csa ? L.gtile : 128) + wt);
+    int want = (int)ceil_div64(num_sms(), B);
+    if (want > kTcCombineMaxSplits) want = kTcCombineMaxSplits;
     if (want < 1) want = 1;
     L.tiles_per_split = (int)ceil_div64(tiles > 0 ? tiles : 1, want);
     L.splits = (int)ceil_div64(tiles > 0 ? tiles : 1, L.tiles_per_split);
@@ -821,7 +846,7 @@ int run_decode_t(const csahca_decode_args* a, cudaStream_t s, char* ws) {
     t.q_norm = a->q_norm; t.eps = eps; t.scale_log2 = scale * kLog2e; t.rope_dims = a->rope_dims;
     t.rope_base = base; t.B = a->B; t.nq = 1; t.N = a->N_cap; t.m = a->m; t.k = a->k; t.w = a->w;
     t.csa = a->kind == CSAHCA_CSA; t.idx = sel; t.decode = 1;
-    t.splits = L.splits; t.tiles_per_split = L.tiles_per_split; t.n_items = a->B * L.splits;
+    t.splits = L.splits; t.tiles_per_split = L.tiles_per_split; t.n_items = a->B * L.splits; t.gtile = L.gtile;
     t.out = nullptr; t.partial = partial;
     st = launch_attn_tc(t, a->kv_cache, (int64_t)a->B * a->N_cap, a->w > 0 ? a->win : nullptr,
                         (int64_t)a->B * a->w, s, a->kind == CSAHCA_CSA ? "attn_decode_csa_tc" : "attn_decode_hca_tc");
@@ -845,12 +870,23 @@ int run_decode_t(const csahca_decode_args* a, cudaStream_t s, char* ws) {
     c.partial = reinterpret_cast<const char*>(partial); c.sinks = a->sinks; c.pos = a->pos;
     c.out = static_cast<__nv_bfloat16*>(a->out);
     c.rows = a->B; c.splits = L.splits; c.rope_dims = a->rope_dims; c.rope_base = base;
-    const int smem = L.splits * 3 * kAttnH * 4;
+    const int smem = tc_combine_smem_bytes(L.splits);
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(attn_combine_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // the partials as [B * splits blocks][516 rows][64 fp16]: one box takes
+    // the m, l headers of every split of a query, one the 16-dim slices
+    CUtensorMap hdr_map, slc_map;
+    const uint64_t blocks = (uint64_t)a->B * L.splits;
+    const uint32_t slc_box = (uint32_t)(L.splits < kTcCombineSlots ? L.splits : kTcCombineSlots);
+    if (!encode_3d(&hdr_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, partial, kAttnH, kTcPartialRows, blocks, kAttnH * 2,
+                   kTcPartialBytes, kAttnH, kTcPartialHeaderRows, (uint32_t)L.splits) ||
+        !encode_3d(&slc_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, partial, kAttnH, kTcPartialRows, blocks, kAttnH * 2,
+                   kTcPartialBytes, kAttnH, kTcCombineDims, slc_box))
+      return CSAHCA_ERR_LAUNCH;
     {
       CSAHCA_TRACE("attn_combine", s);
-      launch_k(attn_combine_tc_kernel, dim3((unsigned)(a->B * (kAttnD / 16))), dim3(128), smem, s, c);
+      launch_k(attn_combine_tc_kernel, dim3((unsigned)(a->B * (kAttnD / kTcCombineDims))), dim3(128), smem, s,
+               hdr_map, slc_map, c);
     }
     CSAHCA_CHECK_LAUNCH();
     return CSAHCA_OK;

@@ -209,6 +209,7 @@ __global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLar
   uint32_t* cnt = p.counters + (int64_t)row * kTopkCounters;
   int* above = p.above + (int64_t)row * p.k;
   uint2* cand = p.cand + (int64_t)row * p.N;
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) hist8[i] = 0;   // first radix digit of the finish
   {
     uint32_t n_above_T;
     int T;
@@ -269,14 +270,47 @@ __global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLar
 
   const uint32_t n_above = min(__ldcg(&cnt[kCntAbove]), (uint32_t)p.k);
   const uint32_t n_cand = min(__ldcg(&cnt[kCntCand]), (uint32_t)p.N);
-  // candidates staged in shared memory when they fit (the usual case), else
-  // read from the scratch in every pass
+  const int words = (v + 31) / 32;
+  constexpr uint32_t kLowMask = (1u << kHistShift) - 1u;
+  // the selected set is built in a v-bit bitmap after the candidate cache:
+  // the taken list's loads go out first, the bitmap is cleared, and the
+  // candidates are staged in shared memory (when they fit, the usual case)
+  // while the first radix digit (bits 20..13) is counted
+  uint32_t* bm = bm_sel + 2 * kTopkCandCache;
+  int abv[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const uint32_t i = threadIdx.x + u * blockDim.x;
+    abv[u] = i < n_above ? __ldcg(above + i) : -1;
+  }
+  for (int i = threadIdx.x; i < words; i += blockDim.x) bm[i] = 0u;
   uint2* cand_s = reinterpret_cast<uint2*>(bm_sel);
   const bool cand_local = n_cand <= (uint32_t)kTopkCandCache;
-  if (cand_local)
-    for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) cand_s[i] = __ldcg(cand + i);
+  for (uint32_t i0 = 0; i0 < n_cand; i0 += 8 * blockDim.x) {
+    uint2 cc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t i = i0 + u * blockDim.x + threadIdx.x;
+      cc[u] = i < n_cand ? __ldcg(cand + i) : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t i = i0 + u * blockDim.x + threadIdx.x;
+      if (i < n_cand) {
+        if (cand_local) cand_s[i] = cc[u];
+        atomicAdd(&hist8[((cc[u].x & kLowMask) >> 13) & 255u], 1u);
+      }
+    }
+  }
   const uint2* C = cand_local ? cand_s : cand;
   __syncthreads();
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    if (abv[u] >= 0) atomicOr(&bm[abv[u] >> 5], 1u << (abv[u] & 31));
+  for (uint32_t i = threadIdx.x + 4 * blockDim.x; i < n_above; i += blockDim.x) {
+    const int j = __ldcg(above + i);
+    atomicOr(&bm[j >> 5], 1u << (j & 31));
+  }
   // radix select of the need-th largest key among the candidates (bits 20..0)
   uint32_t need = (uint32_t)p.k - n_above;
   uint32_t prefix = 0, mask = 0;
@@ -286,11 +320,13 @@ __global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLar
   for (int pass = 0; pass < 3; ++pass) {
     const int shf = shifts[pass];
     const uint32_t dm = (1u << widths[pass]) - 1u;
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist8[i] = 0;
-    __syncthreads();
-    for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
-      const uint32_t key = (cand_local ? C[i].x : __ldcg(&cand[i].x)) & ((1u << kHistShift) - 1u);
-      if ((key & mask) == prefix) atomicAdd(&hist8[(key >> shf) & dm], 1u);
+    if (pass > 0) {
+      for (int i = threadIdx.x; i < 256; i += blockDim.x) hist8[i] = 0;
+      __syncthreads();
+      for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
+        const uint32_t key = (cand_local ? C[i].x : __ldcg(&cand[i].x)) & kLowMask;
+        if ((key & mask) == prefix) atomicAdd(&hist8[(key >> shf) & dm], 1u);
+      }
     }
     __syncthreads();
     if ((threadIdx.x >> 5) == 0) {
@@ -299,68 +335,79 @@ __global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLar
       find_digit_warp(hist8, (int)dm + 1 >= 32 ? (int)dm + 1 : 32, nd, &sh_digit, &sh_need);
     }
     __syncthreads();
-    prefix |= sh_digit << shf;
+    prefix |= sh_digit << shf;                  // sh_digit is next written after two more barriers
     mask |= dm << shf;
-    __syncthreads();
   }
   need = sh_need;                              // keys equal to the threshold still to take
-  // count the keys equal to the threshold
-  if (threadIdx.x == 0) sh_eq = 0;
-  __syncthreads();
-  {
-    uint32_t ne = 0;
-    for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
-      const uint32_t low = (cand_local ? C[i].x : __ldcg(&cand[i].x)) & ((1u << kHistShift) - 1u);
-      ne += low == prefix;
-    }
-    if (ne) atomicAdd(&sh_eq, ne);
-  }
-  __syncthreads();
-  const uint32_t n_eq = sh_eq;
+  // the last pass counted, in the found digit's bin, exactly the keys equal
+  // to the threshold
+  const uint32_t n_eq = hist8[sh_digit];
   if (n_eq == need) {
-    // ---- common path: every key equal to the threshold is taken.  The
-    // selected set goes into a v-bit bitmap (after the candidate cache); each
-    // thread then owns a contiguous range of words, and one block prefix sum
-    // of their popcounts places its indices: the output is in index order.
-    const int words = (v + 31) / 32;
-    uint32_t* bm = bm_sel + 2 * kTopkCandCache;
-    for (int i = threadIdx.x; i < words; i += blockDim.x) bm[i] = 0u;
-    __syncthreads();
-    for (uint32_t i = threadIdx.x; i < n_above; i += blockDim.x) {
-      const int j = __ldcg(above + i);
-      atomicOr(&bm[j >> 5], 1u << (j & 31));
-    }
+    // ---- common path: every key equal to the threshold is taken.  Each
+    // warp owns a contiguous range of bitmap words, read lane-interleaved
+    // (conflict-free); one block prefix sum of the warps' popcounts and a
+    // warp scan per 32 words place the indices: the output is in index order.
     for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
       const uint2 c = cand_local ? C[i] : __ldcg(cand + i);
-      if ((c.x & ((1u << kHistShift) - 1u)) >= prefix) atomicOr(&bm[c.y >> 5], 1u << (c.y & 31));
+      if ((c.x & kLowMask) >= prefix) atomicOr(&bm[c.y >> 5], 1u << (c.y & 31));
     }
     __syncthreads();
-    const int wpt = (words + (int)blockDim.x - 1) / (int)blockDim.x;
-    const int w0 = (int)threadIdx.x * wpt, w1 = min(words, w0 + wpt);
-    int cnt = 0;
-    for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
-    int tot;
-    int pos = block_excl_count(cnt, warp_buf, &tot);
-    for (int w = w0; w < w1; ++w) {
-      uint32_t bits = bm[w];
-      while (bits) {
-        const int j = w * 32 + __ffs(bits) - 1;
-        bits &= bits - 1u;
-        if (pos < p.k) {
-          out[pos] = j;
-          if (p.prefetch_base)
-            bulk_prefetch_l2(p.prefetch_base + ((int64_t)row * p.N + j) * p.prefetch_row_bytes,
-                             (uint32_t)p.prefetch_row_bytes);
-        }
-        ++pos;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    // rounds of 512 words per warp: lane l reads words 32 i + l (conflict
+    // free); the 16 warp scans are independent, so they run interleaved
+    int done = 0;
+    for (int r0 = 0; r0 < words; r0 += nwarps * 512) {
+      const int wb = r0 + warp * 512;
+      uint32_t bits[16];
+      int c[16], incl[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int w = wb + 32 * i + lane;
+        bits[i] = w < words ? bm[w] : 0u;
+        c[i] = __popc(bits[i]);
+        incl[i] = c[i];
       }
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int y = __shfl_up_sync(0xffffffffu, incl[i], o);
+          if (lane >= o) incl[i] += y;
+        }
+      }
+      int goff[16], wtot = 0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        goff[i] = wtot;
+        wtot += __shfl_sync(0xffffffffu, incl[i], 31);
+      }
+      int tot;
+      const int wbase = block_excl_count(lane == 0 ? wtot : 0, warp_buf, &tot);
+      const int pos0 = done + __shfl_sync(0xffffffffu, wbase, 0);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        uint32_t b = bits[i];
+        int q = pos0 + goff[i] + incl[i] - c[i];
+        const int w = wb + 32 * i + lane;
+        while (b) {
+          const int j = w * 32 + __ffs(b) - 1;
+          b &= b - 1u;
+          if (q < p.k) {
+            out[q] = j;
+            if (p.prefetch_base)
+              bulk_prefetch_l2(p.prefetch_base + ((int64_t)row * p.N + j) * p.prefetch_row_bytes,
+                               (uint32_t)p.prefetch_row_bytes);
+          }
+          ++q;
+        }
+      }
+      done += tot;
     }
     return;
   }
   // ---- tie path (more keys equal to the threshold than still to take):
   // the lowest-index ties through a bitmap scan in index order
   __syncthreads();
-  const int words = (v + 31) / 32;
   uint32_t* bm_eq = bm_sel + words;
   for (int i = threadIdx.x; i < 2 * words; i += blockDim.x) bm_sel[i] = 0;
   __syncthreads();
