@@ -838,7 +838,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
 // latency, not one per split.  With more splits than slice slots the slices
 // go in rounds.
 constexpr int kTcCombineMaxSplits = 160;
-constexpr int kTcCombineSlots = 64;
+constexpr int kTcCombineSlots = 48;
+constexpr int kTcCombineThreads = 512;        // four threads per (dim, 8 heads): every fourth split each
 constexpr int kTcCombineDims = 16;
 constexpr int kTcCombineSlice = kTcCombineDims * kAttnH * 2;
 
@@ -862,13 +863,13 @@ __host__ __device__ inline int tc_combine_smem_bytes(int splits) {
 // box [min(splits, 64)][16][64] (16 dims of up to 64 splits).  A bulk copy per
 // split was measured to complete one copy at a time; a box covering every
 // split goes out as one transfer.
-__global__ void __launch_bounds__(128) attn_combine_tc_kernel(const __grid_constant__ CUtensorMap hdr_map,
-                                                              const __grid_constant__ CUtensorMap slc_map,
-                                                              TcCombineParams p) {
+__global__ void __launch_bounds__(kTcCombineThreads) attn_combine_tc_kernel(
+    const __grid_constant__ CUtensorMap hdr_map, const __grid_constant__ CUtensorMap slc_map, TcCombineParams p) {
   extern __shared__ __align__(128) uint8_t cmb_smem[];
   __shared__ uint64_t bar_hdr, bar_slc;
-  __shared__ float red[2][kAttnH];
+  __shared__ float red[8][kAttnH];
   __shared__ float inv_s[kAttnH];
+  __shared__ __align__(16) float acc_s[3][128][8];
   __shared__ __align__(16) __nv_bfloat16 ostage[kAttnH][kTcCombineDims];
   __shared__ volatile int abort_flag;
   constexpr int kChunks = kAttnD / kTcCombineDims;
@@ -897,34 +898,42 @@ __global__ void __launch_bounds__(128) attn_combine_tc_kernel(const __grid_const
     mbar_expect_tx(&bar_slc, (uint32_t)(nslots * kTcCombineSlice));
     tma_load_3d(slots, &slc_map, 0, srow, blk0, &bar_slc);
   }
-  // split weights: thread (head h, half) takes the splits of its parity
-  const int h = tid & (kAttnH - 1), half = tid >> 6;
+  // split weights: thread (head h, part) takes the splits s = part mod 8
+  const int h = tid & (kAttnH - 1), part = tid >> 6;
   bool ok = mbar_wait(&bar_hdr, 0, &abort_flag);
   const float z2 = p.sinks[h] * kLog2e;
   float mx = -INFINITY;
   if (ok) {
 #pragma unroll 4
-    for (int s = half; s < p.splits; s += 2) mx = fmaxf(mx, hdr[s * 2 * kAttnH + h]);
+    for (int s = part; s < p.splits; s += 8) mx = fmaxf(mx, hdr[s * 2 * kAttnH + h]);
   }
-  red[half][h] = mx;
+  red[part][h] = mx;
   __syncthreads();
-  const float M = fmaxf(z2, fmaxf(red[0][h], red[1][h]));
+  float M = z2;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) M = fmaxf(M, red[i][h]);
   float den = 0.f;
   if (ok)
 #pragma unroll 4
-    for (int s = half; s < p.splits; s += 2) {
+    for (int s = part; s < p.splits; s += 8) {
       const float ms = hdr[s * 2 * kAttnH + h];
       const float f = ms == -INFINITY ? 0.f : hdr[s * 2 * kAttnH + kAttnH + h] * exp2f(ms - M);
       hdr[s * 2 * kAttnH + h] = f;
       den += f;
     }
   __syncthreads();                                 // every read of red[] (M) is done
-  red[half][h] = den;
+  red[part][h] = den;
   __syncthreads();
-  if (half == 0) inv_s[h] = 1.f / (exp2f(z2 - M) + red[0][h] + red[1][h]);
-  __syncthreads();
-  // weighted sum over the splits: thread (dim dl, heads 8 hg ..)
-  const int dl = tid >> 3, hg = tid & 7;
+  if (part == 0) {
+    float d = exp2f(z2 - M);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) d += red[i][h];
+    inv_s[h] = 1.f / d;
+  }
+  // weighted sum over the splits: thread (quarter qt, dim dl, heads 8 hg ..)
+  // takes the splits s = qt mod 4
+  const int qt = tid >> 7, lt = tid & 127;
+  const int dl = lt >> 3, hg = lt & 7;
   const int dim = dc * kTcCombineDims + dl;
   float acc[8];
 #pragma unroll
@@ -944,8 +953,8 @@ __global__ void __launch_bounds__(128) attn_combine_tc_kernel(const __grid_const
       const int n = min(p.splits, s0 + nslots) - s0;
       const float* wb = hdr + s0 * 2 * kAttnH + hg * 8;
       const uint8_t* sb = slots + dl * (kAttnH * 2) + hg * 16;
-#pragma unroll 4
-      for (int i = 0; i < n; ++i) {
+#pragma unroll 2
+      for (int i = qt; i < n; i += 4) {
         const float4 w0 = *reinterpret_cast<const float4*>(wb + i * 2 * kAttnH);
         const float4 w1 = *reinterpret_cast<const float4*>(wb + i * 2 * kAttnH + 4);
         uint4 raw = *reinterpret_cast<const uint4*>(sb + i * kTcCombineSlice);
@@ -964,25 +973,36 @@ __global__ void __launch_bounds__(128) attn_combine_tc_kernel(const __grid_const
       }
     }
   }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] *= inv_s[hg * 8 + i];
-  // rope dims: the pair partner (dim ^ 1) is thread tid ^ 8
-  const int r0 = kAttnD - p.rope_dims;
-  float partner[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) partner[i] = __shfl_xor_sync(0xffffffffu, acc[i], 8);
-  if (dim >= r0) {
-    float cs, sn;
-    rope_cos_sin(-(double)p.pos[row], (dim - r0) >> 1, p.rope_dims, p.rope_base, &cs, &sn);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      acc[i] = (dim & 1) ? fmaf(partner[i], sn, acc[i] * cs) : fmaf(-partner[i], sn, acc[i] * cs);
+  if (qt > 0) {
+    *reinterpret_cast<float4*>(&acc_s[qt - 1][lt][0]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    *reinterpret_cast<float4*>(&acc_s[qt - 1][lt][4]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) ostage[hg * 8 + i][dl] = __float2bfloat16_rn(acc[i]);
   ok = __syncthreads_and(ok);
+  if (qt == 0) {
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += acc_s[j][lt][i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] *= inv_s[hg * 8 + i];
+    // rope dims: the pair partner (dim ^ 1) is thread tid ^ 8
+    const int r0 = kAttnD - p.rope_dims;
+    float partner[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) partner[i] = __shfl_xor_sync(0xffffffffu, acc[i], 8);
+    if (dim >= r0) {
+      float cs, sn;
+      rope_cos_sin(-(double)p.pos[row], (dim - r0) >> 1, p.rope_dims, p.rope_base, &cs, &sn);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        acc[i] = (dim & 1) ? fmaf(partner[i], sn, acc[i] * cs) : fmaf(-partner[i], sn, acc[i] * cs);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ostage[hg * 8 + i][dl] = __float2bfloat16_rn(acc[i]);
+  }
+  __syncthreads();
   if (!ok) return;
-  {
+  if (tid < 128) {
     const int hh = tid >> 1, piece = tid & 1;
     *reinterpret_cast<uint4*>(p.out + ((int64_t)row * kAttnH + hh) * kAttnD + dc * kTcCombineDims + piece * 8) =
         *reinterpret_cast<const uint4*>(&ostage[hh][piece * 8]);

@@ -326,7 +326,7 @@ int launch_zero(char* ptr, size_t bytes, cudaStream_t s) {
 // zeroed the scratch and built the row histograms (pass 1) while scoring.
 int launch_topk(const csahca_indexer_args* a, const float* scores, int64_t stride, const int* q_pos, int* idx,
                 int rows, char* scratch, cudaStream_t s, bool hist_ready = false,
-                const void* prefetch_base = nullptr, int64_t prefetch_row_bytes = 0) {
+                const void* prefetch_base = nullptr, int64_t prefetch_row_bytes = 0, bool sorted = true) {
   if (!topk_uses_large(a)) {
     TopkParams tp;
     tp.scores = scores; tp.row_stride = stride; tp.q_pos = q_pos; tp.idx = idx;
@@ -354,6 +354,7 @@ int launch_topk(const csahca_indexer_args* a, const float* scores, int64_t strid
   tp.above = reinterpret_cast<int*>(scratch + L.above);
   tp.cand = reinterpret_cast<uint2*>(scratch + L.cand);
   tp.thresh_ready = hist_ready ? 1 : 0;
+  tp.sorted = sorted ? 1 : 0;
   tp.prefetch_base = static_cast<const char*>(prefetch_base);
   tp.prefetch_row_bytes = prefetch_row_bytes;
   if (!hist_ready) {
@@ -476,7 +477,7 @@ int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* score
 // prefetch_base / prefetch_row_bytes (internal, decode only): every selected
 // row of a long row's top-k is prefetched into L2 from that [B][N] table.
 int run_indexer(const csahca_indexer_args* a, void* stream, const void* prefetch_base = nullptr,
-                int64_t prefetch_row_bytes = 0) {
+                int64_t prefetch_row_bytes = 0, bool sorted = true) {
   int st = validate_indexer(a);
   if (st != CSAHCA_OK) return st;
   if (a->B == 0 || a->nq == 0) return CSAHCA_OK;
@@ -564,7 +565,7 @@ int run_indexer(const csahca_indexer_args* a, void* stream, const void* prefetch
     // addressed per batch entry, so launch per b unless the chunk is the whole nq
     if (qc == a->nq) {
       int st3 = launch_topk(a, base, stride, a->q_pos, a->idx, a->B * qc, scratch, s, fuse_hist,
-                            a->nq == 1 ? prefetch_base : nullptr, prefetch_row_bytes);
+                            a->nq == 1 ? prefetch_base : nullptr, prefetch_row_bytes, sorted);
       if (st3 != CSAHCA_OK) return st3;
     } else {
       for (int b = 0; b < a->B; ++b) {
@@ -830,7 +831,9 @@ int run_decode_t(const csahca_decode_args* a, cudaStream_t s, char* ws) {
       ia.q_pos = a->pos; ia.idx = idx;
       ia.workspace = ws + L.scores_off;
       ia.workspace_bytes = L.idx_off - L.scores_off;
-      int st = run_indexer(&ia, s);
+      // the attention needs the selected set only: index order is kept
+      // when the caller asked for the selection
+      int st = run_indexer(&ia, s, nullptr, 0, a->idx_out != nullptr);
       if (st != CSAHCA_OK) return st;
       sel = idx;
     }
@@ -885,8 +888,8 @@ int run_decode_t(const csahca_decode_args* a, cudaStream_t s, char* ws) {
       return CSAHCA_ERR_LAUNCH;
     {
       CSAHCA_TRACE("attn_combine", s);
-      launch_k(attn_combine_tc_kernel, dim3((unsigned)(a->B * (kAttnD / kTcCombineDims))), dim3(128), smem, s,
-               hdr_map, slc_map, c);
+      launch_k(attn_combine_tc_kernel, dim3((unsigned)(a->B * (kAttnD / kTcCombineDims))), dim3(kTcCombineThreads),
+               smem, s, hdr_map, slc_map, c);
     }
     CSAHCA_CHECK_LAUNCH();
     return CSAHCA_OK;

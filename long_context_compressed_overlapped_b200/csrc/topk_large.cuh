@@ -46,6 +46,7 @@ struct TopkLargeParams {
   uint32_t* hist;                          // [rows][kHistBins]
   uint32_t* counters;                      // [rows][kTopkCounters]: see kCnt* below
   int thresh_ready;                        // the indexer stored T and n_above_T in the counters
+  int sorted;                              // 1: each row's indices in ascending order; 0: any order
   int* above;                              // [rows][k]
   uint2* cand;                             // [rows][N]: (key, index)
   // optional: row j of sequence `row` of a [rows][N] table of prefetch_row_bytes
@@ -176,27 +177,89 @@ __device__ __forceinline__ int bitmap_scan(const uint32_t* bm, int words, int li
 
 constexpr int kTopkSelectThreads = 512;
 constexpr int kTopkCandCache = 4096;       // candidates staged in shared memory (8 bytes each)
+constexpr int kTopkFinishBins = 2048;      // first radix digit of the finish: bits 20..10
+constexpr int kTopkSortMax = 1024;         // k up to this: the selection is sorted, not bitmapped
 
-// Dynamic shared memory of topk_select_kernel: the larger of the tie path
-// (two bitmaps of N bits) and the common path (candidate cache, then one
-// bitmap of N bits).
+// Dynamic shared memory of topk_select_kernel: the candidate cache, the
+// finish histogram and a region for the sorted selection or the v-bit
+// bitmap; the tie path reuses all of it as two bitmaps.
 __host__ __device__ __forceinline__ int topk_select_smem_bytes(int N) {
   const int words = (N + 31) / 32;
   const int ties = 2 * words * 4;
-  const int common = kTopkCandCache * 8 + words * 4;
+  const int common = kTopkCandCache * 8 + kTopkFinishBins * 4 + (words > kTopkSortMax ? words : kTopkSortMax) * 4;
   return ties > common ? ties : common;
 }
 
-// Routing of one slice (pass 2) and, in the last CTA of the row, the exact
-// selection.  Dynamic shared memory: topk_select_smem_bytes(N) (two bitmaps).
-__global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLargeParams p) {
+// Largest digit d of an nb-bin histogram (nb = 2 or 4 x blockDim) with
+// count(digits > d) < need <= count(digits >= d); one thread writes d and
+// need - count(digits > d).  Thread t sums bins [nb - per (t + 1), nb - per t),
+// and one block prefix sum places the crossing.  Every thread calls it.
+__device__ __forceinline__ void find_digit_block(const uint32_t* hist, int nb, uint32_t need, int* warp_buf,
+                                                 uint32_t* out_digit, uint32_t* out_need) {
+  const int per = nb / (int)blockDim.x;
+  const int hi = nb - (int)threadIdx.x * per;
+  uint32_t local = 0;
+  for (int e = 0; e < per; ++e) local += hist[hi - 1 - e];
+  int tot;
+  const uint32_t above = (uint32_t)block_excl_count((int)local, warp_buf, &tot);
+  if (above < need && above + local >= need) {
+    uint32_t cum = above;
+    for (int e = 0; e < per; ++e) {
+      const int b = hi - 1 - e;
+      if (cum + hist[b] >= need) { *out_digit = (uint32_t)b; *out_need = need - cum; break; }
+      cum += hist[b];
+    }
+  }
+}
+
+// Ascending bitonic sort of a[0, 1024) by a block of 512 threads.  Thread
+// (warp w, lane l) holds elements p0 = 64 w + l and p1 = p0 + 32 in
+// registers: strides below 32 are warp shuffles, stride 32 pairs a thread's
+// own two elements, and only the ten steps with stride >= 64 go through
+// shared memory.
+__device__ __forceinline__ int bitonic_cmpx(int mine, int other, int p, int s, int size) {
+  const bool lower = (p & s) == 0, asc = (p & size) == 0;
+  return lower == asc ? min(mine, other) : max(mine, other);
+}
+__device__ __forceinline__ void sort1024_block(int* a) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int p0 = 64 * w + lane, p1 = p0 + 32;
+  int e0 = a[p0], e1 = a[p1];
+  for (int size = 2; size <= 1024; size <<= 1) {
+    for (int s = size >> 1; s > 0; s >>= 1) {
+      if (s >= 64) {
+        __syncthreads();
+        a[p0] = e0;
+        a[p1] = e1;
+        __syncthreads();
+        const int o0 = a[p0 ^ s], o1 = a[p1 ^ s];
+        e0 = bitonic_cmpx(e0, o0, p0, s, size);
+        e1 = bitonic_cmpx(e1, o1, p1, s, size);
+      } else if (s == 32) {
+        const bool asc = (p0 & size) == 0;
+        const int lo = min(e0, e1), hi = max(e0, e1);
+        e0 = asc ? lo : hi;
+        e1 = asc ? hi : lo;
+      } else {
+        const int o0 = __shfl_xor_sync(0xffffffffu, e0, s), o1 = __shfl_xor_sync(0xffffffffu, e1, s);
+        e0 = bitonic_cmpx(e0, o0, p0, s, size);
+        e1 = bitonic_cmpx(e1, o1, p1, s, size);
+      }
+    }
+  }
+  __syncthreads();
+  a[p0] = e0;
+  a[p1] = e1;
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kTopkSelectThreads, 2) topk_select_kernel(TopkLargeParams p) {
   griddep_launch_dependents();
   griddep_wait();
   extern __shared__ uint32_t bm_sel[];               // [words] taken, then [words] ties
   __shared__ uint32_t sh[1024];
-  __shared__ uint32_t hist8[256];
   __shared__ int warp_buf[72];
-  __shared__ uint32_t sh_digit, sh_need, sh_eq, sh_base_t, sh_base_c;
+  __shared__ uint32_t sh_digit, sh_need, sh_base_t, sh_base_c;
   __shared__ int sh_last;
   const int row = blockIdx.x / p.slices, slice = blockIdx.x % p.slices;
   const int v = topk_visible(p, row);
@@ -209,7 +272,6 @@ __global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLar
   uint32_t* cnt = p.counters + (int64_t)row * kTopkCounters;
   int* above = p.above + (int64_t)row * p.k;
   uint2* cand = p.cand + (int64_t)row * p.N;
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) hist8[i] = 0;   // first radix digit of the finish
   {
     uint32_t n_above_T;
     int T;
@@ -272,19 +334,19 @@ __global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLar
   const uint32_t n_cand = min(__ldcg(&cnt[kCntCand]), (uint32_t)p.N);
   const int words = (v + 31) / 32;
   constexpr uint32_t kLowMask = (1u << kHistShift) - 1u;
-  // the selected set is built in a v-bit bitmap after the candidate cache:
-  // the taken list's loads go out first, the bitmap is cleared, and the
-  // candidates are staged in shared memory (when they fit, the usual case)
-  // while the first radix digit (bits 20..13) is counted
-  uint32_t* bm = bm_sel + 2 * kTopkCandCache;
+  uint2* cand_s = reinterpret_cast<uint2*>(bm_sel);                // candidate cache
+  uint32_t* hist = bm_sel + 2 * kTopkCandCache;                     // finish histogram
+  uint32_t* R = hist + kTopkFinishBins;                             // selection or bitmap
+  // the taken list's loads go out first; the candidates are staged in shared
+  // memory (when they fit, the usual case) while the first digit is counted
   int abv[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const uint32_t i = threadIdx.x + u * blockDim.x;
     abv[u] = i < n_above ? __ldcg(above + i) : -1;
   }
-  for (int i = threadIdx.x; i < words; i += blockDim.x) bm[i] = 0u;
-  uint2* cand_s = reinterpret_cast<uint2*>(bm_sel);
+  for (int i = threadIdx.x; i < kTopkFinishBins; i += blockDim.x) hist[i] = 0u;
+  __syncthreads();
   const bool cand_local = n_cand <= (uint32_t)kTopkCandCache;
   for (uint32_t i0 = 0; i0 < n_cand; i0 += 8 * blockDim.x) {
     uint2 cc[8];
@@ -298,55 +360,101 @@ __global__ void __launch_bounds__(kTopkSelectThreads) topk_select_kernel(TopkLar
       const uint32_t i = i0 + u * blockDim.x + threadIdx.x;
       if (i < n_cand) {
         if (cand_local) cand_s[i] = cc[u];
-        atomicAdd(&hist8[((cc[u].x & kLowMask) >> 13) & 255u], 1u);
+        atomicAdd(&hist[(cc[u].x & kLowMask) >> 10], 1u);
       }
     }
   }
   const uint2* C = cand_local ? cand_s : cand;
   __syncthreads();
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-    if (abv[u] >= 0) atomicOr(&bm[abv[u] >> 5], 1u << (abv[u] & 31));
-  for (uint32_t i = threadIdx.x + 4 * blockDim.x; i < n_above; i += blockDim.x) {
-    const int j = __ldcg(above + i);
-    atomicOr(&bm[j >> 5], 1u << (j & 31));
-  }
-  // radix select of the need-th largest key among the candidates (bits 20..0)
+  // radix select of the need-th largest key among the candidates: digit
+  // bits 20..10, then bits 9..0 among the keys of that digit
   uint32_t need = (uint32_t)p.k - n_above;
-  uint32_t prefix = 0, mask = 0;
-  if (threadIdx.x == 0) sh_need = need;
-  const int shifts[3] = {13, 5, 0};
-  const int widths[3] = {8, 8, 5};
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shf = shifts[pass];
-    const uint32_t dm = (1u << widths[pass]) - 1u;
-    if (pass > 0) {
-      for (int i = threadIdx.x; i < 256; i += blockDim.x) hist8[i] = 0;
-      __syncthreads();
-      for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
-        const uint32_t key = (cand_local ? C[i].x : __ldcg(&cand[i].x)) & kLowMask;
-        if ((key & mask) == prefix) atomicAdd(&hist8[(key >> shf) & dm], 1u);
+  find_digit_block(hist, kTopkFinishBins, need, warp_buf, &sh_digit, &sh_need);
+  __syncthreads();
+  const uint32_t d1 = sh_digit;
+  need = sh_need;
+  for (int i = threadIdx.x; i < 1024; i += blockDim.x) hist[i] = 0u;
+  __syncthreads();
+  for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
+    const uint32_t key = (cand_local ? C[i].x : __ldcg(&cand[i].x)) & kLowMask;
+    if ((key >> 10) == d1) atomicAdd(&hist[key & 1023u], 1u);
+  }
+  __syncthreads();
+  find_digit_block(hist, 1024, need, warp_buf, &sh_digit, &sh_need);
+  __syncthreads();
+  const uint32_t prefix = (d1 << 10) | sh_digit;   // low 21 bits of the threshold key
+  need = sh_need;                                   // keys equal to the threshold still to take
+  const uint32_t n_eq = hist[sh_digit];             // keys equal to the threshold
+  if (n_eq == need && !p.sorted) {
+    // ---- common path, any order: the taken list, then the candidates at or
+    // above the threshold (a block prefix sum places them)
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (abv[u] >= 0) out[threadIdx.x + u * blockDim.x] = abv[u];
+    for (uint32_t i = threadIdx.x + 4 * blockDim.x; i < n_above; i += blockDim.x) out[i] = __ldcg(above + i);
+    int mine = 0;
+    for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) mine += ((C[i].x & kLowMask) >= prefix);
+    int tot;
+    int q = (int)n_above + block_excl_count(mine, warp_buf, &tot);
+    for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
+      const uint2 c = cand_local ? C[i] : __ldcg(cand + i);
+      if ((c.x & kLowMask) >= prefix) {
+        if (q < p.k) out[q] = (int)c.y;
+        ++q;
       }
     }
-    __syncthreads();
-    if ((threadIdx.x >> 5) == 0) {
-      const uint32_t nd = sh_need;
-      __syncwarp();
-      find_digit_warp(hist8, (int)dm + 1 >= 32 ? (int)dm + 1 : 32, nd, &sh_digit, &sh_need);
-    }
-    __syncthreads();
-    prefix |= sh_digit << shf;                  // sh_digit is next written after two more barriers
-    mask |= dm << shf;
+    for (int i = (int)n_above + tot + (int)threadIdx.x; i < p.k; i += blockDim.x) out[i] = -1;
+    return;
   }
-  need = sh_need;                              // keys equal to the threshold still to take
-  // the last pass counted, in the found digit's bin, exactly the keys equal
-  // to the threshold
-  const uint32_t n_eq = hist8[sh_digit];
+  if (n_eq == need && p.k <= kTopkSortMax) {
+    // ---- common path: every key equal to the threshold is taken.  The
+    // selection (the taken list, then the candidates at or above the
+    // threshold) is sorted ascending in shared memory: the output is in
+    // index order.
+    int* sel = reinterpret_cast<int*>(R);
+    constexpr int kp = kTopkSortMax;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (abv[u] >= 0) sel[threadIdx.x + u * blockDim.x] = abv[u];
+    for (uint32_t i = threadIdx.x + 4 * blockDim.x; i < n_above; i += blockDim.x) sel[i] = __ldcg(above + i);
+    int mine = 0;
+    for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) mine += ((C[i].x & kLowMask) >= prefix);
+    int tot;
+    int q = (int)n_above + block_excl_count(mine, warp_buf, &tot);
+    for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
+      const uint2 c = cand_local ? C[i] : __ldcg(cand + i);
+      if ((c.x & kLowMask) >= prefix) {
+        if (q < kp) sel[q] = (int)c.y;
+        ++q;
+      }
+    }
+    for (int i = (int)n_above + tot + (int)threadIdx.x; i < kp; i += blockDim.x) sel[i] = INT_MAX;
+    __syncthreads();
+    sort1024_block(sel);
+    for (int i = threadIdx.x; i < p.k; i += blockDim.x) {
+      const int j = sel[i];
+      out[i] = j == INT_MAX ? -1 : j;
+      if (p.prefetch_base && j != INT_MAX)
+        bulk_prefetch_l2(p.prefetch_base + ((int64_t)row * p.N + j) * p.prefetch_row_bytes,
+                         (uint32_t)p.prefetch_row_bytes);
+    }
+    return;
+  }
   if (n_eq == need) {
-    // ---- common path: every key equal to the threshold is taken.  Each
-    // warp owns a contiguous range of bitmap words, read lane-interleaved
-    // (conflict-free); one block prefix sum of the warps' popcounts and a
-    // warp scan per 32 words place the indices: the output is in index order.
+    // ---- common path, k above the sort limit: the selection goes into a
+    // v-bit bitmap; each warp owns a contiguous range of words, read
+    // lane-interleaved (conflict-free); one block prefix sum of the warps'
+    // popcounts and a warp scan per 32 words place the indices in order.
+    uint32_t* bm = R;
+    for (int i = threadIdx.x; i < words; i += blockDim.x) bm[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (abv[u] >= 0) atomicOr(&bm[abv[u] >> 5], 1u << (abv[u] & 31));
+    for (uint32_t i = threadIdx.x + 4 * blockDim.x; i < n_above; i += blockDim.x) {
+      const int j = __ldcg(above + i);
+      atomicOr(&bm[j >> 5], 1u << (j & 31));
+    }
     for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
       const uint2 c = cand_local ? C[i] : __ldcg(cand + i);
       if ((c.x & kLowMask) >= prefix) atomicOr(&bm[c.y >> 5], 1u << (c.y & 31));

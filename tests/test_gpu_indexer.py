@@ -113,6 +113,36 @@ def test_indexer_decode_e4m3_long_rows():
     assert api.device_error() == 0
 
 
+def test_indexer_long_rows_ties_and_large_k():
+    """Rows longer than one CTA's top-k (the multi-CTA select): every score
+    equal (the lowest indices win, bf16 and e4m3 keys), eight distinct key
+    rows (thousands of ties at the threshold, lowest indices first), and k
+    above the sorted-selection limit (the bitmap selection)."""
+    wl = synth.WORKLOADS["decode_1m"]
+    D = synth.Draw(15, DEV)
+    B, N = 2, 40001
+    qI = D.normal("qI", (B, 1, wl.HI, wl.dI), 1.0, torch.bfloat16)
+    w = D.normal("w", (B, 1, wl.HI), 1 / np.sqrt(wl.HI))
+    q_pos = torch.tensor([[4 * N + 3], [4 * N - 1]], device=DEV, dtype=torch.int32)
+    same = D.normal("k1", (B, 1, wl.dI), 1.0, torch.bfloat16).repeat(1, N, 1).contiguous()
+    for kk, sc in ((same, None), synth.quantize_e4m3_rows(same)):
+        idx = api.indexer_topk(qI, w, kk, q_pos, wl.m, 64, kI_scale=sc)
+        for b in range(B):
+            assert npy(idx[b, 0]).tolist() == list(range(64)), f"all-equal b={b}"
+    few = D.normal("k8", (B, 8, wl.dI), 1.0, torch.bfloat16)
+    kf = few[:, torch.arange(N, device=DEV) % 8].contiguous()
+    idx = api.indexer_topk(qI, w, kf, q_pos, wl.m, wl.k)
+    for b in range(B):
+        v = min(O.n_visible(int(q_pos[b, 0]), wl.m), N)
+        s = O.indexer_scores(npy(qI[b, 0]), npy(w[b, 0]), npy(kf[b])[:v])
+        want = np.sort(np.argsort(-s, kind="stable")[:wl.k])
+        assert npy(idx[b, 0]).tolist() == want.tolist(), f"ties b={b}"
+    kr = D.normal("kr", (B, N, wl.dI), 1.0, torch.bfloat16)
+    idx = api.indexer_topk(qI, w, kr, q_pos, wl.m, 5000)
+    _check_rows(idx, qI, w, kr, None, q_pos, wl.m, 5000, [(b, 0) for b in range(B)])
+    assert api.device_error() == 0
+
+
 def test_indexer_edge_cases():
     """No visible entry (t < m - 1, negative t), exactly k visible, k = 1,
     and all-equal scores (ties go to the lower index)."""
