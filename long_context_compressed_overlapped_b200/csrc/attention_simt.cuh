@@ -54,8 +54,8 @@ __device__ __forceinline__ const T* key_row(const SimtAttnParams& p, int b, int 
 
 template <typename T>
 __global__ void __launch_bounds__(32 * kSimtHG) attn_simt_kernel(SimtAttnParams p) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ float smem_at[];
   const int d = p.d, ld = d + 1;
   float* qs = smem_at;                              // [HG][d]
@@ -203,8 +203,8 @@ struct CombineParams {
 
 template <typename T>
 __global__ void __launch_bounds__(128) attn_combine_kernel(CombineParams p) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   // one CTA per (b, q, h); the split weights f_s = e^{m_s - M} / den are
   // computed once into shared memory, then each thread sums 4 dims
   __shared__ float wsplit[kCombineMaxSplits];

@@ -50,6 +50,7 @@ struct AttnTcParams {
   int decode;                   // window = ring [B, w, d] (decode) or finished rows [B, nq, d]
   int n_items, splits, tiles_per_split;
   int gtile;                    // CSA: selected rows per tile (128, 64 or 32); rows gtile..127 stay zero
+  int first_kernel;             // 1: the call's first kernel (inputs are read only after the wait)
   __nv_bfloat16* out;           // final [B, nq, H, D]
   float* partial;               // [B, nq, H, splits, D + 4]
 };
@@ -271,7 +272,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
   const uint32_t tS = tmem;                 // S^T: columns [0, H)
   const uint32_t tO = tmem + 128;           // O^T M-tile j: columns [128 + j*H, ...)
   const uint32_t tL = tmem + 128 + kAttnMT * kAttnH;   // per-key-slot partial sums of p: H columns
-  griddep_launch_dependents();
+  // Programmatic dependent launch: every kernel of the library signals its
+  // dependents only after its own wait, so when a kernel starts, all work
+  // queued before its predecessor has completed and the call's inputs may be
+  // read before the wait.  As the call's first kernel this one waits before
+  // reading anything (query, positions, gain).
+  if (p.first_kernel) {
+    griddep_wait();
+    griddep_launch_dependents();
+  }
 
   if (warp == 8 || warp == 9) {
     // ------------------------------------------------------------ producers
@@ -300,9 +309,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
         if (!ok) { stop = true; break; }
         ++icount;
       }
-      // key rows and selections may come from earlier kernels of this stream;
-      // the query (a caller input) was already on its way
+      // key rows and selections may come from earlier kernels of this stream
       griddep_wait();
+      if (lane == 0 && pw == 0) griddep_launch_dependents();
       for (int tile = it.tile0; tile < it.tile1 && !stop; ++tile, ++tcount) {
         const AttnTile T = attn_tile(p, it, tile);
         const uint32_t ph = tcount & 1;
@@ -888,8 +897,8 @@ __global__ void __launch_bounds__(kTcCombineThreads) attn_combine_tc_kernel(
     tma_prefetch_desc(&slc_map);
   }
   __syncthreads();
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   if (tid == 0) {
     mbar_expect_tx(&bar_hdr, (uint32_t)(p.splits * kTcPartialHeader));
     tma_load_3d(hdr, &hdr_map, 0, 0, blk0, &bar_hdr);

@@ -114,9 +114,11 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes
 // data that an earlier kernel of the library may write (compressed rows,
 // scores, selections, partials) and before its first global write, a thread
 // calls griddep_wait(), which returns once every prerequisite grid has
-// completed and its writes are visible (at once when there is none).  Work
-// before it touches only shared memory, TMEM, kernel parameters and the
-// caller's inputs that no kernel of the library writes.
+// completed and its writes are visible (at once when there is none).  A
+// kernel signals its dependents only after its own wait: so when a kernel
+// starts, everything queued before its predecessor (the caller's work
+// included) has completed, and it may read the call's inputs before its own
+// wait.  The first kernel of a call reads nothing before its wait.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // Lets the next kernel in the stream be scheduled once every CTA of this grid
 // has issued it or exited.

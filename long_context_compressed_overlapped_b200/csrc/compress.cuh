@@ -91,8 +91,8 @@ __device__ __forceinline__ void finish_row(float (&vals)[kMaxChunksPerLane][VEC]
 
 template <typename T, bool kCSA>
 __global__ void __launch_bounds__(256) compress_kernel(CompressParams p) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   constexpr int VEC = Vec16<T>::N;
   const int warp = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
@@ -163,8 +163,8 @@ struct FinishParams {
 
 template <typename T>
 __global__ void __launch_bounds__(256) finish_rows_kernel(FinishParams p) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   constexpr int VEC = Vec16<T>::N;
   const int64_t row = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;

@@ -687,7 +687,7 @@ int run_prefill_t(const csahca_attn_args* a, cudaStream_t s) {
     t.q_norm = a->q_norm; t.eps = eps; t.scale_log2 = scale * kLog2e; t.rope_dims = a->rope_dims;
     t.rope_base = base; t.B = a->B; t.nq = a->n; t.N = a->N; t.m = a->m; t.k = a->k; t.w = a->w;
     t.csa = a->kind == CSAHCA_CSA; t.idx = a->idx; t.decode = 0;
-    t.n_items = a->B * a->n; t.splits = 1; t.tiles_per_split = 0; t.gtile = 128;
+    t.n_items = a->B * a->n; t.splits = 1; t.tiles_per_split = 0; t.gtile = 128; t.first_kernel = a->w > 0 ? 0 : 1;
     t.out = static_cast<__nv_bfloat16*>(a->out); t.partial = nullptr;
     return launch_attn_tc(t, a->kv_comp, (int64_t)a->B * a->N, win_final, (int64_t)a->B * a->n, s,
                           a->kind == CSAHCA_CSA ? "attn_prefill_csa_tc" : "attn_prefill_hca_tc");
@@ -850,6 +850,7 @@ int run_decode_t(const csahca_decode_args* a, cudaStream_t s, char* ws) {
     t.rope_base = base; t.B = a->B; t.nq = 1; t.N = a->N_cap; t.m = a->m; t.k = a->k; t.w = a->w;
     t.csa = a->kind == CSAHCA_CSA; t.idx = sel; t.decode = 1;
     t.splits = L.splits; t.tiles_per_split = L.tiles_per_split; t.n_items = a->B * L.splits; t.gtile = L.gtile;
+    t.first_kernel = (a->kind != CSAHCA_CSA || a->idx_in) ? 1 : 0;
     t.out = nullptr; t.partial = partial;
     st = launch_attn_tc(t, a->kv_cache, (int64_t)a->B * a->N_cap, a->w > 0 ? a->win : nullptr,
                         (int64_t)a->B * a->w, s, a->kind == CSAHCA_CSA ? "attn_decode_csa_tc" : "attn_decode_hca_tc");

@@ -171,8 +171,8 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  griddep_launch_dependents();
   griddep_wait();                                  // keys may come from this stream's compress kernel
+  griddep_launch_dependents();
 
   if (warp == 8 || warp == 11) {
     // ------------------------------------------------------------ producers

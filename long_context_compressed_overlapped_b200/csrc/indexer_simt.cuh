@@ -28,8 +28,8 @@ __device__ __forceinline__ int visible_count(int t, int m, int N) {
 
 template <typename TQ, typename TK, bool kFP8>
 __global__ void __launch_bounds__(256) indexer_scores_simt(IndexerParams p) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ float smem_idx[];
   float* qs = smem_idx;                       // [HI * dI]
   float* ws = qs + p.HI * p.dI;               // [HI]

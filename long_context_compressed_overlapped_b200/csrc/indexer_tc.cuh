@@ -126,8 +126,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  griddep_launch_dependents();
   griddep_wait();                                  // keys may come from this stream's compress kernel
+  griddep_launch_dependents();
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer

@@ -124,8 +124,8 @@ __host__ __device__ __forceinline__ int kslot(int j) { return j + (j >> 5); }
 __host__ __device__ __forceinline__ int topk_rows_smem_bytes(int n) { return (kslot(n) + 1) * 4; }
 
 __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(TopkParams p) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ uint32_t keys[];           // order keys of the row at kslot(j)
   __shared__ uint32_t hist[kTopkSubHist * 256];
   __shared__ int warp_buf[72];

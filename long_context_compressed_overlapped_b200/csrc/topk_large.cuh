@@ -68,15 +68,15 @@ __device__ __forceinline__ int topk_visible(const TopkLargeParams& p, int row) {
 // programmatic dependent launches is not broken; it writes only after the
 // previous kernel has completed.
 __global__ void __launch_bounds__(256) zero16_kernel(uint4* p, int64_t n16) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (int64_t)gridDim.x * blockDim.x)
     p[i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 __global__ void __launch_bounds__(512) topk_hist_kernel(TopkLargeParams p) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   __shared__ uint32_t h[kHistBins];
   const int row = blockIdx.x / p.slices, slice = blockIdx.x % p.slices;
   const int v = topk_visible(p, row);
@@ -254,8 +254,8 @@ __device__ __forceinline__ void sort1024_block(int* a) {
 }
 
 __global__ void __launch_bounds__(kTopkSelectThreads, 2) topk_select_kernel(TopkLargeParams p) {
-  griddep_launch_dependents();
   griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ uint32_t bm_sel[];               // [words] taken, then [words] ties
   __shared__ uint32_t sh[1024];
   __shared__ int warp_buf[72];
