@@ -1,0 +1,49 @@
+"""One decode_1m layer, repeated, for a profiler to capture.
+
+    python -m long_context_compressed_overlapped_b200.profile_case csa --calls 4
+    python -m long_context_compressed_overlapped_b200.profile_case hca --calls 4
+    python -m long_context_compressed_overlapped_b200.profile_case indexer --calls 4
+
+``csa``: one CSA decode layer through ``compressed_attn_decode`` (indexer with
+e4m3 keys, top-k select, attention, combine); ``hca``: one HCA decode layer
+(attention, combine); ``indexer``: ``indexer_topk`` on the CSA layer's indexer
+inputs.  Four sequences at a 1,048,576-token context: 262,144 CSA entries
+(1 GB of bf16 rows, 134 MB of e4m3 indexer keys) or 8,192 HCA entries per
+sequence; about 1.3 GB on the device.  Inputs are the seeded synthetic draw of
+the decode_1m workload.  The process exits non-zero if a bounded device wait
+gave up.
+"""
+
+import argparse
+import sys
+
+import torch
+
+from . import api, synth
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("case", choices=("csa", "hca", "indexer"))
+    ap.add_argument("--calls", type=int, default=4)
+    a = ap.parse_args(argv)
+    wl = synth.WORKLOADS["decode_1m"]
+    kind = "hca" if a.case == "hca" else "csa"
+    L = synth.decode_inputs(wl, "cuda", ctx=wl.ctx, B=wl.B, layers=(kind,))[0]
+    for _ in range(a.calls):
+        if a.case == "indexer":
+            api.indexer_topk(L["qI"][:, None], L["w"][:, None], L["kI"], L["pos"][:, None], L["m"], wl.k,
+                             kI_scale=L["kI_scale"])
+        else:
+            kw = dict(m=L["m"], rope_dims=wl.r, q_gain=L["q_gain"])
+            if kind == "csa":
+                kw.update(k=wl.k, qI=L["qI"], wI=L["w"], kI=L["kI"], kI_scale=L["kI_scale"])
+            api.compressed_attn_decode(kind, L["q"], L["pos"], L["kv"], L["win"], L["sinks"], **kw)
+    torch.cuda.synchronize()
+    err = api.device_error()
+    print(f"profile_case {a.case}: {a.calls} calls, device error {err}")
+    return 1 if err else 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
