@@ -64,10 +64,11 @@ __device__ __forceinline__ int attn_visible(const AttnTcParams& p, int t) {
   return (int)(v < p.N ? v : p.N);
 }
 
+template <bool kDecode>
 __device__ __forceinline__ AttnItem attn_item(const AttnTcParams& p, int id) {
   AttnItem it;
   int qid;
-  if (p.decode) { qid = id / p.splits; it.split = id % p.splits; }
+  if (kDecode) { qid = id / p.splits; it.split = id % p.splits; }
   else {
     // HCA prefill: latest queries (most tiles) first; CSA: all alike.
     qid = p.csa ? id : (p.n_items - 1 - id);
@@ -75,11 +76,11 @@ __device__ __forceinline__ AttnItem attn_item(const AttnTcParams& p, int id) {
   }
   it.b = qid / p.nq;
   it.qi = qid % p.nq;
-  it.t = p.decode ? p.pos[it.b] : it.qi;
+  it.t = kDecode ? p.pos[it.b] : it.qi;
   it.ncomp_tiles = p.csa ? (p.k + p.gtile - 1) / p.gtile : (attn_visible(p, it.t) + 127) / 128;
   it.nwin_tiles = (p.w + 127) / 128;
   const int total = it.ncomp_tiles + it.nwin_tiles;
-  if (p.decode) {
+  if (kDecode) {
     it.tile0 = it.split * p.tiles_per_split;
     it.tile1 = min(total, it.tile0 + p.tiles_per_split);
   } else {
@@ -89,6 +90,7 @@ __device__ __forceinline__ AttnItem attn_item(const AttnTcParams& p, int id) {
   return it;
 }
 
+template <bool kDecode>
 __device__ __forceinline__ AttnTile attn_tile(const AttnTcParams& p, const AttnItem& it, int tile) {
   AttnTile T;
   if (tile < it.ncomp_tiles) {
@@ -109,7 +111,7 @@ __device__ __forceinline__ AttnTile attn_tile(const AttnTcParams& p, const AttnI
     const int wt = tile - it.ncomp_tiles;
     T.src = 2;
     T.list_off = 0;
-    if (p.decode) {
+    if (kDecode) {
       // ring slots [wt*128, wt*128 + 128); slot s is valid iff it holds a
       // position in [pos - w + 1, pos] that is >= 0
       T.row0 = it.b * p.w + wt * 128;
@@ -214,6 +216,7 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+template <bool kDecode>
 __global__ void __launch_bounds__(kAttnTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_constant__ CUtensorMap win_rows,
                const __grid_constant__ CUtensorMap q_rows, const __grid_constant__ CUtensorMap part_rows,
@@ -292,7 +295,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     uint32_t tcount = 0, icount = 0;
     bool stop = false;                       // warp-uniform
     for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
-      const AttnItem it = attn_item(p, id);
+      const AttnItem it = attn_item<kDecode>(p, id);
       if (it.tile1 <= it.tile0) continue;
       if (pw == 0) {
         // raw Q of this item into the Q buffer once the previous item's
@@ -313,13 +316,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       griddep_wait();
       if (lane == 0 && pw == 0) griddep_launch_dependents();
       for (int tile = it.tile0; tile < it.tile1 && !stop; ++tile, ++tcount) {
-        const AttnTile T = attn_tile(p, it, tile);
+        const AttnTile T = attn_tile<kDecode>(p, it, tile);
         const uint32_t ph = tcount & 1;
         // L2 prefetch of the next tile's rows: HBM streams while this tile is
         // processed, and the next tile's shared-memory loads hit L2 (the
         // current tile is loaded right away, so it is not prefetched)
         if (pw == 0 && tile + 1 < it.tile1) {
-          const AttnTile Tn = attn_tile(p, it, tile + 1);
+          const AttnTile Tn = attn_tile<kDecode>(p, it, tile + 1);
           if (Tn.src == 0) {
             const int* L = p.idx + ((int64_t)it.b * p.nq + it.qi) * p.k + Tn.list_off;
 #pragma unroll
@@ -396,7 +399,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       uint32_t tcount = 0, icount = 0;
       bool stop = false;
       for (int id = blockIdx.x; id < p.n_items && !stop && !abort_flag; id += gridDim.x) {
-        const AttnItem it = attn_item(p, id);
+        const AttnItem it = attn_item<kDecode>(p, id);
         if (it.tile1 <= it.tile0) continue;
         if (!mbar_wait(&bar_q_full, icount & 1, &abort_flag)) break;
         ++icount;
@@ -430,14 +433,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       uint32_t tcount = 0;
       bool stop = false;
       for (int id = blockIdx.x; id < p.n_items && !stop && !abort_flag; id += gridDim.x) {
-        const AttnItem it = attn_item(p, id);
+        const AttnItem it = attn_item<kDecode>(p, id);
         for (int tile = it.tile0; tile < it.tile1; ++tile, ++tcount) {
           const uint32_t ph = tcount & 1;
           if (!mbar_wait(&bar_p_full, ph, &abort_flag)) { stop = true; break; }
           tc_fence_after();
           const bool first = tile == it.tile0;
           // key steps past the tile's last valid row hold P = 0 and are skipped
-          const int hi = attn_tile(p, it, tile).hi;
+          const int hi = attn_tile<kDecode>(p, it, tile).hi;
           const int nks = hi <= 16 ? 1 : min(8, (hi + 15) >> 4);
           // M-tile by M-tile, so that chunk pair (2 mt, 2 mt + 1) is released
           // for the next tile's loads as soon as its MMAs complete
@@ -480,7 +483,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     if (st < p.rope_dims / 2) theta_s[st] = rope_theta(st, p.rope_dims, p.rope_base);
     const bool gain_ones = softmax_all256(ones);
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
-      const AttnItem it = attn_item(p, id);
+      const AttnItem it = attn_item<kDecode>(p, id);
       const bool empty = it.tile1 <= it.tile0;
       bool bad = false;                      // uniform over the group; both groups leave together
       // ---- query prologue.  RoPE is linear and the RMSNorm factor is one
@@ -590,7 +593,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
         if (bad) continue;
         const uint32_t ph = tcount & 1;
         const bool first = tile == it.tile0;
-        const AttnTile T = attn_tile(p, it, tile);
+        const AttnTile T = attn_tile<kDecode>(p, it, tile);
         bool valid = tid >= T.lo && tid < T.hi;
         if (valid && T.src == 0) {
           const int e = __ldg(p.idx + ((int64_t)it.b * p.nq + it.qi) * p.k + T.list_off + tid);
@@ -715,7 +718,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       }
       bad = softmax_any256(bad);             // the output stage is entered by both groups or neither
       if (!bad) {
-        if (p.decode) {
+        if (kDecode) {
           // partial block of (query, split): m[H] (log2 units) and l[H] in
           // fp32, then O / l as fp16 [D][H] (a thread writes its dim's 32
           // heads, 64 contiguous bytes, straight from TMEM); an empty split

@@ -658,11 +658,14 @@ int launch_attn_tc(const AttnTcParams& p, const void* kv_comp, int64_t comp_rows
                          (uint64_t)p.B * p.nq * p.splits * kTcPartialRows, kAttnH, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return CSAHCA_ERR_LAUNCH;
   const int smem = AttnSmem::TOTAL;
-  cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  // decode and prefill are separate instances: each carries only its own
+  // epilogue (a smaller kernel stalls less on instruction fetch)
+  auto kern = p.decode ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   if (grid <= 0) return CSAHCA_OK;
   CSAHCA_TRACE(name, s);
-  launch_k(attn_tc_kernel, dim3(grid), dim3(kAttnTcThreads), smem, s, m_rows, m_win, m_q, m_part, p);
+  launch_k(kern, dim3(grid), dim3(kAttnTcThreads), smem, s, m_rows, m_win, m_q, m_part, p);
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
 }
