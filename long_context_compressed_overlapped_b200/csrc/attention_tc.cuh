@@ -43,6 +43,8 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units
 struct AttnTcParams {
   const __nv_bfloat16* q; const float* q_gain; const float* sinks; const int* pos;
   const __nv_bfloat16* kv_comp_ptr;  // [B * N, D] compressed rows (gather source)
+  const __nv_bfloat16* win_ptr;      // window rows (the window tensor map's memory)
+  int64_t comp_rows_total, win_rows_total;   // rows behind kv_comp_ptr / win_ptr
   int q_norm; float eps; float scale_log2; int rope_dims; double rope_base;
   int B, nq, N, m, k, w;
   int csa;                      // 1: keys = idx rows; 0: every visible entry
@@ -318,25 +320,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       for (int tile = it.tile0; tile < it.tile1 && !stop; ++tile, ++tcount) {
         const AttnTile T = attn_tile<kDecode>(p, it, tile);
         const uint32_t ph = tcount & 1;
-        // L2 prefetch of the next tile's rows: HBM streams while this tile is
-        // processed, and the next tile's shared-memory loads hit L2 (the
-        // current tile is loaded right away, so it is not prefetched)
-        if (pw == 0 && tile + 1 < it.tile1) {
-          const AttnTile Tn = attn_tile<kDecode>(p, it, tile + 1);
-          if (Tn.src == 0) {
-            const int* L = p.idx + ((int64_t)it.b * p.nq + it.qi) * p.k + Tn.list_off;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int j = lane + 32 * e;
-              if (j < Tn.hi) {
-                const int v = __ldg(L + j);
-                if (v >= 0 && v < p.N) bulk_prefetch_l2(p.kv_comp_ptr + ((int64_t)it.b * p.N + v) * kAttnD, kAttnD * 2);
-              }
-            }
-          } else if (lane < kAttnChunks && Tn.row0 >= 0) {
-            tma_prefetch_l2_3d(Tn.src == 1 ? &comp_rows : &win_rows, 0, Tn.row0, lane);
-          }
-        }
         if (T.src == 0) {
           // selected rows of this tile (clamped; masked later by the softmax)
           const int* L = p.idx + ((int64_t)it.b * p.nq + it.qi) * p.k + T.list_off;
@@ -379,6 +362,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
             } else {
               mbar_arrive(&bar_kfull[c]);
             }
+          }
+        }
+        // L2 prefetch of the next tile's rows, queued after this tile's
+        // loads: HBM streams while this tile is processed, and the next
+        // tile's loads hit L2.  Contiguous rows: one bulk prefetch (an SM
+        // completes about one TMA op per 580 cycles, so not one per chunk);
+        // gathered rows: line prefetches from the lanes (no TMA op per row)
+        if (!stop && pw == 0 && tile + 1 < it.tile1) {
+          const AttnTile Tn = attn_tile<kDecode>(p, it, tile + 1);
+          if (Tn.src == 0) {
+            const int* L = p.idx + ((int64_t)it.b * p.nq + it.qi) * p.k + Tn.list_off;
+            for (int j = lane >> 3; j < Tn.hi; j += 4) {
+              const int v = __ldg(L + j);
+              if (v >= 0 && v < p.N)
+                prefetch_l2_line(p.kv_comp_ptr + ((int64_t)it.b * p.N + v) * kAttnD + (lane & 7) * 64);
+            }
+          } else if (lane == 0 && Tn.row0 >= 0) {
+            const int64_t total = Tn.src == 1 ? p.comp_rows_total : p.win_rows_total;
+            const int64_t rows = min((int64_t)128, total - Tn.row0);
+            if (rows > 0)
+              bulk_prefetch_l2((Tn.src == 1 ? p.kv_comp_ptr : p.win_ptr) + (int64_t)Tn.row0 * kAttnD,
+                               (uint32_t)(rows * kAttnD * 2));
           }
         }
       }

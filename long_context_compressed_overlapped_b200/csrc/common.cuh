@@ -104,6 +104,10 @@ __device__ __forceinline__ void rope_cos_sin(double pos, int j, int r, double ba
 __host__ __device__ __forceinline__ int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // L2 prefetch of `bytes` contiguous bytes (16-byte aligned address, multiple of 16).
+// One 128-byte line into L2 (a plain load-unit prefetch, no TMA op).
+__device__ __forceinline__ void prefetch_l2_line(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }

@@ -637,8 +637,12 @@ bool attn_tc_shape_ok(int dtype, int H, int d, int rope_dims, int64_t comp_rows,
          win_rows >= 128;
 }
 
-int launch_attn_tc(const AttnTcParams& p, const void* kv_comp, int64_t comp_rows, const void* win,
+int launch_attn_tc(const AttnTcParams& p_in, const void* kv_comp, int64_t comp_rows, const void* win,
                    int64_t win_rows, cudaStream_t s, const char* name) {
+  AttnTcParams p = p_in;
+  p.win_ptr = static_cast<const __nv_bfloat16*>(win ? win : kv_comp);
+  p.comp_rows_total = comp_rows;
+  p.win_rows_total = win ? win_rows : comp_rows;
   // rows of d = 512 bf16 seen as [chunk 8][row][64]: a key box is one chunk
   // of 128 rows (16 KB); the query box is all 8 chunks x 64 heads (64 KB),
   // landing chunk-major with the 128-byte swizzle as the MMA operand wants it
