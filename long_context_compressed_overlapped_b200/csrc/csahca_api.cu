@@ -424,6 +424,7 @@ int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* score
   IdxTcParams p;
   memset(&p, 0, sizeof(p));
   p.hist = hist;
+  p.first_kernel = hist ? 0 : 1;           // with histograms, the zeroing kernel runs first
   p.counters = counters;
   p.k = a->k;
   p.w = a->w; p.kI_scale = a->kI_scale; p.q_pos = a->q_pos;

@@ -171,8 +171,14 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  griddep_wait();                                  // keys may come from this stream's compress kernel
-  griddep_launch_dependents();
+  // As a call's first kernel, nothing is read before the wait (the keys may
+  // come from a compress kernel queued just before).  After the scratch
+  // zeroing kernel of the same call, the key loads and MMAs start at once;
+  // the epilogue waits (before the histograms) and then signals.
+  if (p.first_kernel) {
+    griddep_wait();
+    griddep_launch_dependents();
+  }
 
   if (warp == 8 || warp == 11) {
     // ------------------------------------------------------------ producers
@@ -270,6 +276,7 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
       const IdxItem it = idx_item<1>(p, id);
       const int row = it.b * p.q_count + (it.q0 - p.q_begin);
       if (it.kt1 <= it.kt0) {
+        if (!p.first_kernel) griddep_wait();
         if (do_hist) idx_row_done(p, row, scan_s, &row_flag);   // an empty item still counts
         continue;
       }
@@ -330,6 +337,10 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
         }
       }
       group_sync(bar_id);                            // sW[g] complete
+      if (!p.first_kernel) {
+        griddep_wait();                              // the histograms and counters are zeroed
+        griddep_launch_dependents();
+      }
       const int v = idx_visible(p, it.b, it.q0);
       float* srow = p.scores + ((int64_t)it.b * p.q_count + (it.q0 - p.q_begin)) * p.score_row_stride;
       for (int kt = it.kt0; kt < it.kt1; ++kt, ++acc_iter) {

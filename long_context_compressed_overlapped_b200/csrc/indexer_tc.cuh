@@ -36,6 +36,8 @@ struct IdxTcParams {
   uint32_t* counters;         // with hist: [rows][8] top-k counters (threshold bin stored here)
   int items_per_row;          // with hist: work items per row
   int k;                      // with hist: the top-k size
+  int first_kernel;           // 0: an earlier kernel of the call precedes (the FP8 decode scan may
+                              // then load keys before its wait; the keys are call inputs)
 };
 
 template <int QT, int HI, bool kFP8>
