@@ -32,7 +32,12 @@
 
 namespace csahca {
 
-constexpr int kAttnTcThreads = 384;   // warps 0-7 softmax (two head groups), 8-9 loads, 10-11 MMA
+// Warps 0-7 softmax (two head groups), then the producer warps, then the S
+// and P.V MMA issuers.  Decode: 2 producers (384 threads); prefill: 6 (512
+// threads), since a gather of selected rows runs at about 8 B/cycle per
+// issuing warp.
+template <bool kDecode> __host__ __device__ constexpr int attn_producers() { return kDecode ? 2 : 6; }
+template <bool kDecode> __host__ __device__ constexpr int attn_threads() { return 32 * (10 + attn_producers<kDecode>()); }
 constexpr int kAttnH = 64;          // heads (MMA N of both products)
 constexpr int kAttnD = 512;         // head dim
 constexpr int kAttnChunks = kAttnD / 64;
@@ -219,7 +224,7 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 }
 
 template <bool kDecode>
-__global__ void __launch_bounds__(kAttnTcThreads, 1)
+__global__ void __launch_bounds__(attn_threads<kDecode>(), 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_constant__ CUtensorMap win_rows,
                const __grid_constant__ CUtensorMap q_rows, const __grid_constant__ CUtensorMap part_rows,
                AttnTcParams p) {
@@ -242,13 +247,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
   __shared__ float rope_cs[64], rope_sn[64];
   __shared__ double theta_s[64];                   // RoPE frequency of pair j
   __shared__ __align__(16) float gain_s[kAttnD];
-  __shared__ int rows_s[2][128];
+  __shared__ int rows_s[attn_producers<kDecode>()][128];
   __shared__ int need_rescale[2];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kNP = attn_producers<kDecode>();
+  constexpr int kWarpS = 8 + kNP, kWarpPV = 9 + kNP;
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (int c = 0; c < kAttnChunks; ++c) { mbar_init(&bar_kfull[c], 32); mbar_init(&bar_kempty[c], 1); }
+    for (int c = 0; c < kAttnChunks; ++c) { mbar_init(&bar_kfull[c], kNP == 2 ? 32 : 32 * kNP); mbar_init(&bar_kempty[c], 1); }
     mbar_init(&bar_q_raw, 1);
     mbar_init(&bar_q_empty, 1);
     mbar_init(&bar_q_full, 256);
@@ -259,7 +266,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     mbar_init(&bar_done, 2);                       // both MMA issuers
     mbar_fence_init();
   }
-  if (warp == 10) tmem_alloc(&tmem_base_sh, 512);
+  if (warp == kWarpS) tmem_alloc(&tmem_base_sh, 512);
   if (p.gtile < 128) {
     // rows [gtile, 128) of the key buffer are never written by a gathered
     // tile; zeros there keep the score and P.V MMAs finite (P = 0 there)
@@ -287,9 +294,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     griddep_launch_dependents();
   }
 
-  if (warp == 8 || warp == 9) {
+  // (the decode instance keeps this exact form of the role test: its code
+  // runs once per CTA, fetched cold, and an equivalent range test compiled
+  // to a layout measured 4 us slower per launch)
+  if (kDecode ? (warp == 8 || warp == 9) : (warp >= 8 && warp < 8 + kNP)) {
     // ------------------------------------------------------------ producers
-    // warp 8 loads chunks 0,1,4,5 (and the raw Q); warp 9 chunks 2,3,6,7
+    // decode, two producers: warp 8 loads chunks 0,1,4,5 (and the raw Q),
+    // warp 9 chunks 2,3,6,7, and a chunk barrier expects 32 arrivals.
+    // Prefill, six: every producer loads its share of every chunk (gathered
+    // rows: copy instruction j, rows 4j..4j+3, goes to warp j mod 6;
+    // contiguous rows: chunk c's box is issued by warp c mod 6), and a chunk
+    // barrier expects 32 x 6 arrivals; warp 8 also loads the raw Q
     const int pw = warp - 8;
     tma_prefetch_desc(&comp_rows);
     tma_prefetch_desc(&win_rows);
@@ -332,8 +347,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
           }
           __syncwarp();
         }
-        for (int cc = 0; cc < kAttnChunks / 2; ++cc) {
-          const int c = 4 * (cc >> 1) + 2 * pw + (cc & 1);
+        // two producers (decode): warp pw owns chunks {0,1,4,5} or {2,3,6,7};
+        // more (prefill): every producer takes a share of every chunk
+        constexpr int kChunksPerWarp = kNP == 2 ? kAttnChunks / 2 : kAttnChunks;
+        for (int cc = 0; cc < kChunksPerWarp; ++cc) {
+          const int c = kNP == 2 ? 4 * (cc >> 1) + 2 * pw + (cc & 1) : cc;
           int ok = 1;
           if (lane == 0) ok = mbar_wait(&bar_kempty[c], ph ^ 1, &abort_flag);
           ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -347,16 +365,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
             const int piece = lane & 7, rg = lane >> 3;
             const __nv_bfloat16* src = p.kv_comp_ptr + c * 64 + piece * 8;
             const int nj = p.gtile >> 2;
+            if constexpr (kNP == 2) {
 #pragma unroll 8
-            for (int j = 0; j < nj; ++j) {
-              const int r = 4 * j + rg;
-              cp_async16(dst + sw128_offset(r, piece * 16), src + (int64_t)rows_s[pw][r] * kAttnD);
+              for (int j = 0; j < nj; ++j) {
+                const int r = 4 * j + rg;
+                cp_async16(dst + sw128_offset(r, piece * 16), src + (int64_t)rows_s[pw][r] * kAttnD);
+              }
+            } else {
+#pragma unroll
+              for (int jj = 0; jj < (32 + kNP - 1) / kNP; ++jj) {
+                const int j = pw + jj * kNP;
+                if (j < nj) {
+                  const int r = 4 * j + rg;
+                  cp_async16(dst + sw128_offset(r, piece * 16), src + (int64_t)rows_s[pw][r] * kAttnD);
+                }
+              }
             }
             cp_async_arrive_noinc(&bar_kfull[c]);
           } else {
             // contiguous rows: one 16 KB box per chunk, so the score MMAs of
             // a chunk start as soon as it lands
-            if (lane == 0) {
+            if (lane == 0 && (kNP == 2 || c % kNP == pw)) {
               mbar_expect_tx(&bar_kfull[c], AttnSmem::K_CHUNK);
               tma_load_3d(dst, T.src == 1 ? &comp_rows : &win_rows, 0, T.row0, c, &bar_kfull[c]);
             } else {
@@ -393,7 +422,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     if (lane == 0 && tcount > 0)
       for (int c = 0; c < kAttnChunks; ++c) mbar_wait(&bar_kfull[c], (tcount - 1) & 1, &abort_flag);
     if (pw == 0 && lane == 0 && icount > 0) mbar_wait(&bar_q_raw, (icount - 1) & 1, &abort_flag);
-  } else if (warp == 10) {
+  } else if (warp == kWarpS) {
     // ------------------------------------------------------------ S MMA issuer
     // (a separate thread issues the P.V MMAs, so the S MMAs of tile t+1 go out
     // while those of P.V(t) still do)
@@ -429,7 +458,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       umma_commit(&bar_done);
       mbar_wait(&bar_done, 0, &abort_flag);
     }
-  } else if (warp == 11) {
+  } else if (warp == kWarpPV) {
     // ------------------------------------------------------------ P.V MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_pv = umma_idesc_bf16(128, kAttnH, 1, 1);
@@ -842,7 +871,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 10) tmem_dealloc(tmem, 512);
+  if (warp == kWarpS) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------------------

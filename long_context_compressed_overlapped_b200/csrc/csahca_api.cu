@@ -670,7 +670,8 @@ int launch_attn_tc(const AttnTcParams& p_in, const void* kv_comp, int64_t comp_r
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   if (grid <= 0) return CSAHCA_OK;
   CSAHCA_TRACE(name, s);
-  launch_k(kern, dim3(grid), dim3(kAttnTcThreads), smem, s, m_rows, m_win, m_q, m_part, p);
+  launch_k(kern, dim3(grid), dim3(p.decode ? attn_threads<true>() : attn_threads<false>()), smem, s, m_rows,
+           m_win, m_q, m_part, p);
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
 }
