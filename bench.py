@@ -425,6 +425,7 @@ def main():
     stream = torch.cuda.Stream(device=dev)
     wl = synth.WORKLOADS[args.workload]
     layers = synth.decode_inputs(runtime.shard_workload(wl, rank), dev)
+    io = runtime.StepIO(layers, dev)            # per-step inputs / outputs in one arena each
     eager = runtime.DecodeStep(wl, layers, stream)
     step = eager
     launch_mode = "eager"
@@ -472,22 +473,18 @@ def main():
     step_bytes = decode_step_bytes(wl, wl.ctx)
     step_frac = step_bytes / (ms_per_step / 1000.0) / 1e9 / pk["hbm_gbs"]
 
-    # end to end: pinned host inputs copied in and outputs read back per step
-    host_in, host_out = [], []
-    for L in layers:
-        for name in ("q", "qI", "w", "pos"):
-            if name in L:
-                host_in.append((L[name], L[name].cpu().pin_memory()))
-        host_out.append((L["out"], torch.empty(L["out"].shape, dtype=L["out"].dtype).pin_memory()))
-    h2d = sum(h.numel() * h.element_size() for _, h in host_in)
-    d2h = sum(h.numel() * h.element_size() for _, h in host_out)
+    # end to end: the step's inputs copied in from pinned host memory and its
+    # outputs read back, one copy each way (the layers' tensors are views of
+    # the two arenas)
+    host_inp = io.inp.cpu().pin_memory()
+    host_outp = torch.empty(io.out.shape, dtype=io.out.dtype).pin_memory()
+    h2d = io.inp.numel()
+    d2h = io.out.numel()
 
     def e2e_step():
-        for dv, hv in host_in:
-            dv.copy_(hv, non_blocking=True)
+        io.inp.copy_(host_inp, non_blocking=True)
         step()
-        for dv, hv in host_out:
-            hv.copy_(dv, non_blocking=True)
+        host_outp.copy_(io.out, non_blocking=True)
 
     with torch.cuda.stream(stream):
         e2e_step()

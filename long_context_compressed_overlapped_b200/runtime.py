@@ -35,6 +35,42 @@ def max_over_ranks(x: float, group=None) -> float:
     return float(t.item())
 
 
+class StepIO:
+    """The per-step inputs of every layer (new query, indexer query and
+    weights, positions) placed in one device arena, and the outputs in
+    another: a caller then moves a step's data with one copy each way.  The
+    layers' tensors become views of the arenas (same dtype and shape, slots
+    256-byte aligned); make the DecodeStep after this."""
+
+    IN_NAMES = ("q", "qI", "w", "pos")
+
+    def __init__(self, layers, device):
+        def arena(tensors):
+            offs, off = [], 0
+            for t in tensors:
+                offs.append(off)
+                off = (off + t.numel() * t.element_size() + 255) // 256 * 256
+            return torch.empty(max(off, 256), dtype=torch.uint8, device=device), offs
+
+        def view(buf, off, dtype, shape):
+            n = 1
+            for x in shape:
+                n *= x
+            nbytes = n * torch.empty((), dtype=dtype).element_size()
+            return buf[off:off + nbytes].view(dtype).view(shape)
+
+        ins = [(L, n) for L in layers for n in self.IN_NAMES if L.get(n) is not None]
+        self.inp, offs = arena([L[n] for L, n in ins])
+        for (L, n), o in zip(ins, offs):
+            v = view(self.inp, o, L[n].dtype, tuple(L[n].shape))
+            v.copy_(L[n])
+            L[n] = v
+        outs = [torch.empty_like(L["q"]) for L in layers]
+        self.out, offs = arena(outs)
+        for L, t, o in zip(layers, outs, offs):
+            L["out"] = view(self.out, o, t.dtype, tuple(t.shape))
+
+
 class DecodeStep:
     """One decode step over every layer of `layers` (as made by
     synth.decode_inputs): the C-ABI argument structs and workspaces are
@@ -49,7 +85,7 @@ class DecodeStep:
             if L["kind"] == "csa":
                 kw.update(k=wl.k, qI=L["qI"], wI=L["w"], kI=L["kI"], kI_scale=L["kI_scale"])
             args, out, keep = api.decode_args(L["kind"], L["q"], L["pos"], L["kv"], L["win"],
-                                              L["sinks"], **kw)
+                                              L["sinks"], out=L.get("out"), **kw)
             nbytes = self.lib.csahca_decode_workspace_size(C.byref(args))
             ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=L["q"].device)
             args.workspace = ws.data_ptr()

@@ -55,3 +55,28 @@ def test_two_gloo_ranks_shard_and_reduce():
 
 def test_single_process_max_is_identity():
     assert runtime.max_over_ranks(3.5) == 3.5
+
+
+def test_step_io_arenas_hold_every_input_and_output():
+    """StepIO moves each layer's per-step inputs into one arena (same values,
+    dtypes and shapes, 256-byte aligned slots) and gives every layer an output
+    view of a second arena: a step's data then moves with one copy each way."""
+    g = torch.Generator().manual_seed(0)
+    layers = [
+        dict(q=torch.randn(4, 64, 512, generator=g).bfloat16(), qI=torch.randn(4, 64, 128, generator=g).bfloat16(),
+             w=torch.randn(4, 64, generator=g), pos=torch.arange(4, dtype=torch.int32)),
+        dict(q=torch.randn(4, 64, 512, generator=g).bfloat16(), pos=torch.arange(4, 8, dtype=torch.int32)),
+    ]
+    ref = [{k: v.clone() for k, v in L.items()} for L in layers]
+    io = runtime.StepIO(layers, "cpu")
+    base_in, base_out = io.inp.data_ptr(), io.out.data_ptr()
+    for L, R in zip(layers, ref):
+        for k, v in R.items():
+            assert torch.equal(L[k], v) and L[k].dtype == v.dtype and L[k].shape == v.shape
+            off = L[k].data_ptr() - base_in
+            assert 0 <= off < io.inp.numel() and off % 256 == 0
+        off = L["out"].data_ptr() - base_out
+        assert L["out"].shape == R["q"].shape and 0 <= off < io.out.numel() and off % 256 == 0
+    # the arena is the data: writing it changes the layers' inputs
+    io.inp.zero_()
+    assert all(float(L["q"].float().abs().sum()) == 0.0 for L in layers)
