@@ -57,11 +57,24 @@ Readings where the pages are silent (each is a fixed constant of this code):
   R18 indexer queries stay in their own dtype; only keys are e4m3.
   R20 decode caches hold final rows; the window ring holds final rows, slot
       (p mod w) holding position p.
+  R21 the decode compressor stores a new e4m3 indexer key with the same
+      per-128 rule as R17, every step in float32: scale = amax / 448 (1 for an
+      all-zero block), code = nearest e4m3 of x / scale, ties to even,
+      saturating at 448.
+  R22 between decode steps a compressor keeps the raw streams of its last
+      2m (CSA) or m' (HCA) tokens, token p in ring slot p mod 2m (or p mod m');
+      the window row and the compressed rows share one norm gain.
 
 Pins (what checks each function against something other than itself, in
 ``tests/test_oracle_pins.py`` and ``tests/golden/``):
 
   e4m3_decode           all 256 codes against torch's float8_e4m3fn cast.
+  e4m3_encode           torch's round-to-nearest-even float8_e4m3fn cast on
+                        random values and on every midpoint between codes;
+                        saturation closed form; decode(encode(v)) = v.
+  decode_compress_step  run token by token from position 0, it emits exactly
+                        the rows csa_pool / hca_pool + finish_rows give for the
+                        whole stream, and the window rows of finish_rows.
   csa_pool              hand-worked fixture; constant streams -> 1 (weights sum
                         to 1); equal logits -> plain mean; one-hot logits copy
                         the named token of the named stream/block; causality.
@@ -102,6 +115,38 @@ def e4m3_decode(codes: np.ndarray) -> np.ndarray:
     subnormal = np.ldexp(f / 8.0, -6)
     val = sign * np.where(e == 0, subnormal, normal)
     return np.where((e == 15) & (f == 7), np.nan, val)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Nearest e4m3 ("fn") code of each finite value: the magnitude code whose
+    decoded value is closest to |x|, ties to the code with an even last
+    mantissa bit, magnitudes beyond the largest finite one (448) saturating
+    to it, and the sign bit of x.  Written as the definition: a search over
+    the 127 finite magnitudes."""
+    x = np.asarray(x, np.float64)
+    mags = np.arange(127, dtype=np.uint8)                   # 0x00 .. 0x7E
+    vals = e4m3_decode(mags)
+    ax = np.minimum(np.abs(x), 448.0)
+    dist = np.abs(ax[..., None] - vals)                     # [..., 127]
+    best = dist.min(axis=-1, keepdims=True)
+    rank = np.where(dist == best, (mags & 1).astype(np.int64), 9)
+    code = mags[np.argmin(rank, axis=-1)]
+    return np.where(np.signbit(x), code | np.uint8(0x80), code).astype(np.uint8)
+
+
+def quantize_e4m3_rows_f32(x, block: int = 128):
+    """Per-block e4m3 storage of a key row as the decode compressor writes it
+    (reading R21): with every step in float32, scale = amax / 448 over each
+    ``block`` contiguous elements (1 where amax is 0) and code =
+    e4m3_encode(x / scale).  Returns (codes uint8 [..., d], scales f32
+    [..., d/block])."""
+    x = np.asarray(x, np.float32)
+    d = x.shape[-1]
+    xb = x.reshape(*x.shape[:-1], d // block, block)
+    amax = np.abs(xb).max(axis=-1)
+    scale = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    q = (xb / scale[..., None]).astype(np.float32)
+    return e4m3_encode(q).reshape(x.shape), scale
 
 
 def dequant_e4m3_rows(codes: np.ndarray, scales: np.ndarray, block: int = 128) -> np.ndarray:
@@ -207,6 +252,50 @@ def finish_rows(rows, positions, gain, r: int, base: float = ROPE_BASE,
     With normalize=False the norm is skipped (gain ignored)."""
     y = rms_norm(rows, gain) if normalize else np.asarray(rows, np.float64)
     return rope(y, np.asarray(positions), r, base)
+
+
+# ----------------------------------------------------------------------------
+# one decode step of the compressors  ("Paper Breakdown: DeepSeek-V4",
+# section 4, CSA KV Compression, HCA, Sliding window KV)
+# ----------------------------------------------------------------------------
+
+def decode_compress_step(kind: str, t: int, new, ring, biases, m: int, *, kv_raw=None,
+                         gain=None, r: int = 0, base: float = ROPE_BASE,
+                         normalize: bool = True):
+    """Fold the token at position t into one sequence's compressor state.
+
+    kind "csa": streams a, b, za, zb; kind "hca": a, za.  ``new`` maps each
+    stream name to the token's row [c]; ``ring`` maps it to [R, c] holding
+    token p in slot p % R for the R = 2m (csa) or m (hca) tokens before t.
+    ``biases`` = (bias_a, bias_b) ([m, c] each; bias_b None for hca).
+    Returns (ring', entry, window_row):
+      ring'       the ring with the new token in slot t % R (reading R22);
+      entry       None unless t completes block i = (t+1)/m - 1, else
+                  (i, pooled [c] before finishing, finished [c]) where the
+                  pooling is csa_pool / hca_pool over the tokens of block i
+                  (and block i-1) and finishing is finish_rows at i*m;
+      window_row  finish_rows(kv_raw, t) (None without kv_raw).
+    """
+    streams = ("a", "b", "za", "zb") if kind == "csa" else ("a", "za")
+    R = 2 * m if kind == "csa" else m
+    ring = {s: np.array(ring[s], np.float64, copy=True) for s in streams}
+    for s in streams:
+        ring[s][t % R] = np.asarray(new[s], np.float64)
+    entry = None
+    if (t + 1) % m == 0:
+        i = (t + 1) // m - 1
+        first = max(i - 1, 0) * m if kind == "csa" else i * m
+        toks = np.arange(first, (i + 1) * m)                  # the blocks entry i pools
+        seq = {s: ring[s][toks % R] for s in streams}
+        if kind == "csa":
+            pooled = csa_pool(seq["a"], seq["b"], seq["za"], seq["zb"], biases[0], biases[1], m)[-1]
+        else:
+            pooled = hca_pool(seq["a"], seq["za"], biases[0], m)[-1]
+        entry = (i, pooled, finish_rows(pooled, i * m, gain, r, base, normalize=normalize))
+    win_row = None
+    if kv_raw is not None:
+        win_row = finish_rows(kv_raw, t, gain, r, base, normalize=normalize)
+    return ring, entry, win_row
 
 
 # ----------------------------------------------------------------------------

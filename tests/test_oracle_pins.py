@@ -49,6 +49,51 @@ def test_e4m3_block_scales():
     assert np.array_equal(x[:, 128:], base[:, 128:] * scales[:, 1:])
 
 
+def _e4m3_probe_values():
+    """float32 values across the e4m3 range: random magnitudes, every finite
+    code value, every midpoint between neighbouring codes (the ties), zero
+    and values past the subnormal range, with both signs."""
+    rng = np.random.default_rng(3)
+    mags = O.e4m3_decode(np.arange(127, dtype=np.uint8))
+    mids = (mags[:-1] + mags[1:]) / 2
+    rand = rng.uniform(0, 1, 4000) * np.exp2(rng.integers(-12, 9, 4000))
+    v = np.concatenate([mags, mids, np.clip(rand, 0, 448), [0.0, 2.0 ** -11, 2.0 ** -10, 1e-30]])
+    return np.concatenate([v, -v]).astype(np.float32)
+
+
+def check_e4m3_encode_matches_torch(encode):
+    x = _e4m3_probe_values()
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(encode(x.astype(np.float64)), ref)
+
+
+def test_e4m3_encode_round_to_nearest_even():
+    check_e4m3_encode_matches_torch(O.e4m3_encode)
+
+
+def test_e4m3_encode_saturates_and_round_trips():
+    assert list(O.e4m3_encode(np.array([448.0, 449.0, 480.0, 1e6, -500.0]))) == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE]
+    finite = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    assert np.array_equal(O.e4m3_encode(O.e4m3_decode(finite)), finite)
+
+
+def test_quantize_e4m3_rows_f32():
+    from long_context_compressed_overlapped_b200 import synth
+    rng = np.random.default_rng(4)
+    x = (rng.standard_normal((6, 256)) * np.exp2(rng.integers(-6, 6, (6, 1)))).astype(np.float32)
+    x[2, 128:] = 0.0                                        # an all-zero block: scale 1, codes 0
+    codes, scales = O.quantize_e4m3_rows_f32(x)
+    amax = np.abs(x.reshape(6, 2, 128)).max(axis=-1)
+    assert np.array_equal(scales, np.where(amax > 0, amax / np.float32(448), 1).astype(np.float32))
+    assert scales[2, 1] == 1.0 and not codes[2, 128:].any()
+    # the element of largest magnitude lands on +-448 (code 0x7E or 0xFE)
+    j = np.abs(x[0, :128]).argmax()
+    assert codes[0, j] & 0x7F == 0x7E
+    # the same rule as a torch float32 cast (the harness quantiser)
+    tc, ts = synth.quantize_e4m3_rows(torch.from_numpy(x))
+    assert np.array_equal(codes, tc.numpy()) and np.array_equal(scales, ts.numpy())
+
+
 # ----------------------------------------------------------- compressors ----
 
 def check_csa_golden(pool, fx):
@@ -396,6 +441,48 @@ def test_decode_equals_prefill(kind):
         np.testing.assert_allclose(od, o[p], rtol=1e-12, atol=1e-14)
 
 
+# ------------------------------------------------ decode compressor step ----
+
+def _decode_stream(kind, n, c, m, seed):
+    rng = np.random.default_rng(seed)
+    names = ("a", "b", "za", "zb") if kind == "csa" else ("a", "za")
+    st = {s: rng.standard_normal((n, c)) for s in names}
+    biases = (0.1 * rng.standard_normal((m, c)), 0.1 * rng.standard_normal((m, c)) if kind == "csa" else None)
+    return st, biases, rng.standard_normal((n, c)), rng
+
+
+def check_decode_compress_step(step, kind):
+    n, c, r = 40, 16, 4
+    m = 4 if kind == "csa" else 8
+    R = 2 * m if kind == "csa" else m
+    st, biases, kv_raw, rng = _decode_stream(kind, n, c, m, 7 if kind == "csa" else 8)
+    gain = 1 + 0.1 * rng.standard_normal(c)
+    ring = {s: rng.standard_normal((R, c)) * 1e3 for s in st}    # garbage before position 0
+    if kind == "csa":
+        pooled = O.csa_pool(st["a"], st["b"], st["za"], st["zb"], biases[0], biases[1], m)
+    else:
+        pooled = O.hca_pool(st["a"], st["za"], biases[0], m)
+    want = O.finish_rows(pooled, np.arange(pooled.shape[0]) * m, gain, r)
+    emitted = []
+    for t in range(n):
+        ring, entry, win = step(kind, t, {s: st[s][t] for s in st}, ring, biases, m,
+                                kv_raw=kv_raw[t], gain=gain, r=r)
+        np.testing.assert_allclose(win, O.finish_rows(kv_raw[t], t, gain, r), rtol=1e-13, atol=1e-13)
+        assert (entry is not None) == ((t + 1) % m == 0)
+        if entry is not None:
+            i, raw, fin = entry
+            assert i == (t + 1) // m - 1
+            np.testing.assert_allclose(raw, pooled[i], rtol=1e-13, atol=1e-13)
+            np.testing.assert_allclose(fin, want[i], rtol=1e-13, atol=1e-13)
+            emitted.append(i)
+    assert emitted == list(range(n // m))
+
+
+@pytest.mark.parametrize("kind", ["csa", "hca"])
+def test_decode_compress_step_equals_whole_stream(kind):
+    check_decode_compress_step(O.decode_compress_step, kind)
+
+
 # --------------------------------------------- planted mistakes are caught ----
 
 def test_pins_catch_planted_mistakes(golden_dir):
@@ -453,3 +540,30 @@ def test_pins_catch_planted_mistakes(golden_dir):
 
     with pytest.raises(AssertionError):
         check_e4m3_matches_torch(decode_bias_wrong)
+
+    def encode_ties_away(x):                                # ties away from zero
+        x = np.asarray(x, float)
+        c = O.e4m3_encode(x)
+        up = (c & 0x7F) < 0x7E
+        nxt = O.e4m3_decode(np.where(up, c + 1, c).astype(np.uint8))
+        tie = up & (np.abs(np.abs(nxt) - np.abs(x)) == np.abs(np.abs(x) - np.abs(O.e4m3_decode(c))))
+        return np.where(tie & (np.abs(x) > np.abs(O.e4m3_decode(c))), c + 1, c).astype(np.uint8)
+
+    with pytest.raises(AssertionError):
+        check_e4m3_encode_matches_torch(encode_ties_away)
+
+    def step_ring_not_kept(kind, t, new, ring, biases, m, **kw):      # new token never stored
+        _, entry, win = O.decode_compress_step(kind, t, new, ring, biases, m, **kw)
+        return ring, entry, win
+
+    def step_rope_at_last_token(kind, t, new, ring, biases, m, *, gain=None, r=0, **kw):
+        out_ring, entry, win = O.decode_compress_step(kind, t, new, ring, biases, m, gain=gain, r=r, **kw)
+        if entry is not None:
+            i, raw, _ = entry
+            entry = (i, raw, O.finish_rows(raw, t, gain, r))
+        return out_ring, entry, win
+
+    for kind in ("csa", "hca"):
+        for bad in (step_ring_not_kept, step_rope_at_last_token):
+            with pytest.raises(AssertionError):
+                check_decode_compress_step(bad, kind)
