@@ -219,7 +219,30 @@ def decode_bytes_per_kernel(wl, ctx):
         "topk_rows": B * (vc * 4 + k * 4),
         "attn_decode_csa": B * ((k + w) * d * 2 + qo),
         "attn_decode_hca": B * ((vh + w) * d * 2 + qo),
+        "decode_compress": sum(decode_compress_bytes(wl, kd, ctx) for kd in wl.layers) / len(wl.layers),
     }
+
+
+def decode_compress_bytes(wl, kind, pos):
+    """Algorithmic bytes of one decode_compress launch (B sequences, new token
+    at `pos`): the token's raw streams read and stored in the ring, its raw
+    window row read and the finished row written; when the token completes a
+    block, the other tokens of the pooled blocks (value and logit streams)
+    are read and the entry (and its indexer key) written."""
+    es = 4 if wl.dtype == "f32" else 2
+    m = wl.m if kind == "csa" else wl.m_hca
+    S = 4 if kind == "csa" else 2
+    per = 2 * S * wl.d * es + 2 * wl.d * es
+    if kind == "csa":
+        per += 2 * 4 * wl.dI * es
+    if (pos + 1) % m == 0:
+        i = (pos + 1) // m - 1
+        J = m if (kind == "hca" or i == 0) else 2 * m
+        per += (J - 1) * 2 * wl.d * es + wl.d * es
+        if kind == "csa":
+            key = wl.dI + 4 * (wl.dI // 128) if wl.fp8_keys else wl.dI * es
+            per += (J - 1) * 2 * wl.dI * es + key
+    return wl.B * per
 
 
 def decode_step_bytes(wl, ctx):
@@ -227,6 +250,7 @@ def decode_step_bytes(wl, ctx):
     per = decode_bytes_per_kernel(wl, ctx)
     tot = 0
     for kind in wl.layers:
+        tot += decode_compress_bytes(wl, kind, ctx)
         if kind == "csa":
             tot += per["indexer_scores"] + per["attn_decode_csa"]
         else:
@@ -243,6 +267,8 @@ def kernel_bytes_key(name):
         return "attn_decode_csa"
     if "decode_hca" in name:
         return "attn_decode_hca"
+    if name.startswith("decode_compress"):
+        return "decode_compress"
     return None
 
 
@@ -314,28 +340,63 @@ def blas_threads():
     return os.cpu_count()
 
 
-def oracle_decode_sequence(wl, layers, b):
-    """The oracle's decode step for sequence b over all layers."""
+def oracle_decode_sequence(wl, layers, b, sels=None, scores_out=None):
+    """The oracle's decode step for sequence b over all layers: per layer the
+    compressor step (new token into the ring, its window row, a new entry
+    when it completes a block), then the indexer top-k (CSA) and attention.
+    sels: optional per-layer selections used instead of the oracle's own
+    top-k (None entries keep it); scores_out: a list that receives each CSA
+    layer's indexer scores."""
     from oracle import csahca_oracle as O
 
     def npy(t):
         return t.detach().cpu().to(torch.float64).numpy() if t.dtype != torch.uint8 else t.cpu().numpy()
 
     outs = []
-    for L in layers:
+    for li, L in enumerate(layers):
         pos = int(L["pos"][b])
+        csa = L["kind"] == "csa"
+        m = L["m"]
+        names = ("a", "b", "za", "zb") if csa else ("a", "za")
+        cols = ("ca", "cb", "cza", "czb") if csa else ("ca", "cza")
+        ring = {s_: npy(L["ring"][b, :, j]) for j, s_ in enumerate(names)}
+        new = {s_: npy(L[c_][b]) for s_, c_ in zip(names, cols)}
+        biases = (npy(L["bias_a"]), npy(L["bias_b"]) if csa else None)
+        _, entry, win_row = O.decode_compress_step(L["kind"], pos, new, ring, biases, m,
+                                                   kv_raw=npy(L["kv_raw"][b]), gain=npy(L["kv_gain"]),
+                                                   r=wl.r)
+        win = npy(L["win"][b])
+        win[pos % wl.w] = win_row
+        kv = npy(L["kv"][b])
+        N_cap = kv.shape[0]
+        if entry is not None and entry[0] < N_cap:
+            kv[entry[0]] = entry[2]
         sel = None
-        if L["kind"] == "csa":
-            v = min(O.n_visible(pos, L["m"]), L["kv"].shape[1])
+        if csa:
+            v = min(O.n_visible(pos, m), N_cap)
             if L["kI_scale"] is not None:
                 K = O.dequant_e4m3_rows(npy(L["kI"][b, :v]), npy(L["kI_scale"][b, :v]))
             else:
                 K = npy(L["kI"][b, :v])
+            iring = {s_: npy(L["iring"][b, :, j]) for j, s_ in enumerate(names)}
+            inew = {s_: npy(L[c_][b]) for s_, c_ in zip(names, ("ia", "ib", "iza", "izb"))}
+            _, ientry, _ = O.decode_compress_step("csa", pos, inew, iring,
+                                                  (npy(L["ibias_a"]), npy(L["ibias_b"])), m,
+                                                  normalize=False)
+            if ientry is not None and ientry[0] < v:
+                key = ientry[1]
+                if L["kI_scale"] is not None:
+                    codes, scales = O.quantize_e4m3_rows_f32(key)
+                    key = O.dequant_e4m3_rows(codes, scales)
+                K[ientry[0]] = key
             s = O.indexer_scores(npy(L["qI"][b]), npy(L["w"][b]), K)
+            if scores_out is not None:
+                scores_out.append(s)
             sel = O.top_k_select(s, wl.k)
-        outs.append(O.decode_attention(L["kind"], npy(L["q"][b]), pos, npy(L["kv"][b]),
-                                       npy(L["win"][b]), npy(L["sinks"]), m=L["m"], w=wl.w,
-                                       r=wl.r, q_gain=npy(L["q_gain"]), sel=sel))
+            if sels is not None and sels[li] is not None:
+                sel = np.asarray(sels[li])
+        outs.append(O.decode_attention(L["kind"], npy(L["q"][b]), pos, kv, win, npy(L["sinks"]),
+                                       m=m, w=wl.w, r=wl.r, q_gain=npy(L["q_gain"]), sel=sel))
     return outs
 
 
@@ -426,6 +487,9 @@ def main():
     wl = synth.WORKLOADS[args.workload]
     layers = synth.decode_inputs(runtime.shard_workload(wl, rank), dev)
     io = runtime.StepIO(layers, dev)            # per-step inputs / outputs in one arena each
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    # the oracle's copy of the inputs, taken before any kernel runs
+    layers_host = host_layers(layers) if want_cpu else None
     eager = runtime.DecodeStep(wl, layers, stream)
     step = eager
     launch_mode = "eager"
@@ -514,8 +578,8 @@ def main():
                    "kernels_ms_per_layer": {k_: v[1] / args.prefill_steps for k_, v in ptr.items()}}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, host_layers(layers))
+    if want_cpu:
+        cpu = cpu_baseline(wl, layers_host)
 
     if api.device_error(stream) != 0:
         raise RuntimeError("device error flag set during the timed region")

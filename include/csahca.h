@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define CSAHCA_ABI_VERSION 1
+#define CSAHCA_ABI_VERSION 2
 
 /* ---- status codes ------------------------------------------------------- */
 enum {
@@ -274,6 +274,78 @@ typedef struct {
 int compressed_attn_decode(const csahca_decode_args* args, void* stream);
 size_t csahca_decode_workspace_size(const csahca_decode_args* args);
 
+/* ---- decode_compress --------------------------------------------------------
+ * [P2] CSA KV compression, HCA, sliding window KV, Additional Techniques.
+ * One decode step of one layer's compressors for B sequences, the new token
+ * of sequence b at position t = pos[b] (device int32):
+ *   1. its raw streams go into slot t % R of `ring` (R = 2m for CSA, m for
+ *      HCA; ring [B, R, S, d] with S = 4 streams a, b, za, zb for CSA, 2
+ *      streams a, za for HCA; the indexer streams likewise into `iring`
+ *      [B, 2m, 4, dI]).  The rings are the compressor state between steps:
+ *      slot p % R holds token p for the R tokens before t.
+ *   2. if kv_raw != NULL and w > 0: win[b, t % w] = RoPE_t(RMSNorm(kv_raw[b])
+ *      * kv_gain) (norm only if kv_norm).
+ *   3. if t completes block i = (t+1)/m - 1 and i < N_cap: entry i is pooled
+ *      exactly as csa_compress / hca_compress define it over the ring's tokens
+ *      (token t from the inputs; the slots of other tokens must hold them) and
+ *      kv_cache[b, i] = RoPE_{i*m}(RMSNorm(C_i) * kv_gain); for CSA with
+ *      dI > 0 the indexer key of entry i is pooled from the indexer streams
+ *      (no norm, no RoPE) and stored in kI[b, i] (kI_dtype = dtype), or, for
+ *      kI_dtype E4M3, as e4m3 codes with kI_scale[b, i, j] = amax_j / 448 over
+ *      each 128-element block j (1 for an all-zero block) and codes the
+ *      nearest e4m3 of x / scale (ties to even, saturating at 448), all in
+ *      fp32.  Entries with i >= N_cap are not stored.  A sequence with
+ *      pos[b] < 0 is left untouched.
+ * Layout: pos [B]; kv_raw, a, b, za, zb [B, d] (dtype; b, zb CSA only);
+ *   bias_a, bias_b [m, d] f32; kv_gain [d] f32 or NULL (ones); kv_cache
+ *   [B, N_cap, d]; win [B, w, d]; ia, ib, iza, izb [B, dI] (dtype); ibias_a,
+ *   ibias_b [m, dI] f32; kI [B, N_cap, dI]; kI_scale [B, N_cap, dI/128] f32.
+ * Constraints: dtype F32 (d % 32 == 0) or BF16 (d % 64 == 0), d <= 128 * 16 /
+ *   (element bytes); rope_dims even and <= d; dI = 0 or (CSA) dI % 8 == 0
+ *   with dI / 8 a multiple of the 16-byte vector and dividing 128 (BF16:
+ *   64, 128, 256, 512, 1024; F32: 32, 64, 128, 256, 512); E4M3 keys need
+ *   BF16 and dI % 128 == 0.  No workspace.  Rows of one sequence are written
+ *   by one cluster of eight CTAs, so calls for different layers may overlap.
+ */
+typedef struct {
+  int32_t kind;
+  int32_t dtype;
+  int32_t B, d;
+  int32_t m;
+  int32_t N_cap;
+  int32_t w;
+  int32_t rope_dims;
+  float rope_base;     /* 0 -> 10000 */
+  float eps;           /* 0 -> 1e-6 */
+  int32_t kv_norm;
+  int32_t dI;
+  int32_t kI_dtype;
+  int32_t reserved0;
+  const int32_t* pos;
+  const void* kv_raw;
+  const void* a;
+  const void* b;
+  const void* za;
+  const void* zb;
+  const float* bias_a;
+  const float* bias_b;
+  const float* kv_gain;
+  void* ring;
+  void* kv_cache;
+  void* win;
+  const void* ia;
+  const void* ib;
+  const void* iza;
+  const void* izb;
+  const float* ibias_a;
+  const float* ibias_b;
+  void* iring;
+  void* kI;
+  float* kI_scale;
+} csahca_decode_compress_args;
+
+int decode_compress(const csahca_decode_compress_args* args, void* stream);
+
 /* ---- utilities ------------------------------------------------------------ */
 
 /* Human-readable name of a status code (static string). */
@@ -283,7 +355,8 @@ const char* csahca_status_string(int status);
 int csahca_abi_version(void);
 
 /* sizeof() of the argument structs, for bindings to check their mirrors:
- * which = 0 compress, 1 indexer, 2 prefill, 3 decode; -1 for an unknown id. */
+ * which = 0 compress, 1 indexer, 2 prefill, 3 decode, 4 decode_compress;
+ * -1 for an unknown id. */
 int64_t csahca_struct_size(int which);
 
 /* Device-side error word of the current device: every bounded wait in the

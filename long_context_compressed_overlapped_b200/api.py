@@ -1,4 +1,4 @@
-"""Torch-facing wrappers of the five C-ABI entry points (same names).
+"""Torch-facing wrappers of the C-ABI entry points (same names).
 
 Argument marshalling only: tensors are checked for device, dtype, shape and
 contiguity, outputs and workspaces are allocated with torch when the caller
@@ -181,6 +181,54 @@ def compressed_attn_decode(kind, q, pos, kv_cache, win, sinks, *, m, rope_dims, 
     N.check(L.compressed_attn_decode(C.byref(args), _stream(stream)), "compressed_attn_decode")
     del keep
     return out
+
+
+def decode_compress_args(kind, pos, streams, ring, kv_cache, *, m, bias_a, bias_b=None, kv_raw=None,
+                         win=None, kv_gain=None, kv_norm=True, rope_dims=0, rope_base=10000.0,
+                         eps=1e-6, istreams=None, ibias_a=None, ibias_b=None, iring=None, kI=None,
+                         kI_scale=None):
+    """Build the DecodeCompressArgs struct (and the list of tensors it points to).
+
+    streams: (a, b, za, zb) for "csa" or (a, za) for "hca", each [B, d];
+    ring [B, R, S, d]; istreams: (ia, ib, iza, izb) [B, dI] with iring
+    [B, 2m, 4, dI] and kI / kI_scale (csa only, optional)."""
+    B, d = streams[0].shape
+    keep = []
+
+    def f(t):
+        t = _f32(t)
+        keep.append(t)
+        return t
+
+    pos = pos.to(torch.int32).contiguous()
+    keep.append(pos)
+    csa = kind == "csa"
+    a, b, za, zb = (streams if csa else (streams[0], None, streams[1], None))
+    dI = 0
+    ia = ib = iza = izb = None
+    if csa and istreams is not None:
+        ia, ib, iza, izb = istreams
+        dI = ia.shape[1]
+    args = N.DecodeCompressArgs(
+        kind=N.CSA if csa else N.HCA, dtype=_dt(a), B=B, d=d, m=m, N_cap=kv_cache.shape[1],
+        w=win.shape[1] if win is not None else 0, rope_dims=rope_dims, rope_base=rope_base, eps=eps,
+        kv_norm=int(bool(kv_norm)), dI=dI, kI_dtype=_dt(kI) if dI else 0,
+        pos=_ptr(pos), kv_raw=_ptr(kv_raw), a=_ptr(a), b=_ptr(b), za=_ptr(za), zb=_ptr(zb),
+        bias_a=_ptr(f(bias_a)), bias_b=_ptr(f(bias_b)), kv_gain=_ptr(f(kv_gain)), ring=_ptr(ring),
+        kv_cache=_ptr(kv_cache), win=_ptr(win), ia=_ptr(ia), ib=_ptr(ib), iza=_ptr(iza), izb=_ptr(izb),
+        ibias_a=_ptr(f(ibias_a)), ibias_b=_ptr(f(ibias_b)), iring=_ptr(iring), kI=_ptr(kI),
+        kI_scale=_ptr(kI_scale))
+    return args, keep
+
+
+def decode_compress(kind, pos, streams, ring, kv_cache, *, m, bias_a, stream=None, **kw):
+    """One decode step of one layer's compressors: the new token's raw streams
+    into the ring, its window row (if kv_raw and win are given) and, when the
+    token completes a block, the new compressed entry (and indexer key) into
+    the caches.  Updates ring, win, kv_cache, iring, kI, kI_scale in place."""
+    args, keep = decode_compress_args(kind, pos, streams, ring, kv_cache, m=m, bias_a=bias_a, **kw)
+    N.check(N.lib().decode_compress(C.byref(args), _stream(stream)), "decode_compress")
+    del keep
 
 
 def device_error(stream=None) -> int:

@@ -895,7 +895,7 @@ struct TcCombineParams {
   const int* pos;             // [B] query positions (decode)
   __nv_bfloat16* out;         // [B * nq, H, D]
   int rows, splits, rope_dims;
-  double rope_base;
+  double theta[64];           // base^(-2j/r) per rope pair j (r <= 128), from the host
 };
 
 // dynamic shared memory of the combine: headers of all splits + slice slots
@@ -910,7 +910,8 @@ __host__ __device__ inline int tc_combine_smem_bytes(int splits) {
 // split was measured to complete one copy at a time; a box covering every
 // split goes out as one transfer.
 __global__ void __launch_bounds__(kTcCombineThreads) attn_combine_tc_kernel(
-    const __grid_constant__ CUtensorMap hdr_map, const __grid_constant__ CUtensorMap slc_map, TcCombineParams p) {
+    const __grid_constant__ CUtensorMap hdr_map, const __grid_constant__ CUtensorMap slc_map,
+    const __grid_constant__ TcCombineParams p) {
   extern __shared__ __align__(128) uint8_t cmb_smem[];
   __shared__ uint64_t bar_hdr, bar_slc;
   __shared__ float red[8][kAttnH];
@@ -1038,7 +1039,7 @@ __global__ void __launch_bounds__(kTcCombineThreads) attn_combine_tc_kernel(
     for (int i = 0; i < 8; ++i) partner[i] = __shfl_xor_sync(0xffffffffu, acc[i], 8);
     if (dim >= r0) {
       float cs, sn;
-      rope_cos_sin(-(double)p.pos[row], (dim - r0) >> 1, p.rope_dims, p.rope_base, &cs, &sn);
+      rope_sincos(-(double)p.pos[row], p.theta[(dim - r0) >> 1], &cs, &sn);
 #pragma unroll
       for (int i = 0; i < 8; ++i)
         acc[i] = (dim & 1) ? fmaf(partner[i], sn, acc[i] * cs) : fmaf(-partner[i], sn, acc[i] * cs);

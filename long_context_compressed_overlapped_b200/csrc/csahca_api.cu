@@ -15,6 +15,7 @@
 #include "../../include/csahca.h"
 #include "common.cuh"
 #include "compress.cuh"
+#include "decode_compress.cuh"
 #include "indexer_simt.cuh"
 #include "topk.cuh"
 #include "topk_large.cuh"
@@ -66,6 +67,12 @@ struct Scope {
 
 constexpr double kDefaultRopeBase = 10000.0;
 constexpr float kDefaultEps = 1e-6f;
+
+// theta[j] = base^(-2j/r), the RoPE angle per unit of position of pair j, in
+// double, for the r/2 pairs (at most 64) of kernels that take it as a parameter.
+void rope_theta_table(double* theta, int r, double base) {
+  for (int j = 0; j < 64; ++j) theta[j] = j < r / 2 ? pow(base, -2.0 * j / r) : 0.0;
+}
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -882,7 +889,8 @@ int run_decode_t(const csahca_decode_args* a, cudaStream_t s, char* ws) {
     TcCombineParams c;
     c.partial = reinterpret_cast<const char*>(partial); c.sinks = a->sinks; c.pos = a->pos;
     c.out = static_cast<__nv_bfloat16*>(a->out);
-    c.rows = a->B; c.splits = L.splits; c.rope_dims = a->rope_dims; c.rope_base = base;
+    c.rows = a->B; c.splits = L.splits; c.rope_dims = a->rope_dims;
+    rope_theta_table(c.theta, a->rope_dims, base);              // rope_dims <= 128 on this path
     const int smem = tc_combine_smem_bytes(L.splits);
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(attn_combine_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -928,6 +936,71 @@ int run_decode(const csahca_decode_args* a, void* stream, char* ws, size_t ws_by
   return a->dtype == CSAHCA_F32 ? run_decode_t<float>(a, s, ws) : run_decode_t<__nv_bfloat16>(a, s, ws);
 }
 
+// --------------------------------------------------------- decode_compress --
+
+int run_decode_compress(const csahca_decode_compress_args* a, void* stream) {
+  if (!a) return CSAHCA_ERR_INVALID_ARG;
+  if (a->kind != CSAHCA_CSA && a->kind != CSAHCA_HCA) return CSAHCA_ERR_INVALID_ARG;
+  if (a->dtype != CSAHCA_F32 && a->dtype != CSAHCA_BF16) return CSAHCA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->d <= 0 || a->m < 1 || a->N_cap < 0 || a->w < 0 || a->dI < 0) return CSAHCA_ERR_INVALID_ARG;
+  if (a->rope_dims < 0 || a->rope_dims > a->d || (a->rope_dims & 1)) return CSAHCA_ERR_INVALID_ARG;
+  if (a->rope_dims > 2 * kDcMaxRopePairs) return CSAHCA_ERR_UNSUPPORTED;
+  const bool csa = a->kind == CSAHCA_CSA;
+  const int vec = 16 / dtype_size(a->dtype);
+  if (a->d % (kDcCluster * vec) || a->d / (kDcCluster * vec) > kDcMaxVecs) return CSAHCA_ERR_UNSUPPORTED;
+  const int dI = csa ? a->dI : 0;
+  if (dI) {
+    const int si = dI / kDcCluster;
+    if (dI % kDcCluster || si % vec || 128 % si || si / vec > kDcMaxVecs) return CSAHCA_ERR_UNSUPPORTED;
+    if (a->kI_dtype == CSAHCA_E4M3) {
+      if (a->dtype != CSAHCA_BF16 || dI % 128) return CSAHCA_ERR_UNSUPPORTED;
+    } else if (a->kI_dtype != a->dtype) {
+      return CSAHCA_ERR_UNSUPPORTED;
+    }
+  }
+  if (a->B == 0) return CSAHCA_OK;
+  if (!a->pos || !a->a || !a->za || !a->bias_a || !a->ring || !a->kv_cache) return CSAHCA_ERR_INVALID_ARG;
+  if (csa && (!a->b || !a->zb || !a->bias_b)) return CSAHCA_ERR_INVALID_ARG;
+  if (a->kv_raw && a->w > 0 && !a->win) return CSAHCA_ERR_INVALID_ARG;
+  if (dI && (!a->ia || !a->ib || !a->iza || !a->izb || !a->ibias_a || !a->ibias_b || !a->iring || !a->kI))
+    return CSAHCA_ERR_INVALID_ARG;
+  if (dI && a->kI_dtype == CSAHCA_E4M3 && !a->kI_scale) return CSAHCA_ERR_INVALID_ARG;
+  const void* ptrs[] = {a->pos, a->kv_raw, a->a, a->b, a->za, a->zb, a->bias_a, a->bias_b, a->kv_gain,
+                        a->ring, a->kv_cache, a->win, a->ia, a->ib, a->iza, a->izb, a->ibias_a,
+                        a->ibias_b, a->iring, a->kI, a->kI_scale};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return CSAHCA_ERR_ALIGNMENT;
+  if ((int64_t)a->B * kDcCluster > INT32_MAX) return CSAHCA_ERR_UNSUPPORTED;
+  int st = device_ok();
+  if (st != CSAHCA_OK) return st;
+  DecodeCompressParams p;
+  memset(&p, 0, sizeof(p));
+  p.pos = a->pos; p.kv_raw = a->kv_raw;
+  p.nw[0] = a->a; p.nw[1] = csa ? a->b : a->za; p.nw[2] = csa ? a->za : nullptr; p.nw[3] = csa ? a->zb : nullptr;
+  p.bias_a = a->bias_a; p.bias_b = a->bias_b; p.gain = a->kv_gain;
+  p.ring = a->ring; p.kv_cache = a->kv_cache; p.win = a->win;
+  if (dI) {
+    p.inw[0] = a->ia; p.inw[1] = a->ib; p.inw[2] = a->iza; p.inw[3] = a->izb;
+    p.ibias_a = a->ibias_a; p.ibias_b = a->ibias_b; p.iring = a->iring; p.kI = a->kI; p.kI_scale = a->kI_scale;
+  }
+  p.B = a->B; p.d = a->d; p.dI = dI; p.m = a->m; p.N_cap = a->N_cap; p.w = a->w;
+  p.rope_dims = a->rope_dims; p.kv_norm = a->kv_norm; p.ki_e4m3 = dI && a->kI_dtype == CSAHCA_E4M3;
+  p.eps = a->eps > 0 ? a->eps : kDefaultEps;
+  rope_theta_table(p.theta, a->rope_dims, a->rope_base > 0 ? a->rope_base : kDefaultRopeBase);
+  cudaStream_t s = as_stream(stream);
+  const dim3 grid((unsigned)(a->B * kDcCluster)), block(kDcThreads);
+  CSAHCA_TRACE("decode_compress", s);
+  if (a->dtype == CSAHCA_F32) {
+    if (csa) launch_k(decode_compress_kernel<float, true>, grid, block, 0, s, p);
+    else launch_k(decode_compress_kernel<float, false>, grid, block, 0, s, p);
+  } else {
+    if (csa) launch_k(decode_compress_kernel<__nv_bfloat16, true>, grid, block, 0, s, p);
+    else launch_k(decode_compress_kernel<__nv_bfloat16, false>, grid, block, 0, s, p);
+  }
+  CSAHCA_CHECK_LAUNCH();
+  return CSAHCA_OK;
+}
+
 }  // namespace
 
 // ============================================================== C ABI ======
@@ -954,6 +1027,10 @@ size_t csahca_prefill_workspace_size(const csahca_attn_args* args) {
 int compressed_attn_decode(const csahca_decode_args* args, void* stream) {
   if (!args) return CSAHCA_ERR_INVALID_ARG;
   return run_decode(args, stream, static_cast<char*>(args->workspace), args->workspace_bytes);
+}
+
+int decode_compress(const csahca_decode_compress_args* args, void* stream) {
+  return run_decode_compress(args, stream);
 }
 
 size_t csahca_decode_workspace_size(const csahca_decode_args* args) {
@@ -984,6 +1061,7 @@ int64_t csahca_struct_size(int which) {
     case 1: return (int64_t)sizeof(csahca_indexer_args);
     case 2: return (int64_t)sizeof(csahca_attn_args);
     case 3: return (int64_t)sizeof(csahca_decode_args);
+    case 4: return (int64_t)sizeof(csahca_decode_compress_args);
     default: return -1;
   }
 }

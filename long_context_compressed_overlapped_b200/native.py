@@ -65,11 +65,21 @@ class DecodeArgs(C.Structure):
                 ("workspace_bytes", sz)]
 
 
+class DecodeCompressArgs(C.Structure):
+    _fields_ = [("kind", i32), ("dtype", i32), ("B", i32), ("d", i32), ("m", i32),
+                ("N_cap", i32), ("w", i32), ("rope_dims", i32), ("rope_base", f32), ("eps", f32),
+                ("kv_norm", i32), ("dI", i32), ("kI_dtype", i32), ("reserved0", i32),
+                ("pos", vp), ("kv_raw", vp), ("a", vp), ("b", vp), ("za", vp), ("zb", vp),
+                ("bias_a", vp), ("bias_b", vp), ("kv_gain", vp), ("ring", vp), ("kv_cache", vp),
+                ("win", vp), ("ia", vp), ("ib", vp), ("iza", vp), ("izb", vp), ("ibias_a", vp),
+                ("ibias_b", vp), ("iring", vp), ("kI", vp), ("kI_scale", vp)]
+
+
 class TraceEntry(C.Structure):
     _fields_ = [("name", C.c_char * 48), ("launches", C.c_int64), ("total_ms", C.c_double)]
 
 
-STRUCTS = {0: CompressArgs, 1: IndexerArgs, 2: AttnArgs, 3: DecodeArgs}
+STRUCTS = {0: CompressArgs, 1: IndexerArgs, 2: AttnArgs, 3: DecodeArgs, 4: DecodeCompressArgs}
 
 # Every symbol include/csahca.h declares, with (restype, argtypes).
 SIGNATURES = {
@@ -82,6 +92,7 @@ SIGNATURES = {
     "csahca_prefill_workspace_size": (sz, [C.POINTER(AttnArgs)]),
     "compressed_attn_decode": (C.c_int, [C.POINTER(DecodeArgs), vp]),
     "csahca_decode_workspace_size": (sz, [C.POINTER(DecodeArgs)]),
+    "decode_compress": (C.c_int, [C.POINTER(DecodeCompressArgs), vp]),
     "csahca_status_string": (C.c_char_p, [C.c_int]),
     "csahca_abi_version": (C.c_int, []),
     "csahca_struct_size": (C.c_int64, [C.c_int]),

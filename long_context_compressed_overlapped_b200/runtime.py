@@ -37,12 +37,13 @@ def max_over_ranks(x: float, group=None) -> float:
 
 class StepIO:
     """The per-step inputs of every layer (new query, indexer query and
-    weights, positions) placed in one device arena, and the outputs in
+    weights, positions, the new token's compressor streams and raw window
+    row) placed in one device arena, and the outputs in
     another: a caller then moves a step's data with one copy each way.  The
     layers' tensors become views of the arenas (same dtype and shape, slots
     256-byte aligned); make the DecodeStep after this."""
 
-    IN_NAMES = ("q", "qI", "w", "pos")
+    IN_NAMES = ("q", "qI", "w", "pos", "kv_raw", "ca", "cb", "cza", "czb", "ia", "ib", "iza", "izb")
 
     def __init__(self, layers, device):
         def arena(tensors):
@@ -71,19 +72,42 @@ class StepIO:
             L["out"] = view(self.out, o, t.dtype, tuple(t.shape))
 
 
+def compress_args(wl: synth.Workload, L):
+    """DecodeCompressArgs of one layer of synth.decode_inputs (and the tensors
+    it points to)."""
+    csa = L["kind"] == "csa"
+    streams = tuple(L[n] for n in (("ca", "cb", "cza", "czb") if csa else ("ca", "cza")))
+    kw = {}
+    if csa:
+        kw = dict(istreams=tuple(L[n] for n in ("ia", "ib", "iza", "izb")), ibias_a=L["ibias_a"],
+                  ibias_b=L["ibias_b"], iring=L["iring"], kI=L["kI"], kI_scale=L["kI_scale"])
+    return api.decode_compress_args(L["kind"], L["pos"], streams, L["ring"], L["kv"], m=L["m"],
+                                    bias_a=L["bias_a"], bias_b=L["bias_b"], kv_raw=L["kv_raw"],
+                                    win=L["win"], kv_gain=L["kv_gain"], rope_dims=wl.r, **kw)
+
+
 class DecodeStep:
     """One decode step over every layer of `layers` (as made by
-    synth.decode_inputs): the C-ABI argument structs and workspaces are
-    built once, so a call only enqueues the library's kernels on `stream`."""
+    synth.decode_inputs): per layer, the compressors take in the new token
+    (decode_compress: ring, window row, a new cache entry when the token
+    completes a block), then compressed_attn_decode.  The C-ABI argument
+    structs and workspaces are built once, so a call only enqueues the
+    library's kernels on `stream`."""
 
-    def __init__(self, wl: synth.Workload, layers, stream: torch.cuda.Stream):
+    def __init__(self, wl: synth.Workload, layers, stream: torch.cuda.Stream, keep_idx: bool = False):
         self.lib = native.lib()
         self.stream = stream
         self.calls = []
+        self.compress = [compress_args(wl, L) for L in layers]
+        self.idx = []                            # per layer: the CSA selection (keep_idx) or None
         for L in layers:
             kw = dict(m=L["m"], rope_dims=wl.r, q_gain=L["q_gain"])
+            idx = None
             if L["kind"] == "csa":
-                kw.update(k=wl.k, qI=L["qI"], wI=L["w"], kI=L["kI"], kI_scale=L["kI_scale"])
+                if keep_idx:
+                    idx = torch.empty(L["q"].shape[0], wl.k, dtype=torch.int32, device=L["q"].device)
+                kw.update(k=wl.k, qI=L["qI"], wI=L["w"], kI=L["kI"], kI_scale=L["kI_scale"], idx_out=idx)
+            self.idx.append(idx)
             args, out, keep = api.decode_args(L["kind"], L["q"], L["pos"], L["kv"], L["win"],
                                               L["sinks"], out=L.get("out"), **kw)
             nbytes = self.lib.csahca_decode_workspace_size(C.byref(args))
@@ -96,7 +120,10 @@ class DecodeStep:
 
     def __call__(self):
         sh = self.stream.cuda_stream
-        for args, _, _, _ in self.calls:
+        for (cargs, _), (args, _, _, _) in zip(self.compress, self.calls):
+            st = self.lib.decode_compress(C.byref(cargs), sh)
+            if st != 0:
+                native.check(st, "decode_compress")
             st = self.lib.compressed_attn_decode(C.byref(args), sh)
             if st != 0:
                 native.check(st, "compressed_attn_decode")

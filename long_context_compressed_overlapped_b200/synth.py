@@ -180,10 +180,18 @@ def decode_inputs(wl: Workload, device="cpu", ctx: int | None = None, B: int | N
                   layers=None):
     """Per-layer decode state and new-token inputs.
 
-    For each layer L: caches already final (Gaussian rows as drawn): CSA
-    kv [B, ctx/m, d], indexer keys [B, ctx/m, d_I] (bf16, or e4m3 codes + fp32
-    scales), HCA kv [B, ctx/m', d]; window ring [B, w, d]; new query q
-    [B, H, d] at position ctx, qI [B, H_I, d_I], w [B, H_I]; sinks [H].
+    For each layer L: caches already final (Gaussian rows as drawn), with room
+    for every entry the new token at position ctx completes: CSA kv
+    [B, (ctx+1)/m, d], indexer keys [B, (ctx+1)/m, d_I] (bf16, or e4m3 codes +
+    fp32 scales), HCA kv [B, (ctx+1)/m', d]; window ring [B, w, d]; new query
+    q [B, H, d] at position ctx, qI [B, H_I, d_I], w [B, H_I]; sinks [H].
+    Compressor state and the new token's compressor inputs: ring [B, R, S, d]
+    of the raw streams of the R tokens before it (R = 2m, S = 4 for CSA:
+    a, b, za, zb; R = m', S = 2 for HCA: a, za), its own streams ca, cb, cza,
+    czb (CSA) or ca, cza (HCA) [B, d], its raw window row kv_raw [B, d],
+    biases bias_a, bias_b [m, d] ~ N(0, 0.1^2) and kv_gain (ones); for CSA
+    the indexer streams ia, ib, iza, izb [B, d_I], iring [B, 2m, 4, d_I] and
+    ibias_a, ibias_b [m, d_I].
     """
     D = Draw(wl.seed, device)
     ctx = wl.ctx if ctx is None else ctx
@@ -194,7 +202,7 @@ def decode_inputs(wl: Workload, device="cpu", ctx: int | None = None, B: int | N
     for li, kind in enumerate(layers):
         t = f"L{li}"
         m = wl.m if kind == "csa" else wl.m_hca
-        N = ctx // m
+        N = (ctx + 1) // m
         L = {
             "kind": kind, "m": m,
             "pos": torch.full((B,), ctx, dtype=torch.int32, device=device),
@@ -215,5 +223,23 @@ def decode_inputs(wl: Workload, device="cpu", ctx: int | None = None, B: int | N
             else:
                 L["kI"] = kI
                 L["kI_scale"] = None
+        sd = (1.0 / math.sqrt(wl.d)) if wl.dtype == "f32" else 1.0
+        S = 4 if kind == "csa" else 2
+        R = 2 * m if kind == "csa" else m
+        names = ("ca", "cb", "cza", "czb") if kind == "csa" else ("ca", "cza")
+        L["ring"] = D.normal(f"{t}/ring", (B, R, S, wl.d), sd, dt)
+        for n in names:
+            L[n] = D.normal(f"{t}/{n}", (B, wl.d), sd, dt)
+        L["kv_raw"] = D.normal(f"{t}/kv_raw", (B, wl.d), sd, dt)
+        L["bias_a"] = D.normal(f"{t}/bias_a", (m, wl.d), 0.1, torch.float32)
+        L["bias_b"] = D.normal(f"{t}/bias_b", (m, wl.d), 0.1, torch.float32) if kind == "csa" else None
+        L["kv_gain"] = torch.ones(wl.d, dtype=torch.float32, device=device)
+        if kind == "csa":
+            sdi = (1.0 / math.sqrt(wl.dI)) if wl.dtype == "f32" else 1.0
+            L["iring"] = D.normal(f"{t}/iring", (B, R, 4, wl.dI), sdi, dt)
+            for n in ("ia", "ib", "iza", "izb"):
+                L[n] = D.normal(f"{t}/{n}", (B, wl.dI), sdi, dt)
+            L["ibias_a"] = D.normal(f"{t}/ibias_a", (m, wl.dI), 0.1, torch.float32)
+            L["ibias_b"] = D.normal(f"{t}/ibias_b", (m, wl.dI), 0.1, torch.float32)
         out.append(L)
     return out

@@ -52,7 +52,7 @@ def test_struct_sizes_match(lib):
     for which, st in N.STRUCTS.items():
         assert lib.csahca_struct_size(which) == C.sizeof(st)
     assert lib.csahca_struct_size(99) == -1
-    assert lib.csahca_abi_version() == 1
+    assert lib.csahca_abi_version() == 2
 
 
 def test_status_strings(lib):
@@ -86,6 +86,21 @@ def test_validation_rejects_before_launch(lib):
     assert lib.compressed_attn_prefill(C.byref(aa), None) == N.ERR_INVALID_ARG
     da = N.DecodeArgs(kind=N.HCA, dtype=N.BF16, B=1, H=4, d=48, N_cap=4, m=4)
     assert lib.compressed_attn_decode(C.byref(da), None) == N.ERR_UNSUPPORTED
+    assert lib.decode_compress(None, None) == N.ERR_INVALID_ARG
+    dc = N.DecodeCompressArgs(kind=N.HCA, dtype=N.BF16, B=1, d=96, m=128, N_cap=4)  # d % 64 != 0
+    assert lib.decode_compress(C.byref(dc), None) == N.ERR_UNSUPPORTED
+    dc = N.DecodeCompressArgs(kind=N.CSA, dtype=N.F32, B=1, d=64, m=4, N_cap=4, dI=128, kI_dtype=N.E4M3)
+    assert lib.decode_compress(C.byref(dc), None) == N.ERR_UNSUPPORTED   # e4m3 keys need bf16 rows
+    dc = N.DecodeCompressArgs(kind=N.CSA, dtype=N.BF16, B=1, d=512, m=4, N_cap=4, dI=192, kI_dtype=N.BF16)
+    assert lib.decode_compress(C.byref(dc), None) == N.ERR_UNSUPPORTED   # dI / 8 must divide 128
+    dc = N.DecodeCompressArgs(kind=N.CSA, dtype=N.BF16, B=1, d=512, m=4, N_cap=4, rope_dims=3)
+    assert lib.decode_compress(C.byref(dc), None) == N.ERR_INVALID_ARG
+    dc = N.DecodeCompressArgs(kind=N.HCA, dtype=N.BF16, B=1, d=512, m=128, N_cap=4, pos=16, a=16, za=16,
+                              bias_a=16, ring=16, kv_cache=16)        # HCA needs no b / zb
+    dc.kv_cache = 24
+    assert lib.decode_compress(C.byref(dc), None) == N.ERR_ALIGNMENT
+    dc = N.DecodeCompressArgs(kind=N.CSA, dtype=N.BF16, B=0, d=512, m=4, N_cap=4)
+    assert lib.decode_compress(C.byref(dc), None) == N.OK                 # empty batch: no-op
 
 
 def test_workspace_queries(lib):
@@ -108,3 +123,6 @@ def test_no_device_is_reported_not_faked(lib):
     a = N.CompressArgs(dtype=N.F32, B=1, n=64, c=64, m=4, num_blocks=-1, a=16, b=16, za=16, zb=16, bias_a=16,
                        bias_b=16, out=16)
     assert lib.csa_compress(C.byref(a), None) == N.ERR_NO_DEVICE
+    dc = N.DecodeCompressArgs(kind=N.HCA, dtype=N.BF16, B=1, d=512, m=128, N_cap=4, pos=16, a=16, za=16,
+                              bias_a=16, ring=16, kv_cache=16)
+    assert lib.decode_compress(C.byref(dc), None) == N.ERR_NO_DEVICE

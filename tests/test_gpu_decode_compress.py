@@ -1,0 +1,202 @@
+"""GPU parity of decode_compress, one decode step of a layer's compressors,
+against the float64 oracle.  The step puts the new token's streams in the
+ring and writes its window row.  When the token completes a block it also
+writes the new CSA / HCA entry and the indexer key ("Paper Breakdown:
+DeepSeek-V4", section 4: CSA KV Compression, HCA, Sliding window KV,
+Additional Techniques).  Also covered: the decode step bench.py times
+(compressors, indexer, top-k, attention per layer, replayed as a CUDA graph)
+against the oracle's decode step."""
+
+import ctypes as C
+
+import numpy as np
+import pytest
+import torch
+
+import bench
+from long_context_compressed_overlapped_b200 import api, native, runtime, synth
+from oracle import csahca_oracle as O
+from tests.helpers import check_close, check_topk, npy
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+NAMES = {"csa": ("a", "b", "za", "zb"), "hca": ("a", "za")}
+
+
+def _replay(wl, kind, n, B, lags, gain):
+    """Decode every token of a stream from position 0, one decode_compress
+    call per step; sequence b takes token t - lags[b] at step t."""
+    m = wl.m if kind == "csa" else wl.m_hca
+    wl = synth.Workload(**{**wl.__dict__, "kind": kind})
+    inp = synth.prefill_inputs(wl, DEV, n=n, B=B)
+    names = NAMES[kind]
+    R = 2 * m if kind == "csa" else m
+    dt, d, w = wl.torch_dtype, wl.d, wl.w
+    st = dict(ring=torch.zeros(B, R, len(names), d, dtype=dt, device=DEV),
+              kv=torch.zeros(B, n // m, d, dtype=dt, device=DEV),
+              win=torch.zeros(B, w, d, dtype=dt, device=DEV))
+    if kind == "csa":
+        st["iring"] = torch.zeros(B, R, 4, wl.dI, dtype=dt, device=DEV)
+        st["kI"] = torch.zeros(B, n // m, wl.dI, dtype=dt, device=DEV)
+    ar = torch.arange(B, device=DEV)
+    for t in range(n + max(lags)):
+        p = [t - lag for lag in lags]
+        tok = torch.tensor([min(max(x, 0), n - 1) for x in p], device=DEV)
+        pos = torch.tensor([x if 0 <= x < n else -1 for x in p], dtype=torch.int32, device=DEV)
+        streams = tuple(inp["kv"][s_][ar, tok].contiguous() for s_ in names)
+        kw = {}
+        if kind == "csa":
+            kw = dict(istreams=tuple(inp["ik"][s_][ar, tok].contiguous() for s_ in names),
+                      ibias_a=inp["ik"]["bias_a"], ibias_b=inp["ik"]["bias_b"], iring=st["iring"],
+                      kI=st["kI"])
+        api.decode_compress(kind, pos, streams, st["ring"], st["kv"], m=m, bias_a=inp["kv"]["bias_a"],
+                            bias_b=inp["kv"].get("bias_b"), kv_raw=inp["kv_win"][ar, tok].contiguous(),
+                            win=st["win"], kv_gain=gain, rope_dims=wl.r, **kw)
+    torch.cuda.synchronize()
+    return wl, inp, st, m
+
+
+def _check_replay(wl, kind, inp, st, m, n, B, gain):
+    names = NAMES[kind]
+    R = 2 * m if kind == "csa" else m
+    g = npy(gain)
+    for b in range(B):
+        s = {s_: npy(inp["kv"][s_][b]) for s_ in names}
+        if kind == "csa":
+            pooled = O.csa_pool(s["a"], s["b"], s["za"], s["zb"], npy(inp["kv"]["bias_a"]),
+                                npy(inp["kv"]["bias_b"]), m)
+            ik = {s_: npy(inp["ik"][s_][b]) for s_ in names}
+            keys = O.csa_pool(ik["a"], ik["b"], ik["za"], ik["zb"], npy(inp["ik"]["bias_a"]),
+                              npy(inp["ik"]["bias_b"]), m)
+            check_close(npy(st["kI"][b]), keys, wl.dtype, f"indexer keys b={b}")
+        else:
+            pooled = O.hca_pool(s["a"], s["za"], npy(inp["kv"]["bias_a"]), m)
+        rows = O.finish_rows(pooled, np.arange(pooled.shape[0]) * m, g, wl.r)
+        check_close(npy(st["kv"][b]), rows, wl.dtype, f"{kind} entries b={b}")
+        p = np.arange(n - wl.w, n)
+        wrows = O.finish_rows(npy(inp["kv_win"][b, p]), p, g, wl.r)
+        check_close(npy(st["win"][b, p % wl.w]), wrows, wl.dtype, f"window b={b}")
+        p = np.arange(n - R, n)
+        for j, s_ in enumerate(names):         # the ring holds the last R raw tokens, bit for bit
+            assert torch.equal(st["ring"][b, p % R, j], inp["kv"][s_][b, p])
+
+
+def test_decode_compress_tiny_csa_f32():
+    """tiny_csa_f32 shapes (d 64, r 16, m 4, d_I 32, w 16) in fp32, 40 tokens
+    replayed one call per step, the second sequence 5 tokens behind."""
+    wl = synth.WORKLOADS["tiny_csa_f32"]
+    gain = 1 + 0.1 * torch.randn(wl.d, generator=torch.Generator().manual_seed(5)).to(DEV)
+    wl, inp, st, m = _replay(wl, "csa", 40, 2, [0, 5], gain)
+    _check_replay(wl, "csa", inp, st, m, 40, 2, gain)
+    assert api.device_error() == 0
+
+
+def test_decode_compress_hca_bf16():
+    """hca_8k_bf16 shapes (d 128, r 64, m' 128, w 128): 300 tokens (two
+    entries and a ragged tail), the second sequence 45 tokens behind."""
+    wl = synth.WORKLOADS["hca_8k_bf16"]
+    gain = torch.ones(wl.d, device=DEV)
+    wl, inp, st, m = _replay(wl, "hca", 300, 2, [0, 45], gain)
+    _check_replay(wl, "hca", inp, st, m, 300, 2, gain)
+    assert api.device_error() == 0
+
+
+def _check_e4m3_key(codes, scales, key, what):
+    """codes/scales from the GPU; key: the oracle's pooled fp64 row.  The
+    scale must be the row's amax / 448 and each code a nearest e4m3 of
+    key / scale (a neighbour only where the two are equally near within the
+    fp32 error of the pooling)."""
+    amax = np.abs(key.reshape(-1, 128)).max(axis=1)
+    np.testing.assert_allclose(scales, amax / 448.0, rtol=1e-5, err_msg=what)
+    xs = key / np.repeat(scales.astype(np.float64), 128)
+    want = O.e4m3_encode(xs)
+    d_got = np.abs(O.e4m3_decode(codes) - xs)
+    d_want = np.abs(O.e4m3_decode(want) - xs)
+    assert (d_got <= d_want + 1e-4 * np.maximum(np.abs(xs), 1e-3)).all(), what
+    assert (codes == want).mean() >= 0.99, what
+
+
+def test_decode_compress_decode_1m_shapes():
+    """decode_1m shapes (B 4, d 512, d_I 128 e4m3, m 4, m' 128, w 128), one
+    call per layer with the rings as drawn, at positions that complete a
+    block near 2^20, complete none, complete the first block, and complete
+    block N-2."""
+    wl = synth.WORKLOADS["decode_1m"]
+    ctx = (1 << 20) - 1
+    layers = synth.decode_inputs(wl, DEV, ctx=ctx, layers=("csa", "hca"))
+    for L in layers:
+        m = L["m"]
+        L["pos"] = torch.tensor([ctx, ctx - 1, m - 1, ctx - m], dtype=torch.int32, device=DEV)
+        host = {k_: (v.cpu().clone() if isinstance(v, torch.Tensor) else v) for k_, v in L.items()}
+        args, keep = runtime.compress_args(wl, L)
+        native.check(native.lib().decode_compress(C.byref(args), torch.cuda.current_stream().cuda_stream),
+                     "decode_compress")
+        torch.cuda.synchronize()
+        csa = L["kind"] == "csa"
+        names = NAMES[L["kind"]]
+        cols = ("ca", "cb", "cza", "czb") if csa else ("ca", "cza")
+        R = 2 * m if csa else m
+        for b in range(wl.B):
+            pos = int(host["pos"][b])
+            ring = {s_: npy(host["ring"][b, :, j]) for j, s_ in enumerate(names)}
+            new = {s_: npy(host[c_][b]) for s_, c_ in zip(names, cols)}
+            biases = (npy(host["bias_a"]), npy(host["bias_b"]) if csa else None)
+            _, entry, win_row = O.decode_compress_step(L["kind"], pos, new, ring, biases, m,
+                                                       kv_raw=npy(host["kv_raw"][b]),
+                                                       gain=npy(host["kv_gain"]), r=wl.r)
+            what = f"{L['kind']} b={b} pos={pos}"
+            check_close(npy(L["win"][b, pos % wl.w]), win_row, "bf16", what + " window")
+            for j, c_ in enumerate(cols):
+                assert torch.equal(L["ring"][b, pos % R, j].cpu(), host[c_][b]), what + " ring"
+            emitted = (pos + 1) % m == 0
+            assert (entry is not None) == emitted
+            if emitted:
+                i = entry[0]
+                check_close(npy(L["kv"][b, i]), entry[2], "bf16", what + " entry")
+                lo = max(i - 2, 0)
+                assert torch.equal(L["kv"][b, lo:i].cpu(), host["kv"][b, lo:i]), what + " neighbours"
+            else:
+                i = (pos + 1) // m
+                lo = max(i - 2, 0)
+                assert torch.equal(L["kv"][b, lo:i + 1].cpu(), host["kv"][b, lo:i + 1]), what + " untouched"
+            if csa and emitted:
+                iring = {s_: npy(host["iring"][b, :, j]) for j, s_ in enumerate(names)}
+                inew = {s_: npy(host[c_][b]) for s_, c_ in zip(names, ("ia", "ib", "iza", "izb"))}
+                _, ient, _ = O.decode_compress_step("csa", pos, inew, iring,
+                                                    (npy(host["ibias_a"]), npy(host["ibias_b"])), m,
+                                                    normalize=False)
+                _check_e4m3_key(npy(L["kI"][b, i]), npy(L["kI_scale"][b, i]), ient[1], what + " key")
+        del keep
+    assert api.device_error() == 0
+
+
+def test_bench_decode_step_with_compressors():
+    """The step bench.py times (per layer decode_compress then
+    compressed_attn_decode, CSA, HCA, CSA, HCA, replayed as a CUDA graph) at
+    a 32,767-token context, where the new token completes a CSA and an HCA
+    block, against the oracle's decode step.  Both sequences are checked.
+    Selections must pass the top-k tolerance and outputs are compared on the
+    GPU's selections."""
+    wl = synth.WORKLOADS["decode_1m"]
+    ctx = (1 << 15) - 1
+    layers = synth.decode_inputs(wl, DEV, ctx=ctx, B=2)
+    host = bench.host_layers(layers)
+    stream = torch.cuda.Stream()
+    step = runtime.DecodeStep(wl, layers, stream, keep_idx=True)
+    graph = runtime.DecodeGraph(step)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            graph()                              # replays leave the same state
+    torch.cuda.synchronize()
+    assert api.device_error(stream) == 0
+    for b in range(2):
+        scores = []
+        bench.oracle_decode_sequence(wl, host, b, scores_out=scores)
+        sels = [None if ix is None else npy(ix[b]) for ix in step.idx]
+        si = iter(scores)
+        for li, L in enumerate(layers):
+            if L["kind"] == "csa":
+                check_topk(sels[li], next(si), wl.k, f"layer {li} b={b}")
+        ref = bench.oracle_decode_sequence(wl, host, b, sels=sels)
+        for li, o in enumerate(step.outputs):
+            check_close(npy(o[b]), ref[li], "bf16", f"layer {li} b={b}")
