@@ -60,6 +60,7 @@ struct AttnTcParams {
   int first_kernel;             // 1: the call's first kernel (inputs are read only after the wait)
   __nv_bfloat16* out;           // final [B, nq, H, D]
   float* partial;               // [B, nq, H, splits, D + 4]
+  double theta[64];             // base^(-2j/r) per rope pair j (r <= 128), filled on the host
 };
 
 struct AttnItem { int b, qi, t, tile0, tile1, split, ncomp_tiles, nwin_tiles; };
@@ -227,7 +228,7 @@ template <bool kDecode>
 __global__ void __launch_bounds__(attn_threads<kDecode>(), 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_constant__ CUtensorMap win_rows,
                const __grid_constant__ CUtensorMap q_rows, const __grid_constant__ CUtensorMap part_rows,
-               AttnTcParams p) {
+               const __grid_constant__ AttnTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
@@ -514,7 +515,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       gain_s[x] = gv;
       ones = ones && gv == 1.f;
     }
-    if (st < p.rope_dims / 2) theta_s[st] = rope_theta(st, p.rope_dims, p.rope_base);
+    if (st < p.rope_dims / 2) theta_s[st] = p.theta[st];
     const bool gain_ones = softmax_all256(ones);
     for (int id = blockIdx.x; id < p.n_items; id += gridDim.x) {
       const AttnItem it = attn_item<kDecode>(p, id);

@@ -648,6 +648,7 @@ bool attn_tc_shape_ok(int dtype, int H, int d, int rope_dims, int64_t comp_rows,
 int launch_attn_tc(const AttnTcParams& p_in, const void* kv_comp, int64_t comp_rows, const void* win,
                    int64_t win_rows, cudaStream_t s, const char* name) {
   AttnTcParams p = p_in;
+  rope_theta_table(p.theta, p.rope_dims, p.rope_base);
   p.win_ptr = static_cast<const __nv_bfloat16*>(win ? win : kv_comp);
   p.comp_rows_total = comp_rows;
   p.win_rows_total = win ? win_rows : comp_rows;
