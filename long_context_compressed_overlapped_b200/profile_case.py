@@ -3,11 +3,14 @@
     python -m long_context_compressed_overlapped_b200.profile_case csa --calls 4
     python -m long_context_compressed_overlapped_b200.profile_case hca --calls 4
     python -m long_context_compressed_overlapped_b200.profile_case indexer --calls 4
+    python -m long_context_compressed_overlapped_b200.profile_case compress --calls 4
 
 ``csa``: one CSA decode layer through ``compressed_attn_decode`` (indexer with
 e4m3 keys, top-k select, attention, combine); ``hca``: one HCA decode layer
 (attention, combine); ``indexer``: ``indexer_topk`` on the CSA layer's indexer
-inputs.  Four sequences at a 1,048,576-token context: 262,144 CSA entries
+inputs; ``compress``: ``decode_compress`` of the CSA layer with the new token at
+position 1,048,575, which completes a block (ring store, window row, pooled
+entry and e4m3 indexer key).  Four sequences at a 1,048,576-token context: 262,144 CSA entries
 (1 GB of bf16 rows, 134 MB of e4m3 indexer keys) or 8,192 HCA entries per
 sequence; about 1.3 GB on the device.  Inputs are the seeded synthetic draw of
 the decode_1m workload.  The process exits non-zero if a bounded device wait
@@ -15,23 +18,29 @@ gave up.
 """
 
 import argparse
+import ctypes as C
 import sys
 
 import torch
 
-from . import api, synth
+from . import api, native, runtime, synth
 
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("case", choices=("csa", "hca", "indexer"))
+    ap.add_argument("case", choices=("csa", "hca", "indexer", "compress"))
     ap.add_argument("--calls", type=int, default=4)
     a = ap.parse_args(argv)
     wl = synth.WORKLOADS["decode_1m"]
     kind = "hca" if a.case == "hca" else "csa"
-    L = synth.decode_inputs(wl, "cuda", ctx=wl.ctx, B=wl.B, layers=(kind,))[0]
+    ctx = wl.ctx - 1 if a.case == "compress" else wl.ctx
+    L = synth.decode_inputs(wl, "cuda", ctx=ctx, B=wl.B, layers=(kind,))[0]
+    cargs = runtime.compress_args(wl, L) if a.case == "compress" else None
     for _ in range(a.calls):
-        if a.case == "indexer":
+        if a.case == "compress":
+            native.check(native.lib().decode_compress(C.byref(cargs[0]), torch.cuda.current_stream().cuda_stream),
+                         "decode_compress")
+        elif a.case == "indexer":
             api.indexer_topk(L["qI"][:, None], L["w"][:, None], L["kI"], L["pos"][:, None], L["m"], wl.k,
                              kI_scale=L["kI_scale"])
         else:

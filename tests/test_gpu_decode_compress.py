@@ -200,3 +200,47 @@ def test_bench_decode_step_with_compressors():
         ref = bench.oracle_decode_sequence(wl, host, b, sels=sels)
         for li, o in enumerate(step.outputs):
             check_close(npy(o[b]), ref[li], "bf16", f"layer {li} b={b}")
+
+
+def test_decode_compress_options():
+    """decode_256k shapes (bf16 indexer keys): no RMSNorm (RoPE only), no
+    window row, and an entry past the cache's capacity (not stored); the
+    second sequence's token completes block N_cap, the first's block
+    N_cap - 1."""
+    wl = synth.WORKLOADS["decode_256k"]
+    ctx = 63
+    L = synth.decode_inputs(wl, DEV, ctx=ctx, B=2, layers=("csa",))[0]
+    m = L["m"]
+    N_cap = L["kv"].shape[1]
+    assert N_cap == (ctx + 1) // m
+    L["pos"] = torch.tensor([ctx, ctx + m], dtype=torch.int32, device=DEV)
+    host = {k_: (v.cpu().clone() if isinstance(v, torch.Tensor) else v) for k_, v in L.items()}
+    names = NAMES["csa"]
+    api.decode_compress("csa", L["pos"], tuple(L[c] for c in ("ca", "cb", "cza", "czb")), L["ring"], L["kv"],
+                        m=m, bias_a=L["bias_a"], bias_b=L["bias_b"], kv_raw=None, win=None,
+                        kv_gain=L["kv_gain"], kv_norm=False, rope_dims=wl.r,
+                        istreams=tuple(L[c] for c in ("ia", "ib", "iza", "izb")), ibias_a=L["ibias_a"],
+                        ibias_b=L["ibias_b"], iring=L["iring"], kI=L["kI"])
+    torch.cuda.synchronize()
+    assert torch.equal(L["win"].cpu(), host["win"])                 # no window row
+    for b in range(2):
+        pos = int(host["pos"][b])
+        ring = {s_: npy(host["ring"][b, :, j]) for j, s_ in enumerate(names)}
+        new = {s_: npy(host[c_][b]) for s_, c_ in zip(names, ("ca", "cb", "cza", "czb"))}
+        _, entry, _ = O.decode_compress_step("csa", pos, new, ring, (npy(host["bias_a"]), npy(host["bias_b"])),
+                                             m, r=wl.r, normalize=False)
+        iring = {s_: npy(host["iring"][b, :, j]) for j, s_ in enumerate(names)}
+        inew = {s_: npy(host[c_][b]) for s_, c_ in zip(names, ("ia", "ib", "iza", "izb"))}
+        _, ient, _ = O.decode_compress_step("csa", pos, inew, iring, (npy(host["ibias_a"]), npy(host["ibias_b"])),
+                                            m, normalize=False)
+        i = entry[0]
+        if i < N_cap:
+            check_close(npy(L["kv"][b, i]), entry[2], "bf16", f"b={b} entry without norm")
+            check_close(npy(L["kI"][b, i]), ient[1], "bf16", f"b={b} bf16 key")
+            assert torch.equal(L["kv"][b, :i].cpu(), host["kv"][b, :i])
+        else:                                                         # past the capacity: nothing stored
+            assert torch.equal(L["kv"][b].cpu(), host["kv"][b])
+            assert torch.equal(L["kI"][b].cpu(), host["kI"][b])
+        for j, c_ in enumerate(("ca", "cb", "cza", "czb")):
+            assert torch.equal(L["ring"][b, pos % (2 * m), j].cpu(), host[c_][b])
+    assert api.device_error() == 0
