@@ -301,7 +301,8 @@ size_t csahca_decode_workspace_size(const csahca_decode_args* args);
  *   [B, N_cap, d]; win [B, w, d]; ia, ib, iza, izb [B, dI] (dtype); ibias_a,
  *   ibias_b [m, dI] f32; kI [B, N_cap, dI]; kI_scale [B, N_cap, dI/128] f32.
  * Constraints: dtype F32 (d % 32 == 0) or BF16 (d % 64 == 0), d <= 128 * 16 /
- *   (element bytes); rope_dims even and <= d; dI = 0 or (CSA) dI % 8 == 0
+ *   (element bytes); rope_dims even, <= d and <= 128 (the RoPE angles are
+ *   computed on the host, one per pair); dI = 0 or (CSA) dI % 8 == 0
  *   with dI / 8 a multiple of the 16-byte vector and dividing 128 (BF16:
  *   64, 128, 256, 512, 1024; F32: 32, 64, 128, 256, 512); E4M3 keys need
  *   BF16 and dI % 128 == 0.  No workspace.  Rows of one sequence are written

@@ -95,6 +95,8 @@ def test_validation_rejects_before_launch(lib):
     assert lib.decode_compress(C.byref(dc), None) == N.ERR_UNSUPPORTED   # dI / 8 must divide 128
     dc = N.DecodeCompressArgs(kind=N.CSA, dtype=N.BF16, B=1, d=512, m=4, N_cap=4, rope_dims=3)
     assert lib.decode_compress(C.byref(dc), None) == N.ERR_INVALID_ARG
+    dc = N.DecodeCompressArgs(kind=N.CSA, dtype=N.BF16, B=1, d=512, m=4, N_cap=4, rope_dims=130)
+    assert lib.decode_compress(C.byref(dc), None) == N.ERR_UNSUPPORTED   # at most 64 RoPE pairs
     dc = N.DecodeCompressArgs(kind=N.HCA, dtype=N.BF16, B=1, d=512, m=128, N_cap=4, pos=16, a=16, za=16,
                               bias_a=16, ring=16, kv_cache=16)        # HCA needs no b / zb
     dc.kv_cache = 24
