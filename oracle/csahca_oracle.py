@@ -64,6 +64,11 @@ Readings where the pages are silent (each is a fixed constant of this code):
   R22 between decode steps a compressor keeps the raw streams of its last
       2m (CSA) or m' (HCA) tokens, token p in ring slot p mod 2m (or p mod m');
       the window row and the compressed rows share one norm gain.
+  R23 an FP8 KV cache ("Paper Breakdown: DeepSeek-V4", infrastructure table:
+      KV storage FP8 for the non-RoPE dims, BF16 for the RoPE dims) stores the
+      first d - r dims of a row as e4m3 with one fp32 scale per 64 of them (the
+      R21 rule) and the last r dims as bf16; attention reads the rows it
+      stands for.  The window ring stays bf16.
 
 Pins (what checks each function against something other than itself, in
 ``tests/test_oracle_pins.py`` and ``tests/golden/``):
@@ -72,6 +77,10 @@ Pins (what checks each function against something other than itself, in
   e4m3_encode           torch's round-to-nearest-even float8_e4m3fn cast on
                         random values and on every midpoint between codes;
                         saturation closed form; decode(encode(v)) = v.
+  quantize_kv_rows_fp8  the amax element of each 64-block lands on +-448, an
+                        all-zero block has scale 1 and zero codes, the RoPE dims
+                        are kept bit for bit, and every element of the
+                        dequantised row is within half an e4m3 step of it.
   decode_compress_step  run token by token from position 0, it emits exactly
                         the rows csa_pool / hca_pool + finish_rows give for the
                         whole stream, and the window rows of finish_rows.
@@ -147,6 +156,24 @@ def quantize_e4m3_rows_f32(x, block: int = 128):
     scale = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
     q = (xb / scale[..., None]).astype(np.float32)
     return e4m3_encode(q).reshape(x.shape), scale
+
+
+def quantize_kv_rows_fp8(rows, r: int, block: int = 64):
+    """FP8 storage of KV rows (reading R23): the first d - r ("non-RoPE")
+    dims as e4m3 codes with one fp32 scale per ``block`` of them, quantised
+    exactly as quantize_e4m3_rows_f32; the last r (RoPE) dims kept as given
+    (bf16 in the caches).  Returns (codes uint8 [..., d-r], scales f32
+    [..., (d-r)/block], rope [..., r] float64)."""
+    rows = np.asarray(rows, np.float64)
+    nr = rows.shape[-1] - r
+    codes, scales = quantize_e4m3_rows_f32(rows[..., :nr], block)
+    return codes, scales, rows[..., nr:].copy()
+
+
+def dequant_kv_rows_fp8(codes, scales, rope, block: int = 64) -> np.ndarray:
+    """The KV rows an FP8 cache stands for: decode(code) * scale on the
+    non-RoPE dims, the RoPE dims as stored."""
+    return np.concatenate([dequant_e4m3_rows(codes, scales, block), np.asarray(rope, np.float64)], axis=-1)
 
 
 def dequant_e4m3_rows(codes: np.ndarray, scales: np.ndarray, block: int = 128) -> np.ndarray:

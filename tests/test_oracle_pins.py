@@ -94,6 +94,34 @@ def test_quantize_e4m3_rows_f32():
     assert np.array_equal(codes, tc.numpy()) and np.array_equal(scales, ts.numpy())
 
 
+def check_kv_fp8(quant, dequant):
+    rng = np.random.default_rng(6)
+    d, r = 512, 64
+    x = torch.from_numpy(rng.standard_normal((5, d)) * np.exp2(rng.integers(-4, 4, (5, 1)))).to(
+        torch.bfloat16).to(torch.float64).numpy()
+    x[3, 64:128] = 0.0                                      # an all-zero block
+    codes, scales, rope = quant(x, r)
+    assert codes.shape == (5, d - r) and scales.shape == (5, (d - r) // 64) and rope.shape == (5, r)
+    assert np.array_equal(rope, x[:, d - r:])               # RoPE dims bit for bit
+    assert scales[3, 1] == 1.0 and not codes[3, 64:128].any()
+    blk = np.abs(x[:, :d - r]).reshape(5, -1, 64)
+    j = blk.argmax(axis=-1)
+    got = codes.reshape(5, -1, 64)[np.arange(5)[:, None], np.arange(blk.shape[1])[None], j]
+    nz = blk.max(axis=-1) > 0
+    assert ((got[nz] & 0x7F) == 0x7E).all()                 # the amax element maps to +-448
+    y = dequant(codes, scales, rope)
+    s_ = np.repeat(scales.astype(np.float64), 64, axis=-1)
+    v = np.abs(x[:, :d - r]) / s_
+    e = np.floor(np.log2(np.maximum(v, 2.0 ** -6)))         # e4m3 binade (subnormals share 2^-6's)
+    half_step = np.exp2(e - 4) * s_                         # 3 mantissa bits: half a step is 2^(e-4)
+    assert (np.abs(y[:, :d - r] - x[:, :d - r]) <= half_step * (1 + 1e-6)).all()
+    assert np.array_equal(y[:, d - r:], x[:, d - r:])
+
+
+def test_kv_fp8_rows():
+    check_kv_fp8(O.quantize_kv_rows_fp8, O.dequant_kv_rows_fp8)
+
+
 # ----------------------------------------------------------- compressors ----
 
 def check_csa_golden(pool, fx):
@@ -562,6 +590,17 @@ def test_pins_catch_planted_mistakes(golden_dir):
             i, raw, _ = entry
             entry = (i, raw, O.finish_rows(raw, t, gain, r))
         return out_ring, entry, win
+
+    def kv_quant_block_128(rows, r, block=64):              # scales per 128, read per 64
+        return O.quantize_kv_rows_fp8(rows, r, 128)
+
+    def kv_quant_rope_quantised(rows, r, block=64):         # RoPE dims through e4m3 too
+        c, s, rope = O.quantize_kv_rows_fp8(rows, r, block)
+        return c, s, O.e4m3_decode(O.e4m3_encode(rope)).astype(np.float64)
+
+    for bad in (kv_quant_block_128, kv_quant_rope_quantised):
+        with pytest.raises((AssertionError, ValueError)):
+            check_kv_fp8(bad, O.dequant_kv_rows_fp8)
 
     for kind in ("csa", "hca"):
         for bad in (step_ring_not_kept, step_rope_at_last_token):
