@@ -209,6 +209,8 @@ def decode_compress_args(kind, pos, streams, ring, kv_cache, *, m, bias_a, bias_
     if csa and istreams is not None:
         ia, ib, iza, izb = istreams
         dI = ia.shape[1]
+        if kI is None or iring is None or ibias_a is None or ibias_b is None:
+            raise ValueError("decode_compress: indexer streams need iring, ibias_a, ibias_b and kI")
     args = N.DecodeCompressArgs(
         kind=N.CSA if csa else N.HCA, dtype=_dt(a), B=B, d=d, m=m, N_cap=kv_cache.shape[1],
         w=win.shape[1] if win is not None else 0, rope_dims=rope_dims, rope_base=rope_base, eps=eps,
