@@ -4,7 +4,6 @@ float64 oracle ("Paper Breakdown: DeepSeek-V4", section 4; "How DeepSeek-V4
 architecture and training work together", "Two compressed views of one
 history": interleaved CSA / HCA layers, top-1,024 and a 128-token window)."""
 
-import numpy as np
 import pytest
 import torch
 

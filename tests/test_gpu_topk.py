@@ -5,7 +5,6 @@ scores on both sides the selection must match exactly, including ties, which
 go to the lower index ("Paper Breakdown: DeepSeek-V4", section 4, DSA on
 Compressed KV: the top-k entries by I_{t,s})."""
 
-import numpy as np
 import pytest
 import torch
 

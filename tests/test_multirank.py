@@ -5,7 +5,6 @@ max over ranks; no collective touches the data."""
 import os
 import socket
 
-import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
