@@ -87,8 +87,8 @@ Pins (what checks each function against something other than itself, in
   csa_pool              hand-worked fixture; constant streams -> 1 (weights sum
                         to 1); equal logits -> plain mean; one-hot logits copy
                         the named token of the named stream/block; causality.
-  hca_pool              equals csa_pool with stream b disabled (north-star
-                        invariant) and a hand-worked fixture.
+  hca_pool              equals csa_pool with stream b disabled (one stream, no
+                        overlap, m = m') and a hand-worked fixture.
   rms_norm              output RMS 1, scale invariance.
   rope                  closed form of one pair, orthogonality, composition,
                         relative-position property.

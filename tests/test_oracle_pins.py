@@ -147,8 +147,8 @@ def _streams(rng, n, c, m):
 
 
 def test_csa_pool_weights_sum_to_one():
-    """Spec invariant: pool weights sum to 1 per channel, so constant
-    streams pool to the constant whatever the logits."""
+    """The pool weights are a softmax, so they sum to 1 per channel and
+    constant streams pool to the constant whatever the logits."""
     rng = np.random.default_rng(1)
     s = _streams(rng, 37, 5, 4)
     s["Ca"] = np.full((37, 5), 3.0)
@@ -205,7 +205,8 @@ def test_csa_pool_dependencies():
 
 
 def test_hca_equals_csa_with_stream_b_disabled():
-    """Spec invariant: HCA(m') is CSA with m = m' and no overlap."""
+    """HCA(m') is CSA with m = m', one stream and no overlap ("Paper Breakdown:
+    DeepSeek-V4", section 4, HCA)."""
     rng = np.random.default_rng(5)
     n, c, m = 200, 6, 16
     s = _streams(rng, n, c, m)
@@ -380,8 +381,8 @@ def test_window_alone_is_sliding_window_sdpa():
 
 
 def test_hca_equals_csa_with_all_entries_selected():
-    """Spec invariant at the attention level: dense HCA over the visible
-    entries equals CSA whose top-k keeps every visible entry."""
+    """At the attention level: dense HCA over the visible entries equals CSA
+    whose top-k keeps every visible entry."""
     rng = np.random.default_rng(13)
     n, H, d, m, w, r = 64, 2, 16, 8, 5, 8
     kv = rng.standard_normal((n // m, d))
