@@ -45,3 +45,21 @@ def test_compressor_bytes_when_a_block_completes():
     # the first CSA block has no preceding block: 3 other tokens, stream a only
     assert bench.decode_compress_bytes(wl, "csa", 3) == 4 * (base_csa + 3 * 2 * 512 * 2 + 512 * 2 +
                                                              3 * 2 * 128 * 2 + 128 + 4)
+
+
+def test_prefill_128k_flops_closed_form():
+    """csa_prefill_128k: n = 131,072 = 4Q tokens (Q = 32,768), m = 4, k = 1,024,
+    w = 128, 64 indexer heads of 128 dims, 64 heads of 512 dims.
+    Indexer pairs: sum over u = 1..4Q of floor(u/4) = 2Q^2 - Q.
+    Attention keys: selected min(floor(u/4), 1024) -- 2*1024^2 - 2*1024 up to
+    u = 4,095, then 1,024 for each of the other 126,977 tokens -- plus the
+    window min(128, u): 128*129/2 + (131,072 - 128) * 128."""
+    pw = synth.WORKLOADS["csa_prefill_128k"]
+    Q = 32768
+    pairs = 2 * Q * Q - Q
+    keys = (2 * 1024 * 1024 - 2 * 1024) + (131072 - 4096 + 1) * 1024 + 128 * 129 // 2 + (131072 - 128) * 128
+    idx_fl, att_fl = bench.prefill_flops(pw)
+    assert idx_fl == pairs * 64 * 128 * 2 == 35_183_835_217_920
+    assert att_fl == keys * 64 * 512 * 4
+    assert keys == 148_888_640
+    assert idx_fl + att_fl == 54_698_967_040_000
