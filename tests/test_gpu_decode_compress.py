@@ -170,16 +170,14 @@ def test_decode_compress_decode_1m_shapes():
     assert api.device_error() == 0
 
 
-def test_bench_decode_step_with_compressors():
+def _check_bench_step(ctx, B, seqs):
     """The step bench.py times (per layer decode_compress then
-    compressed_attn_decode, CSA, HCA, CSA, HCA, replayed as a CUDA graph) at
-    a 32,767-token context, where the new token completes a CSA and an HCA
-    block, against the oracle's decode step.  Both sequences are checked.
-    Selections must pass the top-k tolerance and outputs are compared on the
-    GPU's selections."""
+    compressed_attn_decode, CSA, HCA, CSA, HCA, replayed as a CUDA graph)
+    against the oracle's decode step for the sequences `seqs`.  Selections
+    must pass the top-k tolerance and outputs are compared on the GPU's
+    selections."""
     wl = synth.WORKLOADS["decode_1m"]
-    ctx = (1 << 15) - 1
-    layers = synth.decode_inputs(wl, DEV, ctx=ctx, B=2)
+    layers = synth.decode_inputs(wl, DEV, ctx=ctx, B=B)
     host = bench.host_layers(layers)
     stream = torch.cuda.Stream()
     step = runtime.DecodeStep(wl, layers, stream, keep_idx=True)
@@ -189,7 +187,7 @@ def test_bench_decode_step_with_compressors():
             graph()                              # replays leave the same state
     torch.cuda.synchronize()
     assert api.device_error(stream) == 0
-    for b in range(2):
+    for b in seqs:
         scores = []
         bench.oracle_decode_sequence(wl, host, b, scores_out=scores)
         sels = [None if ix is None else npy(ix[b]) for ix in step.idx]
@@ -200,6 +198,20 @@ def test_bench_decode_step_with_compressors():
         ref = bench.oracle_decode_sequence(wl, host, b, sels=sels)
         for li, o in enumerate(step.outputs):
             check_close(npy(o[b]), ref[li], "bf16", f"layer {li} b={b}")
+
+
+def test_bench_decode_step_with_compressors():
+    """At a 32,767-token context, where the new token completes a CSA and an
+    HCA block; both sequences checked."""
+    _check_bench_step((1 << 15) - 1, 2, range(2))
+
+
+@pytest.mark.slow
+def test_bench_decode_step_full_size():
+    """decode_1m exactly as bench.py runs it: B = 4 at the full 1,048,576-token
+    context (262,144 CSA entries with e4m3 keys, 8,192 HCA entries per
+    sequence), the CUDA-graph step with compressors; sequence 0 checked."""
+    _check_bench_step(synth.WORKLOADS["decode_1m"].ctx, 4, [0])
 
 
 def test_decode_compress_options():
