@@ -94,6 +94,13 @@ Pins (what checks each function against something other than itself, in
                         relative-position property.
   indexer_scores        closed forms (ReLU(x)+ReLU(-x) = |x|; orthogonal q).
   top_k_select          brute force rank counting on tiny inputs.
+  attend_query          one key row RoPE_p(y), sink -inf: every head's output is
+                        RoPE_{p-t}(y), the expected value written as a complex
+                        product per pair (p > t included); shifting the query
+                        and every key position by the same delta leaves the
+                        output unchanged; the same closed form through
+                        decode_attention (one selected entry) and
+                        prefill_attention (one-token window).
   sink_attention,
   prefill/decode paths  m=1, all entries selected, no window, no RoPE, sink
                         -inf equals torch's scaled_dot_product_attention;

@@ -470,6 +470,72 @@ def test_decode_equals_prefill(kind):
         np.testing.assert_allclose(od, o[p], rtol=1e-12, atol=1e-14)
 
 
+# ------------------------------------------------- output de-rotation ----
+
+def _rotate_complex(y, delta, r, base=O.ROPE_BASE):
+    """Rotation of the last r dims by delta * base^(-2j/r), written as the
+    complex product (y_2j + i y_2j+1) * e^(i delta theta_j): an independent
+    statement of what RoPE does to one pair."""
+    y = np.array(y, np.float64, copy=True)
+    d = y.shape[-1]
+    theta = base ** (-2.0 * np.arange(r // 2) / r)
+    z = (y[..., d - r::2] + 1j * y[..., d - r + 1::2]) * np.exp(1j * np.asarray(delta, np.float64)[..., None] * theta)
+    y[..., d - r::2] = z.real
+    y[..., d - r + 1::2] = z.imag
+    return y
+
+
+def check_output_derotation(attend):
+    """Reading R7 ("relative position on core outputs"): the output's rope
+    dims are rotated back by -t, so
+      (a) one key row RoPE_p(y) with sink -inf gives every head exactly
+          RoPE_{p-t}(y), whatever the query (p > t included);
+      (b) shifting the query position and every key position by the same
+          delta leaves the output unchanged (only relative positions count).
+    ``attend`` has attend_query's signature."""
+    rng = np.random.default_rng(18)
+    H, d, r = 3, 16, 8
+    tau = 1 / math.sqrt(d)
+    no_sink = np.full(H, -np.inf)
+    for p, t in [(12, 20), (0, 7), (36, 20), (100, 3), (5, 5)]:
+        y = rng.standard_normal(d)
+        q = O.rope(rng.standard_normal((H, d)), t, r)
+        o = attend(q, _rotate_complex(y, p, r)[None], no_sink, t, r, tau)
+        np.testing.assert_allclose(o, np.tile(_rotate_complex(y, p - t, r), (H, 1)), rtol=1e-12, atol=1e-12)
+    ys, x = rng.standard_normal((6, d)), rng.standard_normal((H, d))
+    ps, t, sinks = np.array([0, 4, 8, 20, 31, 33]), 33, rng.standard_normal(H)
+    ref = attend(O.rope(x, t, r), O.rope(ys, ps, r), sinks, t, r, tau)
+    for delta in (1, 57, 1000):
+        got = attend(O.rope(x, t + delta, r), O.rope(ys, ps + delta, r), sinks, t + delta, r, tau)
+        np.testing.assert_allclose(got, ref, rtol=1e-10, atol=1e-12)
+
+
+def test_output_derotation():
+    check_output_derotation(O.attend_query)
+
+
+def test_output_derotation_through_layers():
+    """The same closed form through the decode and prefill paths: one selected
+    entry (finished at i*m) as the only key, and a one-token window (the
+    query's own row, p = t, so the output is the unrotated normed row)."""
+    rng = np.random.default_rng(19)
+    H, d, r, m, N = 2, 16, 8, 4, 30
+    raw = rng.standard_normal((N, d))
+    gain = 1 + 0.1 * rng.standard_normal(d)
+    normed = raw / np.sqrt((raw * raw).mean(-1, keepdims=True) + O.RMS_EPS) * gain
+    kv = O.finish_rows(raw, np.arange(N) * m, gain, r)
+    no_sink = np.full(H, -np.inf)
+    for i, pos in [(3, 50), (7, 29), (20, 41)]:
+        od = O.decode_attention("csa", rng.standard_normal((H, d)), pos, kv, np.zeros((0, d)), no_sink,
+                                m=m, w=0, r=r, sel=np.array([i, -1]))
+        np.testing.assert_allclose(od, np.tile(_rotate_complex(normed[i], i * m - pos, r), (H, 1)),
+                                   rtol=1e-12, atol=1e-12)
+    n = 24
+    op = O.prefill_attention("hca", rng.standard_normal((n, H, d)), np.zeros((0, d)), raw[:n], no_sink,
+                             m=64, w=1, r=r, kv_gain=gain)
+    np.testing.assert_allclose(op, np.repeat(normed[:n, None], H, axis=1), rtol=1e-12, atol=1e-12)
+
+
 # ------------------------------------------------ decode compressor step ----
 
 def _decode_stream(kind, n, c, m, seed):
@@ -607,3 +673,13 @@ def test_pins_catch_planted_mistakes(golden_dir):
         for bad in (step_ring_not_kept, step_rope_at_last_token):
             with pytest.raises(AssertionError):
                 check_decode_compress_step(bad, kind)
+
+    def attend_rotated_forward(q, rows, sinks, t, r, tau, base=O.ROPE_BASE):     # +t, not -t
+        return O.rope(O.sink_attention(q, rows, sinks, tau), t, r, base)
+
+    def attend_not_rotated(q, rows, sinks, t, r, tau, base=O.ROPE_BASE):         # no de-rotation
+        return O.sink_attention(q, rows, sinks, tau)
+
+    for bad in (attend_rotated_forward, attend_not_rotated):
+        with pytest.raises(AssertionError):
+            check_output_derotation(bad)
