@@ -2,14 +2,19 @@
 """Throughput of the CSA + HCA compressed-attention hot path on B200.
 
 One step = one decode step of the decode_1m workload through the C ABI:
-4 sequences x 4 layers (CSA, HCA, CSA, HCA) at a cached context of 1,048,576
-tokens (CSA 4:1 with e4m3 indexer keys and top-1024, HCA 128:1 dense, 128-token
-window, 64 heads of 512 dims).  `value` = tokens/s over all ranks (each rank
-runs its own 4 sequences: weak scaling, no collective on the data path).
-With --prefill the line also carries the csa_prefill_128k layer (one CSA
-prefill of 131,072 tokens: both compressors, indexer top-k, attention).
+4 sequences x 4 layers (CSA, HCA, CSA, HCA) at a cached context of about
+1,048,576 tokens (CSA 4:1 with e4m3 indexer keys and top-1024, HCA 128:1
+dense, 128-token window, 64 heads of 512 dims).  The K timed steps take
+consecutive positions, so the compressors complete a CSA block every fourth
+step and one HCA block mid-run, as in a real decode.  `value` = tokens/s over
+all ranks (each rank runs its own 4 sequences: weak scaling, no collective on
+the data path).  The line also carries the decode_256k workload (8 sequences,
+one CSA + one HCA layer at 262,144 tokens) and the csa_prefill_128k layer (one
+CSA prefill of 131,072 tokens: both compressors, indexer top-k, attention)
+against the sustained dense bf16 peak.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--no-prefill] [--no-256k]
 
 --impl reference times the float64 CPU oracle (the only reference that
 exists for this path) on a bounded sample of the same workload.
@@ -272,34 +277,166 @@ def kernel_bytes_key(name):
     return None
 
 
-def time_steps(step, K, stream, flush, world):
-    """K steps, each bracketed by CUDA events on `stream`, L2 flushed between
-    steps (outside the events).  Returns the max over ranks of the summed
-    device time in ms."""
+def time_steps(step, K, stream, between, world):
+    """K steps, each bracketed by CUDA events on `stream`; between(i) runs
+    before step i outside the events (L2 flush, position of the step).
+    Returns (max over ranks of the summed device time in ms, per-step ms of
+    this rank)."""
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     barrier(world)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         for i in range(K):
-            flush()
+            between(i)
             starts[i].record(stream)
             step()
             ends[i].record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    total = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    return max_over_ranks(total, world)
+    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    return max_over_ranks(sum(per), world), per
+
+
+def run_start(wl, K):
+    """First position of a run of K consecutive decode steps: the cached
+    context is wl.ctx tokens or a few more, CSA blocks complete at every
+    fourth step and one HCA block (position = -1 mod m') completes in the
+    middle of the run."""
+    mh = wl.m_hca
+    return wl.ctx + mh - (K + 1) // 2 - (wl.ctx % mh) if K < mh else wl.ctx
+
+
+def step_kind(wl, pos):
+    """Which compressors complete a block at this position."""
+    hca = any(k == "hca" for k in wl.layers) and (pos + 1) % wl.m_hca == 0
+    csa = any(k == "csa" for k in wl.layers) and (pos + 1) % wl.m == 0
+    return "csa_and_hca_block" if (csa and hca) else "hca_block" if hca else "csa_block" if csa else "no_block"
+
+
+def decode_run(wl, args, dev, stream, world, rank, want_cpu, e2e=True):
+    """Time K consecutive decode steps of workload `wl` (all its layers and
+    sequences) through the C ABI, launched as one CUDA graph per step; a
+    second, traced pass gives the per-kernel times; optionally the same run
+    end to end from host buffers, and the oracle on the host."""
+    K = args.steps
+    p0 = run_start(wl, K)
+    positions = [p0 + i for i in range(K)]
+    layers = synth.decode_inputs(runtime.shard_workload(wl, rank), dev, ctx=p0, room=K)
+    io = runtime.StepIO(layers, dev)            # per-step inputs / outputs in one arena each
+    layers_host = host_layers(layers) if want_cpu else None   # the oracle's copy, before any kernel
+    eager = runtime.DecodeStep(wl, layers, stream)
+    step = eager if args.no_graph else runtime.DecodeGraph(eager)
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def set_pos(p):
+        for L in layers:
+            L["pos"].fill_(p)
+
+    def between(i):
+        flush_buf.random_(0, 255)
+        set_pos(positions[i % K])
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            between(i)
+            step()
+    torch.cuda.synchronize()
+    if api.device_error(stream) != 0:
+        raise RuntimeError("device error flag set during warm-up")
+
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    total_ms, per_step = time_steps(step, K, stream, between, world)
+    clk = clocks.stop()
+    ms_per_step = total_ms / K
+    tokens = world * wl.B * K
+    value = tokens / (total_ms / 1000.0)
+    kinds = {}
+    for p, ms in zip(positions, per_step):
+        kinds.setdefault(step_kind(wl, p), []).append(ms)
+
+    # traced pass: per-kernel device time of the same K steps (eager launches,
+    # so every kernel is bracketed by its own events)
+    api.trace_enable(True)
+    time_steps(eager, K, stream, between, world)
+    traced = api.trace_collect()
+    api.trace_enable(False)
+
+    pk = peaks()
+    per_pos = [decode_bytes_per_kernel(wl, p) for p in positions]
+    per_bytes = {k_: sum(d[k_] for d in per_pos) / K for k_ in per_pos[0]}
+    dom = max(traced.items(), key=lambda kv: kv[1][1])
+    dname, (dl, dms) = dom
+    key = kernel_bytes_key(dname)
+    roof = None
+    if key is not None:
+        ach = per_bytes[key] / (dms / dl / 1000.0) / 1e9
+        roof = {"kernel": dname, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": ach / pk["hbm_gbs"], "traffic": ncu_traffic(dname),
+                "peak_source": pk["source"], "launches": dl, "avg_us": 1000 * dms / dl}
+    step_bytes = sum(decode_step_bytes(wl, p) for p in positions) / K
+    step_frac = step_bytes / (ms_per_step / 1000.0) / 1e9 / pk["hbm_gbs"]
+    out = {
+        "value": value, "ms_per_step": ms_per_step, "tokens_per_step": world * wl.B,
+        "positions": [positions[0], positions[-1]],
+        "ms_per_step_by_kind": {k_: {"steps": len(v), "ms": sum(v) / len(v)} for k_, v in sorted(kinds.items())},
+        "roofline": roof,
+        "step_hbm": {"algorithmic_bytes": step_bytes, "frac": step_frac, "peak": pk["hbm_gbs"],
+                     "peak_source": pk["source"]},
+        "clocks": clk,
+        "gpu_launches": sum(v[0] for v in traced.values()) // K * K,
+        "kernels_ms_per_step": {k_: v[1] / K for k_, v in traced.items()},
+        "launch": "eager" if args.no_graph else "cuda_graph",
+    }
+
+    if e2e:
+        # end to end: each step's inputs (positions included) copied in from
+        # pinned host memory and its outputs read back, one copy each way
+        # (the layers' tensors are views of the two arenas)
+        host_inps = []
+        for p in positions:
+            set_pos(p)
+            host_inps.append(io.inp.cpu().pin_memory())
+        host_outp = torch.empty(io.out.shape, dtype=io.out.dtype).pin_memory()
+        h2d, d2h = io.inp.numel(), io.out.numel()
+        state = {"i": 0}
+
+        def e2e_between(i):
+            flush_buf.random_(0, 255)
+            state["i"] = i
+
+        def e2e_step():
+            io.inp.copy_(host_inps[state["i"] % K], non_blocking=True)
+            step()
+            host_outp.copy_(io.out, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            e2e_step()
+        torch.cuda.synchronize()
+        e2e_ms, _ = time_steps(e2e_step, K, stream, e2e_between, world)
+        out["e2e"] = {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h}
+    if api.device_error(stream) != 0:
+        raise RuntimeError("device error flag set during the timed region")
+    if want_cpu:
+        out["cpu_baseline"] = cpu_baseline(wl, layers_host)
+    del step, eager
+    return out
 
 
 # -------------------------------------------------------------- prefill ----
 
 def prefill_layer_fn(wl, dev, stream):
+    """One csa_prefill_128k layer through the C ABI: both compressors, the
+    indexer top-k and the attention.  Returns (step, inputs, state) where
+    state holds the last step's compressed rows, indexer keys and output."""
     inp = synth.prefill_inputs(wl, dev)
     kvi, ik = inp["kv"], inp["ik"]
     q_pos = torch.arange(wl.n, device=dev, dtype=torch.int32)[None].repeat(wl.B, 1).contiguous()
     idx = torch.empty(wl.B, wl.n, wl.k, dtype=torch.int32, device=dev)
     out = torch.empty_like(inp["q"])
+    state = {"idx": idx, "out": out}
 
     def step():
         with torch.cuda.stream(stream):
@@ -312,7 +449,8 @@ def prefill_layer_fn(wl, dev, stream):
             api.compressed_attn_prefill("csa", inp["q"], kv, inp["kv_win"], inp["sinks"], m=wl.m,
                                         w=wl.w, rope_dims=wl.r, idx=idx, q_gain=inp["q_gain"],
                                         kv_gain=inp["kv_gain"], out=out, stream=stream)
-    return step
+            state["kv"], state["kI"] = kv, kI
+    return step, inp, state
 
 
 def prefill_flops(wl):
@@ -324,6 +462,63 @@ def prefill_flops(wl):
     idx_fl = pairs * wl.HI * wl.dI * 2
     att_fl = keys * wl.H * wl.d * 4
     return idx_fl, att_fl
+
+
+def prefill_row_flops(wl, t):
+    """Algorithmic flops of query t (indexer over its visible entries plus
+    attention over its selected entries and window)."""
+    v = (t + 1) // wl.m
+    return v * wl.HI * wl.dI * 2 + (min(v, wl.k) + min(wl.w, t + 1)) * wl.H * wl.d * 4
+
+
+def prefill_kernel_flops(name, idx_fl, att_fl):
+    if name.startswith("indexer_scores_tc_prefill"):
+        return idx_fl
+    if name.startswith("attn_prefill"):
+        return att_fl
+    return None
+
+
+def prefill_run(args, dev, stream, world, want_cpu):
+    """Time the csa_prefill_128k layer (compressors, indexer top-k, attention)
+    with per-kernel events; roofline against the sustained dense bf16 peak."""
+    pw = synth.WORKLOADS["csa_prefill_128k"]
+    pstep, inp, state = prefill_layer_fn(pw, dev, stream)
+    pstep()
+    torch.cuda.synchronize()
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    api.trace_enable(True)
+    p_ms, _ = time_steps(pstep, args.prefill_steps, stream, lambda i: flush_buf.random_(0, 255), world)
+    ptr = api.trace_collect()
+    api.trace_enable(False)
+    if api.device_error(stream) != 0:
+        raise RuntimeError("device error flag set during the prefill run")
+    idx_fl, att_fl = prefill_flops(pw)
+    tot_fl = idx_fl + att_fl
+    pk = peaks()
+    peak_tf = pk["bf16_tflops_sustained"]
+    ms_layer = p_ms / args.prefill_steps
+    kernels = {k_: {"launches_per_layer": v[0] / args.prefill_steps, "ms_per_layer": v[1] / args.prefill_steps}
+               for k_, v in ptr.items()}
+    dname, (dl, dms) = max(ptr.items(), key=lambda kv: kv[1][1])
+    dfl = prefill_kernel_flops(dname, idx_fl, att_fl)
+    roof = None
+    if dfl is not None:
+        ach = dfl / (dms / args.prefill_steps / 1000.0) / 1e12
+        roof = {"kernel": dname, "bound": "tensor", "achieved": ach, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": ach / peak_tf, "traffic": ncu_traffic(dname), "peak_source": pk["source"] + " (sustained)",
+                "flops_per_layer": dfl, "ms_per_layer": dms / args.prefill_steps}
+    out = {"workload": pw.name, "value": world * pw.n / (ms_layer / 1000), "unit": "tokens/s",
+           "ms_per_layer": ms_layer, "steps": args.prefill_steps,
+           "tflops": tot_fl / (ms_layer / 1000) / 1e12,
+           "frac_of_bf16_peak": tot_fl / (ms_layer / 1000) / 1e12 / peak_tf,
+           "peak_tflops": peak_tf, "peak_source": pk["source"] + " (sustained)",
+           "algorithmic_flops": tot_fl, "roofline": roof,
+           "gpu_launches": sum(v[0] for v in ptr.values()),
+           "kernels": kernels}
+    if want_cpu:
+        out["cpu_baseline"] = prefill_cpu_baseline(pw, inp, state)
+    return out
 
 
 # ------------------------------------------------------------ CPU oracle ----
@@ -427,6 +622,56 @@ def cpu_baseline(wl, layers_host, budget_s=12.0):
                       f"(float64 NumPy, {el:.1f} s)"}
 
 
+def prefill_cpu_baseline(pw, inp, state, rows=96, entries=512):
+    """The oracle on a bounded sample of the csa_prefill_128k layer,
+    extrapolated to the whole layer: both compressors on their first
+    `entries` entries, then for `rows` seeded queries (uniform over t) the
+    indexer scores over every visible entry, the top-k and the attention over
+    the selection and the window.  The compressor time scales by
+    N_c / entries, the query time by the ratio of the algorithmic flops of
+    all n queries to those of the sample."""
+    from oracle import csahca_oracle as O
+
+    def npy(t):
+        return t.detach().cpu().to(torch.float64).numpy()
+
+    m, n = pw.m, pw.n
+    toks = slice(0, entries * m)
+    comp_in = [tuple(npy(st[k_][0, toks]) for k_ in ("a", "b", "za", "zb")) + (npy(st["bias_a"]), npy(st["bias_b"]))
+               for st in (inp["kv"], inp["ik"])]
+    ts = np.sort(np.random.default_rng(2).choice(n, rows, replace=False))
+    sel_t = torch.as_tensor(ts, device=inp["q"].device)
+    KI, KV = npy(state["kI"][0]), npy(state["kv"][0])
+    qI, w = npy(inp["qI"][0].index_select(0, sel_t)), npy(inp["w"][0].index_select(0, sel_t))
+    q = npy(inp["q"][0].index_select(0, sel_t))
+    kv_win = npy(inp["kv_win"][0])
+    sinks, qg, kg = npy(inp["sinks"]), npy(inp["q_gain"]), npy(inp["kv_gain"])
+    t0 = time.perf_counter()
+    for j, args_ in enumerate(comp_in):
+        pooled = O.csa_pool(*args_, m)
+        if j == 0:
+            O.finish_rows(pooled, np.arange(pooled.shape[0]) * m, kg, pw.r)
+    t_comp = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    for j, t in enumerate(ts):
+        t = int(t)
+        sc = O.indexer_scores(qI[j], w[j], KI[: O.n_visible(t, m)])
+        sel = O.top_k_select(sc, pw.k)
+        O.prefill_attention("csa", q[j:j + 1], KV, kv_win, sinks, m=m, w=pw.w, r=pw.r, q_gain=qg,
+                            kv_gain=kg, idx={t: sel}, rows=[t], q_holds_rows=True)
+    t_rows = time.perf_counter() - t1
+    idx_fl, att_fl = prefill_flops(pw)
+    sample_fl = sum(prefill_row_flops(pw, int(t)) for t in ts)
+    n_c = n // m
+    est = t_comp * n_c / entries + t_rows * (idx_fl + att_fl) / sample_fl
+    return {"value": pw.B * n / est, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "extrapolated": True, "measured_s": t_comp + t_rows,
+            "sample": f"extrapolated: both compressors on {entries} of {n_c} entries (x{n_c // entries}) and "
+                      f"{rows} seeded queries of {n} (indexer, top-k, attention; scaled by the algorithmic "
+                      f"flop ratio {(idx_fl + att_fl) / sample_fl:.0f}), float64 NumPy, "
+                      f"{t_comp + t_rows:.1f} s measured"}
+
+
 # ------------------------------------------------------------------ main ----
 
 def run_reference(args, world, rank):
@@ -476,7 +721,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode_1m")
-    ap.add_argument("--prefill", action="store_true", help="also time csa_prefill_128k")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the csa_prefill_128k layer")
+    ap.add_argument("--no-256k", action="store_true", help="skip the decode_256k run")
     ap.add_argument("--prefill-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the decode step eagerly")
@@ -494,123 +740,39 @@ def main():
     dev = torch.device("cuda", local)
     stream = torch.cuda.Stream(device=dev)
     wl = synth.WORKLOADS[args.workload]
-    layers = synth.decode_inputs(runtime.shard_workload(wl, rank), dev)
-    io = runtime.StepIO(layers, dev)            # per-step inputs / outputs in one arena each
     want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
-    # the oracle's copy of the inputs, taken before any kernel runs
-    layers_host = host_layers(layers) if want_cpu else None
-    eager = runtime.DecodeStep(wl, layers, stream)
-    step = eager
-    launch_mode = "eager"
-    if not args.no_graph:
-        step = runtime.DecodeGraph(eager)
-        launch_mode = "cuda_graph"
-    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
-
-    def flush():
-        flush_buf.random_(0, 255)
-
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            step()
-    torch.cuda.synchronize()
-    if api.device_error(stream) != 0:
-        raise RuntimeError("device error flag set during warm-up")
-
-    clocks = ClockSampler(local)
-    clocks.start()
-    total_ms = time_steps(step, args.steps, stream, flush, world)
-    clk = clocks.stop()
-    ms_per_step = total_ms / args.steps
-    tokens = world * wl.B * args.steps
-    value = tokens / (total_ms / 1000.0)
-
-    # traced pass: per-kernel device time of the same K steps (eager launches,
-    # so every kernel is bracketed by its own events)
-    api.trace_enable(True)
-    time_steps(eager, args.steps, stream, flush, world)
-    traced = api.trace_collect()
-    api.trace_enable(False)
-
-    pk = peaks()
-    per_bytes = decode_bytes_per_kernel(wl, wl.ctx)
-    dom = max(traced.items(), key=lambda kv: kv[1][1])
-    dname, (dl, dms) = dom
-    key = kernel_bytes_key(dname)
-    roof = None
-    if key is not None:
-        ach = per_bytes[key] / (dms / dl / 1000.0) / 1e9
-        roof = {"kernel": dname, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": ach / pk["hbm_gbs"], "traffic": ncu_traffic(dname),
-                "peak_source": pk["source"], "launches": dl, "avg_us": 1000 * dms / dl}
-    step_bytes = decode_step_bytes(wl, wl.ctx)
-    step_frac = step_bytes / (ms_per_step / 1000.0) / 1e9 / pk["hbm_gbs"]
-
-    # end to end: the step's inputs copied in from pinned host memory and its
-    # outputs read back, one copy each way (the layers' tensors are views of
-    # the two arenas)
-    host_inp = io.inp.cpu().pin_memory()
-    host_outp = torch.empty(io.out.shape, dtype=io.out.dtype).pin_memory()
-    h2d = io.inp.numel()
-    d2h = io.out.numel()
-
-    def e2e_step():
-        io.inp.copy_(host_inp, non_blocking=True)
-        step()
-        host_outp.copy_(io.out, non_blocking=True)
-
-    with torch.cuda.stream(stream):
-        e2e_step()
-    torch.cuda.synchronize()
-    e2e_ms = time_steps(e2e_step, args.steps, stream, flush, world)
-    e2e_val = tokens / (e2e_ms / 1000.0)
-
+    main_run = decode_run(wl, args, dev, stream, world, rank, want_cpu)
+    extra = None
+    if not args.no_256k and args.workload != "decode_256k":
+        extra = decode_run(synth.WORKLOADS["decode_256k"], args, dev, stream, world, rank, False, e2e=False)
+        extra["workload"] = "decode_256k"
+    torch.cuda.empty_cache()
     prefill = None
-    if args.prefill:
-        pw = synth.WORKLOADS["csa_prefill_128k"]
-        pstep = prefill_layer_fn(pw, dev, stream)
-        for _ in range(max(1, args.warmup // 3)):
-            pstep()
-        torch.cuda.synchronize()
-        api.trace_enable(True)
-        p_ms = time_steps(pstep, args.prefill_steps, stream, flush, world)
-        ptr = api.trace_collect()
-        api.trace_enable(False)
-        idx_fl, att_fl = prefill_flops(pw)
-        tot_fl = idx_fl + att_fl
-        peak_tf = pk["bf16_tflops_sustained"]
-        prefill = {"workload": pw.name, "tokens_per_s": world * pw.n * args.prefill_steps / (p_ms / 1000),
-                   "ms_per_layer": p_ms / args.prefill_steps,
-                   "tflops": tot_fl / (p_ms / args.prefill_steps / 1000) / 1e12,
-                   "frac_of_bf16_peak": tot_fl / (p_ms / args.prefill_steps / 1000) / 1e12 / peak_tf,
-                   "peak_tflops": peak_tf, "algorithmic_flops": tot_fl,
-                   "kernels_ms_per_layer": {k_: v[1] / args.prefill_steps for k_, v in ptr.items()}}
+    if not args.no_prefill:
+        prefill = prefill_run(args, dev, stream, world, want_cpu)
 
-    cpu = None
-    if want_cpu:
-        cpu = cpu_baseline(wl, layers_host)
-
-    if api.device_error(stream) != 0:
-        raise RuntimeError("device error flag set during the timed region")
-    launches = sum(v[0] for v in traced.values()) // args.steps * args.steps
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "metric": METRIC, "value": main_run["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": main_run["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": wl.name, "global_batch": world * wl.B, "seq_len": wl.ctx,
+                   "positions": main_run["positions"],
                    "layers": list(wl.layers), "heads": wl.H, "head_dim": wl.d, "top_k": wl.k,
                    "window": wl.w, "indexer_keys": "e4m3" if wl.fp8_keys else "bf16",
                    "parallelism": f"replicas{world}" if world > 1 else "none",
-                   "launch": launch_mode, "l2": "flushed between timed steps"},
-        "roofline": roof,
-        "step_hbm": {"algorithmic_bytes": step_bytes, "frac": step_frac, "peak": pk["hbm_gbs"]},
-        "clocks": clk,
-        "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches,
-        "kernels_ms_per_step": {k_: v[1] / args.steps for k_, v in traced.items()},
-        "cpu_baseline": cpu,
+                   "launch": main_run["launch"], "l2": "flushed between timed steps",
+                   "steps": "consecutive decode positions; CSA blocks complete every 4th step, "
+                            "one HCA block mid-run"},
+        "roofline": main_run["roofline"],
+        "step_hbm": main_run["step_hbm"],
+        "ms_per_step_by_kind": main_run["ms_per_step_by_kind"],
+        "clocks": main_run["clocks"],
+        "e2e": main_run.get("e2e"),
+        "gpu_launches": main_run["gpu_launches"],
+        "kernels_ms_per_step": main_run["kernels_ms_per_step"],
+        "cpu_baseline": main_run.get("cpu_baseline"),
+        "decode_256k": extra,
         "prefill": prefill,
     }
     if rank == 0:

@@ -167,8 +167,11 @@ size_t csahca_indexer_workspace_size(const csahca_indexer_args* args);
  *     args) exceeds CSAHCA_NOALLOC_SCRATCH_BYTES is rejected with
  *     CSAHCA_ERR_WORKSPACE before any launch.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current, and caches it; make that
- *     first call outside any stream capture.
+ *     (cudaGetSymbolAddress) with that device current, and caches it with the
+ *     id of the current context; make that first call outside any stream
+ *     capture.  After a device reset (cudaDeviceReset, or any teardown of the
+ *     primary context) the next call sees a new context id and looks the
+ *     address up again, so make that call outside capture too.
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents (the parts that must start at zero are cleared by each call).
  *     Calls whose work overlaps on the GPU (other streams, or other host

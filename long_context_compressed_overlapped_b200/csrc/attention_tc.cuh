@@ -211,8 +211,14 @@ struct AttnSmem {
   static constexpr int TOTAL = 1024 + Q_BYTES + K_BYTES + P_BYTES;
 };
 
-// Decode partial of one (query, split): m[H], l[H] fp32, then O / l fp16 [D][H].
-constexpr int kTcPartialHeader = 2 * kAttnH * 4;
+// Decode partial of one (query, split): m[H], l[H] and up[H] fp32, then
+// O / (l up) fp16 [D][H].  up is a power of two, 1 unless the head's largest
+// |O / l| exceeds kPartialMaxAbs: the bf16 value rows behind O / l may be far
+// beyond fp16's range, and scaling them down by an exact power of two keeps
+// the stored partial finite without rounding it any further.
+constexpr int kTcHdrFloats = 3 * kAttnH;
+constexpr int kTcPartialHeader = kTcHdrFloats * 4;
+constexpr float kPartialMaxAbs = 16384.f;
 constexpr int kTcPartialBytes = kTcPartialHeader + kAttnD * kAttnH * 2;
 // The same blocks seen as 128-byte rows (64 fp16), as the TMA store writes them.
 constexpr int kTcPartialRows = kTcPartialBytes / 128;
@@ -241,6 +247,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
   __shared__ volatile int abort_flag;
   __shared__ float red[2][4 * 32];
   __shared__ __align__(16) float stat_a[kAttnH];
+  __shared__ __align__(16) float stat_b[kAttnH];
   __shared__ __align__(16) float m_use[kAttnH];
   __shared__ __align__(16) float sc_h[kAttnH];     // softmax scale of head h (log2 units, times inv_rms_h)
   __shared__ __align__(16) float alpha[kAttnH];
@@ -754,10 +761,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       bad = softmax_any256(bad);             // the output stage is entered by both groups or neither
       if (!bad) {
         if (kDecode) {
-          // partial block of (query, split): m[H] (log2 units) and l[H] in
-          // fp32, then O / l as fp16 [D][H] (a thread writes its dim's 32
-          // heads, 64 contiguous bytes, straight from TMEM); an empty split
-          // writes only m = -inf, which the combine skips
+          // partial block of (query, split): m[H] (log2 units), l[H] and
+          // up[H] in fp32, then O / (l up) as fp16 [D][H] (a thread writes its
+          // dim's 32 heads, 64 contiguous bytes, straight from TMEM); an empty
+          // split writes only its header, m = -inf, which the combine skips
           char* P = reinterpret_cast<char*>(p.partial) +
                     (((int64_t)it.b * p.nq + it.qi) * p.splits + it.split) * kTcPartialBytes;
           float* hdr = reinterpret_cast<float*>(P);
@@ -766,10 +773,40 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
             const float l = empty ? 0.f : l_run[h];
             hdr[h] = empty ? -INFINITY : m_use[h];
             hdr[kAttnH + h] = l;
+            hdr[2 * kAttnH + h] = 1.f;
             stat_a[h] = l > 0.f ? 1.f / l : 0.f;
           }
           group_sync(gid);
           if (!empty) {
+            // per-head largest |O| over the 512 dims (this thread's dim of each
+            // M-tile, then over the group's 128 threads), and from it the
+            // power of two `up` that keeps |O / (l up)| <= kPartialMaxAbs
+            {
+              float amax[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) amax[e] = 0.f;
+#pragma unroll 1
+              for (int mt = 0; mt < kAttnMT; ++mt) {
+                float o[32];
+                tmem_ld32(tO + lane_base + mt * kAttnH + h0, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) amax[e] = fmaxf(amax[e], fabsf(o[e]));
+              }
+              reduce_group32<true>(amax, red[g], stat_b + h0, gid);
+            }
+            if (tid < 32) {
+              const int h = h0 + tid;
+              const float mx = stat_b[h] * stat_a[h];
+              if (mx > kPartialMaxAbs) {
+                int e2 = 0;
+                frexpf(mx / kPartialMaxAbs, &e2);          // mx / kPartialMaxAbs < 2^e2
+                const float up = ldexpf(1.f, e2);
+                hdr[2 * kAttnH + h] = up;
+                stat_a[h] = stat_a[h] / up;                // exact: up is a power of two
+              }
+            }
+            group_sync(gid);
             // O / l of M-tile mt: 128 dims x 64 heads fp16 = 128-byte rows,
             // staged in P's buffer with the 128-byte swizzle (group g writes
             // pieces 4g..4g+3 of row tid) and stored by one TMA box
@@ -877,7 +914,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
 
 // ---------------------------------------------------------------------------
 // Split-KV combine of the tensor-core decode partials, with the sink and the
-// output de-rotation: o = sum_s f_s (O_s / l_s), f_s = l_s 2^(m_s - M) / den,
+// output de-rotation: o = sum_s f_s up_s (O_s / (l_s up_s)), f_s = l_s 2^(m_s - M) / den,
 // den = 2^(z_h log2 e - M) + sum_s l_s 2^(m_s - M), M the largest of them; the
 // rope dims of o are then rotated by -t.  One CTA per (query, 16 dims).  The
 // m, l headers of every split and the 16-dim slices (16 x 64 fp16 per split)
@@ -905,8 +942,8 @@ __host__ __device__ inline int tc_combine_smem_bytes(int splits) {
   return splits * kTcPartialHeader + slots * kTcCombineSlice;
 }
 
-// hdr_map: the partials as [blocks][516 rows][64 fp16], box [splits][4][64]
-// (the m, l headers of all splits of one query); slc_map: the same tensor,
+// hdr_map: the partials as [blocks][518 rows][64 fp16], box [splits][6][64]
+// (the m, l, up headers of all splits of one query); slc_map: the same tensor,
 // box [min(splits, 64)][16][64] (16 dims of up to 64 splits).  A bulk copy per
 // split was measured to complete one copy at a time; a box covering every
 // split goes out as one transfer.
@@ -921,7 +958,7 @@ __global__ void __launch_bounds__(kTcCombineThreads) attn_combine_tc_kernel(
   __shared__ __align__(16) __nv_bfloat16 ostage[kAttnH][kTcCombineDims];
   __shared__ volatile int abort_flag;
   constexpr int kChunks = kAttnD / kTcCombineDims;
-  float* hdr = reinterpret_cast<float*>(cmb_smem);              // [splits][m[H], l[H]]; m slots -> weights
+  float* hdr = reinterpret_cast<float*>(cmb_smem);              // [splits][m[H], l[H], up[H]]; m slots -> weights
   uint8_t* slots = cmb_smem + p.splits * kTcPartialHeader;        // [slots][16 dims][H] fp16
   const int nslots = p.splits < kTcCombineSlots ? p.splits : kTcCombineSlots;
   const int row = blockIdx.x / kChunks, dc = blockIdx.x % kChunks;
@@ -953,7 +990,7 @@ __global__ void __launch_bounds__(kTcCombineThreads) attn_combine_tc_kernel(
   float mx = -INFINITY;
   if (ok) {
 #pragma unroll 4
-    for (int s = part; s < p.splits; s += 8) mx = fmaxf(mx, hdr[s * 2 * kAttnH + h]);
+    for (int s = part; s < p.splits; s += 8) mx = fmaxf(mx, hdr[s * kTcHdrFloats + h]);
   }
   red[part][h] = mx;
   __syncthreads();
@@ -964,9 +1001,9 @@ __global__ void __launch_bounds__(kTcCombineThreads) attn_combine_tc_kernel(
   if (ok)
 #pragma unroll 4
     for (int s = part; s < p.splits; s += 8) {
-      const float ms = hdr[s * 2 * kAttnH + h];
-      const float f = ms == -INFINITY ? 0.f : hdr[s * 2 * kAttnH + kAttnH + h] * exp2f(ms - M);
-      hdr[s * 2 * kAttnH + h] = f;
+      const float ms = hdr[s * kTcHdrFloats + h];
+      const float f = ms == -INFINITY ? 0.f : hdr[s * kTcHdrFloats + kAttnH + h] * exp2f(ms - M);
+      hdr[s * kTcHdrFloats + h] = f * hdr[s * kTcHdrFloats + 2 * kAttnH + h];   // weight of the stored slice
       den += f;
     }
   __syncthreads();                                 // every read of red[] (M) is done
@@ -999,12 +1036,12 @@ __global__ void __launch_bounds__(kTcCombineThreads) attn_combine_tc_kernel(
     ok = mbar_wait(&bar_slc, round & 1, &abort_flag) && ok;
     if (ok) {
       const int n = min(p.splits, s0 + nslots) - s0;
-      const float* wb = hdr + s0 * 2 * kAttnH + hg * 8;
+      const float* wb = hdr + s0 * kTcHdrFloats + hg * 8;
       const uint8_t* sb = slots + dl * (kAttnH * 2) + hg * 16;
 #pragma unroll 2
       for (int i = qt; i < n; i += 4) {
-        const float4 w0 = *reinterpret_cast<const float4*>(wb + i * 2 * kAttnH);
-        const float4 w1 = *reinterpret_cast<const float4*>(wb + i * 2 * kAttnH + 4);
+        const float4 w0 = *reinterpret_cast<const float4*>(wb + i * kTcHdrFloats);
+        const float4 w1 = *reinterpret_cast<const float4*>(wb + i * kTcHdrFloats + 4);
         uint4 raw = *reinterpret_cast<const uint4*>(sb + i * kTcCombineSlice);
         // an empty split (all weights 0) has a header but no written slice
         const bool live = (w0.x != 0.f) | (w0.y != 0.f) | (w0.z != 0.f) | (w0.w != 0.f) | (w1.x != 0.f) |

@@ -895,8 +895,8 @@ int run_decode_t(const csahca_decode_args* a, cudaStream_t s, char* ws) {
     const int smem = tc_combine_smem_bytes(L.splits);
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(attn_combine_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    // the partials as [B * splits blocks][516 rows][64 fp16]: one box takes
-    // the m, l headers of every split of a query, one the 16-dim slices
+    // the partials as [B * splits blocks][518 rows][64 fp16]: one box takes
+    // the m, l, up headers of every split of a query, one the 16-dim slices
     CUtensorMap hdr_map, slc_map;
     const uint64_t blocks = (uint64_t)a->B * L.splits;
     const uint32_t slc_box = (uint32_t)(L.splits < kTcCombineSlots ? L.splits : kTcCombineSlots);
@@ -1135,26 +1135,53 @@ constexpr size_t kNoAllocScratchBytes = CSAHCA_NOALLOC_SCRATCH_BYTES;
 constexpr int kNoAllocMaxDevices = 64;
 
 // Host code must not pass the array's name to a kernel: on the host it is only
-// a stand-in symbol.  Its device address comes from cudaGetSymbolAddress, once
-// per device (with that device current), and is cached here.
+// a stand-in symbol.  Its device address comes from cudaGetSymbolAddress with
+// the device current, and is cached per device together with the id of the
+// context it was looked up in: after a device reset (a new primary context)
+// the next call looks the address up again instead of using a stale one.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kNoAllocMaxDevices];
+struct NoAllocSlot { unsigned long long ctx_id; void* ptr; };
+NoAllocSlot g_noalloc_slot[kNoAllocMaxDevices];
+
+// Unique id of the calling thread's current context (0 if none or unknown).
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  if (!get_cur || !get_id) {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) { (void)cudaGetLastError(); return 0; }
+    get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) { (void)cudaGetLastError(); return 0; }
+    get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 int noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) { (void)cudaGetLastError(); return CSAHCA_ERR_NO_DEVICE; }
   if (dev < 0 || dev >= kNoAllocMaxDevices) return CSAHCA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  NoAllocSlot& slot = g_noalloc_slot[dev];
+  const unsigned long long id = current_context_id();
+  if (!slot.ptr || id == 0 || slot.ctx_id != id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
       (void)cudaGetLastError();
       return CSAHCA_ERR_LAUNCH;
     }
-    g_noalloc_ptr[dev] = p;
+    // (cudaGetSymbolAddress made the primary context current if none was)
+    slot.ptr = p;
+    slot.ctx_id = id != 0 ? id : current_context_id();
   }
-  *out = g_noalloc_ptr[dev];
+  *out = slot.ptr;
   return CSAHCA_OK;
 }
 

@@ -177,13 +177,14 @@ def prefill_inputs(wl: Workload, device="cpu", n: int | None = None, B: int | No
 
 
 def decode_inputs(wl: Workload, device="cpu", ctx: int | None = None, B: int | None = None,
-                  layers=None):
+                  layers=None, room: int = 0):
     """Per-layer decode state and new-token inputs.
 
     For each layer L: caches already final (Gaussian rows as drawn), with room
-    for every entry the new token at position ctx completes: CSA kv
-    [B, (ctx+1)/m, d], indexer keys [B, (ctx+1)/m, d_I] (bf16, or e4m3 codes +
-    fp32 scales), HCA kv [B, (ctx+1)/m', d]; window ring [B, w, d]; new query
+    for every entry the new token at position ctx completes, and for those of
+    ``room`` further positions: CSA kv [B, (ctx+room+1)/m, d], indexer keys
+    [B, (ctx+room+1)/m, d_I] (bf16, or e4m3 codes + fp32 scales), HCA kv
+    [B, (ctx+room+1)/m', d]; window ring [B, w, d]; new query
     q [B, H, d] at position ctx, qI [B, H_I, d_I], w [B, H_I]; sinks [H].
     Compressor state and the new token's compressor inputs: ring [B, R, S, d]
     of the raw streams of the R tokens before it (R = 2m, S = 4 for CSA:
@@ -202,7 +203,7 @@ def decode_inputs(wl: Workload, device="cpu", ctx: int | None = None, B: int | N
     for li, kind in enumerate(layers):
         t = f"L{li}"
         m = wl.m if kind == "csa" else wl.m_hca
-        N = (ctx + 1) // m
+        N = (ctx + room + 1) // m
         L = {
             "kind": kind, "m": m,
             "pos": torch.full((B,), ctx, dtype=torch.int32, device=device),

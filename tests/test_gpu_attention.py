@@ -129,3 +129,81 @@ def test_prefill_hca_64_heads_512_dims(n, w):
         ref = _oracle_rows("hca", inp, kv, None, wl, m, b, rows)
         check_close(npy(out[b, rows]), ref, "bf16", f"hca64 b={b}")
     assert api.device_error() == 0
+
+
+def _gain(name, d, seed):
+    """A non-unit RMSNorm gain, 1 + 0.1 N(0, 1) per dim."""
+    return 1.0 + synth.Draw(seed, DEV).normal(name, (d,), 0.1)
+
+
+@pytest.mark.parametrize("kind", ["csa", "hca"])
+def test_prefill_tc_non_unit_gains(kind):
+    """Non-unit query and KV gains on the tensor-core path (H = 64, d = 512):
+    the query prologue multiplies q by its gain before RoPE (a separate branch
+    from the all-ones one), the compressor and the window rows use the KV gain."""
+    wl = synth.Workload(**{**synth.WORKLOADS["csa_prefill_128k"].__dict__, "kind": kind})
+    n = 4096 + 3 if kind == "csa" else 2048 + 5
+    inp = synth.prefill_inputs(wl, DEV, n=n, B=1)
+    inp["q_gain"] = _gain("q_gain", wl.d, 21)
+    inp["kv_gain"] = _gain("kv_gain", wl.d, 22)
+    kvi = inp["kv"]
+    m = wl.m if kind == "csa" else wl.m_hca
+    idx = None
+    if kind == "csa":
+        kv = api.csa_compress(kvi["a"], kvi["b"], kvi["za"], kvi["zb"], kvi["bias_a"],
+                              kvi["bias_b"], m, gain=inp["kv_gain"], rope_dims=wl.r)
+        ik = inp["ik"]
+        kI = api.csa_compress(ik["a"], ik["b"], ik["za"], ik["zb"], ik["bias_a"], ik["bias_b"], m,
+                              rms_norm=False)
+        q_pos = torch.arange(n, device=DEV, dtype=torch.int32)[None]
+        idx = api.indexer_topk(inp["qI"], inp["w"], kI, q_pos, m, wl.k)
+    else:
+        kv = api.hca_compress(kvi["a"], kvi["za"], kvi["bias_a"], m, gain=inp["kv_gain"],
+                              rope_dims=wl.r)
+    # the compressor rows against the oracle's, gain included
+    from tests.helpers import oracle_compress
+    ents = [0, 1, kv.shape[1] // 2, kv.shape[1] - 1]
+    check_close(npy(kv[0, ents]), oracle_compress(kind, kvi, m, 0, ents, True, inp["kv_gain"], wl.r),
+                "bf16", "compress gain")
+    out = api.compressed_attn_prefill(kind, inp["q"], kv, inp["kv_win"], inp["sinks"], m=m,
+                                      w=wl.w, rope_dims=wl.r, idx=idx, q_gain=inp["q_gain"],
+                                      kv_gain=inp["kv_gain"])
+    rows = _sample(n, [0, 3, 4, 127, 128, m - 1, m, n - 1], seed=5, count=12)
+    ref = _oracle_rows(kind, inp, kv, idx, wl, m, 0, rows)
+    check_close(npy(out[0, rows]), ref, "bf16", f"{kind} prefill gains")
+    assert api.device_error() == 0
+
+
+@pytest.mark.slow
+def test_prefill_csa_128k_full_size_sampled():
+    """csa_prefill_128k at its full size (n = 131,072, the layer bench.py
+    times): both compressors, indexer top-k and attention on the GPU; 64
+    seeded sampled queries checked against the oracle -- queries with fewer
+    visible entries than k (t < 4,096), rows of 16,384 < v <= 32,768 visible
+    entries, block boundaries and t = n - 1.  Top-k sets under the tie-band
+    rule; outputs with the oracle on the GPU's own index set."""
+    from tests.helpers import check_topk
+    wl = synth.WORKLOADS["csa_prefill_128k"]
+    n = wl.n
+    inp, kv, m = _prefill_layer(wl, n, 1)
+    ik = inp["ik"]
+    kI = api.csa_compress(ik["a"], ik["b"], ik["za"], ik["zb"], ik["bias_a"], ik["bias_b"], m,
+                          rms_norm=False)
+    q_pos = torch.arange(n, device=DEV, dtype=torch.int32)[None]
+    idx = api.indexer_topk(inp["qI"], inp["w"], kI, q_pos, m, wl.k)
+    out = api.compressed_attn_prefill("csa", inp["q"], kv, inp["kv_win"], inp["sinks"], m=m,
+                                      w=wl.w, rope_dims=wl.r, idx=idx, q_gain=inp["q_gain"],
+                                      kv_gain=inp["kv_gain"])
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(2)
+    fixed = [0, 3, 4, 4095, 4096, 4 * wl.k - 1, 4 * wl.k, 65535, 65536, 65539, n - 2, n - 1]
+    rows = np.unique(np.r_[fixed, rng.integers(0, 4096, 12), rng.integers(65536, n, 30),
+                           rng.integers(4096, 65536, 10)])[:64]
+    KI = npy(kI[0])
+    for t in rows:
+        v = O.n_visible(int(t), m)
+        s = O.indexer_scores(npy(inp["qI"][0, t]), npy(inp["w"][0, t]), KI[:v])
+        check_topk(npy(idx[0, t]), s, wl.k, f"t={t}")
+    ref = _oracle_rows("csa", inp, kv, idx, wl, m, 0, rows)
+    check_close(npy(out[0, rows]), ref, "bf16", "csa prefill 128k")
+    assert api.device_error() == 0

@@ -103,3 +103,59 @@ def test_decode_1m_full_size_one_sequence_checked():
         out = _decode_layer(L, wl, idx_out=idx)
         _check_layer(L, wl, out, idx, [0])
     assert api.device_error() == 0
+
+
+@pytest.mark.parametrize("wl_name", ["decode_256k", "decode_1m"])
+def test_decode_non_unit_query_gain(wl_name):
+    """A non-unit query gain (1 + 0.1 N(0, 1) per dim) on the tensor-core
+    decode path of both layer kinds: the prologue multiplies q by the gain
+    before RoPE and takes the RMS from the raw values."""
+    wl = synth.WORKLOADS[wl_name]
+    layers = synth.decode_inputs(wl, DEV, ctx=16384 + 3, B=2)
+    for li, L in enumerate(layers):
+        L["q_gain"] = 1.0 + synth.Draw(30 + li, DEV).normal("q_gain", (wl.d,), 0.1)
+        idx = torch.empty(2, wl.k, dtype=torch.int32, device=DEV) if L["kind"] == "csa" else None
+        out = _decode_layer(L, wl, idx_out=idx)
+        _check_layer(L, wl, out, idx, range(2))
+    assert api.device_error() == 0
+
+
+def test_decode_large_value_rows():
+    """Cache and window rows scaled by 1e5 (finite in bf16, far beyond fp16's
+    65,504): the split partials must stay finite and the output match the
+    oracle (compared after dividing both by the scale, with the bf16
+    tolerances).  A query gain of 1e-5 keeps the scores at their usual size,
+    so the softmax weights are as in an unscaled layer and only the values
+    are large."""
+    wl = synth.WORKLOADS["decode_256k"]
+    scale = 1e5
+    layers = synth.decode_inputs(wl, DEV, ctx=8192 + 5, B=2)
+    for L in layers:
+        L["kv"] = (L["kv"].float() * scale).to(torch.bfloat16)
+        L["win"] = (L["win"].float() * scale).to(torch.bfloat16)
+        L["q_gain"] = torch.full((wl.d,), 1.0 / scale, device=DEV)
+        idx = torch.empty(2, wl.k, dtype=torch.int32, device=DEV) if L["kind"] == "csa" else None
+        out = _decode_layer(L, wl, idx_out=idx)
+        assert torch.isfinite(out.float()).all(), f"{L['kind']}: non-finite output"
+        for b in range(2):
+            pos = int(L["pos"][b])
+            sel = npy(idx[b]) if idx is not None else None
+            ref = O.decode_attention(L["kind"], npy(L["q"][b]), pos, npy(L["kv"][b]), npy(L["win"][b]),
+                                     npy(L["sinks"]), m=L["m"], w=wl.w, r=wl.r,
+                                     q_gain=npy(L["q_gain"]), sel=sel)
+            check_close(npy(out[b]) / scale, ref / scale, "bf16", f"{L['kind']} x1e5 b={b}")
+    assert api.device_error() == 0
+
+
+@pytest.mark.slow
+def test_decode_256k_full_size_all_sequences():
+    """decode_256k at its full size: B = 8 sequences at a 262,144-token
+    context (65,536 CSA entries with bf16 indexer keys, 2,048 HCA entries),
+    one CSA and one HCA layer; every sequence checked."""
+    wl = synth.WORKLOADS["decode_256k"]
+    layers = synth.decode_inputs(wl, DEV)
+    for L in layers:
+        idx = torch.empty(wl.B, wl.k, dtype=torch.int32, device=DEV) if L["kind"] == "csa" else None
+        out = _decode_layer(L, wl, idx_out=idx)
+        _check_layer(L, wl, out, idx, range(wl.B))
+    assert api.device_error() == 0
