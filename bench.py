@@ -622,7 +622,7 @@ def cpu_baseline(wl, layers_host, budget_s=12.0):
                       f"(float64 NumPy, {el:.1f} s)"}
 
 
-def prefill_cpu_baseline(pw, inp, state, rows=96, entries=512):
+def prefill_cpu_baseline(pw, inp, state, rows=2048, entries=4096):
     """The oracle on a bounded sample of the csa_prefill_128k layer,
     extrapolated to the whole layer: both compressors on their first
     `entries` entries, then for `rows` seeded queries (uniform over t) the
