@@ -218,12 +218,14 @@ def decode_bytes_per_kernel(wl, ctx):
     vc = (ctx + 1) // wl.m
     vh = (ctx + 1) // wl.m_hca
     key_row = dI + 4 * (dI // 128) if wl.fp8_keys else 2 * dI
+    # a cache row: d bf16, or (FP8 KV) d - r codes + r bf16 + (d - r) / 64 fp32 scales
+    kv_row = (d - wl.r) + 2 * wl.r + 4 * ((d - wl.r) // 64) if wl.fp8_kv else 2 * d
     qo = 2 * H * d * 2
     return {
         "indexer_scores": B * (vc * key_row + HI * dI * 2 + HI * 4),
         "topk_rows": B * (vc * 4 + k * 4),
-        "attn_decode_csa": B * ((k + w) * d * 2 + qo),
-        "attn_decode_hca": B * ((vh + w) * d * 2 + qo),
+        "attn_decode_csa": B * (k * kv_row + w * d * 2 + qo),
+        "attn_decode_hca": B * (vh * kv_row + w * d * 2 + qo),
         "decode_compress": sum(decode_compress_bytes(wl, kd, ctx) for kd in wl.layers) / len(wl.layers),
     }
 
@@ -243,7 +245,8 @@ def decode_compress_bytes(wl, kind, pos):
     if (pos + 1) % m == 0:
         i = (pos + 1) // m - 1
         J = m if (kind == "hca" or i == 0) else 2 * m
-        per += (J - 1) * 2 * wl.d * es + wl.d * es
+        kv_row = (wl.d - wl.r) + 2 * wl.r + 4 * ((wl.d - wl.r) // 64) if wl.fp8_kv else wl.d * es
+        per += (J - 1) * 2 * wl.d * es + kv_row
         if kind == "csa":
             key = wl.dI + 4 * (wl.dI // 128) if wl.fp8_keys else wl.dI * es
             per += (J - 1) * 2 * wl.dI * es + key
@@ -325,6 +328,8 @@ def decode_run(wl, args, dev, stream, world, rank, want_cpu, e2e=True):
     layers = synth.decode_inputs(runtime.shard_workload(wl, rank), dev, ctx=p0, room=K)
     io = runtime.StepIO(layers, dev)            # per-step inputs / outputs in one arena each
     layers_host = host_layers(layers) if want_cpu else None   # the oracle's copy, before any kernel
+    # the inputs are made on the current stream; the step runs on `stream`
+    torch.cuda.synchronize()
     eager = runtime.DecodeStep(wl, layers, stream)
     step = eager if args.no_graph else runtime.DecodeGraph(eager)
     flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
@@ -484,6 +489,7 @@ def prefill_run(args, dev, stream, world, want_cpu):
     with per-kernel events; roofline against the sustained dense bf16 peak."""
     pw = synth.WORKLOADS["csa_prefill_128k"]
     pstep, inp, state = prefill_layer_fn(pw, dev, stream)
+    torch.cuda.synchronize()                    # inputs made on the current stream; the layer runs on `stream`
     pstep()
     torch.cuda.synchronize()
     flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
@@ -562,10 +568,15 @@ def oracle_decode_sequence(wl, layers, b, sels=None, scores_out=None):
                                                    r=wl.r)
         win = npy(L["win"][b])
         win[pos % wl.w] = win_row
-        kv = npy(L["kv"][b])
+        fp8_kv = L["kv"].dtype == torch.uint8
+        if fp8_kv:
+            # the rows an FP8 KV cache stands for, and the new entry as stored
+            kv = O.dequant_kv_rows_fp8(*(npy(t_) for t_ in synth.unpack_kv_rows_fp8(L["kv"][b], wl.d, wl.r)))
+        else:
+            kv = npy(L["kv"][b])
         N_cap = kv.shape[0]
         if entry is not None and entry[0] < N_cap:
-            kv[entry[0]] = entry[2]
+            kv[entry[0]] = O.dequant_kv_rows_fp8(*O.quantize_kv_rows_fp8(entry[2], wl.r)) if fp8_kv else entry[2]
         sel = None
         if csa:
             v = min(O.n_visible(pos, m), N_cap)
@@ -723,6 +734,7 @@ def main():
     ap.add_argument("--workload", default="decode_1m")
     ap.add_argument("--no-prefill", action="store_true", help="skip the csa_prefill_128k layer")
     ap.add_argument("--no-256k", action="store_true", help="skip the decode_256k run")
+    ap.add_argument("--no-fp8kv", action="store_true", help="skip the decode_1m run with FP8 KV caches")
     ap.add_argument("--prefill-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the decode step eagerly")
@@ -746,6 +758,11 @@ def main():
     if not args.no_256k and args.workload != "decode_256k":
         extra = decode_run(synth.WORKLOADS["decode_256k"], args, dev, stream, world, rank, False, e2e=False)
         extra["workload"] = "decode_256k"
+    torch.cuda.empty_cache()
+    fp8kv = None
+    if not args.no_fp8kv and args.workload == "decode_1m":
+        fp8kv = decode_run(synth.WORKLOADS["decode_1m_fp8kv"], args, dev, stream, world, rank, False, e2e=False)
+        fp8kv["workload"] = "decode_1m_fp8kv"
     torch.cuda.empty_cache()
     prefill = None
     if not args.no_prefill:
@@ -773,6 +790,7 @@ def main():
         "kernels_ms_per_step": main_run["kernels_ms_per_step"],
         "cpu_baseline": main_run.get("cpu_baseline"),
         "decode_256k": extra,
+        "decode_1m_fp8kv": fp8kv,
         "prefill": prefill,
     }
     if rank == 0:

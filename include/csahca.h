@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define CSAHCA_ABI_VERSION 2
+#define CSAHCA_ABI_VERSION 4
 
 /* ---- status codes ------------------------------------------------------- */
 enum {
@@ -128,6 +128,14 @@ int hca_compress(const csahca_compress_args* args, void* stream);
  *   only, else NULL); q_pos [B, nq] int32 on the device; idx [B, nq, k] int32.
  *   scores_out: optional [B, nq, N] f32; entries i < v of each row receive
  *   I_{t,i}, the rest is left untouched.  q_pos values < 0 give v = 0.
+ *   sel_scores: optional [B, nq, k] f32; receives I_{t,idx} for each entry
+ *   of idx (-inf where idx = -1): the candidates context parallelism
+ *   exchanges (cp_topk_merge below).
+ *   entry_base (>= 0; 0 for a whole cache): kI holds the global entries
+ *   entry_base .. entry_base + N - 1 of a longer cache (one rank's shard under
+ *   context parallelism).  Local row j is global entry entry_base + j, visible
+ *   iff entry_base + j < (t+1)/m, so v = clamp((t+1)/m - entry_base, 0, N);
+ *   idx, scores_out and sel_scores address LOCAL rows.
  * Constraints: k >= 1; dI % 8 == 0; E4M3 needs dI % 128 == 0 and the same
  *   q_dtype rules; q_dtype == k_dtype unless k_dtype is E4M3 (queries BF16).
  * Workspace: csahca_indexer_workspace_size().
@@ -138,7 +146,7 @@ typedef struct {
   int32_t N;
   int32_t m;
   int32_t k;
-  int32_t reserved0;
+  int32_t entry_base;
   const void* qI;
   const float* w;
   const void* kI;
@@ -146,6 +154,7 @@ typedef struct {
   const int32_t* q_pos;
   int32_t* idx;
   float* scores_out;
+  float* sel_scores;
   void* workspace;
   size_t workspace_bytes;
 } csahca_indexer_args;
@@ -227,6 +236,24 @@ typedef struct {
 int compressed_attn_prefill(const csahca_attn_args* args, void* stream);
 size_t csahca_prefill_workspace_size(const csahca_attn_args* args);
 
+/* ---- FP8 KV cache rows ------------------------------------------------------
+ * [P2] infrastructure table: KV cache storage FP8 for the non-RoPE dims, BF16
+ * for the RoPE dims.  A row of kv_dtype CSAHCA_E4M3 (d and r = rope_dims with
+ * d - r and r multiples of 64) is csahca_kv_row_bytes() bytes:
+ *   bytes [0, d - r)                 e4m3 codes of dims 0 .. d - r - 1
+ *   bytes [d - r, d + r)             the r RoPE dims as bf16
+ *   bytes [d + r, d + r + 4 nb)      fp32 scale of each of the nb = (d - r) / 64
+ *                                    64-dim blocks: amax / 448 (1 for an
+ *                                    all-zero block); codes = nearest e4m3 of
+ *                                    x / scale, ties to even, saturating
+ *   then padding to a multiple of 128 bytes (never read).
+ * Dim j < d - r of the row stands for decode(code_j) * scale_{j / 64}.  The
+ * window ring stays bf16.  d = 512, r = 64: 448 + 128 + 28 -> 640 bytes. */
+
+/* Bytes of one cache row: d times the element size for F32 / BF16, the FP8
+ * layout above for E4M3; 0 for an invalid combination. */
+int64_t csahca_kv_row_bytes(int32_t kv_dtype, int32_t d, int32_t rope_dims);
+
 /* ---- compressed_attn_decode -----------------------------------------------
  * One decode step of one layer (CSA or HCA) for B sequences, one new query
  * token each at position pos[b] (device int32).  Caches hold final rows
@@ -240,6 +267,27 @@ size_t csahca_prefill_workspace_size(const csahca_attn_args* args);
  *   idx_out [B, k] (optional) receives the selection used.
  * HCA: dense over every visible entry.  Output and sink exactly as in
  * compressed_attn_prefill; out [B, H, d] (dtype).
+ * kv_dtype CSAHCA_E4M3: kv_cache holds FP8 KV rows (layout above,
+ *   [B, N_cap, csahca_kv_row_bytes] bytes), read as the rows they stand for;
+ *   dtype BF16, H = 64, d = 512, rope_dims 64 or 128, else
+ *   CSAHCA_ERR_UNSUPPORTED.  Any other kv_dtype: rows of `dtype`.
+ * Context parallelism (one rank's share of a layer whose compressed cache is
+ *   split by entry range across ranks; tensor-core shapes only: BF16, H = 64,
+ *   d = 512, rope_dims <= 128, B * N_cap >= 128 and B * w >= 128, else
+ *   CSAHCA_ERR_UNSUPPORTED):
+ *   entry_base: kv_cache (and kI) hold the global entries entry_base ..
+ *     entry_base + N_cap - 1; visibility as in indexer_topk's entry_base.
+ *     CSA with entry_base > 0 needs idx_in (LOCAL rows, -1 to skip; as
+ *     cp_topk_merge writes them).
+ *   skip_window != 0: the window is left out (another rank attends it); win
+ *     must still point at a [B, w, d] ring (it is not read).
+ *   partial_out != NULL: instead of `out` (which may then be NULL), each row's
+ *     unnormalised share of the softmax is written as one block of
+ *     2H + H*d floats: mx[H], the largest scaled logit of the head in base-2
+ *     units (s * scale * log2(e)), -inf if the rank attends no key; l[H] =
+ *     sum over the keys of 2^(logit2 - mx) (0 if none); o[H][d] = the
+ *     weighted mean of the keys' rows (0 if none).  The sink is left out and
+ *     the output is not de-rotated: cp_attn_merge does both once.
  * Workspace: csahca_decode_workspace_size().
  */
 typedef struct {
@@ -257,6 +305,8 @@ typedef struct {
   int32_t k;
   int32_t HI, dI;
   int32_t qI_dtype, kI_dtype;
+  int32_t kv_dtype;    /* CSAHCA_E4M3: FP8 KV rows; else rows of dtype */
+  int32_t entry_base;  /* context parallelism: first global entry of kv_cache */
   const void* q;
   const int32_t* pos;
   const float* q_gain;
@@ -270,6 +320,9 @@ typedef struct {
   const int32_t* idx_in;
   int32_t* idx_out;
   void* out;
+  float* partial_out;  /* context parallelism: [B, 2H + H*d] f32 instead of out */
+  int32_t skip_window; /* context parallelism: leave the window out */
+  int32_t reserved2;
   void* workspace;
   size_t workspace_bytes;
 } csahca_decode_args;
@@ -298,7 +351,14 @@ size_t csahca_decode_workspace_size(const csahca_decode_args* args);
  *      each 128-element block j (1 for an all-zero block) and codes the
  *      nearest e4m3 of x / scale (ties to even, saturating at 448), all in
  *      fp32.  Entries with i >= N_cap are not stored.  A sequence with
- *      pos[b] < 0 is left untouched.
+ *      pos[b] < 0 is left untouched.  With kv_dtype CSAHCA_E4M3 the entry is
+ *      stored as an FP8 KV row (layout above: the finished row's non-RoPE
+ *      dims quantised in fp32 against their 64-dim block scales, the RoPE
+ *      dims as bf16); dtype BF16, d = 512, rope_dims 64 or 128 only.
+ *   entry_base (>= 0): kv_cache and kI hold the global entries entry_base ..
+ *      entry_base + N_cap - 1 (context parallelism); entry i is stored in local
+ *      row i - entry_base when entry_base <= i < entry_base + N_cap, else not
+ *      at all.  The rings and the window are kept whatever entry_base is.
  * Layout: pos [B]; kv_raw, a, b, za, zb [B, d] (dtype; b, zb CSA only);
  *   bias_a, bias_b [m, d] f32; kv_gain [d] f32 or NULL (ones); kv_cache
  *   [B, N_cap, d]; win [B, w, d]; ia, ib, iza, izb [B, dI] (dtype); ibias_a,
@@ -324,7 +384,9 @@ typedef struct {
   int32_t kv_norm;
   int32_t dI;
   int32_t kI_dtype;
-  int32_t reserved0;
+  int32_t kv_dtype;    /* CSAHCA_E4M3: kv_cache holds FP8 KV rows; else rows of dtype */
+  int32_t entry_base;  /* context parallelism: first global entry of kv_cache / kI */
+  int32_t reserved1;
   const int32_t* pos;
   const void* kv_raw;
   const void* a;
@@ -350,6 +412,74 @@ typedef struct {
 
 int decode_compress(const csahca_decode_compress_args* args, void* stream);
 
+/* ---- context parallelism: the two exchange steps ------------------------------
+ * [P2] infrastructure table, "2-Stage Context Parallel" for compressed
+ * attention (the pages name it and give no steps; the reading taken here):
+ * a layer's compressed cache is split by entry range over R ranks, rank r
+ * holding the global entries bases[r] .. bases[r] + N_r - 1 (ranges
+ * disjoint), and the window and sink are attended once.  A decode step is
+ *   stage 1 (CSA only): each rank runs indexer_topk over its shard
+ *     (entry_base = bases[r], sel_scores), the ranks exchange their k
+ *     candidates (local rows and scores; an all-gather), and every rank
+ *     merges them with cp_topk_merge into the global top-k, which equals the
+ *     top-k over the whole cache (every entry of it is in the top-k of its
+ *     own shard);
+ *   stage 2: each rank runs compressed_attn_decode over its shard (entry_base,
+ *     partial_out; CSA with the merge's local rows as idx_in; skip_window on
+ *     every rank but one), the ranks exchange the partials (an all-gather),
+ *     and cp_attn_merge combines them with the sink and de-rotates the output.
+ * The collectives themselves belong to the caller (NCCL, or anything that
+ * lays the ranks' buffers out rank-major as stated below). */
+#define CSAHCA_CP_MAX_RANKS 64
+
+/* cp_topk_merge: the global top-k of one step from every rank's candidates.
+ * cand_idx [R, rows, k] int32 (rank r's LOCAL rows, -1 = none) and
+ * cand_scores [R, rows, k] f32, as indexer_topk writes idx / sel_scores;
+ * bases[R] on the HOST (copied at the call).  Candidate (r, j) is global
+ * entry bases[r] + cand_idx[r, row, j]; the k of largest score are kept, ties
+ * to the lower global entry, exactly as indexer_topk ranks one cache.
+ * Outputs [rows, k] int32, both optional, in the same order (ascending global
+ * entry, -1 padded when fewer than k candidates exist): idx_global (global
+ * entries) and idx_local (the entry's local row if it belongs to rank
+ * `rank`, else -1: compressed_attn_decode's idx_in for that rank).
+ * Constraints: 1 <= R <= CSAHCA_CP_MAX_RANKS; 1 <= k <= 4096; R * k <= 16384;
+ * bases[r] >= 0 and every global entry < 2^31.  No workspace. */
+typedef struct {
+  int32_t R, rows, k;
+  int32_t rank;
+  const int32_t* bases;
+  const int32_t* cand_idx;
+  const float* cand_scores;
+  int32_t* idx_global;
+  int32_t* idx_local;
+} csahca_cp_topk_merge_args;
+
+int cp_topk_merge(const csahca_cp_topk_merge_args* args, void* stream);
+
+/* cp_attn_merge: the layer's output from every rank's partial (the
+ * partial_out blocks of compressed_attn_decode, laid out [R, rows, 2H + H*d]
+ * f32): per row and head, M = max(z_h log2(e), mx_r), weights
+ * c_r = l_r 2^(mx_r - M), D = sum_r c_r + 2^(z_h log2(e) - M), and
+ * out = sum_r (c_r / D) o_r, whose last rope_dims dims are then rotated back
+ * by -pos[row] (RoPE pairs as above, base rope_base).
+ * Layout: partials [R, rows, 2H + H*d] f32; sinks [H] f32; pos [rows] int32;
+ * out [rows, H, d] (dtype F32 or BF16).  Constraints: 1 <= R <=
+ * CSAHCA_CP_MAX_RANKS; d % 4 == 0, d <= 1024; rope_dims even, <= d and <= 128.
+ * No workspace. */
+typedef struct {
+  int32_t dtype;
+  int32_t R, rows, H, d;
+  int32_t rope_dims;
+  float rope_base;     /* 0 -> 10000 */
+  int32_t reserved0;
+  const float* partials;
+  const float* sinks;
+  const int32_t* pos;
+  void* out;
+} csahca_cp_merge_args;
+
+int cp_attn_merge(const csahca_cp_merge_args* args, void* stream);
+
 /* ---- utilities ------------------------------------------------------------ */
 
 /* Human-readable name of a status code (static string). */
@@ -359,8 +489,8 @@ const char* csahca_status_string(int status);
 int csahca_abi_version(void);
 
 /* sizeof() of the argument structs, for bindings to check their mirrors:
- * which = 0 compress, 1 indexer, 2 prefill, 3 decode, 4 decode_compress;
- * -1 for an unknown id. */
+ * which = 0 compress, 1 indexer, 2 prefill, 3 decode, 4 decode_compress,
+ * 5 cp_topk_merge, 6 cp_attn_merge; -1 for an unknown id. */
 int64_t csahca_struct_size(int which);
 
 /* Device-side error word of the current device: every bounded wait in the

@@ -150,8 +150,12 @@ def decode_args(kind, q, pos, kv_cache, win, sinks, *, m, rope_dims, k=0, qI=Non
     if qI is not None:
         _, HI, dI = qI.shape
         qI_dt, kI_dt = _dt(qI), _dt(kI)
+    # a uint8 cache holds FP8 KV rows (include/csahca.h: e4m3 non-RoPE dims with
+    # one fp32 scale per 64, bf16 RoPE dims)
+    kv_dt = N.E4M3 if kv_cache.dtype == torch.uint8 else _dt(q)
     args = N.DecodeArgs(kind=N.CSA if kind == "csa" else N.HCA, dtype=_dt(q), B=B, H=H, d=d,
                         N_cap=kv_cache.shape[1], m=m, w=win.shape[1] if win is not None else 0,
+                        kv_dtype=kv_dt,
                         rope_dims=rope_dims, rope_base=rope_base, eps=eps, scale=scale,
                         q_norm=int(bool(q_norm)), k=k, HI=HI, dI=dI, qI_dtype=qI_dt,
                         kI_dtype=kI_dt, q=_ptr(q), pos=_ptr(pos), q_gain=_ptr(f(q_gain)),
@@ -215,6 +219,7 @@ def decode_compress_args(kind, pos, streams, ring, kv_cache, *, m, bias_a, bias_
         kind=N.CSA if csa else N.HCA, dtype=_dt(a), B=B, d=d, m=m, N_cap=kv_cache.shape[1],
         w=win.shape[1] if win is not None else 0, rope_dims=rope_dims, rope_base=rope_base, eps=eps,
         kv_norm=int(bool(kv_norm)), dI=dI, kI_dtype=_dt(kI) if dI else 0,
+        kv_dtype=N.E4M3 if kv_cache.dtype == torch.uint8 else _dt(a),
         pos=_ptr(pos), kv_raw=_ptr(kv_raw), a=_ptr(a), b=_ptr(b), za=_ptr(za), zb=_ptr(zb),
         bias_a=_ptr(f(bias_a)), bias_b=_ptr(f(bias_b)), kv_gain=_ptr(f(kv_gain)), ring=_ptr(ring),
         kv_cache=_ptr(kv_cache), win=_ptr(win), ia=_ptr(ia), ib=_ptr(ib), iza=_ptr(iza), izb=_ptr(izb),

@@ -21,9 +21,10 @@
 // load key tiles (cp.async gathers of selected rows, 2D TMA tiles of
 // contiguous rows); warp 10 issues the S MMAs and owns TMEM, warp 11 the P.V
 // MMAs.  Key tiles arrive in 8 chunks of
-// 64 dims with their own barriers; chunk pair (2j, 2j+1) is released as soon
-// as the P.V of O^T M-tile j has read it, so the next tile's loads overlap
-// the tail of the current one.
+// 64 dims with their own barriers, so the score MMAs of a chunk start as soon
+// as it lands; the whole tile is released by the one commit that ends its
+// P.V (a tcgen05.commit costs the tensor pipe a few hundred cycles, so each
+// MMA issuer commits once per tile).
 //
 // Work items: prefill = one query (all its tiles, final output); decode = one
 // query x a range of its tiles (partial max / sum / O for the combine).
@@ -61,15 +62,22 @@ struct AttnTcParams {
   __nv_bfloat16* out;           // final [B, nq, H, D]
   float* partial;               // [B, nq, H, splits, D + 4]
   double theta[64];             // base^(-2j/r) per rope pair j (r <= 128), filled on the host
+  // FP8 KV rows (decode): codes of the non-RoPE dims, RoPE dims bf16, one fp32
+  // scale per 64 dims (the header's layout), kv_row_bytes per row
+  const uint8_t* kv_f8;
+  int64_t kv_row_bytes;
+  int f8_nope_chunks;           // (D - rope_dims) / 64 chunks of e4m3 codes
+  // context parallelism (decode): the cache holds global entries entry_base ..
+  // entry_base + N - 1; skip_window leaves the window to another rank
+  int entry_base;
+  int skip_window;
 };
 
 struct AttnItem { int b, qi, t, tile0, tile1, split, ncomp_tiles, nwin_tiles; };
 struct AttnTile { int src; int row0; int lo, hi; int list_off; };   // src 0 gather, 1 comp rows, 2 window rows
 
 __device__ __forceinline__ int attn_visible(const AttnTcParams& p, int t) {
-  if (t < 0) return 0;
-  const int64_t v = ((int64_t)t + 1) / p.m;
-  return (int)(v < p.N ? v : p.N);
+  return visible_count(t, p.m, p.N, p.entry_base);
 }
 
 template <bool kDecode>
@@ -86,7 +94,7 @@ __device__ __forceinline__ AttnItem attn_item(const AttnTcParams& p, int id) {
   it.qi = qid % p.nq;
   it.t = kDecode ? p.pos[it.b] : it.qi;
   it.ncomp_tiles = p.csa ? (p.k + p.gtile - 1) / p.gtile : (attn_visible(p, it.t) + 127) / 128;
-  it.nwin_tiles = (p.w + 127) / 128;
+  it.nwin_tiles = p.skip_window ? 0 : (p.w + 127) / 128;
   const int total = it.ncomp_tiles + it.nwin_tiles;
   if (kDecode) {
     it.tile0 = it.split * p.tiles_per_split;
@@ -209,45 +217,71 @@ struct AttnSmem {
   static constexpr int K_BYTES = kAttnChunks * K_CHUNK;      // 128 KB
   static constexpr int P_BYTES = 128 * 128;                  // 16 KB
   static constexpr int TOTAL = 1024 + Q_BYTES + K_BYTES + P_BYTES;
+  static constexpr int F8_SCALES = 128 * 32;                 // FP8 rows: 8 scale slots per key row
 };
 
-// Decode partial of one (query, split): m[H], l[H] and up[H] fp32, then
-// O / (l up) fp16 [D][H].  up is a power of two, 1 unless the head's largest
-// |O / l| exceeds kPartialMaxAbs: the bf16 value rows behind O / l may be far
-// beyond fp16's range, and scaling them down by an exact power of two keeps
-// the stored partial finite without rounding it any further.
-constexpr int kTcHdrFloats = 3 * kAttnH;
+// Decode partial of one (query, split): m[H], l[H] fp32, then O / l bf16 [D][H].
+// O / l is a convex combination of bf16 value rows, so bf16 (fp32's exponent
+// range) holds it whatever the rows' magnitude; the combine's output is
+// rounded to bf16 as well, so the partial adds one rounding of the same size.
+constexpr int kTcHdrFloats = 2 * kAttnH;
 constexpr int kTcPartialHeader = kTcHdrFloats * 4;
-constexpr float kPartialMaxAbs = 16384.f;
 constexpr int kTcPartialBytes = kTcPartialHeader + kAttnD * kAttnH * 2;
-// The same blocks seen as 128-byte rows (64 fp16), as the TMA store writes them.
+// The same blocks seen as 128-byte rows (64 bf16), as the TMA store writes them.
 constexpr int kTcPartialRows = kTcPartialBytes / 128;
 constexpr int kTcPartialHeaderRows = kTcPartialHeader / 128;
 static_assert(kTcPartialBytes % 128 == 0 && kTcPartialHeader % 128 == 0, "partial blocks are whole 128-byte rows");
 
-__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
-  const __half2 h = __floats2half2_rn(a, b);
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <bool kDecode>
+// 16 e4m3 codes (codes[i] in byte i) times the block scale -> 16 bf16 at
+// dims 16q .. 16q+15 of row `row` of a 64-dim SW128 chunk.
+__device__ __forceinline__ void f8_piece_to_bf16(uint8_t* chunk, int row, int q, uint4 codes, float scale) {
+  const uint16_t* h = reinterpret_cast<const uint16_t*>(&codes);
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 f = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(h[i]),
+                                                                      __NV_E4M3)));
+    w[i] = pack_bf16x2(f.x * scale, f.y * scale);
+  }
+  *reinterpret_cast<uint4*>(chunk + sw128_offset(row, 32 * q)) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(chunk + sw128_offset(row, 32 * q + 16)) = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+// kF8 (decode only): the compressed rows are FP8 KV rows.  The producers
+// bring each 64-dim chunk's e4m3 codes (64 bytes per row) into the upper half
+// of the chunk's slot, the RoPE chunks (bf16) straight into their slots, and
+// the rows' block scales into a staging area; the softmax warps, idle until
+// the tile's scores, convert the codes in place to the bf16 SW128 rows the
+// MMAs read (every code is read into registers before any row is written).
+// comp_rows then maps the rows' bytes with a 64 x 128 box; f8_rope (128 x 128,
+// 128-byte swizzle) and f8_scale (32 x 128) map the same bytes.
+template <bool kDecode, bool kF8 = false>
 __global__ void __launch_bounds__(attn_threads<kDecode>(), 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_constant__ CUtensorMap win_rows,
                const __grid_constant__ CUtensorMap q_rows, const __grid_constant__ CUtensorMap part_rows,
+               const __grid_constant__ CUtensorMap f8_rope, const __grid_constant__ CUtensorMap f8_scale,
                const __grid_constant__ AttnTcParams p) {
+  static_assert(kDecode || !kF8, "FP8 KV rows are a decode cache format");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
   uint8_t* sK = sQ + AttnSmem::Q_BYTES;
   uint8_t* sP = sK + AttnSmem::K_BYTES;
-  __shared__ uint64_t bar_kfull[kAttnChunks], bar_kempty[kAttnChunks];
-  __shared__ uint64_t bar_q_raw, bar_q_empty, bar_q_full, bar_s_full, bar_s_empty, bar_p_full, bar_pv_done,
-      bar_done;
+  float* sScale = reinterpret_cast<float*>(sP + AttnSmem::P_BYTES);   // kF8: [128 rows][8]
+  __shared__ uint64_t bar_kfull[kAttnChunks];
+  __shared__ uint64_t bar_raw[kF8 ? kAttnChunks : 1], bar_raw_s;    // kF8: codes / scales landed
+  // bar_pv: the tile's P.V MMAs have completed (its key buffer is free, O^T
+  // and P^T may be touched again)
+  __shared__ uint64_t bar_q_raw, bar_q_empty, bar_q_full, bar_s_full, bar_s_empty, bar_p_full, bar_pv, bar_done;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
   __shared__ float red[2][4 * 32];
   __shared__ __align__(16) float stat_a[kAttnH];
-  __shared__ __align__(16) float stat_b[kAttnH];
   __shared__ __align__(16) float m_use[kAttnH];
   __shared__ __align__(16) float sc_h[kAttnH];     // softmax scale of head h (log2 units, times inv_rms_h)
   __shared__ __align__(16) float alpha[kAttnH];
@@ -263,14 +297,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
   constexpr int kWarpS = 8 + kNP, kWarpPV = 9 + kNP;
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    for (int c = 0; c < kAttnChunks; ++c) { mbar_init(&bar_kfull[c], kNP == 2 ? 32 : 32 * kNP); mbar_init(&bar_kempty[c], 1); }
+    // a chunk is full once its producer warp has arrived (TMA bytes or
+    // cp.async completions) and, for FP8 rows, the 256 softmax threads that
+    // convert it (they arrive on every chunk of every tile)
+    for (int c = 0; c < kAttnChunks; ++c) mbar_init(&bar_kfull[c], kF8 ? 32 + 256 : (kNP == 2 ? 32 : 32 * kNP));
+    if constexpr (kF8) {
+      for (int c = 0; c < kAttnChunks; ++c) mbar_init(&bar_raw[c], 32);
+      mbar_init(&bar_raw_s, 32);
+    }
     mbar_init(&bar_q_raw, 1);
     mbar_init(&bar_q_empty, 1);
     mbar_init(&bar_q_full, 256);
     mbar_init(&bar_s_full, 1);
     mbar_init(&bar_s_empty, 256);
     mbar_init(&bar_p_full, 256);
-    mbar_init(&bar_pv_done, 1);
+    mbar_init(&bar_pv, 1);
     mbar_init(&bar_done, 2);                       // both MMA issuers
     mbar_fence_init();
   }
@@ -317,6 +358,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     tma_prefetch_desc(&comp_rows);
     tma_prefetch_desc(&win_rows);
     tma_prefetch_desc(&q_rows);
+    if constexpr (kF8) {
+      tma_prefetch_desc(&f8_rope);
+      tma_prefetch_desc(&f8_scale);
+    }
     uint32_t tcount = 0, icount = 0;
     bool stop = false;                       // warp-uniform
     for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
@@ -355,16 +400,84 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
           }
           __syncwarp();
         }
+        if constexpr (kF8) {
+          // FP8 rows: the tile's block scales (32 bytes per row) by warp 8
+          if (T.src != 2 && pw == 0) {
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait(&bar_pv, ph ^ 1, &abort_flag);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) { stop = true; break; }
+            const int sofs = kAttnD + p.rope_dims;
+            if (T.src == 0) {
+              const int piece = lane & 1, rg = lane >> 1;       // 16 rows per instruction
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int r = 16 * j + rg;
+                cp_async16(reinterpret_cast<uint8_t*>(sScale) + r * 32 + piece * 16,
+                           p.kv_f8 + (int64_t)rows_s[pw][r] * p.kv_row_bytes + sofs + piece * 16);
+              }
+              cp_async_arrive_noinc(&bar_raw_s);
+            } else if (lane == 0) {
+              mbar_expect_tx(&bar_raw_s, AttnSmem::F8_SCALES);
+              tma_load_2d(sScale, &f8_scale, sofs, T.row0, &bar_raw_s);
+            } else {
+              mbar_arrive(&bar_raw_s);
+            }
+          }
+        }
         // two producers (decode): warp pw owns chunks {0,1,4,5} or {2,3,6,7};
         // more (prefill): every producer takes a share of every chunk
         constexpr int kChunksPerWarp = kNP == 2 ? kAttnChunks / 2 : kAttnChunks;
         for (int cc = 0; cc < kChunksPerWarp; ++cc) {
           const int c = kNP == 2 ? 4 * (cc >> 1) + 2 * pw + (cc & 1) : cc;
           int ok = 1;
-          if (lane == 0) ok = mbar_wait(&bar_kempty[c], ph ^ 1, &abort_flag);
+          if (lane == 0) ok = mbar_wait(&bar_pv, ph ^ 1, &abort_flag);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) { stop = true; break; }
           uint8_t* dst = sK + c * AttnSmem::K_CHUNK;
+          if constexpr (kF8) {
+            if (T.src != 2) {
+              if (c < p.f8_nope_chunks) {
+                // e4m3 codes of chunk c, 64 bytes per row, into the slot's upper half
+                uint8_t* raw = dst + AttnSmem::K_CHUNK / 2;
+                if (T.src == 0) {
+                  const int piece = lane & 3, rg = lane >> 2;   // 8 rows per instruction
+                  const uint8_t* src = p.kv_f8 + c * 64 + piece * 16;
+#pragma unroll 8
+                  for (int j = 0; j < 16; ++j) {
+                    const int r = 8 * j + rg;
+                    cp_async16(raw + r * 64 + piece * 16, src + (int64_t)rows_s[pw][r] * p.kv_row_bytes);
+                  }
+                  cp_async_arrive_noinc(&bar_raw[c]);
+                } else if (lane == 0) {
+                  mbar_expect_tx(&bar_raw[c], AttnSmem::K_CHUNK / 2);
+                  tma_load_2d(raw, &comp_rows, c * 64, T.row0, &bar_raw[c]);
+                } else {
+                  mbar_arrive(&bar_raw[c]);
+                }
+                mbar_arrive(&bar_kfull[c]);          // the bf16 rows come from the softmax warps
+              } else {
+                // a RoPE chunk: bf16 bytes at (D - r) + 128 (c - nope) of each row
+                const int rofs = (kAttnD - p.rope_dims) + 128 * (c - p.f8_nope_chunks);
+                if (T.src == 0) {
+                  const int piece = lane & 7, rg = lane >> 3;
+                  const uint8_t* src = p.kv_f8 + rofs + piece * 16;
+#pragma unroll 8
+                  for (int j = 0; j < 32; ++j) {
+                    const int r = 4 * j + rg;
+                    cp_async16(dst + sw128_offset(r, piece * 16), src + (int64_t)rows_s[pw][r] * p.kv_row_bytes);
+                  }
+                  cp_async_arrive_noinc(&bar_kfull[c]);
+                } else if (lane == 0) {
+                  mbar_expect_tx(&bar_kfull[c], AttnSmem::K_CHUNK);
+                  tma_load_2d(dst, &f8_rope, rofs, T.row0, &bar_kfull[c]);
+                } else {
+                  mbar_arrive(&bar_kfull[c]);
+                }
+              }
+              continue;
+            }
+          }
           if (T.src == 0) {
             // gathered rows: 8 lanes per 128-byte row segment (coalesced,
             // conflict-free), 4 rows per instruction, gtile / 4 instructions
@@ -412,15 +525,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
             const int* L = p.idx + ((int64_t)it.b * p.nq + it.qi) * p.k + Tn.list_off;
             for (int j = lane >> 3; j < Tn.hi; j += 4) {
               const int v = __ldg(L + j);
-              if (v >= 0 && v < p.N)
-                prefetch_l2_line(p.kv_comp_ptr + ((int64_t)it.b * p.N + v) * kAttnD + (lane & 7) * 64);
+              if (v >= 0 && v < p.N) {
+                if constexpr (kF8) {
+                  if ((lane & 7) * 128 < p.kv_row_bytes)
+                    prefetch_l2_line(p.kv_f8 + ((int64_t)it.b * p.N + v) * p.kv_row_bytes + (lane & 7) * 128);
+                } else {
+                  prefetch_l2_line(p.kv_comp_ptr + ((int64_t)it.b * p.N + v) * kAttnD + (lane & 7) * 64);
+                }
+              }
             }
           } else if (lane == 0 && Tn.row0 >= 0) {
             const int64_t total = Tn.src == 1 ? p.comp_rows_total : p.win_rows_total;
             const int64_t rows = min((int64_t)128, total - Tn.row0);
-            if (rows > 0)
-              bulk_prefetch_l2((Tn.src == 1 ? p.kv_comp_ptr : p.win_ptr) + (int64_t)Tn.row0 * kAttnD,
-                               (uint32_t)(rows * kAttnD * 2));
+            if (rows > 0) {
+              if (kF8 && Tn.src == 1)
+                bulk_prefetch_l2(p.kv_f8 + Tn.row0 * p.kv_row_bytes, (uint32_t)(rows * p.kv_row_bytes));
+              else
+                bulk_prefetch_l2((Tn.src == 1 ? p.kv_comp_ptr : p.win_ptr) + (int64_t)Tn.row0 * kAttnD,
+                                 (uint32_t)(rows * kAttnD * 2));
+            }
           }
         }
       }
@@ -484,17 +607,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
           // key steps past the tile's last valid row hold P = 0 and are skipped
           const int hi = attn_tile<kDecode>(p, it, tile).hi;
           const int nks = hi <= 16 ? 1 : min(8, (hi + 15) >> 4);
-          // M-tile by M-tile, so that chunk pair (2 mt, 2 mt + 1) is released
-          // for the next tile's loads as soon as its MMAs complete
+          if (nks == 8) {
 #pragma unroll
-          for (int mt = 0; mt < kAttnMT; ++mt) {
-            const uint64_t vd = vdesc + (uint64_t)((2 * mt) * (AttnSmem::K_CHUNK >> 4));
-            for (int ks = 0; ks < nks; ++ks)
-              umma_bf16(tO + mt * kAttnH, vd + 128 * ks, pdesc + 128 * ks, idesc_pv, !(first && ks == 0));
-            umma_commit(&bar_kempty[2 * mt]);
-            umma_commit(&bar_kempty[2 * mt + 1]);
+            for (int mt = 0; mt < kAttnMT; ++mt) {
+              const uint64_t vd = vdesc + (uint64_t)((2 * mt) * (AttnSmem::K_CHUNK >> 4));
+#pragma unroll
+              for (int ks = 0; ks < 8; ++ks)
+                umma_bf16(tO + mt * kAttnH, vd + 128 * ks, pdesc + 128 * ks, idesc_pv, !(first && ks == 0));
+            }
+          } else {
+#pragma unroll
+            for (int mt = 0; mt < kAttnMT; ++mt) {
+              const uint64_t vd = vdesc + (uint64_t)((2 * mt) * (AttnSmem::K_CHUNK >> 4));
+              for (int ks = 0; ks < nks; ++ks)
+                umma_bf16(tO + mt * kAttnH, vd + 128 * ks, pdesc + 128 * ks, idesc_pv, !(first && ks == 0));
+            }
           }
-          umma_commit(&bar_pv_done);
+          umma_commit(&bar_pv);
         }
       }
       umma_commit(&bar_done);
@@ -512,7 +641,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     const int st = threadIdx.x;              // 0..255 over both groups
     const int h0 = 32 * g;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    uint32_t tcount = 0, qcount = 0;
+    uint32_t tcount = 0, qcount = 0, f8count = 0;
     const int r0 = kAttnD - p.rope_dims;
     // q gain (same for every head and query) staged once in shared memory;
     // an all-ones gain (or none) leaves the non-rope dims of q untouched
@@ -632,6 +761,36 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       const float4* sc4 = reinterpret_cast<const float4*>(sc_h + h0);
       const float4* mu4 = reinterpret_cast<const float4*>(m_use + h0);
       for (int tile = it.tile0; tile < it.tile1; ++tile, ++tcount) {
+        if constexpr (kF8) {
+          // FP8 rows: both groups convert the tile's e4m3 chunks to bf16 in
+          // place (a give-up seen by either group ends it for both), and
+          // arrive on every chunk of every tile
+          const AttnTile Tc = attn_tile<kDecode>(p, it, tile);
+          const bool f8 = Tc.src != 2;
+          bool cbad = softmax_any256(bad);
+          if (!cbad && f8) cbad = !softmax_all256(mbar_wait(&bar_raw_s, f8count & 1, &abort_flag));
+          for (int c = 0; c < kAttnChunks; ++c) {
+            if (!cbad && f8 && c < p.f8_nope_chunks) {
+              cbad = !softmax_all256(mbar_wait(&bar_raw[c], f8count & 1, &abort_flag));
+              if (!cbad) {
+                uint8_t* slot = sK + c * AttnSmem::K_CHUNK;
+                const uint8_t* raw = slot + AttnSmem::K_CHUNK / 2;
+                // piece pc = 16 codes: row pc / 4, quarter pc % 4 (raw + 64 row + 16 quarter)
+                const int pc0 = st, pc1 = st + 256;
+                const uint4 in0 = *reinterpret_cast<const uint4*>(raw + pc0 * 16);
+                const uint4 in1 = *reinterpret_cast<const uint4*>(raw + pc1 * 16);
+                const float s0 = sScale[(pc0 >> 2) * 8 + c], s1 = sScale[(pc1 >> 2) * 8 + c];
+                softmax_sync256();                   // every code read before any row is written
+                f8_piece_to_bf16(slot, pc0 >> 2, pc0 & 3, in0, s0);
+                f8_piece_to_bf16(slot, pc1 >> 2, pc1 & 3, in1, s1);
+                fence_proxy_async_smem();
+              }
+            }
+            mbar_arrive(&bar_kfull[c]);
+          }
+          if (f8) ++f8count;
+          bad = bad || cbad;
+        }
         if (bad) continue;
         const uint32_t ph = tcount & 1;
         const bool first = tile == it.tile0;
@@ -694,7 +853,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
         // the previous tile's P.V has finished: P^T may be overwritten and
         // O^T / the partial sums rescaled
         if (!first) {
-          if (!mbar_wait_group(gid, &bar_pv_done, ph ^ 1, &abort_flag)) { bad = true; continue; }
+          if (!mbar_wait_group(gid, &bar_pv, ph ^ 1, &abort_flag)) { bad = true; continue; }
           tc_fence_after();
         }
         if (rescale) {
@@ -749,7 +908,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       }
       // ---- epilogue: wait for the last P.V, reduce the sums, write out
       if (!empty && !bad) {
-        if (!mbar_wait_group(gid, &bar_pv_done, (tcount - 1) & 1, &abort_flag)) bad = true;
+        if (!mbar_wait_group(gid, &bar_pv, (tcount - 1) & 1, &abort_flag)) bad = true;
         else tc_fence_after();
       }
       if (!empty && !bad) {
@@ -761,10 +920,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       bad = softmax_any256(bad);             // the output stage is entered by both groups or neither
       if (!bad) {
         if (kDecode) {
-          // partial block of (query, split): m[H] (log2 units), l[H] and
-          // up[H] in fp32, then O / (l up) as fp16 [D][H] (a thread writes its
-          // dim's 32 heads, 64 contiguous bytes, straight from TMEM); an empty
-          // split writes only its header, m = -inf, which the combine skips
+          // partial block of (query, split): m[H] (log2 units) and l[H] in
+          // fp32, then O / l as bf16 [D][H] (a thread writes its dim's 32
+          // heads, 64 contiguous bytes, straight from TMEM); an empty split
+          // writes only its header, m = -inf, which the combine skips
           char* P = reinterpret_cast<char*>(p.partial) +
                     (((int64_t)it.b * p.nq + it.qi) * p.splits + it.split) * kTcPartialBytes;
           float* hdr = reinterpret_cast<float*>(P);
@@ -773,41 +932,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
             const float l = empty ? 0.f : l_run[h];
             hdr[h] = empty ? -INFINITY : m_use[h];
             hdr[kAttnH + h] = l;
-            hdr[2 * kAttnH + h] = 1.f;
             stat_a[h] = l > 0.f ? 1.f / l : 0.f;
           }
           group_sync(gid);
           if (!empty) {
-            // per-head largest |O| over the 512 dims (this thread's dim of each
-            // M-tile, then over the group's 128 threads), and from it the
-            // power of two `up` that keeps |O / (l up)| <= kPartialMaxAbs
-            {
-              float amax[32];
-#pragma unroll
-              for (int e = 0; e < 32; ++e) amax[e] = 0.f;
-#pragma unroll 1
-              for (int mt = 0; mt < kAttnMT; ++mt) {
-                float o[32];
-                tmem_ld32(tO + lane_base + mt * kAttnH + h0, o);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) amax[e] = fmaxf(amax[e], fabsf(o[e]));
-              }
-              reduce_group32<true>(amax, red[g], stat_b + h0, gid);
-            }
-            if (tid < 32) {
-              const int h = h0 + tid;
-              const float mx = stat_b[h] * stat_a[h];
-              if (mx > kPartialMaxAbs) {
-                int e2 = 0;
-                frexpf(mx / kPartialMaxAbs, &e2);          // mx / kPartialMaxAbs < 2^e2
-                const float up = ldexpf(1.f, e2);
-                hdr[2 * kAttnH + h] = up;
-                stat_a[h] = stat_a[h] / up;                // exact: up is a power of two
-              }
-            }
-            group_sync(gid);
-            // O / l of M-tile mt: 128 dims x 64 heads fp16 = 128-byte rows,
+            // O / l of M-tile mt: 128 dims x 64 heads bf16 = 128-byte rows,
             // staged in P's buffer with the 128-byte swizzle (group g writes
             // pieces 4g..4g+3 of row tid) and stored by one TMA box
             const float4* f4 = reinterpret_cast<const float4*>(stat_a + h0);
@@ -830,10 +959,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 uint4 w;
-                w.x = pack_half2(o[8 * q + 0], o[8 * q + 1]);
-                w.y = pack_half2(o[8 * q + 2], o[8 * q + 3]);
-                w.z = pack_half2(o[8 * q + 4], o[8 * q + 5]);
-                w.w = pack_half2(o[8 * q + 6], o[8 * q + 7]);
+                w.x = pack_bf16x2(o[8 * q + 0], o[8 * q + 1]);
+                w.y = pack_bf16x2(o[8 * q + 2], o[8 * q + 3]);
+                w.z = pack_bf16x2(o[8 * q + 4], o[8 * q + 5]);
+                w.w = pack_bf16x2(o[8 * q + 6], o[8 * q + 7]);
                 *reinterpret_cast<uint4*>(stg + sw128_offset(tid, (4 * g + q) * 16)) = w;
               }
               fence_proxy_async_smem();
@@ -914,10 +1043,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
 
 // ---------------------------------------------------------------------------
 // Split-KV combine of the tensor-core decode partials, with the sink and the
-// output de-rotation: o = sum_s f_s up_s (O_s / (l_s up_s)), f_s = l_s 2^(m_s - M) / den,
+// output de-rotation: o = sum_s f_s (O_s / l_s), f_s = l_s 2^(m_s - M) / den,
 // den = 2^(z_h log2 e - M) + sum_s l_s 2^(m_s - M), M the largest of them; the
 // rope dims of o are then rotated by -t.  One CTA per (query, 16 dims).  The
-// m, l headers of every split and the 16-dim slices (16 x 64 fp16 per split)
+// m, l headers of every split and the 16-dim slices (16 x 64 bf16 per split)
 // reach shared memory by two TMA boxes, so the kernel pays about one memory
 // latency, not one per split.  With more splits than slice slots the slices
 // go in rounds.
@@ -932,6 +1061,9 @@ struct TcCombineParams {
   const float* sinks;         // [H]
   const int* pos;             // [B] query positions (decode)
   __nv_bfloat16* out;         // [B * nq, H, D]
+  // context parallelism: instead of out, the rows' unnormalised shares
+  // [rows][mx[H], l[H], o[H][D]] f32, without the sink and not de-rotated
+  float* partial_out;
   int rows, splits, rope_dims;
   double theta[64];           // base^(-2j/r) per rope pair j (r <= 128), from the host
 };
@@ -942,8 +1074,8 @@ __host__ __device__ inline int tc_combine_smem_bytes(int splits) {
   return splits * kTcPartialHeader + slots * kTcCombineSlice;
 }
 
-// hdr_map: the partials as [blocks][518 rows][64 fp16], box [splits][6][64]
-// (the m, l, up headers of all splits of one query); slc_map: the same tensor,
+// hdr_map: the partials as [blocks][516 rows][64 bf16], box [splits][4][64]
+// (the m, l headers of all splits of one query); slc_map: the same tensor,
 // box [min(splits, 64)][16][64] (16 dims of up to 64 splits).  A bulk copy per
 // split was measured to complete one copy at a time; a box covering every
 // split goes out as one transfer.
@@ -958,8 +1090,8 @@ __global__ void __launch_bounds__(kTcCombineThreads) attn_combine_tc_kernel(
   __shared__ __align__(16) __nv_bfloat16 ostage[kAttnH][kTcCombineDims];
   __shared__ volatile int abort_flag;
   constexpr int kChunks = kAttnD / kTcCombineDims;
-  float* hdr = reinterpret_cast<float*>(cmb_smem);              // [splits][m[H], l[H], up[H]]; m slots -> weights
-  uint8_t* slots = cmb_smem + p.splits * kTcPartialHeader;        // [slots][16 dims][H] fp16
+  float* hdr = reinterpret_cast<float*>(cmb_smem);              // [splits][m[H], l[H]]; m slots -> weights
+  uint8_t* slots = cmb_smem + p.splits * kTcPartialHeader;        // [slots][16 dims][H] bf16
   const int nslots = p.splits < kTcCombineSlots ? p.splits : kTcCombineSlots;
   const int row = blockIdx.x / kChunks, dc = blockIdx.x % kChunks;
   const int blk0 = row * p.splits, srow = kTcPartialHeaderRows + dc * kTcCombineDims;
@@ -986,7 +1118,8 @@ __global__ void __launch_bounds__(kTcCombineThreads) attn_combine_tc_kernel(
   // split weights: thread (head h, part) takes the splits s = part mod 8
   const int h = tid & (kAttnH - 1), part = tid >> 6;
   bool ok = mbar_wait(&bar_hdr, 0, &abort_flag);
-  const float z2 = p.sinks[h] * kLog2e;
+  const bool share = p.partial_out != nullptr;
+  const float z2 = share ? -INFINITY : p.sinks[h] * kLog2e;
   float mx = -INFINITY;
   if (ok) {
 #pragma unroll 4
@@ -1003,17 +1136,22 @@ __global__ void __launch_bounds__(kTcCombineThreads) attn_combine_tc_kernel(
     for (int s = part; s < p.splits; s += 8) {
       const float ms = hdr[s * kTcHdrFloats + h];
       const float f = ms == -INFINITY ? 0.f : hdr[s * kTcHdrFloats + kAttnH + h] * exp2f(ms - M);
-      hdr[s * kTcHdrFloats + h] = f * hdr[s * kTcHdrFloats + 2 * kAttnH + h];   // weight of the stored slice
+      hdr[s * kTcHdrFloats + h] = f;
       den += f;
     }
   __syncthreads();                                 // every read of red[] (M) is done
   red[part][h] = den;
   __syncthreads();
   if (part == 0) {
-    float d = exp2f(z2 - M);
+    float d = share ? 0.f : exp2f(z2 - M);
 #pragma unroll
     for (int i = 0; i < 8; ++i) d += red[i][h];
-    inv_s[h] = 1.f / d;
+    inv_s[h] = share ? (d > 0.f ? 1.f / d : 0.f) : 1.f / d;
+    if (share && dc == 0) {
+      float* hdr_out = p.partial_out + (int64_t)row * (2 * kAttnH + kAttnH * kAttnD);
+      hdr_out[h] = M;
+      hdr_out[kAttnH + h] = d;
+    }
   }
   // weighted sum over the splits: thread (quarter qt, dim dl, heads 8 hg ..)
   // takes the splits s = qt mod 4
@@ -1047,10 +1185,10 @@ __global__ void __launch_bounds__(kTcCombineThreads) attn_combine_tc_kernel(
         const bool live = (w0.x != 0.f) | (w0.y != 0.f) | (w0.z != 0.f) | (w0.w != 0.f) | (w1.x != 0.f) |
                           (w1.y != 0.f) | (w1.z != 0.f) | (w1.w != 0.f);
         raw.x = live ? raw.x : 0u; raw.y = live ? raw.y : 0u; raw.z = live ? raw.z : 0u; raw.w = live ? raw.w : 0u;
-        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-        const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&raw.z));
-        const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&raw.w));
+        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+        const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+        const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.z));
+        const float2 f3 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.w));
         acc[0] = fmaf(w0.x, f0.x, acc[0]); acc[1] = fmaf(w0.y, f0.y, acc[1]);
         acc[2] = fmaf(w0.z, f1.x, acc[2]); acc[3] = fmaf(w0.w, f1.y, acc[3]);
         acc[4] = fmaf(w1.x, f2.x, acc[4]); acc[5] = fmaf(w1.y, f2.y, acc[5]);
@@ -1070,23 +1208,32 @@ __global__ void __launch_bounds__(kTcCombineThreads) attn_combine_tc_kernel(
       for (int i = 0; i < 8; ++i) acc[i] += acc_s[j][lt][i];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] *= inv_s[hg * 8 + i];
-    // rope dims: the pair partner (dim ^ 1) is thread tid ^ 8
-    const int r0 = kAttnD - p.rope_dims;
-    float partner[8];
+    if (share) {
+      // this rank's share: o[h][dim] as fp32 (ok is the block's AND here); the
+      // merge adds the sink and de-rotates
+      float* o = p.partial_out + (int64_t)row * (2 * kAttnH + kAttnH * kAttnD) + 2 * kAttnH;
+      if (ok)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) partner[i] = __shfl_xor_sync(0xffffffffu, acc[i], 8);
-    if (dim >= r0) {
-      float cs, sn;
-      rope_sincos(-(double)p.pos[row], p.theta[(dim - r0) >> 1], &cs, &sn);
+        for (int i = 0; i < 8; ++i) o[(hg * 8 + i) * kAttnD + dim] = acc[i];
+    } else {
+      // rope dims: the pair partner (dim ^ 1) is thread tid ^ 8
+      const int r0 = kAttnD - p.rope_dims;
+      float partner[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        acc[i] = (dim & 1) ? fmaf(partner[i], sn, acc[i] * cs) : fmaf(-partner[i], sn, acc[i] * cs);
+      for (int i = 0; i < 8; ++i) partner[i] = __shfl_xor_sync(0xffffffffu, acc[i], 8);
+      if (dim >= r0) {
+        float cs, sn;
+        rope_sincos(-(double)p.pos[row], p.theta[(dim - r0) >> 1], &cs, &sn);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          acc[i] = (dim & 1) ? fmaf(partner[i], sn, acc[i] * cs) : fmaf(-partner[i], sn, acc[i] * cs);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ostage[hg * 8 + i][dl] = __float2bfloat16_rn(acc[i]);
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) ostage[hg * 8 + i][dl] = __float2bfloat16_rn(acc[i]);
   }
   __syncthreads();
-  if (!ok) return;
+  if (!ok || share) return;
   if (tid < 128) {
     const int hh = tid >> 1, piece = tid & 1;
     *reinterpret_cast<uint4*>(p.out + ((int64_t)row * kAttnH + hh) * kAttnD + dc * kTcCombineDims + piece * 8) =

@@ -23,6 +23,8 @@
 #include "indexer_tc.cuh"
 #include "indexer_f8.cuh"
 #include "attention_tc.cuh"
+#include "context_parallel.cuh"
+#include "attention_small_tc.cuh"
 
 using namespace csahca;
 
@@ -252,7 +254,8 @@ int validate_indexer(const csahca_indexer_args* a, bool shapes_only = false) {
   if (a->q_dtype != CSAHCA_F32 && a->q_dtype != CSAHCA_BF16) return CSAHCA_ERR_INVALID_ARG;
   if (a->k_dtype != CSAHCA_F32 && a->k_dtype != CSAHCA_BF16 && a->k_dtype != CSAHCA_E4M3)
     return CSAHCA_ERR_INVALID_ARG;
-  if (a->B < 0 || a->nq < 0 || a->HI < 1 || a->dI < 1 || a->N < 0 || a->m < 1 || a->k < 1)
+  if (a->B < 0 || a->nq < 0 || a->HI < 1 || a->dI < 1 || a->N < 0 || a->m < 1 || a->k < 1 ||
+      a->entry_base < 0)
     return CSAHCA_ERR_INVALID_ARG;
   if (a->dI % 8) return CSAHCA_ERR_UNSUPPORTED;
   if (a->k_dtype == CSAHCA_E4M3) {
@@ -266,7 +269,8 @@ int validate_indexer(const csahca_indexer_args* a, bool shapes_only = false) {
   if (!a->qI || !a->w || !a->q_pos || !a->idx) return CSAHCA_ERR_INVALID_ARG;
   if (a->N > 0 && !a->kI) return CSAHCA_ERR_INVALID_ARG;
   if (a->k_dtype == CSAHCA_E4M3 && a->N > 0 && !a->kI_scale) return CSAHCA_ERR_INVALID_ARG;
-  const void* ptrs[] = {a->qI, a->w, a->kI, a->kI_scale, a->q_pos, a->idx, a->scores_out, a->workspace};
+  const void* ptrs[] = {a->qI, a->w, a->kI, a->kI_scale, a->q_pos, a->idx, a->scores_out, a->sel_scores,
+                        a->workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return CSAHCA_ERR_ALIGNMENT;
   return CSAHCA_OK;
@@ -333,12 +337,13 @@ int launch_zero(char* ptr, size_t bytes, cudaStream_t s) {
 // zeroed the scratch and built the row histograms (pass 1) while scoring.
 int launch_topk(const csahca_indexer_args* a, const float* scores, int64_t stride, const int* q_pos, int* idx,
                 int rows, char* scratch, cudaStream_t s, bool hist_ready = false,
-                const void* prefetch_base = nullptr, int64_t prefetch_row_bytes = 0, bool sorted = true) {
+                const void* prefetch_base = nullptr, int64_t prefetch_row_bytes = 0, bool sorted = true,
+                bool routed = false) {
   if (!topk_uses_large(a)) {
     TopkParams tp;
     tp.scores = scores; tp.row_stride = stride; tp.q_pos = q_pos; tp.idx = idx;
     tp.B = 1; tp.nq = rows; tp.N = a->N; tp.m = a->m; tp.k = a->k;
-    tp.q_begin = 0; tp.q_count = rows;
+    tp.q_begin = 0; tp.q_count = rows; tp.entry_base = a->entry_base;
     const int smem = topk_rows_smem_bytes(a->N > 0 ? a->N : 1);
     cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     CSAHCA_TRACE("topk_rows", s);
@@ -350,7 +355,7 @@ int launch_topk(const csahca_indexer_args* a, const float* scores, int64_t strid
   const TopkLargeLayout L = topk_large_layout(rows, a->N, a->k);
   TopkLargeParams tp;
   tp.scores = scores; tp.row_stride = stride; tp.q_pos = q_pos; tp.idx = idx;
-  tp.rows = rows; tp.N = a->N; tp.m = a->m; tp.k = a->k;
+  tp.rows = rows; tp.N = a->N; tp.m = a->m; tp.k = a->k; tp.entry_base = a->entry_base;
   int slices = (int)ceil_div64(2 * num_sms(), rows);
   const int max_slices = (int)ceil_div64(a->N, 2048);
   if (slices > max_slices) slices = max_slices;
@@ -364,6 +369,17 @@ int launch_topk(const csahca_indexer_args* a, const float* scores, int64_t strid
   tp.sorted = sorted ? 1 : 0;
   tp.prefetch_base = static_cast<const char*>(prefetch_base);
   tp.prefetch_row_bytes = prefetch_row_bytes;
+  if (routed) {
+    // the indexer has routed every key into the taken / candidate lists
+    const int smem = topk_select_smem_bytes(a->N);
+    cudaFuncSetAttribute(topk_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    {
+      CSAHCA_TRACE("topk_finish", s);
+      launch_k(topk_finish_kernel, dim3(rows), dim3(kTopkSelectThreads), smem, s, tp);
+    }
+    CSAHCA_CHECK_LAUNCH();
+    return CSAHCA_OK;
+  }
   if (!hist_ready) {
     {
       const int st = launch_zero(scratch + L.hist, L.above - L.hist, s);
@@ -426,8 +442,29 @@ int launch_indexer_tc_t(const csahca_indexer_args* a, IdxTcParams p, cudaStream_
 }
 
 // Tensor-core scores for queries [q0, q0 + qc) into scores (row stride N).
+// Decode split of the FP8 scan: each sequence's key tiles over about one CTA per SM.
+void f8_decode_split(const csahca_indexer_args* a, int* tiles_per_split, int* splits) {
+  const int tiles = (int)ceil_div64(a->N, 128);
+  int sp = num_sms() / (a->B > 0 ? a->B : 1);
+  if (sp > tiles) sp = tiles;
+  if (sp < 1) sp = 1;
+  *tiles_per_split = (int)ceil_div64(tiles, sp);
+  *splits = (int)ceil_div64(tiles, *tiles_per_split);
+}
+
+// The FP8 decode scan can route the top-k in its epilogue when every work
+// item has a CTA of its own (a CTA waits for its row's other items) and the
+// item's scores fit in shared memory beside the key stages.
+constexpr int kRouteMaxTiles = 64;
+bool f8_route_ok(const csahca_indexer_args* a) {
+  int tps = 0, sp = 0;
+  f8_decode_split(a, &tps, &sp);
+  return a->B * sp <= num_sms() && tps <= kRouteMaxTiles;
+}
+
 int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* scores, int64_t stride,
-                      cudaStream_t s, uint32_t* hist = nullptr, uint32_t* counters = nullptr) {
+                      cudaStream_t s, uint32_t* hist = nullptr, uint32_t* counters = nullptr, int* above = nullptr,
+                      uint2* cand = nullptr) {
   IdxTcParams p;
   memset(&p, 0, sizeof(p));
   p.hist = hist;
@@ -436,34 +473,33 @@ int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* score
   p.k = a->k;
   p.w = a->w; p.kI_scale = a->kI_scale; p.q_pos = a->q_pos;
   p.scores = scores; p.score_row_stride = stride;
-  p.B = a->B; p.nq = a->nq; p.HI = a->HI; p.N = a->N; p.m = a->m;
+  p.B = a->B; p.nq = a->nq; p.HI = a->HI; p.N = a->N; p.m = a->m; p.entry_base = a->entry_base;
   p.q_begin = q0; p.q_count = qc;
   if (a->k_dtype == CSAHCA_E4M3) {
     // e4m3 keys straight into the FP8 tensor cores, one query per work item;
     // decode spreads each sequence's key tiles over about one CTA per SM
-    const int tiles = (int)ceil_div64(a->N, 128);
     if (qc == 1) {
-      int splits = num_sms() / (a->B > 0 ? a->B : 1);
-      if (splits > tiles) splits = tiles;
-      if (splits < 1) splits = 1;
-      p.tiles_per_split = (int)ceil_div64(tiles, splits);
-      p.splits = (int)ceil_div64(tiles, p.tiles_per_split);
+      f8_decode_split(a, &p.tiles_per_split, &p.splits);
       p.n_items = a->B * p.splits;
     } else {
       p.splits = 0;
       p.n_items = a->B * qc;
     }
     p.items_per_row = p.splits > 0 ? p.splits : 1;
+    p.route = above != nullptr ? 1 : 0;
+    p.above = above;
+    p.cand = cand;
     using Cfg = IdxF8Cfg<64>;
     CUtensorMap kmap;
     if (!encode_2d(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->kI, (uint64_t)a->dI, (uint64_t)a->B * a->N, 128, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B))
       return CSAHCA_ERR_LAUNCH;
-    cudaFuncSetAttribute(indexer_f8_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    const int smem = Cfg::SMEM + (p.route ? p.tiles_per_split * 128 * 4 : 0);
+    cudaFuncSetAttribute(indexer_f8_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
     if (grid <= 0) return CSAHCA_OK;
     CSAHCA_TRACE("indexer_scores_f8", s);
-    launch_k(indexer_f8_kernel<64>, dim3(grid), dim3(kIdxF8Threads), Cfg::SMEM, s, kmap, static_cast<const __nv_bfloat16*>(a->qI), p);
+    launch_k(indexer_f8_kernel<64>, dim3(grid), dim3(kIdxF8Threads), smem, s, kmap, static_cast<const __nv_bfloat16*>(a->qI), p);
     CSAHCA_CHECK_LAUNCH();
     return CSAHCA_OK;
   }
@@ -480,6 +516,18 @@ int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* score
   p.splits = 0;
   p.n_items = a->B * (int)ceil_div64(qc, 4);
   return launch_indexer_tc_t<4, false>(a, p, s);
+}
+
+// sel[r][j] = scores[r][idx[r][j]] for `rows` consecutive rows.
+int launch_select_scores(const float* scores, int64_t stride, const int* idx, float* sel, int rows, int k,
+                         cudaStream_t s) {
+  if (rows <= 0) return CSAHCA_OK;
+  {
+    CSAHCA_TRACE("select_scores", s);
+    launch_k(select_scores_kernel, dim3((unsigned)rows), dim3(256), 0, s, scores, stride, idx, sel, k);
+  }
+  CSAHCA_CHECK_LAUNCH();
+  return CSAHCA_OK;
 }
 
 // prefetch_base / prefetch_row_bytes (internal, decode only): every selected
@@ -499,7 +547,7 @@ int run_indexer(const csahca_indexer_args* a, void* stream, const void* prefetch
     IndexerParams p;
     p.qI = a->qI; p.w = a->w; p.kI = a->kI; p.kI_scale = a->kI_scale; p.q_pos = a->q_pos;
     p.B = a->B; p.nq = a->nq; p.HI = a->HI; p.dI = a->dI; p.N = a->N; p.m = a->m;
-    p.q_begin = q0; p.q_count = qc;
+    p.q_begin = q0; p.q_count = qc; p.entry_base = a->entry_base;
     // scores rows of this chunk: row (b, q) -> b * qc + (q - q0); with
     // scores_out the full [B, nq, N] layout is addressed through the stride.
     float* base;
@@ -535,6 +583,11 @@ int run_indexer(const csahca_indexer_args* a, void* stream, const void* prefetch
         int st3 = launch_topk(a, pb.scores, stride, pb.q_pos + q0, a->idx + ((int64_t)b * a->nq + q0) * a->k, qc,
                               static_cast<char*>(a->workspace), s);
         if (st3 != CSAHCA_OK) return st3;
+        if (a->sel_scores) {
+          const int64_t r0 = (int64_t)b * a->nq + q0;
+          st3 = launch_select_scores(pb.scores, stride, a->idx + r0 * a->k, a->sel_scores + r0 * a->k, qc, a->k, s);
+          if (st3 != CSAHCA_OK) return st3;
+        }
       }
       continue;
     }
@@ -548,15 +601,26 @@ int run_indexer(const csahca_indexer_args* a, void* stream, const void* prefetch
                            a->k_dtype == CSAHCA_E4M3 && a->N <= kTopkLargeMaxN;
     uint32_t* hist = nullptr;
     uint32_t* counters = nullptr;
+    int* above = nullptr;
+    uint2* cand = nullptr;
+    // decode with e4m3 keys and one CTA per work item: the indexer also
+    // routes the keys into the top-k lists from shared memory, and one CTA
+    // per row finishes
+    // (sel_scores reads the scores back: they must reach the workspace)
+    const bool route = fuse_hist && a->nq == 1 && f8_route_ok(a) && !a->sel_scores;
     if (fuse_hist) {
       const TopkLargeLayout L = topk_large_layout((int64_t)a->B * qc, a->N, a->k);
       const int zst = launch_zero(scratch + L.hist, L.above - L.hist, s);
       if (zst != CSAHCA_OK) return zst;
       hist = reinterpret_cast<uint32_t*>(scratch + L.hist);
       counters = reinterpret_cast<uint32_t*>(scratch + L.counters);
+      if (route) {
+        above = reinterpret_cast<int*>(scratch + L.above);
+        cand = reinterpret_cast<uint2*>(scratch + L.cand);
+      }
     }
     if (indexer_tc_eligible(a)) {
-      int st2 = launch_indexer_tc(a, q0, qc, base, stride, s, hist, counters);
+      int st2 = launch_indexer_tc(a, q0, qc, base, stride, s, hist, counters, above, cand);
       if (st2 != CSAHCA_OK) return st2;
     } else if (a->N > 0) {
       if (a->k_dtype == CSAHCA_E4M3) {
@@ -573,13 +637,23 @@ int run_indexer(const csahca_indexer_args* a, void* stream, const void* prefetch
     // addressed per batch entry, so launch per b unless the chunk is the whole nq
     if (qc == a->nq) {
       int st3 = launch_topk(a, base, stride, a->q_pos, a->idx, a->B * qc, scratch, s, fuse_hist,
-                            a->nq == 1 ? prefetch_base : nullptr, prefetch_row_bytes, sorted);
+                            a->nq == 1 ? prefetch_base : nullptr, prefetch_row_bytes, sorted, route);
       if (st3 != CSAHCA_OK) return st3;
+      if (a->sel_scores) {
+        st3 = launch_select_scores(base, stride, a->idx, a->sel_scores, a->B * qc, a->k, s);
+        if (st3 != CSAHCA_OK) return st3;
+      }
     } else {
       for (int b = 0; b < a->B; ++b) {
+        const int64_t r0 = (int64_t)b * a->nq + q0;
         int st3 = launch_topk(a, base + (int64_t)b * qc * stride, stride, a->q_pos + (int64_t)b * a->nq + q0,
-                              a->idx + ((int64_t)b * a->nq + q0) * a->k, qc, scratch, s);
+                              a->idx + r0 * a->k, qc, scratch, s);
         if (st3 != CSAHCA_OK) return st3;
+        if (a->sel_scores) {
+          st3 = launch_select_scores(base + (int64_t)b * qc * stride, stride, a->idx + r0 * a->k,
+                                     a->sel_scores + r0 * a->k, qc, a->k, s);
+          if (st3 != CSAHCA_OK) return st3;
+        }
       }
     }
   }
@@ -645,41 +719,110 @@ bool attn_tc_shape_ok(int dtype, int H, int d, int rope_dims, int64_t comp_rows,
          win_rows >= 128;
 }
 
+// FP8 KV rows (the header's layout): bytes per row, 0 for an invalid combination.
+int64_t kv_f8_row_bytes(int d, int r) {
+  if (d <= 0 || r < 0 || r > d || (d - r) % 64 || r % 64) return 0;
+  const int64_t raw = (int64_t)(d - r) + 2 * (int64_t)r + 4 * (int64_t)((d - r) / 64);
+  return (raw + 127) / 128 * 128;
+}
+
 int launch_attn_tc(const AttnTcParams& p_in, const void* kv_comp, int64_t comp_rows, const void* win,
-                   int64_t win_rows, cudaStream_t s, const char* name) {
+                   int64_t win_rows, cudaStream_t s, const char* name, bool f8 = false) {
   AttnTcParams p = p_in;
   rope_theta_table(p.theta, p.rope_dims, p.rope_base);
+  if (f8) {
+    p.kv_f8 = static_cast<const uint8_t*>(kv_comp);
+    p.kv_row_bytes = kv_f8_row_bytes(kAttnD, p.rope_dims);
+    p.f8_nope_chunks = (kAttnD - p.rope_dims) / 64;
+  }
   p.win_ptr = static_cast<const __nv_bfloat16*>(win ? win : kv_comp);
   p.comp_rows_total = comp_rows;
   p.win_rows_total = win ? win_rows : comp_rows;
   // rows of d = 512 bf16 seen as [chunk 8][row][64]: a key box is one chunk
   // of 128 rows (16 KB); the query box is all 8 chunks x 64 heads (64 KB),
   // landing chunk-major with the 128-byte swizzle as the MMA operand wants it
-  CUtensorMap m_rows, m_win, m_q;
+  CUtensorMap m_rows, m_win, m_q, m_rope, m_scale;
   const uint64_t rs = kAttnD * 2;
-  bool ok = encode_3d(&m_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv_comp, 64, (uint64_t)comp_rows, kAttnChunks, rs,
-                      128, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+  bool ok;
+  if (f8) {
+    // FP8 rows as bytes: 64-byte code boxes, the 128-byte RoPE chunks with the
+    // MMA's swizzle, 32-byte scale boxes (all 128 rows)
+    const uint64_t rb = (uint64_t)p.kv_row_bytes;
+    ok = encode_2d(&m_rows, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kv_comp, rb, (uint64_t)comp_rows, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) &&
+         encode_2d(&m_rope, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kv_comp, rb, (uint64_t)comp_rows, 128, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B) &&
+         encode_2d(&m_scale, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kv_comp, rb, (uint64_t)comp_rows, 32, 128,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+  } else {
+    ok = encode_3d(&m_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv_comp, 64, (uint64_t)comp_rows, kAttnChunks, rs,
+                   128, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+  }
   if (win) ok = ok && encode_3d(&m_win, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, win, 64, (uint64_t)win_rows, kAttnChunks,
                                 rs, 128, 64, 128, 1, CU_TENSOR_MAP_SWIZZLE_128B);
   else m_win = m_rows;
   ok = ok && encode_3d(&m_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.q, 64, (uint64_t)p.B * p.nq * kAttnH, kAttnChunks,
                        rs, 128, 64, kAttnH, kAttnChunks, CU_TENSOR_MAP_SWIZZLE_128B);
-  // decode partials as 128-byte fp16 rows, stored 128 rows (one O^T M-tile) per box
+  // decode partials as 128-byte bf16 rows, stored 128 rows (one O^T M-tile) per box
   CUtensorMap m_part = m_rows;
   if (p.decode)
-    ok = ok && encode_2d(&m_part, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.partial, kAttnH,
+    ok = ok && encode_2d(&m_part, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.partial, kAttnH,
                          (uint64_t)p.B * p.nq * p.splits * kTcPartialRows, kAttnH, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return CSAHCA_ERR_LAUNCH;
-  const int smem = AttnSmem::TOTAL;
+  if (!f8) m_rope = m_scale = m_rows;                  // not read
+  const int smem = AttnSmem::TOTAL + (f8 ? AttnSmem::F8_SCALES : 0);
   // decode and prefill are separate instances: each carries only its own
   // epilogue (a smaller kernel stalls less on instruction fetch)
-  auto kern = p.decode ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  auto kern = p.decode ? (f8 ? attn_tc_kernel<true, true> : attn_tc_kernel<true, false>) : attn_tc_kernel<false, false>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   if (grid <= 0) return CSAHCA_OK;
   CSAHCA_TRACE(name, s);
   launch_k(kern, dim3(grid), dim3(p.decode ? attn_threads<true>() : attn_threads<false>()), smem, s, m_rows,
-           m_win, m_q, m_part, p);
+           m_win, m_q, m_part, m_rope, m_scale, p);
+  CSAHCA_CHECK_LAUNCH();
+  return CSAHCA_OK;
+}
+
+// ---- tensor-core attention for 16 heads of 128 dims (HCA prefill, bf16) ------
+
+bool attn_small_tc_ok(const csahca_attn_args* a) {
+  return a->dtype == CSAHCA_BF16 && a->kind == CSAHCA_HCA && a->H == kSmH && a->d == kSmD &&
+         a->rope_dims <= 128;
+}
+
+int launch_attn_small(const csahca_attn_args* a, const void* win_final, double base, float eps, float scale,
+                      cudaStream_t s) {
+  AttnSmallParams t;
+  memset(&t, 0, sizeof(t));
+  t.q = static_cast<const __nv_bfloat16*>(a->q); t.q_gain = a->q_gain; t.sinks = a->sinks;
+  t.q_norm = a->q_norm; t.eps = eps; t.scale_log2 = scale * kLog2e; t.rope_dims = a->rope_dims;
+  t.B = a->B; t.n = a->n; t.N = a->N; t.m = a->m; t.w = a->w;
+  t.n_items = a->B * (int)ceil_div64(a->n, kSmQ);
+  t.first_kernel = a->w > 0 ? 0 : 1;
+  t.out = static_cast<__nv_bfloat16*>(a->out);
+  rope_theta_table(t.theta, a->rope_dims, base);
+  // rows of 128 bf16 seen as [chunk 2][row][64]: one box = 128 key rows x both
+  // chunks (32 KB), the query box = 64 rows x both chunks (16 KB)
+  const uint64_t rs = kSmD * 2;
+  CUtensorMap m_q, m_comp, m_win;
+  bool ok = encode_3d(&m_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->q, 64, (uint64_t)a->B * a->n * kSmH, 2, rs, 128, 64,
+                      kSmN, 2, CU_TENSOR_MAP_SWIZZLE_128B);
+  m_comp = m_q;
+  m_win = m_q;
+  if ((int64_t)a->B * a->N > 0)
+    ok = ok && encode_3d(&m_comp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->kv_comp, 64, (uint64_t)a->B * a->N, 2, rs,
+                         128, 64, 128, 2, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (a->w > 0)
+    ok = ok && encode_3d(&m_win, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, win_final, 64, (uint64_t)a->B * a->n, 2, rs, 128,
+                         64, 128, 2, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return CSAHCA_ERR_LAUNCH;
+  cudaFuncSetAttribute(attn_small_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SmSmem::TOTAL);
+  int grid = 2 * num_sms();
+  if (grid > t.n_items) grid = t.n_items;
+  if (grid <= 0) return CSAHCA_OK;
+  CSAHCA_TRACE("attn_prefill_hca_small_tc", s);
+  launch_k(attn_small_tc_kernel, dim3(grid), dim3(kSmThreads), SmSmem::TOTAL, s, m_comp, m_win, m_q, t);
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
 }
@@ -696,6 +839,7 @@ int run_prefill_t(const csahca_attn_args* a, cudaStream_t s) {
     if (st != CSAHCA_OK) return st;
   }
   const float scale = a->scale > 0 ? a->scale : 1.0f / sqrtf((float)a->d);
+  if (attn_small_tc_ok(a)) return launch_attn_small(a, win_final, base, eps, scale, s);
   if (attn_tc_shape_ok(a->dtype, a->H, a->d, a->rope_dims, (int64_t)a->B * a->N, (int64_t)a->B * a->n)) {
     AttnTcParams t;
     memset(&t, 0, sizeof(t));
@@ -740,14 +884,24 @@ int run_prefill(const csahca_attn_args* a, void* stream) {
 
 constexpr int kDecodeKeysPerSplit = 256;
 
+bool decode_tc(const csahca_decode_args* a);
+
 int validate_decode(const csahca_decode_args* a, bool shapes_only = false) {
   if (!a) return CSAHCA_ERR_INVALID_ARG;
   if (a->kind != CSAHCA_CSA && a->kind != CSAHCA_HCA) return CSAHCA_ERR_INVALID_ARG;
   if (a->dtype != CSAHCA_F32 && a->dtype != CSAHCA_BF16) return CSAHCA_ERR_INVALID_ARG;
-  if (a->B < 0 || a->H < 1 || a->d < 1 || a->N_cap < 0 || a->m < 1 || a->w < 0)
+  if (a->B < 0 || a->H < 1 || a->d < 1 || a->N_cap < 0 || a->m < 1 || a->w < 0 || a->entry_base < 0)
     return CSAHCA_ERR_INVALID_ARG;
   if (a->rope_dims < 0 || a->rope_dims > a->d || (a->rope_dims & 1)) return CSAHCA_ERR_INVALID_ARG;
   if (a->d % 32 || a->d > 32 * kSimtMaxDPL) return CSAHCA_ERR_UNSUPPORTED;
+  // context parallelism: the tensor-core path only; a CSA shard past the
+  // first takes its selection from cp_topk_merge
+  const bool cp = a->entry_base > 0 || a->partial_out || a->skip_window;
+  if (cp && !decode_tc(a)) return CSAHCA_ERR_UNSUPPORTED;
+  if (a->kind == CSAHCA_CSA && a->entry_base > 0 && !a->idx_in) return CSAHCA_ERR_INVALID_ARG;
+  if (a->kv_dtype == CSAHCA_E4M3 &&
+      (a->dtype != CSAHCA_BF16 || !decode_tc(a) || kv_f8_row_bytes(a->d, a->rope_dims) == 0))
+    return CSAHCA_ERR_UNSUPPORTED;
   if (a->kind == CSAHCA_CSA) {
     if (a->k < 1) return CSAHCA_ERR_INVALID_ARG;
     if (!a->idx_in) {
@@ -761,14 +915,14 @@ int validate_decode(const csahca_decode_args* a, bool shapes_only = false) {
     }
   }
   if (shapes_only || a->B == 0) return CSAHCA_OK;
-  if (!a->q || !a->pos || !a->sinks || !a->out) return CSAHCA_ERR_INVALID_ARG;
+  if (!a->q || !a->pos || !a->sinks || (!a->out && !a->partial_out)) return CSAHCA_ERR_INVALID_ARG;
   if (a->kind == CSAHCA_CSA && !a->idx_in && (!a->qI || !a->wI || (a->N_cap > 0 && !a->kI) ||
                                               (a->kI_dtype == CSAHCA_E4M3 && a->N_cap > 0 && !a->kI_scale)))
     return CSAHCA_ERR_INVALID_ARG;
   if (a->N_cap > 0 && !a->kv_cache) return CSAHCA_ERR_INVALID_ARG;
-  if (a->w > 0 && !a->win) return CSAHCA_ERR_INVALID_ARG;
+  if (a->w > 0 && !a->win && !a->skip_window) return CSAHCA_ERR_INVALID_ARG;
   const void* ptrs[] = {a->q, a->pos, a->q_gain, a->kv_cache, a->win, a->sinks, a->qI, a->wI,
-                        a->kI, a->kI_scale, a->idx_in, a->idx_out, a->out, a->workspace};
+                        a->kI, a->kI_scale, a->idx_in, a->idx_out, a->out, a->partial_out, a->workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return CSAHCA_ERR_ALIGNMENT;
   return CSAHCA_OK;
@@ -783,7 +937,9 @@ struct DecodeLayout {
 };
 
 bool decode_tc(const csahca_decode_args* a) {
-  return attn_tc_shape_ok(a->dtype, a->H, a->d, a->rope_dims, (int64_t)a->B * a->N_cap, (int64_t)a->B * a->w);
+  // (a skipped window is never read: its tensor map falls back to the cache)
+  return attn_tc_shape_ok(a->dtype, a->H, a->d, a->rope_dims, (int64_t)a->B * a->N_cap,
+                          a->skip_window ? 128 : (int64_t)a->B * a->w);
 }
 
 DecodeLayout decode_layout(const csahca_decode_args* a) {
@@ -799,7 +955,7 @@ DecodeLayout decode_layout(const csahca_decode_args* a) {
     // wave (gathered CSA tiles of 128 rows: smaller ones, 64 or 32 rows,
     // measured slower at decode_1m, the per-tile fixed costs dominating)
     const int B = a->B > 0 ? a->B : 1;
-    const int64_t wt = ceil_div64(a->w, 128);
+    const int64_t wt = a->skip_window ? 0 : ceil_div64(a->w, 128);
     const int tiles = (int)(ceil_div64(csa ? a->k : a->N_cap, csa ? L.gtile : 128) + wt);
     int want = (int)ceil_div64(num_sms(), B);
     if (want > kTcCombineMaxSplits) want = kTcCombineMaxSplits;
@@ -866,11 +1022,16 @@ int run_decode_t(const csahca_decode_args* a, cudaStream_t s, char* ws) {
     t.q_norm = a->q_norm; t.eps = eps; t.scale_log2 = scale * kLog2e; t.rope_dims = a->rope_dims;
     t.rope_base = base; t.B = a->B; t.nq = 1; t.N = a->N_cap; t.m = a->m; t.k = a->k; t.w = a->w;
     t.csa = a->kind == CSAHCA_CSA; t.idx = sel; t.decode = 1;
+    t.entry_base = a->entry_base; t.skip_window = a->skip_window ? 1 : 0;
     t.splits = L.splits; t.tiles_per_split = L.tiles_per_split; t.n_items = a->B * L.splits; t.gtile = L.gtile;
     t.first_kernel = (a->kind != CSAHCA_CSA || a->idx_in) ? 1 : 0;
     t.out = nullptr; t.partial = partial;
-    st = launch_attn_tc(t, a->kv_cache, (int64_t)a->B * a->N_cap, a->w > 0 ? a->win : nullptr,
-                        (int64_t)a->B * a->w, s, a->kind == CSAHCA_CSA ? "attn_decode_csa_tc" : "attn_decode_hca_tc");
+    const bool f8 = a->kv_dtype == CSAHCA_E4M3;
+    st = launch_attn_tc(t, a->kv_cache, (int64_t)a->B * a->N_cap, (a->w > 0 && !a->skip_window) ? a->win : nullptr,
+                        (int64_t)a->B * a->w, s,
+                        a->kind == CSAHCA_CSA ? (f8 ? "attn_decode_csa_tc_f8kv" : "attn_decode_csa_tc")
+                                              : (f8 ? "attn_decode_hca_tc_f8kv" : "attn_decode_hca_tc"),
+                        f8);
   } else {
     SimtAttnParams p;
     memset(&p, 0, sizeof(p));
@@ -890,19 +1051,20 @@ int run_decode_t(const csahca_decode_args* a, cudaStream_t s, char* ws) {
     TcCombineParams c;
     c.partial = reinterpret_cast<const char*>(partial); c.sinks = a->sinks; c.pos = a->pos;
     c.out = static_cast<__nv_bfloat16*>(a->out);
+    c.partial_out = a->partial_out;
     c.rows = a->B; c.splits = L.splits; c.rope_dims = a->rope_dims;
     rope_theta_table(c.theta, a->rope_dims, base);              // rope_dims <= 128 on this path
     const int smem = tc_combine_smem_bytes(L.splits);
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(attn_combine_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    // the partials as [B * splits blocks][518 rows][64 fp16]: one box takes
-    // the m, l, up headers of every split of a query, one the 16-dim slices
+    // the partials as [B * splits blocks][516 rows][64 bf16]: one box takes
+    // the m, l headers of every split of a query, one the 16-dim slices
     CUtensorMap hdr_map, slc_map;
     const uint64_t blocks = (uint64_t)a->B * L.splits;
     const uint32_t slc_box = (uint32_t)(L.splits < kTcCombineSlots ? L.splits : kTcCombineSlots);
-    if (!encode_3d(&hdr_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, partial, kAttnH, kTcPartialRows, blocks, kAttnH * 2,
+    if (!encode_3d(&hdr_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, partial, kAttnH, kTcPartialRows, blocks, kAttnH * 2,
                    kTcPartialBytes, kAttnH, kTcPartialHeaderRows, (uint32_t)L.splits) ||
-        !encode_3d(&slc_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, partial, kAttnH, kTcPartialRows, blocks, kAttnH * 2,
+        !encode_3d(&slc_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, partial, kAttnH, kTcPartialRows, blocks, kAttnH * 2,
                    kTcPartialBytes, kAttnH, kTcCombineDims, slc_box))
       return CSAHCA_ERR_LAUNCH;
     {
@@ -943,7 +1105,8 @@ int run_decode_compress(const csahca_decode_compress_args* a, void* stream) {
   if (!a) return CSAHCA_ERR_INVALID_ARG;
   if (a->kind != CSAHCA_CSA && a->kind != CSAHCA_HCA) return CSAHCA_ERR_INVALID_ARG;
   if (a->dtype != CSAHCA_F32 && a->dtype != CSAHCA_BF16) return CSAHCA_ERR_INVALID_ARG;
-  if (a->B < 0 || a->d <= 0 || a->m < 1 || a->N_cap < 0 || a->w < 0 || a->dI < 0) return CSAHCA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->d <= 0 || a->m < 1 || a->N_cap < 0 || a->w < 0 || a->dI < 0 || a->entry_base < 0)
+    return CSAHCA_ERR_INVALID_ARG;
   if (a->rope_dims < 0 || a->rope_dims > a->d || (a->rope_dims & 1)) return CSAHCA_ERR_INVALID_ARG;
   if (a->rope_dims > 2 * kDcMaxRopePairs) return CSAHCA_ERR_UNSUPPORTED;
   const bool csa = a->kind == CSAHCA_CSA;
@@ -966,6 +1129,10 @@ int run_decode_compress(const csahca_decode_compress_args* a, void* stream) {
   if (dI && (!a->ia || !a->ib || !a->iza || !a->izb || !a->ibias_a || !a->ibias_b || !a->iring || !a->kI))
     return CSAHCA_ERR_INVALID_ARG;
   if (dI && a->kI_dtype == CSAHCA_E4M3 && !a->kI_scale) return CSAHCA_ERR_INVALID_ARG;
+  // FP8 KV rows: each CTA of a cluster owns one 64-dim block of the row
+  const bool kv_f8 = a->kv_dtype == CSAHCA_E4M3;
+  if (kv_f8 && (a->dtype != CSAHCA_BF16 || a->d != 64 * kDcCluster || kv_f8_row_bytes(a->d, a->rope_dims) == 0))
+    return CSAHCA_ERR_UNSUPPORTED;
   const void* ptrs[] = {a->pos, a->kv_raw, a->a, a->b, a->za, a->zb, a->bias_a, a->bias_b, a->kv_gain,
                         a->ring, a->kv_cache, a->win, a->ia, a->ib, a->iza, a->izb, a->ibias_a,
                         a->ibias_b, a->iring, a->kI, a->kI_scale};
@@ -986,6 +1153,9 @@ int run_decode_compress(const csahca_decode_compress_args* a, void* stream) {
   }
   p.B = a->B; p.d = a->d; p.dI = dI; p.m = a->m; p.N_cap = a->N_cap; p.w = a->w;
   p.rope_dims = a->rope_dims; p.kv_norm = a->kv_norm; p.ki_e4m3 = dI && a->kI_dtype == CSAHCA_E4M3;
+  p.kv_f8 = kv_f8 ? 1 : 0;
+  p.kv_row_bytes = kv_f8 ? kv_f8_row_bytes(a->d, a->rope_dims) : 0;
+  p.entry_base = a->entry_base;
   p.eps = a->eps > 0 ? a->eps : kDefaultEps;
   rope_theta_table(p.theta, a->rope_dims, a->rope_base > 0 ? a->rope_base : kDefaultRopeBase);
   cudaStream_t s = as_stream(stream);
@@ -997,6 +1167,71 @@ int run_decode_compress(const csahca_decode_compress_args* a, void* stream) {
   } else {
     if (csa) launch_k(decode_compress_kernel<__nv_bfloat16, true>, grid, block, 0, s, p);
     else launch_k(decode_compress_kernel<__nv_bfloat16, false>, grid, block, 0, s, p);
+  }
+  CSAHCA_CHECK_LAUNCH();
+  return CSAHCA_OK;
+}
+
+// ------------------------------------------------------ context parallelism --
+
+int run_cp_topk_merge(const csahca_cp_topk_merge_args* a, void* stream) {
+  if (!a) return CSAHCA_ERR_INVALID_ARG;
+  if (a->R < 1 || a->rows < 0 || a->k < 1 || a->rank < 0 || a->rank >= a->R) return CSAHCA_ERR_INVALID_ARG;
+  if (a->R > kCpMaxRanks || a->k > kCpMaxK || (int64_t)a->R * a->k > kCpMaxCand) return CSAHCA_ERR_UNSUPPORTED;
+  if (a->rows == 0) return CSAHCA_OK;
+  if (!a->bases || !a->cand_idx || !a->cand_scores || (!a->idx_global && !a->idx_local))
+    return CSAHCA_ERR_INVALID_ARG;
+  const void* ptrs[] = {a->cand_idx, a->cand_scores, a->idx_global, a->idx_local};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return CSAHCA_ERR_ALIGNMENT;
+  CpTopkMergeParams p;
+  memset(&p, 0, sizeof(p));
+  for (int r = 0; r < a->R; ++r) {
+    if (a->bases[r] < 0) return CSAHCA_ERR_INVALID_ARG;
+    p.bases[r] = a->bases[r];
+  }
+  int st = device_ok();
+  if (st != CSAHCA_OK) return st;
+  p.cand_idx = a->cand_idx; p.cand_scores = a->cand_scores;
+  p.idx_global = a->idx_global; p.idx_local = a->idx_local;
+  p.R = a->R; p.rows = a->rows; p.k = a->k; p.rank = a->rank;
+  p.kpow2 = 1;
+  while (p.kpow2 < a->k) p.kpow2 <<= 1;
+  const int smem = cp_topk_merge_smem_bytes(a->R, a->k, p.kpow2);
+  cudaFuncSetAttribute(cp_topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaStream_t s = as_stream(stream);
+  {
+    CSAHCA_TRACE("cp_topk_merge", s);
+    launch_k(cp_topk_merge_kernel, dim3((unsigned)a->rows), dim3(kCpMergeThreads), smem, s, p);
+  }
+  CSAHCA_CHECK_LAUNCH();
+  return CSAHCA_OK;
+}
+
+int run_cp_attn_merge(const csahca_cp_merge_args* a, void* stream) {
+  if (!a) return CSAHCA_ERR_INVALID_ARG;
+  if (a->dtype != CSAHCA_F32 && a->dtype != CSAHCA_BF16) return CSAHCA_ERR_INVALID_ARG;
+  if (a->R < 1 || a->rows < 0 || a->H < 1 || a->d < 1) return CSAHCA_ERR_INVALID_ARG;
+  if (a->rope_dims < 0 || a->rope_dims > a->d || (a->rope_dims & 1)) return CSAHCA_ERR_INVALID_ARG;
+  if (a->R > kCpMaxRanks || a->d % 4 || a->d > 1024 || a->rope_dims > 128) return CSAHCA_ERR_UNSUPPORTED;
+  if ((int64_t)a->rows * a->H > INT32_MAX) return CSAHCA_ERR_UNSUPPORTED;
+  if (a->rows == 0) return CSAHCA_OK;
+  if (!a->partials || !a->sinks || !a->pos || !a->out) return CSAHCA_ERR_INVALID_ARG;
+  const void* ptrs[] = {a->partials, a->sinks, a->pos, a->out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return CSAHCA_ERR_ALIGNMENT;
+  int st = device_ok();
+  if (st != CSAHCA_OK) return st;
+  CpMergeParams p;
+  memset(&p, 0, sizeof(p));
+  p.partials = a->partials; p.sinks = a->sinks; p.pos = a->pos; p.out = a->out;
+  p.R = a->R; p.rows = a->rows; p.H = a->H; p.d = a->d; p.rope_dims = a->rope_dims;
+  p.out_bf16 = a->dtype == CSAHCA_BF16 ? 1 : 0;
+  rope_theta_table(p.theta, a->rope_dims, a->rope_base > 0 ? a->rope_base : kDefaultRopeBase);
+  cudaStream_t s = as_stream(stream);
+  {
+    CSAHCA_TRACE("cp_attn_merge", s);
+    launch_k(cp_merge_kernel, dim3((unsigned)(a->rows * a->H)), dim3((unsigned)(a->d / 4)), 0, s, p);
   }
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
@@ -1034,6 +1269,10 @@ int decode_compress(const csahca_decode_compress_args* args, void* stream) {
   return run_decode_compress(args, stream);
 }
 
+int cp_topk_merge(const csahca_cp_topk_merge_args* args, void* stream) { return run_cp_topk_merge(args, stream); }
+
+int cp_attn_merge(const csahca_cp_merge_args* args, void* stream) { return run_cp_attn_merge(args, stream); }
+
 size_t csahca_decode_workspace_size(const csahca_decode_args* args) {
   if (validate_decode(args, true) != CSAHCA_OK) return 0;
   if (args->B == 0) return 0;
@@ -1056,6 +1295,16 @@ const char* csahca_status_string(int status) {
 
 int csahca_abi_version(void) { return CSAHCA_ABI_VERSION; }
 
+int64_t csahca_kv_row_bytes(int32_t kv_dtype, int32_t d, int32_t rope_dims) {
+  if (d <= 0) return 0;
+  switch (kv_dtype) {
+    case CSAHCA_F32: return (int64_t)d * 4;
+    case CSAHCA_BF16: return (int64_t)d * 2;
+    case CSAHCA_E4M3: return kv_f8_row_bytes(d, rope_dims);
+    default: return 0;
+  }
+}
+
 int64_t csahca_struct_size(int which) {
   switch (which) {
     case 0: return (int64_t)sizeof(csahca_compress_args);
@@ -1063,6 +1312,8 @@ int64_t csahca_struct_size(int which) {
     case 2: return (int64_t)sizeof(csahca_attn_args);
     case 3: return (int64_t)sizeof(csahca_decode_args);
     case 4: return (int64_t)sizeof(csahca_decode_compress_args);
+    case 5: return (int64_t)sizeof(csahca_cp_topk_merge_args);
+    case 6: return (int64_t)sizeof(csahca_cp_merge_args);
     default: return -1;
   }
 }

@@ -48,6 +48,9 @@ struct DecodeCompressParams {
   void* kI;                                   // [B, N_cap, dI] (T, or e4m3 codes)
   float* kI_scale;                            // [B, N_cap, dI/128] (e4m3)
   int B, d, dI, m, N_cap, w, rope_dims, kv_norm, ki_e4m3;
+  int kv_f8;                                  // kv_cache holds FP8 KV rows (one 64-dim block per CTA)
+  int64_t kv_row_bytes;
+  int entry_base;                             // local cache row j holds global entry entry_base + j
   float eps;
   // RoPE angle per unit of position of pair j, base^(-2j/r), computed in
   // double on the host: the kernel then carries no pow() of its own
@@ -144,8 +147,11 @@ decode_compress_kernel(const __grid_constant__ DecodeCompressParams p) {
   float wv[VEC];
   if (has_win && tid < nvr) load16(static_cast<const T*>(p.kv_raw) + (int64_t)b * d + tid * VEC, wv);
   const int t = p.pos[b];
-  const bool emit = t >= 0 && (t + 1) % m == 0 && (t + 1) / m - 1 < p.N_cap;
-  const int i = (t + 1) / m - 1;
+  const int64_t t1 = (int64_t)t + 1;          // (no overflow for any position)
+  // global entry i completes; it is stored in local row i - entry_base
+  const bool emit = t >= 0 && t1 % m == 0 && t1 / m - 1 >= p.entry_base && t1 / m - 1 - p.entry_base < p.N_cap;
+  const int i = emit ? (int)(t1 / m - 1) : 0;
+  const int64_t lrow = emit ? (int64_t)i - p.entry_base : 0;
   const bool do_win = has_win && t >= 0;
 
   // ---- the new token into ring slot t % R
@@ -293,11 +299,37 @@ decode_compress_kernel(const __grid_constant__ DecodeCompressParams p) {
 #pragma unroll
     for (int e = 0; e < VEC; ++e) v[e] = pooled[tid * VEC + e];
     dc_finish<VEC>(v, ch, p, rsqrtf(tot[0] / (float)d + p.eps), (double)i * (double)m);
-    store16(static_cast<T*>(p.kv_cache) + ((int64_t)b * p.N_cap + i) * d + ch, v);
+    if (p.kv_f8) {
+      // FP8 KV row: this CTA's slice is one 64-dim block, of codes (with its
+      // scale = amax / 448, codes = nearest e4m3 of x / scale) or of RoPE dims (bf16)
+      uint8_t* row = static_cast<uint8_t*>(p.kv_cache) + ((int64_t)b * p.N_cap + lrow) * p.kv_row_bytes;
+      const int r0 = d - p.rope_dims;
+      if constexpr (VEC == 8) {
+        if (q * sc >= r0) {
+          store16(reinterpret_cast<__nv_bfloat16*>(row + r0 + 2 * (ch - r0)), v);
+        } else {
+          float am = 0.f;
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) am = fmaxf(am, fabsf(v[e]));
+          const unsigned lanes = (1u << nvk) - 1u;            // the slice's threads: lanes 0 .. nvk-1
+          for (int o = 1; o < nvk; o <<= 1) am = fmaxf(am, __shfl_xor_sync(lanes, am, o));
+          const float scale = am > 0.f ? __fdiv_rn(am, 448.0f) : 1.0f;
+          uint32_t w8[2] = {0u, 0u};
+#pragma unroll
+          for (int e = 0; e < VEC; ++e)
+            w8[e / 4] |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(v[e], scale), __NV_SATFINITE, __NV_E4M3)
+                         << (8 * (e % 4));
+          *reinterpret_cast<uint2*>(row + ch) = make_uint2(w8[0], w8[1]);
+          if (tid == 0) *reinterpret_cast<float*>(row + d + p.rope_dims + 4 * (ch / 64)) = scale;
+        }
+      }
+    } else {
+      store16(static_cast<T*>(p.kv_cache) + ((int64_t)b * p.N_cap + lrow) * d + ch, v);
+    }
   } else if (kCSA && tid >= 32 && tid < 32 + nvi) {
     const int u = tid - 32, ch = q * si + u * VEC;
     const float* x = pooled + (nvk + u) * VEC;
-    const int64_t row = (int64_t)b * p.N_cap + i;
+    const int64_t row = (int64_t)b * p.N_cap + lrow;
     float v[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) v[e] = x[e];

@@ -53,7 +53,7 @@ struct IdxF8Cfg {
   static constexpr int B_TERM = HI * 128;           // one e4m3 term: HI rows x 128 bytes
   static constexpr int B_BYTES = 2 * B_TERM;
   static constexpr int A_BYTES = 128 * 128;         // 128 keys x 128 e4m3
-  static constexpr int SMEM = 1024 + B_BYTES + kIdxF8Stages * A_BYTES;
+  static constexpr int SMEM = 1024 + B_BYTES + kIdxF8Stages * A_BYTES;   // plus the fused route's score buffer
   static constexpr int NCOL = 2 * HI;               // MMA N: both terms of every head
   static constexpr int TMEM_COLS = kIdxF8Acc * NCOL <= 256 ? 256 : 512;
   static_assert(kIdxF8Acc * NCOL <= 512, "accumulators fit in TMEM");
@@ -125,11 +125,100 @@ __device__ __forceinline__ void idx_row_done(const IdxTcParams& p, int row, uint
   if (run < k && run + tot >= k) {
 #pragma unroll
     for (int e = 7; e >= 0; --e) {
-      if (run + c[e] >= k) { cnt[kCntT] = (uint32_t)(ept * 8 + e); cnt[kCntAboveT] = run; break; }
+      if (run + c[e] >= k) {
+        cnt[kCntT] = (uint32_t)(ept * 8 + e);
+        cnt[kCntAboveT] = run;
+        if (p.route) {
+          __threadfence();                           // T and the count before the flag
+          atomicExch(&cnt[kCntReady], 1u);
+        }
+        break;
+      }
       run += c[e];
     }
   }
   epi_sync256();
+}
+
+// Exclusive prefix of c over the 256 epilogue threads (named barrier 3);
+// *total receives the sum.  buf: 9 ints.
+__device__ __forceinline__ int epi_excl_count(int c, int* buf, int* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) buf[wid] = incl;
+  epi_sync256();
+  int base = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    const int x = buf[w];
+    base += w < wid ? x : 0;
+    tot += x;
+  }
+  *total = tot;
+  epi_sync256();
+  return base + incl - c;
+}
+
+// Fused routing of one work item (all 256 epilogue threads): wait until the
+// row's last item has stored the threshold bin T (bounded), then send this
+// item's keys above T to the row's taken list and those in T to its
+// candidate list, reserving each list range with one atomic per CTA.
+__device__ __forceinline__ void idx_route(const IdxTcParams& p, int row, int key0, int nkeys, int v,
+                                          const float* sc, int* buf, uint32_t* sh_T, int* sh_ok,
+                                          uint32_t* sh_base, volatile int* abort_flag) {
+  const int ept = threadIdx.x;
+  uint32_t* cnt = p.counters + (int64_t)row * kTopkCounters;
+  if (ept == 0) {
+    int ok = 0;
+    for (uint32_t it = 0; it < kMbarSpinLimit; ++it) {
+      uint32_t r;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(r) : "l"(cnt + kCntReady) : "memory");
+      if (r) { ok = 1; break; }
+      if ((it & 1023u) == 1023u && *abort_flag) break;
+      __nanosleep(64);
+    }
+    if (!ok) { raise_device_error(DEVERR_MBAR_TIMEOUT); *abort_flag = 1; }
+    *sh_ok = ok;
+    *sh_T = ok ? __ldcg(&cnt[kCntT]) : 0u;
+  }
+  epi_sync256();
+  if (!*sh_ok) return;
+  const uint32_t T = *sh_T;
+  int* above = p.above + (int64_t)row * p.k;
+  uint2* cand = p.cand + (int64_t)row * p.N;
+  int nt = 0, nc = 0;
+  for (int i = ept; i < nkeys; i += 256) {
+    if (key0 + i >= v) break;
+    const uint32_t b = order_key(sc[i]) >> kHistShift;
+    nt += b > T;
+    nc += b == T;
+  }
+  int tot;
+  const int off = epi_excl_count(nt | (nc << 16), buf, &tot);
+  if (ept == 0) {
+    sh_base[0] = tot & 0xFFFF ? atomicAdd(&cnt[kCntAbove], (uint32_t)(tot & 0xFFFF)) : 0u;
+    sh_base[1] = tot >> 16 ? atomicAdd(&cnt[kCntCand], (uint32_t)(tot >> 16)) : 0u;
+  }
+  epi_sync256();
+  uint32_t pt = sh_base[0] + (uint32_t)(off & 0xFFFF), pc = sh_base[1] + (uint32_t)(off >> 16);
+  for (int i = ept; i < nkeys; i += 256) {
+    const int j = key0 + i;
+    if (j >= v) break;
+    const uint32_t key = order_key(sc[i]);
+    const uint32_t b = key >> kHistShift;
+    if (b > T) {
+      if (pt < (uint32_t)p.k) above[pt] = j;
+      ++pt;
+    } else if (b == T) {
+      if (pc < (uint32_t)p.N) cand[pc] = make_uint2(key, (uint32_t)j);
+      ++pc;
+    }
+  }
 }
 
 template <int HI>
@@ -151,14 +240,20 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
   __shared__ float sScale[NS][128];               // key row scales of each stage
   __shared__ uint32_t scan_s[512];                // threshold search of a finished row
   __shared__ int row_flag;
+  __shared__ int route_buf[9];
+  __shared__ uint32_t route_T, route_base[2];
+  __shared__ int route_ok;
+  float* sc_s = reinterpret_cast<float*>(sA + NS * Cfg::A_BYTES);   // fused route: this item's scores
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     abort_flag = 0;
     // a stage is full once its key tile (TMA bytes, lane 0's arrive) and its
     // scales (one cp.async arrive per producer lane) have landed; it is empty
-    // once the MMAs have read the keys and the owning epilogue group the scales
-    for (int s = 0; s < NS; ++s) { mbar_init(&bar_a_full[s], 1 + 32); mbar_init(&bar_a_empty[s], 1 + 128); }
+    // once the owning epilogue group has seen the tile's accumulator (so the
+    // MMAs have read the keys) and read the scales: a tcgen05.commit costs the
+    // tensor pipe a few hundred cycles, so the MMA issuers commit once per tile
+    for (int s = 0; s < NS; ++s) { mbar_init(&bar_a_full[s], 1 + 32); mbar_init(&bar_a_empty[s], 128); }
     // (the producer of tile i is warp 8 + (i & 1); its stage has that parity too)
     for (int j = 0; j < NACC; ++j) { mbar_init(&bar_acc_full[j], 1); mbar_init(&bar_acc_empty[j], 128); }
     mbar_init(&bar_b_full, 128);
@@ -251,7 +346,6 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
           const uint32_t d = tmem + j * Cfg::NCOL;
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks) umma_e4m3(d, ad + 2 * ks, bdesc0 + 2 * ks, idesc, ks != 0);
-          umma_commit(&bar_a_empty[s]);
           umma_commit(&bar_acc_full[j]);
         }
         if (!ok) break;
@@ -368,7 +462,8 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
         mbar_arrive(&bar_acc_empty[j]);
         if (key < v) {
           const float score = acc * kscale;
-          srow[key] = score;
+          if (p.route) sc_s[(kt - it.kt0) * 128 + et] = score;
+          else srow[key] = score;
           if (do_hist) atomicAdd(&hist_s[order_key(score) >> kHistShift], 1u);
         }
       }
@@ -380,6 +475,9 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
           if (c) { atomicAdd(gh + i, c); hist_s[i] = 0; }
         }
         idx_row_done(p, row, scan_s, &row_flag);
+        if (p.route && v > p.k)
+          idx_route(p, row, it.kt0 * 128, (it.kt1 - it.kt0) * 128, v, sc_s, route_buf, &route_T, &route_ok,
+                    route_base, &abort_flag);
       }
     }
   }

@@ -18,12 +18,15 @@ struct IndexerParams {
   float* scores; int64_t score_row_stride;   // row r = b * nq + q (within the chunk)
   int B, nq, HI, dI, N, m;
   int q_begin, q_count;                       // query chunk [q_begin, q_begin + q_count)
+  int entry_base;                             // local row j is global entry entry_base + j
 };
 
-__device__ __forceinline__ int visible_count(int t, int m, int N) {
+// Local rows of a cache shard (global entries base .. base + N - 1) visible
+// to the query at position t: entry i is visible iff (i + 1) m - 1 <= t.
+__device__ __forceinline__ int visible_count(int t, int m, int N, int base = 0) {
   if (t < 0) return 0;
-  int v = (int)(((int64_t)t + 1) / m);
-  return v < N ? v : N;
+  const int64_t v = ((int64_t)t + 1) / m - base;
+  return v <= 0 ? 0 : (v < N ? (int)v : N);
 }
 
 template <typename TQ, typename TK, bool kFP8>
@@ -36,7 +39,7 @@ __global__ void __launch_bounds__(256) indexer_scores_simt(IndexerParams p) {
   const int qi = p.q_begin + blockIdx.y;
   const int b = blockIdx.z;
   const int t = p.q_pos[(int64_t)b * p.nq + qi];
-  const int v = visible_count(t, p.m, p.N);
+  const int v = visible_count(t, p.m, p.N, p.entry_base);
   const int key0 = blockIdx.x * 256;
   if (key0 >= v) return;
   const TQ* Q = static_cast<const TQ*>(p.qI) + ((int64_t)b * p.nq + qi) * p.HI * p.dI;

@@ -28,6 +28,7 @@ struct IdxTcParams {
   const float* w; const float* kI_scale; const int* q_pos;
   float* scores; int64_t score_row_stride;
   int B, nq, HI, N, m;
+  int entry_base;             // local row j is global entry entry_base + j
   int q_begin, q_count;
   int n_items;
   int splits;                 // > 0: decode items (b, split); 0: prefill items (b, query tile)
@@ -38,6 +39,13 @@ struct IdxTcParams {
   int k;                      // with hist: the top-k size
   int first_kernel;           // 0: an earlier kernel of the call precedes (the FP8 decode scan may
                               // then load keys before its wait; the keys are call inputs)
+  // fused routing (FP8 decode scan, one work item per CTA): scores stay in
+  // shared memory, and once the row's threshold bin is known every CTA routes
+  // its own keys into the row's taken list `above` [rows][k] and candidate
+  // list `cand` [rows][N]; topk_finish_kernel then selects exactly
+  int route;
+  int* above;
+  uint2* cand;
 };
 
 template <int QT, int HI, bool kFP8>
@@ -58,10 +66,7 @@ struct IdxTcCfg {
 struct IdxItem { int b, q0, qn, kt0, kt1; };
 
 __device__ __forceinline__ int idx_visible(const IdxTcParams& p, int b, int q) {
-  const int t = p.q_pos[(int64_t)b * p.nq + q];
-  if (t < 0) return 0;
-  const int64_t v = ((int64_t)t + 1) / p.m;
-  return (int)(v < p.N ? v : p.N);
+  return visible_count(p.q_pos[(int64_t)b * p.nq + q], p.m, p.N, p.entry_base);
 }
 
 template <int QT>
@@ -113,7 +118,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     abort_flag = 0;
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bar_a_full[s], kFP8 ? 128 : 1);
-      mbar_init(&bar_a_empty[s], 1);
+      // empty once the epilogue has seen the tile's accumulator (the MMAs
+      // have read the keys): one tcgen05.commit per tile, not two
+      mbar_init(&bar_a_empty[s], 128);
       mbar_init(&bar_raw_full[s], 1);
       mbar_init(&bar_raw_empty[s], 128);
     }
@@ -197,7 +204,6 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             for (int ks = 0; ks < 4; ++ks)
               umma_bf16(d, umma_desc_kmajor(sA0 + s * Cfg::A_BYTES + kc * 16384 + ks * 32),
                         umma_desc_kmajor(sB0 + kc * Cfg::B_CHUNK + ks * 32), idesc, (kc | ks) != 0);
-          umma_commit(&bar_a_empty[s]);
           umma_commit(&bar_acc_full[j]);
         }
         umma_commit(&bar_b_empty);
@@ -263,6 +269,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         const int j = acc_iter % NACC;
         const uint32_t aph = (acc_iter / NACC) & 1;
         if (!mbar_wait128(&bar_acc_full[j], aph, &abort_flag)) { stop = true; break; }
+        mbar_arrive(&bar_a_empty[acc_iter % NS]);       // the tile's key stage is free
         tc_fence_after();
         const int key = kt * 128 + et;
         float scale = 1.f;

@@ -116,6 +116,7 @@ struct TopkParams {
   int* idx;                                    // [B, nq, k]
   int B, nq, N, m, k;
   int q_begin, q_count;
+  int entry_base;                              // local row j is global entry entry_base + j
 };
 
 // Shared-memory slot of key j: one pad word per 32 keys keeps both the
@@ -133,8 +134,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(TopkParams p) {
   const int rloc = blockIdx.x;                 // row within the chunk
   const int b = rloc / p.q_count, qi = p.q_begin + rloc % p.q_count;
   const int t = p.q_pos[(int64_t)b * p.nq + qi];
-  int v = 0;
-  if (t >= 0) { int64_t vv = ((int64_t)t + 1) / p.m; v = (int)(vv < p.N ? vv : p.N); }
+  const int v = visible_count(t, p.m, p.N, p.entry_base);
   int* out = p.idx + ((int64_t)b * p.nq + qi) * p.k;
   const float* s = p.scores + (int64_t)rloc * p.row_stride;
   if (v <= p.k) {

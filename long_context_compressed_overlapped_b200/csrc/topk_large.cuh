@@ -33,6 +33,7 @@ constexpr int kCntSlices = 2;              // select CTAs done with the row
 constexpr int kCntItems = 3;               // indexer work items done with the row
 constexpr int kCntT = 4;                   // threshold bin (set by the indexer's last item)
 constexpr int kCntAboveT = 5;              // keys in bins above it
+constexpr int kCntReady = 6;               // 1 once kCntT / kCntAboveT are stored (fused routing)
 constexpr int kHistShift = 21;
 constexpr int kTopkLargeMaxN = 786432;     // two bitmaps of N bits in shared memory
 
@@ -41,6 +42,7 @@ struct TopkLargeParams {
   const int* q_pos;
   int* idx;
   int rows, N, m, k;
+  int entry_base;                          // local row j is global entry entry_base + j
   int slices;                              // CTAs per row in passes 1 and 2
   // workspace (per row)
   uint32_t* hist;                          // [rows][kHistBins]
@@ -57,10 +59,7 @@ struct TopkLargeParams {
 };
 
 __device__ __forceinline__ int topk_visible(const TopkLargeParams& p, int row) {
-  const int t = p.q_pos[row];
-  if (t < 0) return 0;
-  const int64_t v = ((int64_t)t + 1) / p.m;
-  return (int)(v < p.N ? v : p.N);
+  return visible_count(p.q_pos[row], p.m, p.N, p.entry_base);
 }
 
 // Zeroes n16 16-byte words of top-k scratch (histograms and counters).  A
@@ -253,81 +252,16 @@ __device__ __forceinline__ void sort1024_block(int* a) {
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kTopkSelectThreads, 2) topk_select_kernel(TopkLargeParams p) {
-  griddep_wait();
-  griddep_launch_dependents();
-  extern __shared__ uint32_t bm_sel[];               // [words] taken, then [words] ties
-  __shared__ uint32_t sh[1024];
-  __shared__ int warp_buf[72];
-  __shared__ uint32_t sh_digit, sh_need, sh_base_t, sh_base_c;
-  __shared__ int sh_last;
-  const int row = blockIdx.x / p.slices, slice = blockIdx.x % p.slices;
-  const int v = topk_visible(p, row);
-  int* out = p.idx + (int64_t)row * p.k;
-  if (v <= p.k) {
-    if (slice == 0)
-      for (int j = threadIdx.x; j < p.k; j += blockDim.x) out[j] = j < v ? j : -1;
-    return;
-  }
-  uint32_t* cnt = p.counters + (int64_t)row * kTopkCounters;
-  int* above = p.above + (int64_t)row * p.k;
-  uint2* cand = p.cand + (int64_t)row * p.N;
-  {
-    uint32_t n_above_T;
-    int T;
-    if (p.thresh_ready) {
-      T = (int)__ldcg(&cnt[kCntT]);
-      n_above_T = __ldcg(&cnt[kCntAboveT]);
-    } else {
-      T = threshold_bin(p.hist + (int64_t)row * kHistBins, p.k, sh, &n_above_T);
-    }
-    const int per = (v + p.slices - 1) / p.slices;
-    const int j0 = slice * per, j1 = min(v, j0 + per);
-    const float* s = p.scores + (int64_t)row * p.row_stride;
-    // 8 keys per thread per round; the CTA reserves its ranges of the row's
-    // taken / candidate lists with one atomic each (a block prefix sum places
-    // every thread's entries), so the row counters see one atomic per CTA
-    constexpr int kPer = 8;
-    for (int base = j0; base < j1; base += kPer * (int)blockDim.x) {
-      uint32_t key[kPer];
-      int nt = 0, nc = 0;
-#pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const int j = base + u * (int)blockDim.x + (int)threadIdx.x;
-        key[u] = j < j1 ? order_key(__ldcg(s + j)) : 0u;
-        const int bin = (int)(key[u] >> kHistShift);
-        nt += (j < j1 && bin > T);
-        nc += (j < j1 && bin == T);
-      }
-      int tot;
-      const int off = block_excl_count(nt | (nc << 16), warp_buf, &tot);
-      if (threadIdx.x == 0) {
-        sh_base_t = atomicAdd(&cnt[kCntAbove], (uint32_t)(tot & 0xFFFF));
-        sh_base_c = atomicAdd(&cnt[kCntCand], (uint32_t)(tot >> 16));
-      }
-      __syncthreads();
-      uint32_t pt = sh_base_t + (uint32_t)(off & 0xFFFF), pc = sh_base_c + (uint32_t)(off >> 16);
-#pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const int j = base + u * (int)blockDim.x + (int)threadIdx.x;
-        const int bin = (int)(key[u] >> kHistShift);
-        if (j < j1 && bin > T) {
-          if (pt < (uint32_t)p.k) above[pt] = j;
-          ++pt;
-        } else if (j < j1 && bin == T) {
-          if (pc < (uint32_t)p.N) cand[pc] = make_uint2(key[u], (uint32_t)j);
-          ++pc;
-        }
-      }
-      __syncthreads();
-    }
-  }
-  // publish this slice, then let the last CTA of the row finish it
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) sh_last = atomicAdd(&cnt[kCntSlices], 1u) == (uint32_t)(p.slices - 1);
-  __syncthreads();
-  if (!sh_last) return;
+// Exact finish of one row (one CTA, every thread): the taken list holds the
+// keys above the threshold bin T, the candidate list those in T; selects the
+// remaining count among the candidates (radix select of their 21 low bits)
+// and writes the row's k indices (ascending when p.sorted).  The shared
+// arrays are the caller's: bm_sel of topk_select_smem_bytes(N) bytes.
+__device__ __forceinline__ void topk_finish_row(const TopkLargeParams& p, int row, int v, int* out, uint32_t* cnt,
+                                             const int* above, const uint2* cand, uint32_t* bm_sel, int* warp_buf,
+                                             uint32_t* sh_digit_p, uint32_t* sh_need_p) {
+  uint32_t& sh_digit = *sh_digit_p;
+  uint32_t& sh_need = *sh_need_p;
   __threadfence();
 
   const uint32_t n_above = min(__ldcg(&cnt[kCntAbove]), (uint32_t)p.k);
@@ -450,14 +384,14 @@ __global__ void __launch_bounds__(kTopkSelectThreads, 2) topk_select_kernel(Topk
     __syncthreads();
 #pragma unroll
     for (int u = 0; u < 4; ++u)
-      if (abv[u] >= 0) atomicOr(&bm[abv[u] >> 5], 1u << (abv[u] & 31));
+      if (abv[u] >= 0 && abv[u] < v) atomicOr(&bm[abv[u] >> 5], 1u << (abv[u] & 31));
     for (uint32_t i = threadIdx.x + 4 * blockDim.x; i < n_above; i += blockDim.x) {
       const int j = __ldcg(above + i);
-      atomicOr(&bm[j >> 5], 1u << (j & 31));
+      if (j >= 0 && j < v) atomicOr(&bm[j >> 5], 1u << (j & 31));
     }
     for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
       const uint2 c = cand_local ? C[i] : __ldcg(cand + i);
-      if ((c.x & kLowMask) >= prefix) atomicOr(&bm[c.y >> 5], 1u << (c.y & 31));
+      if ((c.x & kLowMask) >= prefix && c.y < (uint32_t)v) atomicOr(&bm[c.y >> 5], 1u << (c.y & 31));
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
@@ -521,11 +455,12 @@ __global__ void __launch_bounds__(kTopkSelectThreads, 2) topk_select_kernel(Topk
   __syncthreads();
   for (uint32_t i = threadIdx.x; i < n_above; i += blockDim.x) {
     const int j = __ldcg(above + i);
-    atomicOr(&bm_sel[j >> 5], 1u << (j & 31));
+    if (j >= 0 && j < v) atomicOr(&bm_sel[j >> 5], 1u << (j & 31));
   }
   for (uint32_t i = threadIdx.x; i < n_cand; i += blockDim.x) {
     const uint2 c = __ldcg(cand + i);
     const uint32_t low = c.x & ((1u << kHistShift) - 1u);
+    if (c.y >= (uint32_t)v) continue;              // (the lists hold indices < v; a bitmap has v bits)
     if (low > prefix) atomicOr(&bm_sel[c.y >> 5], 1u << (c.y & 31));
     else if (low == prefix) atomicOr(&bm_eq[c.y >> 5], 1u << (c.y & 31));
   }
@@ -539,6 +474,105 @@ __global__ void __launch_bounds__(kTopkSelectThreads, 2) topk_select_kernel(Topk
     if (p.prefetch_base) bulk_prefetch_l2(p.prefetch_base + ((int64_t)row * p.N + j) * p.prefetch_row_bytes,
                                           (uint32_t)p.prefetch_row_bytes);
   });
+}
+
+__global__ void __launch_bounds__(kTopkSelectThreads, 2) topk_select_kernel(TopkLargeParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
+  extern __shared__ uint32_t bm_sel[];               // [words] taken, then [words] ties
+  __shared__ uint32_t sh[1024];
+  __shared__ int warp_buf[72];
+  __shared__ uint32_t sh_digit, sh_need, sh_base_t, sh_base_c;
+  __shared__ int sh_last;
+  const int row = blockIdx.x / p.slices, slice = blockIdx.x % p.slices;
+  const int v = topk_visible(p, row);
+  int* out = p.idx + (int64_t)row * p.k;
+  if (v <= p.k) {
+    if (slice == 0)
+      for (int j = threadIdx.x; j < p.k; j += blockDim.x) out[j] = j < v ? j : -1;
+    return;
+  }
+  uint32_t* cnt = p.counters + (int64_t)row * kTopkCounters;
+  int* above = p.above + (int64_t)row * p.k;
+  uint2* cand = p.cand + (int64_t)row * p.N;
+  {
+    uint32_t n_above_T;
+    int T;
+    if (p.thresh_ready) {
+      T = (int)__ldcg(&cnt[kCntT]);
+      n_above_T = __ldcg(&cnt[kCntAboveT]);
+    } else {
+      T = threshold_bin(p.hist + (int64_t)row * kHistBins, p.k, sh, &n_above_T);
+    }
+    const int per = (v + p.slices - 1) / p.slices;
+    const int j0 = slice * per, j1 = min(v, j0 + per);
+    const float* s = p.scores + (int64_t)row * p.row_stride;
+    // 8 keys per thread per round; the CTA reserves its ranges of the row's
+    // taken / candidate lists with one atomic each (a block prefix sum places
+    // every thread's entries), so the row counters see one atomic per CTA
+    constexpr int kPer = 8;
+    for (int base = j0; base < j1; base += kPer * (int)blockDim.x) {
+      uint32_t key[kPer];
+      int nt = 0, nc = 0;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int j = base + u * (int)blockDim.x + (int)threadIdx.x;
+        key[u] = j < j1 ? order_key(__ldcg(s + j)) : 0u;
+        const int bin = (int)(key[u] >> kHistShift);
+        nt += (j < j1 && bin > T);
+        nc += (j < j1 && bin == T);
+      }
+      int tot;
+      const int off = block_excl_count(nt | (nc << 16), warp_buf, &tot);
+      if (threadIdx.x == 0) {
+        sh_base_t = atomicAdd(&cnt[kCntAbove], (uint32_t)(tot & 0xFFFF));
+        sh_base_c = atomicAdd(&cnt[kCntCand], (uint32_t)(tot >> 16));
+      }
+      __syncthreads();
+      uint32_t pt = sh_base_t + (uint32_t)(off & 0xFFFF), pc = sh_base_c + (uint32_t)(off >> 16);
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int j = base + u * (int)blockDim.x + (int)threadIdx.x;
+        const int bin = (int)(key[u] >> kHistShift);
+        if (j < j1 && bin > T) {
+          if (pt < (uint32_t)p.k) above[pt] = j;
+          ++pt;
+        } else if (j < j1 && bin == T) {
+          if (pc < (uint32_t)p.N) cand[pc] = make_uint2(key[u], (uint32_t)j);
+          ++pc;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // publish this slice, then let the last CTA of the row finish it
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) sh_last = atomicAdd(&cnt[kCntSlices], 1u) == (uint32_t)(p.slices - 1);
+  __syncthreads();
+  if (!sh_last) return;
+  topk_finish_row(p, row, v, out, cnt, above, cand, bm_sel, warp_buf, &sh_digit, &sh_need);
+}
+
+// The finish alone, one CTA per row, after a kernel that has routed every
+// key of the row into its taken and candidate lists (the FP8 decode indexer
+// does so in its epilogue, with the scores still on chip).
+__global__ void __launch_bounds__(kTopkSelectThreads) topk_finish_kernel(TopkLargeParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
+  extern __shared__ uint32_t bm_sel[];
+  __shared__ int warp_buf[72];
+  __shared__ uint32_t sh_digit, sh_need;
+  const int row = blockIdx.x;
+  const int v = topk_visible(p, row);
+  int* out = p.idx + (int64_t)row * p.k;
+  if (v <= p.k) {
+    for (int j = threadIdx.x; j < p.k; j += blockDim.x) out[j] = j < v ? j : -1;
+    return;
+  }
+  uint32_t* cnt = p.counters + (int64_t)row * kTopkCounters;
+  topk_finish_row(p, row, v, out, cnt, p.above + (int64_t)row * p.k, p.cand + (int64_t)row * p.N, bm_sel,
+                  warp_buf, &sh_digit, &sh_need);
 }
 
 }  // namespace csahca

@@ -1,20 +1,29 @@
-"""One decode_1m layer, repeated, for a profiler to capture.
+"""One decode_1m layer (or one reduced csa_prefill_128k layer), repeated, for
+a profiler to capture.
 
     python -m long_context_compressed_overlapped_b200.profile_case csa --calls 4
     python -m long_context_compressed_overlapped_b200.profile_case hca --calls 4
+    python -m long_context_compressed_overlapped_b200.profile_case csa_fp8kv --calls 4
     python -m long_context_compressed_overlapped_b200.profile_case indexer --calls 4
     python -m long_context_compressed_overlapped_b200.profile_case compress --calls 4
+    python -m long_context_compressed_overlapped_b200.profile_case prefill --calls 2
 
 ``csa``: one CSA decode layer through ``compressed_attn_decode`` (indexer with
 e4m3 keys, top-k select, attention, combine); ``hca``: one HCA decode layer
-(attention, combine); ``indexer``: ``indexer_topk`` on the CSA layer's indexer
+(attention, combine); ``csa_fp8kv`` / ``hca_fp8kv``: the same layers with FP8
+KV cache rows (decode_1m_fp8kv: 640-byte rows of e4m3 codes, bf16 RoPE dims
+and fp32 scales); ``indexer``: ``indexer_topk`` on the CSA layer's indexer
 inputs; ``compress``: ``decode_compress`` of the CSA layer with the new token at
 position 1,048,575, which completes a block (ring store, window row, pooled
 entry and e4m3 indexer key).  Four sequences at a 1,048,576-token context: 262,144 CSA entries
 (1 GB of bf16 rows, 134 MB of e4m3 indexer keys) or 8,192 HCA entries per
 sequence; about 1.3 GB on the device.  Inputs are the seeded synthetic draw of
-the decode_1m workload.  The process exits non-zero if a bounded device wait
-gave up.
+the decode_1m workload.  ``prefill``: the csa_prefill_128k layer's shapes
+(64 heads of 512 dims, 64 indexer heads of 128 dims, top-1,024, window 128)
+at n = 16,384 tokens: both compressors, indexer_topk (the tensor-core
+indexer over 4-query tiles, then the row top-k) and compressed_attn_prefill;
+about 3 GB on the device.  The process exits non-zero if a bounded device
+wait gave up.
 """
 
 import argparse
@@ -28,11 +37,14 @@ from . import api, native, runtime, synth
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("case", choices=("csa", "hca", "indexer", "compress"))
+    ap.add_argument("case", choices=("csa", "hca", "csa_fp8kv", "hca_fp8kv", "indexer", "compress",
+                                        "prefill"))
     ap.add_argument("--calls", type=int, default=4)
     a = ap.parse_args(argv)
-    wl = synth.WORKLOADS["decode_1m"]
-    kind = "hca" if a.case == "hca" else "csa"
+    if a.case == "prefill":
+        return prefill_case(a.calls)
+    wl = synth.WORKLOADS["decode_1m_fp8kv" if a.case.endswith("_fp8kv") else "decode_1m"]
+    kind = "hca" if a.case.startswith("hca") else "csa"
     ctx = wl.ctx - 1 if a.case == "compress" else wl.ctx
     L = synth.decode_inputs(wl, "cuda", ctx=ctx, B=wl.B, layers=(kind,))[0]
     cargs = runtime.compress_args(wl, L) if a.case == "compress" else None
@@ -51,6 +63,25 @@ def main(argv=None) -> int:
     torch.cuda.synchronize()
     err = api.device_error()
     print(f"profile_case {a.case}: {a.calls} calls, device error {err}")
+    return 1 if err else 0
+
+
+def prefill_case(calls: int, n: int = 16384) -> int:
+    wl = synth.WORKLOADS["csa_prefill_128k"]
+    inp = synth.prefill_inputs(wl, "cuda", n=n)
+    kvi, ik = inp["kv"], inp["ik"]
+    q_pos = torch.arange(n, device="cuda", dtype=torch.int32)[None]
+    for _ in range(calls):
+        kv = api.csa_compress(kvi["a"], kvi["b"], kvi["za"], kvi["zb"], kvi["bias_a"], kvi["bias_b"], wl.m,
+                              gain=inp["kv_gain"], rope_dims=wl.r)
+        kI = api.csa_compress(ik["a"], ik["b"], ik["za"], ik["zb"], ik["bias_a"], ik["bias_b"], wl.m,
+                              rms_norm=False)
+        idx = api.indexer_topk(inp["qI"], inp["w"], kI, q_pos, wl.m, wl.k)
+        api.compressed_attn_prefill("csa", inp["q"], kv, inp["kv_win"], inp["sinks"], m=wl.m, w=wl.w,
+                                    rope_dims=wl.r, idx=idx, q_gain=inp["q_gain"], kv_gain=inp["kv_gain"])
+    torch.cuda.synchronize()
+    err = api.device_error()
+    print(f"profile_case prefill (n={n}): {calls} calls, device error {err}")
     return 1 if err else 0
 
 

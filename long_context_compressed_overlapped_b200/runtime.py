@@ -97,6 +97,10 @@ class DecodeStep:
     def __init__(self, wl: synth.Workload, layers, stream: torch.cuda.Stream, keep_idx: bool = False):
         self.lib = native.lib()
         self.stream = stream
+        # the layers' tensors were written on the current stream: the step's
+        # stream is ordered after that work (later writes are the caller's to order)
+        if isinstance(stream, torch.cuda.Stream):
+            stream.wait_stream(torch.cuda.current_stream(stream.device))
         self.calls = []
         self.compress = [compress_args(wl, L) for L in layers]
         self.idx = []                            # per layer: the CSA selection (keep_idx) or None

@@ -16,6 +16,9 @@ regimes"):
   csa_prefill_128k  B=1 n=131072 H=64 d=512 r=64 m=4 H_I=64 d_I=128 k=1024 w=128
   decode_256k       B=8 ctx=262144, one CSA + one HCA layer, bf16 indexer keys
   decode_1m         B=4 ctx=1048576, CSA,HCA,CSA,HCA, e4m3 indexer keys
+  decode_1m_fp8kv   decode_1m with FP8 KV cache rows (e4m3 non-RoPE dims with
+                    one fp32 scale per 64, bf16 RoPE dims; "Paper Breakdown:
+                    DeepSeek-V4", infrastructure table)
 """
 
 from __future__ import annotations
@@ -46,6 +49,7 @@ class Workload:
     layers: tuple = ()    # decode layer schedule, e.g. ("csa", "hca")
     kind: str = "csa"     # prefill layer kind
     fp8_keys: bool = False
+    fp8_kv: bool = False  # decode caches as FP8 KV rows
 
     @property
     def torch_dtype(self):
@@ -66,6 +70,9 @@ WORKLOADS = {
     "decode_1m": Workload("decode_1m", "bf16", B=4, ctx=1048576, H=64, d=512, r=64, m=4,
                           m_hca=128, HI=64, dI=128, k=1024, w=128, seed=4,
                           layers=("csa", "hca", "csa", "hca"), fp8_keys=True),
+    "decode_1m_fp8kv": Workload("decode_1m_fp8kv", "bf16", B=4, ctx=1048576, H=64, d=512, r=64, m=4,
+                                m_hca=128, HI=64, dI=128, k=1024, w=128, seed=4,
+                                layers=("csa", "hca", "csa", "hca"), fp8_keys=True, fp8_kv=True),
 }
 
 
@@ -118,6 +125,41 @@ def quantize_e4m3_rows(x: torch.Tensor, block: int = 128):
     q = (xb / scale[..., None]).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
     codes = q.view(torch.uint8).reshape(x.shape)
     return codes.contiguous(), scale.contiguous()
+
+
+def kv_fp8_row_bytes(d: int, r: int) -> int:
+    """Bytes of an FP8 KV row (the library's layout, include/csahca.h): d - r
+    e4m3 codes, r bf16 RoPE dims, (d - r) / 64 fp32 scales, padded to a
+    multiple of 128."""
+    raw = (d - r) + 2 * r + 4 * ((d - r) // 64)
+    return (raw + 127) // 128 * 128
+
+
+def pack_kv_rows_fp8(x: torch.Tensor, r: int, block: int = 64) -> torch.Tensor:
+    """FP8 KV storage of rows x [..., d]: the first d - r dims as e4m3 codes
+    with one fp32 scale per `block` of them (quantize_e4m3_rows' rule), the
+    last r dims as bf16, then the scales and zero padding.  Returns uint8
+    [..., kv_fp8_row_bytes(d, r)]."""
+    d = x.shape[-1]
+    nr = d - r
+    codes, scales = quantize_e4m3_rows(x[..., :nr], block)
+    rope = x[..., nr:].to(torch.bfloat16).contiguous().view(torch.uint8)
+    sc = scales.to(torch.float32).contiguous().view(torch.uint8)
+    row = torch.cat([codes, rope, sc], dim=-1)
+    pad = kv_fp8_row_bytes(d, r) - row.shape[-1]
+    if pad:
+        row = torch.cat([row, torch.zeros(*row.shape[:-1], pad, dtype=torch.uint8, device=row.device)], dim=-1)
+    return row.contiguous()
+
+
+def unpack_kv_rows_fp8(packed: torch.Tensor, d: int, r: int, block: int = 64):
+    """The fields of FP8 KV rows: (codes uint8 [..., d-r], scales f32
+    [..., (d-r)/block], rope bf16 [..., r])."""
+    nr = d - r
+    codes = packed[..., :nr]
+    rope = packed[..., nr:nr + 2 * r].contiguous().view(torch.bfloat16)
+    scales = packed[..., nr + 2 * r:nr + 2 * r + 4 * (nr // block)].contiguous().view(torch.float32)
+    return codes, scales, rope
 
 
 # ----------------------------------------------------------------------------
@@ -207,7 +249,8 @@ def decode_inputs(wl: Workload, device="cpu", ctx: int | None = None, B: int | N
         L = {
             "kind": kind, "m": m,
             "pos": torch.full((B,), ctx, dtype=torch.int32, device=device),
-            "kv": D.normal(f"{t}/kv", (B, N, wl.d), 1.0, dt),
+            "kv": (pack_kv_rows_fp8(D.normal(f"{t}/kv", (B, N, wl.d), 1.0, dt), wl.r) if wl.fp8_kv
+                   else D.normal(f"{t}/kv", (B, N, wl.d), 1.0, dt)),
             "win": D.normal(f"{t}/win", (B, wl.w, wl.d), 1.0, dt),
             "q": D.normal(f"{t}/q", (B, wl.H, wl.d), 1.0, dt),
             "sinks": D.normal(f"{t}/sinks", (wl.H,), 1.0, torch.float32),

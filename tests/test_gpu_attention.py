@@ -207,3 +207,23 @@ def test_prefill_csa_128k_full_size_sampled():
     ref = _oracle_rows("csa", inp, kv, idx, wl, m, 0, rows)
     check_close(npy(out[0, rows]), ref, "bf16", "csa prefill 128k")
     assert api.device_error() == 0
+
+
+@pytest.mark.parametrize("n,w,m", [(8192 + 3, 128, 128), (1000, 64, 128), (261, 5, 16), (130, 128, 32)])
+def test_prefill_hca_16_heads_128_dims_tensor_cores(n, w, m):
+    """The 16-head / 128-dim HCA shape (hca_8k_bf16's heads) on the tensor
+    cores: four queries per work item, so ragged tails (n not a multiple of
+    4), blocks whose last query sees one more entry than the first, windows
+    shorter than the block span and non-unit gains are all covered."""
+    wl = synth.Workload(**{**synth.WORKLOADS["hca_8k_bf16"].__dict__, "w": w, "m_hca": m})
+    inp, kv, _ = _prefill_layer(wl, n, 2)
+    inp["q_gain"] = _gain("q_gain16", wl.d, 23)
+    out = api.compressed_attn_prefill("hca", inp["q"], kv, inp["kv_win"], inp["sinks"], m=m,
+                                      w=wl.w, rope_dims=wl.r, q_gain=inp["q_gain"],
+                                      kv_gain=inp["kv_gain"])
+    for b in range(2):
+        rows = _sample(n, [0, 1, 2, 3, m - 2, m - 1, m, 4 * (m // 4) + 3, n - 4, n - 3, n - 2, n - 1],
+                       seed=40 + b, count=16)
+        ref = _oracle_rows("hca", inp, kv, None, wl, m, b, rows)
+        check_close(npy(out[b, rows]), ref, "bf16", f"hca16 n={n} w={w} m={m} b={b}")
+    assert api.device_error() == 0

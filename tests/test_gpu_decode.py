@@ -159,3 +159,54 @@ def test_decode_256k_full_size_all_sequences():
         out = _decode_layer(L, wl, idx_out=idx)
         _check_layer(L, wl, out, idx, range(wl.B))
     assert api.device_error() == 0
+
+
+def _fp8_kv_rows(L, wl, b):
+    """The rows an FP8 KV cache of layer L stands for (sequence b), float64."""
+    return O.dequant_kv_rows_fp8(*(npy(t) for t in synth.unpack_kv_rows_fp8(L["kv"][b], wl.d, wl.r)))
+
+
+@pytest.mark.parametrize("ctx,B", [(32768 + 130, 2), (4096, 4)])
+def test_decode_fp8_kv_layers(ctx, B):
+    """decode_1m with FP8 KV cache rows (e4m3 non-RoPE dims with one fp32
+    scale per 64, bf16 RoPE dims), CSA and HCA layers: the attention reads the
+    rows the cache stands for (the oracle dequantises them); gathered (CSA)
+    and contiguous (HCA) rows, a ragged block tail and partial windows."""
+    wl = synth.WORKLOADS["decode_1m_fp8kv"]
+    layers = synth.decode_inputs(wl, DEV, ctx=ctx, B=B, layers=("csa", "hca"))
+    for L in layers:
+        assert L["kv"].dtype == torch.uint8
+        L["pos"] = torch.tensor([ctx, ctx - 200, 100, 7][:B], device=DEV, dtype=torch.int32)
+        idx = torch.empty(B, wl.k, dtype=torch.int32, device=DEV) if L["kind"] == "csa" else None
+        out = _decode_layer(L, wl, idx_out=idx)
+        for b in range(B):
+            pos = int(L["pos"][b])
+            sel = None
+            if L["kind"] == "csa":
+                v = min(O.n_visible(pos, L["m"]), L["kv"].shape[1])
+                K = O.dequant_e4m3_rows(npy(L["kI"][b, :v]), npy(L["kI_scale"][b, :v]))
+                check_topk(npy(idx[b]), O.indexer_scores(npy(L["qI"][b]), npy(L["w"][b]), K), wl.k,
+                           f"fp8kv b={b}")
+                sel = npy(idx[b])
+            ref = O.decode_attention(L["kind"], npy(L["q"][b]), pos, _fp8_kv_rows(L, wl, b), npy(L["win"][b]),
+                                     npy(L["sinks"]), m=L["m"], w=wl.w, r=wl.r, q_gain=npy(L["q_gain"]),
+                                     sel=sel)
+            check_close(npy(out[b]), ref, "bf16", f"fp8kv {L['kind']} b={b} pos={pos}")
+    assert api.device_error() == 0
+
+
+@pytest.mark.slow
+def test_decode_fp8_kv_full_size():
+    """decode_1m_fp8kv at the full 1,048,576-token context, all four layers,
+    sequence 0 checked."""
+    wl = synth.WORKLOADS["decode_1m_fp8kv"]
+    layers = synth.decode_inputs(wl, DEV)
+    for L in layers:
+        idx = torch.empty(wl.B, wl.k, dtype=torch.int32, device=DEV) if L["kind"] == "csa" else None
+        out = _decode_layer(L, wl, idx_out=idx)
+        pos = int(L["pos"][0])
+        sel = npy(idx[0]) if idx is not None else None
+        ref = O.decode_attention(L["kind"], npy(L["q"][0]), pos, _fp8_kv_rows(L, wl, 0), npy(L["win"][0]),
+                                 npy(L["sinks"]), m=L["m"], w=wl.w, r=wl.r, q_gain=npy(L["q_gain"]), sel=sel)
+        check_close(npy(out[0]), ref, "bf16", f"fp8kv full {L['kind']}")
+    assert api.device_error() == 0

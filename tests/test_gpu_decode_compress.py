@@ -170,13 +170,74 @@ def test_decode_compress_decode_1m_shapes():
     assert api.device_error() == 0
 
 
-def _check_bench_step(ctx, B, seqs):
+def _check_fp8_kv_row(packed, finished, r, what):
+    """An FP8 KV row written by decode_compress against the oracle's quantiser
+    of the finished entry: RoPE dims within the bf16 tolerance, block scales
+    amax / 448 to 1e-5 relative, and each code a nearest e4m3 of x / scale (a
+    neighbour only where the two are equally near within the fp32 error of
+    the pooling; at least 99 % identical)."""
+    d = finished.shape[-1]
+    codes, scales, rope = synth.unpack_kv_rows_fp8(packed, d, r)
+    oc, osc, orope = O.quantize_kv_rows_fp8(finished, r)
+    check_close(npy(rope), orope, "bf16", what + " rope dims")
+    x = finished[: d - r]
+    amax = np.abs(x.reshape(-1, 64)).max(axis=1)
+    np.testing.assert_allclose(npy(scales), amax / 448.0, rtol=1e-5, err_msg=what)
+    xs = x / np.repeat(npy(scales), 64)
+    got = npy(codes)
+    d_got = np.abs(O.e4m3_decode(got) - xs)
+    d_want = np.abs(O.e4m3_decode(O.e4m3_encode(xs)) - xs)
+    assert (d_got <= d_want + 1e-4 * np.maximum(np.abs(xs), 1e-3)).all(), what
+    assert (got == oc).mean() >= 0.99, what
+
+
+def test_decode_compress_fp8_kv_rows():
+    """decode_compress into FP8 KV caches (decode_1m_fp8kv shapes): CSA and
+    HCA layers at positions that complete a block (near 2^20, the first block,
+    block N-2) and one that completes none; the new entry is stored as an FP8
+    KV row and its neighbours are untouched."""
+    wl = synth.WORKLOADS["decode_1m_fp8kv"]
+    ctx = (1 << 20) - 1
+    layers = synth.decode_inputs(wl, DEV, ctx=ctx, layers=("csa", "hca"))
+    for L in layers:
+        m = L["m"]
+        L["pos"] = torch.tensor([ctx, ctx - 1, m - 1, ctx - m], dtype=torch.int32, device=DEV)
+        host = {k_: (v.cpu().clone() if isinstance(v, torch.Tensor) else v) for k_, v in L.items()}
+        args, keep = runtime.compress_args(wl, L)
+        native.check(native.lib().decode_compress(C.byref(args), torch.cuda.current_stream().cuda_stream),
+                     "decode_compress")
+        torch.cuda.synchronize()
+        csa = L["kind"] == "csa"
+        names = NAMES[L["kind"]]
+        cols = ("ca", "cb", "cza", "czb") if csa else ("ca", "cza")
+        for b in range(wl.B):
+            pos = int(host["pos"][b])
+            ring = {s_: npy(host["ring"][b, :, j]) for j, s_ in enumerate(names)}
+            new = {s_: npy(host[c_][b]) for s_, c_ in zip(names, cols)}
+            biases = (npy(host["bias_a"]), npy(host["bias_b"]) if csa else None)
+            _, entry, _ = O.decode_compress_step(L["kind"], pos, new, ring, biases, m,
+                                                 kv_raw=npy(host["kv_raw"][b]), gain=npy(host["kv_gain"]), r=wl.r)
+            what = f"fp8kv {L['kind']} b={b} pos={pos}"
+            if entry is not None:
+                i = entry[0]
+                _check_fp8_kv_row(L["kv"][b, i].cpu(), entry[2], wl.r, what)
+                lo = max(i - 2, 0)
+                assert torch.equal(L["kv"][b, lo:i].cpu(), host["kv"][b, lo:i]), what + " neighbours"
+            else:
+                i = (pos + 1) // m
+                assert torch.equal(L["kv"][b, max(i - 2, 0):i + 1].cpu(),
+                                   host["kv"][b, max(i - 2, 0):i + 1]), what + " untouched"
+        del keep
+    assert api.device_error() == 0
+
+
+def _check_bench_step(ctx, B, seqs, workload="decode_1m"):
     """The step bench.py times (per layer decode_compress then
     compressed_attn_decode, CSA, HCA, CSA, HCA, replayed as a CUDA graph)
     against the oracle's decode step for the sequences `seqs`.  Selections
     must pass the top-k tolerance and outputs are compared on the GPU's
     selections."""
-    wl = synth.WORKLOADS["decode_1m"]
+    wl = synth.WORKLOADS[workload]
     layers = synth.decode_inputs(wl, DEV, ctx=ctx, B=B)
     host = bench.host_layers(layers)
     stream = torch.cuda.Stream()
@@ -204,6 +265,12 @@ def test_bench_decode_step_with_compressors():
     """At a 32,767-token context, where the new token completes a CSA and an
     HCA block; both sequences checked."""
     _check_bench_step((1 << 15) - 1, 2, range(2))
+
+
+def test_bench_decode_step_fp8_kv():
+    """The bench's step with FP8 KV caches at a 32,767-token context (the new
+    token completes a CSA and an HCA block, stored as FP8 KV rows)."""
+    _check_bench_step((1 << 15) - 1, 2, range(2), workload="decode_1m_fp8kv")
 
 
 @pytest.mark.slow
