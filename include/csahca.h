@@ -273,14 +273,14 @@ int64_t csahca_kv_row_bytes(int32_t kv_dtype, int32_t d, int32_t rope_dims);
  *   CSAHCA_ERR_UNSUPPORTED.  Any other kv_dtype: rows of `dtype`.
  * Context parallelism (one rank's share of a layer whose compressed cache is
  *   split by entry range across ranks; tensor-core shapes only: BF16, H = 64,
- *   d = 512, rope_dims <= 128, B * N_cap >= 128 and B * w >= 128, else
- *   CSAHCA_ERR_UNSUPPORTED):
+ *   d = 512, rope_dims <= 128, B * N_cap >= 128 and (unless skip_window)
+ *   B * w >= 128, else CSAHCA_ERR_UNSUPPORTED):
  *   entry_base: kv_cache (and kI) hold the global entries entry_base ..
  *     entry_base + N_cap - 1; visibility as in indexer_topk's entry_base.
  *     CSA with entry_base > 0 needs idx_in (LOCAL rows, -1 to skip; as
  *     cp_topk_merge writes them).
  *   skip_window != 0: the window is left out (another rank attends it); win
- *     must still point at a [B, w, d] ring (it is not read).
+ *     is not read and may be NULL.
  *   partial_out != NULL: instead of `out` (which may then be NULL), each row's
  *     unnormalised share of the softmax is written as one block of
  *     2H + H*d floats: mx[H], the largest scaled logit of the head in base-2
@@ -464,7 +464,8 @@ int cp_topk_merge(const csahca_cp_topk_merge_args* args, void* stream);
  * by -pos[row] (RoPE pairs as above, base rope_base).
  * Layout: partials [R, rows, 2H + H*d] f32; sinks [H] f32; pos [rows] int32;
  * out [rows, H, d] (dtype F32 or BF16).  Constraints: 1 <= R <=
- * CSAHCA_CP_MAX_RANKS; d % 4 == 0, d <= 1024; rope_dims even, <= d and <= 128.
+ * CSAHCA_CP_MAX_RANKS; H even; d % 4 == 0, d <= 1024; rope_dims even, <= d
+ * and <= 128.
  * No workspace. */
 typedef struct {
   int32_t dtype;

@@ -75,12 +75,15 @@ def hca_compress(a, za, bias_a, m, **kw):
 
 
 def indexer_topk(qI, w, kI, q_pos, m, k, *, kI_scale=None, idx=None, scores_out=None,
-                 stream=None):
+                 sel_scores=None, entry_base=0, stream=None):
     """Lightning-indexer scores over the visible compressed keys and the
     per-query top-k (ties to the lower index), sorted ascending, -1 padded.
 
     qI [B, nq, HI, dI]; w [B, nq, HI] f32; kI [B, N, dI] (f32/bf16, or uint8
-    e4m3 codes with kI_scale [B, N, dI/128]); q_pos [B, nq] int32."""
+    e4m3 codes with kI_scale [B, N, dI/128]); q_pos [B, nq] int32.
+    Context parallelism: kI holds the global entries entry_base ..
+    entry_base + N - 1 (idx then holds local rows), and sel_scores
+    [B, nq, k] f32 receives the score of each selected row."""
     B, nq, HI, dI = qI.shape
     Nk = kI.shape[1]
     if idx is None:
@@ -90,7 +93,8 @@ def indexer_topk(qI, w, kI, q_pos, m, k, *, kI_scale=None, idx=None, scores_out=
     args = N.IndexerArgs(q_dtype=_dt(qI), k_dtype=_dt(kI), B=B, nq=nq, HI=HI, dI=dI, N=Nk, m=m,
                          k=k, qI=_ptr(qI), w=_ptr(w), kI=_ptr(kI),
                          kI_scale=_ptr(_f32(kI_scale)), q_pos=_ptr(q_pos), idx=_ptr(idx),
-                         scores_out=_ptr(scores_out))
+                         scores_out=_ptr(scores_out), sel_scores=_ptr(sel_scores),
+                         entry_base=int(entry_base))
     L = N.lib()
     ws_bytes = L.csahca_indexer_workspace_size(C.byref(args))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=qI.device) if ws_bytes else None
@@ -130,7 +134,8 @@ def compressed_attn_prefill(kind, q, kv_comp, kv_win, sinks, *, m, w, rope_dims,
 
 def decode_args(kind, q, pos, kv_cache, win, sinks, *, m, rope_dims, k=0, qI=None, wI=None,
                 kI=None, kI_scale=None, idx_in=None, idx_out=None, q_gain=None, q_norm=True,
-                rope_base=10000.0, eps=1e-6, scale=0.0, out=None):
+                rope_base=10000.0, eps=1e-6, scale=0.0, out=None, entry_base=0, partial_out=None,
+                skip_window=False):
     """Build the DecodeArgs struct (and keep the tensors it points to alive in
     the returned list)."""
     B, H, d = q.shape
@@ -143,7 +148,7 @@ def decode_args(kind, q, pos, kv_cache, win, sinks, *, m, rope_dims, k=0, qI=Non
 
     pos = pos.to(torch.int32).contiguous()
     keep.append(pos)
-    if out is None:
+    if out is None and partial_out is None:
         out = torch.empty_like(q)
     HI = dI = 0
     qI_dt = kI_dt = 0
@@ -161,21 +166,28 @@ def decode_args(kind, q, pos, kv_cache, win, sinks, *, m, rope_dims, k=0, qI=Non
                         kI_dtype=kI_dt, q=_ptr(q), pos=_ptr(pos), q_gain=_ptr(f(q_gain)),
                         kv_cache=_ptr(kv_cache), win=_ptr(win), sinks=_ptr(f(sinks)),
                         qI=_ptr(qI), wI=_ptr(f(wI)), kI=_ptr(kI), kI_scale=_ptr(f(kI_scale)),
-                        idx_in=_ptr(idx_in), idx_out=_ptr(idx_out), out=_ptr(out))
+                        idx_in=_ptr(idx_in), idx_out=_ptr(idx_out), out=_ptr(out),
+                        entry_base=int(entry_base), partial_out=_ptr(partial_out),
+                        skip_window=int(bool(skip_window)))
     return args, out, keep
 
 
 def compressed_attn_decode(kind, q, pos, kv_cache, win, sinks, *, m, rope_dims, k=0, qI=None,
                            wI=None, kI=None, kI_scale=None, idx_in=None, idx_out=None,
                            q_gain=None, q_norm=True, rope_base=10000.0, eps=1e-6, scale=0.0,
-                           out=None, workspace=None, stream=None):
+                           out=None, entry_base=0, partial_out=None, skip_window=False,
+                           workspace=None, stream=None):
     """One decode step of one CSA or HCA layer for B sequences (one new query
     each at pos[b]); CSA selects with the lightning indexer unless idx_in is
-    given.  Returns out [B, H, d]."""
+    given.  Returns out [B, H, d], or partial_out [B, 2H + H*d] f32 (this
+    rank's share of a context-parallel layer whose cache shard starts at
+    global entry entry_base) when that is given."""
     args, out, keep = decode_args(kind, q, pos, kv_cache, win, sinks, m=m, rope_dims=rope_dims,
                                   k=k, qI=qI, wI=wI, kI=kI, kI_scale=kI_scale, idx_in=idx_in,
                                   idx_out=idx_out, q_gain=q_gain, q_norm=q_norm,
-                                  rope_base=rope_base, eps=eps, scale=scale, out=out)
+                                  rope_base=rope_base, eps=eps, scale=scale, out=out,
+                                  entry_base=entry_base, partial_out=partial_out,
+                                  skip_window=skip_window)
     L = N.lib()
     ws_bytes = L.csahca_decode_workspace_size(C.byref(args))
     if workspace is None or workspace.numel() < ws_bytes:
@@ -184,13 +196,13 @@ def compressed_attn_decode(kind, q, pos, kv_cache, win, sinks, *, m, rope_dims, 
     args.workspace_bytes = workspace.numel()
     N.check(L.compressed_attn_decode(C.byref(args), _stream(stream)), "compressed_attn_decode")
     del keep
-    return out
+    return out if partial_out is None else partial_out
 
 
 def decode_compress_args(kind, pos, streams, ring, kv_cache, *, m, bias_a, bias_b=None, kv_raw=None,
                          win=None, kv_gain=None, kv_norm=True, rope_dims=0, rope_base=10000.0,
                          eps=1e-6, istreams=None, ibias_a=None, ibias_b=None, iring=None, kI=None,
-                         kI_scale=None):
+                         kI_scale=None, entry_base=0):
     """Build the DecodeCompressArgs struct (and the list of tensors it points to).
 
     streams: (a, b, za, zb) for "csa" or (a, za) for "hca", each [B, d];
@@ -219,7 +231,7 @@ def decode_compress_args(kind, pos, streams, ring, kv_cache, *, m, bias_a, bias_
         kind=N.CSA if csa else N.HCA, dtype=_dt(a), B=B, d=d, m=m, N_cap=kv_cache.shape[1],
         w=win.shape[1] if win is not None else 0, rope_dims=rope_dims, rope_base=rope_base, eps=eps,
         kv_norm=int(bool(kv_norm)), dI=dI, kI_dtype=_dt(kI) if dI else 0,
-        kv_dtype=N.E4M3 if kv_cache.dtype == torch.uint8 else _dt(a),
+        kv_dtype=N.E4M3 if kv_cache.dtype == torch.uint8 else _dt(a), entry_base=int(entry_base),
         pos=_ptr(pos), kv_raw=_ptr(kv_raw), a=_ptr(a), b=_ptr(b), za=_ptr(za), zb=_ptr(zb),
         bias_a=_ptr(f(bias_a)), bias_b=_ptr(f(bias_b)), kv_gain=_ptr(f(kv_gain)), ring=_ptr(ring),
         kv_cache=_ptr(kv_cache), win=_ptr(win), ia=_ptr(ia), ib=_ptr(ib), iza=_ptr(iza), izb=_ptr(izb),
@@ -236,6 +248,48 @@ def decode_compress(kind, pos, streams, ring, kv_cache, *, m, bias_a, stream=Non
     args, keep = decode_compress_args(kind, pos, streams, ring, kv_cache, m=m, bias_a=bias_a, **kw)
     N.check(N.lib().decode_compress(C.byref(args), _stream(stream)), "decode_compress")
     del keep
+
+
+def cp_partial_floats(H: int, d: int) -> int:
+    """Floats of one row's context-parallel attention share: mx[H], l[H], o[H][d]."""
+    return 2 * H + H * d
+
+
+def cp_topk_merge(cand_idx, cand_scores, bases, rank, *, idx_global=None, idx_local=None, stream=None):
+    """Stage 1 of context parallelism: the global top-k from every rank's
+    candidates.  cand_idx / cand_scores [R, rows, k] (local rows and their
+    scores, as indexer_topk writes idx / sel_scores); bases: the R shards'
+    first global entries (host ints).  Returns (idx_global, idx_local), each
+    [rows, k] int32 in ascending global order, -1 padded; idx_local holds the
+    rows of rank `rank` and -1 for the other ranks' entries."""
+    R, rows, k = cand_idx.shape
+    dev = cand_idx.device
+    if idx_global is None:
+        idx_global = torch.empty(rows, k, dtype=torch.int32, device=dev)
+    if idx_local is None:
+        idx_local = torch.empty(rows, k, dtype=torch.int32, device=dev)
+    b = (C.c_int32 * R)(*[int(x) for x in bases])
+    args = N.CpTopkMergeArgs(R=R, rows=rows, k=k, rank=int(rank), bases=C.cast(b, C.c_void_p),
+                             cand_idx=_ptr(cand_idx), cand_scores=_ptr(cand_scores),
+                             idx_global=_ptr(idx_global), idx_local=_ptr(idx_local))
+    N.check(N.lib().cp_topk_merge(C.byref(args), _stream(stream)), "cp_topk_merge")
+    return idx_global, idx_local
+
+
+def cp_attn_merge(partials, sinks, pos, *, H, d, rope_dims, dtype=torch.bfloat16, rope_base=10000.0,
+                  out=None, stream=None):
+    """Stage 2 of context parallelism: the layer output [rows, H, d] from the
+    ranks' shares partials [R, rows, 2H + H*d] f32, with the sink and the
+    output de-rotation by -pos."""
+    R, rows, _ = partials.shape
+    if out is None:
+        out = torch.empty(rows, H, d, dtype=dtype, device=partials.device)
+    keep = _f32(sinks)
+    pos = pos.to(torch.int32).contiguous()
+    args = N.CpMergeArgs(dtype=_dt(out), R=R, rows=rows, H=H, d=d, rope_dims=rope_dims, rope_base=rope_base,
+                         partials=_ptr(partials), sinks=_ptr(keep), pos=_ptr(pos), out=_ptr(out))
+    N.check(N.lib().cp_attn_merge(C.byref(args), _stream(stream)), "cp_attn_merge")
+    return out
 
 
 def device_error(stream=None) -> int:

@@ -1213,7 +1213,9 @@ int run_cp_attn_merge(const csahca_cp_merge_args* a, void* stream) {
   if (a->dtype != CSAHCA_F32 && a->dtype != CSAHCA_BF16) return CSAHCA_ERR_INVALID_ARG;
   if (a->R < 1 || a->rows < 0 || a->H < 1 || a->d < 1) return CSAHCA_ERR_INVALID_ARG;
   if (a->rope_dims < 0 || a->rope_dims > a->d || (a->rope_dims & 1)) return CSAHCA_ERR_INVALID_ARG;
-  if (a->R > kCpMaxRanks || a->d % 4 || a->d > 1024 || a->rope_dims > 128) return CSAHCA_ERR_UNSUPPORTED;
+  // (H even and d % 4 == 0 keep every row's o[h] 16-byte aligned for float4 loads)
+  if (a->R > kCpMaxRanks || a->H % 2 || a->d % 4 || a->d > 1024 || a->rope_dims > 128)
+    return CSAHCA_ERR_UNSUPPORTED;
   if ((int64_t)a->rows * a->H > INT32_MAX) return CSAHCA_ERR_UNSUPPORTED;
   if (a->rows == 0) return CSAHCA_OK;
   if (!a->partials || !a->sinks || !a->pos || !a->out) return CSAHCA_ERR_INVALID_ARG;

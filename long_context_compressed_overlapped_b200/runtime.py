@@ -72,9 +72,9 @@ class StepIO:
             L["out"] = view(self.out, o, t.dtype, tuple(t.shape))
 
 
-def compress_args(wl: synth.Workload, L):
+def compress_args(wl: synth.Workload, L, entry_base: int = 0):
     """DecodeCompressArgs of one layer of synth.decode_inputs (and the tensors
-    it points to)."""
+    it points to); entry_base: the first global entry of L's cache shard."""
     csa = L["kind"] == "csa"
     streams = tuple(L[n] for n in (("ca", "cb", "cza", "czb") if csa else ("ca", "cza")))
     kw = {}
@@ -83,7 +83,8 @@ def compress_args(wl: synth.Workload, L):
                   ibias_b=L["ibias_b"], iring=L["iring"], kI=L["kI"], kI_scale=L["kI_scale"])
     return api.decode_compress_args(L["kind"], L["pos"], streams, L["ring"], L["kv"], m=L["m"],
                                     bias_a=L["bias_a"], bias_b=L["bias_b"], kv_raw=L["kv_raw"],
-                                    win=L["win"], kv_gain=L["kv_gain"], rope_dims=wl.r, **kw)
+                                    win=L["win"], kv_gain=L["kv_gain"], rope_dims=wl.r, entry_base=entry_base,
+                                    **kw)
 
 
 class DecodeStep:
