@@ -34,11 +34,21 @@
 namespace csahca {
 
 // Warps 0-7 softmax (two head groups), then the producer warps, then the S
-// and P.V MMA issuers.  Decode: 2 producers (384 threads); prefill: 6 (512
-// threads), since a gather of selected rows runs at about 8 B/cycle per
-// issuing warp.
-template <bool kDecode> __host__ __device__ constexpr int attn_producers() { return kDecode ? 2 : 6; }
-template <bool kDecode> __host__ __device__ constexpr int attn_threads() { return 32 * (10 + attn_producers<kDecode>()); }
+// and P.V MMA issuers.  Decode: 2 producers (384 threads).  Prefill: 16
+// producers (896 threads, the last two warps idle): a gather of selected rows
+// from L2 runs at a few B/cycle per issuing warp and the prefill attention is
+// bound by it.  Its registers are split per warpgroup (setmaxnreg, one role per
+// warpgroup, launched at 72 a thread): softmax warpgroups 0-1, producer
+// warpgroups 2-5, and warpgroup 6 (the two MMA issuers and two idle warps).
+template <bool kDecode> __host__ __device__ constexpr int attn_producers() { return kDecode ? 2 : 16; }
+template <bool kDecode> __host__ __device__ constexpr int attn_threads() { return kDecode ? 32 * 12 : 32 * 28; }
+constexpr int kAttnRegsSoftmax = 128;   // prefill: warps 0-7
+constexpr int kAttnRegsProducer = 48;   // prefill: warps 8-23
+constexpr int kAttnRegsMma = 56;        // prefill: warps 24-27
+__host__ __device__ constexpr int attn_prefill_regs_needed() {
+  return 256 * kAttnRegsSoftmax + 512 * kAttnRegsProducer + 128 * kAttnRegsMma;
+}
+static_assert(attn_prefill_regs_needed() <= 72 * 896, "the prefill register split fits a 72-register launch");
 constexpr int kAttnH = 64;          // heads (MMA N of both products)
 constexpr int kAttnD = 512;         // head dim
 constexpr int kAttnChunks = kAttnD / 64;
@@ -289,7 +299,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
   __shared__ float rope_cs[64], rope_sn[64];
   __shared__ double theta_s[64];                   // RoPE frequency of pair j
   __shared__ __align__(16) float gain_s[kAttnD];
-  __shared__ int rows_s[attn_producers<kDecode>()][128];
+  __shared__ int rows_s[kDecode ? attn_producers<kDecode>() : 1][128];   // decode: each producer's rows
   __shared__ int need_rescale[2];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -342,18 +352,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     griddep_wait();
     griddep_launch_dependents();
   }
+  static_assert(kDecode || (kNP % 4 == 0 && kWarpPV < attn_threads<kDecode>() / 32 &&
+                            attn_threads<kDecode>() == 32 * (8 + kNP + 4)),
+                "prefill: whole warpgroups per role (softmax, producers, MMA issuers)");
 
   // (the decode instance keeps this exact form of the role test: its code
   // runs once per CTA, fetched cold, and an equivalent range test compiled
   // to a layout measured 4 us slower per launch)
   if (kDecode ? (warp == 8 || warp == 9) : (warp >= 8 && warp < 8 + kNP)) {
+    if constexpr (!kDecode) setmaxnreg_dec<kAttnRegsProducer>();
     // ------------------------------------------------------------ producers
     // decode, two producers: warp 8 loads chunks 0,1,4,5 (and the raw Q),
     // warp 9 chunks 2,3,6,7, and a chunk barrier expects 32 arrivals.
-    // Prefill, six: every producer loads its share of every chunk (gathered
-    // rows: copy instruction j, rows 4j..4j+3, goes to warp j mod 6;
-    // contiguous rows: chunk c's box is issued by warp c mod 6), and a chunk
-    // barrier expects 32 x 6 arrivals; warp 8 also loads the raw Q
+    // Prefill, eighteen: every producer loads its share of every chunk
+    // (gathered rows: copy instruction j, rows 4j..4j+3, goes to warp j mod
+    // 18, which looks its rows up once per tile into registers; contiguous
+    // rows: chunk c's box is issued by warp c mod 18), and a chunk barrier
+    // expects 32 x 18 arrivals; warp 8 also loads the raw Q
     const int pw = warp - 8;
     tma_prefetch_desc(&comp_rows);
     tma_prefetch_desc(&win_rows);
@@ -364,6 +379,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     }
     uint32_t tcount = 0, icount = 0;
     bool stop = false;                       // warp-uniform
+    constexpr int kRowGroups = (32 + kNP - 1) / kNP;   // prefill: 4-row copy groups per warp
+    int rowreg[kRowGroups];
+#pragma unroll
+    for (int jj = 0; jj < kRowGroups; ++jj) rowreg[jj] = 0;
     for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
       const AttnItem it = attn_item<kDecode>(p, id);
       if (it.tile1 <= it.tile0) continue;
@@ -391,14 +410,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
         if (T.src == 0) {
           // selected rows of this tile (clamped; masked later by the softmax)
           const int* L = p.idx + ((int64_t)it.b * p.nq + it.qi) * p.k + T.list_off;
+          if constexpr (kNP == 2) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = lane + 32 * e;
-            int v = (j < T.hi) ? __ldg(L + j) : 0;
-            v = (v < 0 || v >= p.N) ? 0 : v;
-            rows_s[pw][j] = it.b * p.N + v;
+            for (int e = 0; e < 4; ++e) {
+              const int j = lane + 32 * e;
+              int v = (j < T.hi) ? __ldg(L + j) : 0;
+              v = (v < 0 || v >= p.N) ? 0 : v;
+              rows_s[pw][j] = it.b * p.N + v;
+            }
+            __syncwarp();
+          } else {
+            // prefill: this lane's rows, 4j + (lane >> 3) of instructions j = pw + jj * kNP
+#pragma unroll
+            for (int jj = 0; jj < kRowGroups; ++jj) {
+              const int r = 4 * (pw + jj * kNP) + (lane >> 3);
+              int v = (r < T.hi) ? __ldg(L + r) : 0;
+              v = (v < 0 || v >= p.N) ? 0 : v;
+              rowreg[jj] = it.b * p.N + v;
+            }
           }
-          __syncwarp();
         }
         if constexpr (kF8) {
           // FP8 rows: the tile's block scales (32 bytes per row) by warp 8
@@ -494,11 +524,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
               }
             } else {
 #pragma unroll
-              for (int jj = 0; jj < (32 + kNP - 1) / kNP; ++jj) {
+              for (int jj = 0; jj < kRowGroups; ++jj) {
                 const int j = pw + jj * kNP;
                 if (j < nj) {
                   const int r = 4 * j + rg;
-                  cp_async16(dst + sw128_offset(r, piece * 16), src + (int64_t)rows_s[pw][r] * kAttnD);
+                  cp_async16(dst + sw128_offset(r, piece * 16), src + (int64_t)rowreg[jj] * kAttnD);
                 }
               }
             }
@@ -553,7 +583,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     if (lane == 0 && tcount > 0)
       for (int c = 0; c < kAttnChunks; ++c) mbar_wait(&bar_kfull[c], (tcount - 1) & 1, &abort_flag);
     if (pw == 0 && lane == 0 && icount > 0) mbar_wait(&bar_q_raw, (icount - 1) & 1, &abort_flag);
-  } else if (warp == kWarpS) {
+  } else if (warp >= kWarpS) {
+    if constexpr (!kDecode) setmaxnreg_dec<kAttnRegsMma>();
+    if (warp == kWarpS) {
     // ------------------------------------------------------------ S MMA issuer
     // (a separate thread issues the P.V MMAs, so the S MMAs of tile t+1 go out
     // while those of P.V(t) still do)
@@ -589,7 +621,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       umma_commit(&bar_done);
       mbar_wait(&bar_done, 0, &abort_flag);
     }
-  } else if (warp == kWarpPV) {
+    } else if (warp == kWarpPV) {
     // ------------------------------------------------------------ P.V MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_pv = umma_idesc_bf16(128, kAttnH, 1, 1);
@@ -629,7 +661,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
       umma_commit(&bar_done);
       mbar_wait(&bar_done, 0, &abort_flag);
     }
+    }
   } else if (warp < 8) {
+    if constexpr (!kDecode) setmaxnreg_inc<kAttnRegsSoftmax>();
     // ------------------------------------------------------------ softmax / epilogue
     // Two groups of 4 warps; group g owns heads [32g, 32g + 32): its columns
     // of S^T, O^T and the row sums in TMEM, and its 64 bytes of each P^T row.

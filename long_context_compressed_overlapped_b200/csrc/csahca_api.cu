@@ -344,10 +344,8 @@ int launch_topk(const csahca_indexer_args* a, const float* scores, int64_t strid
     tp.scores = scores; tp.row_stride = stride; tp.q_pos = q_pos; tp.idx = idx;
     tp.B = 1; tp.nq = rows; tp.N = a->N; tp.m = a->m; tp.k = a->k;
     tp.q_begin = 0; tp.q_count = rows; tp.entry_base = a->entry_base;
-    const int smem = topk_rows_smem_bytes(a->N > 0 ? a->N : 1);
-    cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     CSAHCA_TRACE("topk_rows", s);
-    launch_k(topk_rows_kernel, dim3(rows), dim3(kTopkThreads), smem, s, tp);
+    launch_k(topk_rows_stream_kernel, dim3(rows), dim3(kTopkStreamThreads), 0, s, tp);
     CSAHCA_CHECK_LAUNCH();
     return CSAHCA_OK;
   }
@@ -775,6 +773,16 @@ int launch_attn_tc(const AttnTcParams& p_in, const void* kv_comp, int64_t comp_r
   // epilogue (a smaller kernel stalls less on instruction fetch)
   auto kern = p.decode ? (f8 ? attn_tc_kernel<true, true> : attn_tc_kernel<true, false>) : attn_tc_kernel<false, false>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (!p.decode) {
+    // the prefill instance moves registers between warpgroups: the counts after
+    // the move must fit the launch allocation, else an increase would wait
+    static int launch_regs = -1;
+    if (launch_regs < 0) {
+      cudaFuncAttributes fa;
+      launch_regs = cudaFuncGetAttributes(&fa, kern) == cudaSuccess ? fa.numRegs : 0;
+    }
+    if ((int64_t)launch_regs * attn_threads<false>() < attn_prefill_regs_needed()) return CSAHCA_ERR_UNSUPPORTED;
+  }
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   if (grid <= 0) return CSAHCA_OK;
   CSAHCA_TRACE(name, s);

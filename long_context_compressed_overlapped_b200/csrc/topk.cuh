@@ -1,56 +1,25 @@
 // Per-query top-k over indexer scores ("Paper Breakdown: DeepSeek-V4",
 // section 4, DSA on Compressed KV: the top-k entries by I_{t,s}).
 //
-// Radix select on order-preserving 32-bit keys: four 8-bit digit passes find
-// the exact key T of the k-th largest score and how many keys equal to T are
-// taken; a last pass in index order takes every key > T and the lowest-index
-// keys == T (ties to the lower index), and block prefix sums place each taken
-// index, so the output comes out sorted ascending with no sort.
-//
-// Rows up to kTopkSmemMaxN long: one CTA per row, the row's keys read from
-// HBM once into shared memory; histograms are spread over 8 sub-histograms
-// (warp % 8) to cut atomic contention; the digit that crosses k is found by
-// one warp with a shuffle scan.
+// Radix select on order-preserving 32-bit keys gives the exact key T of the
+// k-th largest score and how many keys equal to T are taken; a pass in index
+// order then takes every key > T and the lowest-index keys == T (ties to the
+// lower index), placed by prefix counts, so the output comes out sorted
+// ascending with no sort.  This file holds the shared pieces (order key,
+// block prefix counts) and the kernel for rows up to kTopkSmemMaxN keys;
+// longer rows use topk_large.cuh.
 #pragma once
 #include "common.cuh"
 
 namespace csahca {
 
-constexpr int kTopkThreads = 1024;
-constexpr int kTopkSmemMaxN = 32768;        // keys held in shared memory (128 KB)
-constexpr int kTopkSubHist = 8;
+constexpr int kTopkSmemMaxN = 32768;        // rows up to this length: topk_rows_stream_kernel
+                                            // (16-bit candidate indices)
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   if (f == 0.0f) f = 0.0f;                    // -0 and +0 are one value
   uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// Exclusive block scan of 0/1 flags (blockDim.x a multiple of 32, <= 1024);
-// returns the exclusive prefix of this thread and writes the block total to
-// *total.
-__device__ __forceinline__ int block_excl_scan(int flag, int* warp_buf, int* total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  unsigned ballot = __ballot_sync(0xffffffffu, flag);
-  int in_warp = __popc(ballot & ((1u << lane) - 1u));
-  if (lane == 0) warp_buf[wid] = __popc(ballot);
-  __syncthreads();
-  if (wid == 0) {
-    int x = lane < (int)(blockDim.x >> 5) ? warp_buf[lane] : 0;
-    int incl = x;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    warp_buf[32 + lane] = incl - x;
-    if (lane == 31) warp_buf[64] = incl;
-  }
-  __syncthreads();
-  int res = warp_buf[32 + wid] + in_warp;
-  *total = warp_buf[64];
-  __syncthreads();
-  return res;
 }
 
 // Exclusive block prefix sum of per-thread counts (blockDim.x a multiple of
@@ -83,33 +52,6 @@ __device__ __forceinline__ int block_excl_count(int c, int* warp_buf, int* total
   return res;
 }
 
-// Executed by one full warp: hist[0, nb) with nb a multiple of 32 (<= 256).
-// Finds the largest digit d with sum_{e >= d} hist[e] >= need and stores d and
-// need - sum_{e > d} hist[e] (the count still to take inside bin d).
-__device__ __forceinline__ void find_digit_warp(const uint32_t* hist, int nb, uint32_t need,
-                                                uint32_t* out_digit, uint32_t* out_need) {
-  const int lane = threadIdx.x & 31;
-  const int per = nb / 32;
-  const int hi = nb - lane * per;              // this lane's bins: [hi - per, hi), top bins at lane 0
-  uint32_t local = 0;
-  for (int e = 0; e < per; ++e) local += hist[hi - 1 - e];
-  uint32_t incl = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  const uint32_t above = incl - local;
-  if (above < need && incl >= need) {
-    uint32_t cum = above;
-    for (int e = 0; e < per; ++e) {
-      const int b = hi - 1 - e;
-      if (cum + hist[b] >= need) { *out_digit = (uint32_t)b; *out_need = need - cum; break; }
-      cum += hist[b];
-    }
-  }
-}
-
 struct TopkParams {
   const float* scores; int64_t row_stride;     // row r of the chunk
   const int* q_pos;                            // [B, nq]
@@ -119,19 +61,103 @@ struct TopkParams {
   int entry_base;                              // local row j is global entry entry_base + j
 };
 
-// Shared-memory slot of key j: one pad word per 32 keys keeps both the
-// strided (histogram) and the per-thread-segment (output) reads conflict-free.
-__host__ __device__ __forceinline__ int kslot(int j) { return j + (j >> 5); }
-__host__ __device__ __forceinline__ int topk_rows_smem_bytes(int n) { return (kslot(n) + 1) * 4; }
+// ---- rows up to kTopkSmemMaxN ---------------------------------------------------
+// One CTA of 256 threads per row and ~21 KB of shared memory (the row itself
+// is not held there), so several rows run per SM and the reads of one hide
+// the latency of another; a first version holding each row in shared memory
+// (128 KB, one row per SM) took 13.0 ms over csa_prefill_128k's score rows
+// against 10.3 ms for this one.
+//   pass 1 (the row from HBM): histogram of the order keys' bits 31..21 ->
+//     the bin B of the k-th largest key;
+//   pass 2 (from L2): each warp walks its own contiguous range of the row,
+//     counting the keys in bins above B and appending the keys in B (with
+//     their indices) to a candidate list in shared memory;
+//   the exact key T of the k-th largest and the number of keys equal to T to
+//     take follow from two histograms over the candidates (bits 20..10, then
+//     9..0), and so do each warp's counts of keys > T and == T;
+//   output pass (from L2): the same walk places every key > T and the
+//     lowest-index keys == T by warp ballots, so the output is in index order.
+// When bin B holds more keys than the list, the two digits come from passes
+// over the row instead and a counting pass precedes the output pass.
+constexpr int kTopkStreamThreads = 256;
+constexpr int kTopkStreamWarps = kTopkStreamThreads / 32;
+constexpr int kTopkStreamCand = 2048;
+static_assert(kTopkSmemMaxN <= 65536, "candidate indices are 16-bit");
 
-__global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(TopkParams p) {
+// One digit of the radix select over `nb` bins (nb = 8 or 4 per thread): the
+// largest digit d with sum_{e >= d} hist[e] >= need; stores d and
+// need - sum_{e > d} hist[e].  All threads call it.
+__device__ __forceinline__ void find_digit_stream(const uint32_t* hist, int nb, uint32_t need, uint32_t* wsum,
+                                                  uint32_t* out_digit, uint32_t* out_need) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int per = nb / kTopkStreamThreads;           // bins per thread (8 or 4)
+  const int hi = nb - threadIdx.x * per;              // this thread's bins [hi - per, hi), top bins first
+  uint32_t local = 0;
+  for (int e = 0; e < per; ++e) local += hist[hi - 1 - e];
+  uint32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[wid] = incl;
+  __syncthreads();
+  uint32_t before = 0;
+#pragma unroll
+  for (int w = 0; w < kTopkStreamWarps; ++w) before += w < wid ? wsum[w] : 0u;
+  const uint32_t above = before + incl - local;        // keys in the bins above this thread's
+  if (above < need && above + local >= need) {
+    uint32_t cum = above;
+    for (int e = 0; e < per; ++e) {
+      const int b = hi - 1 - e;
+      if (cum + hist[b] >= need) { *out_digit = (uint32_t)b; *out_need = need - cum; break; }
+      cum += hist[b];
+    }
+  }
+  __syncthreads();
+}
+
+// Histogram pass over the row: bins (u >> shift) & (nb - 1) of the keys u
+// whose bits above hshift equal `prefix` (every key for hshift = 32).
+__device__ __forceinline__ void stream_hist_pass(const float* s, int v, bool vec, uint32_t* hist, int nb, int shift,
+                                                 int hshift, uint32_t prefix) {
+  for (int x = threadIdx.x; x < nb; x += blockDim.x) hist[x] = 0u;
+  __syncthreads();
+  const uint32_t dmask = (uint32_t)nb - 1u;
+  const int v4 = vec ? (v >> 2) : 0;
+  const float4* s4 = reinterpret_cast<const float4*>(s);
+  auto count = [&](float f) {
+    const uint32_t u = order_key(f);
+    if (hshift == 32 || (u >> hshift) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
+  };
+  for (int base = 0; base < v4; base += 4 * blockDim.x) {
+    float4 f[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j4 = base + u * blockDim.x + threadIdx.x;
+      f[u] = j4 < v4 ? __ldg(s4 + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j4 = base + u * blockDim.x + threadIdx.x;
+      if (j4 < v4) { count(f[u].x); count(f[u].y); count(f[u].z); count(f[u].w); }
+    }
+  }
+  for (int j = 4 * v4 + threadIdx.x; j < v; j += blockDim.x) count(__ldg(s + j));
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kTopkStreamThreads) topk_rows_stream_kernel(TopkParams p) {
   griddep_wait();
   griddep_launch_dependents();
-  extern __shared__ uint32_t keys[];           // order keys of the row at kslot(j)
-  __shared__ uint32_t hist[kTopkSubHist * 256];
-  __shared__ int warp_buf[72];
+  __shared__ uint32_t hist[2048];
+  __shared__ uint32_t cand_key[kTopkStreamCand];
+  __shared__ uint16_t cand_idx[kTopkStreamCand];
+  __shared__ uint32_t wsum[kTopkStreamWarps];
   __shared__ uint32_t sh_digit, sh_need;
-  const int rloc = blockIdx.x;                 // row within the chunk
+  __shared__ int n_cand;
+  __shared__ int wcnt[kTopkStreamWarps][2];          // per warp: keys > T, keys == T
+  const int rloc = blockIdx.x;                       // row within the chunk
   const int b = rloc / p.q_count, qi = p.q_begin + rloc % p.q_count;
   const int t = p.q_pos[(int64_t)b * p.nq + qi];
   const int v = visible_count(t, p.m, p.N, p.entry_base);
@@ -141,84 +167,106 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(TopkParams p) {
     for (int j = threadIdx.x; j < p.k; j += blockDim.x) out[j] = j < v ? j : -1;
     return;
   }
-  // row -> shared keys: 16-byte loads, four in flight per thread (rows are
-  // 16-byte aligned when the row stride is a multiple of 4; else scalar)
-  if ((p.row_stride & 3) == 0) {
-    const int v4 = v >> 2;
-    const float4* s4 = reinterpret_cast<const float4*>(s);
-    for (int base = 0; base < v4; base += 4 * blockDim.x) {
-      float4 f[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j4 = base + u * blockDim.x + threadIdx.x;
-        f[u] = j4 < v4 ? __ldg(s4 + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j4 = base + u * blockDim.x + threadIdx.x;
-        if (j4 < v4) {
-          keys[kslot(4 * j4 + 0)] = order_key(f[u].x); keys[kslot(4 * j4 + 1)] = order_key(f[u].y);
-          keys[kslot(4 * j4 + 2)] = order_key(f[u].z); keys[kslot(4 * j4 + 3)] = order_key(f[u].w);
-        }
-      }
+  const bool vec = (p.row_stride & 3) == 0;          // 16-byte aligned rows (the base is)
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  // warp w walks [j0, j1), 32 keys at a time, in the candidate and output passes
+  const int L = ((v + kTopkStreamWarps * 32 - 1) / (kTopkStreamWarps * 32)) * 32;
+  const int j0 = wid * L, j1 = min(v, j0 + L);
+
+  // pass 1: bin of the k-th largest key
+  if (threadIdx.x == 0) n_cand = 0;
+  if (threadIdx.x < kTopkStreamWarps) { wcnt[threadIdx.x][0] = 0; wcnt[threadIdx.x][1] = 0; }
+  stream_hist_pass(s, v, vec, hist, 2048, 21, 32, 0u);
+  find_digit_stream(hist, 2048, (uint32_t)p.k, wsum, &sh_digit, &sh_need);
+  const uint32_t B1 = sh_digit;
+  uint32_t need = sh_need;
+
+  // pass 2: keys above the bin per warp; the bin's keys to the candidate list
+  int n_above = 0;
+  for (int j = j0 + lane; j - lane < j1; j += 32) {
+    const bool in = j < j1;
+    const uint32_t u = in ? order_key(__ldg(s + j)) : 0u;
+    const uint32_t bin = u >> 21;
+    n_above += __popc(__ballot_sync(0xffffffffu, in && bin > B1));
+    if (in && bin == B1) {
+      const int slot = atomicAdd(&n_cand, 1);
+      if (slot < kTopkStreamCand) { cand_key[slot] = u; cand_idx[slot] = (uint16_t)j; }
     }
-    for (int j = 4 * v4 + threadIdx.x; j < v; j += blockDim.x) keys[kslot(j)] = order_key(__ldg(s + j));
-  } else {
-    for (int j = threadIdx.x; j < v; j += blockDim.x) keys[kslot(j)] = order_key(__ldg(s + j));
   }
-  const int wid = threadIdx.x >> 5;
-  uint32_t* myhist = hist + (wid % kTopkSubHist) * 256;
-  uint32_t prefix = 0, mask = 0, need = (uint32_t)p.k;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int x = threadIdx.x; x < kTopkSubHist * 256; x += blockDim.x) hist[x] = 0;
-    __syncthreads();
-    for (int j = threadIdx.x; j < v; j += blockDim.x) {
-      const uint32_t u = keys[kslot(j)];
-      if ((u & mask) == prefix) atomicAdd(&myhist[(u >> shift) & 255u], 1u);
-    }
-    __syncthreads();
-    if (threadIdx.x < 256) {
-      uint32_t tot = 0;
-#pragma unroll
-      for (int h = 0; h < kTopkSubHist; ++h) tot += hist[h * 256 + threadIdx.x];
-      hist[threadIdx.x] = tot;                  // sub-histogram 0 <- total (own column only)
-    }
-    __syncthreads();
-    if (wid == 0) find_digit_warp(hist, 256, need, &sh_digit, &sh_need);
-    __syncthreads();
-    prefix |= sh_digit << shift;
-    mask |= 255u << shift;
-    need = sh_need;
-    __syncthreads();
-  }
-  // prefix = key of the k-th largest; take all keys > prefix and the first
-  // `need` keys == prefix in index order.  Thread i owns the contiguous
-  // segment [i*seg, (i+1)*seg): one block scan of its count of equal keys
-  // ranks the ties, one of its count of taken keys places its output.
   __syncthreads();
-  const int seg = (v + blockDim.x - 1) / blockDim.x;
-  const int j0 = threadIdx.x * seg, j1 = min(v, j0 + seg);
-  int n_eq = 0, n_gt = 0;
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t u = keys[kslot(j)];
-    n_eq += (u == prefix);
-    n_gt += (u > prefix);
-  }
-  int tot;
-  const int eq_before = block_excl_count(n_eq, warp_buf, &tot);
-  int eq_take = (int)need - eq_before;                  // ties this thread may still take
-  eq_take = eq_take < 0 ? 0 : (eq_take > n_eq ? n_eq : eq_take);
-  const int pos0 = block_excl_count(n_gt + eq_take, warp_buf, &tot);
-  int pos = pos0, eq_used = 0;
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t u = keys[kslot(j)];
-    bool take = u > prefix;
-    if (u == prefix && eq_used < eq_take) { take = true; ++eq_used; }
-    if (take) {
-      if (pos < p.k) out[pos] = j;
-      ++pos;
+  const int nc = n_cand;
+  uint32_t T;
+  if (nc <= kTopkStreamCand) {
+    // the two lower digits from the candidates
+    for (int x = threadIdx.x; x < 2048; x += blockDim.x) hist[x] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < nc; i += blockDim.x) atomicAdd(&hist[(cand_key[i] >> 10) & 2047u], 1u);
+    __syncthreads();
+    find_digit_stream(hist, 2048, need, wsum, &sh_digit, &sh_need);
+    const uint32_t pre22 = (B1 << 11) | sh_digit;
+    need = sh_need;
+    for (int x = threadIdx.x; x < 1024; x += blockDim.x) hist[x] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < nc; i += blockDim.x)
+      if ((cand_key[i] >> 10) == pre22) atomicAdd(&hist[cand_key[i] & 1023u], 1u);
+    __syncthreads();
+    find_digit_stream(hist, 1024, need, wsum, &sh_digit, &sh_need);
+    T = (pre22 << 10) | sh_digit;
+    need = sh_need;
+    // per-warp counts: keys above the bin (pass 2) plus the candidates > T, == T
+    for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+      const uint32_t u = cand_key[i];
+      const int w = (int)cand_idx[i] / L;
+      if (u > T) atomicAdd(&wcnt[w][0], 1);
+      else if (u == T) atomicAdd(&wcnt[w][1], 1);
     }
+    if (lane == 0) atomicAdd(&wcnt[wid][0], n_above);
+  } else {
+    // more keys in the bin than the list holds: the digits by passes over the row
+    stream_hist_pass(s, v, vec, hist, 2048, 10, 21, B1);
+    find_digit_stream(hist, 2048, need, wsum, &sh_digit, &sh_need);
+    const uint32_t pre22 = (B1 << 11) | sh_digit;
+    need = sh_need;
+    stream_hist_pass(s, v, vec, hist, 1024, 0, 10, pre22);
+    find_digit_stream(hist, 1024, need, wsum, &sh_digit, &sh_need);
+    T = (pre22 << 10) | sh_digit;
+    need = sh_need;
+    int n_gt = 0, n_eq = 0;
+    for (int j = j0 + lane; j - lane < j1; j += 32) {
+      const bool in = j < j1;
+      const uint32_t u = in ? order_key(__ldg(s + j)) : 0u;
+      n_gt += __popc(__ballot_sync(0xffffffffu, in && u > T));
+      n_eq += __popc(__ballot_sync(0xffffffffu, in && u == T));
+    }
+    if (lane == 0) { wcnt[wid][0] = n_gt; wcnt[wid][1] = n_eq; }
+  }
+  __syncthreads();
+  const int n_eq = wcnt[wid][1];
+  int eq_before = 0, out_before = 0;
+  for (int w = 0; w < wid; ++w) {
+    const int eb = eq_before;
+    eq_before += wcnt[w][1];
+    int et = (int)need - eb;
+    et = et < 0 ? 0 : (et > wcnt[w][1] ? wcnt[w][1] : et);
+    out_before += wcnt[w][0] + et;
+  }
+  int eq_take = (int)need - eq_before;               // ties this warp takes (lowest indices first)
+  eq_take = eq_take < 0 ? 0 : (eq_take > n_eq ? n_eq : eq_take);
+  // output pass: keys > T and the first eq_take keys == T of this warp's range
+  int pos = out_before, eq_seen = 0;
+  for (int j = j0 + lane; j - lane < j1; j += 32) {
+    const bool in = j < j1;
+    const uint32_t u = in ? order_key(__ldg(s + j)) : 0u;
+    const uint32_t eqb = __ballot_sync(0xffffffffu, in && u == T);
+    const bool take = in && (u > T || (u == T && eq_seen + __popc(eqb & lt) < eq_take));
+    const uint32_t tb = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int o = pos + __popc(tb & lt);
+      if (o < p.k) out[o] = j;
+    }
+    pos += __popc(tb);
+    eq_seen += __popc(eqb);
   }
 }
 

@@ -7,6 +7,7 @@ a profiler to capture.
     python -m long_context_compressed_overlapped_b200.profile_case indexer --calls 4
     python -m long_context_compressed_overlapped_b200.profile_case compress --calls 4
     python -m long_context_compressed_overlapped_b200.profile_case prefill --calls 2
+    python -m long_context_compressed_overlapped_b200.profile_case prefill_tail --calls 2
 
 ``csa``: one CSA decode layer through ``compressed_attn_decode`` (indexer with
 e4m3 keys, top-k select, attention, combine); ``hca``: one HCA decode layer
@@ -22,7 +23,10 @@ the decode_1m workload.  ``prefill``: the csa_prefill_128k layer's shapes
 (64 heads of 512 dims, 64 indexer heads of 128 dims, top-1,024, window 128)
 at n = 16,384 tokens: both compressors, indexer_topk (the tensor-core
 indexer over 4-query tiles, then the row top-k) and compressed_attn_prefill;
-about 3 GB on the device.  The process exits non-zero if a bounded device
+about 3 GB on the device.  ``prefill_tail``: indexer_topk for the last 16,384
+queries of csa_prefill_128k (positions 114,688 .. 131,071 against the layer's
+32,768 indexer keys: the longest score rows, 28,673 .. 32,768 entries);
+about 2.3 GB on the device.  The process exits non-zero if a bounded device
 wait gave up.
 """
 
@@ -38,11 +42,13 @@ from . import api, native, runtime, synth
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("case", choices=("csa", "hca", "csa_fp8kv", "hca_fp8kv", "indexer", "compress",
-                                        "prefill"))
+                                        "prefill", "prefill_tail"))
     ap.add_argument("--calls", type=int, default=4)
     a = ap.parse_args(argv)
     if a.case == "prefill":
         return prefill_case(a.calls)
+    if a.case == "prefill_tail":
+        return prefill_tail_case(a.calls)
     wl = synth.WORKLOADS["decode_1m_fp8kv" if a.case.endswith("_fp8kv") else "decode_1m"]
     kind = "hca" if a.case.startswith("hca") else "csa"
     ctx = wl.ctx - 1 if a.case == "compress" else wl.ctx
@@ -82,6 +88,22 @@ def prefill_case(calls: int, n: int = 16384) -> int:
     torch.cuda.synchronize()
     err = api.device_error()
     print(f"profile_case prefill (n={n}): {calls} calls, device error {err}")
+    return 1 if err else 0
+
+
+def prefill_tail_case(calls: int, nq: int = 16384) -> int:
+    wl = synth.WORKLOADS["csa_prefill_128k"]
+    D = synth.Draw(wl.seed + 100, "cuda")
+    N = wl.n // wl.m
+    qI = D.normal("qI", (1, nq, wl.HI, wl.dI), 1.0, torch.bfloat16)
+    w = D.normal("w", (1, nq, wl.HI), 1.0 / wl.HI ** 0.5)
+    kI = D.normal("kI", (1, N, wl.dI), 1.0, torch.bfloat16)
+    q_pos = torch.arange(wl.n - nq, wl.n, device="cuda", dtype=torch.int32)[None]
+    for _ in range(calls):
+        api.indexer_topk(qI, w, kI, q_pos, wl.m, wl.k)
+    torch.cuda.synchronize()
+    err = api.device_error()
+    print(f"profile_case prefill_tail ({nq} queries, {N} keys): {calls} calls, device error {err}")
     return 1 if err else 0
 
 
