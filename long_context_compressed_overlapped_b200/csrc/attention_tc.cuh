@@ -288,6 +288,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
   // bar_pv: the tile's P.V MMAs have completed (its key buffer is free, O^T
   // and P^T may be touched again)
   __shared__ uint64_t bar_q_raw, bar_q_empty, bar_q_full, bar_s_full, bar_s_empty, bar_p_full, bar_pv, bar_done;
+  // prefill: bar_pvm[j], the tile's P.V MMAs of O^T M-tiles 0..j have completed
+  // (key chunks 2j, 2j + 1 are free), j < 3; M-tile 3 completes bar_pv
+  __shared__ uint64_t bar_pvm[kAttnMT - 1];
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
   __shared__ float red[2][4 * 32];
@@ -322,6 +325,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
     mbar_init(&bar_s_empty, 256);
     mbar_init(&bar_p_full, 256);
     mbar_init(&bar_pv, 1);
+    if constexpr (!kDecode)
+      for (int j = 0; j < kAttnMT - 1; ++j) mbar_init(&bar_pvm[j], 1);
     mbar_init(&bar_done, 2);                       // both MMA issuers
     mbar_fence_init();
   }
@@ -461,7 +466,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
         for (int cc = 0; cc < kChunksPerWarp; ++cc) {
           const int c = kNP == 2 ? 4 * (cc >> 1) + 2 * pw + (cc & 1) : cc;
           int ok = 1;
-          if (lane == 0) ok = mbar_wait(&bar_pv, ph ^ 1, &abort_flag);
+          // prefill: a chunk pair is free once the P.V of its O^T M-tile has
+          // completed, so the next tile's rows start landing during the P.V
+          uint64_t* freed = (!kDecode && c / 2 < kAttnMT - 1) ? &bar_pvm[c / 2] : &bar_pv;
+          if (lane == 0) ok = mbar_wait(freed, ph ^ 1, &abort_flag);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) { stop = true; break; }
           uint8_t* dst = sK + c * AttnSmem::K_CHUNK;
@@ -646,6 +654,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
 #pragma unroll
               for (int ks = 0; ks < 8; ++ks)
                 umma_bf16(tO + mt * kAttnH, vd + 128 * ks, pdesc + 128 * ks, idesc_pv, !(first && ks == 0));
+              if (!kDecode && mt < kAttnMT - 1) umma_commit(&bar_pvm[mt]);
             }
           } else {
 #pragma unroll
@@ -653,6 +662,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
               const uint64_t vd = vdesc + (uint64_t)((2 * mt) * (AttnSmem::K_CHUNK >> 4));
               for (int ks = 0; ks < nks; ++ks)
                 umma_bf16(tO + mt * kAttnH, vd + 128 * ks, pdesc + 128 * ks, idesc_pv, !(first && ks == 0));
+              if (!kDecode && mt < kAttnMT - 1) umma_commit(&bar_pvm[mt]);
             }
           }
           umma_commit(&bar_pv);
