@@ -10,8 +10,11 @@
 //
 // Roles (320 threads): warps 0-3 epilogue, warp 4 TMA producer, warp 5 MMA
 // issuer (and TMEM owner), warps 6-9 convert e4m3 key tiles to bf16 (exact)
-// when the keys are stored in e4m3; for e4m3 keys the per-row fp32 scale is
-// applied to the score (a positive per-row factor commutes with ReLU).
+// when the keys are stored in e4m3 (the per-row fp32 scale is applied to the
+// score: a positive per-row factor commutes with ReLU), and with bf16 keys
+// form a second epilogue group: the two groups take alternate tiles (and
+// accumulators), since one group's TMEM reads and weighted sums took longer
+// than the tile's MMAs.
 //
 // Work items: prefill = (sequence, tile of QT queries, every key tile any of
 // its queries can see), longest first; decode = (sequence, contiguous range of
@@ -58,7 +61,7 @@ struct IdxTcCfg {
   static constexpr int B_BYTES = 2 * B_CHUNK;
   static constexpr int A_BYTES = 2 * 128 * 128;                 // 128 keys x 128 dims bf16
   static constexpr int RAW_BYTES = kFP8 ? 128 * 128 : 0;        // 128 keys x 128 e4m3
-  static constexpr int SMEM = 1024 + B_BYTES + NSTAGE * (A_BYTES + RAW_BYTES) + QT * HI * 4 + 1024;
+  static constexpr int SMEM = 1024 + B_BYTES + NSTAGE * (A_BYTES + RAW_BYTES) + 2 * QT * HI * 4 + 1024;
   static_assert(NCOL % 16 == 0 && NCOL <= 256, "MMA N");
   static_assert(HI % 32 == 0, "heads per query must be a multiple of 32");
 };
@@ -211,9 +214,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
       umma_commit(&bar_done);
       mbar_wait(&bar_done, 0, &abort_flag);
     }
-  } else if (warp >= 6) {
+  } else if (kFP8 && warp >= 6) {
     // ------------------------------------------------------------ e4m3 -> bf16
-    if (kFP8) {
+    {
       const int ct = threadIdx.x - 192;                 // 0..127
       uint32_t a_iter = 0;
       for (int id = blockIdx.x; id < p.n_items && !abort_flag; id += gridDim.x) {
@@ -249,44 +252,52 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 0-3)
-    const int et = threadIdx.x;                         // key lane 0..127
+    // ------------------------------------------------------------ epilogue: warps 0-3 (and 6-9)
+    // group eg (bf16 keys: eg = 1 for warps 6-9) takes the tiles of parity eg
+    // (one group takes every tile when the keys are e4m3)
+    constexpr int kGroups = kFP8 ? 1 : 2;
+    const int eg = warp >= 6 ? 1 : 0;
+    const int quad = warp & 3;                          // TMEM lane quarter of this warp
+    const int et = quad * 32 + lane;                    // key lane 0..127
+    float* sWg = sW + eg * QT * HI;
     uint32_t acc_iter = 0;
-    bool stop = false;                                  // uniform over the 128 threads
+    bool stop = false;                                  // uniform over the group's 128 threads
     for (int id = blockIdx.x; id < p.n_items && !stop; id += gridDim.x) {
       const IdxItem it = idx_item<QT>(p, id);
       if (it.kt1 <= it.kt0) continue;
-      named_sync128();
+      group_sync(1 + eg);
       for (int x = et; x < QT * HI; x += 128) {
         const int q = x / HI;
-        sW[x] = q < it.qn ? p.w[((int64_t)it.b * p.nq + it.q0 + q) * HI + (x % HI)] : 0.f;
+        sWg[x] = q < it.qn ? p.w[((int64_t)it.b * p.nq + it.q0 + q) * HI + (x % HI)] : 0.f;
       }
-      named_sync128();
+      group_sync(1 + eg);
       int vq[QT];
 #pragma unroll
       for (int q = 0; q < QT; ++q) vq[q] = q < it.qn ? idx_visible(p, it.b, it.q0 + q) : 0;
       for (int kt = it.kt0; kt < it.kt1; ++kt, ++acc_iter) {
+        if (kGroups == 2 && (int)(acc_iter & 1u) != eg) continue;
         const int j = acc_iter % NACC;
         const uint32_t aph = (acc_iter / NACC) & 1;
-        if (!mbar_wait128(&bar_acc_full[j], aph, &abort_flag)) { stop = true; break; }
+        if (!mbar_wait_group(1 + eg, &bar_acc_full[j], aph, &abort_flag)) { stop = true; break; }
         mbar_arrive(&bar_a_empty[acc_iter % NS]);       // the tile's key stage is free
         tc_fence_after();
         const int key = kt * 128 + et;
         float scale = 1.f;
         if (kFP8 && key < p.N) scale = __ldg(p.kI_scale + (int64_t)it.b * p.N + key);
-        const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + j * NCOL;
+        const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + j * NCOL;
 #pragma unroll
         for (int q = 0; q < QT; ++q) {
+          // the query's HI columns in flight together, one wait
+          float v[HI / 32][32];
+#pragma unroll
+          for (int c = 0; c < HI / 32; ++c) tmem_ld32(tbase + q * HI + c * 32, v[c]);
+          tmem_wait_ld();
           float acc = 0.f;
+          const float* wq = sWg + q * HI;
 #pragma unroll
-          for (int c = 0; c < HI / 32; ++c) {
-            float v[32];
-            tmem_ld32(tbase + q * HI + c * 32, v);
-            tmem_wait_ld();
-            const float* wq = sW + q * HI + c * 32;
+          for (int c = 0; c < HI / 32; ++c)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) acc = fmaf(wq[e], fmaxf(v[e], 0.f), acc);
-          }
+            for (int e = 0; e < 32; ++e) acc = fmaf(wq[c * 32 + e], fmaxf(v[c][e], 0.f), acc);
           if (key < vq[q])
             p.scores[((int64_t)it.b * p.q_count + (it.q0 + q - p.q_begin)) * p.score_row_stride + key] = acc * scale;
         }
