@@ -453,7 +453,6 @@ void f8_decode_split(const csahca_indexer_args* a, int* tiles_per_split, int* sp
 // The FP8 decode scan can route the top-k in its epilogue when every work
 // item has a CTA of its own (a CTA waits for its row's other items) and the
 // item's scores fit in shared memory beside the key stages.
-constexpr int kRouteMaxTiles = 64;
 bool f8_route_ok(const csahca_indexer_args* a) {
   int tps = 0, sp = 0;
   f8_decode_split(a, &tps, &sp);

@@ -31,9 +31,8 @@ constexpr int kCntAbove = 0;               // keys routed to the taken list
 constexpr int kCntCand = 1;                // keys routed to the candidate list
 constexpr int kCntSlices = 2;              // select CTAs done with the row
 constexpr int kCntItems = 3;               // indexer work items done with the row
-constexpr int kCntT = 4;                   // threshold bin (set by the indexer's last item)
+constexpr int kCntT = 4;                   // threshold bin (set by the indexer's last item; unrouted rows)
 constexpr int kCntAboveT = 5;              // keys in bins above it
-constexpr int kCntReady = 6;               // 1 once kCntT / kCntAboveT are stored (fused routing)
 constexpr int kHistShift = 21;
 constexpr int kTopkLargeMaxN = 786432;     // two bitmaps of N bits in shared memory
 
