@@ -77,26 +77,45 @@ __device__ __forceinline__ void dc_cluster_wait() {
 }
 
 // RMSNorm scale and gain, then RoPE at `pos` on the pairs of one vector whose
-// channels fall in the last r.
+// channels fall in the last r; split in two so that the per-channel factors
+// (gain, cos / sin of the angle) can be formed before the row's norm is known.
 template <int VEC>
-__device__ __forceinline__ void dc_finish(float (&v)[VEC], int ch0, const DecodeCompressParams& p, float inv,
-                                          double pos) {
+__device__ __forceinline__ void dc_finish_coef(int ch0, const DecodeCompressParams& p, double pos, float (&g)[VEC],
+                                               float (&cs)[VEC / 2], float (&sn)[VEC / 2]) {
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) g[e] = (p.kv_norm && p.gain) ? __ldg(p.gain + ch0 + e) : 1.f;
+  const int r = p.rope_dims, r0 = p.d - r;
+#pragma unroll
+  for (int e = 0; e < VEC; e += 2) {
+    cs[e / 2] = 1.f;
+    sn[e / 2] = 0.f;
+    if (r > 0 && ch0 + e >= r0) rope_sincos(pos, p.theta[(ch0 + e - r0) >> 1], &cs[e / 2], &sn[e / 2]);
+  }
+}
+template <int VEC>
+__device__ __forceinline__ void dc_finish_apply(float (&v)[VEC], int ch0, const DecodeCompressParams& p, float inv,
+                                                const float (&g)[VEC], const float (&cs)[VEC / 2],
+                                                const float (&sn)[VEC / 2]) {
   if (p.kv_norm) {
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) v[e] = v[e] * inv * (p.gain ? __ldg(p.gain + ch0 + e) : 1.f);
+    for (int e = 0; e < VEC; ++e) v[e] = v[e] * inv * g[e];
   }
   const int r = p.rope_dims, r0 = p.d - r;
 #pragma unroll
   for (int e = 0; e < VEC; e += 2) {
-    const int cc = ch0 + e;
-    if (r > 0 && cc >= r0) {
-      float cs, sn;
-      rope_sincos(pos, p.theta[(cc - r0) >> 1], &cs, &sn);
+    if (r > 0 && ch0 + e >= r0) {
       const float x0 = v[e], x1 = v[e + 1];
-      v[e] = x0 * cs - x1 * sn;
-      v[e + 1] = x0 * sn + x1 * cs;
+      v[e] = x0 * cs[e / 2] - x1 * sn[e / 2];
+      v[e + 1] = x0 * sn[e / 2] + x1 * cs[e / 2];
     }
   }
+}
+template <int VEC>
+__device__ __forceinline__ void dc_finish(float (&v)[VEC], int ch0, const DecodeCompressParams& p, float inv,
+                                          double pos) {
+  float g[VEC], cs[VEC / 2], sn[VEC / 2];
+  dc_finish_coef<VEC>(ch0, p, pos, g, cs, sn);
+  dc_finish_apply<VEC>(v, ch0, p, inv, g, cs, sn);
 }
 
 template <typename T, bool kCSA>
@@ -153,6 +172,12 @@ decode_compress_kernel(const __grid_constant__ DecodeCompressParams p) {
   const int i = emit ? (int)(t1 / m - 1) : 0;
   const int64_t lrow = emit ? (int64_t)i - p.entry_base : 0;
   const bool do_win = has_win && t >= 0;
+  // this CTA's slice of the window row: its per-channel factors are formed
+  // now, while the row's sum of squares is gathered, so that only the
+  // scaling is left after the barrier
+  const bool fin_win = do_win && tid >= q * nvk && tid < (q + 1) * nvk;
+  float wg[VEC], wcs[VEC / 2], wsn[VEC / 2];
+  if (fin_win) dc_finish_coef<VEC>(tid * VEC, p, (double)t, wg, wcs, wsn);
 
   // ---- the new token into ring slot t % R
   if (t >= 0 && n_s >= 0) {
@@ -237,10 +262,10 @@ decode_compress_kernel(const __grid_constant__ DecodeCompressParams p) {
   __syncthreads();
 
   // ---- window row: this CTA's slice, normalised and rotated to position t
-  if (do_win && tid >= q * nvk && tid < (q + 1) * nvk) {
+  if (fin_win) {
     float tw = 0.f;
     for (int k = 0; k < (nvr + 31) / 32; ++k) tw += wss[k];
-    dc_finish<VEC>(wv, tid * VEC, p, rsqrtf(tw / (float)d + p.eps), (double)t);
+    dc_finish_apply<VEC>(wv, tid * VEC, p, rsqrtf(tw / (float)d + p.eps), wg, wcs, wsn);
     store16(static_cast<T*>(p.win) + ((int64_t)b * p.w + t % p.w) * d + tid * VEC, wv);
   }
   if (!emit) return;                          // uniform over the cluster: one position per sequence
