@@ -345,7 +345,7 @@ int launch_topk(const csahca_indexer_args* a, const float* scores, int64_t strid
     tp.B = 1; tp.nq = rows; tp.N = a->N; tp.m = a->m; tp.k = a->k;
     tp.q_begin = 0; tp.q_count = rows; tp.entry_base = a->entry_base;
     CSAHCA_TRACE("topk_rows", s);
-    launch_k(topk_rows_stream_kernel, dim3(rows), dim3(kTopkStreamThreads), 0, s, tp);
+    launch_k(topk_rows_sample_kernel, dim3(rows), dim3(kTopkStreamThreads), 0, s, tp);
     CSAHCA_CHECK_LAUNCH();
     return CSAHCA_OK;
   }

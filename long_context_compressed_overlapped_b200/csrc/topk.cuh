@@ -13,7 +13,7 @@
 
 namespace csahca {
 
-constexpr int kTopkSmemMaxN = 32768;        // rows up to this length: topk_rows_stream_kernel
+constexpr int kTopkSmemMaxN = 32768;        // rows up to this length: topk_rows_sample_kernel
                                             // (16-bit candidate indices)
 
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -61,12 +61,9 @@ struct TopkParams {
   int entry_base;                              // local row j is global entry entry_base + j
 };
 
-// ---- rows up to kTopkSmemMaxN ---------------------------------------------------
-// One CTA of 256 threads per row and ~21 KB of shared memory (the row itself
-// is not held there), so several rows run per SM and the reads of one hide
-// the latency of another; a first version holding each row in shared memory
-// (128 KB, one row per SM) took 13.0 ms over csa_prefill_128k's score rows
-// against 10.3 ms for this one.
+// ---- rows up to kTopkSmemMaxN: three passes over the row ---------------------
+// The fallback of topk_rows_sample_kernel (below), one CTA of 256 threads per
+// row, the row itself not held in shared memory:
 //   pass 1 (the row from HBM): histogram of the order keys' bits 31..21 ->
 //     the bin B of the k-th largest key;
 //   pass 2 (from L2): each warp walks its own contiguous range of the row,
@@ -147,26 +144,25 @@ __device__ __forceinline__ void stream_hist_pass(const float* s, int v, bool vec
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kTopkStreamThreads) topk_rows_stream_kernel(TopkParams p) {
-  griddep_wait();
-  griddep_launch_dependents();
-  __shared__ uint32_t hist[2048];
-  __shared__ uint32_t cand_key[kTopkStreamCand];
-  __shared__ uint16_t cand_idx[kTopkStreamCand];
-  __shared__ uint32_t wsum[kTopkStreamWarps];
-  __shared__ uint32_t sh_digit, sh_need;
-  __shared__ int n_cand;
-  __shared__ int wcnt[kTopkStreamWarps][2];          // per warp: keys > T, keys == T
-  const int rloc = blockIdx.x;                       // row within the chunk
-  const int b = rloc / p.q_count, qi = p.q_begin + rloc % p.q_count;
-  const int t = p.q_pos[(int64_t)b * p.nq + qi];
-  const int v = visible_count(t, p.m, p.N, p.entry_base);
-  int* out = p.idx + ((int64_t)b * p.nq + qi) * p.k;
-  const float* s = p.scores + (int64_t)rloc * p.row_stride;
-  if (v <= p.k) {
-    for (int j = threadIdx.x; j < p.k; j += blockDim.x) out[j] = j < v ? j : -1;
-    return;
-  }
+// Shared memory of one row's selection (both kernels below).
+struct TopkRowSmem {
+  uint32_t hist[2048];
+  uint32_t wsum[kTopkStreamWarps];
+  uint32_t sh_digit, sh_need;
+  int n_cand;
+  int wcnt[kTopkStreamWarps][2];                     // per warp: keys > T, keys == T
+};
+
+// The three-pass selection of one row of v > k keys (every thread of the
+// CTA): see the comment above kTopkStreamThreads.
+__device__ __forceinline__ void topk_row_passes(const TopkParams& p, const float* s, int v, int* out,
+                                                TopkRowSmem& sm, uint32_t* cand_key, uint16_t* cand_idx) {
+  uint32_t* hist = sm.hist;
+  uint32_t* wsum = sm.wsum;
+  uint32_t& sh_digit = sm.sh_digit;
+  uint32_t& sh_need = sm.sh_need;
+  int& n_cand = sm.n_cand;
+  auto& wcnt = sm.wcnt;
   const bool vec = (p.row_stride & 3) == 0;          // 16-byte aligned rows (the base is)
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const uint32_t lt = (1u << lane) - 1u;
@@ -264,6 +260,196 @@ __global__ void __launch_bounds__(kTopkStreamThreads) topk_rows_stream_kernel(To
     if (take) {
       const int o = pos + __popc(tb & lt);
       if (o < p.k) out[o] = j;
+    }
+    pos += __popc(tb);
+    eq_seen += __popc(eqb);
+  }
+}
+
+// Row r of the chunk: its position, visible count, output and scores.
+struct TopkRow { int v; int* out; const float* s; };
+__device__ __forceinline__ TopkRow topk_row(const TopkParams& p) {
+  const int rloc = blockIdx.x;                       // row within the chunk
+  const int b = rloc / p.q_count, qi = p.q_begin + rloc % p.q_count;
+  const int t = p.q_pos[(int64_t)b * p.nq + qi];
+  TopkRow r;
+  r.v = visible_count(t, p.m, p.N, p.entry_base);
+  r.out = p.idx + ((int64_t)b * p.nq + qi) * p.k;
+  r.s = p.scores + (int64_t)rloc * p.row_stride;
+  return r;
+}
+
+// ---- rows up to kTopkSmemMaxN, one pass over the row --------------------------
+// topk_rows_sample_kernel (256 threads, ~33 KB of shared memory):
+//   bound: a row whose warp ranges fit the warps' candidate lists keeps
+//     every key; otherwise a histogram of one 32-key segment in 8 gives the
+//     bin of the sample's k_s-th largest key, k_s = the sample's share of k
+//     plus a margin, and every key in that bin or above is kept (the k-th
+//     largest of the row is in a bin at least as high unless the sample
+//     misleads, which the count below detects);
+//   collect (the row from HBM, once): each warp walks its contiguous range of
+//     the row in index order and appends the kept keys with their indices to
+//     its own list in shared memory (warp ballots place them);
+//   when the lists hold at least k keys and none overflowed, the exact key T
+//     of the k-th largest and the ties to take come from three histograms
+//     over the lists (bits 31..21, 20..10, 9..0), and each warp writes its
+//     list's keys > T and its share of the lowest-index keys == T, in index
+//     order; otherwise the row takes the three passes of topk_row_passes.
+constexpr int kTopkSampPerWarp = 512;
+constexpr int kTopkSampCand = kTopkSampPerWarp * kTopkStreamWarps;
+static_assert(kTopkSampCand >= kTopkStreamCand, "the fallback's candidate list fits the sample lists");
+
+__global__ void __launch_bounds__(kTopkStreamThreads) topk_rows_sample_kernel(TopkParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
+  __shared__ TopkRowSmem sm;
+  __shared__ uint32_t ck[kTopkSampCand];
+  __shared__ uint16_t ci[kTopkSampCand];
+  __shared__ int wn[kTopkStreamWarps];
+  const TopkRow r = topk_row(p);
+  const int v = r.v;
+  int* out = r.out;
+  const float* s = r.s;
+  if (v <= p.k) {
+    for (int j = threadIdx.x; j < p.k; j += blockDim.x) out[j] = j < v ? j : -1;
+    return;
+  }
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int L = ((v + kTopkStreamWarps * 32 - 1) / (kTopkStreamWarps * 32)) * 32;
+  const int j0 = wid * L, j1 = min(v, j0 + L);
+  const uint32_t k = (uint32_t)p.k;
+
+  // ---- the bin from which keys are kept
+  uint32_t Blo = 0;
+  if (L > kTopkSampPerWarp) {
+    for (int x = threadIdx.x; x < 2048; x += blockDim.x) sm.hist[x] = 0u;
+    __syncthreads();
+    const int nseg = (v + 31) / 32;                  // 32-key segments; segment 8 g is sampled
+    // warp w takes sampled segments 8 g, g = w + 8 i; eight loads go out
+    // before any is used (the row comes from HBM)
+    for (int g0 = wid; 8 * g0 < nseg; g0 += 8 * kTopkStreamWarps) {
+      float f[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        const int j = 8 * (g0 + x * kTopkStreamWarps) * 32 + lane;
+        f[x] = j < v ? __ldg(s + j) : 0.f;
+      }
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        const int j = 8 * (g0 + x * kTopkStreamWarps) * 32 + lane;
+        if (j < v) atomicAdd(&sm.hist[order_key(f[x]) >> 21], 1u);
+      }
+    }
+    __syncthreads();
+    // the sample size, then its k_s-th largest bin
+    const int nfull = nseg / 8 + (nseg % 8 != 0 ? 1 : 0);
+    const int last = 8 * (nfull - 1);                // the last sampled segment may be short
+    const int ns = (nfull - 1) * 32 + min(32, v - 32 * last);
+    const int ks0 = (int)(((int64_t)p.k * ns + v - 1) / v);
+    const int ks = min(ns, ks0 + max(64, ks0 / 4));
+    find_digit_stream(sm.hist, 2048, (uint32_t)ks, sm.wsum, &sm.sh_digit, &sm.sh_need);
+    Blo = sm.sh_digit;
+  }
+
+  // ---- collect: each warp's kept keys, in index order, into its list
+  uint32_t* lk = ck + wid * kTopkSampPerWarp;
+  uint16_t* li = ci + wid * kTopkSampPerWarp;
+  int cnt = 0;
+  // eight 32-key steps per round: their loads go out before any is used
+  for (int base = j0; base < j1; base += 8 * 32) {
+    float f[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      const int j = base + 32 * x + lane;
+      f[x] = j < j1 ? __ldg(s + j) : 0.f;
+    }
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      const int j = base + 32 * x + lane;
+      const bool in = j < j1;
+      const uint32_t u = order_key(f[x]);
+      const bool keep = in && (u >> 21) >= Blo;
+      const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+      if (keep) {
+        const int o = cnt + __popc(kb & lt);
+        if (o < kTopkSampPerWarp) { lk[o] = u; li[o] = (uint16_t)j; }
+      }
+      cnt += __popc(kb);
+    }
+  }
+  if (lane == 0) wn[wid] = cnt;
+  __syncthreads();
+  int total = 0;
+  bool over = false;
+#pragma unroll
+  for (int w = 0; w < kTopkStreamWarps; ++w) {
+    total += wn[w];
+    over = over || wn[w] > kTopkSampPerWarp;
+  }
+  if (over || total < (int)k) {
+    // the sample misled or one bin holds too many keys: the three passes
+    // (every thread takes this branch together: total and over are uniform)
+    if (threadIdx.x == 0) sm.n_cand = 0;
+    if (threadIdx.x < kTopkStreamWarps) { sm.wcnt[threadIdx.x][0] = 0; sm.wcnt[threadIdx.x][1] = 0; }
+    __syncthreads();
+    topk_row_passes(p, s, v, out, sm, ck, ci);
+    return;
+  }
+
+  // ---- the exact threshold over the lists: three digits of 11, 11, 10 bits
+  uint32_t need = k, prefix = 0;
+  const int shifts[3] = {21, 10, 0};
+  const int bins[3] = {2048, 2048, 1024};
+#pragma unroll 1
+  for (int dgt = 0; dgt < 3; ++dgt) {
+    const int sh = shifts[dgt], nb = bins[dgt], hs = dgt == 0 ? 32 : shifts[dgt - 1];
+    for (int x = threadIdx.x; x < 2048; x += blockDim.x) sm.hist[x] = 0u;
+    __syncthreads();
+    for (int x = threadIdx.x; x < kTopkSampCand; x += blockDim.x) {
+      const int w = x / kTopkSampPerWarp, o = x % kTopkSampPerWarp;
+      if (o < wn[w]) {
+        const uint32_t u = ck[x];
+        if (hs == 32 || (u >> hs) == prefix) atomicAdd(&sm.hist[(u >> sh) & (uint32_t)(nb - 1)], 1u);
+      }
+    }
+    __syncthreads();
+    find_digit_stream(sm.hist, nb, need, sm.wsum, &sm.sh_digit, &sm.sh_need);
+    prefix = dgt == 0 ? sm.sh_digit : ((prefix << (dgt == 1 ? 11 : 10)) | sm.sh_digit);
+    need = sm.sh_need;
+  }
+  const uint32_t T = prefix;                         // the k-th largest key; `need` ties at T to take
+
+  // ---- per-warp counts, then each warp writes its list's selection in order
+  int n_gt = 0, n_eq = 0;
+  for (int o = lane; o - lane < wn[wid]; o += 32) {
+    const bool in = o < wn[wid];
+    const uint32_t u = in ? lk[o] : 0u;
+    n_gt += __popc(__ballot_sync(0xffffffffu, in && u > T));
+    n_eq += __popc(__ballot_sync(0xffffffffu, in && u == T));
+  }
+  if (lane == 0) { sm.wcnt[wid][0] = n_gt; sm.wcnt[wid][1] = n_eq; }
+  __syncthreads();
+  int eq_before = 0, out_before = 0;
+  for (int w = 0; w < wid; ++w) {
+    const int eb = eq_before;
+    eq_before += sm.wcnt[w][1];
+    int et = (int)need - eb;
+    et = et < 0 ? 0 : (et > sm.wcnt[w][1] ? sm.wcnt[w][1] : et);
+    out_before += sm.wcnt[w][0] + et;
+  }
+  int eq_take = (int)need - eq_before;               // ties this warp takes (lowest indices first)
+  eq_take = eq_take < 0 ? 0 : (eq_take > n_eq ? n_eq : eq_take);
+  int pos = out_before, eq_seen = 0;
+  for (int o = lane; o - lane < wn[wid]; o += 32) {
+    const bool in = o < wn[wid];
+    const uint32_t u = in ? lk[o] : 0u;
+    const uint32_t eqb = __ballot_sync(0xffffffffu, in && u == T);
+    const bool take = in && (u > T || (u == T && eq_seen + __popc(eqb & lt) < eq_take));
+    const uint32_t tb = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int q = pos + __popc(tb & lt);
+      if (q < p.k) out[q] = (int)li[o];
     }
     pos += __popc(tb);
     eq_seen += __popc(eqb);
