@@ -352,7 +352,14 @@ __global__ void __launch_bounds__(kTopkStreamThreads) topk_rows_sample_kernel(To
     Blo = sm.sh_digit;
   }
 
-  // ---- collect: each warp's kept keys, in index order, into its list
+  // ---- collect: each warp's kept keys, in index order, into its list.  A key
+  // is kept when its order key is at least Blo << 21, i.e. when its score is
+  // at least the score fb whose order key that is (order keys are monotone in
+  // the score), so the walk compares scores and forms order keys for kept
+  // keys only
+  // (bins below 4 hold no finite score: every key is kept from there)
+  const uint32_t klo = Blo << 21;
+  const float fb = Blo < 4 ? -INFINITY : __uint_as_float((klo & 0x80000000u) ? (klo & 0x7fffffffu) : ~klo);
   uint32_t* lk = ck + wid * kTopkSampPerWarp;
   uint16_t* li = ci + wid * kTopkSampPerWarp;
   int cnt = 0;
@@ -367,13 +374,11 @@ __global__ void __launch_bounds__(kTopkStreamThreads) topk_rows_sample_kernel(To
 #pragma unroll
     for (int x = 0; x < 8; ++x) {
       const int j = base + 32 * x + lane;
-      const bool in = j < j1;
-      const uint32_t u = order_key(f[x]);
-      const bool keep = in && (u >> 21) >= Blo;
+      const bool keep = j < j1 && f[x] >= fb;
       const uint32_t kb = __ballot_sync(0xffffffffu, keep);
       if (keep) {
         const int o = cnt + __popc(kb & lt);
-        if (o < kTopkSampPerWarp) { lk[o] = u; li[o] = (uint16_t)j; }
+        if (o < kTopkSampPerWarp) { lk[o] = order_key(f[x]); li[o] = (uint16_t)j; }
       }
       cnt += __popc(kb);
     }
