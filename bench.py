@@ -406,15 +406,16 @@ def decode_run(wl, args, dev, stream, world, rank, want_cpu, e2e=True):
         host_outp = torch.empty(io.out.shape, dtype=io.out.dtype).pin_memory()
         h2d, d2h = io.inp.numel(), io.out.numel()
         state = {"i": 0}
+        # one graph per step's host buffer: the copies pipelined layer by layer
+        # with the kernels (runtime.HostIOGraph)
+        graphs = [runtime.HostIOGraph(eager, io, h, host_outp) for h in host_inps]
 
         def e2e_between(i):
             flush_buf.random_(0, 255)
             state["i"] = i
 
         def e2e_step():
-            io.inp.copy_(host_inps[state["i"] % K], non_blocking=True)
-            step()
-            host_outp.copy_(io.out, non_blocking=True)
+            graphs[state["i"] % K]()
 
         with torch.cuda.stream(stream):
             e2e_step()

@@ -60,16 +60,23 @@ class StepIO:
             nbytes = n * torch.empty((), dtype=dtype).element_size()
             return buf[off:off + nbytes].view(dtype).view(shape)
 
-        ins = [(L, n) for L in layers for n in self.IN_NAMES if L.get(n) is not None]
-        self.inp, offs = arena([L[n] for L, n in ins])
-        for (L, n), o in zip(ins, offs):
+        ins = [(li, L, n) for li, L in enumerate(layers) for n in self.IN_NAMES if L.get(n) is not None]
+        self.inp, offs = arena([L[n] for _, L, n in ins])
+        # layer l's inputs and output occupy one contiguous byte range of each
+        # arena (the slots are layer-major), so they can move layer by layer
+        self.in_ranges = [[self.inp.numel(), 0] for _ in layers]
+        for (li, L, n), o in zip(ins, offs):
             v = view(self.inp, o, L[n].dtype, tuple(L[n].shape))
             v.copy_(L[n])
             L[n] = v
+            r = self.in_ranges[li]
+            r[0], r[1] = min(r[0], o), max(r[1], o + v.numel() * v.element_size())
         outs = [torch.empty_like(L["q"]) for L in layers]
         self.out, offs = arena(outs)
+        self.out_ranges = []
         for L, t, o in zip(layers, outs, offs):
             L["out"] = view(self.out, o, t.dtype, tuple(t.shape))
+            self.out_ranges.append((o, o + t.numel() * t.element_size()))
 
 
 def compress_args(wl: synth.Workload, L, entry_base: int = 0):
@@ -123,15 +130,19 @@ class DecodeStep:
             self.calls.append((args, out, keep, ws))
         self.outputs = [c[1] for c in self.calls]
 
-    def __call__(self):
+    def layer(self, i: int):
+        """Enqueue layer i alone: its compressors' step, then its attention."""
         sh = self.stream.cuda_stream
-        for (cargs, _), (args, _, _, _) in zip(self.compress, self.calls):
-            st = self.lib.decode_compress(C.byref(cargs), sh)
-            if st != 0:
-                native.check(st, "decode_compress")
-            st = self.lib.compressed_attn_decode(C.byref(args), sh)
-            if st != 0:
-                native.check(st, "compressed_attn_decode")
+        st = self.lib.decode_compress(C.byref(self.compress[i][0]), sh)
+        if st != 0:
+            native.check(st, "decode_compress")
+        st = self.lib.compressed_attn_decode(C.byref(self.calls[i][0]), sh)
+        if st != 0:
+            native.check(st, "compressed_attn_decode")
+
+    def __call__(self):
+        for i in range(len(self.calls)):
+            self.layer(i)
 
 
 class DecodeGraph:
@@ -146,6 +157,54 @@ class DecodeGraph:
         torch.cuda.synchronize()
         with torch.cuda.graph(self.graph, stream=step.stream, capture_error_mode="thread_local"):
             step()
+        torch.cuda.synchronize()
+
+    def __call__(self):
+        self.graph.replay()
+
+
+class HostIOGraph:
+    """A decode step fed from host memory, captured as one CUDA graph with the
+    host copies pipelined layer by layer: every layer's input slice starts
+    for the device on a copy stream at once (layer l's kernels wait only for
+    its own slice, so the later slices arrive while earlier layers run), and
+    each layer's output leaves on another copy stream as soon as the layer
+    is done.  host_in and host_out are pinned host buffers shaped like
+    io.inp and io.out (one host_in per graph: a buffer the host rewrites
+    must not be one a replay may still be reading).  Make it after the step
+    has run once (the library's first-call set-up happens outside capture)."""
+
+    def __init__(self, step: DecodeStep, io: StepIO, host_in: torch.Tensor, host_out: torch.Tensor):
+        self.graph = torch.cuda.CUDAGraph()
+        main = step.stream
+        cin = torch.cuda.Stream(main.device)
+        cout = torch.cuda.Stream(main.device)
+        n = len(step.calls)
+        ev_in = [torch.cuda.Event() for _ in range(n)]
+        ev_out = [torch.cuda.Event() for _ in range(n)]
+
+        def enqueue():
+            cin.wait_stream(main)
+            cout.wait_stream(main)
+            with torch.cuda.stream(cin):
+                for li, (a, b) in enumerate(io.in_ranges):
+                    io.inp[a:b].copy_(host_in[a:b], non_blocking=True)
+                    ev_in[li].record(cin)
+            for li in range(n):
+                main.wait_event(ev_in[li])
+                step.layer(li)
+                ev_out[li].record(main)
+                cout.wait_event(ev_out[li])
+                a, b = io.out_ranges[li]
+                with torch.cuda.stream(cout):
+                    host_out[a:b].copy_(io.out[a:b], non_blocking=True)
+            main.wait_stream(cin)
+            main.wait_stream(cout)
+
+        # (capture only: the step has run before, so the library's lazy set-up is done)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(self.graph, stream=main, capture_error_mode="thread_local"):
+            enqueue()
         torch.cuda.synchronize()
 
     def __call__(self):

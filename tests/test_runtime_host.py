@@ -57,3 +57,29 @@ def test_decode_step_runs_compressor_then_attention_per_layer(monkeypatch):
         for n in ("kv_raw", "ca", "cza"):
             assert io.inp.data_ptr() <= L[n].data_ptr() < io.inp.data_ptr() + io.inp.numel()
     assert torch.equal(layers[0]["pos"], torch.full((2,), 2047, dtype=torch.int32))
+
+
+def test_step_io_layer_ranges_partition_the_arenas():
+    """Layer l's inputs and output lie in one byte range of each arena, the
+    ranges in layer order and disjoint: the end-to-end graph moves them layer
+    by layer."""
+    wl = synth.WORKLOADS["decode_1m"]
+    layers = synth.decode_inputs(wl, "cpu", ctx=2047, B=2)
+    io = runtime.StepIO(layers, "cpu")
+    base_in, base_out = io.inp.data_ptr(), io.out.data_ptr()
+    assert len(io.in_ranges) == len(io.out_ranges) == len(layers)
+    prev_in = prev_out = 0
+    for li, L in enumerate(layers):
+        a, b = io.in_ranges[li]
+        assert prev_in <= a < b <= io.inp.numel()
+        prev_in = b
+        for n in runtime.StepIO.IN_NAMES:
+            t = L.get(n)
+            if t is not None:
+                lo = t.data_ptr() - base_in
+                assert a <= lo and lo + t.numel() * t.element_size() <= b, (li, n)
+        a, b = io.out_ranges[li]
+        assert prev_out <= a < b <= io.out.numel()
+        prev_out = b
+        lo = L["out"].data_ptr() - base_out
+        assert (a, b) == (lo, lo + L["out"].numel() * L["out"].element_size())
