@@ -43,7 +43,9 @@ class StepIO:
     layers' tensors become views of the arenas (same dtype and shape, slots
     256-byte aligned); make the DecodeStep after this."""
 
-    IN_NAMES = ("q", "qI", "w", "pos", "kv_raw", "ca", "cb", "cza", "czb", "ia", "ib", "iza", "izb")
+    # per layer: the compressors' inputs (and the positions) first, then the attention's
+    COMP_NAMES = ("pos", "kv_raw", "ca", "cb", "cza", "czb", "ia", "ib", "iza", "izb")
+    IN_NAMES = COMP_NAMES + ("qI", "w", "q")
 
     def __init__(self, layers, device):
         def arena(tensors):
@@ -63,14 +65,20 @@ class StepIO:
         ins = [(li, L, n) for li, L in enumerate(layers) for n in self.IN_NAMES if L.get(n) is not None]
         self.inp, offs = arena([L[n] for _, L, n in ins])
         # layer l's inputs and output occupy one contiguous byte range of each
-        # arena (the slots are layer-major), so they can move layer by layer
+        # arena (the slots are layer-major), so they can move layer by layer;
+        # within a layer the compressors' inputs come first (comp_ends[l]:
+        # the end of that part)
         self.in_ranges = [[self.inp.numel(), 0] for _ in layers]
+        self.comp_ends = [0 for _ in layers]
         for (li, L, n), o in zip(ins, offs):
             v = view(self.inp, o, L[n].dtype, tuple(L[n].shape))
             v.copy_(L[n])
             L[n] = v
             r = self.in_ranges[li]
-            r[0], r[1] = min(r[0], o), max(r[1], o + v.numel() * v.element_size())
+            end = o + v.numel() * v.element_size()
+            r[0], r[1] = min(r[0], o), max(r[1], end)
+            if n in self.COMP_NAMES:
+                self.comp_ends[li] = max(self.comp_ends[li], end)
         outs = [torch.empty_like(L["q"]) for L in layers]
         self.out, offs = arena(outs)
         self.out_ranges = []
@@ -130,15 +138,22 @@ class DecodeStep:
             self.calls.append((args, out, keep, ws))
         self.outputs = [c[1] for c in self.calls]
 
-    def layer(self, i: int):
-        """Enqueue layer i alone: its compressors' step, then its attention."""
-        sh = self.stream.cuda_stream
-        st = self.lib.decode_compress(C.byref(self.compress[i][0]), sh)
+    def compress_step(self, i: int):
+        """Enqueue layer i's compressors' step."""
+        st = self.lib.decode_compress(C.byref(self.compress[i][0]), self.stream.cuda_stream)
         if st != 0:
             native.check(st, "decode_compress")
-        st = self.lib.compressed_attn_decode(C.byref(self.calls[i][0]), sh)
+
+    def attention(self, i: int):
+        """Enqueue layer i's attention (indexer top-k for CSA, then attention)."""
+        st = self.lib.compressed_attn_decode(C.byref(self.calls[i][0]), self.stream.cuda_stream)
         if st != 0:
             native.check(st, "compressed_attn_decode")
+
+    def layer(self, i: int):
+        """Enqueue layer i alone: its compressors' step, then its attention."""
+        self.compress_step(i)
+        self.attention(i)
 
     def __call__(self):
         for i in range(len(self.calls)):
@@ -165,11 +180,12 @@ class DecodeGraph:
 
 class HostIOGraph:
     """A decode step fed from host memory, captured as one CUDA graph with the
-    host copies pipelined layer by layer: every layer's input slice starts
-    for the device on a copy stream at once (layer l's kernels wait only for
-    its own slice, so the later slices arrive while earlier layers run), and
-    each layer's output leaves on another copy stream as soon as the layer
-    is done.  host_in and host_out are pinned host buffers shaped like
+    host copies pipelined: on a copy stream the first layer's compressor
+    inputs go first, then its attention inputs, then each later layer's
+    slice; the first layer's compressor step waits only for the first part,
+    its attention for the second, and each later layer for its own slice
+    (which lands while the earlier layers run).  Each layer's output leaves on another
+    copy stream as soon as the layer is done.  host_in and host_out are pinned host buffers shaped like
     io.inp and io.out (one host_in per graph: a buffer the host rewrites
     must not be one a replay may still be reading).  Make it after the step
     has run once (the library's first-call set-up happens outside capture)."""
@@ -180,19 +196,29 @@ class HostIOGraph:
         cin = torch.cuda.Stream(main.device)
         cout = torch.cuda.Stream(main.device)
         n = len(step.calls)
-        ev_in = [torch.cuda.Event() for _ in range(n)]
+        a0, b0 = io.in_ranges[0]
+        c0 = io.comp_ends[0]
+        parts = [(a0, c0), (c0, b0)] + [tuple(r) for r in io.in_ranges[1:]]
+        ev_in = [torch.cuda.Event() for _ in parts]
         ev_out = [torch.cuda.Event() for _ in range(n)]
 
         def enqueue():
             cin.wait_stream(main)
             cout.wait_stream(main)
             with torch.cuda.stream(cin):
-                for li, (a, b) in enumerate(io.in_ranges):
-                    io.inp[a:b].copy_(host_in[a:b], non_blocking=True)
-                    ev_in[li].record(cin)
+                for k, (a, b) in enumerate(parts):
+                    if b > a:
+                        io.inp[a:b].copy_(host_in[a:b], non_blocking=True)
+                    ev_in[k].record(cin)
             for li in range(n):
-                main.wait_event(ev_in[li])
-                step.layer(li)
+                if li == 0:
+                    main.wait_event(ev_in[0])
+                    step.compress_step(0)
+                    main.wait_event(ev_in[1])
+                    step.attention(0)
+                else:
+                    main.wait_event(ev_in[li + 1])
+                    step.layer(li)
                 ev_out[li].record(main)
                 cout.wait_event(ev_out[li])
                 a, b = io.out_ranges[li]

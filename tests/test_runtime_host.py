@@ -73,11 +73,16 @@ def test_step_io_layer_ranges_partition_the_arenas():
         a, b = io.in_ranges[li]
         assert prev_in <= a < b <= io.inp.numel()
         prev_in = b
+        c = io.comp_ends[li]
+        assert a < c <= b
         for n in runtime.StepIO.IN_NAMES:
             t = L.get(n)
             if t is not None:
                 lo = t.data_ptr() - base_in
-                assert a <= lo and lo + t.numel() * t.element_size() <= b, (li, n)
+                hi = lo + t.numel() * t.element_size()
+                assert a <= lo and hi <= b, (li, n)
+                # the compressors' inputs before comp_ends, the attention's after
+                assert (hi <= c) if n in runtime.StepIO.COMP_NAMES else (lo >= c), (li, n)
         a, b = io.out_ranges[li]
         assert prev_out <= a < b <= io.out.numel()
         prev_out = b
