@@ -430,18 +430,21 @@ int launch_indexer_tc_t(const csahca_indexer_args* a, IdxTcParams p, cudaStream_
                        (uint64_t)a->B * a->nq * a->HI, 64, (uint32_t)Cfg::NCOL, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return CSAHCA_ERR_LAUNCH;
   auto kern = indexer_tc_kernel<QT, 64, kFP8>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+  // a routed decode scan keeps its item's scores beside the key stages
+  const int smem = Cfg::SMEM + (p.route ? p.tiles_per_split * 128 * 4 : 0);
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   if (grid <= 0) return CSAHCA_OK;
   CSAHCA_TRACE(QT == 1 ? "indexer_scores_tc_decode" : "indexer_scores_tc_prefill", s);
-  launch_k(kern, dim3(grid), dim3(kIdxTcThreads), Cfg::SMEM, s, kmap, qmap, p);
+  launch_k(kern, dim3(grid), dim3(kIdxTcThreads), smem, s, kmap, qmap, p);
   CSAHCA_CHECK_LAUNCH();
   return CSAHCA_OK;
 }
 
 // Tensor-core scores for queries [q0, q0 + qc) into scores (row stride N).
-// Decode split of the FP8 scan: each sequence's key tiles over about one CTA per SM.
-void f8_decode_split(const csahca_indexer_args* a, int* tiles_per_split, int* splits) {
+// Decode split of a routed scan: each sequence's key tiles over about one CTA
+// per SM, one work item per CTA.
+void decode_split(const csahca_indexer_args* a, int* tiles_per_split, int* splits) {
   const int tiles = (int)ceil_div64(a->N, 128);
   int sp = num_sms() / (a->B > 0 ? a->B : 1);
   if (sp > tiles) sp = tiles;
@@ -450,12 +453,12 @@ void f8_decode_split(const csahca_indexer_args* a, int* tiles_per_split, int* sp
   *splits = (int)ceil_div64(tiles, *tiles_per_split);
 }
 
-// The FP8 decode scan can route the top-k in its epilogue when every work
-// item has a CTA of its own (a CTA waits for its row's other items) and the
-// item's scores fit in shared memory beside the key stages.
-bool f8_route_ok(const csahca_indexer_args* a) {
+// A decode scan (e4m3 or bf16 keys) can route the top-k in its epilogue when
+// every work item has a CTA of its own (a CTA waits for its row's other
+// items) and the item's scores fit in shared memory beside the key stages.
+bool decode_route_ok(const csahca_indexer_args* a) {
   int tps = 0, sp = 0;
-  f8_decode_split(a, &tps, &sp);
+  decode_split(a, &tps, &sp);
   return a->B * sp <= num_sms() && tps <= kRouteMaxTiles;
 }
 
@@ -476,7 +479,7 @@ int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* score
     // e4m3 keys straight into the FP8 tensor cores, one query per work item;
     // decode spreads each sequence's key tiles over about one CTA per SM
     if (qc == 1) {
-      f8_decode_split(a, &p.tiles_per_split, &p.splits);
+      decode_split(a, &p.tiles_per_split, &p.splits);
       p.n_items = a->B * p.splits;
     } else {
       p.splits = 0;
@@ -501,13 +504,23 @@ int launch_indexer_tc(const csahca_indexer_args* a, int q0, int qc, float* score
     return CSAHCA_OK;
   }
   if (qc == 1) {
-    const int tiles = (int)ceil_div64(a->N, 128);
-    int splits = (int)ceil_div64(2 * num_sms(), a->B);
-    if (splits > tiles) splits = tiles;
-    if (splits < 1) splits = 1;
-    p.tiles_per_split = (int)ceil_div64(tiles, splits);
-    p.splits = (int)ceil_div64(tiles, p.tiles_per_split);
+    if (above != nullptr) {
+      // routed: one work item per CTA; the epilogue keeps the item's scores
+      // and histogram and routes its keys (indexer_tc.cuh)
+      decode_split(a, &p.tiles_per_split, &p.splits);
+      p.route = 1;
+      p.above = above;
+      p.cand = cand;
+    } else {
+      const int tiles = (int)ceil_div64(a->N, 128);
+      int splits = (int)ceil_div64(2 * num_sms(), a->B);
+      if (splits > tiles) splits = tiles;
+      if (splits < 1) splits = 1;
+      p.tiles_per_split = (int)ceil_div64(tiles, splits);
+      p.splits = (int)ceil_div64(tiles, p.tiles_per_split);
+    }
     p.n_items = a->B * p.splits;
+    p.items_per_row = p.splits;
     return launch_indexer_tc_t<1, false>(a, p, s);
   }
   p.splits = 0;
@@ -594,8 +607,11 @@ int run_indexer(const csahca_indexer_args* a, void* stream, const void* prefetch
     char* scratch = static_cast<char*>(a->workspace) + indexer_scores_bytes(a);
     // decode with e4m3 keys: the FP8 indexer builds the top-k row histograms
     // while it writes the scores (the scratch it adds into is zeroed first)
-    const bool fuse_hist = qc == a->nq && topk_uses_large(a) && indexer_tc_eligible(a) &&
-                           a->k_dtype == CSAHCA_E4M3 && a->N <= kTopkLargeMaxN;
+    // (with bf16 keys only when the scan also routes: its epilogue has no
+    // last-item threshold for the select kernel)
+    const bool fuse_hist = qc == a->nq && topk_uses_large(a) && indexer_tc_eligible(a) && a->N <= kTopkLargeMaxN &&
+                           (a->k_dtype == CSAHCA_E4M3 ||
+                            (a->k_dtype == CSAHCA_BF16 && a->nq == 1 && decode_route_ok(a) && !a->sel_scores));
     uint32_t* hist = nullptr;
     uint32_t* counters = nullptr;
     int* above = nullptr;
@@ -604,7 +620,7 @@ int run_indexer(const csahca_indexer_args* a, void* stream, const void* prefetch
     // routes the keys into the top-k lists from shared memory, and one CTA
     // per row finishes
     // (sel_scores reads the scores back: they must reach the workspace)
-    const bool route = fuse_hist && a->nq == 1 && f8_route_ok(a) && !a->sel_scores;
+    const bool route = fuse_hist && a->nq == 1 && decode_route_ok(a) && !a->sel_scores;
     if (fuse_hist) {
       const TopkLargeLayout L = topk_large_layout((int64_t)a->B * qc, a->N, a->k);
       const int zst = launch_zero(scratch + L.hist, L.above - L.hist, s);

@@ -84,19 +84,6 @@ __device__ __forceinline__ void cp_async4_zfill(void* dst_smem, const void* src_
                : "memory");
 }
 
-// Named barrier 3 over the 256 threads of both epilogue groups.
-__device__ __forceinline__ void epi_sync256() { asm volatile("bar.sync 3, 256;" ::: "memory"); }
-__device__ __forceinline__ bool epi_any256(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 3, 256, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v)
-      : "memory");
-  return r != 0;
-}
-
 // Unrouted rows: the last work item of a top-k row (counted after a fence)
 // sees the row's histogram complete, so the 256 epilogue threads find its
 // threshold bin T (fewer than k keys in bins above T, at least k from T up)
@@ -139,131 +126,6 @@ __device__ __forceinline__ void idx_row_done(const IdxTcParams& p, int row, uint
   }
   epi_sync256();
 }
-
-// Exclusive prefix of c over the 256 epilogue threads (named barrier 3);
-// *total receives the sum.  buf: 9 ints.
-__device__ __forceinline__ int epi_excl_count(int c, int* buf, int* total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int incl = c;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) buf[wid] = incl;
-  epi_sync256();
-  int base = 0, tot = 0;
-#pragma unroll
-  for (int w = 0; w < 8; ++w) {
-    const int x = buf[w];
-    base += w < wid ? x : 0;
-    tot += x;
-  }
-  *total = tot;
-  epi_sync256();
-  return base + incl - c;
-}
-
-// Fused routing of one work item (all 256 epilogue threads), run by every
-// item of a top-k row once its scores and histogram adds are done: count the
-// item as done, wait (bounded) until every item of the row has counted, find
-// the row's threshold bin T from the row's histogram (fewer than k keys in
-// bins above T, at least k from T up), and send this item's keys above T to
-// the row's taken list and those in T to its candidate list, reserving each
-// list range with one atomic per CTA.  Every item finds T itself, so no item
-// waits for another to publish it.  Requires every item of the row to be
-// resident at once (one CTA per item), and nkeys <= 32 * 256.  An item
-// with no keys passes v = 0: it only counts.
-__device__ __forceinline__ void idx_route(const IdxTcParams& p, int row, int key0, int nkeys, int v,
-                                          const float* sc, int* buf, uint32_t* sh_T, int* sh_ok,
-                                          uint32_t* sh_base, volatile int* abort_flag) {
-  const int ept = threadIdx.x, lane = ept & 31, wid = ept >> 5;
-  uint32_t* cnt = p.counters + (int64_t)row * kTopkCounters;
-  __threadfence();                                   // this item's histogram adds
-  epi_sync256();
-  if (v <= p.k) {                                    // the row takes every visible key: count only
-    if (ept == 0) atomicAdd(&cnt[kCntItems], 1u);
-    return;
-  }
-  if (ept == 0) {
-    atomicAdd(&cnt[kCntItems], 1u);
-    int ok = 0;
-    for (uint32_t it = 0; it < kMbarSpinLimit; ++it) {
-      uint32_t r;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(r) : "l"(cnt + kCntItems) : "memory");
-      if (r >= (uint32_t)p.items_per_row) { ok = 1; break; }
-      if ((it & 1023u) == 1023u && *abort_flag) break;
-      __nanosleep(32);
-    }
-    if (!ok) { raise_device_error(DEVERR_MBAR_TIMEOUT); *abort_flag = 1; }
-    *sh_ok = ok;
-  }
-  epi_sync256();
-  if (!*sh_ok) return;
-  // the row's histogram: thread ept holds bins [8 ept, 8 ept + 8); a suffix
-  // sum over the threads gives the keys in bins above each thread's group
-  const uint4* g4 = reinterpret_cast<const uint4*>(p.hist + (int64_t)row * kHistBins) + 2 * ept;
-  const uint4 h0 = __ldcg(g4), h1 = __ldcg(g4 + 1);
-  const uint32_t c[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-  uint32_t tot = 0;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) tot += c[e];
-  uint32_t suf = tot;                                // inclusive suffix sum within the warp
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_down_sync(0xffffffffu, suf, o);
-    if (lane + o < 32) suf += y;
-  }
-  if (lane == 0) buf[wid] = (int)suf;                // the warp's total
-  epi_sync256();
-  uint32_t run = suf - tot;                          // keys in bins above this thread's group
-#pragma unroll
-  for (int w = 0; w < 8; ++w) run += w > wid ? (uint32_t)buf[w] : 0u;
-  const uint32_t k = (uint32_t)p.k;
-  if (run < k && run + tot >= k) {
-#pragma unroll
-    for (int e = 7; e >= 0; --e) {
-      if (run + c[e] >= k) { *sh_T = (uint32_t)(ept * 8 + e); break; }
-      run += c[e];
-    }
-  }
-  epi_sync256();
-  const uint32_t T = *sh_T;
-  // one pass over this item's scores: bit j of ma / me marks key ept + 256 j
-  // above T / in T
-  uint32_t ma = 0u, me = 0u;
-  const int lim = min(nkeys, v - key0);
-#pragma unroll 4
-  for (int j = 0; j < 32; ++j) {
-    const int i = ept + 256 * j;
-    if (i < lim) {
-      const uint32_t b = order_key(sc[i]) >> kHistShift;
-      ma |= (uint32_t)(b > T) << j;
-      me |= (uint32_t)(b == T) << j;
-    }
-  }
-  int tot2;
-  const int off = epi_excl_count(__popc(ma) | (__popc(me) << 16), buf, &tot2);
-  if (ept == 0) {
-    sh_base[0] = tot2 & 0xFFFF ? atomicAdd(&cnt[kCntAbove], (uint32_t)(tot2 & 0xFFFF)) : 0u;
-    sh_base[1] = tot2 >> 16 ? atomicAdd(&cnt[kCntCand], (uint32_t)(tot2 >> 16)) : 0u;
-  }
-  epi_sync256();
-  int* above = p.above + (int64_t)row * p.k;
-  uint2* cand = p.cand + (int64_t)row * p.N;
-  uint32_t pt = sh_base[0] + (uint32_t)(off & 0xFFFF), pc = sh_base[1] + (uint32_t)(off >> 16);
-  for (; ma; ma &= ma - 1u, ++pt)
-    if (pt < (uint32_t)p.k) above[pt] = key0 + ept + 256 * (__ffs(ma) - 1);
-  for (; me; me &= me - 1u, ++pc) {
-    const int i = ept + 256 * (__ffs(me) - 1);
-    if (pc < (uint32_t)p.N) cand[pc] = make_uint2(order_key(sc[i]), (uint32_t)(key0 + i));
-  }
-}
-
-// Route bound: the scores of a routed work item stay in shared memory, and
-// the routing marks each thread's keys in one 32-bit mask.
-constexpr int kRouteMaxTiles = 64;
-static_assert(kRouteMaxTiles * 128 <= 32 * 256, "a routed item's keys fit the per-thread masks");
 
 template <int HI>
 __global__ void __launch_bounds__(kIdxF8Threads, 1)
@@ -417,7 +279,7 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
         if (!p.first_kernel) griddep_wait();
         // an empty item still counts
         if (do_hist) {
-          if (p.route) idx_route(p, row, 0, 0, 0, sc_s, route_buf, &route_T, &route_ok, route_base, &abort_flag);
+          if (p.route) idx_route(p, threadIdx.x, row, 0, 0, 0, sc_s, route_buf, &route_T, &route_ok, route_base, &abort_flag);
           else idx_row_done(p, row, scan_s, &row_flag);
         }
         continue;
@@ -523,7 +385,7 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
           if (c) { atomicAdd(gh + i, c); hist_s[i] = 0; }
         }
         if (p.route)
-          idx_route(p, row, it.kt0 * 128, (it.kt1 - it.kt0) * 128, v, sc_s, route_buf, &route_T, &route_ok,
+          idx_route(p, threadIdx.x, row, it.kt0 * 128, (it.kt1 - it.kt0) * 128, v, sc_s, route_buf, &route_T, &route_ok,
                     route_base, &abort_flag);
         else
           idx_row_done(p, row, scan_s, &row_flag);
