@@ -99,6 +99,32 @@ def test_prefill_csa_bf16_prefill_shapes():
     assert api.device_error() == 0
 
 
+def test_prefill_csa_tc_ragged_tiles():
+    """Tensor-core CSA prefill (H = 64, d = 512) with k and w that are not
+    multiples of the key tile (k = 200: a full tile of selected rows and a
+    ragged one; w = 100: one ragged window tile), two sequences, and queries
+    with fewer visible entries than k (lists padded with -1) or a window
+    clipped at t = 0."""
+    base = synth.WORKLOADS["csa_prefill_128k"]
+    wl = synth.Workload(**{**base.__dict__, "k": 200, "w": 100})
+    n, B = 1500 + 7, 2
+    inp, kv, m = _prefill_layer(wl, n, B)
+    ik = inp["ik"]
+    kI = api.csa_compress(ik["a"], ik["b"], ik["za"], ik["zb"], ik["bias_a"], ik["bias_b"], m,
+                          rms_norm=False)
+    q_pos = torch.arange(n, device=DEV, dtype=torch.int32)[None].expand(B, n).contiguous()
+    idx = api.indexer_topk(inp["qI"], inp["w"], kI, q_pos, m, wl.k)
+    out = api.compressed_attn_prefill("csa", inp["q"], kv, inp["kv_win"], inp["sinks"], m=m,
+                                      w=wl.w, rope_dims=wl.r, idx=idx, q_gain=inp["q_gain"],
+                                      kv_gain=inp["kv_gain"])
+    for b in range(B):
+        rows = _sample(n, [0, 1, 3, 63, 64, 99, 100, 255, 256, 4 * wl.k - 1, 4 * wl.k, n - 1], seed=7 + b,
+                       count=10)
+        ref = _oracle_rows("csa", inp, kv, idx, wl, m, b, rows)
+        check_close(npy(out[b, rows]), ref, "bf16", f"csa prefill ragged b={b}")
+    assert api.device_error() == 0
+
+
 def test_prefill_no_window_no_sink_edge():
     """w = 0 with the first queries (no visible entry): the output is 0 for
     t < m - 1 (only the sink in the denominator)."""
