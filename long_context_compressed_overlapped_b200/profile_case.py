@@ -5,6 +5,7 @@ a profiler to capture.
     python -m long_context_compressed_overlapped_b200.profile_case hca --calls 4
     python -m long_context_compressed_overlapped_b200.profile_case csa_fp8kv --calls 4
     python -m long_context_compressed_overlapped_b200.profile_case indexer --calls 4
+    python -m long_context_compressed_overlapped_b200.profile_case indexer_256k --calls 4
     python -m long_context_compressed_overlapped_b200.profile_case compress --calls 4
     python -m long_context_compressed_overlapped_b200.profile_case prefill --calls 2
     python -m long_context_compressed_overlapped_b200.profile_case prefill_tail --calls 2
@@ -14,7 +15,9 @@ e4m3 keys, top-k select, attention, combine); ``hca``: one HCA decode layer
 (attention, combine); ``csa_fp8kv`` / ``hca_fp8kv``: the same layers with FP8
 KV cache rows (decode_1m_fp8kv: 640-byte rows of e4m3 codes, bf16 RoPE dims
 and fp32 scales); ``indexer``: ``indexer_topk`` on the CSA layer's indexer
-inputs; ``compress``: ``decode_compress`` of the CSA layer with the new token at
+inputs; ``indexer_256k``: the same on the decode_256k CSA layer (eight
+sequences at a 262,144-token context, 65,536 bf16 indexer keys each, 134 MB,
+routed by the bf16 indexer); ``compress``: ``decode_compress`` of the CSA layer with the new token at
 position 1,048,575, which completes a block (ring store, window row, pooled
 entry and e4m3 indexer key).  Four sequences at a 1,048,576-token context: 262,144 CSA entries
 (1 GB of bf16 rows, 134 MB of e4m3 indexer keys) or 8,192 HCA entries per
@@ -41,7 +44,7 @@ from . import api, native, runtime, synth
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("case", choices=("csa", "hca", "csa_fp8kv", "hca_fp8kv", "indexer", "compress",
+    ap.add_argument("case", choices=("csa", "hca", "csa_fp8kv", "hca_fp8kv", "indexer", "indexer_256k", "compress",
                                         "prefill", "prefill_tail"))
     ap.add_argument("--calls", type=int, default=4)
     a = ap.parse_args(argv)
@@ -49,7 +52,8 @@ def main(argv=None) -> int:
         return prefill_case(a.calls)
     if a.case == "prefill_tail":
         return prefill_tail_case(a.calls)
-    wl = synth.WORKLOADS["decode_1m_fp8kv" if a.case.endswith("_fp8kv") else "decode_1m"]
+    wl = synth.WORKLOADS["decode_1m_fp8kv" if a.case.endswith("_fp8kv") else
+                         "decode_256k" if a.case.endswith("_256k") else "decode_1m"]
     kind = "hca" if a.case.startswith("hca") else "csa"
     ctx = wl.ctx - 1 if a.case == "compress" else wl.ctx
     L = synth.decode_inputs(wl, "cuda", ctx=ctx, B=wl.B, layers=(kind,))[0]
@@ -58,7 +62,7 @@ def main(argv=None) -> int:
         if a.case == "compress":
             native.check(native.lib().decode_compress(C.byref(cargs[0]), torch.cuda.current_stream().cuda_stream),
                          "decode_compress")
-        elif a.case == "indexer":
+        elif a.case in ("indexer", "indexer_256k"):
             api.indexer_topk(L["qI"][:, None], L["w"][:, None], L["kI"], L["pos"][:, None], L["m"], wl.k,
                              kI_scale=L["kI_scale"])
         else:
