@@ -586,8 +586,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap comp_rows, const __grid_const
         }
       }
     }
-    // drain the last loads before the CTA may exit
-    cp_async_wait_all();
+    // drain the last loads before the CTA may exit: the last tile's chunk
+    // barriers complete only once every producer lane's copies have landed
+    // (the gathers are not committed to cp.async groups, so the group wait
+    // orders nothing; this form of the drain measured fastest in decode)
+    cp_async_wait<0>();
     if (lane == 0 && tcount > 0)
       for (int c = 0; c < kAttnChunks; ++c) mbar_wait(&bar_kfull[c], (tcount - 1) & 1, &abort_flag);
     if (pw == 0 && lane == 0 && icount > 0) mbar_wait(&bar_q_raw, (icount - 1) & 1, &abort_flag);

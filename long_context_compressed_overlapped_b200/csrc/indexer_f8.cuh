@@ -217,7 +217,9 @@ indexer_f8_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16*
       }
     }
     // drain: every fill this warp issued has landed before the CTA may exit
-    cp_async_wait_all();
+    // (the stage barriers complete only once the lanes' copies have; the
+    // group wait orders nothing, the copies being uncommitted)
+    cp_async_wait<0>();
     if (lane == 0)
       for (uint32_t i = (a_iter > NS ? a_iter - NS : 0); i < a_iter; ++i)
         if ((i & 1u) == pe) mbar_wait(&bar_a_full[i % NS], (i / NS) & 1, &abort_flag);
