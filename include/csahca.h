@@ -496,10 +496,18 @@ int64_t csahca_struct_size(int which);
 
 /* Device-side error word of the current device: every bounded wait in the
  * kernels that gives up ORs a code into it and the kernel returns early
- * instead of hanging.  Synchronises `stream`, stores the word in *code (0 =
- * no error) and clears it.  Returns CSAHCA_OK, or CSAHCA_ERR_LAUNCH if the
- * stream itself reports a CUDA error. */
+ * instead of hanging (1: a barrier wait reached its iteration limit; 2: a
+ * selection index outside [0, N) was skipped).  Synchronises `stream`, stores
+ * the word in *code (0 = no error) and clears it.  Returns CSAHCA_OK, or
+ * CSAHCA_ERR_LAUNCH if the stream itself reports a CUDA error. */
 int csahca_device_error(void* stream, int32_t* code);
+
+/* Self-test of that failure path: launches one kernel on `stream` whose
+ * bounded wait on a barrier that nothing completes gives up (well under a
+ * second), so that csahca_device_error() on the same stream then reports
+ * code 1 and the device stays usable for the calls that follow.  Returns
+ * CSAHCA_OK, CSAHCA_ERR_NO_DEVICE without a B200, or CSAHCA_ERR_LAUNCH. */
+int csahca_selftest_bounded_wait(void* stream);
 
 /* ---- tracing ---------------------------------------------------------------
  * Optional per-kernel timing.  While enabled, every kernel the library

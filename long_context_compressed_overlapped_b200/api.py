@@ -299,6 +299,12 @@ def device_error(stream=None) -> int:
     return int(code.value)
 
 
+def selftest_bounded_wait(stream=None) -> None:
+    """Launch the library's failure-path self-test: a kernel whose bounded
+    wait gives up; device_error() on the same stream then reports code 1."""
+    N.check(N.lib().csahca_selftest_bounded_wait(_stream(stream)), "csahca_selftest_bounded_wait")
+
+
 def trace_enable(on: bool = True) -> None:
     """Bracket every library kernel launch with CUDA events (see trace_collect)."""
     N.check(N.lib().csahca_trace_enable(int(bool(on))), "csahca_trace_enable")

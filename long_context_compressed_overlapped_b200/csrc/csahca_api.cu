@@ -1266,6 +1266,21 @@ int run_cp_attn_merge(const csahca_cp_merge_args* a, void* stream) {
 
 // ============================================================== C ABI ======
 
+// Self-test of the failure detection: one thread waits on an mbarrier that
+// nothing arrives at; the bounded wait gives up after its iteration limit,
+// ORs DEVERR_MBAR_TIMEOUT into the device error word and the kernel returns.
+__global__ void selftest_bounded_wait_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, &abort_flag);
+}
+
 extern "C" {
 
 int csa_compress(const csahca_compress_args* args, void* stream) { return run_compress(args, stream, true); }
@@ -1378,6 +1393,14 @@ int csahca_trace_collect(csahca_trace_entry* out, int max_entries, int* n_entrie
   for (; n < (int)acc.size() && n < max_entries; ++n) out[n] = acc[n];
   *n_entries = n;
   return status;
+}
+
+int csahca_selftest_bounded_wait(void* stream) {
+  const int st = device_ok();
+  if (st != CSAHCA_OK) return st;
+  selftest_bounded_wait_kernel<<<1, 32, 0, as_stream(stream)>>>();
+  CSAHCA_CHECK_LAUNCH();
+  return CSAHCA_OK;
 }
 
 int csahca_device_error(void* stream, int32_t* code) {

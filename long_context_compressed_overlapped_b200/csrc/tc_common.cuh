@@ -17,7 +17,12 @@
 
 namespace csahca {
 
-constexpr uint32_t kMbarSpinLimit = 1u << 22;   // bounded waits (well under a second)
+// Polls before a bounded wait gives up.  On the B200 a try_wait on a pending
+// phase suspends the thread ~4 us before it returns false (2^22 polls took
+// 16.6 s), so 2^18 polls give up after about a second; the routing flag
+// wait's polls (an L2 round trip and a short nap) end sooner.  The waits of a
+// working call last microseconds.
+constexpr uint32_t kMbarSpinLimit = 1u << 18;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

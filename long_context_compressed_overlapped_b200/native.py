@@ -116,6 +116,7 @@ SIGNATURES = {
     "csahca_kv_row_bytes": (C.c_int64, [C.c_int32, C.c_int32, C.c_int32]),
     "csahca_struct_size": (C.c_int64, [C.c_int]),
     "csahca_device_error": (C.c_int, [vp, C.POINTER(i32)]),
+    "csahca_selftest_bounded_wait": (C.c_int, [vp]),
     "csahca_trace_enable": (C.c_int, [C.c_int]),
     "csahca_trace_collect": (C.c_int, [C.POINTER(TraceEntry), C.c_int, C.POINTER(C.c_int)]),
 }

@@ -179,6 +179,7 @@ def test_no_device_is_reported_not_faked(lib):
     dc = N.DecodeCompressArgs(kind=N.HCA, dtype=N.BF16, B=1, d=512, m=128, N_cap=4, pos=16, a=16, za=16,
                               bias_a=16, ring=16, kv_cache=16)
     assert lib.decode_compress(C.byref(dc), None) == N.ERR_NO_DEVICE
+    assert lib.csahca_selftest_bounded_wait(None) == N.ERR_NO_DEVICE
 
 
 def test_kv_row_bytes_matches_the_binding(lib):
